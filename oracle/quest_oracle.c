@@ -1,0 +1,345 @@
+/*
+ * QuEST oracle: a plain, slow, deliberately literal CPU implementation of the
+ * QuEST quantizer, trust-mask backward and integer linear layer, in fp64 / int64.
+ *
+ * TEST INFRASTRUCTURE ONLY. Only the test-suite, the package smoke check and
+ * the benchmark's CPU-baseline leg may load this library. The product (the CUDA
+ * library) shares no code with it and never calls it.
+ *
+ * What it follows (method source: "QuEST: Stable Training of LLMs with 1-Bit
+ * Weights and Activations", Panferov et al., arXiv 2502.05003):
+ *   - pith.science review, "What carries the argument": a Hadamard transform of
+ *     weights and activations, projection onto a uniform grid whose scale
+ *     minimises the L2 error against a standard Gaussian, and a backward pass
+ *     that multiplies the gradient *in the Hadamard domain* by a binary mask
+ *     zeroing entries whose quantization error exceeds half an interval.
+ *   - atlas.scime.ai summary, "Approach": Hadamard transform with RMS
+ *     normalisation, MSE-optimal clipping fitted to a Gaussian, trust threshold.
+ *   - pith.science review, "Assumptions & free parameters": after RMS
+ *     normalisation the data is treated as N(0,1) plus tails; alpha* comes from
+ *     a fixed N(0,1) target; Hadamard matrices are orthogonal, so a transform
+ *     applied to both matmul operands leaves the product unchanged.
+ *   - pith.science review, Figure 2 caption: two Hadamard transforms on the
+ *     forward pass, two inverse transforms on the backward pass.
+ *
+ * Readings where the pages are silent (each is listed with its reason in the
+ * design notes of the repository):
+ *   - Hadamard matrix: Sylvester order, H[i][j] = (-1)^popcount(i & j),
+ *     normalised by 1/sqrt(n); the inverse is the same matrix (symmetric,
+ *     orthogonal).
+ *   - RMS is taken over the transformed values y of an "rms group" (a multiple
+ *     of the Hadamard block that divides the row).
+ *   - Grid: symmetric midrise, 2^b levels at (i + 1/2) * Delta,
+ *     i = -2^(b-1) .. 2^(b-1)-1, Delta = alpha_b * r / 2^(b-1).
+ *   - alpha_b = 2^(b-1) * Delta*, Delta* the step minimising the Gaussian MSE.
+ *   - Code q = clamp(floor(y / Delta)); mask m = [ |t - (q + 1/2)| <= T/2 ].
+ *   - A group with r == 0 gives Delta = 0, q = 0, dequant 0, m = 1.
+ *   - No gradient flows through r.
+ *   - GEMM operand form c = 2q + 1, Y = acc * Delta_x * Delta_w / 4.
+ *
+ * Every computation is the definition written out: an explicit n x n Hadamard
+ * matrix and an O(n^2) matrix-vector product per block, a golden-section
+ * minimisation of the closed-form Gaussian MSE, and a triple-loop integer GEMM.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+#define ORACLE_OK 0
+#define ORACLE_EINVAL -1
+
+/* ------------------------------------------------------------------------- */
+/* Hadamard matrix (Sylvester construction, natural order).                   */
+/* ------------------------------------------------------------------------- */
+
+static int popcount_int(unsigned v) {
+    int c = 0;
+    while (v) {
+        c += (int)(v & 1u);
+        v >>= 1;
+    }
+    return c;
+}
+
+static int is_pow2(int64_t n) { return n > 0 && (n & (n - 1)) == 0; }
+
+/* Fills H (n x n, row-major) with the UNNORMALISED entries (-1)^popcount(i&j). */
+int oracle_hadamard(int n, double* H) {
+    if (!is_pow2(n) || n > 4096) return ORACLE_EINVAL;
+    for (int i = 0; i < n; ++i)
+        for (int j = 0; j < n; ++j)
+            H[(int64_t)i * n + j] = (popcount_int((unsigned)(i & j)) & 1) ? -1.0 : 1.0;
+    return ORACLE_OK;
+}
+
+/* y = (1/sqrt(n)) * H * x for one block; H is the unnormalised matrix. */
+static void hadamard_block(const double* H, int n, const double* x, double* y) {
+    const double norm = 1.0 / sqrt((double)n);
+    for (int i = 0; i < n; ++i) {
+        double acc = 0.0;
+        for (int j = 0; j < n; ++j) acc += H[(int64_t)i * n + j] * x[j];
+        y[i] = acc * norm;
+    }
+}
+
+/* ------------------------------------------------------------------------- */
+/* Gaussian MSE of the midrise uniform quantizer and its minimiser.           */
+/* ------------------------------------------------------------------------- */
+
+static double phi(double x) { return exp(-0.5 * x * x) / sqrt(2.0 * M_PI); }
+
+/* P(a <= X < b) for X ~ N(0,1); b may be +INFINITY. */
+static double gauss_mass(double a, double b) {
+    double ub = isinf(b) ? 0.0 : erfc(b / sqrt(2.0));
+    return 0.5 * (erfc(a / sqrt(2.0)) - ub);
+}
+
+/* Integral over [a, b) of (x - c)^2 phi(x) dx, using
+ *   int x^2 phi = [Phi] + a phi(a) - b phi(b),   int x phi = phi(a) - phi(b). */
+static double cell_sq_error(double a, double b, double c) {
+    double mass = gauss_mass(a, b);
+    double pa = phi(a);
+    double pb = isinf(b) ? 0.0 : phi(b);
+    double bpb = isinf(b) ? 0.0 : b * pb;
+    double m2 = mass + a * pa - bpb;
+    double m1 = pa - pb;
+    return m2 - 2.0 * c * m1 + c * c * mass;
+}
+
+/* E[(X - Q(X))^2], X ~ N(0,1), Q the 2^bits-level midrise quantizer of step
+ * delta: levels (i + 1/2) delta, decision thresholds at integer multiples of
+ * delta, outermost cells open to +-infinity. Uses the symmetry X -> -X. */
+double oracle_gauss_mse(int bits, double delta) {
+    if (bits < 1 || bits > 16 || !(delta > 0.0)) return NAN;
+    const int half = 1 << (bits - 1);
+    double total = 0.0;
+    for (int i = 0; i < half; ++i) {
+        double a = i * delta;
+        double b = (i == half - 1) ? INFINITY : (i + 1) * delta;
+        double c = (i + 0.5) * delta;
+        total += cell_sq_error(a, b, c);
+    }
+    return 2.0 * total;
+}
+
+/* Golden-section minimisation of oracle_gauss_mse over delta in [lo, hi]. */
+static double golden_min(int bits, double lo, double hi, double tol) {
+    const double g = (sqrt(5.0) - 1.0) / 2.0;
+    double a = lo, b = hi;
+    double c = b - g * (b - a), d = a + g * (b - a);
+    double fc = oracle_gauss_mse(bits, c), fd = oracle_gauss_mse(bits, d);
+    while (b - a > tol) {
+        if (fc < fd) {
+            b = d; d = c; fd = fc;
+            c = b - g * (b - a); fc = oracle_gauss_mse(bits, c);
+        } else {
+            a = c; c = d; fc = fd;
+            d = a + g * (b - a); fd = oracle_gauss_mse(bits, d);
+        }
+    }
+    return 0.5 * (a + b);
+}
+
+/* alpha_b = 2^(b-1) * argmin_delta MSE(delta): the clip edge of the grid.
+ * Also returns the optimal step and the minimal Gaussian MSE. */
+int oracle_alpha(int bits, double* alpha, double* delta_opt, double* mse_opt) {
+    if (bits < 1 || bits > 16) return ORACLE_EINVAL;
+    double d = golden_min(bits, 1e-4, 4.0, 1e-13);
+    if (alpha) *alpha = ldexp(d, bits - 1);
+    if (delta_opt) *delta_opt = d;
+    if (mse_opt) *mse_opt = oracle_gauss_mse(bits, d);
+    return ORACLE_OK;
+}
+
+/* ------------------------------------------------------------------------- */
+/* Forward quantizer.                                                         */
+/* ------------------------------------------------------------------------- */
+
+/* Distance from t to the nearest point where the mask value changes, given
+ * the code cell q(t). Flip points are c +- T/2 (c = q + 1/2) that lie inside
+ * the t-range of their own cell; the element's own cell and both neighbours are
+ * searched. */
+static double mask_flip_distance(double t, int q, int lo, int hi, double trust) {
+    double best = INFINITY;
+    for (int k = q - 1; k <= q + 1; ++k) {
+        if (k < lo || k > hi) continue;
+        double cell_lo = (k == lo) ? -INFINITY : (double)k;
+        double cell_hi = (k == hi) ? INFINITY : (double)(k + 1);
+        double c = k + 0.5;
+        double f[2] = {c - 0.5 * trust, c + 0.5 * trust};
+        for (int s = 0; s < 2; ++s)
+            if (f[s] > cell_lo && f[s] < cell_hi) {
+                double dd = fabs(t - f[s]);
+                if (dd < best) best = dd;
+            }
+    }
+    return best;
+}
+
+/*
+ * Quantizes x [rows, cols] (row stride ld, fp64 values) block by block.
+ *   had       Hadamard block size (power of two), divides cols.
+ *   rms_group RMS group length (multiple of had, divides cols).
+ *   bits      1..8; trust T > 0; alpha the grid clip for this bit-width.
+ * Outputs (all dense, row-major, may be NULL unless stated):
+ *   y      [rows, cols]   transformed values (Hadamard domain)
+ *   t      [rows, cols]   pre-round value y / Delta (0 where Delta == 0)
+ *   q      [rows, cols]   integer code                        (required)
+ *   yhat   [rows, cols]   dequantised value (q + 1/2) Delta, Hadamard domain
+ *   mask   [rows, cols]   1 = gradient kept, 0 = zeroed
+ *   scale  [rows, cols / rms_group]   Delta per group
+ *   d_round [rows, cols]  distance of t to the nearest code decision boundary
+ *   d_mask  [rows, cols]  distance of t to the nearest mask flip point
+ */
+int oracle_quantize(const double* x, int64_t rows, int64_t cols, int64_t ld, int had,
+                    int64_t rms_group, int bits, double trust, double alpha, double* y_out,
+                    double* t_out, int32_t* q, double* yhat, uint8_t* mask, double* scale,
+                    double* d_round, double* d_mask) {
+    if (rows < 0 || cols <= 0 || ld < cols || !is_pow2(had) || cols % had != 0) return ORACLE_EINVAL;
+    if (rms_group <= 0 || rms_group % had != 0 || cols % rms_group != 0) return ORACLE_EINVAL;
+    if (bits < 1 || bits > 8 || !(trust > 0.0) || !(alpha > 0.0) || q == NULL) return ORACLE_EINVAL;
+
+    const int lo = -(1 << (bits - 1)), hi = (1 << (bits - 1)) - 1;
+    const double levels_half = ldexp(1.0, bits - 1);
+    double* H = (double*)malloc(sizeof(double) * had * had);
+    double* y = (double*)malloc(sizeof(double) * cols);
+    if (!H || !y) { free(H); free(y); return ORACLE_EINVAL; }
+    oracle_hadamard(had, H);
+
+    for (int64_t r = 0; r < rows; ++r) {
+        const double* xr = x + r * ld;
+        /* Step 1: blockwise Hadamard transform of the row. */
+        for (int64_t b0 = 0; b0 < cols; b0 += had) hadamard_block(H, had, xr + b0, y + b0);
+
+        for (int64_t g0 = 0; g0 < cols; g0 += rms_group) {
+            /* Step 2: RMS of the transformed values of the group. */
+            double ss = 0.0;
+            for (int64_t j = 0; j < rms_group; ++j) ss += y[g0 + j] * y[g0 + j];
+            double rms = sqrt(ss / (double)rms_group);
+            /* Step 3: Gaussian-fitted step. */
+            double delta = alpha * rms / levels_half;
+            if (scale) scale[r * (cols / rms_group) + g0 / rms_group] = delta;
+            /* Step 4: project onto the grid; step 5: trust mask. */
+            for (int64_t j = 0; j < rms_group; ++j) {
+                int64_t idx = r * cols + g0 + j;
+                double yv = y[g0 + j];
+                double tv, dr, dm;
+                int qv;
+                uint8_t mv;
+                if (delta == 0.0) {
+                    tv = 0.0; qv = 0; mv = 1; dr = INFINITY; dm = INFINITY;
+                } else {
+                    tv = yv / delta;
+                    double fl = floor(tv);
+                    if (fl < lo) fl = lo;
+                    if (fl > hi) fl = hi;
+                    qv = (int)fl;
+                    double err = fabs(tv - (qv + 0.5));
+                    mv = (err <= 0.5 * trust) ? 1 : 0;
+                    /* nearest interior code boundary: integers lo+1 .. hi */
+                    double k = nearbyint(tv);
+                    if (k < lo + 1) k = lo + 1;
+                    if (k > hi) k = hi;
+                    dr = (hi > lo) ? fabs(tv - k) : INFINITY;
+                    dm = mask_flip_distance(tv, qv, lo, hi, trust);
+                }
+                if (y_out) y_out[idx] = yv;
+                if (t_out) t_out[idx] = tv;
+                q[idx] = qv;
+                if (yhat) yhat[idx] = (qv + 0.5) * delta;
+                if (mask) mask[idx] = mv;
+                if (d_round) d_round[idx] = dr;
+                if (d_mask) d_mask[idx] = dm;
+            }
+        }
+    }
+    free(H);
+    free(y);
+    return ORACLE_OK;
+}
+
+/* ------------------------------------------------------------------------- */
+/* Trust backward: g_x = H^T (m . g) / sqrt(n) per Hadamard block.            */
+/* ------------------------------------------------------------------------- */
+
+int oracle_trust_bwd(const double* g, const uint8_t* mask, int64_t rows, int64_t cols, int had,
+                     double* gx) {
+    if (rows < 0 || cols <= 0 || !is_pow2(had) || cols % had != 0) return ORACLE_EINVAL;
+    double* H = (double*)malloc(sizeof(double) * had * had);
+    double* mg = (double*)malloc(sizeof(double) * had);
+    if (!H || !mg) { free(H); free(mg); return ORACLE_EINVAL; }
+    oracle_hadamard(had, H);
+    const double norm = 1.0 / sqrt((double)had);
+    for (int64_t r = 0; r < rows; ++r)
+        for (int64_t b0 = 0; b0 < cols; b0 += had) {
+            const int64_t base = r * cols + b0;
+            for (int j = 0; j < had; ++j) mg[j] = mask[base + j] ? g[base + j] : 0.0;
+            /* transpose product: out[i] = sum_j H[j][i] * mg[j] */
+            for (int i = 0; i < had; ++i) {
+                double acc = 0.0;
+                for (int j = 0; j < had; ++j) acc += H[(int64_t)j * had + i] * mg[j];
+                gx[base + i] = acc * norm;
+            }
+        }
+    free(H);
+    free(mg);
+    return ORACLE_OK;
+}
+
+/* ------------------------------------------------------------------------- */
+/* Integer linear layer.                                                      */
+/* ------------------------------------------------------------------------- */
+
+/* acc[m][n] = sum_k A[m][k] * B[n][k]  (A: [M,K], B: [N,K], both K-contiguous). */
+int oracle_gemm_i8(const int8_t* A, const int8_t* B, int64_t M, int64_t N, int64_t K,
+                   int64_t* acc) {
+    if (M < 0 || N < 0 || K < 0) return ORACLE_EINVAL;
+    for (int64_t m = 0; m < M; ++m)
+        for (int64_t n = 0; n < N; ++n) {
+            int64_t s = 0;
+            for (int64_t k = 0; k < K; ++k) s += (int64_t)A[m * K + k] * (int64_t)B[n * K + k];
+            acc[m * N + n] = s;
+        }
+    return ORACLE_OK;
+}
+
+/* Y[m][n] = acc[m][n] * (Delta_a[m] / 2) * (Delta_b[n] / 2): the c = 2q+1 codes
+ * carry a factor 2 each relative to (q + 1/2). */
+int oracle_dequant_linear(const int64_t* acc, const double* delta_a, const double* delta_b,
+                          int64_t M, int64_t N, double* y) {
+    if (M < 0 || N < 0) return ORACLE_EINVAL;
+    for (int64_t m = 0; m < M; ++m)
+        for (int64_t n = 0; n < N; ++n)
+            y[m * N + n] = (double)acc[m * N + n] * (delta_a[m] * 0.5) * (delta_b[n] * 0.5);
+    return ORACLE_OK;
+}
+
+/* ------------------------------------------------------------------------- */
+/* Rounding of an fp64 value to bfloat16, round-to-nearest-even, one rounding. */
+/* ------------------------------------------------------------------------- */
+
+uint16_t oracle_bf16_rne(double v) {
+    if (isnan(v)) return 0x7FC0;
+    uint16_t sign = signbit(v) ? 0x8000 : 0;
+    double a = fabs(v);
+    if (isinf(a)) return sign | 0x7F80;
+    if (a == 0.0) return sign;
+    /* quantum of the bf16 grid at this magnitude: 8 significant bits for
+     * normals (|a| >= 2^-126), fixed 2^-133 for subnormals. */
+    int e;
+    frexp(a, &e); /* a = f * 2^e, f in [0.5, 1) */
+    double quantum = (a >= ldexp(1.0, -126)) ? ldexp(1.0, e - 8) : ldexp(1.0, -133);
+    double k = a / quantum;              /* exact: quantum is a power of two */
+    double kr = nearbyint(k);            /* default mode: ties to even */
+    double rv = kr * quantum;
+    if (rv >= ldexp(1.0, 128)) return sign | 0x7F80;
+    float f = (float)rv;                 /* exact: rv has <= 8 significant bits */
+    uint32_t bits;
+    memcpy(&bits, &f, sizeof bits);
+    return (uint16_t)(sign | (uint16_t)((bits >> 16) & 0x7FFF));
+}
+
+void oracle_bf16_rne_array(const double* v, int64_t n, uint16_t* out) {
+    for (int64_t i = 0; i < n; ++i) out[i] = oracle_bf16_rne(v[i]);
+}
