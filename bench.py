@@ -1,0 +1,489 @@
+#!/usr/bin/env python3
+"""Benchmark of the QuEST hot path on B200: one step = one pass of the whole path
+over one batch of the activation workload.
+
+Step (all kernels of libquest_b200.so, on one CUDA stream):
+  1. quest_quantize_fwd   X [16384, 2048] bf16 -> 4-bit codes, trust mask bits,
+                          per-128-group scales (the QAT forward quantizer)
+  2. quest_trust_bwd      G [16384, 2048] bf16 + that mask -> grad_in bf16
+  3. quest_quantize_fwd   X -> int8 operand codes, one scale per row
+  4. quest_quantize_fwd   W_up [5632, 2048] -> int8 operand codes, one scale per row
+  5. quest_w4a4_linear    Y [16384, 5632] bf16 = dequant(cX @ cW^T)
+
+Metric: algorithmic GB/s of the whole step (bytes every kernel must move: inputs
+read once, outputs written once) and, per part, GB/s as a fraction of the
+measured HBM copy bandwidth or int8 TOPS as a fraction of the int8 tensor peak.
+Multi-GPU: every rank runs its own full workload (the path shards by rows with
+no exchange), weak scaling, time = max over ranks.
+
+``--impl reference`` times the CPU oracle (single-threaded C, fp64) on a bounded
+row sample of the same step instead.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+BITS = 4
+HB = 128
+R, C = 16384, 2048          # activation / gradient tensors
+NW = 5632                   # up-projection width (8/3 * 2048 padded to 256)
+L2_FLUSH_BYTES = 512 << 20  # written between steps (L2 is 126 MB)
+METRIC = "QuEST quantizer GB/s (frac of HBM peak); W4A4 linear TOPS (frac of int8 TC)"
+WORKLOAD = ("QuEST hot path on the 16384x2048 bf16 activation workload (Student-t nu=3, "
+            "16 outlier channels x20), b=4, Hadamard block 128: quantize_fwd with trust mask "
+            "(RMS per 128-group) + trust backward on a 16384x2048 N(0,1e-6) gradient + W4A4 "
+            "linear vs the 5632x2048 up-projection (operands quantized with one RMS per row)")
+
+
+def part_bytes():
+    """Algorithmic bytes per step for each kernel (inputs read once, outputs written once)."""
+    e = R * C
+    return {
+        "quantize_fwd": 2 * e + e // 2 + e // 8 + 4 * (e // HB),       # bf16 in, 4-bit codes, mask bits, scales
+        "trust_bwd": 2 * e + e // 8 + 2 * e,                           # grad in, mask in, grad out
+        "quantize_operand_x": 2 * e + e + 4 * R,                       # bf16 in, int8 codes, row scales
+        "quantize_operand_w": 3 * NW * C + 4 * NW,
+        "w4a4_linear": R * C + NW * C + 4 * (R + NW) + 2 * R * NW,     # codes, scales in, bf16 out
+    }
+
+
+GEMM_OPS = 2 * R * NW * C
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return {"hbm_gbs": float(p["hbm_gbs"]), "bf16_tflops": float(p["bf16_tflops"]),
+                "bf16_tflops_sustained": float(p.get("bf16_tflops_sustained", p["bf16_tflops"])),
+                "source": "measured"}
+    except Exception:
+        return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+                "source": "fallback"}
+
+
+# ---------------------------------------------------------------------------
+# clocks during the timed region (NVML, polled from a thread)
+# ---------------------------------------------------------------------------
+class ClockSampler:
+    def __init__(self, torch_device_index, period_s=0.01):
+        self.period = period_s
+        self.samples = []
+        self.max_mhz = None
+        self._stop = threading.Event()
+        self._thr = None
+        self.ok = False
+        try:
+            import pynvml
+            import torch
+            pynvml.nvmlInit()
+            props = torch.cuda.get_device_properties(torch_device_index)
+            handle = None
+            try:
+                bus = f"{props.pci_domain_id:08X}:{props.pci_bus_id:02X}:{props.pci_device_id:02X}.0"
+                handle = pynvml.nvmlDeviceGetHandleByPciBusId(bus)
+            except Exception:
+                handle = pynvml.nvmlDeviceGetHandleByIndex(torch_device_index)
+            self.nv = pynvml
+            self.h = handle
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(handle, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception as e:  # no NVML: report that instead of guessing
+            self.err = str(e)
+
+    def _run(self):
+        nv = self.nv
+        while not self._stop.is_set():
+            try:
+                mhz = nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM)
+                rs = nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                self.samples.append((mhz, rs))
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def start(self):
+        if self.ok:
+            self._thr = threading.Thread(target=self._run, daemon=True)
+            self._thr.start()
+
+    def stop(self):
+        if self._thr:
+            self._stop.set()
+            self._thr.join()
+
+    def summary(self):
+        if not self.ok:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "note": "NVML unavailable"}
+        nv = self.nv
+        names = {
+            "gpu_idle": nv.nvmlClocksEventReasonGpuIdle,
+            "applications_clocks_setting": nv.nvmlClocksEventReasonApplicationsClocksSetting,
+            "sw_power_cap": nv.nvmlClocksEventReasonSwPowerCap,
+            "hw_slowdown": nv.nvmlClocksEventReasonHwSlowdown,
+            "sync_boost": nv.nvmlClocksEventReasonSyncBoost,
+            "sw_thermal_slowdown": nv.nvmlClocksEventReasonSwThermalSlowdown,
+            "hw_thermal_slowdown": nv.nvmlClocksEventReasonHwThermalSlowdown,
+            "hw_power_brake_slowdown": nv.nvmlClocksEventReasonHwPowerBrakeSlowdown,
+        }
+        reasons = set()
+        for _, rs in self.samples:
+            for n, bit in names.items():
+                if rs & bit and n != "gpu_idle":
+                    reasons.add(n)
+        mhz = [m for m, _ in self.samples]
+        return {"sm_mhz": statistics.median(mhz) if mhz else None, "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(reasons), "samples": len(mhz)}
+
+
+# ---------------------------------------------------------------------------
+# distributed plumbing (timing only; the data path has no collective)
+# ---------------------------------------------------------------------------
+def dist_setup(n_gpus):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import torch.distributed as dist
+        import torch
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    return world, rank, local
+
+
+def dist_max(value, world):
+    if world == 1:
+        return value
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([value], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def dist_barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+# ---------------------------------------------------------------------------
+# the B200 arm
+# ---------------------------------------------------------------------------
+class Step:
+    """Buffers and launches of one step of the hot path (device-resident inputs)."""
+
+    def __init__(self, dev, x, g, w):
+        import torch
+        import bit_quantization_aware_blockwise_b200 as q
+        self.q, self.torch = q, torch
+        self.dev = dev
+        self.x, self.g, self.w = x, g, w
+        e = R * C
+        u8 = torch.uint8
+        self.codes = torch.empty(q.codes_bytes(R, C, BITS), dtype=u8, device=dev)
+        self.scales = torch.empty((R, C // HB), dtype=torch.float32, device=dev)
+        self.mask = torch.empty(e // 8, dtype=u8, device=dev)
+        self.grad_in = torch.empty((R, C), dtype=torch.bfloat16, device=dev)
+        self.cx = torch.empty((R, C), dtype=torch.int8, device=dev)
+        self.sx = torch.empty((R, 1), dtype=torch.float32, device=dev)
+        self.cw = torch.empty((NW, C), dtype=torch.int8, device=dev)
+        self.sw = torch.empty((NW, 1), dtype=torch.float32, device=dev)
+        self.y = torch.empty((R, NW), dtype=torch.bfloat16, device=dev)
+        self.launches_per_step = 5
+
+    def parts(self, stream):
+        """The five launches, each a zero-argument callable (raw C-ABI calls)."""
+        q, s = self.q, stream.cuda_stream
+        x, g, w = self.x, self.g, self.w
+        return [
+            ("quantize_fwd", lambda: q.quantize_fwd_raw(
+                x.data_ptr(), 0, R, C, C, BITS, HB, HB, 1.0, q.CODES_PACKED, self.codes.data_ptr(),
+                self.scales.data_ptr(), q.MASK_BITS, self.mask.data_ptr(), None, 0, s)),
+            ("trust_bwd", lambda: q.trust_bwd_raw(
+                g.data_ptr(), self.mask.data_ptr(), q.MASK_BITS, R, C, HB, self.grad_in.data_ptr(), s)),
+            ("quantize_operand_x", lambda: q.quantize_fwd_raw(
+                x.data_ptr(), 0, R, C, C, BITS, HB, C, 1.0, q.CODES_GEMM_OPERAND, self.cx.data_ptr(),
+                self.sx.data_ptr(), q.MASK_BITS, None, None, 0, s)),
+            ("quantize_operand_w", lambda: q.quantize_fwd_raw(
+                w.data_ptr(), 0, NW, C, C, BITS, HB, C, 1.0, q.CODES_GEMM_OPERAND, self.cw.data_ptr(),
+                self.sw.data_ptr(), q.MASK_BITS, None, None, 0, s)),
+            ("w4a4_linear", lambda: q.w4a4_linear_raw(
+                self.cx.data_ptr(), self.sx.data_ptr(), self.cw.data_ptr(), self.sw.data_ptr(),
+                R, NW, C, self.y.data_ptr(), None, s)),
+        ]
+
+
+def run_b200(args, world, rank, local):
+    import torch
+    import bit_quantization_aware_blockwise_b200 as q
+    from bit_quantization_aware_blockwise_b200 import inputs
+
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    q.load_library()
+    peaks = load_peaks()
+    x_cpu = inputs.activation_input()
+    g_cpu = inputs.grad_input()
+    w_cpu = inputs.weight_up()
+    x, g, w = x_cpu.to(dev), g_cpu.to(dev), w_cpu.to(dev)
+    step = Step(dev, x, g, w)
+    stream = torch.cuda.current_stream(dev)
+    parts = step.parts(stream)
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    names = [n for n, _ in parts]
+
+    def one_step(evs=None):
+        for i, (_, f) in enumerate(parts):
+            if evs is not None:
+                evs[i][0].record(stream)
+            f()
+            if evs is not None:
+                evs[i][1].record(stream)
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        one_step()
+    torch.cuda.synchronize()
+    q.device_status()
+
+    evs = [[[torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)]
+            for _ in parts] for _ in range(args.steps)]
+    clocks = ClockSampler(local)
+    dist_barrier(world)
+    torch.cuda.synchronize()
+    clocks.start()
+    t0 = time.perf_counter()
+    for k in range(args.steps):
+        flush.zero_()  # L2 flush between timed steps (outside the per-step events)
+        one_step(evs[k])
+    torch.cuda.synchronize()
+    wall = time.perf_counter() - t0
+    clocks.stop()
+    dist_barrier(world)
+    q.device_status()
+
+    part_ms = {n: [] for n in names}
+    step_ms = []
+    for k in range(args.steps):
+        tot = 0.0
+        for i, n in enumerate(names):
+            t = evs[k][i][0].elapsed_time(evs[k][i][1])
+            part_ms[n].append(t)
+            tot += t
+        step_ms.append(tot)
+    my_ms = sum(step_ms) / args.steps
+    ms = dist_max(my_ms, world)
+    pbytes = part_bytes()
+    step_bytes = sum(pbytes.values())
+    value = step_bytes * world / (ms * 1e-3) / 1e9
+
+    hbm = peaks["hbm_gbs"]
+    int8_peak = peaks["bf16_tflops"] * 2.0   # nominal int8 : bf16 dense ratio 4.5 : 2.25
+    breakdown = {}
+    for n in names:
+        m = statistics.median(part_ms[n])
+        d = {"ms": round(m, 5), "gbs": round(pbytes[n] / (m * 1e-3) / 1e9, 1)}
+        d["frac_hbm"] = round(d["gbs"] / hbm, 4)
+        if n == "w4a4_linear":
+            d["tops"] = round(GEMM_OPS / (m * 1e-3) / 1e12, 1)
+            d["frac_int8_peak"] = round(d["tops"] / int8_peak, 4)
+        breakdown[n] = d
+    dominant = max(names, key=lambda n: breakdown[n]["ms"])
+    avg = {n: sum(part_ms[n]) / len(part_ms[n]) for n in names}
+    if dominant == "w4a4_linear":
+        achieved = GEMM_OPS / (avg[dominant] * 1e-3) / 1e12
+        roofline = {"kernel": "w4a4_gemm_kernel", "bound": "tensor", "achieved": round(achieved, 1),
+                    "peak": round(int8_peak, 1), "unit": "TOPS",
+                    "frac": round(achieved / int8_peak, 4),
+                    "peak_source": f"{peaks['source']} bf16 burst x 2 (nominal int8/bf16 dense ratio)",
+                    "traffic": None}
+    else:
+        achieved = pbytes[dominant] / (avg[dominant] * 1e-3) / 1e9
+        roofline = {"kernel": dominant, "bound": "hbm", "achieved": round(achieved, 1),
+                    "peak": hbm, "unit": "GB/s", "frac": round(achieved / hbm, 4),
+                    "peak_source": peaks["source"], "traffic": None}
+
+    # ---- end to end: pinned host inputs -> device, the step, results -> host
+    e2e = None
+    if not args.no_e2e:
+        e2e = run_e2e(args, dev, step, parts, x_cpu, g_cpu, w_cpu, flush, world)
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(args)
+
+    result = {
+        "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 5),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "fp32 math on bf16 I/O; int8 x int8 -> int32 tensor cores", "data": "synthetic",
+        "config": {"workload": WORKLOAD, "bits": BITS, "had_block": HB,
+                   "shapes": {"x": [R, C], "grad": [R, C], "w_up": [NW, C], "y": [R, NW]},
+                   "l2": f"flushed between timed steps ({L2_FLUSH_BYTES >> 20} MiB write, untimed)",
+                   "parallelism": f"dp{world} (independent row shards, no collective)"},
+        "parts": breakdown,
+        "w4a4_tops": breakdown["w4a4_linear"]["tops"],
+        "roofline": roofline,
+        "gpu_launches": step.launches_per_step * args.steps,
+        "clocks": clocks.summary(),
+        "wall_s_timed_loop": round(wall, 4),
+        "e2e": e2e,
+        "cpu_baseline": cpu,
+    }
+    if rank == 0:
+        print(json.dumps(result), flush=True)
+
+
+def run_e2e(args, dev, step, parts, x_cpu, g_cpu, w_cpu, flush, world):
+    import torch
+    xp, gp, wp = x_cpu.pin_memory(), g_cpu.pin_memory(), w_cpu.pin_memory()
+    outs = [step.codes, step.scales, step.mask, step.grad_in, step.y]
+    host_outs = [torch.empty(o.shape, dtype=o.dtype, pin_memory=True) for o in outs]
+    stream = torch.cuda.current_stream(dev)
+
+    def e2e_step():
+        step.x.copy_(xp, non_blocking=True)
+        step.g.copy_(gp, non_blocking=True)
+        step.w.copy_(wp, non_blocking=True)
+        for _, f in parts:
+            f()
+        for h, o in zip(host_outs, outs):
+            h.copy_(o, non_blocking=True)
+
+    n = max(3, min(args.steps, 10))
+    for _ in range(2):
+        e2e_step()
+    torch.cuda.synchronize()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(n)]
+    dist_barrier(world)
+    for k in range(n):
+        flush.zero_()
+        ev[k][0].record(stream)
+        e2e_step()
+        ev[k][1].record(stream)
+    torch.cuda.synchronize()
+    ms = sum(a.elapsed_time(b) for a, b in ev) / n
+    ms = dist_max(ms, world)
+    h2d = sum(t.numel() * t.element_size() for t in (x_cpu, g_cpu, w_cpu))
+    d2h = sum(o.numel() * o.element_size() for o in outs)
+    value = sum(part_bytes().values()) * world / (ms * 1e-3) / 1e9
+    return {"value": round(value, 2), "unit": "GB/s", "ms_per_step": round(ms, 4),
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": n,
+            "path": "pinned host -> cudaMemcpyAsync -> quest_* C-ABI calls -> pinned host"}
+
+
+# ---------------------------------------------------------------------------
+# CPU oracle (cpu_baseline leg and the reference arm)
+# ---------------------------------------------------------------------------
+def oracle_sample(rows_x=256, rows_w=88, gemm_rows=16):
+    """Runs the oracle on a bounded row sample of one step; returns (seconds, bytes)."""
+    import oracle
+    from bit_quantization_aware_blockwise_b200 import inputs
+    x = inputs.to_f64(inputs.activation_input(rows=rows_x))
+    g = inputs.to_f64(inputs.grad_input(rows=rows_x))
+    w = inputs.to_f64(inputs.weight_up(rows=rows_w))
+    w_full_rows = NW
+    t0 = time.perf_counter()
+    o = oracle.quantize(x, bits=BITS, had=HB)
+    oracle.trust_bwd(g, o["mask"], had=HB)
+    ox = oracle.quantize(x, bits=BITS, had=HB, rms_group=C)
+    ow = oracle.quantize(w, bits=BITS, had=HB, rms_group=C)
+    cx = (2 * ox["q"][:gemm_rows] + 1).astype(np.int8)
+    cw = (2 * ow["q"] + 1).astype(np.int8)
+    # the GEMM sample: gemm_rows output rows against all NW weight rows (codes of the
+    # sampled weight rows are tiled to the full width: the cost is the triple loop)
+    cw_full = np.resize(cw, (w_full_rows, C))
+    acc = oracle.gemm_i8(cx, cw_full)
+    sw = np.resize(ow["scale"][:, 0], w_full_rows)
+    oracle.dequant_linear(acc, ox["scale"][:gemm_rows, 0], sw)
+    dt = time.perf_counter() - t0
+    e = rows_x * C
+    nbytes = ((2 * e + e // 2 + e // 8 + 4 * (e // HB)) + (2 * e + e // 8 + 2 * e) + (3 * e + 4 * rows_x)
+              + (3 * rows_w * C + 4 * rows_w)
+              + (gemm_rows * C + NW * C + 4 * (gemm_rows + NW) + 2 * gemm_rows * NW))
+    sample = (f"oracle on {rows_x} activation/gradient rows (quantize + trust backward + operand "
+              f"quantize), {rows_w} weight rows, and a {gemm_rows}x{NW}x{C} GEMM block; "
+              f"single-threaded C, fp64/int64")
+    return dt, nbytes, sample
+
+
+def cpu_baseline(args):
+    import oracle
+    oracle.build()
+    dt, nbytes, sample = oracle_sample()
+    return {"value": round(nbytes / dt / 1e9, 5), "unit": "GB/s", "cores": 1, "kind": "oracle",
+            "sample": sample, "seconds": round(dt, 3)}
+
+
+def run_reference(args, world, rank):
+    if rank != 0:
+        return
+    import oracle
+    oracle.build()
+    times, nb, sample = [], 0, ""
+    for _ in range(max(args.warmup, 0) and 1):
+        oracle_sample(rows_x=64, rows_w=22, gemm_rows=4)
+    for _ in range(args.steps):
+        dt, nb, sample = oracle_sample(rows_x=64, rows_w=22, gemm_rows=4)
+        times.append(dt)
+    ms = 1e3 * sum(times) / len(times)
+    value = nb / (ms * 1e-3) / 1e9
+    line = {
+        "impl": "reference", "metric": METRIC, "value": round(value, 5), "unit": "GB/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 3),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "f64/int64 (CPU oracle)", "data": "synthetic",
+        "config": {"workload": WORKLOAD, "bits": BITS, "had_block": HB,
+                   "note": "each step is a bounded row sample of the workload"},
+        "cpu_baseline": {"value": round(value, 5), "unit": "GB/s", "cores": 1, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": round(value, 5), "unit": "GB/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+        "gpu_launches": 0,
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["b200", "reference"], default="b200")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3 and args.impl == "b200":
+        args.warmup = 3
+    world, rank, local = (int(os.environ.get("WORLD_SIZE", "1")), int(os.environ.get("RANK", "0")),
+                          int(os.environ.get("LOCAL_RANK", "0")))
+    if args.impl == "reference":
+        run_reference(args, world, rank)
+        return
+    world, rank, local = dist_setup(args.gpus)
+    try:
+        run_b200(args, world, rank, local)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

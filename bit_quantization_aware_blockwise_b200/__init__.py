@@ -1,0 +1,36 @@
+"""QuEST quantizer hot path on B200 (sm_100a).
+
+The product is the C-ABI library ``libquest_b200.so`` (declared in
+``include/quest.h``); this package is its thin Python binding. Importing the
+package loads nothing: the library is loaded on first use, and every call fails
+loudly (``QuestError``) when it is missing or no CUDA device is present. There
+is no CPU fallback.
+"""
+from ._binding import (  # noqa: F401
+    QuestError,
+    CODES_PACKED,
+    CODES_INT8,
+    CODES_GEMM_OPERAND,
+    MASK_BITS,
+    MASK_BYTES,
+    library_path,
+    load_library,
+    alpha,
+    codes_bytes,
+    mask_bytes,
+    container_bits,
+    quantize_fwd,
+    trust_bwd,
+    w4a4_linear,
+    quantize_fwd_raw,
+    trust_bwd_raw,
+    w4a4_linear_raw,
+    device_status,
+)
+
+__all__ = [
+    "QuestError", "CODES_PACKED", "CODES_INT8", "CODES_GEMM_OPERAND", "MASK_BITS",
+    "MASK_BYTES", "library_path", "load_library", "alpha", "codes_bytes", "mask_bytes",
+    "container_bits", "quantize_fwd", "trust_bwd", "w4a4_linear", "quantize_fwd_raw",
+    "trust_bwd_raw", "w4a4_linear_raw", "device_status",
+]

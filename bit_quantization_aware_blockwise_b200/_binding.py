@@ -1,0 +1,230 @@
+"""ctypes binding of ``libquest_b200.so`` (see ``include/quest.h``).
+
+Argument marshalling only: every step of the quantizer, trust backward and
+integer linear layer runs in the library's CUDA kernels. PyTorch supplies
+device memory and the current stream. The library is loaded on first use; if
+it is missing, or a call fails, ``QuestError`` is raised. There is no fallback.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_LIB_NAME = "libquest_b200.so"
+
+CODES_PACKED, CODES_INT8, CODES_GEMM_OPERAND = 0, 1, 2
+MASK_BITS, MASK_BYTES = 0, 1
+BF16, FP32 = 0, 1
+_STATUS = {0: "ok", 1: "invalid argument", 2: "unsupported", 3: "CUDA error", 4: "device wait timed out"}
+
+# Every symbol the header declares, with (restype, argtypes).
+_p, _i64, _int, _f32, _f64, _sz = (ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_float,
+                                   ctypes.c_double, ctypes.c_size_t)
+SIGNATURES = {
+    "quest_quantize_fwd": (_int, [_p, _int, _i64, _i64, _i64, _int, _int, _i64, _f32, _int, _p, _p,
+                                  _int, _p, _p, _int, _p]),
+    "quest_trust_bwd": (_int, [_p, _p, _int, _i64, _i64, _int, _p, _p]),
+    "quest_w4a4_linear": (_int, [_p, _p, _p, _p, _i64, _i64, _i64, _p, _p, _p]),
+    "quest_device_status": (_int, [_p]),
+    "quest_alpha": (_f64, [_int]),
+    "quest_container_bits": (_int, [_int]),
+    "quest_codes_bytes": (_sz, [_i64, _i64, _int, _int]),
+    "quest_mask_bytes": (_sz, [_i64, _i64, _int]),
+    "quest_status_string": (ctypes.c_char_p, [_int]),
+    "quest_last_error_message": (ctypes.c_char_p, []),
+    "quest_version": (_int, []),
+}
+
+_lock = threading.Lock()
+_lib = None
+
+
+class QuestError(RuntimeError):
+    """A quest_* call failed (or the library could not be loaded)."""
+
+    def __init__(self, msg, status=None):
+        super().__init__(msg)
+        self.status = status
+
+
+def library_path() -> str:
+    return os.environ.get("QUEST_B200_LIB", os.path.join(_HERE, _LIB_NAME))
+
+
+def load_library():
+    """Load the library (once). Raises QuestError if it is not built."""
+    global _lib
+    with _lock:
+        if _lib is not None:
+            return _lib
+        path = library_path()
+        if not os.path.exists(path):
+            raise QuestError(f"{path} not found: build it with "
+                             "`python -m bit_quantization_aware_blockwise_b200.build`")
+        try:
+            lib = ctypes.CDLL(path)
+        except OSError as e:
+            raise QuestError(f"cannot load {path}: {e}") from e
+        for name, (res, args) in SIGNATURES.items():
+            f = getattr(lib, name)
+            f.restype = res
+            f.argtypes = args
+        _lib = lib
+        return lib
+
+
+def _check(status: int, what: str):
+    if status != 0:
+        detail = load_library().quest_last_error_message().decode(errors="replace")
+        raise QuestError(f"{what}: {_STATUS.get(status, status)}: {detail}", status)
+
+
+# ---------------------------------------------------------------------------
+# Raw entry points (integer device pointers and stream handle)
+# ---------------------------------------------------------------------------
+
+def quantize_fwd_raw(x, x_dtype, rows, cols, ld_x, bits, had_block, rms_group, trust, code_mode,
+                     codes, scales, mask_mode, mask, dequant, dequant_dtype, stream=0):
+    _check(load_library().quest_quantize_fwd(x, x_dtype, rows, cols, ld_x, bits, had_block,
+                                             rms_group, trust, code_mode, codes, scales,
+                                             mask_mode, mask, dequant, dequant_dtype, stream),
+           "quest_quantize_fwd")
+
+
+def trust_bwd_raw(grad_out, mask, mask_mode, rows, cols, had_block, grad_in, stream=0):
+    _check(load_library().quest_trust_bwd(grad_out, mask, mask_mode, rows, cols, had_block,
+                                          grad_in, stream), "quest_trust_bwd")
+
+
+def w4a4_linear_raw(a_codes, a_scales, w_codes, w_scales, M, N, K, y, acc=None, stream=0):
+    _check(load_library().quest_w4a4_linear(a_codes, a_scales, w_codes, w_scales, M, N, K, y, acc,
+                                            stream), "quest_w4a4_linear")
+
+
+def device_status(stream=0):
+    """Synchronise ``stream`` and raise QuestError if a bounded device wait gave up."""
+    _check(load_library().quest_device_status(stream), "quest_device_status")
+
+
+def alpha(bits: int) -> float:
+    return float(load_library().quest_alpha(bits))
+
+
+def container_bits(bits: int) -> int:
+    return int(load_library().quest_container_bits(bits))
+
+
+def codes_bytes(rows: int, cols: int, bits: int, code_mode: int = CODES_PACKED) -> int:
+    return int(load_library().quest_codes_bytes(rows, cols, bits, code_mode))
+
+
+def mask_bytes(rows: int, cols: int, mask_mode: int = MASK_BITS) -> int:
+    return int(load_library().quest_mask_bytes(rows, cols, mask_mode))
+
+
+# ---------------------------------------------------------------------------
+# torch-tensor wrappers (allocate outputs with torch, pass pointers)
+# ---------------------------------------------------------------------------
+
+def _torch():
+    import torch
+    return torch
+
+
+def _stream_handle(stream, device):
+    torch = _torch()
+    s = stream if stream is not None else torch.cuda.current_stream(device)
+    return s.cuda_stream
+
+
+def _require_cuda(t, name):
+    if not t.is_cuda:
+        raise QuestError(f"{name} must be a CUDA tensor (there is no CPU path)")
+
+
+def quantize_fwd(x, bits: int, had_block: int = 128, rms_group: int | None = None,
+                 trust: float = 1.0, code_mode: int = CODES_PACKED, mask_mode: int | None = MASK_BITS,
+                 dequant: str | None = None, out: dict | None = None, stream=None) -> dict:
+    """Quantize the rows of a 2-D CUDA tensor ``x`` (bf16 or fp32, unit stride along
+    columns). Returns ``{"codes", "scales", "mask", "dequant"}`` (mask/dequant None
+    when not requested). ``rms_group`` defaults to ``had_block``; pass ``x.shape[1]``
+    for one RMS per row. Outputs may be supplied in ``out`` to avoid allocation."""
+    torch = _torch()
+    _require_cuda(x, "x")
+    if x.dim() != 2 or x.stride(1) != 1:
+        raise QuestError("x must be 2-D with unit column stride")
+    if x.dtype == torch.bfloat16:
+        xd = BF16
+    elif x.dtype == torch.float32:
+        xd = FP32
+    else:
+        raise QuestError("x must be bfloat16 or float32")
+    rows, cols = x.shape
+    rms_group = had_block if rms_group is None else int(rms_group)
+    out = {} if out is None else out
+    dev = x.device
+    codes = out.get("codes")
+    if codes is None:
+        codes = torch.empty(max(codes_bytes(rows, cols, bits, code_mode), 1), dtype=torch.uint8, device=dev)
+    scales = out.get("scales")
+    if scales is None:
+        scales = torch.empty((rows, cols // rms_group if rms_group else 0), dtype=torch.float32, device=dev)
+    mask = out.get("mask")
+    if mask is None and mask_mode is not None:
+        mask = torch.empty(max(mask_bytes(rows, cols, mask_mode), 1), dtype=torch.uint8, device=dev)
+    deq = out.get("dequant")
+    deq_dtype = BF16
+    if dequant is not None:
+        deq_dtype = BF16 if dequant == "bf16" else FP32
+        if deq is None:
+            deq = torch.empty((rows, cols), dtype=torch.bfloat16 if deq_dtype == BF16 else torch.float32,
+                              device=dev)
+    quantize_fwd_raw(x.data_ptr(), xd, rows, cols, x.stride(0) if rows > 1 else cols, bits,
+                     had_block, rms_group, float(trust), code_mode, codes.data_ptr(),
+                     scales.data_ptr(), MASK_BITS if mask_mode is None else mask_mode,
+                     mask.data_ptr() if mask is not None else None,
+                     deq.data_ptr() if deq is not None else None, deq_dtype,
+                     _stream_handle(stream, dev))
+    return {"codes": codes, "scales": scales, "mask": mask, "dequant": deq}
+
+
+def trust_bwd(grad_out, mask, had_block: int = 128, mask_mode: int = MASK_BITS, out=None,
+              stream=None):
+    """grad_in = H (m * grad_out) / sqrt(n) per block; bf16 in and out."""
+    torch = _torch()
+    _require_cuda(grad_out, "grad_out")
+    _require_cuda(mask, "mask")
+    if grad_out.dtype != torch.bfloat16 or grad_out.dim() != 2 or not grad_out.is_contiguous():
+        raise QuestError("grad_out must be a contiguous 2-D bfloat16 tensor")
+    rows, cols = grad_out.shape
+    if out is None:
+        out = torch.empty_like(grad_out)
+    trust_bwd_raw(grad_out.data_ptr(), mask.data_ptr(), mask_mode, rows, cols, had_block,
+                  out.data_ptr(), _stream_handle(stream, grad_out.device))
+    return out
+
+
+def w4a4_linear(a_codes, a_scales, w_codes, w_scales, out=None, acc: bool = False, stream=None):
+    """y = bf16((a_codes @ w_codes^T) * (a_scales/2)[:, None] * (w_scales/2)[None, :]).
+    Codes are int8 [M, K] and [N, K]; returns y (and the int32 accumulator if acc)."""
+    torch = _torch()
+    for t, n in ((a_codes, "a_codes"), (w_codes, "w_codes"), (a_scales, "a_scales"), (w_scales, "w_scales")):
+        _require_cuda(t, n)
+    if a_codes.dtype not in (torch.int8, torch.uint8) or w_codes.dtype not in (torch.int8, torch.uint8):
+        raise QuestError("codes must be int8")
+    if not (a_codes.is_contiguous() and w_codes.is_contiguous()):
+        raise QuestError("codes must be contiguous")
+    M, K = a_codes.shape
+    N, K2 = w_codes.shape
+    if K != K2:
+        raise QuestError("a_codes and w_codes disagree on K")
+    dev = a_codes.device
+    if out is None:
+        out = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+    acc_t = torch.empty((M, N), dtype=torch.int32, device=dev) if acc else None
+    w4a4_linear_raw(a_codes.data_ptr(), a_scales.data_ptr(), w_codes.data_ptr(), w_scales.data_ptr(),
+                    M, N, K, out.data_ptr(), acc_t.data_ptr() if acc_t is not None else None,
+                    _stream_handle(stream, dev))
+    return (out, acc_t) if acc else out

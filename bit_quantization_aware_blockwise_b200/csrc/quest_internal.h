@@ -1,0 +1,68 @@
+// Internal (non-ABI) declarations shared by the host entry points and the
+// kernel launchers.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "quest.h"
+
+namespace quest {
+
+// Per-call constants of the forward quantizer (host-computed, passed by value).
+struct QuantConsts {
+    float c_delta;      // alpha_b / 2^(b-1): Delta = c_delta * r
+    float inv_count;    // 1 / (HB * G): mean of the normalised y^2 = sum(y_u^2) * inv_count
+    float sqrt_hb;      // sqrt(HB): y = y_u / sqrt(HB)
+    float edge;         // 2^(b-1) + (T-1)/2: for T >= 1, m = [|t| <= edge]
+    float half_trust;   // T / 2 (general mask rule)
+    float s_lo, s_hi;   // kMagic + lo, kMagic + hi (clamp bounds of the biased code)
+    uint32_t pack_mult; // 1, or 2 for the c = 2q+1 operand form
+    uint32_t pack_add;  // additive constant of the modular packing (see quantize_fwd.cu)
+    uint32_t pack_xor;  // un-biasing mask of the packed word
+    int trust_ge1;      // 1: use m = [|t| <= edge]
+    int mask_mode;      // -1 none, 0 bits, 1 bytes
+    int deq_mode;       // -1 none, 0 bf16, 1 fp32
+};
+
+struct QuantArgs {
+    const char* x;
+    int64_t ld_x_bytes;      // row pitch of x in bytes
+    int64_t rows, cols;
+    int dense;               // 1 when x rows are contiguous (ld == cols)
+    uint8_t* codes;
+    int64_t codes_row_bytes;
+    float* scales;
+    uint8_t* mask;
+    int64_t mask_row_bytes;
+    uint8_t* deq;
+    int64_t deq_row_bytes;
+    QuantConsts c;
+};
+
+struct TrustArgs {
+    const uint16_t* g;       // bf16 [rows, cols]
+    const uint8_t* mask;     // bits or bytes
+    int mask_mode;           // 0 bits, 1 bytes
+    int64_t rows, cols;
+    uint16_t* out;           // bf16 [rows, cols]
+    float inv_sqrt_hb;
+};
+
+// Launchers (return cudaSuccess or the launch error).
+cudaError_t launch_quantize(const QuantArgs& a, quest_dtype x_dtype, int had_block, int cbits,
+                            bool row_mode, cudaStream_t stream);
+cudaError_t launch_trust_bwd(const TrustArgs& a, int had_block, cudaStream_t stream);
+cudaError_t launch_w4a4(const int8_t* A, const float* sa, const int8_t* B, const float* sb,
+                        int64_t M, int64_t N, int64_t K, uint16_t* y, int32_t* acc,
+                        cudaStream_t stream);
+
+// Reads (synchronising `stream`) and clears the integer linear layer's device
+// status word; returns its value (0 or a quest_status).
+int read_and_clear_gemm_status(cudaStream_t stream, cudaError_t* err);
+
+// Number of SMs and max resident CTAs of `func` per SM on the current device.
+int sm_count();
+int max_ctas_per_sm(const void* func, int threads, size_t smem);
+
+}  // namespace quest

@@ -1,0 +1,494 @@
+// Integer linear layer on QuEST codes: tcgen05 kind::i8 GEMM with TMEM
+// accumulators and a fused dequantisation epilogue (sm_100a).
+//
+//   acc[m][n] = sum_k A[m][k] * B[n][k]        (int8 x int8 -> int32, exact)
+//   y[m][n]   = bf16_rne(acc * (sa[m]/2) * (sb[n]/2))
+//
+// The pages run the QuEST linear layers as INT4 kernels on the integer codes
+// (atlas.scime.ai summary of QuEST, "Key results"; pith.science review,
+// Figure 5). On sm_100a the codes travel as int8 (c = 2q + 1, |c| <= 15 at
+// b = 4), which makes the int8 tensor-core product exact.
+//
+// Structure (one persistent CTA per SM, 192 threads):
+//   warp 0     TMA producer: A [128 x 128] and B [256 x 128] int8 tiles,
+//              128-byte swizzle, kStages-deep smem ring guarded by mbarriers.
+//   warp 1     TMEM allocator and MMA issuer: one thread issues four
+//              tcgen05.mma (K = 32 each) per stage into a 128 x 256 int32
+//              accumulator; two accumulators (512 TMEM columns) alternate so
+//              the epilogue of tile i overlaps the mainloop of tile i + 1.
+//   warps 2-5  epilogue: tcgen05.ld 32 columns at a time, scale, round to
+//              bf16, stage in 64-byte-swizzled smem, TMA store.
+// No cluster, no multicast. Every mbarrier wait is bounded in time; on
+// timeout the CTA records QUEST_ETIMEOUT in a device status word, drains its
+// in-flight copies and MMAs, frees TMEM and returns.
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include <mutex>
+
+#include "quest_internal.h"
+
+namespace quest {
+
+// Device-side status word of the integer linear layer (0 = fine). Written only
+// when a bounded wait gives up; read and cleared by quest_device_status().
+__device__ int g_gemm_status = 0;
+
+namespace {
+
+constexpr int BM = 128, BN = 256, BK = 128;   // BK in int8 elements (= bytes)
+constexpr int kStages = 4;
+constexpr int kUmmaK = 32;                    // K of one kind::i8 MMA
+constexpr int kThreads = 192;
+constexpr int kEpiThreads = 128;
+constexpr int kChunkCols = 32;                // epilogue columns per TMEM load / TMA store
+constexpr uint32_t kTmemCols = 512;           // two 256-column accumulators
+constexpr uint32_t kStageA = BM * BK, kStageB = BN * BK, kStageBytes = kStageA + kStageB;
+constexpr uint32_t kCBytes = BM * kChunkCols * 2;  // one bf16 staging chunk (8 KB)
+constexpr uint32_t kSmemA = 0;
+constexpr uint32_t kSmemB = kSmemA + kStages * kStageA;
+constexpr uint32_t kSmemC = kSmemB + kStages * kStageB;
+constexpr uint32_t kSmemScale = kSmemC + 2 * kCBytes;       // float[BN]
+constexpr uint32_t kSmemBar = kSmemScale + BN * 4;
+constexpr uint32_t kNumBars = 2 * kStages + 4 + 1;
+constexpr uint32_t kSmemTmemSlot = kSmemBar + kNumBars * 8;
+constexpr uint32_t kSmemAbort = kSmemTmemSlot + 4;
+constexpr uint32_t kSmemUsed = kSmemAbort + 4;
+constexpr uint32_t kSmemTotal = kSmemUsed + 1024;           // slack for 1 KB alignment
+constexpr uint64_t kWaitLimitNs = 2000000000ull;            // 2 s per wait
+
+// Instruction descriptor of tcgen05.mma kind::i8: D int32, A and B signed
+// int8, both K-major, M = 128, N = 256.
+constexpr uint32_t kIdesc = (2u << 4)           // D format: s32
+                            | (1u << 7)         // A: signed 8-bit
+                            | (1u << 10)        // B: signed 8-bit
+                            | (uint32_t(BN >> 3) << 17) | (uint32_t(BM >> 4) << 24);
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
+}
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
+                 : "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+__device__ __forceinline__ uint64_t global_timer_ns() {
+    uint64_t t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+
+// Bounded wait for the phase of `bar` with parity `parity`. Returns false when
+// the CTA is aborting (another role timed out) or this wait timed out.
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag,
+                                          uint64_t limit_ns = kWaitLimitNs) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = global_timer_ns();
+    for (uint32_t it = 1;; ++it) {
+        if (mbar_try_wait(bar, parity)) return true;
+        if ((it & 63u) == 0) {
+            if (*abort_flag) return false;
+            if (global_timer_ns() - t0 > limit_ns) {
+                *abort_flag = 1;
+                atomicExch(&g_gemm_status, (int)QUEST_ETIMEOUT);
+                return false;
+            }
+        }
+    }
+}
+
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, int c0, int c1,
+                                            uint32_t bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes "
+        "[%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(bar)
+        : "memory");
+}
+__device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, uint32_t src, int c0, int c1) {
+    asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%1, %2}], [%3];" ::"l"(
+                     reinterpret_cast<uint64_t>(map)),
+                 "r"(c0), "r"(c1), "r"(src)
+                 : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait_read_le1() {
+    asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
+}
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+__device__ __forceinline__ void fence_proxy_async_smem() {
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+__device__ __forceinline__ void epi_bar() { asm volatile("bar.sync 1, %0;" ::"n"(kEpiThreads) : "memory"); }
+// OR-vote over the 128 epilogue threads (named barrier 1).
+__device__ __forceinline__ bool epi_any(bool pred) {
+    uint32_t out;
+    asm volatile(
+        "{\n\t.reg .pred p, q;\n\t"
+        "setp.ne.u32 p, %1, 0;\n\t"
+        "bar.red.or.pred q, 1, %2, p;\n\t"
+        "selp.u32 %0, 1, 0, q;\n\t}"
+        : "=r"(out)
+        : "r"((uint32_t)pred), "n"(kEpiThreads)
+        : "memory");
+    return out != 0;
+}
+
+__device__ __forceinline__ void tc_fence_before() {
+    asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after() {
+    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_commit(uint32_t bar) {
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
+                 : "memory");
+}
+__device__ __forceinline__ void tc_mma_i8(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
+                                          uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::i8 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(adesc), "l"(bdesc), "r"(kIdesc), "r"(accumulate)
+        : "memory");
+}
+
+// Shared-memory matrix descriptor of a K-major tile with 128-byte rows and the
+// 128-byte swizzle written by TMA: 8-row core groups 1024 bytes apart.
+__device__ __forceinline__ uint64_t smem_desc_k128(uint32_t addr) {
+    uint64_t d = 0;
+    d |= uint64_t((addr >> 4) & 0x3FFFu);          // start address
+    d |= uint64_t(1) << 16;                        // leading byte offset (unused for swizzled K-major)
+    d |= uint64_t(1024 >> 4) << 32;                // stride byte offset: 8 rows x 128 B
+    d |= uint64_t(1) << 46;                        // descriptor version (sm_100)
+    d |= uint64_t(2) << 61;                        // layout: 128-byte swizzle
+    return d;
+}
+
+#define QUEST_TMEM_LD32(taddr, r)                                                              \
+    asm volatile(                                                                              \
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 "                                             \
+        "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"                              \
+        "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"             \
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), \
+          "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),          \
+          "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]),       \
+          "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]),       \
+          "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]),       \
+          "=r"(r[31])                                                                          \
+        : "r"(taddr))
+
+__device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+
+struct GemmParams {
+    const float* sa;
+    const float* sb;
+    int32_t* acc;       // optional int32 copy of the accumulator
+    int M, N, K;
+    int num_m, num_n, num_k;
+};
+
+__global__ void __launch_bounds__(kThreads, 1)
+w4a4_gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_b,
+                 const __grid_constant__ CUtensorMap map_y, const GemmParams p) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const uint32_t sbase = smem_u32(smem);
+    const uint32_t bar_full = sbase + kSmemBar;                  // [kStages]
+    const uint32_t bar_empty = bar_full + 8 * kStages;           // [kStages]
+    const uint32_t bar_tfull = bar_empty + 8 * kStages;          // [2]
+    const uint32_t bar_tempty = bar_tfull + 16;                  // [2]
+    const uint32_t bar_drain = bar_tempty + 16;                  // [1] MMA drain on abort
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + kSmemAbort);
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kSmemTmemSlot);
+    float* s_scale = reinterpret_cast<float*>(smem + kSmemScale);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int num_tiles = p.num_m * p.num_n;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kStages; ++s) {
+            mbar_init(bar_full + 8 * s, 1);
+            mbar_init(bar_empty + 8 * s, 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(bar_tfull + 8 * b, 1);
+            mbar_init(bar_tempty + 8 * b, kEpiThreads);
+        }
+        mbar_init(bar_drain, 1);
+        *abort_flag = 0;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&map_a)) : "memory");
+        asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&map_b)) : "memory");
+        asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&map_y)) : "memory");
+    }
+    if (warp == 1) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                         smem_u32(tmem_slot)),
+                     "r"(kTmemCols)
+                     : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+
+    if (warp == 0) {
+        // ------------------------------------------------------------ TMA producer
+        if (lane == 0) {
+            uint32_t stage = 0, phase = 0;
+            uint64_t issued = 0;
+            bool ok = true;
+            for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
+                const int m0 = (tile % p.num_m) * BM, n0 = (tile / p.num_m) * BN;
+                for (int kb = 0; kb < p.num_k; ++kb) {
+                    if (!mbar_wait(bar_empty + 8 * stage, phase ^ 1, abort_flag)) { ok = false; break; }
+                    const uint32_t fb = bar_full + 8 * stage;
+                    mbar_arrive_expect_tx(fb, kStageBytes);
+                    tma_load_2d(sbase + kSmemA + stage * kStageA, &map_a, kb * BK, m0, fb);
+                    tma_load_2d(sbase + kSmemB + stage * kStageB, &map_b, kb * BK, n0, fb);
+                    ++issued;
+                    if (++stage == kStages) { stage = 0; phase ^= 1; }
+                }
+            }
+            if (!ok) {
+                // drain: the last min(issued, kStages) loads may still be landing
+                const uint64_t n = issued < kStages ? issued : kStages;
+                for (uint64_t i = issued - n; i < issued; ++i) {
+                    const uint32_t st = uint32_t(i % kStages), ph = uint32_t((i / kStages) & 1);
+                    const uint64_t t0 = global_timer_ns();
+                    while (!mbar_try_wait(bar_full + 8 * st, ph) && global_timer_ns() - t0 < kWaitLimitNs) {
+                    }
+                }
+            }
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            uint32_t stage = 0, phase = 0;
+            bool ok = true;
+            int local = 0;
+            for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x, ++local) {
+                const uint32_t buf = local & 1, bphase = (local >> 1) & 1;
+                if (!mbar_wait(bar_tempty + 8 * buf, bphase ^ 1, abort_flag)) { ok = false; break; }
+                tc_fence_after();
+                const uint32_t d_tmem = tmem_base + buf * BN;
+                for (int kb = 0; kb < p.num_k; ++kb) {
+                    if (!mbar_wait(bar_full + 8 * stage, phase, abort_flag)) { ok = false; break; }
+                    tc_fence_after();
+                    const uint32_t a_addr = sbase + kSmemA + stage * kStageA;
+                    const uint32_t b_addr = sbase + kSmemB + stage * kStageB;
+#pragma unroll
+                    for (int kk = 0; kk < BK / kUmmaK; ++kk) {
+                        tc_mma_i8(d_tmem, smem_desc_k128(a_addr + kk * kUmmaK),
+                                  smem_desc_k128(b_addr + kk * kUmmaK), (kb | kk) != 0);
+                    }
+                    tc_commit(bar_empty + 8 * stage);  // frees the smem stage when these MMAs finish
+                    if (++stage == kStages) { stage = 0; phase ^= 1; }
+                }
+                if (!ok) break;
+                tc_commit(bar_tfull + 8 * buf);        // accumulator ready for the epilogue
+            }
+            // make sure every issued MMA has finished before TMEM is released
+            tc_commit(bar_drain);
+            const uint64_t t0 = global_timer_ns();
+            while (!mbar_try_wait(bar_drain, 0) && global_timer_ns() - t0 < kWaitLimitNs) {
+            }
+        }
+    } else {
+        // ------------------------------------------------------------ epilogue (warps 2..5)
+        const int et = threadIdx.x - 64;             // 0..127
+        const int quarter = warp & 3;                // this warp may read TMEM lanes 32*quarter..+31
+        const int row_in_tile = quarter * 32 + lane; // accumulator row = TMEM lane
+        const uint32_t lane_addr = uint32_t(quarter * 32) << 16;
+        int local = 0;
+        int cbuf = 0;
+        for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++local) {
+            const int m0 = (tile % p.num_m) * BM, n0 = (tile / p.num_m) * BN;
+            const uint32_t buf = local & 1, bphase = (local >> 1) & 1;
+            epi_bar();  // everyone is done with the previous tile's column scales
+            for (int c = et; c < BN; c += kEpiThreads) {
+                const int n = n0 + c;
+                s_scale[c] = n < p.N ? p.sb[n] * 0.5f : 0.0f;
+            }
+            const int m = m0 + row_in_tile;
+            const float sa_half = m < p.M ? p.sa[m] * 0.5f : 0.0f;
+            const bool got = mbar_wait(bar_tfull + 8 * buf, bphase, abort_flag);
+            if (epi_any(!got)) break;  // all 128 threads leave together
+            tc_fence_after();
+            const uint32_t t_acc = tmem_base + lane_addr + buf * BN;
+#pragma unroll 1
+            for (int c = 0; c < BN / kChunkCols; ++c) {
+                uint32_t r[32];
+                QUEST_TMEM_LD32(t_acc + c * kChunkCols, r);
+                tmem_wait_ld();
+                const float* sc = s_scale + c * kChunkCols;
+                const uint32_t stg = sbase + kSmemC + cbuf * kCBytes + row_in_tile * (kChunkCols * 2);
+                const uint32_t swz = (row_in_tile >> 1) & 3;
+#pragma unroll
+                for (int q16 = 0; q16 < 4; ++q16) {
+                    uint32_t w[4];
+#pragma unroll
+                    for (int h = 0; h < 4; ++h) {
+                        const int i = q16 * 8 + h * 2;
+                        const float y0 = (float)(int32_t)r[i] * sa_half * sc[i];
+                        const float y1 = (float)(int32_t)r[i + 1] * sa_half * sc[i + 1];
+                        __nv_bfloat162 hb = __floats2bfloat162_rn(y0, y1);
+                        w[h] = *reinterpret_cast<uint32_t*>(&hb);
+                    }
+                    const uint32_t dst = stg + ((q16 ^ swz) << 4);
+                    asm volatile("st.shared.v4.u32 [%0], {%1,%2,%3,%4};" ::"r"(dst), "r"(w[0]),
+                                 "r"(w[1]), "r"(w[2]), "r"(w[3])
+                                 : "memory");
+                }
+                if (p.acc != nullptr && m < p.M) {
+                    int32_t* arow = p.acc + int64_t(m) * p.N;
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) {
+                        const int n = n0 + c * kChunkCols + i;
+                        if (n < p.N) arow[n] = (int32_t)r[i];
+                    }
+                }
+                fence_proxy_async_smem();
+                epi_bar();
+                if (et == 0) {
+                    tma_store_2d(&map_y, sbase + kSmemC + cbuf * kCBytes, n0 + c * kChunkCols, m0);
+                    bulk_commit();
+                    bulk_wait_read_le1();  // the other staging buffer is free again
+                }
+                epi_bar();
+                cbuf ^= 1;
+            }
+            tc_fence_before();
+            mbar_arrive(bar_tempty + 8 * buf);
+        }
+        if (et == 0) bulk_wait_all();
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base),
+                     "r"(kTmemCols)
+                     : "memory");
+    }
+}
+
+// Writes zeros (K == 0: the empty sum).
+__global__ void zero_fill_kernel(uint16_t* y, int32_t* acc, int64_t n) {
+    for (int64_t i = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; i < n;
+         i += int64_t(gridDim.x) * blockDim.x) {
+        y[i] = 0;
+        if (acc) acc[i] = 0;
+    }
+}
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    });
+    return fn;
+}
+
+bool make_map_2d(CUtensorMap* map, CUtensorMapDataType dt, const void* base, uint64_t inner,
+                 uint64_t outer, uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer,
+                 CUtensorMapSwizzle swz) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    const cuuint64_t dims[2] = {inner, outer};
+    const cuuint64_t strides[1] = {row_bytes};
+    const cuuint32_t box[2] = {box_inner, box_outer};
+    const cuuint32_t estr[2] = {1, 1};
+    return fn(map, dt, 2, const_cast<void*>(base), dims, strides, box, estr,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+}  // namespace
+
+cudaError_t launch_w4a4(const int8_t* A, const float* sa, const int8_t* B, const float* sb,
+                        int64_t M, int64_t N, int64_t K, uint16_t* y, int32_t* acc,
+                        cudaStream_t stream) {
+    if (M == 0 || N == 0) return cudaSuccess;
+    if (K == 0) {
+        const int64_t n = M * N;
+        int64_t blocks = (n + 255) / 256;
+        if (blocks > 4096) blocks = 4096;
+        zero_fill_kernel<<<(int)blocks, 256, 0, stream>>>(y, acc, n);
+        return cudaGetLastError();
+    }
+    CUtensorMap ma, mb, my;
+    if (!make_map_2d(&ma, CU_TENSOR_MAP_DATA_TYPE_UINT8, A, K, M, K, BK, BM, CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !make_map_2d(&mb, CU_TENSOR_MAP_DATA_TYPE_UINT8, B, K, N, K, BK, BN, CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !make_map_2d(&my, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, y, N, M, N * 2, kChunkCols, BM,
+                     CU_TENSOR_MAP_SWIZZLE_64B))
+        return cudaErrorInvalidValue;
+    GemmParams p;
+    p.sa = sa; p.sb = sb; p.acc = acc;
+    p.M = (int)M; p.N = (int)N; p.K = (int)K;
+    p.num_m = (int)((M + BM - 1) / BM);
+    p.num_n = (int)((N + BN - 1) / BN);
+    p.num_k = (int)((K + BK - 1) / BK);
+    static thread_local int attr_dev = -1;
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (attr_dev != dev) {
+        cudaError_t e = cudaFuncSetAttribute(w4a4_gemm_kernel,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemTotal);
+        if (e != cudaSuccess) return e;
+        attr_dev = dev;
+    }
+    const int tiles = p.num_m * p.num_n;
+    const int sms = sm_count();
+    const int grid = tiles < sms ? tiles : sms;
+    w4a4_gemm_kernel<<<grid, kThreads, kSmemTotal, stream>>>(ma, mb, my, p);
+    return cudaGetLastError();
+}
+
+int read_and_clear_gemm_status(cudaStream_t stream, cudaError_t* err) {
+    int v = 0, zero = 0;
+    cudaError_t e = cudaMemcpyFromSymbolAsync(&v, g_gemm_status, sizeof(int), 0,
+                                              cudaMemcpyDeviceToHost, stream);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(stream);
+    if (e == cudaSuccess && v != 0)
+        e = cudaMemcpyToSymbolAsync(g_gemm_status, &zero, sizeof(int), 0, cudaMemcpyHostToDevice, stream);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(stream);
+    *err = e;
+    return v;
+}
+
+}  // namespace quest

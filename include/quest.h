@@ -1,0 +1,211 @@
+/*
+ * quest.h -- C ABI of the QuEST quantizer hot path for NVIDIA B200 (sm_100a).
+ *
+ * Method: "QuEST: Stable Training of LLMs with 1-Bit Weights and Activations"
+ * (Panferov, Chen, Tabesh, Castro, Nikdan, Alistarh; arXiv 2502.05003), as
+ * described on the pith.science review page ("What carries the argument",
+ * "Assumptions & free parameters", Figures 2 and 5) and the atlas.scime.ai
+ * summary ("Approach", "Key results").
+ *
+ * General conventions
+ *   - Every tensor argument is a DEVICE pointer to memory the caller owns
+ *     (allocated by the caller, e.g. through PyTorch). The library allocates no
+ *     device memory, keeps no per-call state and never synchronises: every
+ *     entry point validates its arguments on the host, enqueues its kernel(s) on
+ *     `stream` and returns.
+ *   - `stream` is a cudaStream_t passed as void*; NULL means the legacy default
+ *     stream. The current CUDA device must be the device owning the pointers.
+ *   - Matrices are row-major. "rows" is the number of independent vectors, "cols"
+ *     the length along which the Hadamard transform and the RMS groups run (the
+ *     reduction dimension of the linear layer that consumes the codes).
+ *   - bf16 means IEEE bfloat16 (1-8-7), stored as 16-bit little-endian words.
+ *   - Errors: a non-zero quest_status. Argument errors are detected before any
+ *     launch and leave every output untouched; QUEST_ECUDA reports a launch or
+ *     driver error (the CUDA error string is available from
+ *     quest_last_error_message()). Nothing in the library traps or asserts on
+ *     the device.
+ *   - Thread safety: all entry points may be called concurrently from several
+ *     host threads (the per-thread error message is thread-local).
+ */
+#ifndef QUEST_B200_H
+#define QUEST_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum quest_status {
+    QUEST_OK = 0,
+    QUEST_EINVAL = 1,         /* an argument is out of range, NULL or misaligned */
+    QUEST_EUNSUPPORTED = 2,   /* a valid request this build does not implement */
+    QUEST_ECUDA = 3,          /* CUDA launch / driver error */
+    QUEST_ETIMEOUT = 4        /* a bounded device-side wait gave up */
+} quest_status;
+
+typedef enum quest_dtype {
+    QUEST_BF16 = 0,
+    QUEST_FP32 = 1
+} quest_dtype;
+
+/* How integer codes are stored.
+ *   QUEST_CODES_PACKED        two's-complement code q in a container of
+ *                             1/2/4/4/8/8/8/8 bits for b = 1..8, packed little-
+ *                             endian inside each byte (element 2j in the low
+ *                             nibble at 4-bit, element 8j in bit 0 at 1-bit).
+ *                             Row stride: cols * container_bits / 8 bytes.
+ *   QUEST_CODES_INT8          one int8 per element holding q.
+ *   QUEST_CODES_GEMM_OPERAND  one int8 per element holding c = 2q + 1 (odd,
+ *                             |c| <= 2^b - 1), the exact integer form of the
+ *                             midrise level (q + 1/2); requires b <= 7. */
+typedef enum quest_code_mode {
+    QUEST_CODES_PACKED = 0,
+    QUEST_CODES_INT8 = 1,
+    QUEST_CODES_GEMM_OPERAND = 2
+} quest_code_mode;
+
+/* How the trust mask is stored (1 = gradient kept, 0 = gradient zeroed).
+ *   QUEST_MASK_BITS   uint32 words [rows, cols/32]; bit j of word w is column
+ *                     32w + j (equivalently bytes [rows, cols/8], bit j of byte
+ *                     i is column 8i + j).
+ *   QUEST_MASK_BYTES  uint8 [rows, cols], one 0/1 byte per element. */
+typedef enum quest_mask_mode {
+    QUEST_MASK_BITS = 0,
+    QUEST_MASK_BYTES = 1
+} quest_mask_mode;
+
+/*
+ * quest_quantize_fwd -- QuEST forward quantizer with trust mask.
+ *
+ * Follows pith.science review, "What carries the argument" (Hadamard transform,
+ * then projection onto a uniform grid whose scale minimises the L2 error
+ * against a standard Gaussian; the mask zeroes entries whose quantization error
+ * exceeds half a quantization interval), atlas.scime.ai summary, "Approach"
+ * (Hadamard transform with RMS normalisation, MSE-optimal Gaussian clipping,
+ * trust threshold) and pith.science review, "Assumptions & free parameters"
+ * (alpha fixed from an N(0,1) target). For every row and every Hadamard block
+ * of `had_block` consecutive columns:
+ *     y     = H x_block / sqrt(had_block)      (Sylvester order, H_ij = (-1)^popcount(i&j))
+ *     r     = sqrt(mean(y^2))   over the rms group (`rms_group` consecutive columns)
+ *     Delta = alpha_b * r / 2^(b-1)            (alpha_b = quest_alpha(bits))
+ *     t     = y / Delta
+ *     q     = clamp(floor(t), -2^(b-1), 2^(b-1) - 1)
+ *     yhat  = (q + 1/2) * Delta                (stays in the Hadamard domain)
+ *     m     = [ |t - (q + 1/2)| <= trust / 2 ]
+ * A group with r == 0 yields Delta = 0, q = 0, yhat = 0, m = 1. Inputs holding
+ * NaN or Inf propagate into that group's outputs (codes become unspecified but
+ * in range); they are not checked.
+ *
+ * Arguments
+ *   x          device, x_dtype [rows, ld_x] (only the first `cols` columns read);
+ *              16-byte aligned; ld_x * sizeof(x_dtype) a multiple of 16 bytes.
+ *   rows       >= 0 (0 is a no-op).   cols > 0, a multiple of had_block.
+ *   bits       1..8.   had_block: 16, 32, 64, 128 or 256.
+ *   rms_group  had_block (one RMS per Hadamard block) or cols (one RMS per row,
+ *              the per-row scale form used by the integer linear layer; then
+ *              cols <= 16384).
+ *   trust      trust factor T > 0 (1.0 = half an interval; the 1-bit runs of the
+ *              pages widen the outer trust region with s* = 1.30).
+ *   code_mode  storage of `codes` (see quest_code_mode); codes must be aligned to
+ *              8 bytes (4 for 4-bit packed, 2 for 2-bit, 1 for 1-bit).
+ *   codes      device, required: quest_codes_bytes(rows, cols, bits, code_mode) bytes.
+ *   scales     device, required: fp32 [rows, cols / rms_group], Delta per group.
+ *   mask_mode, mask   device, optional (NULL = not written): quest_mask_bytes() bytes.
+ *   dequant    device, optional (NULL = not written): dequant_dtype [rows, cols],
+ *              16-byte aligned, yhat.
+ * Returns QUEST_OK, QUEST_EINVAL (bad argument), QUEST_EUNSUPPORTED, QUEST_ECUDA.
+ */
+quest_status quest_quantize_fwd(const void* x, quest_dtype x_dtype, int64_t rows, int64_t cols,
+                                int64_t ld_x, int bits, int had_block, int64_t rms_group,
+                                float trust, quest_code_mode code_mode, void* codes,
+                                float* scales, quest_mask_mode mask_mode, void* mask,
+                                void* dequant, quest_dtype dequant_dtype, void* stream);
+
+/*
+ * quest_trust_bwd -- trust-estimator backward.
+ *
+ * Follows pith.science review, "What carries the argument" (the gradient is
+ * multiplied in the Hadamard domain by the binary mask) and Figure 2's caption
+ * (two inverse Hadamard transforms on the backward pass, one per operand). For
+ * every row and block:
+ *     grad_in_block = H^T (m . grad_out_block) / sqrt(had_block)
+ * (H is symmetric, so the inverse of the normalised transform is itself). No
+ * gradient flows through the RMS scale.
+ *
+ * Arguments
+ *   grad_out   device, bf16 [rows, cols], dL/dyhat in the Hadamard domain; 16-byte aligned.
+ *   mask       device, the mask written by quest_quantize_fwd in `mask_mode`.
+ *   rows >= 0; cols > 0, a multiple of had_block.
+ *   had_block  16, 32, 64, 128 or 256 (the value used in the forward pass).
+ *   grad_in    device, bf16 [rows, cols], dL/dx; 16-byte aligned; may not alias grad_out.
+ */
+quest_status quest_trust_bwd(const void* grad_out, const void* mask, quest_mask_mode mask_mode,
+                             int64_t rows, int64_t cols, int had_block, void* grad_in,
+                             void* stream);
+
+/*
+ * quest_w4a4_linear -- integer linear layer on QuEST codes.
+ *
+ * The pages' GPU kernels run the linear layers of a QuEST INT4 model on the
+ * integer codes, with quantization, dequantization and Hadamard costs included
+ * (atlas.scime.ai summary, "Key results"; pith.science review, Figure 5). Because
+ * the Hadamard matrix is orthogonal, transforming both operands leaves the
+ * product unchanged (pith.science review, "Assumptions & free parameters"), so
+ * the product of the two Hadamard-domain operands is the layer output:
+ *     acc[m][n] = sum_k a_codes[m][k] * w_codes[n][k]          (exact, int32)
+ *     y[m][n]   = bf16_rne( acc[m][n] * (a_scales[m] / 2) * (w_scales[n] / 2) )
+ * With codes in GEMM-operand form (c = 2q + 1) and per-row scales Delta
+ * (rms_group = cols), y equals yhat_a . yhat_w^T.
+ *
+ * Arguments
+ *   a_codes    device, int8 [M, K] row-major (K contiguous); 16-byte aligned.
+ *   a_scales   device, fp32 [M].
+ *   w_codes    device, int8 [N, K] row-major (the nn.Linear weight layout).
+ *   w_scales   device, fp32 [N].
+ *   M >= 0, N >= 0 (0 = no-op); N a multiple of 8; K >= 0, a multiple of 16,
+ *   K < 131072 (so that any int8 products fit the int32 accumulator).
+ *   y          device, bf16 [M, N]; 16-byte aligned.
+ *   acc        device, optional int32 [M, N] copy of the accumulator (NULL = not
+ *              written); meant for exactness checks.
+ */
+quest_status quest_w4a4_linear(const int8_t* a_codes, const float* a_scales,
+                               const int8_t* w_codes, const float* w_scales, int64_t M,
+                               int64_t N, int64_t K, void* y, int32_t* acc, void* stream);
+
+/*
+ * quest_device_status -- synchronises `stream`, then reports (and clears) the
+ * device-side status of the integer linear layer on the current device:
+ * QUEST_ETIMEOUT if one of its bounded pipeline waits gave up since the last
+ * call (its output is then incomplete), QUEST_OK otherwise, QUEST_ECUDA on a
+ * CUDA error. The quantizer and trust kernels have no waits and never set it.
+ */
+quest_status quest_device_status(void* stream);
+
+/* alpha_b, the clip edge of the b-bit grid (2^(b-1) times the step that minimises
+ * the MSE of the midrise uniform quantizer for X ~ N(0,1)); bits 1..8. Computed on
+ * the host at first use. Returns NaN for an invalid bit-width. */
+double quest_alpha(int bits);
+
+/* Bits of the storage container of a b-bit packed code: 1, 2, 4, 4, 8, 8, 8, 8. 0 if invalid. */
+int quest_container_bits(int bits);
+
+/* Bytes needed for `codes` / `mask` of a rows x cols tensor; 0 for invalid arguments. */
+size_t quest_codes_bytes(int64_t rows, int64_t cols, int bits, quest_code_mode mode);
+size_t quest_mask_bytes(int64_t rows, int64_t cols, quest_mask_mode mode);
+
+/* Static description of a status code. */
+const char* quest_status_string(quest_status s);
+
+/* Detail of the last error on the calling host thread ("" if none). */
+const char* quest_last_error_message(void);
+
+/* ABI version (major * 10000 + minor * 100 + patch). */
+int quest_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* QUEST_B200_H */

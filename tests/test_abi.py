@@ -1,0 +1,132 @@
+"""C-ABI checks that need no GPU: the library loads, exports every function the
+header declares, computes alpha_b on the host, and rejects invalid arguments
+before touching the device."""
+import ctypes
+import math
+import os
+import re
+
+import pytest
+
+import oracle
+import bit_quantization_aware_blockwise_b200 as q
+from bit_quantization_aware_blockwise_b200 import _binding
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared_functions():
+    names = set()
+    for fn in os.listdir(os.path.join(ROOT, "include")):
+        if fn.endswith(".h"):
+            text = open(os.path.join(ROOT, "include", fn)).read()
+            text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+            names |= set(re.findall(r"\b(quest_\w+)\s*\(", text))
+    return names
+
+
+def test_library_exports_every_declared_symbol():
+    lib = q.load_library()
+    declared = _declared_functions()
+    assert "quest_quantize_fwd" in declared and "quest_w4a4_linear" in declared
+    for name in sorted(declared):
+        assert hasattr(lib, name), name
+    # and the binding knows the signature of each
+    assert declared == set(_binding.SIGNATURES)
+
+
+def test_version_and_status_strings():
+    lib = q.load_library()
+    assert lib.quest_version() >= 10000
+    for s in range(5):
+        assert lib.quest_status_string(s)
+
+
+@pytest.mark.parametrize("bits", range(1, 9))
+def test_alpha_table_matches_oracle(bits):
+    # The library finds alpha_b by bisection on the stationarity condition; the
+    # oracle by golden-section search on the MSE itself. The golden section only
+    # locates a flat minimum to ~sqrt(eps) of its argument.
+    a_lib = q.alpha(bits)
+    a_ref, _, _ = oracle.alpha(bits)
+    assert a_lib == pytest.approx(a_ref, rel=3e-7)
+
+
+def test_alpha_one_bit_exact():
+    assert q.alpha(1) == pytest.approx(2 * math.sqrt(2 / math.pi), rel=1e-14)
+    assert math.isnan(q.alpha(0)) and math.isnan(q.alpha(9))
+
+
+def test_sizes():
+    assert [q.container_bits(b) for b in range(1, 9)] == [1, 2, 4, 4, 8, 8, 8, 8]
+    assert q.codes_bytes(16384, 2048, 4) == 16384 * 2048 // 2
+    assert q.codes_bytes(3, 128, 1) == 3 * 16
+    assert q.codes_bytes(3, 128, 4, q.CODES_GEMM_OPERAND) == 3 * 128
+    assert q.mask_bytes(16384, 2048, q.MASK_BITS) == 16384 * 2048 // 8
+    assert q.mask_bytes(2, 128, q.MASK_BYTES) == 256
+    assert q.codes_bytes(1, 128, 0) == 0 and q.mask_bytes(1, 12, q.MASK_BITS) == 0
+
+
+# Invalid calls: the library must return QUEST_EINVAL / EUNSUPPORTED before any
+# CUDA call, so these run without a GPU. The pointers are never dereferenced.
+FAKE = 1 << 20  # 16-byte aligned, never touched
+
+
+def _qf(**kw):
+    args = dict(x=FAKE, x_dtype=0, rows=4, cols=256, ld_x=256, bits=4, had_block=128,
+                rms_group=128, trust=1.0, code_mode=0, codes=FAKE, scales=FAKE, mask_mode=0,
+                mask=FAKE, dequant=None, dequant_dtype=0, stream=None)
+    args.update(kw)
+    lib = q.load_library()
+    return lib.quest_quantize_fwd(*args.values())
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(bits=0), 1), (dict(bits=9), 1), (dict(had_block=100), 1), (dict(had_block=512), 1),
+    (dict(cols=200), 1), (dict(ld_x=128), 1), (dict(rms_group=64), 1), (dict(trust=0.0), 1),
+    (dict(trust=-1.0), 1), (dict(trust=float("inf")), 1), (dict(code_mode=7), 1),
+    (dict(code_mode=2, bits=8), 1), (dict(x=None), 1), (dict(codes=None), 1),
+    (dict(scales=None), 1), (dict(x=FAKE + 4), 1), (dict(ld_x=260), 1),
+    (dict(codes=FAKE + 2), 1), (dict(x_dtype=5), 1), (dict(mask_mode=3), 1),
+    (dict(dequant=FAKE + 8), 1), (dict(rows=-1), 1),
+    (dict(cols=16384 * 2, ld_x=16384 * 2, rms_group=16384 * 2), 2),
+])
+def test_quantize_rejects_invalid_arguments(kw, status):
+    assert _qf(**kw) == status
+    assert q.load_library().quest_last_error_message()
+
+
+def test_quantize_zero_rows_is_a_noop():
+    assert _qf(rows=0, x=None, codes=None, scales=None, mask=None) == 0
+
+
+def test_trust_bwd_rejects_invalid_arguments():
+    lib = q.load_library()
+    ok = dict(g=FAKE, m=FAKE, mm=0, rows=4, cols=256, hb=128, out=FAKE * 4, s=None)
+    def call(**kw):
+        a = dict(ok); a.update(kw)
+        return lib.quest_trust_bwd(*a.values())
+    assert call(hb=100) == 1
+    assert call(cols=100) == 1
+    assert call(mm=2) == 1
+    assert call(g=None) == 1
+    assert call(out=FAKE + 2) == 1
+    assert call(out=FAKE) == 1            # aliasing grad_out
+    assert call(mm=1, m=FAKE + 4) == 1    # byte mask misaligned
+    assert call(rows=0, g=None, m=None, out=None) == 0
+
+
+def test_w4a4_rejects_invalid_arguments():
+    lib = q.load_library()
+    ok = dict(a=FAKE, sa=FAKE, w=FAKE, sw=FAKE, M=128, N=256, K=2048, y=FAKE, acc=None, s=None)
+    def call(**kw):
+        a = dict(ok); a.update(kw)
+        return lib.quest_w4a4_linear(*a.values())
+    assert call(K=100) == 1
+    assert call(N=100) == 1
+    assert call(K=131072) == 1
+    assert call(M=-1) == 1
+    assert call(a=FAKE + 8) == 1
+    assert call(y=None) == 1
+    assert call(sa=FAKE + 2) == 1
+    assert call(M=0) == 0 and call(N=0) == 0   # empty output: nothing to do
