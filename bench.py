@@ -166,14 +166,20 @@ def dist_setup(n_gpus):
     return world, rank, local
 
 
-def dist_max(value, world):
+def dist_max(value, world, device="cuda"):
+    """Max of a per-rank number over all ranks (timing plumbing, not the data path)."""
     if world == 1:
         return value
     import torch
     import torch.distributed as dist
-    t = torch.tensor([value], dtype=torch.float64, device="cuda")
+    t = torch.tensor([value], dtype=torch.float64, device=device)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def aggregate_throughput(bytes_per_rank_step, world, ms_max):
+    """Whole-job GB/s: the units every rank processed over the slowest rank's time."""
+    return bytes_per_rank_step * world / (ms_max * 1e-3) / 1e9
 
 
 def dist_barrier(world):
@@ -291,7 +297,7 @@ def run_b200(args, world, rank, local):
     ms = dist_max(my_ms, world)
     pbytes = part_bytes()
     step_bytes = sum(pbytes.values())
-    value = step_bytes * world / (ms * 1e-3) / 1e9
+    value = aggregate_throughput(step_bytes, world, ms)
 
     hbm = peaks["hbm_gbs"]
     int8_peak = peaks["bf16_tflops"] * 2.0   # nominal int8 : bf16 dense ratio 4.5 : 2.25
@@ -437,7 +443,7 @@ def run_reference(args, world, rank):
     import oracle
     oracle.build()
     times, nb, sample = [], 0, ""
-    for _ in range(max(args.warmup, 0) and 1):
+    if args.warmup > 0:
         oracle_sample(rows_x=64, rows_w=22, gemm_rows=4)
     for _ in range(args.steps):
         dt, nb, sample = oracle_sample(rows_x=64, rows_w=22, gemm_rows=4)
@@ -460,6 +466,32 @@ def run_reference(args, world, rank):
     print(json.dumps(line), flush=True)
 
 
+def run_profile_kernels(args):
+    """One launch of every kernel on a case sized for an ncu capture: inputs larger
+    than L2 (32768 x 2048 bf16 = 134 MB) but a few hundred MB in all."""
+    import torch
+    import bit_quantization_aware_blockwise_b200 as q
+    from bit_quantization_aware_blockwise_b200 import inputs
+    rows = args.profile_rows
+    dev = torch.device("cuda", 0)
+    x = inputs.activations(rows, C, seed=1).to(dev)
+    g = inputs.upstream_grad(rows, C, seed=4).to(dev)
+    a = torch.from_numpy(inputs.gemm_codes(4096, C, seed=31)).to(dev)
+    b = torch.from_numpy(inputs.gemm_codes(NW, C, seed=32)).to(dev)
+    sa = torch.from_numpy(inputs.positive_scales(4096, 33)).to(dev)
+    sb = torch.from_numpy(inputs.positive_scales(NW, 34)).to(dev)
+    torch.cuda.synchronize()
+    out = q.quantize_fwd(x, BITS, mask_mode=q.MASK_BITS)                               # 1
+    gi = q.trust_bwd(g, out["mask"])                                                   # 2
+    op = q.quantize_fwd(x, BITS, rms_group=C, code_mode=q.CODES_GEMM_OPERAND, mask_mode=None)  # 3
+    y = q.w4a4_linear(a, sa, b, sb)                                                    # 4
+    torch.cuda.synchronize()
+    q.device_status()
+    print(json.dumps({"profile_kernels": "ok", "rows": rows, "checksum": [
+        float(out["scales"].sum()), float(gi.float().abs().sum()), float(op["scales"].sum()),
+        float(y.float().abs().sum())]}))
+
+
 def main():
     ap = argparse.ArgumentParser(description=__doc__)
     ap.add_argument("--gpus", type=int, default=1)
@@ -468,7 +500,13 @@ def main():
     ap.add_argument("--impl", choices=["b200", "reference"], default="b200")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--profile-kernels", action="store_true",
+                    help="launch each kernel once on an ncu-sized case and exit")
+    ap.add_argument("--profile-rows", type=int, default=32768)
     args = ap.parse_args()
+    if args.profile_kernels:
+        run_profile_kernels(args)
+        return
     if args.warmup < 3 and args.impl == "b200":
         args.warmup = 3
     world, rank, local = (int(os.environ.get("WORLD_SIZE", "1")), int(os.environ.get("RANK", "0")),

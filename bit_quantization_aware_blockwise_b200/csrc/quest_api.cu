@@ -14,6 +14,7 @@
 #include "quest.h"
 #include "quest_device.cuh"
 #include "quest_internal.h"
+#include "quest_sync.cuh"
 
 namespace quest {
 namespace {
@@ -98,7 +99,32 @@ int code_bits(int bits, quest_code_mode mode) {
 
 // Constants of the modular code packing (see quantize_fwd.cu): a packed word is
 // (sum_i bits(s_i) * mult * 2^(cb*i) + add) ^ xr, where bits(s_i) = kMagicBits
-// + q_i, so that every field holds q_i + bias (or 2 q_i + 1 + bias) in [0, 2^cb).
+// plus the code, so that every field holds the code plus a bias in [0, 2^cb).
+//
+// Half-slab kernels: codes biased as q_b = q + 2^(b-1) in [0, 2^b - 1];
+// field = q_b + 2^(cb-1) - 2^(b-1), or 2 q_b + 129 - 2^b for the operand form.
+void pack_constants_biased(int cb, int bits, quest_code_mode mode, uint32_t* mult, uint32_t* add,
+                           uint32_t* xr) {
+    // the half-slab kernels pack full 32-bit words: 32, 16, 8 or 4 fields
+    uint32_t rep;
+    switch (cb) {
+        case 1: rep = 0xFFFFFFFFu; *xr = 0xFFFFFFFFu; break;
+        case 2: rep = 0x55555555u; *xr = 0xAAAAAAAAu; break;
+        case 4: rep = 0x11111111u; *xr = 0x88888888u; break;
+        default: rep = 0x01010101u; *xr = 0x80808080u; break;
+    }
+    const uint32_t half_cb = 1u << (cb - 1), half_b = 1u << (bits - 1);
+    if (mode == QUEST_CODES_GEMM_OPERAND) {
+        *mult = 2;
+        *add = ((129u - (1u << bits)) - 2u * kMagicBits) * rep;
+    } else {
+        *mult = 1;
+        *add = ((half_cb - half_b) - kMagicBits) * rep;
+    }
+}
+
+// Direct kernels: 8 fields per word for cb < 8 (4 for cb = 8), codes q; field =
+// q + 2^(cb-1), or 2 q + 1 + 128 for the operand form.
 void pack_constants(int cb, quest_code_mode mode, uint32_t* mult, uint32_t* add, uint32_t* xr) {
     uint32_t bias, rep, m = 1;
     switch (cb) {
@@ -146,6 +172,37 @@ int max_ctas_per_sm(const void* func, int threads, size_t smem) {
         n = 1;
     g_occ[key] = n;
     return n;
+}
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+bool encode_tensor_map(CUtensorMap* map, CUtensorMapDataType dt, int rank, const void* base,
+                       const uint64_t* dims, const uint64_t* strides_bytes, const uint32_t* box,
+                       CUtensorMapSwizzle swz) {
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    });
+    if (!fn || rank < 1 || rank > 5) return false;
+    cuuint64_t d[5], st[4];
+    cuuint32_t b[5], es[5];
+    for (int i = 0; i < rank; ++i) {
+        d[i] = dims[i];
+        b[i] = box[i];
+        es[i] = 1;
+        if (i + 1 < rank) st[i] = strides_bytes[i];
+    }
+    return fn(map, dt, (cuuint32_t)rank, const_cast<void*>(base), d, st, b, es,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 }  // namespace quest
@@ -258,11 +315,18 @@ quest_status quest_quantize_fwd(const void* x, quest_dtype x_dtype, int64_t rows
     c.s_lo = kMagic + (float)lo;
     c.s_hi = kMagic + (float)hi;
     pack_constants(cb, code_mode, &c.pack_mult, &c.pack_add, &c.pack_xor);
+    c.inv_levels = (float)ldexp(1.0, -bits);
+    c.half_levels = (float)ldexp(1.0, bits - 1);
+    c.sat_k = (float)(ldexp(1.0, bits) * (1.0 - ldexp(1.0, -23)));
+    c.s_mid = kMagic + (float)ldexp(1.0, bits - 1);
+    c.s_top = kMagic + (float)(ldexp(1.0, bits) - 1.0);
+    c.cell_center = (float)(0.5 - ldexp(1.0, bits - 1));
+    pack_constants_biased(cb, bits, code_mode, &c.pack2_mult, &c.pack2_add, &c.pack2_xor);
     c.trust_ge1 = trust >= 1.0f;
     c.mask_mode = mask ? (int)mask_mode : -1;
     c.deq_mode = dequant ? (int)dequant_dtype : -1;
 
-    cudaError_t e = launch_quantize(a, x_dtype, had_block, cb, row_mode, static_cast<cudaStream_t>(stream));
+    cudaError_t e = launch_quantize(a, x_dtype, had_block, cb, bits, row_mode, static_cast<cudaStream_t>(stream));
     if (e != cudaSuccess) return cuda_fail(e, "quest_quantize_fwd launch");
     return QUEST_OK;
 }
@@ -327,10 +391,17 @@ quest_status quest_w4a4_linear(const int8_t* a_codes, const float* a_scales,
 
 quest_status quest_device_status(void* stream) {
     g_last_error.clear();
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
     cudaError_t e = cudaSuccess;
-    const int v = read_and_clear_gemm_status(static_cast<cudaStream_t>(stream), &e);
+    const int vg = read_and_clear_gemm_status(s, &e);
     if (e != cudaSuccess) return cuda_fail(e, "quest_device_status");
-    if (v != 0) return fail((quest_status)v, "a bounded device-side wait in quest_w4a4_linear gave up");
+    const int vq = read_and_clear_quant_status(s, &e);
+    if (e != cudaSuccess) return cuda_fail(e, "quest_device_status");
+    const int vt = read_and_clear_trust_status(s, &e);
+    if (e != cudaSuccess) return cuda_fail(e, "quest_device_status");
+    if (vg != 0) return fail((quest_status)vg, "a bounded device-side wait in quest_w4a4_linear gave up");
+    if (vq != 0) return fail((quest_status)vq, "a bounded device-side wait in quest_quantize_fwd gave up");
+    if (vt != 0) return fail((quest_status)vt, "a bounded device-side wait in quest_trust_bwd gave up");
     return QUEST_OK;
 }
 

@@ -20,6 +20,14 @@ struct QuantConsts {
     uint32_t pack_mult; // 1, or 2 for the c = 2q+1 operand form
     uint32_t pack_add;  // additive constant of the modular packing (see quantize_fwd.cu)
     uint32_t pack_xor;  // un-biasing mask of the packed word
+    // half-slab (TMA-staged) decision path, codes biased as q_b = q + 2^(b-1)
+    float inv_levels;   // 2^-b
+    float half_levels;  // 2^(b-1)
+    float sat_k;        // 2^b (1 - 2^-23)
+    float s_mid;        // kMagic + 2^(b-1)
+    float s_top;        // kMagic + 2^b - 1
+    float cell_center;  // 1/2 - 2^(b-1): q + 1/2 = q_b + cell_center
+    uint32_t pack2_mult, pack2_add, pack2_xor;
     int trust_ge1;      // 1: use m = [|t| <= edge]
     int mask_mode;      // -1 none, 0 bits, 1 bytes
     int deq_mode;       // -1 none, 0 bf16, 1 fp32
@@ -51,7 +59,9 @@ struct TrustArgs {
 
 // Launchers (return cudaSuccess or the launch error).
 cudaError_t launch_quantize(const QuantArgs& a, quest_dtype x_dtype, int had_block, int cbits,
-                            bool row_mode, cudaStream_t stream);
+                            int bits, bool row_mode, cudaStream_t stream);
+int read_and_clear_quant_status(cudaStream_t stream, cudaError_t* err);
+int read_and_clear_trust_status(cudaStream_t stream, cudaError_t* err);
 cudaError_t launch_trust_bwd(const TrustArgs& a, int had_block, cudaStream_t stream);
 cudaError_t launch_w4a4(const int8_t* A, const float* sa, const int8_t* B, const float* sb,
                         int64_t M, int64_t N, int64_t K, uint16_t* y, int32_t* acc,

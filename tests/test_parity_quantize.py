@@ -70,8 +70,8 @@ def test_smoke_config_fp32_256x512(cuda_device):
     o = oracle.quantize(inputs.to_f64(x), bits=4, had=128)
     res = run_gpu(x, 4, code_mode=q.CODES_INT8, mask_mode=q.MASK_BYTES, dequant="fp32")
     n_ex = check_all(res, o, 4, q.CODES_INT8)
-    assert n_ex <= 2
-    assert np.array_equal(res["codes"], o["q"]) or n_ex > 0
+    # the exempt set is a property of the data: values within 1e-5 of a boundary
+    assert n_ex <= 1e-4 * x.numel()
 
 
 @pytest.mark.parametrize("bits", [1, 2, 3, 4, 5, 6, 7, 8])
@@ -118,7 +118,7 @@ def test_row_rms_operand_codes(cuda_device, cols):
     check_all(res, o, 4, q.CODES_GEMM_OPERAND)
 
 
-@pytest.mark.parametrize("had,cols", [(16, 8192), (64, 1024), (256, 4096)])
+@pytest.mark.parametrize("had,cols", [(16, 8192), (32, 2048), (64, 1024), (256, 4096), (16, 1024)])
 def test_row_rms_other_blocks(cuda_device, had, cols):
     x = inputs.weights(9, cols, seed=had)
     o = oracle.quantize(inputs.to_f64(x), bits=2, had=had, rms_group=cols)
@@ -198,3 +198,41 @@ def test_mask_rate_on_gaussian_rows(cuda_device):
         p = 2 * scipy.stats.norm.sf(q.alpha(bits))
         n = res["mask"].size
         assert abs(rate - p) < 5 * np.sqrt(p * (1 - p) / n) + 2e-4
+
+
+@pytest.mark.parametrize("had,cols", [(16, 80), (32, 96), (64, 192), (64, 320)])
+def test_rows_not_multiple_of_128_use_the_direct_kernel(cuda_device, had, cols):
+    x = inputs.activations(29, cols, seed=cols)
+    for bits in (1, 4):
+        o = oracle.quantize(inputs.to_f64(x), bits=bits, had=had)
+        check_all(run_gpu(x, bits, had=had), o, bits)
+        o = oracle.quantize(inputs.to_f64(x), bits=bits, had=had, rms_group=cols)
+        check_all(run_gpu(x, bits, had=had, rms_group=cols), o, bits)
+
+
+@pytest.mark.parametrize("bits", [2, 4, 8])
+def test_under_aligned_outputs_use_the_direct_kernel(cuda_device, bits):
+    # codes (and mask bits) just past an allocation's start: valid for the ABI, too
+    # little alignment for the staged kernel's vector stores.
+    dev = torch.device("cuda:0")
+    x_cpu = inputs.activations(40, 512, seed=bits)
+    x = x_cpu.to(dev)
+    nb = q.codes_bytes(40, 512, bits)
+    codes = torch.zeros(nb + 64, dtype=torch.uint8, device=dev)
+    mask = torch.zeros(40 * 512 // 8 + 64, dtype=torch.uint8, device=dev)
+    scales = torch.zeros(40 * 4, dtype=torch.float32, device=dev)
+    # the ABI's own minimum alignment for this container, but not 16 bytes
+    off = {1: 1, 2: 2, 4: 4, 8: 8}[q.container_bits(bits)]
+    q.quantize_fwd_raw(x.data_ptr(), 0, 40, 512, 512, bits, 128, 128, 1.0, q.CODES_PACKED,
+                       codes.data_ptr() + off, scales.data_ptr(), q.MASK_BITS, mask.data_ptr() + 1,
+                       None, 0, torch.cuda.current_stream().cuda_stream)
+    torch.cuda.synchronize()
+    o = oracle.quantize(inputs.to_f64(x_cpu), bits=bits, had=128)
+    res = {"codes": unpack_codes(codes.cpu().numpy()[off:off + nb], 40, 512, bits, q.CODES_PACKED),
+           "scales": scales.cpu().numpy().reshape(40, 4),
+           "mask": unpack_mask_bits(mask.cpu().numpy()[1:1 + 40 * 64], 40, 512)}
+    check_all(res, o, bits)
+
+
+def test_device_status_is_clean_after_the_suite(cuda_device):
+    q.device_status()

@@ -102,3 +102,27 @@ def test_empty(cuda_device):
     out = q.trust_bwd(g, m)
     torch.cuda.synchronize()
     assert out.shape == (0, 256)
+
+
+def test_under_aligned_mask_uses_the_direct_kernel(cuda_device):
+    dev = torch.device("cuda:0")
+    g = inputs.upstream_grad(24, 512, seed=3)
+    m = inputs.random_mask(24, 512, seed=4, keep_prob=0.9)
+    bits = torch.from_numpy(inputs.pack_mask_bits(m).view(np.uint8).reshape(-1))
+    buf = torch.zeros(bits.numel() + 16, dtype=torch.uint8)
+    buf[3:3 + bits.numel()] = bits
+    buf = buf.to(dev)
+    gd = g.to(dev)
+    out = torch.empty_like(gd)
+    q.trust_bwd_raw(gd.data_ptr(), buf.data_ptr() + 3, q.MASK_BITS, 24, 512, 128, out.data_ptr(),
+                    torch.cuda.current_stream().cuda_stream)
+    torch.cuda.synchronize()
+    ref = oracle.trust_bwd(inputs.to_f64(g), m, had=128)
+    check_bf16(out.cpu().view(torch.int16).numpy().view(np.uint16), ref, floor=_block_rms(ref, 128))
+
+
+@pytest.mark.parametrize("had,cols", [(16, 48), (64, 192)])
+def test_rows_not_multiple_of_128(cuda_device, had, cols):
+    g = inputs.upstream_grad(17, cols, seed=cols)
+    m = inputs.random_mask(17, cols, seed=1, keep_prob=0.8)
+    check(g, m, had, q.MASK_BYTES)
