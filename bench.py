@@ -62,6 +62,30 @@ def part_bytes():
 
 GEMM_OPS = 2 * R * NW * C
 
+# DRAM traffic per launch of the dominant kernel, from one ncu capture of the full
+# workload (dram__bytes_read.sum + dram__bytes_write.sum, one pass; the summary is in
+# profiles/launches_hot_path_16384x2048.md). Reported only while the kernel's source
+# file is byte-identical to the one that was captured; otherwise null.
+NCU_TRAFFIC = {
+    "w4a4_linear": {"source": "bit_quantization_aware_blockwise_b200/csrc/w4a4_gemm.cu",
+                    "sha256": "ddc0e88b8a8950c47e30c5caff33b44293baa26c0ffd328eff565ec84e9bb928",
+                    "dram_read": 65479168, "dram_write": 145387008},
+}
+
+
+def ncu_traffic(part):
+    import hashlib
+    rec = NCU_TRAFFIC.get(part)
+    if rec is None:
+        return None
+    try:
+        with open(os.path.join(ROOT, rec["source"]), "rb") as f:
+            if hashlib.sha256(f.read()).hexdigest() != rec["sha256"]:
+                return None
+    except OSError:
+        return None
+    return rec["dram_read"] + rec["dram_write"]
+
 
 def load_peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
@@ -80,7 +104,7 @@ def load_peaks():
 # clocks during the timed region (NVML, polled from a thread)
 # ---------------------------------------------------------------------------
 class ClockSampler:
-    def __init__(self, torch_device_index, period_s=0.01):
+    def __init__(self, torch_device_index, period_s=0.001):
         self.period = period_s
         self.samples = []
         self.max_mhz = None
@@ -318,12 +342,13 @@ def run_b200(args, world, rank, local):
                     "peak": round(int8_peak, 1), "unit": "TOPS",
                     "frac": round(achieved / int8_peak, 4),
                     "peak_source": f"{peaks['source']} bf16 burst x 2 (nominal int8/bf16 dense ratio)",
-                    "traffic": None}
+                    "traffic": ncu_traffic(dominant), "traffic_unit": "bytes per launch (ncu DRAM read+write)"}
     else:
         achieved = pbytes[dominant] / (avg[dominant] * 1e-3) / 1e9
         roofline = {"kernel": dominant, "bound": "hbm", "achieved": round(achieved, 1),
                     "peak": hbm, "unit": "GB/s", "frac": round(achieved / hbm, 4),
-                    "peak_source": peaks["source"], "traffic": None}
+                    "peak_source": peaks["source"], "traffic": ncu_traffic(dominant),
+                    "traffic_unit": "bytes per launch (ncu DRAM read+write)"}
 
     # ---- end to end: pinned host inputs -> device, the step, results -> host
     e2e = None
@@ -495,7 +520,7 @@ def run_profile_kernels(args):
 def main():
     ap = argparse.ArgumentParser(description=__doc__)
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["b200", "reference"], default="b200")
     ap.add_argument("--no-e2e", action="store_true")

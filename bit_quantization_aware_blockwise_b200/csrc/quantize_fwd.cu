@@ -313,15 +313,16 @@ cudaError_t launch_dtype(const QuantArgs& a, int hb, int cbits, bool row_mode, c
 
 }  // namespace
 // ===========================================================================
-// TMA-staged quantizer (dense rows whose length is a multiple of 128).
+// TMA-staged quantizer, one RMS group per Hadamard block (rows whose length is
+// a multiple of 128).
 //
 // One persistent CTA per SM: warp 0 streams tiles of whole 128-element slabs
 // into a ring of shared-memory stages with 3-D TMA copies (128-byte swizzle);
-// 8 consumer warps take each stage, two lanes per slab (half-slab layout,
-// quest_device.cuh), transform with packed fp32x2 butterflies and write codes,
-// mask bits, scales and (optionally) dequantised values straight to global
-// memory (every store covers whole 32-byte sectors). A stage is released as
-// soon as its consumers have its data in registers.
+// 11 consumer warps (8 for fp32 input) take each stage, two lanes per slab
+// (half-slab layout, quest_device.cuh), transform with packed fp32x2
+// butterflies and write codes, mask bits, scales and (optionally) dequantised
+// values to global memory with 8- and 16-byte vector stores. A stage is
+// released as soon as its consumers have its data in registers.
 //
 // Per element, the decision path is: u = sat(y_u * a + c) (one FMA that also
 // clamps), s = fma_rd(u, 2^b (1 - 2^-23), 1.5*2^23) (packed: the biased code
@@ -334,7 +335,6 @@ cudaError_t launch_dtype(const QuantArgs& a, int hb, int cbits, bool row_mode, c
 namespace tma {
 
 constexpr int kStageBudget = 192 * 1024;
-constexpr int kNamedBar = 1;
 
 // Shape of the CTA and its stage ring: bf16 inputs run 11 consumer warps (176
 // slabs, 44 KB per stage, 4 stages), fp32 inputs 8 (128 slabs, 64 KB, 3 stages).
@@ -354,11 +354,9 @@ struct Geo {
     static constexpr int kStages = kStageBudget / kStageBytes; // 4 (bf16) or 3 (fp32)
     static constexpr int kMaxSlabCols = 256 / (2 * kRowsPerHalf);  // box dim 1 <= 256
     static constexpr int kBarOffset = kStages * kStageBytes;
-    // bars: full[kStages], empty[kStages]; then abort flag; partial sums; row sums
+    // bars: full[kStages], empty[kStages]; then the abort flag
     static constexpr int kAbortOffset = kBarOffset + 16 * kStages;
-    static constexpr int kPartialOffset = kAbortOffset + 16;
-    static constexpr int kRowSumOffset = kPartialOffset + 4 * kConsumerThreads;
-    static constexpr int kSmemUsed = kRowSumOffset + 4 * kSlabsPerStage;
+    static constexpr int kSmemUsed = kAbortOffset + 16;
     static constexpr int kSmemTotal = kSmemUsed + 1024;
 };
 
@@ -584,7 +582,7 @@ __device__ __forceinline__ void emit_half(const QuantArgs& A, const float2 (&P)[
     }
 }
 
-template <typename Tin, int HB, int CB, bool MULT2, bool ROW_MODE, bool SAT>
+template <typename Tin, int HB, int CB, bool MULT2, bool SAT>
 __global__ void __launch_bounds__(Geo<Tin>::kThreads, 1)
 quantize_tma_kernel(const __grid_constant__ CUtensorMap map_x, const QuantArgs A, const TileGeo g) {
     using Gm = Geo<Tin>;
@@ -596,8 +594,6 @@ quantize_tma_kernel(const __grid_constant__ CUtensorMap map_x, const QuantArgs A
     const uint32_t bar_full = sbase + Gm::kBarOffset;
     const uint32_t bar_empty = bar_full + 8 * Gm::kStages;
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Gm::kAbortOffset);
-    float* partial = reinterpret_cast<float*>(smem + Gm::kPartialOffset);
-    float* rowsum = reinterpret_cast<float*>(smem + Gm::kRowSumOffset);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
     if (threadIdx.x == 0) {
@@ -648,11 +644,7 @@ quantize_tma_kernel(const __grid_constant__ CUtensorMap map_x, const QuantArgs A
         const uint32_t st = it % Gm::kStages, ph = (it / Gm::kStages) & 1;
         const bool got = sync::mbar_wait(bar_full + 8 * st, ph, abort_flag, &g_quant_status,
                                          (int)QUEST_ETIMEOUT);
-        // on a timeout the lanes of a warp leave together (row mode: the whole CTA,
-        // at the first reduction barrier below)
-        if constexpr (!ROW_MODE) {
-            if (__any_sync(0xFFFFFFFFu, !got)) break;
-        }
+        if (__any_sync(0xFFFFFFFFu, !got)) break;   // on a timeout the warp leaves together
         float2 P[32];
         read_half_slab<Tin>(sbase + st * Gm::kStageBytes, row0, P);
         sync::mbar_arrive(bar_empty + 8 * st);
@@ -679,56 +671,31 @@ quantize_tma_kernel(const __grid_constant__ CUtensorMap map_x, const QuantArgs A
             ssb[b] = slot_ok ? acc[0].x + acc[0].y : 0.0f;
         }
         GroupK G[BPL];
-        if constexpr (ROW_MODE) {
-            float lane_ss = 0.0f;
 #pragma unroll
-            for (int b = 0; b < BPL; ++b) lane_ss += ssb[b];
-            partial[L] = got ? lane_ss : 0.0f;
-            if (sync::named_bar_any(kNamedBar, Gm::kConsumerThreads, !got)) break;
-            // one warp per tile row sums that row's 2*S_c lane partials in a fixed order
-            for (int r = warp - 1; r < g.R_t; r += Gm::kConsumerWarps) {
-                const int base = r * 2 * g.S_c;
-                float v = 0.0f;
-                for (int i = lane; i < 2 * g.S_c; i += 32) v += partial[base + i];
-#pragma unroll
-                for (int s = 16; s >= 1; s >>= 1) v += __shfl_xor_sync(0xFFFFFFFFu, v, s);
-                if (lane == 0) rowsum[r] = v;
-            }
-            sync::named_bar(kNamedBar, Gm::kConsumerThreads);
-            G[0] = make_group(A.c, slot_ok ? rowsum[sr] : 0.0f);
-#pragma unroll
-            for (int b = 1; b < BPL; ++b) G[b] = G[0];   // one RMS group per row
-        } else {
-#pragma unroll
-            for (int b = 0; b < BPL; ++b) {
-                float v = ssb[b];
-                if constexpr (HB >= 128) v += __shfl_xor_sync(0xFFFFFFFFu, v, 1);
-                if constexpr (HB >= 256) v += __shfl_xor_sync(0xFFFFFFFFu, v, 2);
-                G[b] = make_group(A.c, v);
-            }
+        for (int b = 0; b < BPL; ++b) {
+            float v = ssb[b];
+            if constexpr (HB >= 128) v += __shfl_xor_sync(0xFFFFFFFFu, v, 1);
+            if constexpr (HB >= 256) v += __shfl_xor_sync(0xFFFFFFFFu, v, 2);
+            G[b] = make_group(A.c, v);
         }
         if (valid) {
             const int64_t e0 = int64_t(scol) * 128 + half * 64;
             emit_half<HB, CB, MULT2, SAT>(A, P, G, row, e0);
-            if constexpr (ROW_MODE) {
-                if (sc == 0 && half == 0) A.scales[row] = G[0].delta;
+            const int64_t gpr = A.cols / HB;   // groups per row
+            if constexpr (HB >= 128) {
+                if ((L & (HB / 64 - 1)) == 0) A.scales[row * gpr + e0 / HB] = G[0].delta;
             } else {
-                const int64_t gpr = A.cols / HB;   // groups per row
-                if constexpr (HB >= 128) {
-                    if ((L & (HB / 64 - 1)) == 0) A.scales[row * gpr + e0 / HB] = G[0].delta;
-                } else {
 #pragma unroll
-                    for (int b = 0; b < BPL; ++b) A.scales[row * gpr + e0 / HB + b] = G[b].delta;
-                }
+                for (int b = 0; b < BPL; ++b) A.scales[row * gpr + e0 / HB + b] = G[b].delta;
             }
         }
     }
 }
 
-template <typename Tin, int HB, int CB, bool MULT2, bool ROW, bool SAT>
+template <typename Tin, int HB, int CB, bool MULT2, bool SAT>
 cudaError_t launch_tma_t(const QuantArgs& a, const TileGeo& g, const CUtensorMap& map, cudaStream_t s) {
     using Gm = Geo<Tin>;
-    auto fn = quantize_tma_kernel<Tin, HB, CB, MULT2, ROW, SAT>;
+    auto fn = quantize_tma_kernel<Tin, HB, CB, MULT2, SAT>;
     static thread_local int attr_dev = -1;
     int dev = 0;
     cudaGetDevice(&dev);
@@ -744,45 +711,37 @@ cudaError_t launch_tma_t(const QuantArgs& a, const TileGeo& g, const CUtensorMap
 }
 
 template <typename Tin, int HB, int CB, bool MULT2>
-cudaError_t launch_tma_cb(const QuantArgs& a, int bits, bool row, const TileGeo& g,
-                          const CUtensorMap& map, cudaStream_t s) {
-    const bool sat = bits <= 6;
-    if (row) return sat ? launch_tma_t<Tin, HB, CB, MULT2, true, true>(a, g, map, s)
-                        : launch_tma_t<Tin, HB, CB, MULT2, true, false>(a, g, map, s);
-    return sat ? launch_tma_t<Tin, HB, CB, MULT2, false, true>(a, g, map, s)
-               : launch_tma_t<Tin, HB, CB, MULT2, false, false>(a, g, map, s);
+cudaError_t launch_tma_cb(const QuantArgs& a, int bits, const TileGeo& g, const CUtensorMap& map,
+                          cudaStream_t s) {
+    return bits <= 6 ? launch_tma_t<Tin, HB, CB, MULT2, true>(a, g, map, s)
+                     : launch_tma_t<Tin, HB, CB, MULT2, false>(a, g, map, s);
 }
 
 template <typename Tin, int HB>
-cudaError_t launch_tma_hb(const QuantArgs& a, int bits, int cb, bool row, const TileGeo& g,
+cudaError_t launch_tma_hb(const QuantArgs& a, int bits, int cb, const TileGeo& g,
                           const CUtensorMap& map, cudaStream_t s) {
     switch (cb) {
-        case 1: return launch_tma_cb<Tin, HB, 1, false>(a, bits, row, g, map, s);
-        case 2: return launch_tma_cb<Tin, HB, 2, false>(a, bits, row, g, map, s);
-        case 4: return launch_tma_cb<Tin, HB, 4, false>(a, bits, row, g, map, s);
-        case 8: return a.c.pack2_mult == 2 ? launch_tma_cb<Tin, HB, 8, true>(a, bits, row, g, map, s)
-                                           : launch_tma_cb<Tin, HB, 8, false>(a, bits, row, g, map, s);
+        case 1: return launch_tma_cb<Tin, HB, 1, false>(a, bits, g, map, s);
+        case 2: return launch_tma_cb<Tin, HB, 2, false>(a, bits, g, map, s);
+        case 4: return launch_tma_cb<Tin, HB, 4, false>(a, bits, g, map, s);
+        case 8: return a.c.pack2_mult == 2 ? launch_tma_cb<Tin, HB, 8, true>(a, bits, g, map, s)
+                                           : launch_tma_cb<Tin, HB, 8, false>(a, bits, g, map, s);
     }
     return cudaErrorInvalidValue;
 }
 
 template <typename Tin>
-cudaError_t launch_tma(const QuantArgs& a, int bits, int hb, int cb, bool row, cudaStream_t s) {
+cudaError_t launch_tma(const QuantArgs& a, int bits, int hb, int cb, cudaStream_t s) {
     using Gm = Geo<Tin>;
     TileGeo g;
     g.spr = (int)(a.cols / 128);
-    if (row) {
-        g.S_c = g.spr;
-        g.R_t = Gm::kSlabsPerStage / g.S_c;
-    } else {
-        g.S_c = g.spr < Gm::kMaxSlabCols ? g.spr : Gm::kMaxSlabCols;
-        if (g.S_c > Gm::kSlabsPerStage) g.S_c = Gm::kSlabsPerStage;
-        g.R_t = Gm::kSlabsPerStage / g.S_c;
-        // keep at least ~4 tiles per SM on small tensors
-        const int64_t want_tiles = 4LL * sm_count();
-        while (g.R_t > 1 && ((a.rows + g.R_t - 1) / g.R_t) * ((g.spr + g.S_c - 1) / g.S_c) < want_tiles)
-            g.R_t = (g.R_t + 1) / 2;
-    }
+    g.S_c = g.spr < Gm::kMaxSlabCols ? g.spr : Gm::kMaxSlabCols;
+    if (g.S_c > Gm::kSlabsPerStage) g.S_c = Gm::kSlabsPerStage;
+    g.R_t = Gm::kSlabsPerStage / g.S_c;
+    // keep at least ~4 tiles per SM on small tensors
+    const int64_t want_tiles = 4LL * sm_count();
+    while (g.R_t > 1 && ((a.rows + g.R_t - 1) / g.R_t) * ((g.spr + g.S_c - 1) / g.S_c) < want_tiles)
+        g.R_t = (g.R_t + 1) / 2;
     g.tiles_c = (g.spr + g.S_c - 1) / g.S_c;
     const int64_t tiles_r = (a.rows + g.R_t - 1) / g.R_t;
     if (tiles_r * g.tiles_c > 0x7FFFFFFF) return cudaErrorInvalidValue;
@@ -796,11 +755,11 @@ cudaError_t launch_tma(const QuantArgs& a, int bits, int hb, int cb, bool row, c
                            3, a.x, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B))
         return cudaErrorInvalidValue;
     switch (hb) {
-        case 16: return launch_tma_hb<Tin, 16>(a, bits, cb, row, g, map, s);
-        case 32: return launch_tma_hb<Tin, 32>(a, bits, cb, row, g, map, s);
-        case 64: return launch_tma_hb<Tin, 64>(a, bits, cb, row, g, map, s);
-        case 128: return launch_tma_hb<Tin, 128>(a, bits, cb, row, g, map, s);
-        case 256: return launch_tma_hb<Tin, 256>(a, bits, cb, row, g, map, s);
+        case 16: return launch_tma_hb<Tin, 16>(a, bits, cb, g, map, s);
+        case 32: return launch_tma_hb<Tin, 32>(a, bits, cb, g, map, s);
+        case 64: return launch_tma_hb<Tin, 64>(a, bits, cb, g, map, s);
+        case 128: return launch_tma_hb<Tin, 128>(a, bits, cb, g, map, s);
+        case 256: return launch_tma_hb<Tin, 256>(a, bits, cb, g, map, s);
     }
     return cudaErrorInvalidValue;
 }
@@ -808,7 +767,13 @@ cudaError_t launch_tma(const QuantArgs& a, int bits, int hb, int cb, bool row, c
 }  // namespace tma
 
 // Whether the TMA-staged kernel handles this request (otherwise the direct one does).
+// Path choice, from measurements on B200 at the 16384 x 2048 activation shape:
+// the staged kernel wins for one RMS per block (b = 4: 32.8 vs 37.9 us), the
+// direct kernel for one RMS per row (36.9 vs 37.9 us; 18.5 vs 20.5 us for the
+// 5632 x 2048 weights). Staged streaming tops out near 4.7 TB/s on this part,
+// below plain 16-byte loads, so the direct kernel keeps the rows it wins.
 bool tma_path_ok(const QuantArgs& a, quest_dtype x_dtype, int cbits, bool row_mode) {
+    if (row_mode) return false;
     if (a.cols % 128 != 0) return false;
     const int esize = x_dtype == QUEST_BF16 ? 2 : 4;
     if (a.ld_x_bytes % 16 != 0 || (reinterpret_cast<uintptr_t>(a.x) & 15) != 0) return false;
@@ -824,8 +789,8 @@ bool tma_path_ok(const QuantArgs& a, quest_dtype x_dtype, int cbits, bool row_mo
 cudaError_t launch_quantize(const QuantArgs& a, quest_dtype x_dtype, int had_block, int cbits,
                             int bits, bool row_mode, cudaStream_t stream) {
     if (tma_path_ok(a, x_dtype, cbits, row_mode)) {
-        if (x_dtype == QUEST_BF16) return tma::launch_tma<__nv_bfloat16>(a, bits, had_block, cbits, row_mode, stream);
-        return tma::launch_tma<float>(a, bits, had_block, cbits, row_mode, stream);
+        if (x_dtype == QUEST_BF16) return tma::launch_tma<__nv_bfloat16>(a, bits, had_block, cbits, stream);
+        return tma::launch_tma<float>(a, bits, had_block, cbits, stream);
     }
     if (x_dtype == QUEST_BF16) return launch_dtype<__nv_bfloat16>(a, had_block, cbits, row_mode, stream);
     return launch_dtype<float>(a, had_block, cbits, row_mode, stream);

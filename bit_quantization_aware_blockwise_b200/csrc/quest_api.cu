@@ -397,11 +397,8 @@ quest_status quest_device_status(void* stream) {
     if (e != cudaSuccess) return cuda_fail(e, "quest_device_status");
     const int vq = read_and_clear_quant_status(s, &e);
     if (e != cudaSuccess) return cuda_fail(e, "quest_device_status");
-    const int vt = read_and_clear_trust_status(s, &e);
-    if (e != cudaSuccess) return cuda_fail(e, "quest_device_status");
     if (vg != 0) return fail((quest_status)vg, "a bounded device-side wait in quest_w4a4_linear gave up");
     if (vq != 0) return fail((quest_status)vq, "a bounded device-side wait in quest_quantize_fwd gave up");
-    if (vt != 0) return fail((quest_status)vt, "a bounded device-side wait in quest_trust_bwd gave up");
     return QUEST_OK;
 }
 

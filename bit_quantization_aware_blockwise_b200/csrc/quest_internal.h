@@ -61,7 +61,6 @@ struct TrustArgs {
 cudaError_t launch_quantize(const QuantArgs& a, quest_dtype x_dtype, int had_block, int cbits,
                             int bits, bool row_mode, cudaStream_t stream);
 int read_and_clear_quant_status(cudaStream_t stream, cudaError_t* err);
-int read_and_clear_trust_status(cudaStream_t stream, cudaError_t* err);
 cudaError_t launch_trust_bwd(const TrustArgs& a, int had_block, cudaStream_t stream);
 cudaError_t launch_w4a4(const int8_t* A, const float* sa, const int8_t* B, const float* sb,
                         int64_t M, int64_t N, int64_t K, uint16_t* y, int32_t* acc,
