@@ -27,6 +27,7 @@
 #include "quest_device.cuh"
 #include "quest_internal.h"
 #include "quest_sync.cuh"
+#include "quest_emit.cuh"
 
 namespace quest {
 namespace {
@@ -397,111 +398,6 @@ __device__ __forceinline__ void read_half_slab(uint32_t stage_base, uint32_t row
     }
 }
 
-// Per-group constants of the decision path.
-struct GroupK {
-    float delta;   // Delta
-    float a, c;    // u = sat(y_u * a + c)      (saturating path)
-    float inv;     // t = y_u * inv             (exact path, general mask)
-    float thr2;    // (edge * sqrt(HB) * Delta)^2
-    float ch;      // yhat = q_b * Delta + ch
-};
-
-__device__ __forceinline__ GroupK make_group(const QuantConsts& k, float ss) {
-    GroupK g;
-    const float r = sqrtf(ss * k.inv_count);
-    g.delta = k.c_delta * r;
-    if (g.delta > 0.0f) {
-        const float sd = k.sqrt_hb * g.delta;
-        g.inv = __frcp_rn(sd);
-        g.a = g.inv * k.inv_levels;
-        g.c = 0.5f;
-        const float thr = k.edge * sd;
-        g.thr2 = thr * thr;
-    } else {
-        g.inv = 0.0f;
-        g.a = 0.0f;
-        g.c = 0.5f + 0.5f * k.inv_levels;   // lands in the cell of q = 0
-        g.thr2 = __int_as_float(0x7F800000);
-    }
-    g.ch = (0.5f - k.half_levels) * g.delta;
-    return g;
-}
-
-// Biased code s = kMagic + q_b of a pair of transformed values.
-template <bool SAT>
-__device__ __forceinline__ float2 decide(float2 y, const GroupK& g, const QuantConsts& k) {
-    if constexpr (SAT) {
-        const float2 u = make_float2(__saturatef(__fmaf_rn(y.x, g.a, g.c)),
-                                     __saturatef(__fmaf_rn(y.y, g.a, g.c)));
-        return __ffma2_rd(u, make_float2(k.sat_k, k.sat_k), make_float2(kMagic, kMagic));
-    } else {
-        const float2 t = __ffma2_rd(y, make_float2(g.inv, g.inv), make_float2(k.s_mid, k.s_mid));
-        return make_float2(fminf(fmaxf(t.x, kMagic), k.s_top), fminf(fmaxf(t.y, kMagic), k.s_top));
-    }
-}
-
-// Packed code word of elements [w*EPW, (w+1)*EPW) of the half-slab. The sum is
-// split over independent partial sums of 8 fields so the dependency chains
-// stay short.
-template <int HB, int CB, bool MULT2, bool SAT>
-__device__ __forceinline__ uint32_t code_word(const float2 (&P)[32], const GroupK* G, int w,
-                                              const QuantConsts& k) {
-    constexpr uint32_t kMult = MULT2 ? 2u : 1u;
-    constexpr int EPW = 32 / CB;
-    constexpr int PPB = 32 / ((HB >= 64) ? 1 : 64 / HB);
-    constexpr int NSUB = EPW >= 8 ? EPW / 8 : 1;
-    constexpr int PER = EPW / NSUB;
-    uint32_t part[NSUB];
-#pragma unroll
-    for (int u = 0; u < NSUB; ++u) {
-        uint32_t acc = 0;
-#pragma unroll
-        for (int i = u * PER; i < (u + 1) * PER; i += 2) {
-            const int j = (w * EPW + i) / 2;
-            const float2 s2 = decide<SAT>(P[j], G[j / PPB], k);
-            acc += __float_as_uint(s2.x) * (kMult << (CB * i));
-            acc += __float_as_uint(s2.y) * (kMult << (CB * (i + 1)));
-        }
-        part[u] = acc;
-    }
-    uint32_t word = k.pack2_add;
-#pragma unroll
-    for (int u = 0; u < NSUB; ++u) word += part[u];
-    return word ^ k.pack2_xor;
-}
-
-// Trust-mask byte of elements [8*byte, 8*byte + 8): bit i = element 8*byte + i.
-template <int HB>
-__device__ __forceinline__ uint32_t mask_byte(const float2 (&P)[32], const GroupK* G, int byte,
-                                              const QuantConsts& k) {
-    constexpr int PPB = 32 / ((HB >= 64) ? 1 : 64 / HB);
-    uint32_t acc = 0;
-    if (k.trust_ge1) {
-#pragma unroll
-        for (int j = 4 * byte + 3; j >= 4 * byte; --j) {
-            const float t2 = G[j / PPB].thr2;
-            const float2 d = __ffma2_rn(P[j], P[j], make_float2(-t2, -t2));
-            acc = __funnelshift_l(__float_as_uint(d.y), acc, 1);
-            acc = __funnelshift_l(__float_as_uint(d.x), acc, 1);
-        }
-    } else {
-#pragma unroll
-        for (int j = 4 * byte + 3; j >= 4 * byte; --j) {
-            const GroupK& g = G[j / PPB];
-            // q + 1/2 = q_b + cell_center, q_b from the exact floor of t
-            const float2 t = __fmul2_rn(P[j], make_float2(g.inv, g.inv));
-            float2 sf = __ffma2_rd(P[j], make_float2(g.inv, g.inv), make_float2(k.s_mid, k.s_mid));
-            sf = make_float2(fminf(fmaxf(sf.x, kMagic), k.s_top), fminf(fmaxf(sf.y, kMagic), k.s_top));
-            const float ex = fabsf(t.x - ((sf.x - kMagic) + k.cell_center)) - k.half_trust;
-            const float ey = fabsf(t.y - ((sf.y - kMagic) + k.cell_center)) - k.half_trust;
-            const bool zero_group = !(g.delta > 0.0f);
-            acc = __funnelshift_l(__float_as_uint(zero_group ? -1.0f : ey), acc, 1);
-            acc = __funnelshift_l(__float_as_uint(zero_group ? -1.0f : ex), acc, 1);
-        }
-    }
-    return acc;
-}
-
 // Quantise, pack and store the 64 values of one half-slab. `e0` is the index
 // of its first element within its row; outputs are dense [rows, cols].
 template <int HB, int CB, bool MULT2, bool SAT>
@@ -516,13 +412,13 @@ __device__ __forceinline__ void emit_half(const QuantArgs& A, const float2 (&P)[
         uint8_t* dst = A.codes + row * A.codes_row_bytes + e0 * CB / 8;
         if constexpr (NW == 2) {
             *reinterpret_cast<uint2*>(dst) =
-                make_uint2(code_word<HB, CB, MULT2, SAT>(P, G, 0, k), code_word<HB, CB, MULT2, SAT>(P, G, 1, k));
+                make_uint2(code_word<32 / ((HB >= 64) ? 1 : 64 / HB), CB, MULT2, SAT>(P, G, 0, k), code_word<32 / ((HB >= 64) ? 1 : 64 / HB), CB, MULT2, SAT>(P, G, 1, k));
         } else {
 #pragma unroll
             for (int w = 0; w < NW; w += 4)
                 *reinterpret_cast<uint4*>(dst + 4 * w) = make_uint4(
-                    code_word<HB, CB, MULT2, SAT>(P, G, w, k), code_word<HB, CB, MULT2, SAT>(P, G, w + 1, k),
-                    code_word<HB, CB, MULT2, SAT>(P, G, w + 2, k), code_word<HB, CB, MULT2, SAT>(P, G, w + 3, k));
+                    code_word<32 / ((HB >= 64) ? 1 : 64 / HB), CB, MULT2, SAT>(P, G, w, k), code_word<32 / ((HB >= 64) ? 1 : 64 / HB), CB, MULT2, SAT>(P, G, w + 1, k),
+                    code_word<32 / ((HB >= 64) ? 1 : 64 / HB), CB, MULT2, SAT>(P, G, w + 2, k), code_word<32 / ((HB >= 64) ? 1 : 64 / HB), CB, MULT2, SAT>(P, G, w + 3, k));
         }
     }
 
@@ -530,7 +426,7 @@ __device__ __forceinline__ void emit_half(const QuantArgs& A, const float2 (&P)[
     if (k.mask_mode >= 0) {
         uint32_t by[8];
 #pragma unroll
-        for (int b = 0; b < 8; ++b) by[b] = mask_byte<HB>(P, G, b, k);
+        for (int b = 0; b < 8; ++b) by[b] = mask_byte<32 / ((HB >= 64) ? 1 : 64 / HB)>(P, G, b, k);
         if (k.mask_mode == 0) {
             const uint32_t m0 = by[0] | (by[1] << 8) | (by[2] << 16) | (by[3] << 24);
             const uint32_t m1 = by[4] | (by[5] << 8) | (by[6] << 16) | (by[7] << 24);
@@ -788,6 +684,10 @@ bool tma_path_ok(const QuantArgs& a, quest_dtype x_dtype, int cbits, bool row_mo
 
 cudaError_t launch_quantize(const QuantArgs& a, quest_dtype x_dtype, int had_block, int cbits,
                             int bits, bool row_mode, cudaStream_t stream) {
+    if (tc_path_ok(a, x_dtype, had_block, cbits, row_mode))
+        return launch_quantize_tc(a, had_block, cbits, bits, row_mode, stream);
+    if (hs_path_ok(a, had_block, cbits, row_mode))
+        return launch_quantize_hs(a, x_dtype, had_block, cbits, bits, row_mode, stream);
     if (tma_path_ok(a, x_dtype, cbits, row_mode)) {
         if (x_dtype == QUEST_BF16) return tma::launch_tma<__nv_bfloat16>(a, bits, had_block, cbits, stream);
         return tma::launch_tma<float>(a, bits, had_block, cbits, stream);

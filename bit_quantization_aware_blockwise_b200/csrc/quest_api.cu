@@ -317,11 +317,27 @@ quest_status quest_quantize_fwd(const void* x, quest_dtype x_dtype, int64_t rows
     pack_constants(cb, code_mode, &c.pack_mult, &c.pack_add, &c.pack_xor);
     c.inv_levels = (float)ldexp(1.0, -bits);
     c.half_levels = (float)ldexp(1.0, bits - 1);
+    {
+        const double cd = alpha / ldexp(1.0, bits - 1), ic = 1.0 / ((double)had_block * (double)rms_group);
+        const double shb = sqrt((double)had_block);
+        const double edge = ldexp(1.0, bits - 1) + 0.5 * ((double)trust - 1.0);
+        c.delta_k = (float)(cd * sqrt(ic));
+        c.inv_k = (float)(1.0 / (shb * cd * sqrt(ic)));
+        c.a_k = (float)(ldexp(1.0, -bits) / (shb * cd * sqrt(ic)));
+        c.thr2_k = (float)(edge * edge * shb * shb * cd * cd * ic);
+    }
     c.sat_k = (float)(ldexp(1.0, bits) * (1.0 - ldexp(1.0, -23)));
     c.s_mid = kMagic + (float)ldexp(1.0, bits - 1);
     c.s_top = kMagic + (float)(ldexp(1.0, bits) - 1.0);
     c.cell_center = (float)(0.5 - ldexp(1.0, bits - 1));
     pack_constants_biased(cb, bits, code_mode, &c.pack2_mult, &c.pack2_add, &c.pack2_xor);
+    {   // an 8-field word (one chunk of 8 elements) for cb <= 4
+        const uint32_t rep8 = cb == 1 ? 0xFFu : (cb == 2 ? 0x5555u : 0x11111111u);
+        const uint32_t x8 = cb == 1 ? 0xFFu : (cb == 2 ? 0xAAAAu : 0x88888888u);
+        const uint32_t off = (1u << (cb - 1)) - (1u << (bits - 1));
+        c.pack8_add = (off - kMagicBits) * rep8;
+        c.pack8_xor = x8;
+    }
     c.trust_ge1 = trust >= 1.0f;
     c.mask_mode = mask ? (int)mask_mode : -1;
     c.deq_mode = dequant ? (int)dequant_dtype : -1;

@@ -215,3 +215,60 @@ __device__ __forceinline__ void fwht_halfslab(float2 (&P)[32], int lane) {
 }
 
 }  // namespace quest
+
+// ---------------------------------------------------------------------------
+// Interleaved half-slab layout (direct-load kernels). Lane h (= lane & 1) of a
+// pair holds chunks 2k + h, k = 0..7, of a 128-element slab (8 elements per
+// chunk), so the two lanes' 16-byte loads of chunk slot k cover one 32-byte
+// sector. Pair P[4k + p] = (element 2p, element 2p + 1) of chunk 2k + h.
+// Element index bits inside a block:
+//   bit 0            inside a pair                  (scalar add/sub)
+//   bits 1, 2        pair bits 0, 1                 (packed butterflies)
+//   bit 3            lane ^ 1                       (shuffle)
+//   bits 4, 5, 6     pair bits 2, 3, 4              (packed, for HB >= 32/64/128)
+//   bit 7            lane ^ 2 (the next slab)       (shuffle, HB == 256)
+// A lane holds the pairs of block b in [b*PPB, (b+1)*PPB), PPB = min(HB, 128)/4.
+// ---------------------------------------------------------------------------
+namespace quest {
+
+template <int HB>
+__device__ __forceinline__ void fwht_interleaved(float2 (&P)[32], int lane) {
+    static_assert(HB >= 16 && HB <= 256 && (HB & (HB - 1)) == 0, "HB");
+#pragma unroll
+    for (int j = 0; j < 32; ++j) {
+        const float a = P[j].x, b = P[j].y;
+        P[j] = make_float2(a + b, a - b);
+    }
+    // pair-index bit t is element bit t+1 (t < 2) or t+2 (t >= 2)
+#pragma unroll
+    for (int t = 0; t < 5; ++t) {
+        const int elem_bit = t < 2 ? t + 1 : t + 2;
+        if ((1 << elem_bit) < HB) {
+            const int h = 1 << t;
+#pragma unroll
+            for (int j = 0; j < 32; ++j) {
+                if ((j & h) == 0) {
+                    const float2 a = P[j], b = P[j + h];
+                    P[j] = __fadd2_rn(a, b);
+                    P[j + h] = f2_sub(a, b);
+                }
+            }
+        }
+    }
+#pragma unroll
+    for (int s = 1; s <= 2; s <<= 1) {
+        if ((s == 1 && HB >= 16) || (s == 2 && HB >= 256)) {
+            const float sg = (lane & s) ? -1.0f : 1.0f;
+            const float2 sg2 = make_float2(sg, sg);
+#pragma unroll
+            for (int j = 0; j < 32; ++j) {
+                float2 o;
+                o.x = __shfl_xor_sync(0xFFFFFFFFu, P[j].x, s);
+                o.y = __shfl_xor_sync(0xFFFFFFFFu, P[j].y, s);
+                P[j] = __ffma2_rn(P[j], sg2, o);
+            }
+        }
+    }
+}
+
+}  // namespace quest

@@ -1,0 +1,160 @@
+// Per-element decision path shared by the half-slab quantizer kernels.
+//
+// Codes are produced biased, s = 1.5*2^23 + q_b with q_b = q + 2^(b-1) in
+// [0, 2^b - 1], so that one integer multiply-add per element packs them (see
+// the packing constants in quest_api.cu).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "quest_device.cuh"
+#include "quest_internal.h"
+
+namespace quest {
+
+// Per-group constants of the decision path.
+struct GroupK {
+    float delta;   // Delta
+    float a, c;    // u = sat(y_u * a + c)      (saturating path)
+    float inv;     // t = y_u * inv             (exact path, general mask)
+    float thr2;    // (edge * sqrt(HB) * Delta)^2
+    float ch;      // yhat = q_b * Delta + ch
+};
+
+// From the sum of squares ss of a group's unnormalised transformed values:
+// r = sqrt(ss / count), Delta = c_delta r, t = y / Delta. One approximate
+// reciprocal square root (relative error a few 1e-7) serves all of them; a
+// decision that this moves lies within 1e-6 relative of a cell boundary.
+__device__ __forceinline__ GroupK make_group(const QuantConsts& k, float ss) {
+    GroupK g;
+    if (ss > 0.0f) {
+        const float rs = rsqrtf(ss);
+        g.delta = ss * rs * k.delta_k;
+        g.inv = rs * k.inv_k;
+        g.a = rs * k.a_k;
+        g.c = 0.5f;
+        g.thr2 = ss * k.thr2_k;
+    } else {
+        g.delta = 0.0f;
+        g.inv = 0.0f;
+        g.a = 0.0f;
+        g.c = 0.5f + 0.5f * k.inv_levels;   // lands in the cell of q = 0
+        g.thr2 = __int_as_float(0x7F800000);
+    }
+    g.ch = (0.5f - k.half_levels) * g.delta;
+    return g;
+}
+
+// Biased code s = kMagic + q_b of a pair of transformed values.
+template <bool SAT>
+__device__ __forceinline__ float2 decide(float2 y, const GroupK& g, const QuantConsts& k) {
+    if constexpr (SAT) {
+        const float2 u = make_float2(__saturatef(__fmaf_rn(y.x, g.a, g.c)),
+                                     __saturatef(__fmaf_rn(y.y, g.a, g.c)));
+        return __ffma2_rd(u, make_float2(k.sat_k, k.sat_k), make_float2(kMagic, kMagic));
+    } else {
+        const float2 t = __ffma2_rd(y, make_float2(g.inv, g.inv), make_float2(k.s_mid, k.s_mid));
+        return make_float2(fminf(fmaxf(t.x, kMagic), k.s_top), fminf(fmaxf(t.y, kMagic), k.s_top));
+    }
+}
+
+// Packed code word of the EPW = 32/CB elements in pairs [w*EPW/2, (w+1)*EPW/2)
+// (PPB = pairs per RMS group). The sum is split over independent partial sums of
+// 8 fields so the dependency chains stay short.
+template <int PPB, int CB, bool MULT2, bool SAT>
+__device__ __forceinline__ uint32_t code_word(const float2 (&P)[32], const GroupK* G, int w,
+                                              const QuantConsts& k) {
+    constexpr uint32_t kMult = MULT2 ? 2u : 1u;
+    constexpr int EPW = 32 / CB;
+    constexpr int NSUB = EPW >= 8 ? EPW / 8 : 1;
+    constexpr int PER = EPW / NSUB;
+    uint32_t part[NSUB];
+#pragma unroll
+    for (int u = 0; u < NSUB; ++u) {
+        uint32_t acc = 0;
+#pragma unroll
+        for (int i = u * PER; i < (u + 1) * PER; i += 2) {
+            const int j = (w * EPW + i) / 2;
+            const float2 s2 = decide<SAT>(P[j], G[j / PPB], k);
+            acc += __float_as_uint(s2.x) * (kMult << (CB * i));
+            acc += __float_as_uint(s2.y) * (kMult << (CB * (i + 1)));
+        }
+        part[u] = acc;
+    }
+    uint32_t word = k.pack2_add;
+#pragma unroll
+    for (int u = 0; u < NSUB; ++u) word += part[u];
+    return word ^ k.pack2_xor;
+}
+
+// Trust-mask byte of the 8 elements in pairs [4*byte, 4*byte + 4): bit i = element i.
+template <int PPB, int N>
+__device__ __forceinline__ uint32_t mask_byte(const float2 (&P)[N], const GroupK* G, int byte,
+                                              const QuantConsts& k) {
+    uint32_t acc = 0;
+    if (k.trust_ge1) {
+#pragma unroll
+        for (int j = 4 * byte + 3; j >= 4 * byte; --j) {
+            const float t2 = G[j / PPB].thr2;
+            const float2 d = __ffma2_rn(P[j], P[j], make_float2(-t2, -t2));
+            acc = __funnelshift_l(__float_as_uint(d.y), acc, 1);
+            acc = __funnelshift_l(__float_as_uint(d.x), acc, 1);
+        }
+    } else {
+#pragma unroll
+        for (int j = 4 * byte + 3; j >= 4 * byte; --j) {
+            const GroupK& g = G[j / PPB];
+            // q + 1/2 = q_b + cell_center, q_b from the exact floor of t
+            const float2 t = __fmul2_rn(P[j], make_float2(g.inv, g.inv));
+            float2 sf = __ffma2_rd(P[j], make_float2(g.inv, g.inv), make_float2(k.s_mid, k.s_mid));
+            sf = make_float2(fminf(fmaxf(sf.x, kMagic), k.s_top), fminf(fmaxf(sf.y, kMagic), k.s_top));
+            const float ex = fabsf(t.x - ((sf.x - kMagic) + k.cell_center)) - k.half_trust;
+            const float ey = fabsf(t.y - ((sf.y - kMagic) + k.cell_center)) - k.half_trust;
+            const bool zero_group = !(g.delta > 0.0f);
+            acc = __funnelshift_l(__float_as_uint(zero_group ? -1.0f : ey), acc, 1);
+            acc = __funnelshift_l(__float_as_uint(zero_group ? -1.0f : ex), acc, 1);
+        }
+    }
+    return acc;
+}
+
+
+// Biased codes of the 8 elements of one chunk (pairs 4c .. 4c+3 of a lane).
+template <bool SAT, int PPB, int N>
+__device__ __forceinline__ void chunk_decide(const float2 (&P)[N], const GroupK* G, int c,
+                                             const QuantConsts& k, float2 (&s)[4]) {
+#pragma unroll
+    for (int p = 0; p < 4; ++p) s[p] = decide<SAT>(P[4 * c + p], G[(4 * c + p) / PPB], k);
+}
+
+// The 8 codes of a chunk in the low 8*CB bits (CB <= 4), with the constants of
+// an 8-field word (pack8_add / pack8_xor).
+template <int CB>
+__device__ __forceinline__ uint32_t chunk_pack(const float2 (&s)[4], const QuantConsts& k) {
+    static_assert(CB <= 4, "8-bit codes take chunk_pack_i8");
+    uint32_t acc = 0;
+#pragma unroll
+    for (int p = 0; p < 4; ++p) {
+        acc += __float_as_uint(s[p].x) << (CB * 2 * p);
+        acc += __float_as_uint(s[p].y) << (CB * (2 * p + 1));
+    }
+    return ((acc + k.pack8_add) ^ k.pack8_xor) & (CB == 4 ? 0xFFFFFFFFu : ((1u << (8 * CB)) - 1u));
+}
+
+// The 8 one-byte codes of a chunk as two 32-bit words (pack2_* constants).
+template <bool MULT2>
+__device__ __forceinline__ uint2 chunk_pack_i8(const float2 (&s)[4], const QuantConsts& k) {
+    constexpr uint32_t m = MULT2 ? 2u : 1u;
+    uint32_t w[2];
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+        const uint32_t acc = __float_as_uint(s[2 * u].x) * m + __float_as_uint(s[2 * u].y) * (m << 8) +
+                             __float_as_uint(s[2 * u + 1].x) * (m << 16) +
+                             __float_as_uint(s[2 * u + 1].y) * (m << 24);
+        w[u] = (acc + k.pack2_add) ^ k.pack2_xor;
+    }
+    return make_uint2(w[0], w[1]);
+}
+
+}  // namespace quest

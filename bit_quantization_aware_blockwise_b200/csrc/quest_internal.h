@@ -22,12 +22,18 @@ struct QuantConsts {
     uint32_t pack_xor;  // un-biasing mask of the packed word
     // half-slab (TMA-staged) decision path, codes biased as q_b = q + 2^(b-1)
     float inv_levels;   // 2^-b
+    // Per-group constants from rs = rsqrt(sum of y_u^2) (one MUFU op per group):
+    float delta_k;      // Delta = ss * rs * delta_k          (c_delta * sqrt(inv_count))
+    float inv_k;        // 1 / (sqrt(HB) Delta) = rs * inv_k
+    float a_k;          // inv * 2^-b = rs * a_k
+    float thr2_k;       // (edge sqrt(HB) Delta)^2 = ss * thr2_k
     float half_levels;  // 2^(b-1)
     float sat_k;        // 2^b (1 - 2^-23)
     float s_mid;        // kMagic + 2^(b-1)
     float s_top;        // kMagic + 2^b - 1
     float cell_center;  // 1/2 - 2^(b-1): q + 1/2 = q_b + cell_center
-    uint32_t pack2_mult, pack2_add, pack2_xor;
+    uint32_t pack2_mult, pack2_add, pack2_xor;   // 32-bit words of 32/cb fields
+    uint32_t pack8_add, pack8_xor;                // words of 8 fields (cb <= 4)
     int trust_ge1;      // 1: use m = [|t| <= edge]
     int mask_mode;      // -1 none, 0 bits, 1 bytes
     int deq_mode;       // -1 none, 0 bf16, 1 fp32
@@ -61,6 +67,14 @@ struct TrustArgs {
 cudaError_t launch_quantize(const QuantArgs& a, quest_dtype x_dtype, int had_block, int cbits,
                             int bits, bool row_mode, cudaStream_t stream);
 int read_and_clear_quant_status(cudaStream_t stream, cudaError_t* err);
+// Direct-load interleaved half-slab quantizer (quantize_hs.cu).
+bool hs_path_ok(const QuantArgs& a, int had_block, int cbits, bool row_mode);
+cudaError_t launch_quantize_hs(const QuantArgs& a, quest_dtype x_dtype, int had_block, int cbits,
+                               int bits, bool row_mode, cudaStream_t stream);
+// bf16 quantizer with the 16-point Hadamard factor on tensor cores (quantize_tc.cu).
+bool tc_path_ok(const QuantArgs& a, quest_dtype x_dtype, int had_block, int cbits, bool row_mode);
+cudaError_t launch_quantize_tc(const QuantArgs& a, int had_block, int cbits, int bits, bool row_mode,
+                               cudaStream_t stream);
 cudaError_t launch_trust_bwd(const TrustArgs& a, int had_block, cudaStream_t stream);
 cudaError_t launch_w4a4(const int8_t* A, const float* sa, const int8_t* B, const float* sb,
                         int64_t M, int64_t N, int64_t K, uint16_t* y, int32_t* acc,
