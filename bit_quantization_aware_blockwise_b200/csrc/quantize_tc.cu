@@ -7,20 +7,8 @@
 //
 // Why. On B200 the CUDA-core quantizer is bound by instruction issue, not by
 // HBM: its butterflies, bf16 unpacking and cross-lane shuffles are about a third
-// of ~14.5 instructions per element. The Sylvester matrix factors over the bits
-// of the element index, H_128 = H_2 (x) ... (x) H_2, so any four of the seven
-// bits can be transformed at once by a 16 x 16 matrix product. Here each lane's
-// 16-byte load of 8 bf16 values is, unchanged, its part of the A operand of an
-// m16n8k16 bf16 MMA (fp32 accumulation, exact products of inputs with +-1), the
-// result lands on the same lane in the same element order, and only the three
-// remaining index bits are butterflies in registers.
-//
-// Layout. A warp step covers 8 slabs of 128 values. Lane = 4 g + t: slab g,
-// chunks c = t + 4 f (f = 0..3) of 8 values each. With element index bits
-// b0..b6 within the slab: b0 = position in a 32-bit word, (b1, b2) = word of the
-// chunk, (b3, b4) = t, (b5, b6) = f. MMA f transforms bits (b0, b3, b4, b1) as
-// its k bits; b2 is the row half of the fragment; b2, b5, b6 (and the slab bit
-// for 256-blocks) are done in registers / by one shuffle.
+// of ~14.5 instructions per element. Here four of the seven index bits go through
+// a 16 x 16 tensor-core product (quest_tc.cuh, which also gives the data layout).
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
@@ -28,121 +16,10 @@
 #include "quest_device.cuh"
 #include "quest_emit.cuh"
 #include "quest_internal.h"
+#include "quest_tc.cuh"
 
 namespace quest {
 namespace tc {
-
-constexpr int kThreads = 128;
-
-__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
-    uint32_t d;
-    asm("prmt.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(sel));
-    return d;
-}
-
-// 16 x 16 transform matrix on the MMA's k / n bits: entry (k, n) is the product
-// over the 4 bits of H_2 (bit in `tmask`) or I_2 (bit not in the block).
-__device__ __forceinline__ float mat_entry(int k, int n, int tmask) {
-    int neg = 0;
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        const int ki = (k >> i) & 1, ni = (n >> i) & 1;
-        if ((tmask >> i) & 1) neg ^= ki & ni;
-        else if (ki != ni) return 0.0f;
-    }
-    return neg ? -1.0f : 1.0f;
-}
-
-__device__ __forceinline__ uint32_t bf16x2_bits(float lo, float hi) {
-    const uint32_t l = __bfloat16_as_ushort(__float2bfloat16_rn(lo));
-    const uint32_t h = __bfloat16_as_ushort(__float2bfloat16_rn(hi));
-    return l | (h << 16);
-}
-
-// B fragments (k = 2t, 2t+1 and 2t+8, 2t+9; n = g + 8 tile) of the transform matrix.
-struct BFrag {
-    uint32_t b[2][2];   // [n tile][register]
-};
-
-__device__ __forceinline__ BFrag make_bfrag(int lane, int tmask) {
-    const int g = lane >> 2, t = lane & 3;
-    BFrag f;
-#pragma unroll
-    for (int tile = 0; tile < 2; ++tile) {
-        const int n = g + 8 * tile;
-        f.b[tile][0] = bf16x2_bits(mat_entry(2 * t, n, tmask), mat_entry(2 * t + 1, n, tmask));
-        f.b[tile][1] = bf16x2_bits(mat_entry(2 * t + 8, n, tmask), mat_entry(2 * t + 9, n, tmask));
-    }
-    return f;
-}
-
-__device__ __forceinline__ void mma16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
-                                         uint32_t b0, uint32_t b1) {
-    asm("mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
-        "{%10,%10,%10,%10};"
-        : "=f"(d[0]), "=f"(d[1]), "=f"(d[2]), "=f"(d[3])
-        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1), "f"(0.0f));
-}
-
-// The 4 chunks (16 bytes each) this lane loads from a slab at `src`.
-__device__ __forceinline__ void load_slab(const char* src, int t, uint4 (&r)[4]) {
-#pragma unroll
-    for (int f = 0; f < 4; ++f) r[f] = ld_stream_v4(src + (t + 4 * f) * 16);
-}
-
-__device__ __forceinline__ void zero4(uint4 (&r)[4]) {
-#pragma unroll
-    for (int f = 0; f < 4; ++f) r[f] = make_uint4(0u, 0u, 0u, 0u);
-}
-
-// Transform bits (b0, b1, b3, b4) by MMA: P[4f + w] = values 2w, 2w+1 of chunk f.
-__device__ __forceinline__ void mma_stage(const uint4 (&r)[4], const BFrag& B, float2 (&P)[16]) {
-#pragma unroll
-    for (int f = 0; f < 4; ++f) {
-        // A registers: (row g, k3 = 0) = word 0, (row g+8, k3 = 0) = word 2,
-        //              (row g, k3 = 1) = word 1, (row g+8, k3 = 1) = word 3
-        float d0[4], d1[4];
-        mma16816(d0, r[f].x, r[f].z, r[f].y, r[f].w, B.b[0][0], B.b[0][1]);
-        mma16816(d1, r[f].x, r[f].z, r[f].y, r[f].w, B.b[1][0], B.b[1][1]);
-        P[4 * f + 0] = make_float2(d0[0], d0[1]);   // word 0: b1 = 0, b2 = 0
-        P[4 * f + 1] = make_float2(d1[0], d1[1]);   // word 1: b1 = 1, b2 = 0
-        P[4 * f + 2] = make_float2(d0[2], d0[3]);   // word 2: b1 = 0, b2 = 1
-        P[4 * f + 3] = make_float2(d1[2], d1[3]);   // word 3: b1 = 1, b2 = 1
-    }
-}
-
-__device__ __forceinline__ void bfly(float2& a, float2& b) {
-    const float2 s = __fadd2_rn(a, b);
-    b = f2_sub(a, b);
-    a = s;
-}
-
-// Remaining in-register bits: b2 (index stride 2), b5 (stride 4), b6 (stride 8);
-// for 256-blocks also the slab bit (lane ^ 4).
-template <int HB>
-__device__ __forceinline__ void reg_stages(float2 (&P)[16], int lane) {
-#pragma unroll
-    for (int j = 0; j < 16; ++j)
-        if ((j & 2) == 0) bfly(P[j], P[j + 2]);
-    if constexpr (HB >= 64) {
-#pragma unroll
-        for (int j = 0; j < 16; ++j)
-            if ((j & 4) == 0) bfly(P[j], P[j + 4]);
-    }
-    if constexpr (HB >= 128) {
-#pragma unroll
-        for (int j = 0; j < 8; ++j) bfly(P[j], P[j + 8]);
-    }
-    if constexpr (HB == 256) {
-        const float sgn = (lane & 4) ? -1.0f : 1.0f;   // odd slab of the pair takes a - b
-#pragma unroll
-        for (int j = 0; j < 16; ++j) {
-            const float2 o = make_float2(__shfl_xor_sync(0xFFFFFFFFu, P[j].x, 4),
-                                         __shfl_xor_sync(0xFFFFFFFFu, P[j].y, 4));
-            P[j] = __ffma2_rn(P[j], make_float2(sgn, sgn), o);
-        }
-    }
-}
 
 // Blocks per lane and pairs of one block in a lane.
 template <int HB>
@@ -165,15 +42,6 @@ __device__ __forceinline__ void lane_sums(const float2 (&P)[16], float (&ss)[Blk
         const float2 a = __fadd2_rn(acc0, acc1);
         ss[b] = a.x + a.y;
     }
-}
-
-// Byte transpose across a lane quad: lane t holds byte f = value of chunk t + 4f;
-// returns the word of chunks 4t .. 4t+3 (byte j = chunk 4t + j).
-__device__ __forceinline__ uint32_t quad_transpose_bytes(uint32_t x, int t) {
-    const uint32_t p1 = __shfl_xor_sync(0xFFFFFFFFu, x, 1);
-    const uint32_t z = prmt(x, p1, (t & 1) ? 0x3715u : 0x6240u);
-    const uint32_t p2 = __shfl_xor_sync(0xFFFFFFFFu, z, 2);
-    return prmt(z, p2, (t & 2) ? 0x3276u : 0x5410u);
 }
 
 // Quantise and store this lane's 32 values: chunks c = t + 4f of the slab whose
@@ -199,7 +67,6 @@ __device__ __forceinline__ void emit(const QuantArgs& A, const float2 (&P)[16], 
         } else {
             cbytes |= chunk_pack<1>(s, k) << (8 * f);
         }
-        if (do_mask) mbytes |= mask_byte<PPB>(P, G, f, k) << (8 * f);
         if (do_deq) {
             // yhat = q_b Delta + (1/2 - 2^(b-1)) Delta
             float2 y[4];
@@ -221,6 +88,17 @@ __device__ __forceinline__ void emit(const QuantArgs& A, const float2 (&P)[16], 
                 *reinterpret_cast<uint4*>(dst + 16) = make_uint4(__float_as_uint(y[2].x), __float_as_uint(y[2].y),
                                                                  __float_as_uint(y[3].x), __float_as_uint(y[3].y));
             }
+        }
+    }
+    // trust mask bytes: one loop per form of the test, so that neither is predicated
+    // into the other's path
+    if (do_mask) {
+        if (k.trust_ge1) {
+#pragma unroll
+            for (int f = 0; f < 4; ++f) mbytes |= mask_byte_edge<PPB>(P, G, f) << (8 * f);
+        } else {
+#pragma unroll
+            for (int f = 0; f < 4; ++f) mbytes |= mask_byte_cell<PPB>(P, G, f, k) << (8 * f);
         }
     }
     if constexpr (CB == 1) {
@@ -245,12 +123,51 @@ __device__ __forceinline__ void emit(const QuantArgs& A, const float2 (&P)[16], 
     }
 }
 
-template <int HB>
-constexpr int tmask_of() { return HB == 16 ? 0xB : 0xF; }   // HB = 16 leaves b4 alone
+
+// Everything after the MMA for one slab of the group-RMS kernel.
+template <int HB, int CB, bool MULT2, bool SAT>
+__device__ __forceinline__ void group_slab(const QuantArgs& A, float2 (&P)[16], int64_t slab, bool valid,
+                                           int lane) {
+    constexpr int NBL = Blk<HB>::NBL, PPB = Blk<HB>::PPB;
+    const int g = lane >> 2, t = lane & 3;
+    reg_stages<HB>(P, lane);
+    float ss[NBL];
+    lane_sums<HB>(P, ss);
+    GroupK G[NBL];
+#pragma unroll
+    for (int b = 0; b < NBL; ++b) {
+        float v = ss[b] + __shfl_xor_sync(0xFFFFFFFFu, ss[b], 1);
+        if constexpr (HB >= 32) v += __shfl_xor_sync(0xFFFFFFFFu, v, 2);
+        if constexpr (HB == 256) v += __shfl_xor_sync(0xFFFFFFFFu, v, 4);
+        G[b] = make_group(A.c, v);
+    }
+    const int64_t E = slab * 128;   // dense outputs: row 0 with a flat offset
+    emit<PPB, CB, MULT2, SAT>(A, P, G, 0, E, t, valid);
+    if (valid) {
+        float* sp = A.scales + E / HB;
+        if constexpr (HB == 256) {
+            if ((g & 1) == 0 && t == 0) sp[0] = G[0].delta;
+        } else if constexpr (HB == 128) {
+            if (t == 0) sp[0] = G[0].delta;
+        } else if constexpr (HB == 64) {
+            if (t < 2) sp[t] = t ? G[1].delta : G[0].delta;   // block = b6
+        } else if constexpr (HB == 32) {
+            sp[t] = t == 0 ? G[0].delta : t == 1 ? G[1].delta : t == 2 ? G[2].delta : G[3].delta;   // block = f
+        } else {
+            // 16-blocks: index b4 + 2 (b5 + 2 b6) = (t >> 1) + 2 f; lanes t and t ^ 1 agree
+            const int t1 = t >> 1, lo = (t & 1) ? 2 : 0;
+            sp[t1 + 2 * lo] = (t & 1) ? G[2].delta : G[0].delta;
+            sp[t1 + 2 * (lo + 1)] = (t & 1) ? G[3].delta : G[1].delta;
+        }
+    }
+}
+
+// Loads run kDepth warp steps ahead of the arithmetic (on B200 a second step in
+// flight costs more in registers, and so in resident warps, than it hides).
+constexpr int kDepth = 1;
 
 template <int HB, int CB, bool MULT2, bool SAT>
 __global__ void __launch_bounds__(kThreads) quantize_tc_groups(const QuantArgs A) {
-    constexpr int NBL = Blk<HB>::NBL, PPB = Blk<HB>::PPB;
     const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
     const int64_t spr = A.cols / 128;
     const int64_t total = A.rows * spr;
@@ -263,45 +180,25 @@ __global__ void __launch_bounds__(kThreads) quantize_tc_groups(const QuantArgs A
         return A.x + row * A.ld_x_bytes + sc * 256;
     };
 
-    uint4 raw[4];
-    if (warp0 * 8 + g < total) load_slab(src_of(warp0 * 8 + g), t, raw);
-    else zero4(raw);
-    for (int64_t s0 = warp0 * 8; s0 < total; s0 += step) {
-        const int64_t slab = s0 + g;
-        const bool valid = slab < total;
-        float2 P[16];
-        mma_stage(raw, B, P);
-        if (slab + step < total) load_slab(src_of(slab + step), t, raw);
-        else zero4(raw);
-        reg_stages<HB>(P, lane);
-        float ss[NBL];
-        lane_sums<HB>(P, ss);
-        GroupK G[NBL];
+    uint4 raw[kDepth][4];
 #pragma unroll
-        for (int b = 0; b < NBL; ++b) {
-            float v = ss[b] + __shfl_xor_sync(0xFFFFFFFFu, ss[b], 1);
-            if constexpr (HB >= 32) v += __shfl_xor_sync(0xFFFFFFFFu, v, 2);
-            if constexpr (HB == 256) v += __shfl_xor_sync(0xFFFFFFFFu, v, 4);
-            G[b] = make_group(A.c, v);
-        }
-        const int64_t E = slab * 128;   // dense outputs: row 0 with a flat offset
-        emit<PPB, CB, MULT2, SAT>(A, P, G, 0, E, t, valid);
-        if (valid) {
-            float* sp = A.scales + E / HB;
-            if constexpr (HB == 256) {
-                if ((g & 1) == 0 && t == 0) sp[0] = G[0].delta;
-            } else if constexpr (HB == 128) {
-                if (t == 0) sp[0] = G[0].delta;
-            } else if constexpr (HB == 64) {
-                if (t < 2) sp[t] = t ? G[1].delta : G[0].delta;   // block = b6
-            } else if constexpr (HB == 32) {
-                sp[t] = t == 0 ? G[0].delta : t == 1 ? G[1].delta : t == 2 ? G[2].delta : G[3].delta;   // block = f
-            } else {
-                // 16-blocks: index b4 + 2 (b5 + 2 b6) = (t >> 1) + 2 f; lanes t and t ^ 1 agree
-                const int t1 = t >> 1, lo = (t & 1) ? 2 : 0;
-                sp[t1 + 2 * lo] = (t & 1) ? G[2].delta : G[0].delta;
-                sp[t1 + 2 * (lo + 1)] = (t & 1) ? G[3].delta : G[1].delta;
-            }
+    for (int d = 0; d < kDepth; ++d) {
+        const int64_t slab = warp0 * 8 + g + d * step;
+        if (slab < total) load_slab(src_of(slab), t, raw[d]);
+        else zero4(raw[d]);
+    }
+    for (int64_t s0 = warp0 * 8; s0 < total; s0 += kDepth * step) {
+#pragma unroll
+        for (int d = 0; d < kDepth; ++d) {
+            const int64_t base = s0 + d * step;
+            if (base >= total) break;   // warp-uniform
+            const int64_t slab = base + g;
+            float2 P[16];
+            mma_stage(raw[d], B, P);
+            const int64_t next = slab + kDepth * step;
+            if (next < total) load_slab(src_of(next), t, raw[d]);
+            else zero4(raw[d]);
+            group_slab<HB, CB, MULT2, SAT>(A, P, slab, slab < total, lane);
         }
     }
 }
@@ -309,7 +206,7 @@ __global__ void __launch_bounds__(kThreads) quantize_tc_groups(const QuantArgs A
 // One RMS over each row of spr slabs. SUB = slabs per lane group (spr / 8 when
 // spr >= 8, so a warp holds a whole row); for spr < 8 a warp step covers 8 / spr rows.
 template <int HB, int CB, bool MULT2, bool SAT, int SUB>
-__global__ void __launch_bounds__(kThreads) quantize_tc_rows(const QuantArgs A, int spr) {
+__global__ void __launch_bounds__(kThreads, 4) quantize_tc_rows(const QuantArgs A, int spr) {
     constexpr int NBL = Blk<HB>::NBL, PPB = Blk<HB>::PPB;
     const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
     const int rps = SUB > 1 ? 1 : 8 / spr;          // rows per warp step

@@ -89,36 +89,46 @@ __device__ __forceinline__ uint32_t code_word(const float2 (&P)[32], const Group
 }
 
 // Trust-mask byte of the 8 elements in pairs [4*byte, 4*byte + 4): bit i = element i.
+// For T >= 1: m = [y^2 <= thr^2], read off the sign of y^2 - thr^2.
 template <int PPB, int N>
-__device__ __forceinline__ uint32_t mask_byte(const float2 (&P)[N], const GroupK* G, int byte,
-                                              const QuantConsts& k) {
+__device__ __forceinline__ uint32_t mask_byte_edge(const float2 (&P)[N], const GroupK* G, int byte) {
     uint32_t acc = 0;
-    if (k.trust_ge1) {
 #pragma unroll
-        for (int j = 4 * byte + 3; j >= 4 * byte; --j) {
-            const float t2 = G[j / PPB].thr2;
-            const float2 d = __ffma2_rn(P[j], P[j], make_float2(-t2, -t2));
-            acc = __funnelshift_l(__float_as_uint(d.y), acc, 1);
-            acc = __funnelshift_l(__float_as_uint(d.x), acc, 1);
-        }
-    } else {
-#pragma unroll
-        for (int j = 4 * byte + 3; j >= 4 * byte; --j) {
-            const GroupK& g = G[j / PPB];
-            // q + 1/2 = q_b + cell_center, q_b from the exact floor of t
-            const float2 t = __fmul2_rn(P[j], make_float2(g.inv, g.inv));
-            float2 sf = __ffma2_rd(P[j], make_float2(g.inv, g.inv), make_float2(k.s_mid, k.s_mid));
-            sf = make_float2(fminf(fmaxf(sf.x, kMagic), k.s_top), fminf(fmaxf(sf.y, kMagic), k.s_top));
-            const float ex = fabsf(t.x - ((sf.x - kMagic) + k.cell_center)) - k.half_trust;
-            const float ey = fabsf(t.y - ((sf.y - kMagic) + k.cell_center)) - k.half_trust;
-            const bool zero_group = !(g.delta > 0.0f);
-            acc = __funnelshift_l(__float_as_uint(zero_group ? -1.0f : ey), acc, 1);
-            acc = __funnelshift_l(__float_as_uint(zero_group ? -1.0f : ex), acc, 1);
-        }
+    for (int j = 4 * byte + 3; j >= 4 * byte; --j) {
+        const float t2 = G[j / PPB].thr2;
+        const float2 d = __ffma2_rn(P[j], P[j], make_float2(-t2, -t2));
+        acc = __funnelshift_l(__float_as_uint(d.y), acc, 1);
+        acc = __funnelshift_l(__float_as_uint(d.x), acc, 1);
     }
     return acc;
 }
 
+// General T: m = [|t - (q + 1/2)| <= T/2] with q from the exact floor of t.
+template <int PPB, int N>
+__device__ __forceinline__ uint32_t mask_byte_cell(const float2 (&P)[N], const GroupK* G, int byte,
+                                                   const QuantConsts& k) {
+    uint32_t acc = 0;
+#pragma unroll
+    for (int j = 4 * byte + 3; j >= 4 * byte; --j) {
+        const GroupK& g = G[j / PPB];
+        // q + 1/2 = q_b + cell_center, q_b from the exact floor of t
+        const float2 t = __fmul2_rn(P[j], make_float2(g.inv, g.inv));
+        float2 sf = __ffma2_rd(P[j], make_float2(g.inv, g.inv), make_float2(k.s_mid, k.s_mid));
+        sf = make_float2(fminf(fmaxf(sf.x, kMagic), k.s_top), fminf(fmaxf(sf.y, kMagic), k.s_top));
+        const float ex = fabsf(t.x - ((sf.x - kMagic) + k.cell_center)) - k.half_trust;
+        const float ey = fabsf(t.y - ((sf.y - kMagic) + k.cell_center)) - k.half_trust;
+        const bool zero_group = !(g.delta > 0.0f);
+        acc = __funnelshift_l(__float_as_uint(zero_group ? -1.0f : ey), acc, 1);
+        acc = __funnelshift_l(__float_as_uint(zero_group ? -1.0f : ex), acc, 1);
+    }
+    return acc;
+}
+
+template <int PPB, int N>
+__device__ __forceinline__ uint32_t mask_byte(const float2 (&P)[N], const GroupK* G, int byte,
+                                              const QuantConsts& k) {
+    return k.trust_ge1 ? mask_byte_edge<PPB>(P, G, byte) : mask_byte_cell<PPB>(P, G, byte, k);
+}
 
 // Biased codes of the 8 elements of one chunk (pairs 4c .. 4c+3 of a lane).
 template <bool SAT, int PPB, int N>

@@ -76,6 +76,9 @@ bool tc_path_ok(const QuantArgs& a, quest_dtype x_dtype, int had_block, int cbit
 cudaError_t launch_quantize_tc(const QuantArgs& a, int had_block, int cbits, int bits, bool row_mode,
                                cudaStream_t stream);
 cudaError_t launch_trust_bwd(const TrustArgs& a, int had_block, cudaStream_t stream);
+// Trust backward with the tensor-core Hadamard factor (trust_tc.cu).
+bool trust_tc_ok(const TrustArgs& a, int had_block);
+cudaError_t launch_trust_tc(const TrustArgs& a, int had_block, cudaStream_t stream);
 cudaError_t launch_w4a4(const int8_t* A, const float* sa, const int8_t* B, const float* sb,
                         int64_t M, int64_t N, int64_t K, uint16_t* y, int32_t* acc,
                         cudaStream_t stream);

@@ -100,10 +100,10 @@ cudaError_t launch_hb(const TrustArgs& a, cudaStream_t stream) {
 
 }  // namespace
 
-// Direct loads only: on B200 this kernel streams the 16384 x 2048 gradient at
-// 4.8 TB/s, where a TMA-staged variant reached 3.6 TB/s (staged streaming tops
-// out near 4.7 TB/s on this part even with no arithmetic).
+// Rows of whole 128-value slabs take the tensor-core kernel (trust_tc.cu); this
+// CUDA-core kernel covers the rest (any cols that are a multiple of the block).
 cudaError_t launch_trust_bwd(const TrustArgs& a, int had_block, cudaStream_t stream) {
+    if (trust_tc_ok(a, had_block)) return launch_trust_tc(a, had_block, stream);
     switch (had_block) {
         case 16: return launch_hb<16>(a, stream);
         case 32: return launch_hb<32>(a, stream);
