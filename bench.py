@@ -457,7 +457,9 @@ def oracle_sample(rows_x=256, rows_w=88, gemm_rows=16):
 def cpu_baseline(args):
     import oracle
     oracle.build()
-    dt, nbytes, sample = oracle_sample()
+    # the full activation, gradient and weight legs and a 512-row block of the GEMM:
+    # about 10-20 s of single-threaded CPU work
+    dt, nbytes, sample = oracle_sample(rows_x=R, rows_w=NW, gemm_rows=512)
     return {"value": round(nbytes / dt / 1e9, 5), "unit": "GB/s", "cores": 1, "kind": "oracle",
             "sample": sample, "seconds": round(dt, 3)}
 
