@@ -61,6 +61,7 @@ def part_bytes():
 
 
 GEMM_OPS = 2 * R * NW * C
+NOMINAL_HBM_GBS = 8000.0     # nominal B200 HBM3e bandwidth (about 8 TB/s); the roofline peak is the measured copy
 
 # DRAM traffic per launch of the dominant kernel, from one ncu capture of the full
 # workload (dram__bytes_read.sum + dram__bytes_write.sum, one pass; the summary is in
@@ -330,6 +331,7 @@ def run_b200(args, world, rank, local):
         m = statistics.median(part_ms[n])
         d = {"ms": round(m, 5), "gbs": round(pbytes[n] / (m * 1e-3) / 1e9, 1)}
         d["frac_hbm"] = round(d["gbs"] / hbm, 4)
+        d["frac_nominal_8tbs"] = round(d["gbs"] / NOMINAL_HBM_GBS, 4)
         if n == "w4a4_linear":
             d["tops"] = round(GEMM_OPS / (m * 1e-3) / 1e12, 1)
             d["frac_int8_peak"] = round(d["tops"] / int8_peak, 4)
@@ -355,6 +357,8 @@ def run_b200(args, world, rank, local):
     if not args.no_e2e:
         e2e = run_e2e(args, dev, step, parts, x_cpu, g_cpu, w_cpu, flush, world)
 
+    probe = mma_probe(dev, breakdown["w4a4_linear"]["tops"])
+
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = cpu_baseline(args)
@@ -371,6 +375,7 @@ def run_b200(args, world, rank, local):
         "parts": breakdown,
         "w4a4_tops": breakdown["w4a4_linear"]["tops"],
         "roofline": roofline,
+        "int8_mma_probe": probe,
         "gpu_launches": step.launches_per_step * args.steps,
         "clocks": clocks.summary(),
         "wall_s_timed_loop": round(wall, 4),
@@ -379,6 +384,30 @@ def run_b200(args, world, rank, local):
     }
     if rank == 0:
         print(json.dumps(result), flush=True)
+
+
+def mma_probe(dev, gemm_tops, iters=20000, reps=5):
+    """int8 tensor-core rate with no memory traffic (back-to-back tcgen05.mma
+    kind::i8, M 128 N 256 K 32, one CTA per SM): context for the GEMM's fraction."""
+    import statistics
+    import torch
+    import bit_quantization_aware_blockwise_b200 as q
+    stream = torch.cuda.current_stream(dev)
+    q.probe_mma_i8(iters, stream.cuda_stream)
+    ts, ctas = [], 0
+    for _ in range(reps):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        ctas = q.probe_mma_i8(iters, stream.cuda_stream)
+        b.record(stream)
+        torch.cuda.synchronize()
+        ts.append(a.elapsed_time(b))
+    q.probe_status(stream.cuda_stream)
+    ms = statistics.median(ts)
+    tops = 2.0 * 128 * 256 * 32 * iters * ctas / (ms * 1e-3) / 1e12
+    return {"tops": round(tops, 1), "iters": iters, "ctas": ctas,
+            "gemm_frac_of_probe": round(gemm_tops / tops, 4),
+            "note": "timed alone right after the bench loop; the roofline peak stays the measured bf16 x 2"}
 
 
 def run_e2e(args, dev, step, parts, x_cpu, g_cpu, w_cpu, flush, world):
@@ -454,14 +483,37 @@ def oracle_sample(rows_x=256, rows_w=88, gemm_rows=16):
     return dt, nbytes, sample
 
 
+def _oracle_shard(shape):
+    return oracle_sample(*shape)[:2]
+
+
+def oracle_all_cores(rows_x, rows_w, gemm_rows):
+    """The same sample split into row shards over every host core (one process per
+    core, spawned; the oracle itself unchanged). Returns (seconds, bytes, cores)."""
+    import multiprocessing as mp
+    n = max(1, os.cpu_count() or 1)
+    shard = (max(1, rows_x // n), max(1, rows_w // n), max(1, gemm_rows // n))
+    with mp.get_context("spawn").Pool(n) as pool:
+        pool.map(_oracle_shard, [(2, 2, 1)] * n)          # start-up and imports, untimed
+        t0 = time.perf_counter()
+        res = pool.map(_oracle_shard, [shard] * n)
+        dt = time.perf_counter() - t0
+    return dt, sum(b for _, b in res), n
+
+
 def cpu_baseline(args):
     import oracle
     oracle.build()
     # the full activation, gradient and weight legs and a 512-row block of the GEMM:
     # about 10-20 s of single-threaded CPU work
     dt, nbytes, sample = oracle_sample(rows_x=R, rows_w=NW, gemm_rows=512)
-    return {"value": round(nbytes / dt / 1e9, 5), "unit": "GB/s", "cores": 1, "kind": "oracle",
-            "sample": sample, "seconds": round(dt, 3)}
+    out = {"value": round(nbytes / dt / 1e9, 5), "unit": "GB/s", "cores": 1, "kind": "oracle",
+           "sample": sample, "seconds": round(dt, 3)}
+    dt_n, bytes_n, n = oracle_all_cores(R, NW, 512)
+    out["all_cores"] = {"value": round(bytes_n / dt_n / 1e9, 5), "unit": "GB/s", "cores": n,
+                        "seconds": round(dt_n, 3),
+                        "sample": "the same sample split into row shards, one spawned process per core"}
+    return out
 
 
 def run_reference(args, world, rank):
@@ -491,6 +543,157 @@ def run_reference(args, world, rank):
         "gpu_launches": 0,
     }
     print(json.dumps(line), flush=True)
+
+
+def _timed(f, flush, stream, warmup=10, reps=50):
+    """Median and p10 (us) of `reps` launches of f, L2 flushed before each (untimed)."""
+    import statistics
+    import torch
+    for _ in range(warmup):
+        f()
+    torch.cuda.synchronize()
+    ts = []
+    for _ in range(reps):
+        flush.zero_()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        f()
+        b.record(stream)
+        torch.cuda.synchronize()
+        ts.append(a.elapsed_time(b) * 1e3)
+    ts.sort()
+    return statistics.median(ts), ts[len(ts) // 10]
+
+
+def _graph_us(make_launch, sets, stream, n=20):
+    """One CUDA graph of n launches cycling over `sets` buffer sets; us per launch."""
+    import torch
+    for k in range(len(sets)):
+        make_launch(sets[k])()
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        for i in range(n):
+            make_launch(sets[i % len(sets)])()
+    g.replay()
+    torch.cuda.synchronize()
+    ts = []
+    for _ in range(10):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        g.replay()
+        b.record(stream)
+        torch.cuda.synchronize()
+        ts.append(a.elapsed_time(b) * 1e3 / n)
+    del g
+    return sorted(ts)[len(ts) // 2]
+
+
+def run_configs(args):
+    """Kernel timings for every workload configuration of the hot path (not the
+    bench line): median and p10 of 50 launches after 10 warm-ups, L2 flushed
+    before each launch outside the events; the weight tensors also as a CUDA graph
+    of 20 launches rotating over 16 buffer sets (> 3x L2)."""
+    import torch
+    import bit_quantization_aware_blockwise_b200 as q
+    from bit_quantization_aware_blockwise_b200 import inputs
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.Stream(dev)     # a non-default stream, so launches can be graph-captured
+    torch.cuda.set_stream(stream)
+    s = stream.cuda_stream
+    peaks = load_peaks()
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    rows = []
+
+    def add(name, f, nbytes, unit_ops=None, extra=None):
+        med, p10 = _timed(f, flush, stream)
+        r = {"case": name, "median_us": round(med, 2), "p10_us": round(p10, 2), "bytes": nbytes,
+             "gbs": round(nbytes / (med * 1e-6) / 1e9, 1)}
+        r["frac_hbm_measured"] = round(r["gbs"] / peaks["hbm_gbs"], 4)
+        r["frac_nominal_8tbs"] = round(r["gbs"] / NOMINAL_HBM_GBS, 4)
+        if unit_ops:
+            r["tops"] = round(unit_ops / (med * 1e-6) / 1e12, 1)
+            r["frac_int8_peak"] = round(r["tops"] / (peaks["bf16_tflops"] * 2.0), 4)
+        if extra:
+            r.update(extra)
+        rows.append(r)
+        print(json.dumps(r), flush=True)
+
+    def quant(x, bits, rms, code_mode, mask_mode, deq_dtype=None):
+        rr, cc = x.shape
+        codes = torch.empty(q.codes_bytes(rr, cc, bits, code_mode), dtype=torch.uint8, device=dev)
+        scales = torch.empty(rr * (cc // rms), dtype=torch.float32, device=dev)
+        mask = torch.empty(q.mask_bytes(rr, cc, mask_mode), dtype=torch.uint8, device=dev) \
+            if mask_mode is not None else None
+        deq = None
+        if deq_dtype is not None:
+            deq = torch.empty((rr, cc), dtype=torch.bfloat16 if deq_dtype == q.BF16 else torch.float32,
+                              device=dev)
+        xd = q.FP32 if x.dtype == torch.float32 else q.BF16
+        f = lambda: q.quantize_fwd_raw(
+            x.data_ptr(), xd, rr, cc, cc, bits, HB, rms, 1.0, code_mode, codes.data_ptr(), scales.data_ptr(),
+            mask_mode if mask_mode is not None else 0, mask.data_ptr() if mask is not None else None,
+            deq.data_ptr() if deq is not None else None, deq_dtype if deq is not None else 0, s)
+        esz = x.element_size()
+        e = rr * cc
+        nbytes = esz * e + codes.numel() + (mask.numel() if mask is not None else 0) + 4 * scales.numel() \
+            + (deq.numel() * deq.element_size() if deq is not None else 0)
+        return f, nbytes, (codes, scales, mask)
+
+    # config 1: fp32 256 x 512, int8 codes, fp32 dequant, byte mask
+    x1 = inputs.smoke_input().to(dev)
+    f, nb, _ = quant(x1, 4, HB, q.CODES_INT8, q.MASK_BYTES, q.FP32)
+    add("cfg1 quantize fp32 256x512 b4 int8+fp32 deq+byte mask", f, nb)
+    # config 2: activations 16384 x 2048
+    x2 = inputs.activation_input().to(dev)
+    for bits in (1, 2, 3, 4, 8):
+        f, nb, _ = quant(x2, bits, HB, q.CODES_PACKED, q.MASK_BITS)
+        add(f"cfg2 quantize 16384x2048 b{bits} codes+mask", f, nb)
+    f, nb, _ = quant(x2, 4, HB, q.CODES_PACKED, q.MASK_BITS, q.BF16)
+    add("cfg2 quantize 16384x2048 b4 codes+mask+bf16 yhat", f, nb)
+    # config 3: weights, with the CUDA-graph batch over rotated buffers
+    for wname, wt in (("W_up 5632x2048", inputs.weight_up()), ("W_down 2048x5632", inputs.weight_down())):
+        w = wt.to(dev)
+        for bits in (1, 4):
+            f, nb, _ = quant(w, bits, HB, q.CODES_PACKED, q.MASK_BITS)
+            sets = [quant(w.clone(), bits, HB, q.CODES_PACKED, q.MASK_BITS)[0] for _ in range(16)]
+            g_us = _graph_us(lambda fn: fn, sets, stream)
+            add(f"cfg3 quantize {wname} b{bits} codes+mask", f, nb,
+                extra={"graph_us_per_launch": round(g_us, 2),
+                       "graph_gbs": round(nb / (g_us * 1e-6) / 1e9, 1)})
+            del sets
+    # config 4: trust backward with config 2's b = 4 mask
+    fq, _, (codes, scales, mask) = quant(x2, 4, HB, q.CODES_PACKED, q.MASK_BITS)
+    fq()
+    g = inputs.grad_input().to(dev)
+    gi = torch.empty_like(g)
+    f = lambda: q.trust_bwd_raw(g.data_ptr(), mask.data_ptr(), q.MASK_BITS, R, C, HB, gi.data_ptr(), s)
+    add("cfg4 trust backward 16384x2048", f, 4 * R * C + R * C // 8)
+    # config 5: operand codes (one RMS per row) and the linear layer
+    fx, nbx, (cx, sx, _) = quant(x2, 4, C, q.CODES_GEMM_OPERAND, None)
+    add("cfg5 operand quantize X 16384x2048 (row RMS)", fx, nbx)
+    w = inputs.weight_up().to(dev)
+    fw, nbw, (cw, sw, _) = quant(w, 4, C, q.CODES_GEMM_OPERAND, None)
+    add("cfg5 operand quantize W_up 5632x2048 (row RMS)", fw, nbw)
+    fx(); fw()
+    y = torch.empty((R, NW), dtype=torch.bfloat16, device=dev)
+    f = lambda: q.w4a4_linear_raw(cx.data_ptr(), sx.data_ptr(), cw.data_ptr(), sw.data_ptr(), R, NW, C,
+                                  y.data_ptr(), None, s)
+    add("cfg5 W4A4 linear 16384x5632x2048", f, R * C + NW * C + 4 * (R + NW) + 2 * R * NW, unit_ops=GEMM_OPS)
+    # the 1-bit path: b = 1 operand codes (c in {-1, +1}) through the same GEMM
+    fx1, nbx1, (cx1, sx1, _) = quant(x2, 1, C, q.CODES_GEMM_OPERAND, None)
+    fw1, nbw1, (cw1, sw1, _) = quant(w, 1, C, q.CODES_GEMM_OPERAND, None)
+    add("W1A1 operand quantize X 16384x2048 b1 (row RMS)", fx1, nbx1)
+    fx1(); fw1()
+    f = lambda: q.w4a4_linear_raw(cx1.data_ptr(), sx1.data_ptr(), cw1.data_ptr(), sw1.data_ptr(), R, NW, C,
+                                  y.data_ptr(), None, s)
+    add("W1A1 linear 16384x5632x2048 (+-1 codes)", f, R * C + NW * C + 4 * (R + NW) + 2 * R * NW,
+        unit_ops=GEMM_OPS)
+    gemm_tops = rows[-3]["tops"]
+    q.device_status()
+    probe = mma_probe(dev, gemm_tops)
+    print(json.dumps({"configs": rows, "int8_mma_probe": probe, "peaks": peaks}), flush=True)
 
 
 def run_profile_kernels(args):
@@ -530,9 +733,14 @@ def main():
     ap.add_argument("--profile-kernels", action="store_true",
                     help="launch each kernel once on an ncu-sized case and exit")
     ap.add_argument("--profile-rows", type=int, default=32768)
+    ap.add_argument("--configs", action="store_true",
+                    help="time every workload configuration (median / p10 per kernel) and exit")
     args = ap.parse_args()
     if args.profile_kernels:
         run_profile_kernels(args)
+        return
+    if args.configs:
+        run_configs(args)
         return
     if args.warmup < 3 and args.impl == "b200":
         args.warmup = 3

@@ -13,6 +13,8 @@ from ._binding import (  # noqa: F401
     CODES_GEMM_OPERAND,
     MASK_BITS,
     MASK_BYTES,
+    BF16,
+    FP32,
     library_path,
     load_library,
     alpha,
@@ -26,11 +28,13 @@ from ._binding import (  # noqa: F401
     trust_bwd_raw,
     w4a4_linear_raw,
     device_status,
+    probe_mma_i8,
+    probe_status,
 )
 
 __all__ = [
     "QuestError", "CODES_PACKED", "CODES_INT8", "CODES_GEMM_OPERAND", "MASK_BITS",
-    "MASK_BYTES", "library_path", "load_library", "alpha", "codes_bytes", "mask_bytes",
+    "MASK_BYTES", "BF16", "FP32", "library_path", "load_library", "alpha", "codes_bytes", "mask_bytes",
     "container_bits", "quantize_fwd", "trust_bwd", "w4a4_linear", "quantize_fwd_raw",
-    "trust_bwd_raw", "w4a4_linear_raw", "device_status",
+    "trust_bwd_raw", "w4a4_linear_raw", "device_status", "probe_mma_i8", "probe_status",
 ]

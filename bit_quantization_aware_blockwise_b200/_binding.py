@@ -35,6 +35,8 @@ SIGNATURES = {
     "quest_status_string": (ctypes.c_char_p, [_int]),
     "quest_last_error_message": (ctypes.c_char_p, []),
     "quest_version": (_int, []),
+    "quest_probe_mma_i8": (_int, [_int, _p, _p]),
+    "quest_probe_status": (_int, [_p]),
 }
 
 _lock = threading.Lock()
@@ -228,3 +230,14 @@ def w4a4_linear(a_codes, a_scales, w_codes, w_scales, out=None, acc: bool = Fals
                     M, N, K, out.data_ptr(), acc_t.data_ptr() if acc_t is not None else None,
                     _stream_handle(stream, dev))
     return (out, acc_t) if acc else out
+
+
+def probe_mma_i8(iters, stream=0):
+    """Enqueue the int8 tensor-core peak probe; returns the number of CTAs launched."""
+    ctas = ctypes.c_int(0)
+    _check(load_library().quest_probe_mma_i8(iters, ctypes.byref(ctas), stream), "quest_probe_mma_i8")
+    return ctas.value
+
+
+def probe_status(stream=0):
+    _check(load_library().quest_probe_status(stream), "quest_probe_status")

@@ -1,0 +1,132 @@
+// Tensor-core peak probe: back-to-back tcgen05.mma kind::i8 (M = 128, N = 256,
+// K = 32, the integer linear layer's instruction shape) from shared-memory
+// operands into one TMEM accumulator, one CTA per SM, no loads and no epilogue.
+// The caller times a launch; 2 * 128 * 256 * 32 * iters * SMs / time is the
+// int8 MMA rate this part sustains at its current clocks, the denominator the
+// GEMM's tensor-core fraction can be read against besides the nominal figure.
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "quest.h"
+#include "quest_internal.h"
+#include "quest_probe.h"
+
+namespace quest {
+
+__device__ int g_probe_status = 0;
+
+namespace {
+
+constexpr int kProbeThreads = 128;
+constexpr uint32_t kProbeSmem = 120 * 1024;   // more than half an SM: one CTA per SM
+constexpr uint32_t kA = 0, kB = 128 * 128;     // A 128 x 128 B, B 256 x 128 B (swizzled rows)
+constexpr uint32_t kBar = kB + 256 * 128;
+constexpr uint32_t kSlot = kBar + 8;
+constexpr uint32_t kIdescProbe = (2u << 4) | (1u << 7) | (1u << 10) | (uint32_t(256 >> 3) << 17) |
+                                 (uint32_t(128 >> 4) << 24);
+
+__device__ __forceinline__ uint64_t probe_desc(uint32_t addr) {
+    uint64_t d = 0;
+    d |= uint64_t((addr >> 4) & 0x3FFFu);
+    d |= uint64_t(1) << 16;
+    d |= uint64_t(1024 >> 4) << 32;
+    d |= uint64_t(1) << 46;
+    d |= uint64_t(2) << 61;
+    return d;
+}
+
+__global__ void __launch_bounds__(kProbeThreads, 1) probe_mma_i8_kernel(int iters) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const uint32_t sbase = static_cast<uint32_t>(__cvta_generic_to_shared(smem));
+    for (uint32_t i = threadIdx.x * 16; i < kBar; i += kProbeThreads * 16)
+        *reinterpret_cast<uint4*>(smem + i) = make_uint4(0x01010101u, 0x01010101u, 0x01010101u, 0x01010101u);
+    const uint32_t bar = sbase + kBar;
+    if (threadIdx.x == 0) {
+        asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(bar) : "memory");
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    const int warp = threadIdx.x >> 5;
+    if (warp == 0) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], 256;" ::"r"(sbase + kSlot)
+                     : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    }
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");   // operand writes -> tensor core
+    asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+    __syncthreads();
+    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+    const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(smem + kSlot);
+
+    if (threadIdx.x == 0) {
+        const uint64_t a = probe_desc(sbase + kA), b = probe_desc(sbase + kB);
+        for (int i = 0; i < iters; ++i) {
+            asm volatile(
+                "{\n\t.reg .pred p;\n\t"
+                "setp.ne.b32 p, %4, 0;\n\t"
+                "tcgen05.mma.cta_group::1.kind::i8 [%0], %1, %2, %3, p;\n\t}" ::"r"(tmem),
+                "l"(a), "l"(b), "r"(kIdescProbe), "r"(i)
+                : "memory");
+        }
+        asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
+                     : "memory");
+        // bounded wait for the MMAs to finish (2 s)
+        uint64_t t0, t;
+        asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t0));
+        for (;;) {
+            uint32_t ok;
+            asm volatile(
+                "{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], 0;\n\t"
+                "selp.u32 %0, 1, 0, p;\n\t}"
+                : "=r"(ok)
+                : "r"(bar)
+                : "memory");
+            if (ok) break;
+            asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+            if (t - t0 > 2000000000ull) {
+                atomicExch(&g_probe_status, (int)QUEST_ETIMEOUT);
+                break;
+            }
+        }
+    }
+    asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+    __syncthreads();
+    if (warp == 0) {
+        asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, 256;" ::"r"(tmem) : "memory");
+    }
+}
+
+}  // namespace
+}  // namespace quest
+
+extern "C" quest_status quest_probe_mma_i8(int iters, int* ctas, void* stream) {
+    using namespace quest;
+    if (iters < 1 || iters > (1 << 24) || ctas == nullptr) return QUEST_EINVAL;
+    static thread_local int attr_dev = -1;
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (attr_dev != dev) {
+        if (cudaFuncSetAttribute(probe_mma_i8_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 kProbeSmem + 1024) != cudaSuccess)
+            return QUEST_ECUDA;
+        attr_dev = dev;
+    }
+    *ctas = sm_count();
+    probe_mma_i8_kernel<<<*ctas, kProbeThreads, kProbeSmem + 1024, static_cast<cudaStream_t>(stream)>>>(iters);
+    return cudaGetLastError() == cudaSuccess ? QUEST_OK : QUEST_ECUDA;
+}
+
+extern "C" quest_status quest_probe_status(void* stream) {
+    int v = 0, zero = 0;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (cudaMemcpyFromSymbolAsync(&v, quest::g_probe_status, sizeof(int), 0, cudaMemcpyDeviceToHost, s) !=
+            cudaSuccess ||
+        cudaStreamSynchronize(s) != cudaSuccess)
+        return QUEST_ECUDA;
+    if (v != 0) {
+        cudaMemcpyToSymbolAsync(quest::g_probe_status, &zero, sizeof(int), 0, cudaMemcpyHostToDevice, s);
+        cudaStreamSynchronize(s);
+    }
+    return static_cast<quest_status>(v);
+}

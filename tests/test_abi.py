@@ -130,3 +130,11 @@ def test_w4a4_rejects_invalid_arguments():
     assert call(y=None) == 1
     assert call(sa=FAKE + 2) == 1
     assert call(M=0) == 0 and call(N=0) == 0   # empty output: nothing to do
+
+
+def test_probe_rejects_invalid_arguments():
+    lib = q.load_library()
+    n = ctypes.c_int(0)
+    assert lib.quest_probe_mma_i8(0, ctypes.byref(n), None) == 1
+    assert lib.quest_probe_mma_i8(1 << 25, ctypes.byref(n), None) == 1
+    assert lib.quest_probe_mma_i8(100, None, None) == 1

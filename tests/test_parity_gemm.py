@@ -140,3 +140,40 @@ def test_quantized_linear_end_to_end(cuda_device):
     exact = inputs.to_f64(X) @ inputs.to_f64(W).T
     rel = np.linalg.norm(oracle.bf16_bits_to_f64(yb) - exact) / np.linalg.norm(exact)
     assert rel < 0.3
+
+
+def test_w1a1_linear_end_to_end(cuda_device):
+    # The 1-bit path: X and W quantized at b = 1 (one RMS per row, operand codes
+    # c = 2q + 1 in {-1, +1}) and multiplied by the same int8 tensor-core GEMM.
+    dev = torch.device("cuda:0")
+    X = inputs.activation_input(rows=384)
+    W = inputs.weight_up(rows=512)
+    K = X.shape[1]
+    qx = q.quantize_fwd(X.to(dev), 1, rms_group=K, code_mode=q.CODES_GEMM_OPERAND, mask_mode=None)
+    qw = q.quantize_fwd(W.to(dev), 1, rms_group=K, code_mode=q.CODES_GEMM_OPERAND, mask_mode=None)
+    cx = qx["codes"].view(torch.int8).reshape(384, K)
+    cw = qw["codes"].view(torch.int8).reshape(512, K)
+    y, acc_gpu = q.w4a4_linear(cx, qx["scales"].reshape(-1), cw, qw["scales"].reshape(-1), acc=True)
+    q.device_status()
+    gpu_cx = unpack_codes(cx.cpu().numpy(), 384, K, 1, 2)
+    gpu_cw = unpack_codes(cw.cpu().numpy(), 512, K, 1, 2)
+    assert set(np.unique(gpu_cx)) <= {-1, 1} and set(np.unique(gpu_cw)) <= {-1, 1}
+    ox = oracle.quantize(inputs.to_f64(X), bits=1, had=128, rms_group=K)
+    ow = oracle.quantize(inputs.to_f64(W), bits=1, had=128, rms_group=K)
+    check_codes_operand(gpu_cx, ox)
+    check_codes_operand(gpu_cw, ow)
+    acc = oracle.gemm_i8((2 * ox["q"] + 1).astype(np.int8), (2 * ow["q"] + 1).astype(np.int8))
+    ref = oracle.dequant_linear(acc, ox["scale"][:, 0], ow["scale"][:, 0])
+    rows_same = np.all(gpu_cx == 2 * ox["q"] + 1, axis=1)
+    cols_same = np.all(gpu_cw == 2 * ow["q"] + 1, axis=1)
+    same = rows_same[:, None] & cols_same[None, :]
+    assert same.mean() > 0.95
+    # the accumulator is exact wherever both code rows agree with the oracle's
+    assert np.array_equal(acc_gpu.cpu().numpy()[same], acc[same].astype(np.int32))
+    yb = y.cpu().view(torch.int16).numpy().view(np.uint16)
+    check_bf16(yb, ref, skip=~same, what="y end to end (W1A1)")
+    # sanity, not parity: the 1-bit product still tracks X W^T
+    exact = inputs.to_f64(X) @ inputs.to_f64(W).T
+    yv = oracle.bf16_bits_to_f64(yb)
+    corr = np.sum(yv * exact) / (np.linalg.norm(yv) * np.linalg.norm(exact))
+    assert corr > 0.5
