@@ -75,6 +75,8 @@ def _load():
         lib.oracle_gemm_i8.restype = _int
         lib.oracle_dequant_linear.argtypes = [_p, _p, _p, _i64, _i64, _p]
         lib.oracle_dequant_linear.restype = _int
+        lib.oracle_linear_grouped.argtypes = [_p, _p, _p, _p, _i64, _i64, _i64, _i64, _p, _p]
+        lib.oracle_linear_grouped.restype = _int
         lib.oracle_bf16_rne.argtypes = [_dbl]
         lib.oracle_bf16_rne.restype = ctypes.c_uint16
         lib.oracle_bf16_rne_array.argtypes = [_p, _i64, _p]
@@ -169,6 +171,23 @@ def dequant_linear(acc, delta_a, delta_b) -> np.ndarray:
     _check(_load().oracle_dequant_linear(_ptr(acc), _ptr(da), _ptr(db), acc.shape[0],
                                          acc.shape[1], _ptr(y)), "dequant_linear")
     return y
+
+
+def linear_grouped(a, b, delta_a, delta_b, group: int = 128):
+    """Y = sum_g (Delta_a[:, g]/2)(Delta_b[:, g]/2) * (A_g @ B_g^T) in fp64, with A_g the
+    int8 codes of K-group g; returns (Y, sum_g |term_g|)."""
+    a = np.ascontiguousarray(np.asarray(a, dtype=np.int8))
+    b = np.ascontiguousarray(np.asarray(b, dtype=np.int8))
+    da = np.ascontiguousarray(np.asarray(delta_a, dtype=np.float64))
+    db = np.ascontiguousarray(np.asarray(delta_b, dtype=np.float64))
+    M, K = a.shape
+    N = b.shape[0]
+    assert b.shape[1] == K and da.shape == (M, K // group) and db.shape == (N, K // group)
+    y = np.empty((M, N), dtype=np.float64)
+    mag = np.empty((M, N), dtype=np.float64)
+    _check(_load().oracle_linear_grouped(_ptr(a), _ptr(b), _ptr(da), _ptr(db), M, N, K, group,
+                                         _ptr(y), _ptr(mag)), "linear_grouped")
+    return y, mag
 
 
 def bf16_rne(v) -> np.ndarray:

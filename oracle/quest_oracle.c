@@ -315,6 +315,34 @@ int oracle_dequant_linear(const int64_t* acc, const double* delta_a, const doubl
     return ORACLE_OK;
 }
 
+/* Linear layer with one scale per (row, group of `group` consecutive K
+ * indices) on both operands:
+ *   Y[m][n] = sum_g (Delta_a[m][g] / 2) * (Delta_b[n][g] / 2) * acc_g[m][n],
+ *   acc_g[m][n] = sum over k in group g of A[m][k] * B[n][k]   (int64).
+ * `mag` (nullable) receives sum_g |term_g|, the scale of the rounding error
+ * of any finite-precision sum of the G terms. */
+int oracle_linear_grouped(const int8_t* A, const int8_t* B, const double* delta_a,
+                          const double* delta_b, int64_t M, int64_t N, int64_t K, int64_t group,
+                          double* y, double* mag) {
+    if (M < 0 || N < 0 || K < 0 || group <= 0 || K % group != 0) return ORACLE_EINVAL;
+    const int64_t G = K / group;
+    for (int64_t m = 0; m < M; ++m)
+        for (int64_t n = 0; n < N; ++n) {
+            double sum = 0.0, abs_sum = 0.0;
+            for (int64_t g = 0; g < G; ++g) {
+                int64_t acc = 0;
+                for (int64_t k = g * group; k < (g + 1) * group; ++k)
+                    acc += (int64_t)A[m * K + k] * (int64_t)B[n * K + k];
+                const double term = (double)acc * (delta_a[m * G + g] * 0.5) * (delta_b[n * G + g] * 0.5);
+                sum += term;
+                abs_sum += fabs(term);
+            }
+            y[m * N + n] = sum;
+            if (mag) mag[m * N + n] = abs_sum;
+        }
+    return ORACLE_OK;
+}
+
 /* ------------------------------------------------------------------------- */
 /* Rounding of an fp64 value to bfloat16, round-to-nearest-even, one rounding. */
 /* ------------------------------------------------------------------------- */

@@ -416,3 +416,48 @@ def test_bf16_rne_ties_to_even_and_single_rounding():
     assert oracle.bf16_rne(np.array([-(one + 2 ** -8 + 2 ** -40)]))[0] == 0xBF81
     vals = oracle.bf16_bits_to_f64(np.array([0x3F80, 0xC020, 0x0001], dtype=np.uint16))
     assert list(vals) == [1.0, -2.5, 2.0 ** -133]
+
+
+# --- per-group-scaled linear layer -------------------------------------------
+def _grouped_case(M, N, K, seed):
+    g = np.random.default_rng(seed)
+    a = (2 * g.integers(-8, 8, size=(M, K)) + 1).astype(np.int8)
+    b = (2 * g.integers(-8, 8, size=(N, K)) + 1).astype(np.int8)
+    sa = np.exp(g.uniform(-6, -2, size=(M, K // 128)))
+    sb = np.exp(g.uniform(-6, -2, size=(N, K // 128)))
+    return a, b, sa, sb
+
+
+def test_grouped_linear_equals_product_of_scaled_operands():
+    # Scale-then-multiply with a library matmul against the oracle's
+    # multiply-then-scale per group: the same bilinear form in another order.
+    a, b, sa, sb = _grouped_case(7, 9, 512, 1)
+    y, mag = oracle.linear_grouped(a, b, sa, sb)
+    at = a.astype(np.float64) * np.repeat(sa / 2, 128, axis=1)
+    bt = b.astype(np.float64) * np.repeat(sb / 2, 128, axis=1)
+    ref = at @ bt.T
+    assert np.allclose(y, ref, rtol=0, atol=1e-12 * np.max(mag))
+    assert np.all(mag >= np.abs(y) * (1 - 1e-15))
+
+
+def test_grouped_linear_with_row_constant_scales_is_the_row_scaled_layer():
+    # Constant scales along K reduce the grouped layer to one int32 accumulator
+    # per output and the per-row dequantisation.
+    a, b, _, _ = _grouped_case(5, 6, 384, 2)
+    ra = np.exp(np.random.default_rng(3).uniform(-5, -1, size=5))
+    rb = np.exp(np.random.default_rng(4).uniform(-5, -1, size=6))
+    y, _ = oracle.linear_grouped(a, b, np.repeat(ra[:, None], 3, axis=1), np.repeat(rb[:, None], 3, axis=1))
+    ref = oracle.dequant_linear(oracle.gemm_i8(a, b), ra, rb)
+    assert np.allclose(y, ref, rtol=1e-14, atol=0)
+
+
+def test_grouped_linear_groups_are_independent():
+    # Zeroing the scales of one group removes exactly that group's K-slice.
+    a, b, sa, sb = _grouped_case(4, 5, 512, 5)
+    sa0 = sa.copy()
+    sa0[:, 2] = 0.0
+    y0, _ = oracle.linear_grouped(a, b, sa0, sb)
+    a_cut = a.copy()
+    a_cut[:, 256:384] = 0
+    y_cut, _ = oracle.linear_grouped(a_cut, b, sa, sb)
+    assert np.allclose(y0, y_cut, rtol=1e-14, atol=0)
