@@ -690,7 +690,18 @@ def run_configs(args):
                                   y.data_ptr(), None, s)
     add("W1A1 linear 16384x5632x2048 (+-1 codes)", f, R * C + NW * C + 4 * (R + NW) + 2 * R * NW,
         unit_ops=GEMM_OPS)
-    gemm_tops = rows[-3]["tops"]
+    # per-128-group scales on both operands: E4M3 operand codes and the grouped layer
+    E4 = q.CODES_GEMM_OPERAND_E4M3
+    fxg, nbxg, (cxg, sxg, _) = quant(x2, 4, HB, E4, None)
+    fwg, nbwg, (cwg, swg, _) = quant(w, 4, HB, E4, None)
+    add("grouped operand quantize X 16384x2048 b4 E4M3 (RMS per 128-group)", fxg, nbxg)
+    fxg(); fwg()
+    G = C // HB
+    f = lambda: q.w4a4_linear_grouped_raw(cxg.data_ptr(), sxg.data_ptr(), cwg.data_ptr(), swg.data_ptr(),
+                                          R, NW, C, HB, y.data_ptr(), None, s)
+    add("grouped linear 16384x5632x2048 (E4M3 codes, scales per 128-group)", f,
+        R * C + NW * C + 4 * G * (R + NW) + 2 * R * NW, unit_ops=GEMM_OPS)
+    gemm_tops = rows[-5]["tops"]
     q.device_status()
     probe = mma_probe(dev, gemm_tops)
     print(json.dumps({"configs": rows, "int8_mma_probe": probe, "peaks": peaks}), flush=True)

@@ -11,6 +11,7 @@ from ._binding import (  # noqa: F401
     CODES_PACKED,
     CODES_INT8,
     CODES_GEMM_OPERAND,
+    CODES_GEMM_OPERAND_E4M3,
     MASK_BITS,
     MASK_BYTES,
     BF16,
@@ -27,14 +28,16 @@ from ._binding import (  # noqa: F401
     quantize_fwd_raw,
     trust_bwd_raw,
     w4a4_linear_raw,
+    w4a4_linear_grouped,
+    w4a4_linear_grouped_raw,
     device_status,
     probe_mma_i8,
     probe_status,
 )
 
 __all__ = [
-    "QuestError", "CODES_PACKED", "CODES_INT8", "CODES_GEMM_OPERAND", "MASK_BITS",
+    "QuestError", "CODES_PACKED", "CODES_INT8", "CODES_GEMM_OPERAND", "CODES_GEMM_OPERAND_E4M3", "MASK_BITS",
     "MASK_BYTES", "BF16", "FP32", "library_path", "load_library", "alpha", "codes_bytes", "mask_bytes",
     "container_bits", "quantize_fwd", "trust_bwd", "w4a4_linear", "quantize_fwd_raw",
-    "trust_bwd_raw", "w4a4_linear_raw", "device_status", "probe_mma_i8", "probe_status",
+    "trust_bwd_raw", "w4a4_linear_raw", "w4a4_linear_grouped", "w4a4_linear_grouped_raw", "device_status", "probe_mma_i8", "probe_status",
 ]

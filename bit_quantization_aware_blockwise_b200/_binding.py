@@ -14,7 +14,7 @@ import threading
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _LIB_NAME = "libquest_b200.so"
 
-CODES_PACKED, CODES_INT8, CODES_GEMM_OPERAND = 0, 1, 2
+CODES_PACKED, CODES_INT8, CODES_GEMM_OPERAND, CODES_GEMM_OPERAND_E4M3 = 0, 1, 2, 3
 MASK_BITS, MASK_BYTES = 0, 1
 BF16, FP32 = 0, 1
 _STATUS = {0: "ok", 1: "invalid argument", 2: "unsupported", 3: "CUDA error", 4: "device wait timed out"}
@@ -27,6 +27,7 @@ SIGNATURES = {
                                   _int, _p, _p, _int, _p]),
     "quest_trust_bwd": (_int, [_p, _p, _int, _i64, _i64, _int, _p, _p]),
     "quest_w4a4_linear": (_int, [_p, _p, _p, _p, _i64, _i64, _i64, _p, _p, _p]),
+    "quest_w4a4_linear_grouped": (_int, [_p, _p, _p, _p, _i64, _i64, _i64, _i64, _p, _p, _p]),
     "quest_device_status": (_int, [_p]),
     "quest_alpha": (_f64, [_int]),
     "quest_container_bits": (_int, [_int]),
@@ -103,6 +104,11 @@ def trust_bwd_raw(grad_out, mask, mask_mode, rows, cols, had_block, grad_in, str
 def w4a4_linear_raw(a_codes, a_scales, w_codes, w_scales, M, N, K, y, acc=None, stream=0):
     _check(load_library().quest_w4a4_linear(a_codes, a_scales, w_codes, w_scales, M, N, K, y, acc,
                                             stream), "quest_w4a4_linear")
+
+
+def w4a4_linear_grouped_raw(a_codes, a_scales, w_codes, w_scales, M, N, K, group, y, y_f32=None, stream=0):
+    _check(load_library().quest_w4a4_linear_grouped(a_codes, a_scales, w_codes, w_scales, M, N, K, group, y,
+                                                    y_f32, stream), "quest_w4a4_linear_grouped")
 
 
 def device_status(stream=0):
@@ -230,6 +236,37 @@ def w4a4_linear(a_codes, a_scales, w_codes, w_scales, out=None, acc: bool = Fals
                     M, N, K, out.data_ptr(), acc_t.data_ptr() if acc_t is not None else None,
                     _stream_handle(stream, dev))
     return (out, acc_t) if acc else out
+
+
+def w4a4_linear_grouped(a_codes, a_scales, w_codes, w_scales, out=None, y_f32: bool = False,
+                        group: int = 128, stream=None):
+    """y = bf16(sum_g (a_scales[:, g]/2)(w_scales[:, g]/2) * (A_g @ W_g^T)), A_g / W_g the
+    codes of K-group g. Codes are FP8 E4M3 bytes [M, K] / [N, K] (float8_e4m3fn or uint8:
+    the CODES_GEMM_OPERAND_E4M3 form); scales fp32 [M, K/group] / [N, K/group].
+    Returns y (and the fp32 result before rounding if y_f32)."""
+    torch = _torch()
+    for t, n in ((a_codes, "a_codes"), (w_codes, "w_codes"), (a_scales, "a_scales"), (w_scales, "w_scales")):
+        _require_cuda(t, n)
+    ok = (torch.uint8, torch.float8_e4m3fn)
+    if a_codes.dtype not in ok or w_codes.dtype not in ok:
+        raise QuestError("codes must be FP8 E4M3 (float8_e4m3fn or uint8 bytes)")
+    if not (a_codes.is_contiguous() and w_codes.is_contiguous() and a_scales.is_contiguous()
+            and w_scales.is_contiguous()):
+        raise QuestError("codes and scales must be contiguous")
+    M, K = a_codes.shape
+    N, K2 = w_codes.shape
+    if K != K2:
+        raise QuestError("a_codes and w_codes disagree on K")
+    if group <= 0 or K % group != 0 or a_scales.numel() != M * (K // group) or w_scales.numel() != N * (K // group):
+        raise QuestError("scales must be [M, K/group] and [N, K/group]")
+    dev = a_codes.device
+    if out is None:
+        out = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+    y32 = torch.empty((M, N), dtype=torch.float32, device=dev) if y_f32 else None
+    w4a4_linear_grouped_raw(a_codes.data_ptr(), a_scales.data_ptr(), w_codes.data_ptr(), w_scales.data_ptr(),
+                            M, N, K, group, out.data_ptr(), y32.data_ptr() if y32 is not None else None,
+                            _stream_handle(stream, dev))
+    return (out, y32) if y_f32 else out
 
 
 def probe_mma_i8(iters, stream=0):

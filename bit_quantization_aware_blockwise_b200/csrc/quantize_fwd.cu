@@ -688,6 +688,7 @@ cudaError_t launch_quantize(const QuantArgs& a, quest_dtype x_dtype, int had_blo
         return launch_quantize_tc(a, had_block, cbits, bits, row_mode, stream);
     if (hs_path_ok(a, had_block, cbits, row_mode))
         return launch_quantize_hs(a, x_dtype, had_block, cbits, bits, row_mode, stream);
+    if (a.c.code_fp8) return cudaErrorNotSupported;   // E4M3 codes only on the two layouts above
     if (tma_path_ok(a, x_dtype, cbits, row_mode)) {
         if (x_dtype == QUEST_BF16) return tma::launch_tma<__nv_bfloat16>(a, bits, had_block, cbits, stream);
         return tma::launch_tma<float>(a, bits, had_block, cbits, stream);

@@ -125,7 +125,7 @@ __device__ __forceinline__ uint4 exchange_halves(const uint32_t (&w)[4], int h) 
 // element index (within its row) of the slab's first element. One pass over
 // the 8 chunks computes each chunk's decisions once and uses them for its
 // codes, mask byte and dequantised values, so a chunk's registers die early.
-template <int PPB, int CB, bool MULT2, bool SAT>
+template <int PPB, int CB, int FMT, bool SAT>
 __device__ __forceinline__ void emit(const QuantArgs& A, const float2 (&P)[32], const GroupK* G,
                                      int64_t row, int64_t e_slab, int h, bool valid) {
     const QuantConsts& k = A.c;
@@ -138,7 +138,7 @@ __device__ __forceinline__ void emit(const QuantArgs& A, const float2 (&P)[32], 
         float2 s[4];
         chunk_decide<SAT, PPB>(P, G, c, k, s);
         if constexpr (CB == 8) {
-            if (valid) *reinterpret_cast<uint2*>(codes + (2 * c + h) * 8) = chunk_pack_i8<MULT2>(s, k);
+            if (valid) *reinterpret_cast<uint2*>(codes + (2 * c + h) * 8) = chunk_pack_i8<FMT>(s, k);
         } else {
             W[c] = chunk_pack<CB>(s, k);
         }
@@ -238,7 +238,7 @@ __device__ __forceinline__ void block_sums(const float2 (&P)[32], float (&ss)[32
     }
 }
 
-template <typename Tin, int HB, int CB, bool MULT2, bool SAT>
+template <typename Tin, int HB, int CB, int FMT, bool SAT>
 __global__ void __launch_bounds__(kThreads, Pipe<Tin>::kMinBlocks) quantize_hs_groups(const QuantArgs A) {
     constexpr int PPB = (HB >= 128 ? 128 : HB) / 4;   // pairs of one block in this lane
     constexpr int BPL = 32 / PPB;
@@ -283,7 +283,7 @@ __global__ void __launch_bounds__(kThreads, Pipe<Tin>::kMinBlocks) quantize_hs_g
             G[b] = make_group(A.c, v);
         }
         // row 0 with a flat offset addresses every dense output
-        emit<PPB, CB, MULT2, SAT>(A, P, G, 0, E, h, valid);
+        emit<PPB, CB, FMT, SAT>(A, P, G, 0, E, h, valid);
         if (valid) {
             float* sp = A.scales + E / HB;   // scales are dense [rows, cols / HB]
             if constexpr (HB == 256) {
@@ -300,7 +300,7 @@ __global__ void __launch_bounds__(kThreads, Pipe<Tin>::kMinBlocks) quantize_hs_g
     }
 }
 
-template <typename Tin, int HB, int CB, bool MULT2, bool SAT>
+template <typename Tin, int HB, int CB, int FMT, bool SAT>
 __global__ void __launch_bounds__(kThreads, Pipe<Tin>::kMinBlocks) quantize_hs_rows(const QuantArgs A, int spr) {
     constexpr int PPB = (HB >= 128 ? 128 : HB) / 4;
     constexpr int BPL = 32 / PPB;
@@ -343,26 +343,26 @@ __global__ void __launch_bounds__(kThreads, Pipe<Tin>::kMinBlocks) quantize_hs_r
         G[0] = make_group(A.c, v);
 #pragma unroll
         for (int b = 1; b < BPL; ++b) G[b] = G[0];
-        emit<PPB, CB, MULT2, SAT>(A, P, G, row, int64_t(sc) * 128, h, valid);
+        emit<PPB, CB, FMT, SAT>(A, P, G, row, int64_t(sc) * 128, h, valid);
         if (valid && sc == 0 && h == 0) A.scales[row] = G[0].delta;
     }
 }
 
-template <typename Tin, int HB, int CB, bool MULT2, bool SAT>
+template <typename Tin, int HB, int CB, int FMT, bool SAT>
 cudaError_t launch_t(const QuantArgs& a, bool row_mode, cudaStream_t s) {
     const int sms = sm_count();
     if (row_mode) {
         const int spr = (int)(a.cols / 128);
         const int rpw = 16 / spr;
         const int64_t warps = (a.rows + rpw - 1) / rpw;
-        auto fn = quantize_hs_rows<Tin, HB, CB, MULT2, SAT>;
+        auto fn = quantize_hs_rows<Tin, HB, CB, FMT, SAT>;
         const int64_t cap = int64_t(sms) * max_ctas_per_sm((const void*)fn, kThreads, 0);
         const int64_t want = (warps + kThreads / 32 - 1) / (kThreads / 32);
         fn<<<(int)(want < cap ? want : cap), kThreads, 0, s>>>(a, spr);
     } else {
         const int64_t slabs = a.rows * (a.cols / 128);
         const int64_t warps = (slabs + 15) / 16;
-        auto fn = quantize_hs_groups<Tin, HB, CB, MULT2, SAT>;
+        auto fn = quantize_hs_groups<Tin, HB, CB, FMT, SAT>;
         const int64_t cap = int64_t(sms) * max_ctas_per_sm((const void*)fn, kThreads, 0);
         const int64_t want = (warps + kThreads / 32 - 1) / (kThreads / 32);
         fn<<<(int)(want < cap ? want : cap), kThreads, 0, s>>>(a);
@@ -370,20 +370,22 @@ cudaError_t launch_t(const QuantArgs& a, bool row_mode, cudaStream_t s) {
     return cudaGetLastError();
 }
 
-template <typename Tin, int HB, int CB, bool MULT2>
+template <typename Tin, int HB, int CB, int FMT>
 cudaError_t launch_sat(const QuantArgs& a, int bits, bool row, cudaStream_t s) {
-    return bits <= 6 ? launch_t<Tin, HB, CB, MULT2, true>(a, row, s)
-                     : launch_t<Tin, HB, CB, MULT2, false>(a, row, s);
+    if constexpr (FMT == 2) return launch_t<Tin, HB, CB, FMT, true>(a, row, s);   // E4M3 codes: b <= 4
+    else return bits <= 6 ? launch_t<Tin, HB, CB, FMT, true>(a, row, s)
+                          : launch_t<Tin, HB, CB, FMT, false>(a, row, s);
 }
 
 template <typename Tin, int HB>
 cudaError_t launch_hb(const QuantArgs& a, int bits, int cb, bool row, cudaStream_t s) {
     switch (cb) {
-        case 1: return launch_sat<Tin, HB, 1, false>(a, bits, row, s);
-        case 2: return launch_sat<Tin, HB, 2, false>(a, bits, row, s);
-        case 4: return launch_sat<Tin, HB, 4, false>(a, bits, row, s);
-        case 8: return a.c.pack2_mult == 2 ? launch_sat<Tin, HB, 8, true>(a, bits, row, s)
-                                           : launch_sat<Tin, HB, 8, false>(a, bits, row, s);
+        case 1: return launch_sat<Tin, HB, 1, 0>(a, bits, row, s);
+        case 2: return launch_sat<Tin, HB, 2, 0>(a, bits, row, s);
+        case 4: return launch_sat<Tin, HB, 4, 0>(a, bits, row, s);
+        case 8: return a.c.code_fp8 ? launch_sat<Tin, HB, 8, 2>(a, bits, row, s)
+                                    : a.c.pack2_mult == 2 ? launch_sat<Tin, HB, 8, 1>(a, bits, row, s)
+                                                          : launch_sat<Tin, HB, 8, 0>(a, bits, row, s);
     }
     return cudaErrorInvalidValue;
 }

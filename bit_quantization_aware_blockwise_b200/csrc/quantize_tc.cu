@@ -46,7 +46,7 @@ __device__ __forceinline__ void lane_sums(const float2 (&P)[16], float (&ss)[Blk
 
 // Quantise and store this lane's 32 values: chunks c = t + 4f of the slab whose
 // first element is `e_slab` in row `row`.
-template <int PPB, int CB, bool MULT2, bool SAT>
+template <int PPB, int CB, int FMT, bool SAT>
 __device__ __forceinline__ void emit(const QuantArgs& A, const float2 (&P)[16], const GroupK* G, int64_t row,
                                      int64_t e_slab, int t, bool valid) {
     const QuantConsts& k = A.c;
@@ -59,7 +59,7 @@ __device__ __forceinline__ void emit(const QuantArgs& A, const float2 (&P)[16], 
         float2 s[4];
         chunk_decide<SAT, PPB>(P, G, f, k, s);
         if constexpr (CB == 8) {
-            if (valid) *reinterpret_cast<uint2*>(codes + 8 * c) = chunk_pack_i8<MULT2>(s, k);
+            if (valid) *reinterpret_cast<uint2*>(codes + 8 * c) = chunk_pack_i8<FMT>(s, k);
         } else if constexpr (CB == 4) {
             if (valid) *reinterpret_cast<uint32_t*>(codes + 4 * c) = chunk_pack<4>(s, k);
         } else if constexpr (CB == 2) {
@@ -125,7 +125,7 @@ __device__ __forceinline__ void emit(const QuantArgs& A, const float2 (&P)[16], 
 
 
 // Everything after the MMA for one slab of the group-RMS kernel.
-template <int HB, int CB, bool MULT2, bool SAT>
+template <int HB, int CB, int FMT, bool SAT>
 __device__ __forceinline__ void group_slab(const QuantArgs& A, float2 (&P)[16], int64_t slab, bool valid,
                                            int lane) {
     constexpr int NBL = Blk<HB>::NBL, PPB = Blk<HB>::PPB;
@@ -142,7 +142,7 @@ __device__ __forceinline__ void group_slab(const QuantArgs& A, float2 (&P)[16], 
         G[b] = make_group(A.c, v);
     }
     const int64_t E = slab * 128;   // dense outputs: row 0 with a flat offset
-    emit<PPB, CB, MULT2, SAT>(A, P, G, 0, E, t, valid);
+    emit<PPB, CB, FMT, SAT>(A, P, G, 0, E, t, valid);
     if (valid) {
         float* sp = A.scales + E / HB;
         if constexpr (HB == 256) {
@@ -166,7 +166,7 @@ __device__ __forceinline__ void group_slab(const QuantArgs& A, float2 (&P)[16], 
 // flight costs more in registers, and so in resident warps, than it hides).
 constexpr int kDepth = 1;
 
-template <int HB, int CB, bool MULT2, bool SAT>
+template <int HB, int CB, int FMT, bool SAT>
 __global__ void __launch_bounds__(kThreads) quantize_tc_groups(const QuantArgs A) {
     const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
     const int64_t spr = A.cols / 128;
@@ -198,14 +198,14 @@ __global__ void __launch_bounds__(kThreads) quantize_tc_groups(const QuantArgs A
             const int64_t next = slab + kDepth * step;
             if (next < total) load_slab(src_of(next), t, raw[d]);
             else zero4(raw[d]);
-            group_slab<HB, CB, MULT2, SAT>(A, P, slab, slab < total, lane);
+            group_slab<HB, CB, FMT, SAT>(A, P, slab, slab < total, lane);
         }
     }
 }
 
 // One RMS over each row of spr slabs. SUB = slabs per lane group (spr / 8 when
 // spr >= 8, so a warp holds a whole row); for spr < 8 a warp step covers 8 / spr rows.
-template <int HB, int CB, bool MULT2, bool SAT, int SUB>
+template <int HB, int CB, int FMT, bool SAT, int SUB>
 __global__ void __launch_bounds__(kThreads, 4) quantize_tc_rows(const QuantArgs A, int spr) {
     constexpr int NBL = Blk<HB>::NBL, PPB = Blk<HB>::PPB;
     const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
@@ -249,12 +249,12 @@ __global__ void __launch_bounds__(kThreads, 4) quantize_tc_rows(const QuantArgs 
         for (int b = 1; b < NBL; ++b) G[b] = G[0];
 #pragma unroll
         for (int u = 0; u < SUB; ++u)
-            emit<PPB, CB, MULT2, SAT>(A, P[u], G, row, int64_t(sc0 + 8 * u) * 128, t, valid);
+            emit<PPB, CB, FMT, SAT>(A, P[u], G, row, int64_t(sc0 + 8 * u) * 128, t, valid);
         if (valid && sc0 == 0 && t == 0) A.scales[row] = G[0].delta;
     }
 }
 
-template <int HB, int CB, bool MULT2, bool SAT>
+template <int HB, int CB, int FMT, bool SAT>
 cudaError_t launch_t(const QuantArgs& a, bool row_mode, cudaStream_t s) {
     const int sms = sm_count();
     if (row_mode) {
@@ -265,13 +265,13 @@ cudaError_t launch_t(const QuantArgs& a, bool row_mode, cudaStream_t s) {
             const int64_t want = (warps + kThreads / 32 - 1) / (kThreads / 32);
             fn<<<(int)(want < cap ? want : cap), kThreads, 0, s>>>(a, spr);
         };
-        if (spr == 16) go(quantize_tc_rows<HB, CB, MULT2, SAT, 2>, 1);
-        else if (spr == 8) go(quantize_tc_rows<HB, CB, MULT2, SAT, 1>, 1);
-        else go(quantize_tc_rows<HB, CB, MULT2, SAT, 1>, 8 / spr);
+        if (spr == 16) go(quantize_tc_rows<HB, CB, FMT, SAT, 2>, 1);
+        else if (spr == 8) go(quantize_tc_rows<HB, CB, FMT, SAT, 1>, 1);
+        else go(quantize_tc_rows<HB, CB, FMT, SAT, 1>, 8 / spr);
     } else {
         const int64_t slabs = a.rows * (a.cols / 128);
         const int64_t warps = (slabs + 7) / 8;
-        auto fn = quantize_tc_groups<HB, CB, MULT2, SAT>;
+        auto fn = quantize_tc_groups<HB, CB, FMT, SAT>;
         const int64_t cap = int64_t(sms) * max_ctas_per_sm((const void*)fn, kThreads, 0);
         const int64_t want = (warps + kThreads / 32 - 1) / (kThreads / 32);
         fn<<<(int)(want < cap ? want : cap), kThreads, 0, s>>>(a);
@@ -279,19 +279,21 @@ cudaError_t launch_t(const QuantArgs& a, bool row_mode, cudaStream_t s) {
     return cudaGetLastError();
 }
 
-template <int HB, int CB, bool MULT2>
+template <int HB, int CB, int FMT>
 cudaError_t launch_sat(const QuantArgs& a, int bits, bool row, cudaStream_t s) {
-    return bits <= 6 ? launch_t<HB, CB, MULT2, true>(a, row, s) : launch_t<HB, CB, MULT2, false>(a, row, s);
+    if constexpr (FMT == 2) return launch_t<HB, CB, FMT, true>(a, row, s);   // E4M3 codes: b <= 4
+    else return bits <= 6 ? launch_t<HB, CB, FMT, true>(a, row, s) : launch_t<HB, CB, FMT, false>(a, row, s);
 }
 
 template <int HB>
 cudaError_t launch_hb(const QuantArgs& a, int bits, int cb, bool row, cudaStream_t s) {
     switch (cb) {
-        case 1: return launch_sat<HB, 1, false>(a, bits, row, s);
-        case 2: return launch_sat<HB, 2, false>(a, bits, row, s);
-        case 4: return launch_sat<HB, 4, false>(a, bits, row, s);
-        case 8: return a.c.pack2_mult == 2 ? launch_sat<HB, 8, true>(a, bits, row, s)
-                                           : launch_sat<HB, 8, false>(a, bits, row, s);
+        case 1: return launch_sat<HB, 1, 0>(a, bits, row, s);
+        case 2: return launch_sat<HB, 2, 0>(a, bits, row, s);
+        case 4: return launch_sat<HB, 4, 0>(a, bits, row, s);
+        case 8: return a.c.code_fp8 ? launch_sat<HB, 8, 2>(a, bits, row, s)
+                                    : a.c.pack2_mult == 2 ? launch_sat<HB, 8, 1>(a, bits, row, s)
+                                                          : launch_sat<HB, 8, 0>(a, bits, row, s);
     }
     return cudaErrorInvalidValue;
 }

@@ -223,7 +223,8 @@ int quest_container_bits(int bits) { return container_bits_of(bits); }
 
 size_t quest_codes_bytes(int64_t rows, int64_t cols, int bits, quest_code_mode mode) {
     if (rows < 0 || cols <= 0 || bits < 1 || bits > 8) return 0;
-    if (mode != QUEST_CODES_PACKED && mode != QUEST_CODES_INT8 && mode != QUEST_CODES_GEMM_OPERAND)
+    if (mode != QUEST_CODES_PACKED && mode != QUEST_CODES_INT8 && mode != QUEST_CODES_GEMM_OPERAND &&
+        mode != QUEST_CODES_GEMM_OPERAND_E4M3)
         return 0;
     const int cb = code_bits(bits, mode);
     if ((cols * cb) % 8 != 0) return 0;
@@ -268,10 +269,13 @@ quest_status quest_quantize_fwd(const void* x, quest_dtype x_dtype, int64_t rows
     if (row_mode && cols > row_mode_max_cols(had_block))
         return fail(QUEST_EUNSUPPORTED, "rms_group == cols supports at most 16384 columns (8192 for had_block 16)");
     if (!(trust > 0.0f) || isinf(trust)) return fail(QUEST_EINVAL, "trust must be finite and > 0");
-    if (code_mode != QUEST_CODES_PACKED && code_mode != QUEST_CODES_INT8 && code_mode != QUEST_CODES_GEMM_OPERAND)
+    if (code_mode != QUEST_CODES_PACKED && code_mode != QUEST_CODES_INT8 && code_mode != QUEST_CODES_GEMM_OPERAND &&
+        code_mode != QUEST_CODES_GEMM_OPERAND_E4M3)
         return fail(QUEST_EINVAL, "invalid code_mode");
     if (code_mode == QUEST_CODES_GEMM_OPERAND && bits > 7)
         return fail(QUEST_EINVAL, "the GEMM operand form c = 2q+1 needs bits <= 7 to fit int8");
+    if (code_mode == QUEST_CODES_GEMM_OPERAND_E4M3 && bits > 4)
+        return fail(QUEST_EINVAL, "the E4M3 operand form holds c = 2q+1 exactly only for bits <= 4");
     if (mask && mask_mode != QUEST_MASK_BITS && mask_mode != QUEST_MASK_BYTES)
         return fail(QUEST_EINVAL, "invalid mask_mode");
     if (dequant && dequant_dtype != QUEST_BF16 && dequant_dtype != QUEST_FP32)
@@ -330,7 +334,9 @@ quest_status quest_quantize_fwd(const void* x, quest_dtype x_dtype, int64_t rows
     c.s_mid = kMagic + (float)ldexp(1.0, bits - 1);
     c.s_top = kMagic + (float)(ldexp(1.0, bits) - 1.0);
     c.cell_center = (float)(0.5 - ldexp(1.0, bits - 1));
-    pack_constants_biased(cb, bits, code_mode, &c.pack2_mult, &c.pack2_add, &c.pack2_xor);
+    pack_constants_biased(cb, bits, code_mode == QUEST_CODES_GEMM_OPERAND_E4M3 ? QUEST_CODES_GEMM_OPERAND : code_mode,
+                          &c.pack2_mult, &c.pack2_add, &c.pack2_xor);
+    c.code_fp8 = code_mode == QUEST_CODES_GEMM_OPERAND_E4M3;
     {   // an 8-field word (one chunk of 8 elements) for cb <= 4
         const uint32_t rep8 = cb == 1 ? 0xFFu : (cb == 2 ? 0x5555u : 0x11111111u);
         const uint32_t x8 = cb == 1 ? 0xFFu : (cb == 2 ? 0xAAAAu : 0x88888888u);
@@ -343,6 +349,9 @@ quest_status quest_quantize_fwd(const void* x, quest_dtype x_dtype, int64_t rows
     c.deq_mode = dequant ? (int)dequant_dtype : -1;
 
     cudaError_t e = launch_quantize(a, x_dtype, had_block, cb, bits, row_mode, static_cast<cudaStream_t>(stream));
+    if (e == cudaErrorNotSupported)
+        return fail(QUEST_EUNSUPPORTED, "the E4M3 operand form needs rows of whole 128-value slabs, 8-byte aligned "
+                                        "codes and at most 16 slabs per row in row-RMS mode");
     if (e != cudaSuccess) return cuda_fail(e, "quest_quantize_fwd launch");
     return QUEST_OK;
 }
@@ -402,6 +411,36 @@ quest_status quest_w4a4_linear(const int8_t* a_codes, const float* a_scales,
                                 static_cast<uint16_t*>(y), acc, static_cast<cudaStream_t>(stream));
     if (e == cudaErrorInvalidValue) return fail(QUEST_ECUDA, "quest_w4a4_linear: tensor map encoding failed");
     if (e != cudaSuccess) return cuda_fail(e, "quest_w4a4_linear launch");
+    return QUEST_OK;
+}
+
+quest_status quest_w4a4_linear_grouped(const uint8_t* a_codes, const float* a_scales,
+                                       const uint8_t* w_codes, const float* w_scales, int64_t M,
+                                       int64_t N, int64_t K, int64_t group, void* y, float* y_f32,
+                                       void* stream) {
+    g_last_error.clear();
+    if (M < 0 || N < 0 || K < 0) return fail(QUEST_EINVAL, "M, N and K must be >= 0");
+    if (M >= (int64_t(1) << 31) || N >= (int64_t(1) << 31)) return fail(QUEST_EINVAL, "M and N must be < 2^31");
+    if (group != 128) return fail(QUEST_EUNSUPPORTED, "quest_w4a4_linear_grouped: group must be 128");
+    if (K % group != 0) return fail(QUEST_EINVAL, "K must be a multiple of the group");
+    if (K >= (int64_t(1) << 24)) return fail(QUEST_EINVAL, "K must be < 2^24");
+    if (N % 8 != 0) return fail(QUEST_EINVAL, "N must be a multiple of 8");
+    if (M > 0 && N > 0) {
+        if (!y) return fail(QUEST_EINVAL, "y must be non-NULL");
+        if (K > 0 && (!a_codes || !w_codes || !a_scales || !w_scales))
+            return fail(QUEST_EINVAL, "codes and scales must be non-NULL");
+        if (K > 0 && (!aligned(a_codes, 16) || !aligned(w_codes, 16)))
+            return fail(QUEST_EINVAL, "codes must be 16-byte aligned");
+        if (!aligned(y, 16)) return fail(QUEST_EINVAL, "y must be 16-byte aligned");
+        if ((a_scales && !aligned(a_scales, 4)) || (w_scales && !aligned(w_scales, 4)) ||
+            (y_f32 && !aligned(y_f32, 4)))
+            return fail(QUEST_EINVAL, "scales and y_f32 must be 4-byte aligned");
+    }
+    cudaError_t e = launch_w4a4_grouped(reinterpret_cast<const int8_t*>(a_codes), a_scales,
+                                        reinterpret_cast<const int8_t*>(w_codes), w_scales, M, N, K,
+                                        static_cast<uint16_t*>(y), y_f32, static_cast<cudaStream_t>(stream));
+    if (e == cudaErrorInvalidValue) return fail(QUEST_ECUDA, "quest_w4a4_linear_grouped: tensor map encoding failed");
+    if (e != cudaSuccess) return cuda_fail(e, "quest_w4a4_linear_grouped launch");
     return QUEST_OK;
 }
 

@@ -5,6 +5,7 @@
 // the packing constants in quest_api.cu).
 #pragma once
 
+#include <cuda_fp8.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -152,17 +153,32 @@ __device__ __forceinline__ uint32_t chunk_pack(const float2 (&s)[4], const Quant
     return ((acc + k.pack8_add) ^ k.pack8_xor) & (CB == 4 ? 0xFFFFFFFFu : ((1u << (8 * CB)) - 1u));
 }
 
-// The 8 one-byte codes of a chunk as two 32-bit words (pack2_* constants).
-template <bool MULT2>
+// The 8 one-byte codes of a chunk as two 32-bit words. FMT 0: q and 1: c = 2q + 1
+// as int8 (pack2_* constants); FMT 2: c as FP8 E4M3 (exact for |c| <= 15).
+template <int FMT>
 __device__ __forceinline__ uint2 chunk_pack_i8(const float2 (&s)[4], const QuantConsts& k) {
-    constexpr uint32_t m = MULT2 ? 2u : 1u;
     uint32_t w[2];
+    if constexpr (FMT == 2) {
+        uint32_t h[4];
 #pragma unroll
-    for (int u = 0; u < 2; ++u) {
-        const uint32_t acc = __float_as_uint(s[2 * u].x) * m + __float_as_uint(s[2 * u].y) * (m << 8) +
-                             __float_as_uint(s[2 * u + 1].x) * (m << 16) +
-                             __float_as_uint(s[2 * u + 1].y) * (m << 24);
-        w[u] = (acc + k.pack2_add) ^ k.pack2_xor;
+        for (int p = 0; p < 4; ++p) {
+            // q_b = s - 1.5*2^23 exactly; c = 2 (q_b + 1/2 - 2^(b-1))
+            const float2 qb = __fadd2_rn(s[p], make_float2(-kMagic, -kMagic));
+            const float2 c = __ffma2_rn(qb, make_float2(2.0f, 2.0f),
+                                        make_float2(2.0f * k.cell_center, 2.0f * k.cell_center));
+            h[p] = __nv_cvt_float2_to_fp8x2(c, __NV_SATFINITE, __NV_E4M3);
+        }
+        w[0] = h[0] | (h[1] << 16);
+        w[1] = h[2] | (h[3] << 16);
+    } else {
+        constexpr uint32_t m = FMT == 1 ? 2u : 1u;
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+            const uint32_t acc = __float_as_uint(s[2 * u].x) * m + __float_as_uint(s[2 * u].y) * (m << 8) +
+                                 __float_as_uint(s[2 * u + 1].x) * (m << 16) +
+                                 __float_as_uint(s[2 * u + 1].y) * (m << 24);
+            w[u] = (acc + k.pack2_add) ^ k.pack2_xor;
+        }
     }
     return make_uint2(w[0], w[1]);
 }

@@ -35,6 +35,7 @@ struct QuantConsts {
     uint32_t pack2_mult, pack2_add, pack2_xor;   // 32-bit words of 32/cb fields
     uint32_t pack8_add, pack8_xor;                // words of 8 fields (cb <= 4)
     int trust_ge1;      // 1: use m = [|t| <= edge]
+    int code_fp8;       // operand codes c = 2q + 1 stored as FP8 E4M3
     int mask_mode;      // -1 none, 0 bits, 1 bytes
     int deq_mode;       // -1 none, 0 bf16, 1 fp32
 };
@@ -86,6 +87,9 @@ cudaError_t launch_w4a4(const int8_t* A, const float* sa, const int8_t* B, const
 // Reads (synchronising `stream`) and clears the integer linear layer's device
 // status word; returns its value (0 or a quest_status).
 int read_and_clear_gemm_status(cudaStream_t stream, cudaError_t* err);
+cudaError_t launch_w4a4_grouped(const int8_t* A, const float* sa, const int8_t* B, const float* sb,
+                                int64_t M, int64_t N, int64_t K, uint16_t* y, float* y32,
+                                cudaStream_t stream);
 
 // Number of SMs and max resident CTAs of `func` per SM on the current device.
 int sm_count();

@@ -59,11 +59,21 @@ typedef enum quest_dtype {
  *   QUEST_CODES_INT8          one int8 per element holding q.
  *   QUEST_CODES_GEMM_OPERAND  one int8 per element holding c = 2q + 1 (odd,
  *                             |c| <= 2^b - 1), the exact integer form of the
- *                             midrise level (q + 1/2); requires b <= 7. */
+ *                             midrise level (q + 1/2); requires b <= 7.
+ *   QUEST_CODES_GEMM_OPERAND_E4M3
+ *                             one byte per element holding the same c in the
+ *                             OCP FP8 E4M3 format (sign, 4-bit exponent with
+ *                             bias 7, 3-bit mantissa), exact for |c| <= 15:
+ *                             requires b <= 4. It is the operand of
+ *                             quest_w4a4_linear_grouped. Supported where the
+ *                             rows are whole 128-value slabs with 8-byte aligned
+ *                             codes and at most 16 slabs per row in row-RMS mode
+ *                             (QUEST_EUNSUPPORTED otherwise). */
 typedef enum quest_code_mode {
     QUEST_CODES_PACKED = 0,
     QUEST_CODES_INT8 = 1,
-    QUEST_CODES_GEMM_OPERAND = 2
+    QUEST_CODES_GEMM_OPERAND = 2,
+    QUEST_CODES_GEMM_OPERAND_E4M3 = 3
 } quest_code_mode;
 
 /* How the trust mask is stored (1 = gradient kept, 0 = gradient zeroed).
@@ -173,6 +183,40 @@ quest_status quest_trust_bwd(const void* grad_out, const void* mask, quest_mask_
 quest_status quest_w4a4_linear(const int8_t* a_codes, const float* a_scales,
                                const int8_t* w_codes, const float* w_scales, int64_t M,
                                int64_t N, int64_t K, void* y, int32_t* acc, void* stream);
+
+/*
+ * quest_w4a4_linear_grouped -- linear layer on QuEST codes with one scale per
+ * row and per group of 128 consecutive K indices on both operands (the codes of
+ * a quantize_fwd call with rms_group = had_block = 128 in the
+ * QUEST_CODES_GEMM_OPERAND_E4M3 form).
+ *
+ * Same layer as quest_w4a4_linear (pith.science review, "Assumptions & free
+ * parameters": a Hadamard transform applied to both operands leaves the product
+ * unchanged), with the scales varying along K, so each group's exact integer
+ * product is scaled on its own:
+ *     acc_g[m][n] = sum over k in group g of a_codes[m][k] * w_codes[n][k]
+ *     y[m][n]     = bf16_rne( sum_g (a_scales[m][g]/2) (w_scales[n][g]/2) acc_g[m][n] )
+ * acc_g is exact (FP8 E4M3 tensor-core products accumulated in fp32) whenever
+ * every partial sum is an integer below 2^24 in magnitude, which holds for
+ * codes c = 2q + 1 with |c| <= 15; the group sum runs in fp32 (its rounding
+ * error is below 1e-6 of sum_g |term_g|); the pages do not fix this precision.
+ *
+ * Arguments
+ *   a_codes    device, FP8 E4M3 bytes [M, K] row-major; 16-byte aligned.
+ *   a_scales   device, fp32 [M, K / group] row-major.
+ *   w_codes    device, FP8 E4M3 bytes [N, K] row-major; 16-byte aligned.
+ *   w_scales   device, fp32 [N, K / group] row-major.
+ *   M >= 0, N >= 0 (0 = no-op); N a multiple of 8; K >= 0, a multiple of
+ *   `group`, K < 2^24.
+ *   group      must be 128 (QUEST_EUNSUPPORTED otherwise).
+ *   y          device, bf16 [M, N]; 16-byte aligned.
+ *   y_f32      device, optional fp32 [M, N] copy of y before the bf16 rounding
+ *              (NULL = not written); meant for exactness checks.
+ */
+quest_status quest_w4a4_linear_grouped(const uint8_t* a_codes, const float* a_scales,
+                                       const uint8_t* w_codes, const float* w_scales, int64_t M,
+                                       int64_t N, int64_t K, int64_t group, void* y, float* y_f32,
+                                       void* stream);
 
 /*
  * quest_device_status -- synchronises `stream`, then reports (and clears) the

@@ -15,10 +15,37 @@ EXEMPT_REL = 1e-5
 FLOAT_REL = 2e-3
 
 
+def e4m3_decode(raw):
+    """Value of OCP FP8 E4M3 bytes by the format's definition: sign, 4-bit exponent
+    with bias 7 (0 = subnormal), 3-bit mantissa; 0x7F / 0xFF are NaN."""
+    b = np.asarray(raw, dtype=np.uint8).astype(np.int64)
+    sign = np.where(b >> 7, -1.0, 1.0)
+    e = (b >> 3) & 15
+    m = (b & 7).astype(np.float64)
+    v = np.where(e == 0, m / 8.0 * 2.0 ** -6, (1.0 + m / 8.0) * np.exp2(e - 7.0))
+    v = np.where((e == 15) & ((b & 7) == 7), np.nan, v)
+    return sign * v
+
+
+def e4m3_encode_int(c):
+    """E4M3 bytes of integers exactly representable in the format (|c| <= 15 here)."""
+    c = np.asarray(c, dtype=np.int64)
+    a = np.abs(c)
+    assert np.all(a <= 15)
+    e = np.where(a > 0, np.floor(np.log2(np.maximum(a, 1))).astype(np.int64), 0)
+    m = np.where(a > 0, (a * 8) // (1 << e) - 8, 0)
+    byte = np.where(a > 0, ((e + 7) << 3) | m, 0) | np.where(c < 0, 0x80, 0)
+    return byte.astype(np.uint8)
+
+
 def unpack_codes(raw, rows, cols, bits, mode):
     """Decode the library's code buffer into int codes [rows, cols] (q, or c=2q+1 for
-    the GEMM operand form)."""
+    the GEMM operand forms)."""
     raw = np.asarray(raw, dtype=np.uint8).reshape(-1)
+    if mode == 3:  # E4M3 operand form
+        v = e4m3_decode(raw[: rows * cols]).reshape(rows, cols)
+        assert np.all(v == np.round(v)), "E4M3 operand codes must be integers"
+        return v.astype(np.int32)
     if mode in (1, 2):  # int8 forms
         return raw[: rows * cols].view(np.int8).reshape(rows, cols).astype(np.int32)
     cb = [0, 1, 2, 4, 4, 8, 8, 8, 8][bits]

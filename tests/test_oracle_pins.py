@@ -461,3 +461,18 @@ def test_grouped_linear_groups_are_independent():
     a_cut[:, 256:384] = 0
     y_cut, _ = oracle.linear_grouped(a_cut, b, sa, sb)
     assert np.allclose(y0, y_cut, rtol=1e-14, atol=0)
+
+
+def test_e4m3_helpers_match_torch():
+    # the test-side E4M3 codec against torch's float8_e4m3fn conversion
+    import sys, os
+    sys.path.insert(0, os.path.dirname(__file__))
+    from parity import e4m3_decode, e4m3_encode_int
+    c = np.arange(-15, 16)
+    ref = torch.tensor(c, dtype=torch.float32).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    assert np.array_equal(e4m3_encode_int(c), ref)
+    allb = np.arange(256, dtype=np.uint8)
+    tv = torch.from_numpy(allb).view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    dv = e4m3_decode(allb)
+    assert np.array_equal(np.isnan(tv), np.isnan(dv))
+    assert np.array_equal(tv[~np.isnan(tv)], dv[~np.isnan(dv)])

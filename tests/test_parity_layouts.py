@@ -12,6 +12,7 @@ import pytest
 import oracle
 import bit_quantization_aware_blockwise_b200 as q
 from bit_quantization_aware_blockwise_b200 import inputs
+from parity import check_codes_operand
 from test_parity_quantize import check_all, run_gpu
 
 pytestmark = pytest.mark.gpu
@@ -54,3 +55,21 @@ def test_row_rms_all_slab_counts(cuda_device, dtype, had, spr):
     o = oracle.quantize(inputs.to_f64(x), bits=2, had=had, rms_group=cols, trust=0.7)
     res = run_gpu(x, 2, had=had, rms_group=cols, trust=0.7, mask_mode=q.MASK_BYTES, dequant="fp32")
     check_all(res, o, 2)
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "fp32"])
+@pytest.mark.parametrize("bits", [1, 2, 3, 4])
+@pytest.mark.parametrize("rms", ["group", "row"])
+def test_e4m3_operand_codes(cuda_device, dtype, bits, rms):
+    # c = 2q + 1 stored as FP8 E4M3 (the grouped linear layer's operand)
+    x = inputs.activations(45, 1024, seed=bits, dtype=dtype)
+    rg = 128 if rms == "group" else 1024
+    o = oracle.quantize(inputs.to_f64(x), bits=bits, had=128, rms_group=rg)
+    res = run_gpu(x, bits, rms_group=rg, code_mode=q.CODES_GEMM_OPERAND_E4M3, mask_mode=None, dequant=None)
+    check_codes_operand(res["codes"], o)
+
+
+def test_e4m3_operand_codes_reject_wide_codes(cuda_device):
+    x = inputs.activations(4, 256, seed=1).to("cuda")
+    with pytest.raises(q.QuestError):
+        q.quantize_fwd(x, 5, code_mode=q.CODES_GEMM_OPERAND_E4M3, mask_mode=None)
