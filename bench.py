@@ -726,11 +726,15 @@ def run_profile_kernels(args):
     gi = q.trust_bwd(g, out["mask"])                                                   # 2
     op = q.quantize_fwd(x, BITS, rms_group=C, code_mode=q.CODES_GEMM_OPERAND, mask_mode=None)  # 3
     y = q.w4a4_linear(a, sa, b, sb)                                                    # 4
+    a8, b8 = a.float().to(torch.float8_e4m3fn), b.float().to(torch.float8_e4m3fn)
+    sag = sa[:, None].repeat(1, C // HB).contiguous()
+    sbg = sb[:, None].repeat(1, C // HB).contiguous()
+    yg = q.w4a4_linear_grouped(a8, sag, b8, sbg)                                       # 5
     torch.cuda.synchronize()
     q.device_status()
     print(json.dumps({"profile_kernels": "ok", "rows": rows, "checksum": [
         float(out["scales"].sum()), float(gi.float().abs().sum()), float(op["scales"].sum()),
-        float(y.float().abs().sum())]}))
+        float(y.float().abs().sum()), float(yg.float().abs().sum())]}))
 
 
 def main():

@@ -724,9 +724,9 @@ constexpr uint32_t kGStageA = 128 * BK, kGStageB = (kGBN / 2) * BK;   // per CTA
 constexpr uint32_t kGTxBytes = 2 * (kGStageA + kGStageB);
 constexpr uint32_t kGSmemA = 0;
 constexpr uint32_t kGSmemB = kGSmemA + kGStages * kGStageA;
-constexpr uint32_t kGSmemSW = kGSmemB + kGStages * kGStageB;          // float [16][128]
-constexpr uint32_t kGSmemSX = kGSmemSW + kGScaleBlock * kGBN * 4;     // float [16][128]
-constexpr uint32_t kGSmemC = kGSmemSX + kGScaleBlock * 128 * 4;       // 8 warps x 2 x 2 KB
+constexpr uint32_t kGScaleBytes = kGScaleBlock * (kGBN + 128) * 4;    // one block: sb [16][128], sa [16][128]
+constexpr uint32_t kGSmemS = kGSmemB + kGStages * kGStageB;           // two blocks (double buffer)
+constexpr uint32_t kGSmemC = kGSmemS + 2 * kGScaleBytes;              // 8 warps x 2 x 2 KB
 constexpr uint32_t kGCBytes = 32 * 32 * 2;                            // 32 rows x 32 bf16
 constexpr uint32_t kGSmemBar = kGSmemC + 8 * 2 * kGCBytes;
 constexpr uint32_t kGNumBars = 2 * kGStages + kGSlots + 1;
@@ -768,6 +768,13 @@ __device__ __forceinline__ bool gepi_any(bool pred) {
     return out != 0;
 }
 
+__device__ __forceinline__ void cp_async4(uint32_t dst, const float* src, bool valid) {
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;" ::"r"(dst), "l"(src), "r"(valid ? 4 : 0)
+                 : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
+
 struct GroupedParams {
     const float* sa;    // [M, K / 128]
     const float* sb;    // [N, K / 128]
@@ -788,8 +795,8 @@ w4a4_gemm_grouped_kernel(const __grid_constant__ CUtensorMap map_a, const __grid
     const uint32_t bar_drain = bar_tempty + 8 * kGSlots;
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + kGSmemAbort);
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kGSmemTmemSlot);
-    float* s_w = reinterpret_cast<float*>(smem + kGSmemSW);      // [16][128]: sb[n0 + n][g] / 2
-    float* s_x = reinterpret_cast<float*>(smem + kGSmemSX);      // [16][128]: sa[m0 + r][g] / 2
+    // scale blocks (double buffer): [16][128] sb[n0 + n][g0 + gg], then [16][128] sa[m0 + r][g0 + gg]
+    float* s_sc = reinterpret_cast<float*>(smem + kGSmemS);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const uint32_t rank = cluster_rank();
@@ -899,9 +906,32 @@ w4a4_gemm_grouped_kernel(const __grid_constant__ CUtensorMap map_a, const __grid
         const uint32_t tempty_even = map_to_rank(bar_tempty, 0);
         const uint32_t stg0 = sbase + kGSmemC + uint32_t(ew) * 2 * kGCBytes;
         const int Gs = p.K / kGroup;                       // scale columns per row
+        // issue the copies of scale block (tile, g0) into buffer b: transposed to [group][column]
+        auto prefetch = [&](int tile, int g0, int b) {
+            if (tile < num_tiles) {
+                const int pm0 = (tile % p.num_m2) * 256 + 128 * int(rank), pn0 = (tile / p.num_m2) * kGBN;
+                const int nb = (G - g0) < kGScaleBlock ? (G - g0) : kGScaleBlock;
+                const uint32_t base = sbase + kGSmemS + uint32_t(b) * kGScaleBytes;
+#pragma unroll
+                for (int k = 0; k < kGScaleBlock * kGBN / kGEpiThreads; ++k) {
+                    const int i = et + k * kGEpiThreads, n = i / kGScaleBlock, gg = i % kGScaleBlock;
+                    const bool v = gg < nb && pn0 + n < p.N;
+                    cp_async4(base + 4 * (gg * kGBN + n), p.sb + (v ? int64_t(pn0 + n) * Gs + g0 + gg : 0), v);
+                }
+#pragma unroll
+                for (int k = 0; k < kGScaleBlock * 128 / kGEpiThreads; ++k) {
+                    const int i = et + k * kGEpiThreads, r = i / kGScaleBlock, gg = i % kGScaleBlock;
+                    const bool v = gg < nb && pm0 + r < p.M;
+                    cp_async4(base + 4 * (kGScaleBlock * kGBN + gg * 128 + r),
+                              p.sa + (v ? int64_t(pm0 + r) * Gs + g0 + gg : 0), v);
+                }
+            }
+            cp_async_commit();
+        };
         uint32_t gcount = 0;
-        int cbuf = 0;
+        int cbuf = 0, sbuf = 0;
         bool aborted = false;
+        prefetch(pair, 0, 0);
         for (int tile = pair; tile < num_tiles && !aborted; tile += num_pairs) {
             const int m0 = (tile % p.num_m2) * 256 + 128 * int(rank), n0 = (tile / p.num_m2) * kGBN;
             float2 acc[32];   // columns 64*half + 2j, +1
@@ -911,31 +941,12 @@ w4a4_gemm_grouped_kernel(const __grid_constant__ CUtensorMap map_a, const __grid
                 if ((g % kGScaleBlock) == 0) {
                     // a thread whose wait gave up stops the whole epilogue here (uniform exit)
                     if (gepi_any(aborted)) break;
-                    // stage the scales of groups g .. g+15, halved (c = 2q + 1 carries a factor 2)
+                    // this block's scales have landed, and every thread is done with the other
+                    // buffer: start copying the next block into it (one tile ahead at most)
+                    cp_async_wait_all();
                     gepi_bar();
-                    const int nb = (G - g) < kGScaleBlock ? (G - g) : kGScaleBlock;
-                    float vw[kGScaleBlock * kGBN / kGEpiThreads], vx[kGScaleBlock * 128 / kGEpiThreads];
-#pragma unroll
-                    for (int k = 0; k < kGScaleBlock * kGBN / kGEpiThreads; ++k) {
-                        const int i = et + k * kGEpiThreads, n = i / kGScaleBlock, gg = i % kGScaleBlock;
-                        vw[k] = (gg < nb && n0 + n < p.N) ? __ldg(p.sb + int64_t(n0 + n) * Gs + g + gg) : 0.0f;
-                    }
-#pragma unroll
-                    for (int k = 0; k < kGScaleBlock * 128 / kGEpiThreads; ++k) {
-                        const int i = et + k * kGEpiThreads, r = i / kGScaleBlock, gg = i % kGScaleBlock;
-                        vx[k] = (gg < nb && m0 + r < p.M) ? __ldg(p.sa + int64_t(m0 + r) * Gs + g + gg) : 0.0f;
-                    }
-#pragma unroll
-                    for (int k = 0; k < kGScaleBlock * kGBN / kGEpiThreads; ++k) {
-                        const int i = et + k * kGEpiThreads;
-                        s_w[(i % kGScaleBlock) * kGBN + i / kGScaleBlock] = vw[k] * 0.5f;
-                    }
-#pragma unroll
-                    for (int k = 0; k < kGScaleBlock * 128 / kGEpiThreads; ++k) {
-                        const int i = et + k * kGEpiThreads;
-                        s_x[(i % kGScaleBlock) * 128 + i / kGScaleBlock] = vx[k] * 0.5f;
-                    }
-                    gepi_bar();
+                    if (g + kGScaleBlock < G) prefetch(tile, g + kGScaleBlock, sbuf ^ 1);
+                    else prefetch(tile + num_pairs, 0, sbuf ^ 1);
                 }
                 // group gcount's MMAs are complete when its stage's empty barrier completes
                 // that use; the epilogue trails the MMA by at most kGSlots < kGStages groups,
@@ -954,8 +965,11 @@ w4a4_gemm_grouped_kernel(const __grid_constant__ CUtensorMap map_a, const __grid
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive_remote(tempty_even + 8 * slot);
-                const float sx = s_x[(g % kGScaleBlock) * 128 + row_in_tile];
-                const float4* sw4 = reinterpret_cast<const float4*>(s_w + (g % kGScaleBlock) * kGBN + 64 * half);
+                // (sa/2)(sb/2): the factor 1/4 rides on the row scale
+                const float* sblk = s_sc + sbuf * (kGScaleBytes / 4);
+                const float sx = 0.25f * sblk[kGScaleBlock * kGBN + (g % kGScaleBlock) * 128 + row_in_tile];
+                const float4* sw4 = reinterpret_cast<const float4*>(sblk + (g % kGScaleBlock) * kGBN + 64 * half);
+                if ((g % kGScaleBlock) == kGScaleBlock - 1 || g == G - 1) sbuf ^= 1;   // next block, other buffer
 #pragma unroll
                 for (int q4 = 0; q4 < 16; ++q4) {
                     const float4 w4 = sw4[q4];
@@ -1009,6 +1023,7 @@ w4a4_gemm_grouped_kernel(const __grid_constant__ CUtensorMap map_a, const __grid
                 cbuf ^= 1;
             }
         }
+        cp_async_wait_all();   // no copy may still target shared memory at exit
         if (lane == 0) bulk_wait_all();
     }
 
