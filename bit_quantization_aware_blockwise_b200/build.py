@@ -17,7 +17,7 @@ CSRC = os.path.join(HERE, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(HERE, "libquest_b200.so")
 SOURCES = ["quest_api.cu", "quantize_fwd.cu", "quantize_hs.cu", "quantize_tc.cu", "trust_bwd.cu", "trust_tc.cu", "w4a4_gemm.cu", "probe_mma.cu"]
-HEADERS = ["quest_device.cuh", "quest_internal.h", "quest_sync.cuh", "quest_emit.cuh", "quest_tc.cuh"]
+HEADERS = ["quest_device.cuh", "quest_internal.h", "quest_emit.cuh", "quest_tc.cuh"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
 

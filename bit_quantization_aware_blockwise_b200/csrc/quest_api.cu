@@ -14,7 +14,6 @@
 #include "quest.h"
 #include "quest_device.cuh"
 #include "quest_internal.h"
-#include "quest_sync.cuh"
 
 namespace quest {
 namespace {
@@ -172,37 +171,6 @@ int max_ctas_per_sm(const void* func, int threads, size_t smem) {
         n = 1;
     g_occ[key] = n;
     return n;
-}
-
-using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
-                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
-                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
-                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-bool encode_tensor_map(CUtensorMap* map, CUtensorMapDataType dt, int rank, const void* base,
-                       const uint64_t* dims, const uint64_t* strides_bytes, const uint32_t* box,
-                       CUtensorMapSwizzle swz) {
-    static EncodeTiledFn fn = nullptr;
-    static std::once_flag once;
-    std::call_once(once, [] {
-        void* p = nullptr;
-        cudaDriverEntryPointQueryResult q;
-        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
-            q == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<EncodeTiledFn>(p);
-    });
-    if (!fn || rank < 1 || rank > 5) return false;
-    cuuint64_t d[5], st[4];
-    cuuint32_t b[5], es[5];
-    for (int i = 0; i < rank; ++i) {
-        d[i] = dims[i];
-        b[i] = box[i];
-        es[i] = 1;
-        if (i + 1 < rank) st[i] = strides_bytes[i];
-    }
-    return fn(map, dt, (cuuint32_t)rank, const_cast<void*>(base), d, st, b, es,
-              CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 }  // namespace quest
@@ -450,10 +418,7 @@ quest_status quest_device_status(void* stream) {
     cudaError_t e = cudaSuccess;
     const int vg = read_and_clear_gemm_status(s, &e);
     if (e != cudaSuccess) return cuda_fail(e, "quest_device_status");
-    const int vq = read_and_clear_quant_status(s, &e);
-    if (e != cudaSuccess) return cuda_fail(e, "quest_device_status");
     if (vg != 0) return fail((quest_status)vg, "a bounded device-side wait in quest_w4a4_linear gave up");
-    if (vq != 0) return fail((quest_status)vq, "a bounded device-side wait in quest_quantize_fwd gave up");
     return QUEST_OK;
 }
 

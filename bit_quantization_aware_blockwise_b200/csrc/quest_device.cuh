@@ -179,41 +179,6 @@ __device__ __forceinline__ float2 f2_sub(float2 a, float2 b) {
     return __ffma2_rn(b, make_float2(-1.0f, -1.0f), a);  // a - b, one rounding
 }
 
-// Unnormalised Walsh-Hadamard transform (Sylvester order) of every HB-block
-// held in the half-slab layout; in place.
-template <int HB>
-__device__ __forceinline__ void fwht_halfslab(float2 (&P)[32], int lane) {
-    static_assert(HB >= 16 && HB <= 256 && (HB & (HB - 1)) == 0, "HB");
-#pragma unroll
-    for (int j = 0; j < 32; ++j) {
-        const float a = P[j].x, b = P[j].y;
-        P[j] = make_float2(a + b, a - b);
-    }
-#pragma unroll
-    for (int h = 1; h < 32 && 2 * h < HB; h <<= 1) {
-#pragma unroll
-        for (int j = 0; j < 32; ++j) {
-            if ((j & h) == 0) {
-                const float2 a = P[j], b = P[j + h];
-                P[j] = __fadd2_rn(a, b);
-                P[j + h] = f2_sub(a, b);
-            }
-        }
-    }
-#pragma unroll
-    for (int s = 1; s < 4 && 64 * s < HB; s <<= 1) {
-        const float sg = (lane & s) ? -1.0f : 1.0f;
-        const float2 sg2 = make_float2(sg, sg);
-#pragma unroll
-        for (int j = 0; j < 32; ++j) {
-            float2 o;
-            o.x = __shfl_xor_sync(0xFFFFFFFFu, P[j].x, s);
-            o.y = __shfl_xor_sync(0xFFFFFFFFu, P[j].y, s);
-            P[j] = __ffma2_rn(P[j], sg2, o);
-        }
-    }
-}
-
 }  // namespace quest
 
 // ---------------------------------------------------------------------------

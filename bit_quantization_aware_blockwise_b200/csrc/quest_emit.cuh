@@ -60,35 +60,6 @@ __device__ __forceinline__ float2 decide(float2 y, const GroupK& g, const QuantC
     }
 }
 
-// Packed code word of the EPW = 32/CB elements in pairs [w*EPW/2, (w+1)*EPW/2)
-// (PPB = pairs per RMS group). The sum is split over independent partial sums of
-// 8 fields so the dependency chains stay short.
-template <int PPB, int CB, bool MULT2, bool SAT>
-__device__ __forceinline__ uint32_t code_word(const float2 (&P)[32], const GroupK* G, int w,
-                                              const QuantConsts& k) {
-    constexpr uint32_t kMult = MULT2 ? 2u : 1u;
-    constexpr int EPW = 32 / CB;
-    constexpr int NSUB = EPW >= 8 ? EPW / 8 : 1;
-    constexpr int PER = EPW / NSUB;
-    uint32_t part[NSUB];
-#pragma unroll
-    for (int u = 0; u < NSUB; ++u) {
-        uint32_t acc = 0;
-#pragma unroll
-        for (int i = u * PER; i < (u + 1) * PER; i += 2) {
-            const int j = (w * EPW + i) / 2;
-            const float2 s2 = decide<SAT>(P[j], G[j / PPB], k);
-            acc += __float_as_uint(s2.x) * (kMult << (CB * i));
-            acc += __float_as_uint(s2.y) * (kMult << (CB * (i + 1)));
-        }
-        part[u] = acc;
-    }
-    uint32_t word = k.pack2_add;
-#pragma unroll
-    for (int u = 0; u < NSUB; ++u) word += part[u];
-    return word ^ k.pack2_xor;
-}
-
 // Trust-mask byte of the 8 elements in pairs [4*byte, 4*byte + 4): bit i = element i.
 // For T >= 1: m = [y^2 <= thr^2], read off the sign of y^2 - thr^2.
 template <int PPB, int N>

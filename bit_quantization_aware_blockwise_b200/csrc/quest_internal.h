@@ -67,7 +67,6 @@ struct TrustArgs {
 // Launchers (return cudaSuccess or the launch error).
 cudaError_t launch_quantize(const QuantArgs& a, quest_dtype x_dtype, int had_block, int cbits,
                             int bits, bool row_mode, cudaStream_t stream);
-int read_and_clear_quant_status(cudaStream_t stream, cudaError_t* err);
 // Direct-load interleaved half-slab quantizer (quantize_hs.cu).
 bool hs_path_ok(const QuantArgs& a, int had_block, int cbits, bool row_mode);
 cudaError_t launch_quantize_hs(const QuantArgs& a, quest_dtype x_dtype, int had_block, int cbits,

@@ -213,7 +213,7 @@ def test_rows_not_multiple_of_128_use_the_direct_kernel(cuda_device, had, cols):
 @pytest.mark.parametrize("bits", [2, 4, 8])
 def test_under_aligned_outputs_use_the_direct_kernel(cuda_device, bits):
     # codes (and mask bits) just past an allocation's start: valid for the ABI, too
-    # little alignment for the staged kernel's vector stores.
+    # little alignment for the vector stores of the slab-layout kernels.
     dev = torch.device("cuda:0")
     x_cpu = inputs.activations(40, 512, seed=bits)
     x = x_cpu.to(dev)
