@@ -205,8 +205,10 @@ __global__ void __launch_bounds__(kThreads) quantize_tc_groups(const QuantArgs A
 
 // One RMS over each row of spr slabs. SUB = slabs per lane group (spr / 8 when
 // spr >= 8, so a warp holds a whole row); for spr < 8 a warp step covers 8 / spr rows.
+// As in the group kernel, the loads of a warp's next row are issued as soon as the
+// MMA has consumed the current row's registers, so they land during its arithmetic.
 template <int HB, int CB, int FMT, bool SAT, int SUB>
-__global__ void __launch_bounds__(kThreads, 4) quantize_tc_rows(const QuantArgs A, int spr) {
+__global__ void __launch_bounds__(kThreads, 3) quantize_tc_rows(const QuantArgs A, int spr) {
     constexpr int NBL = Blk<HB>::NBL, PPB = Blk<HB>::PPB;
     const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
     const int rps = SUB > 1 ? 1 : 8 / spr;          // rows per warp step
@@ -214,24 +216,26 @@ __global__ void __launch_bounds__(kThreads, 4) quantize_tc_rows(const QuantArgs 
     const int64_t warp0 = (int64_t(blockIdx.x) * kThreads + threadIdx.x) >> 5;
     const int64_t step = int64_t(gridDim.x) * (kThreads / 32) * rps;
     const BFrag B = make_bfrag(lane, tmask_of<HB>());
-    auto src_of = [&](int64_t row, int u) -> const char* {
-        return A.x + row * A.ld_x_bytes + int64_t(sc0 + 8 * u) * 256;
+    auto load_row = [&](int64_t row, uint4 (&raw)[SUB][4]) {
+#pragma unroll
+        for (int u = 0; u < SUB; ++u) {
+            if (row < A.rows) load_slab(A.x + row * A.ld_x_bytes + int64_t(sc0 + 8 * u) * 256, t, raw[u]);
+            else zero4(raw[u]);
+        }
     };
 
+    uint4 raw[SUB][4];
+    load_row(warp0 * rps + r_in, raw);
     for (int64_t r0 = warp0 * rps; r0 < A.rows; r0 += step) {
         const int64_t row = r0 + r_in;
         const bool valid = row < A.rows;
-        uint4 raw[SUB][4];
-#pragma unroll
-        for (int u = 0; u < SUB; ++u) {
-            if (valid) load_slab(src_of(row, u), t, raw[u]);
-            else zero4(raw[u]);
-        }
         float2 P[SUB][16];
+#pragma unroll
+        for (int u = 0; u < SUB; ++u) mma_stage(raw[u], B, P[u]);
+        load_row(row + step, raw);
         float v = 0.0f;
 #pragma unroll
         for (int u = 0; u < SUB; ++u) {
-            mma_stage(raw[u], B, P[u]);
             reg_stages<HB>(P[u], lane);
             float ss[NBL];
             lane_sums<HB>(P[u], ss);

@@ -50,6 +50,19 @@ def test_codes_full_range(cuda_device, M, N, K):
     check(a, b, sa, sb)
 
 
+@pytest.mark.parametrize("M,N,K", [
+    (2560, 2080, 384),   # 10 x 9 = 90 pair tiles: a full wave of 74, then 16
+    (3072, 2560, 128),   # 12 x 10 = 120 pair tiles: a full wave, then 46
+])
+def test_two_wave_schedules(cuda_device, M, N, K):
+    # More tiles than CTA pairs, so pairs take a second tile with the TMEM
+    # accumulator and stage rings carried over; the first shape's last column
+    # block (N = 2080) is ragged, its second 128-column half wholly past N.
+    a = inputs.gemm_codes(M, K, seed=M + 7)
+    b = inputs.gemm_codes(N, K, seed=N + 9)
+    check(a, b, inputs.positive_scales(M, seed=11), inputs.positive_scales(N, seed=12))
+
+
 def test_int8_extremes(cuda_device):
     # every int8 value, including -128 * -128 products
     M, N, K = 256, 256, 1024
