@@ -69,8 +69,8 @@ NOMINAL_HBM_GBS = 8000.0     # nominal B200 HBM3e bandwidth (about 8 TB/s); the 
 # file is byte-identical to the one that was captured; otherwise null.
 NCU_TRAFFIC = {
     "w4a4_linear": {"source": "bit_quantization_aware_blockwise_b200/csrc/w4a4_gemm.cu",
-                    "sha256": "5f25a0ca49d096b9bae2d3c290d3e0be8bf89b2ac59feddcb19d914829ec7328",
-                    "dram_read": 65654656, "dram_write": 145804928},
+                    "sha256": "d8849045eb06987486af384f050ec8599ce31d380b90fedb80e6bd00f96c3ad9",
+                    "dram_read": 65884160, "dram_write": 145072384},
 }
 
 
