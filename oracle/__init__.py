@@ -69,6 +69,17 @@ def _load():
         lib.oracle_quantize.argtypes = [_p, _i64, _i64, _i64, _int, _i64, _int, _dbl, _dbl,
                                         _p, _p, _p, _p, _p, _p, _p, _p]
         lib.oracle_quantize.restype = _int
+        lib.oracle_e2m1_value.argtypes = [_int]
+        lib.oracle_e2m1_value.restype = _dbl
+        lib.oracle_e2m1_round.argtypes = [_dbl]
+        lib.oracle_e2m1_round.restype = _int
+        lib.oracle_fp4_gauss_mse.argtypes = [_dbl]
+        lib.oracle_fp4_gauss_mse.restype = _dbl
+        lib.oracle_fp4_scale.argtypes = [_p, _p]
+        lib.oracle_fp4_scale.restype = _int
+        lib.oracle_quantize_fp4.argtypes = [_p, _i64, _i64, _i64, _int, _i64, _dbl, _dbl,
+                                            _p, _p, _p, _p, _p, _p, _p, _p, _p]
+        lib.oracle_quantize_fp4.restype = _int
         lib.oracle_trust_bwd.argtypes = [_p, _p, _i64, _i64, _int, _p]
         lib.oracle_trust_bwd.restype = _int
         lib.oracle_gemm_i8.argtypes = [_p, _p, _i64, _i64, _i64, _p]
@@ -135,6 +146,52 @@ def quantize(x, bits: int, had: int = 128, rms_group: int | None = None, trust: 
         _ptr(out["y"]), _ptr(out["t"]), _ptr(out["q"]), _ptr(out["yhat"]),
         _ptr(out["mask"]), _ptr(out["scale"]), _ptr(out["d_round"]), _ptr(out["d_mask"]))
     _check(rc, "quantize")
+    return out
+
+
+def e2m1_value(code: int) -> float:
+    """Value of a 4-bit E2M1 code (bit 3 sign, 2 exponent bits with bias 1, 1 mantissa bit)."""
+    return float(_load().oracle_e2m1_value(int(code)))
+
+
+def e2m1_round(t: float) -> int:
+    """E2M1 code nearest to t (ties to the even mantissa, saturating at +-6, sign of t kept)."""
+    return int(_load().oracle_e2m1_round(float(t)))
+
+
+def fp4_gauss_mse(s: float) -> float:
+    """E[(X - s Q(X/s))^2] for X ~ N(0,1), Q round-to-nearest onto the E2M1 grid."""
+    return float(_load().oracle_fp4_gauss_mse(float(s)))
+
+
+def alpha_fp4():
+    """(s*, minimal Gaussian MSE): the scale of the E2M1 grid that minimises the MSE."""
+    s, m = _dbl(), _dbl()
+    _check(_load().oracle_fp4_scale(ctypes.byref(s), ctypes.byref(m)), "fp4_scale")
+    return s.value, m.value
+
+
+def quantize_fp4(x, had: int = 128, rms_group: int | None = None, trust: float = 1.0):
+    """FP4 (E2M1) grid quantizer of the rows of ``x``. Returns a dict of numpy arrays:
+    y, t, code (4-bit E2M1), value (grid value Q), yhat, mask, scale, d_round, d_mask."""
+    x = np.ascontiguousarray(np.asarray(x, dtype=np.float64))
+    if x.ndim != 2:
+        raise ValueError("x must be 2-D")
+    rows, cols = x.shape
+    rms_group = had if rms_group is None else int(rms_group)
+    s, _ = alpha_fp4()
+    out = {
+        "y": np.empty((rows, cols)), "t": np.empty((rows, cols)),
+        "code": np.empty((rows, cols), dtype=np.uint8), "value": np.empty((rows, cols)),
+        "yhat": np.empty((rows, cols)), "mask": np.empty((rows, cols), dtype=np.uint8),
+        "scale": np.empty((rows, cols // rms_group if rms_group else 0)),
+        "d_round": np.empty((rows, cols)), "d_mask": np.empty((rows, cols)),
+    }
+    rc = _load().oracle_quantize_fp4(
+        _ptr(x), rows, cols, cols, had, rms_group, float(trust), s,
+        _ptr(out["y"]), _ptr(out["t"]), _ptr(out["code"]), _ptr(out["value"]), _ptr(out["yhat"]),
+        _ptr(out["mask"]), _ptr(out["scale"]), _ptr(out["d_round"]), _ptr(out["d_mask"]))
+    _check(rc, "quantize_fp4")
     return out
 
 

@@ -260,6 +260,169 @@ int oracle_quantize(const double* x, int64_t rows, int64_t cols, int64_t ld, int
 }
 
 /* ------------------------------------------------------------------------- */
+/* FP4 (E2M1) grid variant.                                                   */
+/*                                                                           */
+/* The pages evaluate QuEST on an FP4 grid as well as the INT4 one (pith.science */
+/* review, "What carries the argument" and its results list) without spelling */
+/* the variant out. Reading: the same Hadamard transform and RMS, the grid is   */
+/* the 15 signed E2M1 values scaled by Delta = s* r, s* minimising the Gaussian */
+/* MSE of round-to-nearest onto that grid, and the trust mask keeps an element  */
+/* whose error is at most T/2 of the grid interval that holds it (the last one, */
+/* [4, 6], beyond the grid).                                                  */
+/* ------------------------------------------------------------------------- */
+
+/* Value of a 4-bit E2M1 code: bit 3 sign, bits 2..1 exponent (bias 1), bit 0
+ * mantissa; exponent 0 is subnormal (0 or 0.5). No infinities or NaNs. */
+double oracle_e2m1_value(int code) {
+    int sign = (code >> 3) & 1, e = (code >> 1) & 3, m = code & 1;
+    double mag = (e == 0) ? 0.5 * m : ldexp(1.0 + 0.5 * m, e - 1);
+    return sign ? -mag : mag;
+}
+
+/* The 8 non-negative grid magnitudes in increasing order (codes 0..7). */
+static void e2m1_magnitudes(double v[8]) {
+    for (int c = 0; c < 8; ++c) v[c] = oracle_e2m1_value(c);
+}
+
+/* E[(X - s Q(X / s))^2] for X ~ N(0,1), Q round-to-nearest onto the E2M1 grid
+ * (saturating at +-6): cell k of the positive side runs from the midpoint
+ * below level k to the midpoint above it, the last cell is open. */
+double oracle_fp4_gauss_mse(double s) {
+    if (!(s > 0.0)) return NAN;
+    double v[8];
+    e2m1_magnitudes(v);
+    double total = 0.0;
+    for (int k = 0; k < 8; ++k) {
+        double a = (k == 0) ? 0.0 : 0.5 * (v[k - 1] + v[k]) * s;
+        double b = (k == 7) ? INFINITY : 0.5 * (v[k] + v[k + 1]) * s;
+        total += cell_sq_error(a, b, v[k] * s);
+    }
+    return 2.0 * total;
+}
+
+/* s* = argmin_s oracle_fp4_gauss_mse(s), golden section over [lo, hi]. */
+int oracle_fp4_scale(double* s_opt, double* mse_opt) {
+    const double g = (sqrt(5.0) - 1.0) / 2.0;
+    double a = 0.01, b = 2.0;
+    double c = b - g * (b - a), d = a + g * (b - a);
+    double fc = oracle_fp4_gauss_mse(c), fd = oracle_fp4_gauss_mse(d);
+    while (b - a > 1e-13) {
+        if (fc < fd) {
+            b = d; d = c; fd = fc;
+            c = b - g * (b - a); fc = oracle_fp4_gauss_mse(c);
+        } else {
+            a = c; c = d; fc = fd;
+            d = a + g * (b - a); fd = oracle_fp4_gauss_mse(d);
+        }
+    }
+    double sv = 0.5 * (a + b);
+    if (s_opt) *s_opt = sv;
+    if (mse_opt) *mse_opt = oracle_fp4_gauss_mse(sv);
+    return ORACLE_OK;
+}
+
+/* Round-to-nearest of t onto the E2M1 grid by search over all 16 codes; a tie
+ * goes to the code with mantissa bit 0 (nearest-even). The sign bit is the sign
+ * bit of t, so small negative t gives the code of -0. */
+int oracle_e2m1_round(double t) {
+    int best = -1;
+    double bd = INFINITY;
+    for (int c = 0; c < 8; ++c) {
+        double d = fabs(fabs(t) - oracle_e2m1_value(c));
+        if (d < bd || (d == bd && (c & 1) == 0)) { bd = d; best = c; }
+    }
+    return best | (signbit(t) ? 8 : 0);
+}
+
+/* Width of the grid interval that holds |t| (the last interval beyond 6). */
+static double e2m1_interval(double t) {
+    double v[8], a = fabs(t);
+    e2m1_magnitudes(v);
+    for (int k = 0; k < 7; ++k)
+        if (a < v[k + 1]) return v[k + 1] - v[k];
+    return v[7] - v[6];
+}
+
+/*
+ * FP4-grid quantizer, same argument conventions as oracle_quantize; `s_opt` is
+ * the Gaussian-optimal scale of the grid (Delta = s_opt * rms). Outputs:
+ *   code  [rows, cols]  4-bit E2M1 code (required)
+ *   value [rows, cols]  Q(t), the grid value of the code
+ *   yhat = value * Delta; mask; scale = Delta; t; y;
+ *   d_round  distance of t to the nearest decision point (a midpoint between
+ *            neighbouring grid values, or 0 where the sign bit flips)
+ *   d_mask   distance of t to the nearest point where the mask changes
+ */
+int oracle_quantize_fp4(const double* x, int64_t rows, int64_t cols, int64_t ld, int had,
+                        int64_t rms_group, double trust, double s_opt, double* y_out, double* t_out,
+                        uint8_t* code, double* value, double* yhat, uint8_t* mask, double* scale,
+                        double* d_round, double* d_mask) {
+    if (rows < 0 || cols <= 0 || ld < cols || !is_pow2(had) || cols % had != 0) return ORACLE_EINVAL;
+    if (rms_group <= 0 || rms_group % had != 0 || cols % rms_group != 0) return ORACLE_EINVAL;
+    if (!(trust > 0.0) || !(s_opt > 0.0) || code == NULL) return ORACLE_EINVAL;
+
+    double v[8];
+    e2m1_magnitudes(v);
+    double* H = (double*)malloc(sizeof(double) * had * had);
+    double* y = (double*)malloc(sizeof(double) * cols);
+    if (!H || !y) { free(H); free(y); return ORACLE_EINVAL; }
+    oracle_hadamard(had, H);
+
+    for (int64_t r = 0; r < rows; ++r) {
+        const double* xr = x + r * ld;
+        for (int64_t b0 = 0; b0 < cols; b0 += had) hadamard_block(H, had, xr + b0, y + b0);
+        for (int64_t g0 = 0; g0 < cols; g0 += rms_group) {
+            double ss = 0.0;
+            for (int64_t j = 0; j < rms_group; ++j) ss += y[g0 + j] * y[g0 + j];
+            double delta = s_opt * sqrt(ss / (double)rms_group);
+            if (scale) scale[r * (cols / rms_group) + g0 / rms_group] = delta;
+            for (int64_t j = 0; j < rms_group; ++j) {
+                int64_t idx = r * cols + g0 + j;
+                double yv = y[g0 + j], tv, qv, dr, dm;
+                int cv;
+                uint8_t mv;
+                if (delta == 0.0) {
+                    tv = 0.0; cv = 0; qv = 0.0; mv = 1; dr = INFINITY; dm = INFINITY;
+                } else {
+                    tv = yv / delta;
+                    cv = oracle_e2m1_round(tv);
+                    qv = oracle_e2m1_value(cv);
+                    mv = (fabs(tv - qv) <= 0.5 * trust * e2m1_interval(tv)) ? 1 : 0;
+                    /* decision points: 0 and the midpoints between neighbours */
+                    double a = fabs(tv);
+                    dr = a;
+                    for (int k = 0; k < 7; ++k) {
+                        double d = fabs(a - 0.5 * (v[k] + v[k + 1]));
+                        if (d < dr) dr = d;
+                    }
+                    /* mask flips: 6 + T beyond the grid; for T < 1 also
+                     * v_k + (T/2) w_k and v_(k+1) - (T/2) w_k in each interval */
+                    dm = fabs(a - (v[7] + 0.5 * trust * (v[7] - v[6])));
+                    if (trust < 1.0)
+                        for (int k = 0; k < 7; ++k) {
+                            double w = v[k + 1] - v[k];
+                            double f0 = v[k] + 0.5 * trust * w, f1 = v[k + 1] - 0.5 * trust * w;
+                            if (fabs(a - f0) < dm) dm = fabs(a - f0);
+                            if (fabs(a - f1) < dm) dm = fabs(a - f1);
+                        }
+                }
+                if (y_out) y_out[idx] = yv;
+                if (t_out) t_out[idx] = tv;
+                code[idx] = (uint8_t)cv;
+                if (value) value[idx] = qv;
+                if (yhat) yhat[idx] = qv * delta;
+                if (mask) mask[idx] = mv;
+                if (d_round) d_round[idx] = dr;
+                if (d_mask) d_mask[idx] = dm;
+            }
+        }
+    }
+    free(H);
+    free(y);
+    return ORACLE_OK;
+}
+
+/* ------------------------------------------------------------------------- */
 /* Trust backward: g_x = H^T (m . g) / sqrt(n) per Hadamard block.            */
 /* ------------------------------------------------------------------------- */
 
