@@ -744,7 +744,21 @@ def run_configs(args):
                                           R, NW, C, HB, y.data_ptr(), None, s)
     add("grouped linear 16384x5632x2048 (E4M3 codes, scales per 128-group)", f,
         R * C + NW * C + 4 * G * (R + NW) + 2 * R * NW, unit_ops=GEMM_OPS)
-    gemm_tops = rows[-5]["tops"]
+    # the FP4 (E2M1) grid: packed codes + mask per 128-group, int8 c = 2Q operands
+    # (one RMS per row) and the same int8 layer on them
+    F4, F4OP = q.CODES_FP4_PACKED, q.CODES_FP4_OPERAND
+    f, nb, _ = quant(x2, 4, HB, F4, q.MASK_BITS)
+    add("FP4 quantize 16384x2048 E2M1 codes+mask (RMS per 128-group)", f, nb)
+    fx4, nbx4, (cx4, sx4, _) = quant(x2, 4, C, F4OP, None)
+    fw4, nbw4, (cw4, sw4, _) = quant(w, 4, C, F4OP, None)
+    add("FP4 operand quantize X 16384x2048 c=2Q (row RMS)", fx4, nbx4)
+    add("FP4 operand quantize W_up 5632x2048 c=2Q (row RMS)", fw4, nbw4)
+    fx4(); fw4()
+    f = lambda: q.w4a4_linear_raw(cx4.data_ptr(), sx4.data_ptr(), cw4.data_ptr(), sw4.data_ptr(), R, NW, C,
+                                  y.data_ptr(), None, s)
+    add("FP4 linear 16384x5632x2048 (c=2Q codes, int8 tensor cores)", f,
+        R * C + NW * C + 4 * (R + NW) + 2 * R * NW, unit_ops=GEMM_OPS)
+    gemm_tops = next(r["tops"] for r in rows if r["case"].startswith("cfg5 W4A4 linear"))
     q.device_status()
     probe = mma_probe(dev, gemm_tops)
     print(json.dumps({"configs": rows, "int8_mma_probe": probe, "peaks": peaks}), flush=True)
@@ -773,11 +787,12 @@ def run_profile_kernels(args):
     sag = sa[:, None].repeat(1, C // HB).contiguous()
     sbg = sb[:, None].repeat(1, C // HB).contiguous()
     yg = q.w4a4_linear_grouped(a8, sag, b8, sbg)                                       # 5
+    f4 = q.quantize_fwd(x, 4, code_mode=q.CODES_FP4_PACKED, mask_mode=q.MASK_BITS)    # 6
     torch.cuda.synchronize()
     q.device_status()
     print(json.dumps({"profile_kernels": "ok", "rows": rows, "checksum": [
         float(out["scales"].sum()), float(gi.float().abs().sum()), float(op["scales"].sum()),
-        float(y.float().abs().sum()), float(yg.float().abs().sum())]}))
+        float(y.float().abs().sum()), float(yg.float().abs().sum()), float(f4["scales"].sum())]}))
 
 
 def main():

@@ -15,6 +15,7 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 _LIB_NAME = "libquest_b200.so"
 
 CODES_PACKED, CODES_INT8, CODES_GEMM_OPERAND, CODES_GEMM_OPERAND_E4M3 = 0, 1, 2, 3
+CODES_FP4_PACKED, CODES_FP4_OPERAND = 4, 5   # FP4 (E2M1) grid, bits = 4
 MASK_BITS, MASK_BYTES = 0, 1
 BF16, FP32 = 0, 1
 _STATUS = {0: "ok", 1: "invalid argument", 2: "unsupported", 3: "CUDA error", 4: "device wait timed out"}
@@ -30,6 +31,7 @@ SIGNATURES = {
     "quest_w4a4_linear_grouped": (_int, [_p, _p, _p, _p, _i64, _i64, _i64, _i64, _p, _p, _p]),
     "quest_device_status": (_int, [_p]),
     "quest_alpha": (_f64, [_int]),
+    "quest_alpha_fp4": (_f64, []),
     "quest_container_bits": (_int, [_int]),
     "quest_codes_bytes": (_sz, [_i64, _i64, _int, _int]),
     "quest_mask_bytes": (_sz, [_i64, _i64, _int]),
@@ -118,6 +120,11 @@ def device_status(stream=0):
 
 def alpha(bits: int) -> float:
     return float(load_library().quest_alpha(bits))
+
+
+def alpha_fp4() -> float:
+    """s*, the Gaussian-MSE-optimal scale of the E2M1 grid (Delta = s* r)."""
+    return float(load_library().quest_alpha_fp4())
 
 
 def container_bits(bits: int) -> int:

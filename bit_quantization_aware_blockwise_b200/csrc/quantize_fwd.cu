@@ -317,7 +317,8 @@ cudaError_t launch_quantize(const QuantArgs& a, quest_dtype x_dtype, int had_blo
         return launch_quantize_tc(a, had_block, cbits, bits, row_mode, stream);
     if (hs_path_ok(a, had_block, cbits, row_mode))
         return launch_quantize_hs(a, x_dtype, had_block, cbits, bits, row_mode, stream);
-    if (a.c.code_fp8) return cudaErrorNotSupported;   // E4M3 codes only on the two layouts above
+    // E4M3 operand codes and the FP4 grid only on the two layouts above
+    if (a.c.code_fp8 || a.c.grid_fp4) return cudaErrorNotSupported;
     if (x_dtype == QUEST_BF16) return launch_dtype<__nv_bfloat16>(a, had_block, cbits, row_mode, stream);
     return launch_dtype<float>(a, had_block, cbits, row_mode, stream);
 }

@@ -135,27 +135,43 @@ __device__ __forceinline__ void emit(const QuantArgs& A, const float2 (&P)[32], 
     uint32_t mlo = 0, mhi = 0;
 #pragma unroll
     for (int c = 0; c < 8; ++c) {
-        float2 s[4];
-        chunk_decide<SAT, PPB>(P, G, c, k, s);
-        if constexpr (CB == 8) {
-            if (valid) *reinterpret_cast<uint2*>(codes + (2 * c + h) * 8) = chunk_pack_i8<FMT>(s, k);
+        float2 y[4];   // dequantised values of the chunk (when requested)
+        uint32_t m = 0;
+        if constexpr (FMT >= 3) {
+            // FP4 grid: FMT 3 packed E2M1 codes, FMT 4 int8 c = 2Q
+            const uint32_t w4 = chunk_fp4<PPB>(P, G, c);
+            if constexpr (FMT == 3) {
+                W[c] = w4;
+            } else {
+                if (valid) *reinterpret_cast<uint2*>(codes + (2 * c + h) * 8) = fp4_operand_i8(w4);
+            }
+            if (do_mask)
+                m = k.trust_ge1 ? mask_byte_edge<PPB>(P, G, c) : mask_byte_fp4_cell<PPB>(P, G, c, w4, k);
+            if (do_deq) fp4_dequant<PPB>(w4, G, c, y);
         } else {
-            W[c] = chunk_pack<CB>(s, k);
+            float2 s[4];
+            chunk_decide<SAT, PPB>(P, G, c, k, s);
+            if constexpr (CB == 8) {
+                if (valid) *reinterpret_cast<uint2*>(codes + (2 * c + h) * 8) = chunk_pack_i8<FMT>(s, k);
+            } else {
+                W[c] = chunk_pack<CB>(s, k);
+            }
+            if (do_mask) m = mask_byte<PPB>(P, G, c, k);
+            if (do_deq) {
+                // yhat = q_b Delta + (1/2 - 2^(b-1)) Delta
+#pragma unroll
+                for (int p = 0; p < 4; ++p) {
+                    const GroupK& g = G[(4 * c + p) / PPB];
+                    const float2 qb = __fadd2_rn(s[p], make_float2(-kMagic, -kMagic));
+                    y[p] = __ffma2_rn(qb, make_float2(g.delta, g.delta), make_float2(g.ch, g.ch));
+                }
+            }
         }
         if (do_mask) {
-            const uint32_t m = mask_byte<PPB>(P, G, c, k);
             if (c < 4) mlo |= m << (8 * c);
             else mhi |= m << (8 * (c - 4));
         }
         if (do_deq) {
-            // yhat = q_b Delta + (1/2 - 2^(b-1)) Delta
-            float2 y[4];
-#pragma unroll
-            for (int p = 0; p < 4; ++p) {
-                const GroupK& g = G[(4 * c + p) / PPB];
-                const float2 qb = __fadd2_rn(s[p], make_float2(-kMagic, -kMagic));
-                y[p] = __ffma2_rn(qb, make_float2(g.delta, g.delta), make_float2(g.ch, g.ch));
-            }
             const int64_t e = e_slab + (2 * c + h) * 8;
             if (k.deq_mode == 0) {
                 *reinterpret_cast<uint4*>(A.deq + row * A.deq_row_bytes + 2 * e) =
@@ -372,7 +388,8 @@ cudaError_t launch_t(const QuantArgs& a, bool row_mode, cudaStream_t s) {
 
 template <typename Tin, int HB, int CB, int FMT>
 cudaError_t launch_sat(const QuantArgs& a, int bits, bool row, cudaStream_t s) {
-    if constexpr (FMT == 2) return launch_t<Tin, HB, CB, FMT, true>(a, row, s);   // E4M3 codes: b <= 4
+    // E4M3 codes (b <= 4) and the FP4 grid (no integer decision path)
+    if constexpr (FMT >= 2) return launch_t<Tin, HB, CB, FMT, true>(a, row, s);
     else return bits <= 6 ? launch_t<Tin, HB, CB, FMT, true>(a, row, s)
                           : launch_t<Tin, HB, CB, FMT, false>(a, row, s);
 }
@@ -382,8 +399,10 @@ cudaError_t launch_hb(const QuantArgs& a, int bits, int cb, bool row, cudaStream
     switch (cb) {
         case 1: return launch_sat<Tin, HB, 1, 0>(a, bits, row, s);
         case 2: return launch_sat<Tin, HB, 2, 0>(a, bits, row, s);
-        case 4: return launch_sat<Tin, HB, 4, 0>(a, bits, row, s);
-        case 8: return a.c.code_fp8 ? launch_sat<Tin, HB, 8, 2>(a, bits, row, s)
+        case 4: return a.c.grid_fp4 ? launch_sat<Tin, HB, 4, 3>(a, bits, row, s)
+                                    : launch_sat<Tin, HB, 4, 0>(a, bits, row, s);
+        case 8: return a.c.grid_fp4 ? launch_sat<Tin, HB, 8, 4>(a, bits, row, s)
+                : a.c.code_fp8 ? launch_sat<Tin, HB, 8, 2>(a, bits, row, s)
                                     : a.c.pack2_mult == 2 ? launch_sat<Tin, HB, 8, 1>(a, bits, row, s)
                                                           : launch_sat<Tin, HB, 8, 0>(a, bits, row, s);
     }

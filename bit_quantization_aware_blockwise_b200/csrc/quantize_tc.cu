@@ -56,26 +56,40 @@ __device__ __forceinline__ void emit(const QuantArgs& A, const float2 (&P)[16], 
 #pragma unroll
     for (int f = 0; f < 4; ++f) {
         const int c = t + 4 * f;
-        float2 s[4];
-        chunk_decide<SAT, PPB>(P, G, f, k, s);
-        if constexpr (CB == 8) {
-            if (valid) *reinterpret_cast<uint2*>(codes + 8 * c) = chunk_pack_i8<FMT>(s, k);
-        } else if constexpr (CB == 4) {
-            if (valid) *reinterpret_cast<uint32_t*>(codes + 4 * c) = chunk_pack<4>(s, k);
-        } else if constexpr (CB == 2) {
-            if (valid) *reinterpret_cast<uint16_t*>(codes + 2 * c) = (uint16_t)chunk_pack<2>(s, k);
+        float2 y[4];   // dequantised values of the chunk (when requested)
+        if constexpr (FMT >= 3) {
+            // FP4 grid: FMT 3 packed E2M1 codes, FMT 4 int8 c = 2Q
+            const uint32_t w4 = chunk_fp4<PPB>(P, G, f);
+            if constexpr (FMT == 3) {
+                if (valid) *reinterpret_cast<uint32_t*>(codes + 4 * c) = w4;
+            } else {
+                if (valid) *reinterpret_cast<uint2*>(codes + 8 * c) = fp4_operand_i8(w4);
+            }
+            if (do_mask && !k.trust_ge1) mbytes |= mask_byte_fp4_cell<PPB>(P, G, f, w4, k) << (8 * f);
+            if (do_deq) fp4_dequant<PPB>(w4, G, f, y);
         } else {
-            cbytes |= chunk_pack<1>(s, k) << (8 * f);
+            float2 s[4];
+            chunk_decide<SAT, PPB>(P, G, f, k, s);
+            if constexpr (CB == 8) {
+                if (valid) *reinterpret_cast<uint2*>(codes + 8 * c) = chunk_pack_i8<FMT>(s, k);
+            } else if constexpr (CB == 4) {
+                if (valid) *reinterpret_cast<uint32_t*>(codes + 4 * c) = chunk_pack<4>(s, k);
+            } else if constexpr (CB == 2) {
+                if (valid) *reinterpret_cast<uint16_t*>(codes + 2 * c) = (uint16_t)chunk_pack<2>(s, k);
+            } else {
+                cbytes |= chunk_pack<1>(s, k) << (8 * f);
+            }
+            if (do_deq) {
+                // yhat = q_b Delta + (1/2 - 2^(b-1)) Delta
+#pragma unroll
+                for (int p = 0; p < 4; ++p) {
+                    const GroupK& g = G[(4 * f + p) / PPB];
+                    const float2 qb = __fadd2_rn(s[p], make_float2(-kMagic, -kMagic));
+                    y[p] = __ffma2_rn(qb, make_float2(g.delta, g.delta), make_float2(g.ch, g.ch));
+                }
+            }
         }
         if (do_deq) {
-            // yhat = q_b Delta + (1/2 - 2^(b-1)) Delta
-            float2 y[4];
-#pragma unroll
-            for (int p = 0; p < 4; ++p) {
-                const GroupK& g = G[(4 * f + p) / PPB];
-                const float2 qb = __fadd2_rn(s[p], make_float2(-kMagic, -kMagic));
-                y[p] = __ffma2_rn(qb, make_float2(g.delta, g.delta), make_float2(g.ch, g.ch));
-            }
             const int64_t e = e_slab + 8 * c;
             if (k.deq_mode == 0) {
                 *reinterpret_cast<uint4*>(A.deq + row * A.deq_row_bytes + 2 * e) =
@@ -91,12 +105,12 @@ __device__ __forceinline__ void emit(const QuantArgs& A, const float2 (&P)[16], 
         }
     }
     // trust mask bytes: one loop per form of the test, so that neither is predicated
-    // into the other's path
+    // into the other's path (the FP4 grid's general form was taken with its codes)
     if (do_mask) {
         if (k.trust_ge1) {
 #pragma unroll
             for (int f = 0; f < 4; ++f) mbytes |= mask_byte_edge<PPB>(P, G, f) << (8 * f);
-        } else {
+        } else if constexpr (FMT < 3) {
 #pragma unroll
             for (int f = 0; f < 4; ++f) mbytes |= mask_byte_cell<PPB>(P, G, f, k) << (8 * f);
         }
@@ -285,7 +299,8 @@ cudaError_t launch_t(const QuantArgs& a, bool row_mode, cudaStream_t s) {
 
 template <int HB, int CB, int FMT>
 cudaError_t launch_sat(const QuantArgs& a, int bits, bool row, cudaStream_t s) {
-    if constexpr (FMT == 2) return launch_t<HB, CB, FMT, true>(a, row, s);   // E4M3 codes: b <= 4
+    // E4M3 codes (b <= 4) and the FP4 grid (no integer decision path)
+    if constexpr (FMT >= 2) return launch_t<HB, CB, FMT, true>(a, row, s);
     else return bits <= 6 ? launch_t<HB, CB, FMT, true>(a, row, s) : launch_t<HB, CB, FMT, false>(a, row, s);
 }
 
@@ -294,8 +309,9 @@ cudaError_t launch_hb(const QuantArgs& a, int bits, int cb, bool row, cudaStream
     switch (cb) {
         case 1: return launch_sat<HB, 1, 0>(a, bits, row, s);
         case 2: return launch_sat<HB, 2, 0>(a, bits, row, s);
-        case 4: return launch_sat<HB, 4, 0>(a, bits, row, s);
-        case 8: return a.c.code_fp8 ? launch_sat<HB, 8, 2>(a, bits, row, s)
+        case 4: return a.c.grid_fp4 ? launch_sat<HB, 4, 3>(a, bits, row, s) : launch_sat<HB, 4, 0>(a, bits, row, s);
+        case 8: return a.c.grid_fp4 ? launch_sat<HB, 8, 4>(a, bits, row, s)
+                : a.c.code_fp8 ? launch_sat<HB, 8, 2>(a, bits, row, s)
                                     : a.c.pack2_mult == 2 ? launch_sat<HB, 8, 1>(a, bits, row, s)
                                                           : launch_sat<HB, 8, 0>(a, bits, row, s);
     }

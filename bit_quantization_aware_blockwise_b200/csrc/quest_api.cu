@@ -87,12 +87,49 @@ void init_alpha() {
     for (int b = 1; b <= 8; ++b) g_alpha[b] = ldexp(optimal_step(b), b - 1);
 }
 
+// s* of the FP4 grid: the non-negative E2M1 values v_k with round-to-nearest
+// cells [s (v_(k-1) + v_k) / 2, s (v_k + v_(k+1)) / 2) (the first from 0, the last
+// open). The midpoint thresholds cancel the boundary terms of dMSE/ds again, so
+// the optimum is the root of  g(s) = sum_k v_k (phi(a_k) - phi(b_k)) - s sum_k v_k^2 P(cell_k),
+// positive below it; found by bisection.
+constexpr double kE2M1[8] = {0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0};
+
+double fp4_stationarity_residual(double s) {
+    double first = 0.0, second = 0.0;
+    for (int k = 0; k < 8; ++k) {
+        const double a = k == 0 ? 0.0 : 0.5 * (kE2M1[k - 1] + kE2M1[k]) * s;
+        const double b = k == 7 ? INFINITY : 0.5 * (kE2M1[k] + kE2M1[k + 1]) * s;
+        first += kE2M1[k] * (std_normal_pdf(a) - std_normal_pdf(b));
+        second += kE2M1[k] * kE2M1[k] * cell_prob(a, b);
+    }
+    return first - s * second;
+}
+
+double g_alpha_fp4 = NAN;
+std::once_flag g_alpha_fp4_once;
+
+void init_alpha_fp4() {
+    double lo = 1e-2, hi = 2.0;
+    for (int it = 0; it < 200; ++it) {
+        const double mid = 0.5 * (lo + hi);
+        if (mid <= lo || mid >= hi) break;
+        if (fp4_stationarity_residual(mid) > 0.0)
+            lo = mid;
+        else
+            hi = mid;
+    }
+    g_alpha_fp4 = 0.5 * (lo + hi);
+}
+
+bool is_fp4_mode(quest_code_mode m) { return m == QUEST_CODES_FP4_PACKED || m == QUEST_CODES_FP4_OPERAND; }
+
 int container_bits_of(int bits) {
     static const int t[9] = {0, 1, 2, 4, 4, 8, 8, 8, 8};
     return (bits >= 1 && bits <= 8) ? t[bits] : 0;
 }
 
 int code_bits(int bits, quest_code_mode mode) {
+    if (mode == QUEST_CODES_FP4_PACKED) return 4;
     return mode == QUEST_CODES_PACKED ? container_bits_of(bits) : 8;
 }
 
@@ -187,13 +224,19 @@ double quest_alpha(int bits) {
     return g_alpha[bits];
 }
 
+double quest_alpha_fp4(void) {
+    std::call_once(g_alpha_fp4_once, init_alpha_fp4);
+    return g_alpha_fp4;
+}
+
 int quest_container_bits(int bits) { return container_bits_of(bits); }
 
 size_t quest_codes_bytes(int64_t rows, int64_t cols, int bits, quest_code_mode mode) {
     if (rows < 0 || cols <= 0 || bits < 1 || bits > 8) return 0;
     if (mode != QUEST_CODES_PACKED && mode != QUEST_CODES_INT8 && mode != QUEST_CODES_GEMM_OPERAND &&
-        mode != QUEST_CODES_GEMM_OPERAND_E4M3)
+        mode != QUEST_CODES_GEMM_OPERAND_E4M3 && !is_fp4_mode(mode))
         return 0;
+    if (is_fp4_mode(mode) && bits != 4) return 0;
     const int cb = code_bits(bits, mode);
     if ((cols * cb) % 8 != 0) return 0;
     return (size_t)(rows * (cols * cb / 8));
@@ -238,8 +281,10 @@ quest_status quest_quantize_fwd(const void* x, quest_dtype x_dtype, int64_t rows
         return fail(QUEST_EUNSUPPORTED, "rms_group == cols supports at most 16384 columns (8192 for had_block 16)");
     if (!(trust > 0.0f) || isinf(trust)) return fail(QUEST_EINVAL, "trust must be finite and > 0");
     if (code_mode != QUEST_CODES_PACKED && code_mode != QUEST_CODES_INT8 && code_mode != QUEST_CODES_GEMM_OPERAND &&
-        code_mode != QUEST_CODES_GEMM_OPERAND_E4M3)
+        code_mode != QUEST_CODES_GEMM_OPERAND_E4M3 && !is_fp4_mode(code_mode))
         return fail(QUEST_EINVAL, "invalid code_mode");
+    const bool fp4 = is_fp4_mode(code_mode);
+    if (fp4 && bits != 4) return fail(QUEST_EINVAL, "the FP4 (E2M1) grid needs bits == 4");
     if (code_mode == QUEST_CODES_GEMM_OPERAND && bits > 7)
         return fail(QUEST_EINVAL, "the GEMM operand form c = 2q+1 needs bits <= 7 to fit int8");
     if (code_mode == QUEST_CODES_GEMM_OPERAND_E4M3 && bits > 4)
@@ -265,6 +310,10 @@ quest_status quest_quantize_fwd(const void* x, quest_dtype x_dtype, int64_t rows
 
     const double alpha = quest_alpha(bits);
     const int lo = -(1 << (bits - 1)), hi = (1 << (bits - 1)) - 1;
+    // the FP4 grid: Delta = s* r, mask edge 6 + T for T >= 1 (the last grid
+    // interval [4, 6] is 2 wide, so T of its halves reach 6 + T)
+    const double cd_grid = fp4 ? quest_alpha_fp4() : alpha / ldexp(1.0, bits - 1);
+    const double edge_grid = fp4 ? 6.0 + (double)trust : ldexp(1.0, bits - 1) + 0.5 * ((double)trust - 1.0);
     QuantArgs a;
     a.x = static_cast<const char*>(x);
     a.ld_x_bytes = ld_x * esize;
@@ -279,20 +328,20 @@ quest_status quest_quantize_fwd(const void* x, quest_dtype x_dtype, int64_t rows
     a.deq = static_cast<uint8_t*>(dequant);
     a.deq_row_bytes = cols * (dequant_dtype == QUEST_BF16 ? 2 : 4);
     QuantConsts& c = a.c;
-    c.c_delta = (float)(alpha / ldexp(1.0, bits - 1));
+    c.c_delta = (float)cd_grid;
     c.inv_count = (float)(1.0 / ((double)had_block * (double)rms_group));
     c.sqrt_hb = (float)sqrt((double)had_block);
-    c.edge = (float)(ldexp(1.0, bits - 1) + 0.5 * ((double)trust - 1.0));
+    c.edge = (float)edge_grid;
     c.half_trust = 0.5f * trust;
     c.s_lo = kMagic + (float)lo;
     c.s_hi = kMagic + (float)hi;
-    pack_constants(cb, code_mode, &c.pack_mult, &c.pack_add, &c.pack_xor);
+    pack_constants(cb, fp4 ? QUEST_CODES_INT8 : code_mode, &c.pack_mult, &c.pack_add, &c.pack_xor);
     c.inv_levels = (float)ldexp(1.0, -bits);
     c.half_levels = (float)ldexp(1.0, bits - 1);
     {
-        const double cd = alpha / ldexp(1.0, bits - 1), ic = 1.0 / ((double)had_block * (double)rms_group);
+        const double cd = cd_grid, ic = 1.0 / ((double)had_block * (double)rms_group);
         const double shb = sqrt((double)had_block);
-        const double edge = ldexp(1.0, bits - 1) + 0.5 * ((double)trust - 1.0);
+        const double edge = edge_grid;
         c.delta_k = (float)(cd * sqrt(ic));
         c.inv_k = (float)(1.0 / (shb * cd * sqrt(ic)));
         c.a_k = (float)(ldexp(1.0, -bits) / (shb * cd * sqrt(ic)));
@@ -302,9 +351,11 @@ quest_status quest_quantize_fwd(const void* x, quest_dtype x_dtype, int64_t rows
     c.s_mid = kMagic + (float)ldexp(1.0, bits - 1);
     c.s_top = kMagic + (float)(ldexp(1.0, bits) - 1.0);
     c.cell_center = (float)(0.5 - ldexp(1.0, bits - 1));
-    pack_constants_biased(cb, bits, code_mode == QUEST_CODES_GEMM_OPERAND_E4M3 ? QUEST_CODES_GEMM_OPERAND : code_mode,
+    pack_constants_biased(cb, bits, code_mode == QUEST_CODES_GEMM_OPERAND_E4M3 ? QUEST_CODES_GEMM_OPERAND
+                                    : fp4 ? QUEST_CODES_INT8 : code_mode,
                           &c.pack2_mult, &c.pack2_add, &c.pack2_xor);
     c.code_fp8 = code_mode == QUEST_CODES_GEMM_OPERAND_E4M3;
+    c.grid_fp4 = code_mode == QUEST_CODES_FP4_PACKED ? 1 : (code_mode == QUEST_CODES_FP4_OPERAND ? 2 : 0);
     {   // an 8-field word (one chunk of 8 elements) for cb <= 4
         const uint32_t rep8 = cb == 1 ? 0xFFu : (cb == 2 ? 0x5555u : 0x11111111u);
         const uint32_t x8 = cb == 1 ? 0xFFu : (cb == 2 ? 0xAAAAu : 0x88888888u);
@@ -318,8 +369,8 @@ quest_status quest_quantize_fwd(const void* x, quest_dtype x_dtype, int64_t rows
 
     cudaError_t e = launch_quantize(a, x_dtype, had_block, cb, bits, row_mode, static_cast<cudaStream_t>(stream));
     if (e == cudaErrorNotSupported)
-        return fail(QUEST_EUNSUPPORTED, "the E4M3 operand form needs rows of whole 128-value slabs, 8-byte aligned "
-                                        "codes and at most 16 slabs per row in row-RMS mode");
+        return fail(QUEST_EUNSUPPORTED, "the E4M3 operand form and the FP4 grid need rows of whole 128-value slabs, "
+                                        "aligned codes and at most 16 slabs per row in row-RMS mode");
     if (e != cudaSuccess) return cuda_fail(e, "quest_quantize_fwd launch");
     return QUEST_OK;
 }

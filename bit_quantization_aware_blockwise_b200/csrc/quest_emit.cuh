@@ -5,6 +5,8 @@
 // the packing constants in quest_api.cu).
 #pragma once
 
+#include <cuda_fp16.h>
+#include <cuda_fp4.h>
 #include <cuda_fp8.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
@@ -152,6 +154,81 @@ __device__ __forceinline__ uint2 chunk_pack_i8(const float2 (&s)[4], const Quant
         }
     }
     return make_uint2(w[0], w[1]);
+}
+
+// ---------------------------------------------------------------------------
+// FP4 (E2M1) grid. A chunk's 8 codes form one 32-bit word, element j of the
+// chunk in nibble j; t = y_u * inv is rounded onto the grid by the hardware
+// conversion (nearest, ties to the even mantissa, saturating at +-6, the sign
+// of t kept, so a small negative t gives -0).
+// ---------------------------------------------------------------------------
+template <int PPB, int N>
+__device__ __forceinline__ uint32_t chunk_fp4(const float2 (&P)[N], const GroupK* G, int c) {
+    uint32_t w = 0;
+#pragma unroll
+    for (int p = 0; p < 4; ++p) {
+        const GroupK& g = G[(4 * c + p) / PPB];
+        const float2 t = __fmul2_rn(P[4 * c + p], make_float2(g.inv, g.inv));
+        w |= uint32_t(__nv_cvt_float2_to_fp4x2(t, __NV_E2M1, cudaRoundNearest)) << (8 * p);
+    }
+    return w;
+}
+
+// The grid values of a pair of codes (byte p of a chunk word) as fp32.
+__device__ __forceinline__ float2 fp4_pair_value(uint32_t w, int p) {
+    const __half2_raw h = __nv_cvt_fp4x2_to_halfraw2((__nv_fp4x2_storage_t)((w >> (8 * p)) & 0xFFu), __NV_E2M1);
+    return __half22float2(*reinterpret_cast<const __half2*>(&h));
+}
+
+// int8 c = 2 Q of a chunk word. Each pair of grid values is decoded to an f16
+// pair (exact), then 2 Q + 1152 (exact: f16 holds the integers of [1024, 2048)
+// with unit spacing) leaves c + 128 in the low byte of each half; one byte
+// permutation gathers four of them and an XOR with 0x80 removes the bias.
+__device__ __forceinline__ uint32_t fp4_prmt(uint32_t a, uint32_t b, uint32_t sel) {
+    uint32_t d;
+    asm("prmt.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(sel));
+    return d;
+}
+__device__ __forceinline__ uint2 fp4_operand_i8(uint32_t w) {
+    uint32_t h[4];
+#pragma unroll
+    for (int p = 0; p < 4; ++p) {
+        const __half2_raw r = __nv_cvt_fp4x2_to_halfraw2((__nv_fp4x2_storage_t)((w >> (8 * p)) & 0xFFu), __NV_E2M1);
+        const __half2 u = __hfma2(*reinterpret_cast<const __half2*>(&r), __floats2half2_rn(2.0f, 2.0f),
+                                  __floats2half2_rn(1152.0f, 1152.0f));
+        h[p] = *reinterpret_cast<const uint32_t*>(&u);
+    }
+    return make_uint2(fp4_prmt(h[0], h[1], 0x6420u) ^ 0x80808080u, fp4_prmt(h[2], h[3], 0x6420u) ^ 0x80808080u);
+}
+
+// yhat = Q Delta for the 4 pairs of chunk c.
+template <int PPB>
+__device__ __forceinline__ void fp4_dequant(uint32_t w, const GroupK* G, int c, float2 (&y)[4]) {
+#pragma unroll
+    for (int p = 0; p < 4; ++p) {
+        const float d = G[(4 * c + p) / PPB].delta;
+        y[p] = __fmul2_rn(fp4_pair_value(w, p), make_float2(d, d));
+    }
+}
+
+// General-T trust mask byte of chunk c on the FP4 grid: m = [|t - Q| <= (T/2) w],
+// w the width of the grid interval that holds |t| (0.5 below 2, 1 below 4, else 2).
+template <int PPB, int N>
+__device__ __forceinline__ uint32_t mask_byte_fp4_cell(const float2 (&P)[N], const GroupK* G, int c,
+                                                       uint32_t w, const QuantConsts& k) {
+    uint32_t acc = 0;
+#pragma unroll
+    for (int p = 0; p < 4; ++p) {
+        const GroupK& g = G[(4 * c + p) / PPB];
+        const float2 t = __fmul2_rn(P[4 * c + p], make_float2(g.inv, g.inv));
+        const float2 q = fp4_pair_value(w, p);
+        const float ax = fabsf(t.x), ay = fabsf(t.y);
+        const float wx = ax < 2.0f ? 0.5f : (ax < 4.0f ? 1.0f : 2.0f);
+        const float wy = ay < 2.0f ? 0.5f : (ay < 4.0f ? 1.0f : 2.0f);
+        acc |= uint32_t(fabsf(t.x - q.x) <= k.half_trust * wx) << (2 * p);
+        acc |= uint32_t(fabsf(t.y - q.y) <= k.half_trust * wy) << (2 * p + 1);
+    }
+    return acc;
 }
 
 }  // namespace quest

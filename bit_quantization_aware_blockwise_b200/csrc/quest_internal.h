@@ -36,6 +36,7 @@ struct QuantConsts {
     uint32_t pack8_add, pack8_xor;                // words of 8 fields (cb <= 4)
     int trust_ge1;      // 1: use m = [|t| <= edge]
     int code_fp8;       // operand codes c = 2q + 1 stored as FP8 E4M3
+    int grid_fp4;       // 0 integer grid; 1 FP4 grid, packed E2M1 codes; 2 FP4 grid, int8 c = 2Q
     int mask_mode;      // -1 none, 0 bits, 1 bytes
     int deq_mode;       // -1 none, 0 bf16, 1 fp32
 };

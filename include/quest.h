@@ -68,12 +68,28 @@ typedef enum quest_dtype {
  *                             quest_w4a4_linear_grouped. Supported where the
  *                             rows are whole 128-value slabs with 8-byte aligned
  *                             codes and at most 16 slabs per row in row-RMS mode
- *                             (QUEST_EUNSUPPORTED otherwise). */
+ *                             (QUEST_EUNSUPPORTED otherwise).
+ * The FP4 grid (bits must be 4; see quest_quantize_fwd for the grid, scale and
+ * mask of this variant):
+ *   QUEST_CODES_FP4_PACKED    4-bit OCP E2M1 codes (bit 3 sign, bits 2..1
+ *                             exponent with bias 1, bit 0 mantissa), two per
+ *                             byte, element 2j in the low nibble. Row stride
+ *                             cols / 2 bytes; codes 4-byte aligned.
+ *   QUEST_CODES_FP4_OPERAND   one int8 per element holding c = 2 Q, twice the
+ *                             grid value Q (c in {0, +-1, +-2, +-3, +-4, +-6,
+ *                             +-8, +-12}): the exact integer operand of
+ *                             quest_w4a4_linear, whose Y = acc (Delta_x / 2)
+ *                             (Delta_w / 2) then equals sum Q_x Q_w Delta_x Delta_w.
+ * Both FP4 forms are supported where the rows are whole 128-value slabs with
+ * aligned codes and at most 16 slabs per row in row-RMS mode (QUEST_EUNSUPPORTED
+ * otherwise). */
 typedef enum quest_code_mode {
     QUEST_CODES_PACKED = 0,
     QUEST_CODES_INT8 = 1,
     QUEST_CODES_GEMM_OPERAND = 2,
-    QUEST_CODES_GEMM_OPERAND_E4M3 = 3
+    QUEST_CODES_GEMM_OPERAND_E4M3 = 3,
+    QUEST_CODES_FP4_PACKED = 4,
+    QUEST_CODES_FP4_OPERAND = 5
 } quest_code_mode;
 
 /* How the trust mask is stored (1 = gradient kept, 0 = gradient zeroed).
@@ -107,6 +123,22 @@ typedef enum quest_mask_mode {
  * A group with r == 0 yields Delta = 0, q = 0, yhat = 0, m = 1. Inputs holding
  * NaN or Inf propagate into that group's outputs (codes become unspecified but
  * in range); they are not checked.
+ *
+ * FP4 grid (code_mode QUEST_CODES_FP4_*, bits = 4). The pages report QuEST on an
+ * FP4 grid too and that it trails INT4 through a higher Gaussian MSE once
+ * clipping is allowed (pith.science review, "What carries the argument" and its
+ * results list); they do not spell the variant out. This library reads it as the
+ * same transform and RMS with the grid and mask replaced:
+ *     Delta = s* r                             (s* = quest_alpha_fp4(), the scale
+ *                                               of the E2M1 grid minimising the
+ *                                               MSE on N(0,1))
+ *     Q     = the E2M1 value nearest to t = y / Delta (ties to the even mantissa,
+ *             saturating at +-6; the code of a small negative t is -0)
+ *     yhat  = Q * Delta
+ *     m     = [ |t - Q| <= trust / 2 * w(t) ],  w = the width of the grid
+ *             interval that holds |t| (0.5 below 2, 1 below 4, 2 above; beyond 6
+ *             the last interval [4, 6] counts), so for trust >= 1:
+ *             m = [ |t| <= 6 + trust ].
  *
  * Arguments
  *   x          device, x_dtype [rows, ld_x] (only the first `cols` columns read);
@@ -231,6 +263,11 @@ quest_status quest_device_status(void* stream);
  * the MSE of the midrise uniform quantizer for X ~ N(0,1)); bits 1..8. Computed on
  * the host at first use. Returns NaN for an invalid bit-width. */
 double quest_alpha(int bits);
+
+/* s*, the scale of the OCP E2M1 (FP4) grid {0, +-0.5, +-1, +-1.5, +-2, +-3, +-4, +-6}
+ * that minimises E[(X - s Q(X / s))^2] for X ~ N(0,1), Q round-to-nearest onto the
+ * grid (the FP4 code modes use Delta = s* r). Computed on the host at first use. */
+double quest_alpha_fp4(void);
 
 /* Bits of the storage container of a b-bit packed code: 1, 2, 4, 4, 8, 8, 8, 8. 0 if invalid. */
 int quest_container_bits(int bits);

@@ -52,6 +52,13 @@ def test_alpha_table_matches_oracle(bits):
     assert a_lib == pytest.approx(a_ref, rel=3e-7)
 
 
+def test_alpha_fp4_matches_oracle():
+    # library: bisection on the stationarity condition of the E2M1 grid; oracle:
+    # golden section on its closed-form Gaussian MSE
+    s_ref, _ = oracle.alpha_fp4()
+    assert q.alpha_fp4() == pytest.approx(s_ref, rel=3e-7)
+
+
 def test_alpha_one_bit_exact():
     assert q.alpha(1) == pytest.approx(2 * math.sqrt(2 / math.pi), rel=1e-14)
     assert math.isnan(q.alpha(0)) and math.isnan(q.alpha(9))
@@ -65,6 +72,9 @@ def test_sizes():
     assert q.mask_bytes(16384, 2048, q.MASK_BITS) == 16384 * 2048 // 8
     assert q.mask_bytes(2, 128, q.MASK_BYTES) == 256
     assert q.codes_bytes(1, 128, 0) == 0 and q.mask_bytes(1, 12, q.MASK_BITS) == 0
+    assert q.codes_bytes(3, 256, 4, q.CODES_FP4_PACKED) == 3 * 128
+    assert q.codes_bytes(3, 256, 4, q.CODES_FP4_OPERAND) == 3 * 256
+    assert q.codes_bytes(3, 256, 3, q.CODES_FP4_PACKED) == 0
 
 
 # Invalid calls: the library must return QUEST_EINVAL / EUNSUPPORTED before any
@@ -90,6 +100,10 @@ def _qf(**kw):
     (dict(codes=FAKE + 2), 1), (dict(x_dtype=5), 1), (dict(mask_mode=3), 1),
     (dict(dequant=FAKE + 8), 1), (dict(rows=-1), 1),
     (dict(cols=16384 * 2, ld_x=16384 * 2, rms_group=16384 * 2), 2),
+    (dict(code_mode=4, bits=3), 1), (dict(code_mode=5, bits=8), 1),
+    # the FP4 grid runs only on the slab layouts: rows of 96 columns are not whole slabs
+    (dict(code_mode=4, cols=96, ld_x=96, had_block=32, rms_group=32), 2),
+    (dict(code_mode=5, cols=96, ld_x=96, had_block=32, rms_group=32), 2),
 ])
 def test_quantize_rejects_invalid_arguments(kw, status):
     assert _qf(**kw) == status
