@@ -207,6 +207,20 @@ def trust_bwd(g, mask, had: int = 128) -> np.ndarray:
     return out
 
 
+def trust_bwd_linear(g_y, w_hat, mask, had: int = 128) -> np.ndarray:
+    """Input gradient of a linear layer y = x_hat w_hat^T whose quantized input carried
+    trust mask m (pith.science review, "What carries the argument" and Figure 2
+    caption: the gradient is masked in the Hadamard domain, then transformed back):
+        G   = g_y @ w_hat            [rows, K]  (fp64; numpy's matmul)
+        g_x = H^T (m * G) / sqrt(had) per block (``trust_bwd``)
+    g_y [rows, N], w_hat [N, K] (the dequantised weights, Hadamard domain), mask [rows, K]."""
+    g_y = np.asarray(g_y, dtype=np.float64)
+    w_hat = np.asarray(w_hat, dtype=np.float64)
+    if g_y.ndim != 2 or w_hat.ndim != 2 or g_y.shape[1] != w_hat.shape[0]:
+        raise ValueError("g_y [rows, N] and w_hat [N, K] expected")
+    return trust_bwd(g_y @ w_hat, mask, had)
+
+
 def gemm_i8(a, b) -> np.ndarray:
     """acc = A @ B^T in int64 by a triple loop; A [M,K], B [N,K] int8."""
     a = np.ascontiguousarray(np.asarray(a, dtype=np.int8))

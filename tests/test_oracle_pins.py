@@ -476,3 +476,27 @@ def test_e4m3_helpers_match_torch():
     dv = e4m3_decode(allb)
     assert np.array_equal(np.isnan(tv), np.isnan(dv))
     assert np.array_equal(tv[~np.isnan(tv)], dv[~np.isnan(dv)])
+
+
+def test_trust_bwd_linear_composition_pins():
+    # the fused backward is the product followed by the pinned trust backward: pin
+    # the product by a brute-force triple loop on a tiny case, and the whole chain
+    # by two closed forms (all-ones mask and w_hat = [I; 0]: H G / sqrt(n) with G
+    # the first K columns of g_y; all-zero mask: 0)
+    g = np.random.default_rng(21)
+    gy = g.standard_normal((3, 5))
+    w = g.standard_normal((5, 16))
+    m = g.integers(0, 2, size=(3, 16)).astype(np.uint8)
+    G = np.zeros((3, 16))
+    for i in range(3):
+        for k in range(16):
+            G[i, k] = sum(gy[i, n] * w[n, k] for n in range(5))
+    assert np.allclose(oracle.trust_bwd_linear(gy, w, m, had=16), oracle.trust_bwd(G, m, had=16),
+                       rtol=0, atol=1e-12)
+    gy = g.standard_normal((4, 40))
+    eye = np.zeros((40, 32))
+    eye[:32, :32] = np.eye(32)
+    H = scipy.linalg.hadamard(32) / np.sqrt(32)
+    out = oracle.trust_bwd_linear(gy, eye, np.ones((4, 32), np.uint8), had=32)
+    assert np.allclose(out, gy[:, :32] @ H.T, rtol=0, atol=1e-12)
+    assert not oracle.trust_bwd_linear(gy, eye, np.zeros((4, 32), np.uint8), had=32).any()
