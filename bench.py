@@ -649,13 +649,16 @@ def run_configs(args):
     flush = L2Flush(dev)
     rows = []
 
-    def add(name, f, nbytes, unit_ops=None, extra=None):
+    def add(name, f, nbytes, unit_ops=None, extra=None, bf16=False):
         med, p10 = _timed(f, flush, stream)
         r = {"case": name, "median_us": round(med, 2), "p10_us": round(p10, 2), "bytes": nbytes,
              "gbs": round(nbytes / (med * 1e-6) / 1e9, 1)}
         r["frac_hbm_measured"] = round(r["gbs"] / peaks["hbm_gbs"], 4)
         r["frac_nominal_8tbs"] = round(r["gbs"] / NOMINAL_HBM_GBS, 4)
-        if unit_ops:
+        if unit_ops and bf16:
+            r["tflops"] = round(unit_ops / (med * 1e-6) / 1e12, 1)
+            r["frac_bf16_peak"] = round(r["tflops"] / peaks["bf16_tflops"], 4)
+        elif unit_ops:
             r["tops"] = round(unit_ops / (med * 1e-6) / 1e12, 1)
             r["frac_int8_peak"] = round(r["tops"] / (peaks["bf16_tflops"] * 2.0), 4)
         if extra:
@@ -758,6 +761,35 @@ def run_configs(args):
                                   y.data_ptr(), None, s)
     add("FP4 linear 16384x5632x2048 (c=2Q codes, int8 tensor cores)", f,
         R * C + NW * C + 4 * (R + NW) + 2 * R * NW, unit_ops=GEMM_OPS)
+    # the input gradient of the layer with the trust backward fused into the bf16
+    # product: w_hat from the weight quantizer's bf16 dequant, laid out [K, N] by the
+    # library's transpose, X's trust mask from config 4
+    fwq, _, _ = quant(w, 4, C, q.CODES_GEMM_OPERAND, None)
+    w_hat = torch.empty((NW, C), dtype=torch.bfloat16, device=dev)
+    cwq = torch.empty(NW * C, dtype=torch.uint8, device=dev)
+    swq = torch.empty(NW, dtype=torch.float32, device=dev)
+    q.quantize_fwd_raw(w.data_ptr(), q.BF16, NW, C, C, 4, HB, C, 1.0, q.CODES_GEMM_OPERAND, cwq.data_ptr(),
+                       swq.data_ptr(), 0, None, w_hat.data_ptr(), q.BF16, s)
+    wt = torch.empty((C, NW), dtype=torch.bfloat16, device=dev)
+    f = lambda: q.transpose_bf16_raw(w_hat.data_ptr(), NW, C, wt.data_ptr(), s)
+    add("transpose w_hat 5632x2048 bf16 (operand layout of the fused backward)", f, 4 * NW * C)
+    f()
+    gyl = inputs.layer_output_grad().to(dev)
+    gx = torch.empty((R, C), dtype=torch.bfloat16, device=dev)
+    f = lambda: q.trust_bwd_linear_raw(gyl.data_ptr(), wt.data_ptr(), mask.data_ptr(), R, NW, C, HB,
+                                       gx.data_ptr(), s)
+    add("fused input gradient 16384x5632->2048 (bf16 tcgen05, trust backward in the epilogue)", f,
+        2 * R * NW + 2 * C * NW + R * C // 8 + 2 * R * C, unit_ops=GEMM_OPS, bf16=True)
+    # comparison only (not a path of the library): the same result unfused, torch's
+    # cuBLAS bf16 product writing G to HBM, then the trust backward kernel reading it
+    G = torch.empty((R, C), dtype=torch.bfloat16, device=dev)
+    gx2 = torch.empty_like(gx)
+
+    def unfused():
+        torch.matmul(gyl, w_hat, out=G)
+        q.trust_bwd_raw(G.data_ptr(), mask.data_ptr(), q.MASK_BITS, R, C, HB, gx2.data_ptr(), s)
+    add("comparison: cuBLAS bf16 product then trust backward (unfused, G through HBM)", unfused,
+        2 * R * NW + 2 * C * NW + R * C // 8 + 2 * R * C, unit_ops=GEMM_OPS, bf16=True)
     gemm_tops = next(r["tops"] for r in rows if r["case"].startswith("cfg5 W4A4 linear"))
     q.device_status()
     probe = mma_probe(dev, gemm_tops)
@@ -788,11 +820,15 @@ def run_profile_kernels(args):
     sbg = sb[:, None].repeat(1, C // HB).contiguous()
     yg = q.w4a4_linear_grouped(a8, sag, b8, sbg)                                       # 5
     f4 = q.quantize_fwd(x, 4, code_mode=q.CODES_FP4_PACKED, mask_mode=q.MASK_BITS)    # 6
+    gyl = inputs.upstream_grad(8192, NW, seed=5).to(dev)
+    wt = q.transpose_bf16(inputs.weight_up().to(dev))                                  # 7
+    gx = q.trust_bwd_linear(gyl, wt, out["mask"][: 8192 * C // 8])                     # 8
     torch.cuda.synchronize()
     q.device_status()
     print(json.dumps({"profile_kernels": "ok", "rows": rows, "checksum": [
         float(out["scales"].sum()), float(gi.float().abs().sum()), float(op["scales"].sum()),
-        float(y.float().abs().sum()), float(yg.float().abs().sum()), float(f4["scales"].sum())]}))
+        float(y.float().abs().sum()), float(yg.float().abs().sum()), float(f4["scales"].sum()),
+        float(gx.float().abs().sum())]}))
 
 
 def main():

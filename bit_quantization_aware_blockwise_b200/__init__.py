@@ -33,6 +33,10 @@ from ._binding import (  # noqa: F401
     w4a4_linear_raw,
     w4a4_linear_grouped,
     w4a4_linear_grouped_raw,
+    trust_bwd_linear,
+    trust_bwd_linear_raw,
+    transpose_bf16,
+    transpose_bf16_raw,
     device_status,
     probe_mma_i8,
     probe_status,
@@ -43,5 +47,6 @@ __all__ = [
     "CODES_FP4_OPERAND", "MASK_BITS",
     "MASK_BYTES", "BF16", "FP32", "library_path", "load_library", "alpha", "alpha_fp4", "codes_bytes", "mask_bytes",
     "container_bits", "quantize_fwd", "trust_bwd", "w4a4_linear", "quantize_fwd_raw",
-    "trust_bwd_raw", "w4a4_linear_raw", "w4a4_linear_grouped", "w4a4_linear_grouped_raw", "device_status", "probe_mma_i8", "probe_status",
+    "trust_bwd_raw", "w4a4_linear_raw", "w4a4_linear_grouped", "w4a4_linear_grouped_raw",
+    "trust_bwd_linear", "trust_bwd_linear_raw", "transpose_bf16", "transpose_bf16_raw", "device_status", "probe_mma_i8", "probe_status",
 ]

@@ -29,6 +29,8 @@ SIGNATURES = {
     "quest_trust_bwd": (_int, [_p, _p, _int, _i64, _i64, _int, _p, _p]),
     "quest_w4a4_linear": (_int, [_p, _p, _p, _p, _i64, _i64, _i64, _p, _p, _p]),
     "quest_w4a4_linear_grouped": (_int, [_p, _p, _p, _p, _i64, _i64, _i64, _i64, _p, _p, _p]),
+    "quest_trust_bwd_linear": (_int, [_p, _p, _p, _i64, _i64, _i64, _int, _p, _p]),
+    "quest_transpose_bf16": (_int, [_p, _i64, _i64, _p, _p]),
     "quest_device_status": (_int, [_p]),
     "quest_alpha": (_f64, [_int]),
     "quest_alpha_fp4": (_f64, []),
@@ -106,6 +108,15 @@ def trust_bwd_raw(grad_out, mask, mask_mode, rows, cols, had_block, grad_in, str
 def w4a4_linear_raw(a_codes, a_scales, w_codes, w_scales, M, N, K, y, acc=None, stream=0):
     _check(load_library().quest_w4a4_linear(a_codes, a_scales, w_codes, w_scales, M, N, K, y, acc,
                                             stream), "quest_w4a4_linear")
+
+
+def trust_bwd_linear_raw(grad_y, w_hat_t, mask, M, N, K, had_block, grad_x, stream=0):
+    _check(load_library().quest_trust_bwd_linear(grad_y, w_hat_t, mask, M, N, K, had_block, grad_x, stream),
+           "quest_trust_bwd_linear")
+
+
+def transpose_bf16_raw(src, rows, cols, dst, stream=0):
+    _check(load_library().quest_transpose_bf16(src, rows, cols, dst, stream), "quest_transpose_bf16")
 
 
 def w4a4_linear_grouped_raw(a_codes, a_scales, w_codes, w_scales, M, N, K, group, y, y_f32=None, stream=0):
@@ -218,6 +229,41 @@ def trust_bwd(grad_out, mask, had_block: int = 128, mask_mode: int = MASK_BITS, 
         out = torch.empty_like(grad_out)
     trust_bwd_raw(grad_out.data_ptr(), mask.data_ptr(), mask_mode, rows, cols, had_block,
                   out.data_ptr(), _stream_handle(stream, grad_out.device))
+    return out
+
+
+def trust_bwd_linear(grad_y, w_hat_t, mask, had_block: int = 128, out=None, stream=None):
+    """grad_x = H (m * (grad_y @ w_hat_t^T)) / sqrt(128) per 128-column block: the input
+    gradient of a quantized linear layer. grad_y bf16 [M, N], w_hat_t bf16 [K, N] (the
+    dequantised weight, transposed), mask = the input's trust mask bits [M, K/8]."""
+    torch = _torch()
+    for t, n in ((grad_y, "grad_y"), (w_hat_t, "w_hat_t"), (mask, "mask")):
+        _require_cuda(t, n)
+    if grad_y.dtype != torch.bfloat16 or w_hat_t.dtype != torch.bfloat16:
+        raise QuestError("grad_y and w_hat_t must be bfloat16")
+    if grad_y.dim() != 2 or w_hat_t.dim() != 2 or not (grad_y.is_contiguous() and w_hat_t.is_contiguous()):
+        raise QuestError("grad_y and w_hat_t must be contiguous 2-D tensors")
+    M, N = grad_y.shape
+    K = w_hat_t.shape[0]
+    if w_hat_t.shape[1] != N:
+        raise QuestError("w_hat_t must be [K, N] with grad_y [M, N]")
+    if out is None:
+        out = torch.empty((M, K), dtype=torch.bfloat16, device=grad_y.device)
+    trust_bwd_linear_raw(grad_y.data_ptr(), w_hat_t.data_ptr(), mask.data_ptr(), M, N, K, had_block,
+                         out.data_ptr(), _stream_handle(stream, grad_y.device))
+    return out
+
+
+def transpose_bf16(src, out=None, stream=None):
+    """[rows, cols] bf16 -> [cols, rows] (a library kernel)."""
+    torch = _torch()
+    _require_cuda(src, "src")
+    if src.dtype != torch.bfloat16 or src.dim() != 2 or not src.is_contiguous():
+        raise QuestError("src must be a contiguous 2-D bfloat16 tensor")
+    rows, cols = src.shape
+    if out is None:
+        out = torch.empty((cols, rows), dtype=torch.bfloat16, device=src.device)
+    transpose_bf16_raw(src.data_ptr(), rows, cols, out.data_ptr(), _stream_handle(stream, src.device))
     return out
 
 

@@ -463,6 +463,47 @@ quest_status quest_w4a4_linear_grouped(const uint8_t* a_codes, const float* a_sc
     return QUEST_OK;
 }
 
+quest_status quest_trust_bwd_linear(const void* grad_y, const void* w_hat_t, const void* mask, int64_t M,
+                                    int64_t N, int64_t K, int had_block, void* grad_x, void* stream) {
+    g_last_error.clear();
+    if (M < 0 || N < 0 || K < 0) return fail(QUEST_EINVAL, "M, N and K must be >= 0");
+    if (M >= (int64_t(1) << 31) || K >= (int64_t(1) << 31) || N >= (int64_t(1) << 31))
+        return fail(QUEST_EINVAL, "M, N and K must be < 2^31");
+    if (!valid_had(had_block)) return fail(QUEST_EINVAL, "had_block must be 16, 32, 64, 128 or 256");
+    if (had_block != 128) return fail(QUEST_EUNSUPPORTED, "quest_trust_bwd_linear: had_block must be 128");
+    if (K % 128 != 0) return fail(QUEST_EINVAL, "K must be a multiple of 128");
+    if (N % 8 != 0) return fail(QUEST_EINVAL, "N must be a multiple of 8 (16-byte rows)");
+    if (M > 0 && K > 0) {
+        if (!grad_x || !mask) return fail(QUEST_EINVAL, "mask and grad_x must be non-NULL");
+        if (N > 0 && (!grad_y || !w_hat_t)) return fail(QUEST_EINVAL, "grad_y and w_hat_t must be non-NULL");
+        if (!aligned(grad_x, 16) || !aligned(mask, 16) || (N > 0 && (!aligned(grad_y, 16) || !aligned(w_hat_t, 16))))
+            return fail(QUEST_EINVAL, "grad_y, w_hat_t, mask and grad_x must be 16-byte aligned");
+    }
+    cudaError_t e = launch_trust_linear(static_cast<const uint16_t*>(grad_y), static_cast<const uint16_t*>(w_hat_t),
+                                        static_cast<const uint8_t*>(mask), M, N, K, static_cast<uint16_t*>(grad_x),
+                                        static_cast<cudaStream_t>(stream));
+    if (e == cudaErrorInvalidValue) return fail(QUEST_ECUDA, "quest_trust_bwd_linear: tensor map encoding failed");
+    if (e != cudaSuccess) return cuda_fail(e, "quest_trust_bwd_linear launch");
+    return QUEST_OK;
+}
+
+quest_status quest_transpose_bf16(const void* src, int64_t rows, int64_t cols, void* dst, void* stream) {
+    g_last_error.clear();
+    if (rows < 0 || cols < 0) return fail(QUEST_EINVAL, "rows and cols must be >= 0");
+    if (rows > 0 && cols > 0) {
+        if (!src || !dst) return fail(QUEST_EINVAL, "src and dst must be non-NULL");
+        if (!aligned(src, 2) || !aligned(dst, 2)) return fail(QUEST_EINVAL, "src and dst must be 2-byte aligned");
+        const char* a = static_cast<const char*>(src);
+        const char* b = static_cast<const char*>(dst);
+        const int64_t bytes = rows * cols * 2;
+        if (a < b + bytes && b < a + bytes) return fail(QUEST_EINVAL, "src and dst must not overlap");
+    }
+    cudaError_t e = launch_transpose_bf16(static_cast<const uint16_t*>(src), rows, cols, static_cast<uint16_t*>(dst),
+                                          static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "quest_transpose_bf16 launch");
+    return QUEST_OK;
+}
+
 quest_status quest_device_status(void* stream) {
     g_last_error.clear();
     cudaStream_t s = static_cast<cudaStream_t>(stream);

@@ -131,3 +131,8 @@ def weight_down(rows: int = HIDDEN, cols: int = MLP_WIDTH) -> torch.Tensor:
 def grad_input(rows: int = TOKENS, cols: int = HIDDEN) -> torch.Tensor:
     """bf16 [16384, 2048] upstream gradient N(0, 1e-3^2), seed 4."""
     return upstream_grad(rows, cols, seed=4)
+
+
+def layer_output_grad(rows: int = TOKENS, cols: int = MLP_WIDTH) -> torch.Tensor:
+    """bf16 [16384, 5632] gradient of the up-projection's output, N(0, 1e-3^2), seed 5."""
+    return upstream_grad(rows, cols, seed=5)

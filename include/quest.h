@@ -251,11 +251,48 @@ quest_status quest_w4a4_linear_grouped(const uint8_t* a_codes, const float* a_sc
                                        void* stream);
 
 /*
+ * quest_trust_bwd_linear -- input gradient of a QuEST linear layer with the
+ * trust backward fused into the product.
+ *
+ * Backward pass of y = x_hat w_hat^T, where x_hat is the quantized input in the
+ * Hadamard domain carrying trust mask m (pith.science review, "What carries the
+ * argument": the gradient is masked in the Hadamard domain; Figure 2 caption:
+ * the inverse transforms run on the backward pass):
+ *     G      = grad_y w_hat                              [M, K]  (fp32 accumulation)
+ *     grad_x = H (m * G) / sqrt(128) per 128-column block          (bf16, RNE)
+ * which equals quest_trust_bwd applied to G, with G kept on chip.
+ *
+ * Arguments
+ *   grad_y   device bf16 [M, N], the gradient of the layer output, row-major.
+ *   w_hat_t  device bf16 [K, N]: the dequantised weights w_hat [N, K] (Hadamard
+ *            domain, e.g. quest_quantize_fwd's `dequant` of the weight)
+ *            transposed, so that both operands run along N (see quest_transpose_bf16).
+ *   mask     device, the trust mask bits of x_hat [M, K] (QUEST_MASK_BITS layout).
+ *   M, N, K  >= 0; N a multiple of 8, K a multiple of 128; M, K < 2^31.
+ *   had_block  128 (QUEST_EUNSUPPORTED otherwise).
+ *   grad_x   device bf16 [M, K].
+ * grad_y, w_hat_t, mask and grad_x 16-byte aligned. N == 0 writes zeros.
+ * Returns QUEST_OK, QUEST_EINVAL, QUEST_EUNSUPPORTED or QUEST_ECUDA; a bounded wait
+ * that gives up is reported by quest_device_status as QUEST_ETIMEOUT.
+ */
+quest_status quest_trust_bwd_linear(const void* grad_y, const void* w_hat_t, const void* mask, int64_t M,
+                                    int64_t N, int64_t K, int had_block, void* grad_x, void* stream);
+
+/*
+ * quest_transpose_bf16 -- dst[c][r] = src[r][c] for a bf16 [rows, cols] matrix
+ * (row-major, dense); dst is [cols, rows]. Produces the w_hat_t operand of
+ * quest_trust_bwd_linear from a dequantised weight. src and dst must not overlap.
+ * Returns QUEST_OK, QUEST_EINVAL or QUEST_ECUDA.
+ */
+quest_status quest_transpose_bf16(const void* src, int64_t rows, int64_t cols, void* dst, void* stream);
+
+/*
  * quest_device_status -- synchronises `stream`, then reports (and clears) the
  * device-side status of the integer linear layer on the current device:
  * QUEST_ETIMEOUT if one of its bounded pipeline waits gave up since the last
  * call (its output is then incomplete), QUEST_OK otherwise, QUEST_ECUDA on a
- * CUDA error. The quantizer and trust kernels have no waits and never set it.
+ * CUDA error. The quantizer and trust kernels have no waits and never set it;
+ * quest_trust_bwd_linear shares the linear layer's status word.
  */
 quest_status quest_device_status(void* stream);
 

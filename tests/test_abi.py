@@ -152,3 +152,22 @@ def test_probe_rejects_invalid_arguments():
     assert lib.quest_probe_mma_i8(0, ctypes.byref(n), None) == 1
     assert lib.quest_probe_mma_i8(1 << 25, ctypes.byref(n), None) == 1
     assert lib.quest_probe_mma_i8(100, None, None) == 1
+
+
+def test_trust_bwd_linear_rejects_invalid_arguments():
+    lib = q.load_library()
+    ok = dict(gy=FAKE, wt=FAKE, mask=FAKE, M=4, N=64, K=256, had=128, gx=FAKE)
+
+    def call(**kw):
+        a = dict(ok)
+        a.update(kw)
+        return lib.quest_trust_bwd_linear(a["gy"], a["wt"], a["mask"], a["M"], a["N"], a["K"], a["had"],
+                                          a["gx"], None)
+    for kw, st in [(dict(M=-1), 1), (dict(K=200), 1), (dict(N=12), 1), (dict(had=64), 2), (dict(had=100), 1),
+                   (dict(gx=None), 1), (dict(mask=None), 1), (dict(gy=None), 1), (dict(gy=FAKE + 8), 1),
+                   (dict(mask=FAKE + 4), 1), (dict(M=1 << 31), 1)]:
+        assert call(**kw) == st, kw
+    assert call(M=0, gy=None, wt=None, mask=None, gx=None) == 0
+    assert lib.quest_transpose_bf16(FAKE, -1, 4, FAKE, None) == 1
+    assert lib.quest_transpose_bf16(FAKE, 4, 4, FAKE + 8, None) == 1      # overlapping
+    assert lib.quest_transpose_bf16(None, 0, 4, None, None) == 0
