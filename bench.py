@@ -69,8 +69,8 @@ NOMINAL_HBM_GBS = 8000.0     # nominal B200 HBM3e bandwidth (about 8 TB/s); the 
 # file is byte-identical to the one that was captured; otherwise null.
 NCU_TRAFFIC = {
     "w4a4_linear": {"source": "bit_quantization_aware_blockwise_b200/csrc/w4a4_gemm.cu",
-                    "sha256": "d8849045eb06987486af384f050ec8599ce31d380b90fedb80e6bd00f96c3ad9",
-                    "dram_read": 65884160, "dram_write": 145072384},
+                    "sha256": "747a9bf4a9f2430d821282a5f35dcb6815f80a7ff304b7c2832382999935302f",
+                    "dram_read": 66429056, "dram_write": 145147520},
 }
 
 
