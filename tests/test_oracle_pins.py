@@ -7,6 +7,7 @@ off-by-one in the grid) fails at least one of them. No expected value here comes
 from the CUDA library.
 """
 import math
+import os
 
 import numpy as np
 import pytest
@@ -500,3 +501,30 @@ def test_trust_bwd_linear_composition_pins():
     out = oracle.trust_bwd_linear(gy, eye, np.ones((4, 32), np.uint8), had=32)
     assert np.allclose(out, gy[:, :32] @ H.T, rtol=0, atol=1e-12)
     assert not oracle.trust_bwd_linear(gy, eye, np.zeros((4, 32), np.uint8), had=32).any()
+
+
+def _golden(name):
+    path = os.path.join(os.path.dirname(__file__), "golden", "pages_parameters.txt")
+    for line in open(path):
+        if line.strip() and not line.startswith("#"):
+            k, v = line.split()[:2]
+            if k == name:
+                return float(v)
+    raise KeyError(name)
+
+
+def test_one_bit_outer_trust_from_the_pages():
+    # The 1-bit runs widen the outer trust region with s* (printed by the pages), passed as
+    # T: for T >= 1 the mask keeps |t| <= 2^(b-1) + (T-1)/2 = 1.15 at b = 1. On a long
+    # N(0,1) row with whole-row RMS, t = y / (alpha_1 r) and the masked fraction is the
+    # Gaussian tail mass beyond 1.15 alpha_1.
+    s_star = _golden("outer_trust_scale_1bit")
+    assert s_star == 1.30
+    x = np.random.default_rng(13).standard_normal((1, 1 << 20))
+    o = oracle.quantize(x, bits=1, had=128, rms_group=1 << 20, trust=s_star)
+    edge = 1.0 + (s_star - 1.0) / 2.0
+    assert np.array_equal(o["mask"], (np.abs(o["t"]) <= edge).astype(np.uint8))
+    a1, _, _ = oracle.alpha(1)
+    p = 2 * scipy.stats.norm.sf(edge * a1)
+    rate = 1 - o["mask"].mean()
+    assert abs(rate - p) < 4 * math.sqrt(p * (1 - p) / x.size)

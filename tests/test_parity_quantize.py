@@ -236,3 +236,17 @@ def test_under_aligned_outputs_use_the_direct_kernel(cuda_device, bits):
 
 def test_device_status_is_clean_after_the_suite(cuda_device):
     q.device_status()
+
+
+@pytest.mark.parametrize("rms", ["group", "row"])
+def test_one_bit_outer_trust_from_the_pages(cuda_device, rms):
+    # the 1-bit runs widen the outer trust region with the factor s* the pages print
+    # (tests/golden/pages_parameters.txt), passed as the trust argument
+    from test_oracle_pins import _golden
+    s_star = _golden("outer_trust_scale_1bit")
+    x = inputs.activations(64, 2048, seed=17)
+    rg = 128 if rms == "group" else 2048
+    o = oracle.quantize(inputs.to_f64(x), bits=1, had=128, rms_group=rg, trust=s_star)
+    res = run_gpu(x, 1, rms_group=rg, trust=s_star)
+    check_all(res, o, 1)
+    assert 0 < 1 - res["mask"].mean() < 0.2
