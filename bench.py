@@ -6,9 +6,9 @@ Step (all kernels of libquest_b200.so, on one CUDA stream):
   1. quest_quantize_fwd   X [16384, 2048] bf16 -> 4-bit codes, trust mask bits,
                           per-128-group scales (the QAT forward quantizer)
   2. quest_trust_bwd      G [16384, 2048] bf16 + that mask -> grad_in bf16
-  3. quest_quantize_fwd   X -> int8 operand codes, one scale per row
-  4. quest_quantize_fwd   W_up [5632, 2048] -> int8 operand codes, one scale per row
-  5. quest_w4a4_linear    Y [16384, 5632] bf16 = dequant(cX @ cW^T)
+  3. quest_quantize_operands  X and W_up [5632, 2048] -> int8 operand codes, one
+                          scale per row (one launch for both operands of the layer)
+  4. quest_w4a4_linear    Y [16384, 5632] bf16 = dequant(cX @ cW^T)
 
 Metric: algorithmic GB/s of the whole step (bytes every kernel must move: inputs
 read once, outputs written once) and, per part, GB/s as a fraction of the
@@ -54,8 +54,7 @@ def part_bytes():
     return {
         "quantize_fwd": 2 * e + e // 2 + e // 8 + 4 * (e // HB),       # bf16 in, 4-bit codes, mask bits, scales
         "trust_bwd": 2 * e + e // 8 + 2 * e,                           # grad in, mask in, grad out
-        "quantize_operand_x": 2 * e + e + 4 * R,                       # bf16 in, int8 codes, row scales
-        "quantize_operand_w": 3 * NW * C + 4 * NW,
+        "quantize_operands": 3 * e + 4 * R + 3 * NW * C + 4 * NW,      # X and W_up: bf16 in, int8 codes, row scales
         "w4a4_linear": R * C + NW * C + 4 * (R + NW) + 2 * R * NW,     # codes, scales in, bf16 out
     }
 
@@ -258,10 +257,10 @@ class Step:
         self.cw = torch.empty((NW, C), dtype=torch.int8, device=dev)
         self.sw = torch.empty((NW, 1), dtype=torch.float32, device=dev)
         self.y = torch.empty((R, NW), dtype=torch.bfloat16, device=dev)
-        self.launches_per_step = 5
+        self.launches_per_step = 4
 
     def parts(self, stream):
-        """The five launches, each a zero-argument callable (raw C-ABI calls)."""
+        """The four launches, each a zero-argument callable (raw C-ABI calls)."""
         q, s = self.q, stream.cuda_stream
         x, g, w = self.x, self.g, self.w
         return [
@@ -270,12 +269,9 @@ class Step:
                 self.scales.data_ptr(), q.MASK_BITS, self.mask.data_ptr(), None, 0, s)),
             ("trust_bwd", lambda: q.trust_bwd_raw(
                 g.data_ptr(), self.mask.data_ptr(), q.MASK_BITS, R, C, HB, self.grad_in.data_ptr(), s)),
-            ("quantize_operand_x", lambda: q.quantize_fwd_raw(
-                x.data_ptr(), 0, R, C, C, BITS, HB, C, 1.0, q.CODES_GEMM_OPERAND, self.cx.data_ptr(),
-                self.sx.data_ptr(), q.MASK_BITS, None, None, 0, s)),
-            ("quantize_operand_w", lambda: q.quantize_fwd_raw(
-                w.data_ptr(), 0, NW, C, C, BITS, HB, C, 1.0, q.CODES_GEMM_OPERAND, self.cw.data_ptr(),
-                self.sw.data_ptr(), q.MASK_BITS, None, None, 0, s)),
+            ("quantize_operands", lambda: q.quantize_operands_raw(
+                x.data_ptr(), R, w.data_ptr(), NW, C, q.BF16, BITS, HB, q.CODES_GEMM_OPERAND, self.cx.data_ptr(),
+                self.sx.data_ptr(), self.cw.data_ptr(), self.sw.data_ptr(), s)),
             ("w4a4_linear", lambda: q.w4a4_linear_raw(
                 self.cx.data_ptr(), self.sx.data_ptr(), self.cw.data_ptr(), self.sw.data_ptr(),
                 R, NW, C, self.y.data_ptr(), None, s)),

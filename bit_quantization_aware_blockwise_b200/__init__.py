@@ -26,6 +26,8 @@ from ._binding import (  # noqa: F401
     mask_bytes,
     container_bits,
     quantize_fwd,
+    quantize_operands,
+    quantize_operands_raw,
     trust_bwd,
     w4a4_linear,
     quantize_fwd_raw,
@@ -46,7 +48,7 @@ __all__ = [
     "QuestError", "CODES_PACKED", "CODES_INT8", "CODES_GEMM_OPERAND", "CODES_GEMM_OPERAND_E4M3", "CODES_FP4_PACKED",
     "CODES_FP4_OPERAND", "MASK_BITS",
     "MASK_BYTES", "BF16", "FP32", "library_path", "load_library", "alpha", "alpha_fp4", "codes_bytes", "mask_bytes",
-    "container_bits", "quantize_fwd", "trust_bwd", "w4a4_linear", "quantize_fwd_raw",
+    "container_bits", "quantize_fwd", "quantize_operands", "quantize_operands_raw", "trust_bwd", "w4a4_linear", "quantize_fwd_raw",
     "trust_bwd_raw", "w4a4_linear_raw", "w4a4_linear_grouped", "w4a4_linear_grouped_raw",
     "trust_bwd_linear", "trust_bwd_linear_raw", "transpose_bf16", "transpose_bf16_raw", "device_status", "probe_mma_i8", "probe_status",
 ]

@@ -27,6 +27,7 @@ SIGNATURES = {
     "quest_quantize_fwd": (_int, [_p, _int, _i64, _i64, _i64, _int, _int, _i64, _f32, _int, _p, _p,
                                   _int, _p, _p, _int, _p]),
     "quest_trust_bwd": (_int, [_p, _p, _int, _i64, _i64, _int, _p, _p]),
+    "quest_quantize_operands": (_int, [_p, _i64, _p, _i64, _i64, _int, _int, _int, _int, _p, _p, _p, _p, _p]),
     "quest_w4a4_linear": (_int, [_p, _p, _p, _p, _i64, _i64, _i64, _p, _p, _p]),
     "quest_w4a4_linear_grouped": (_int, [_p, _p, _p, _p, _i64, _i64, _i64, _i64, _p, _p, _p]),
     "quest_trust_bwd_linear": (_int, [_p, _p, _p, _i64, _i64, _i64, _int, _p, _p]),
@@ -98,6 +99,12 @@ def quantize_fwd_raw(x, x_dtype, rows, cols, ld_x, bits, had_block, rms_group, t
                                              rms_group, trust, code_mode, codes, scales,
                                              mask_mode, mask, dequant, dequant_dtype, stream),
            "quest_quantize_fwd")
+
+
+def quantize_operands_raw(x, M, w, N, K, dtype, bits, had_block, code_mode, x_codes, x_scales, w_codes,
+                          w_scales, stream=0):
+    _check(load_library().quest_quantize_operands(x, M, w, N, K, dtype, bits, had_block, code_mode, x_codes,
+                                                  x_scales, w_codes, w_scales, stream), "quest_quantize_operands")
 
 
 def trust_bwd_raw(grad_out, mask, mask_mode, rows, cols, had_block, grad_in, stream=0):
@@ -214,6 +221,34 @@ def quantize_fwd(x, bits: int, had_block: int = 128, rms_group: int | None = Non
                      deq.data_ptr() if deq is not None else None, deq_dtype,
                      _stream_handle(stream, dev))
     return {"codes": codes, "scales": scales, "mask": mask, "dequant": deq}
+
+
+def quantize_operands(x, w, bits: int = 4, had_block: int = 128, code_mode: int = CODES_GEMM_OPERAND,
+                      stream=None):
+    """Operand codes of a linear layer, one RMS per row: x [M, K] and w [N, K] (same dtype,
+    contiguous) in one call. Returns ({"codes", "scales"} for x, the same for w)."""
+    torch = _torch()
+    _require_cuda(x, "x")
+    _require_cuda(w, "w")
+    if x.dim() != 2 or w.dim() != 2 or x.shape[1] != w.shape[1] or x.dtype != w.dtype:
+        raise QuestError("x [M, K] and w [N, K] of one dtype expected")
+    if not (x.is_contiguous() and w.is_contiguous()):
+        raise QuestError("x and w must be contiguous")
+    if x.dtype == torch.bfloat16:
+        dt = BF16
+    elif x.dtype == torch.float32:
+        dt = FP32
+    else:
+        raise QuestError("x and w must be bfloat16 or float32")
+    (M, K), N = x.shape, w.shape[0]
+    dev = x.device
+    cx = torch.empty(max(codes_bytes(M, K, bits, code_mode), 1), dtype=torch.uint8, device=dev)
+    cw = torch.empty(max(codes_bytes(N, K, bits, code_mode), 1), dtype=torch.uint8, device=dev)
+    sx = torch.empty(max(M, 1), dtype=torch.float32, device=dev)
+    sw = torch.empty(max(N, 1), dtype=torch.float32, device=dev)
+    quantize_operands_raw(x.data_ptr(), M, w.data_ptr(), N, K, dt, bits, had_block, code_mode, cx.data_ptr(),
+                          sx.data_ptr(), cw.data_ptr(), sw.data_ptr(), _stream_handle(stream, dev))
+    return {"codes": cx, "scales": sx[:M]}, {"codes": cw, "scales": sw[:N]}
 
 
 def trust_bwd(grad_out, mask, had_block: int = 128, mask_mode: int = MASK_BITS, out=None,

@@ -221,6 +221,8 @@ __global__ void __launch_bounds__(kThreads) quantize_tc_groups(const QuantArgs A
 // spr >= 8, so a warp holds a whole row); for spr < 8 a warp step covers 8 / spr rows.
 // As in the group kernel, the loads of a warp's next row are issued as soon as the
 // MMA has consumed the current row's registers, so they land during its arithmetic.
+// The rows of a second tensor (A.rows2 > 0, the other operand of a linear layer)
+// follow those of the first in one virtual row space, so both take one launch.
 template <int HB, int CB, int FMT, bool SAT, int SUB>
 __global__ void __launch_bounds__(kThreads, 3) quantize_tc_rows(const QuantArgs A, int spr) {
     constexpr int NBL = Blk<HB>::NBL, PPB = Blk<HB>::PPB;
@@ -229,24 +231,26 @@ __global__ void __launch_bounds__(kThreads, 3) quantize_tc_rows(const QuantArgs 
     const int r_in = SUB > 1 ? 0 : g / spr, sc0 = SUB > 1 ? g : g % spr;
     const int64_t warp0 = (int64_t(blockIdx.x) * kThreads + threadIdx.x) >> 5;
     const int64_t step = int64_t(gridDim.x) * (kThreads / 32) * rps;
+    const int64_t total = A.rows + A.rows2;
     const BFrag B = make_bfrag(lane, tmask_of<HB>());
-    auto load_row = [&](int64_t row, uint4 (&raw)[SUB][4]) {
+    auto load_row = [&](int64_t vrow, uint4 (&raw)[SUB][4]) {
+        const char* src = vrow < A.rows ? A.x + vrow * A.ld_x_bytes : A.x2 + (vrow - A.rows) * A.ld_x_bytes;
 #pragma unroll
         for (int u = 0; u < SUB; ++u) {
-            if (row < A.rows) load_slab(A.x + row * A.ld_x_bytes + int64_t(sc0 + 8 * u) * 256, t, raw[u]);
+            if (vrow < total) load_slab(src + int64_t(sc0 + 8 * u) * 256, t, raw[u]);
             else zero4(raw[u]);
         }
     };
 
     uint4 raw[SUB][4];
     load_row(warp0 * rps + r_in, raw);
-    for (int64_t r0 = warp0 * rps; r0 < A.rows; r0 += step) {
-        const int64_t row = r0 + r_in;
-        const bool valid = row < A.rows;
+    for (int64_t r0 = warp0 * rps; r0 < total; r0 += step) {
+        const int64_t vrow = r0 + r_in;
+        const bool valid = vrow < total;
         float2 P[SUB][16];
 #pragma unroll
         for (int u = 0; u < SUB; ++u) mma_stage(raw[u], B, P[u]);
-        load_row(row + step, raw);
+        load_row(vrow + step, raw);
         float v = 0.0f;
 #pragma unroll
         for (int u = 0; u < SUB; ++u) {
@@ -265,10 +269,18 @@ __global__ void __launch_bounds__(kThreads, 3) quantize_tc_rows(const QuantArgs 
         G[0] = make_group(A.c, v);
 #pragma unroll
         for (int b = 1; b < NBL; ++b) G[b] = G[0];
+        // the tensor this row belongs to
+        QuantArgs T = A;
+        int64_t row = vrow;
+        if (vrow >= A.rows) {
+            T.codes = A.codes2;
+            T.scales = A.scales2;
+            row = vrow - A.rows;
+        }
 #pragma unroll
         for (int u = 0; u < SUB; ++u)
-            emit<PPB, CB, FMT, SAT>(A, P[u], G, row, int64_t(sc0 + 8 * u) * 128, t, valid);
-        if (valid && sc0 == 0 && t == 0) A.scales[row] = G[0].delta;
+            emit<PPB, CB, FMT, SAT>(T, P[u], G, row, int64_t(sc0 + 8 * u) * 128, t, valid);
+        if (valid && sc0 == 0 && t == 0) T.scales[row] = G[0].delta;
     }
 }
 
@@ -278,7 +290,7 @@ cudaError_t launch_t(const QuantArgs& a, bool row_mode, cudaStream_t s) {
     if (row_mode) {
         const int spr = (int)(a.cols / 128);
         auto go = [&](auto fn, int64_t rows_per_warp) {
-            const int64_t warps = (a.rows + rows_per_warp - 1) / rows_per_warp;
+            const int64_t warps = (a.rows + a.rows2 + rows_per_warp - 1) / rows_per_warp;
             const int64_t cap = int64_t(sms) * max_ctas_per_sm((const void*)fn, kThreads, 0);
             const int64_t want = (warps + kThreads / 32 - 1) / (kThreads / 32);
             fn<<<(int)(want < cap ? want : cap), kThreads, 0, s>>>(a, spr);

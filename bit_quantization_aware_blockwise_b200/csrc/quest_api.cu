@@ -214,6 +214,116 @@ int max_ctas_per_sm(const void* func, int threads, size_t smem) {
 
 using namespace quest;
 
+// Validates the arguments of one quantizer call and fills the kernel arguments
+// (QuEST forward quantizer; see quest_quantize_fwd in quest.h). `a.rows` == 0 means
+// there is nothing to launch.
+static quest_status prepare_quantize(const void* x, quest_dtype x_dtype, int64_t rows, int64_t cols, int64_t ld_x,
+                              int bits, int had_block, int64_t rms_group, float trust,
+                              quest_code_mode code_mode, void* codes, float* scales,
+                              quest_mask_mode mask_mode, void* mask, void* dequant, quest_dtype dequant_dtype,
+                              QuantArgs& a, bool& row_mode, int& cb) {
+    a = QuantArgs{};
+    if (x_dtype != QUEST_BF16 && x_dtype != QUEST_FP32) return fail(QUEST_EINVAL, "x_dtype must be QUEST_BF16 or QUEST_FP32");
+    if (rows < 0) return fail(QUEST_EINVAL, "rows must be >= 0");
+    if (bits < 1 || bits > 8) return fail(QUEST_EINVAL, "bits must be in 1..8");
+    if (!valid_had(had_block)) return fail(QUEST_EINVAL, "had_block must be 16, 32, 64, 128 or 256");
+    if (cols <= 0 || cols % had_block != 0) return fail(QUEST_EINVAL, "cols must be a positive multiple of had_block");
+    if (ld_x < cols) return fail(QUEST_EINVAL, "ld_x must be >= cols");
+    if (rms_group != had_block && rms_group != cols)
+        return fail(QUEST_EINVAL, "rms_group must equal had_block or cols");
+    row_mode = rms_group != had_block;
+    if (row_mode && cols > row_mode_max_cols(had_block))
+        return fail(QUEST_EUNSUPPORTED, "rms_group == cols supports at most 16384 columns (8192 for had_block 16)");
+    if (!(trust > 0.0f) || isinf(trust)) return fail(QUEST_EINVAL, "trust must be finite and > 0");
+    if (code_mode != QUEST_CODES_PACKED && code_mode != QUEST_CODES_INT8 && code_mode != QUEST_CODES_GEMM_OPERAND &&
+        code_mode != QUEST_CODES_GEMM_OPERAND_E4M3 && !is_fp4_mode(code_mode))
+        return fail(QUEST_EINVAL, "invalid code_mode");
+    const bool fp4 = is_fp4_mode(code_mode);
+    if (fp4 && bits != 4) return fail(QUEST_EINVAL, "the FP4 (E2M1) grid needs bits == 4");
+    if (code_mode == QUEST_CODES_GEMM_OPERAND && bits > 7)
+        return fail(QUEST_EINVAL, "the GEMM operand form c = 2q+1 needs bits <= 7 to fit int8");
+    if (code_mode == QUEST_CODES_GEMM_OPERAND_E4M3 && bits > 4)
+        return fail(QUEST_EINVAL, "the E4M3 operand form holds c = 2q+1 exactly only for bits <= 4");
+    if (mask && mask_mode != QUEST_MASK_BITS && mask_mode != QUEST_MASK_BYTES)
+        return fail(QUEST_EINVAL, "invalid mask_mode");
+    if (dequant && dequant_dtype != QUEST_BF16 && dequant_dtype != QUEST_FP32)
+        return fail(QUEST_EINVAL, "invalid dequant_dtype");
+    const int esize = x_dtype == QUEST_BF16 ? 2 : 4;
+    cb = code_bits(bits, code_mode);
+    if (rows > 0) {
+        if (!x || !codes || !scales) return fail(QUEST_EINVAL, "x, codes and scales must be non-NULL");
+        if (!aligned(x, 16) || (ld_x * esize) % 16 != 0)
+            return fail(QUEST_EINVAL, "x must be 16-byte aligned with a row pitch that is a multiple of 16 bytes");
+        if (!aligned(codes, cb == 8 ? 8 : (cb == 4 ? 4 : (cb == 2 ? 2 : 1))))
+            return fail(QUEST_EINVAL, "codes is not aligned to its store width (8 bytes for int8 forms)");
+        if (!aligned(scales, 4)) return fail(QUEST_EINVAL, "scales must be 4-byte aligned");
+        if (mask && mask_mode == QUEST_MASK_BYTES && !aligned(mask, 8))
+            return fail(QUEST_EINVAL, "a byte mask must be 8-byte aligned");
+        if (dequant && !aligned(dequant, 16)) return fail(QUEST_EINVAL, "dequant must be 16-byte aligned");
+    }
+    if (rows == 0) return QUEST_OK;
+
+    const double alpha = quest_alpha(bits);
+    const int lo = -(1 << (bits - 1)), hi = (1 << (bits - 1)) - 1;
+    // the FP4 grid: Delta = s* r, mask edge 6 + T for T >= 1 (the last grid
+    // interval [4, 6] is 2 wide, so T of its halves reach 6 + T)
+    const double cd_grid = fp4 ? quest_alpha_fp4() : alpha / ldexp(1.0, bits - 1);
+    const double edge_grid = fp4 ? 6.0 + (double)trust : ldexp(1.0, bits - 1) + 0.5 * ((double)trust - 1.0);
+    a.x = static_cast<const char*>(x);
+    a.ld_x_bytes = ld_x * esize;
+    a.rows = rows;
+    a.cols = cols;
+    a.dense = ld_x == cols;
+    a.codes = static_cast<uint8_t*>(codes);
+    a.codes_row_bytes = cols * cb / 8;
+    a.scales = scales;
+    a.mask = static_cast<uint8_t*>(mask);
+    a.mask_row_bytes = mask_mode == QUEST_MASK_BITS ? cols / 8 : cols;
+    a.deq = static_cast<uint8_t*>(dequant);
+    a.deq_row_bytes = cols * (dequant_dtype == QUEST_BF16 ? 2 : 4);
+    QuantConsts& c = a.c;
+    c.c_delta = (float)cd_grid;
+    c.inv_count = (float)(1.0 / ((double)had_block * (double)rms_group));
+    c.sqrt_hb = (float)sqrt((double)had_block);
+    c.edge = (float)edge_grid;
+    c.half_trust = 0.5f * trust;
+    c.s_lo = kMagic + (float)lo;
+    c.s_hi = kMagic + (float)hi;
+    pack_constants(cb, fp4 ? QUEST_CODES_INT8 : code_mode, &c.pack_mult, &c.pack_add, &c.pack_xor);
+    c.inv_levels = (float)ldexp(1.0, -bits);
+    c.half_levels = (float)ldexp(1.0, bits - 1);
+    {
+        const double cd = cd_grid, ic = 1.0 / ((double)had_block * (double)rms_group);
+        const double shb = sqrt((double)had_block);
+        const double edge = edge_grid;
+        c.delta_k = (float)(cd * sqrt(ic));
+        c.inv_k = (float)(1.0 / (shb * cd * sqrt(ic)));
+        c.a_k = (float)(ldexp(1.0, -bits) / (shb * cd * sqrt(ic)));
+        c.thr2_k = (float)(edge * edge * shb * shb * cd * cd * ic);
+    }
+    c.sat_k = (float)(ldexp(1.0, bits) * (1.0 - ldexp(1.0, -23)));
+    c.s_mid = kMagic + (float)ldexp(1.0, bits - 1);
+    c.s_top = kMagic + (float)(ldexp(1.0, bits) - 1.0);
+    c.cell_center = (float)(0.5 - ldexp(1.0, bits - 1));
+    pack_constants_biased(cb, bits, code_mode == QUEST_CODES_GEMM_OPERAND_E4M3 ? QUEST_CODES_GEMM_OPERAND
+                                    : fp4 ? QUEST_CODES_INT8 : code_mode,
+                          &c.pack2_mult, &c.pack2_add, &c.pack2_xor);
+    c.code_fp8 = code_mode == QUEST_CODES_GEMM_OPERAND_E4M3;
+    c.grid_fp4 = code_mode == QUEST_CODES_FP4_PACKED ? 1 : (code_mode == QUEST_CODES_FP4_OPERAND ? 2 : 0);
+    {   // an 8-field word (one chunk of 8 elements) for cb <= 4
+        const uint32_t rep8 = cb == 1 ? 0xFFu : (cb == 2 ? 0x5555u : 0x11111111u);
+        const uint32_t x8 = cb == 1 ? 0xFFu : (cb == 2 ? 0xAAAAu : 0x88888888u);
+        const uint32_t off = (1u << (cb - 1)) - (1u << (bits - 1));
+        c.pack8_add = (off - kMagicBits) * rep8;
+        c.pack8_xor = x8;
+    }
+    c.trust_ge1 = trust >= 1.0f;
+    c.mask_mode = mask ? (int)mask_mode : -1;
+    c.deq_mode = dequant ? (int)dequant_dtype : -1;
+
+    return QUEST_OK;
+}
+
 extern "C" {
 
 int quest_version(void) { return 10000; }
@@ -268,110 +378,54 @@ quest_status quest_quantize_fwd(const void* x, quest_dtype x_dtype, int64_t rows
                                 float* scales, quest_mask_mode mask_mode, void* mask,
                                 void* dequant, quest_dtype dequant_dtype, void* stream) {
     g_last_error.clear();
-    if (x_dtype != QUEST_BF16 && x_dtype != QUEST_FP32) return fail(QUEST_EINVAL, "x_dtype must be QUEST_BF16 or QUEST_FP32");
-    if (rows < 0) return fail(QUEST_EINVAL, "rows must be >= 0");
-    if (bits < 1 || bits > 8) return fail(QUEST_EINVAL, "bits must be in 1..8");
-    if (!valid_had(had_block)) return fail(QUEST_EINVAL, "had_block must be 16, 32, 64, 128 or 256");
-    if (cols <= 0 || cols % had_block != 0) return fail(QUEST_EINVAL, "cols must be a positive multiple of had_block");
-    if (ld_x < cols) return fail(QUEST_EINVAL, "ld_x must be >= cols");
-    if (rms_group != had_block && rms_group != cols)
-        return fail(QUEST_EINVAL, "rms_group must equal had_block or cols");
-    const bool row_mode = rms_group != had_block;
-    if (row_mode && cols > row_mode_max_cols(had_block))
-        return fail(QUEST_EUNSUPPORTED, "rms_group == cols supports at most 16384 columns (8192 for had_block 16)");
-    if (!(trust > 0.0f) || isinf(trust)) return fail(QUEST_EINVAL, "trust must be finite and > 0");
-    if (code_mode != QUEST_CODES_PACKED && code_mode != QUEST_CODES_INT8 && code_mode != QUEST_CODES_GEMM_OPERAND &&
-        code_mode != QUEST_CODES_GEMM_OPERAND_E4M3 && !is_fp4_mode(code_mode))
-        return fail(QUEST_EINVAL, "invalid code_mode");
-    const bool fp4 = is_fp4_mode(code_mode);
-    if (fp4 && bits != 4) return fail(QUEST_EINVAL, "the FP4 (E2M1) grid needs bits == 4");
-    if (code_mode == QUEST_CODES_GEMM_OPERAND && bits > 7)
-        return fail(QUEST_EINVAL, "the GEMM operand form c = 2q+1 needs bits <= 7 to fit int8");
-    if (code_mode == QUEST_CODES_GEMM_OPERAND_E4M3 && bits > 4)
-        return fail(QUEST_EINVAL, "the E4M3 operand form holds c = 2q+1 exactly only for bits <= 4");
-    if (mask && mask_mode != QUEST_MASK_BITS && mask_mode != QUEST_MASK_BYTES)
-        return fail(QUEST_EINVAL, "invalid mask_mode");
-    if (dequant && dequant_dtype != QUEST_BF16 && dequant_dtype != QUEST_FP32)
-        return fail(QUEST_EINVAL, "invalid dequant_dtype");
-    const int esize = x_dtype == QUEST_BF16 ? 2 : 4;
-    const int cb = code_bits(bits, code_mode);
-    if (rows > 0) {
-        if (!x || !codes || !scales) return fail(QUEST_EINVAL, "x, codes and scales must be non-NULL");
-        if (!aligned(x, 16) || (ld_x * esize) % 16 != 0)
-            return fail(QUEST_EINVAL, "x must be 16-byte aligned with a row pitch that is a multiple of 16 bytes");
-        if (!aligned(codes, cb == 8 ? 8 : (cb == 4 ? 4 : (cb == 2 ? 2 : 1))))
-            return fail(QUEST_EINVAL, "codes is not aligned to its store width (8 bytes for int8 forms)");
-        if (!aligned(scales, 4)) return fail(QUEST_EINVAL, "scales must be 4-byte aligned");
-        if (mask && mask_mode == QUEST_MASK_BYTES && !aligned(mask, 8))
-            return fail(QUEST_EINVAL, "a byte mask must be 8-byte aligned");
-        if (dequant && !aligned(dequant, 16)) return fail(QUEST_EINVAL, "dequant must be 16-byte aligned");
-    }
-    if (rows == 0) return QUEST_OK;
-
-    const double alpha = quest_alpha(bits);
-    const int lo = -(1 << (bits - 1)), hi = (1 << (bits - 1)) - 1;
-    // the FP4 grid: Delta = s* r, mask edge 6 + T for T >= 1 (the last grid
-    // interval [4, 6] is 2 wide, so T of its halves reach 6 + T)
-    const double cd_grid = fp4 ? quest_alpha_fp4() : alpha / ldexp(1.0, bits - 1);
-    const double edge_grid = fp4 ? 6.0 + (double)trust : ldexp(1.0, bits - 1) + 0.5 * ((double)trust - 1.0);
     QuantArgs a;
-    a.x = static_cast<const char*>(x);
-    a.ld_x_bytes = ld_x * esize;
-    a.rows = rows;
-    a.cols = cols;
-    a.dense = ld_x == cols;
-    a.codes = static_cast<uint8_t*>(codes);
-    a.codes_row_bytes = cols * cb / 8;
-    a.scales = scales;
-    a.mask = static_cast<uint8_t*>(mask);
-    a.mask_row_bytes = mask_mode == QUEST_MASK_BITS ? cols / 8 : cols;
-    a.deq = static_cast<uint8_t*>(dequant);
-    a.deq_row_bytes = cols * (dequant_dtype == QUEST_BF16 ? 2 : 4);
-    QuantConsts& c = a.c;
-    c.c_delta = (float)cd_grid;
-    c.inv_count = (float)(1.0 / ((double)had_block * (double)rms_group));
-    c.sqrt_hb = (float)sqrt((double)had_block);
-    c.edge = (float)edge_grid;
-    c.half_trust = 0.5f * trust;
-    c.s_lo = kMagic + (float)lo;
-    c.s_hi = kMagic + (float)hi;
-    pack_constants(cb, fp4 ? QUEST_CODES_INT8 : code_mode, &c.pack_mult, &c.pack_add, &c.pack_xor);
-    c.inv_levels = (float)ldexp(1.0, -bits);
-    c.half_levels = (float)ldexp(1.0, bits - 1);
-    {
-        const double cd = cd_grid, ic = 1.0 / ((double)had_block * (double)rms_group);
-        const double shb = sqrt((double)had_block);
-        const double edge = edge_grid;
-        c.delta_k = (float)(cd * sqrt(ic));
-        c.inv_k = (float)(1.0 / (shb * cd * sqrt(ic)));
-        c.a_k = (float)(ldexp(1.0, -bits) / (shb * cd * sqrt(ic)));
-        c.thr2_k = (float)(edge * edge * shb * shb * cd * cd * ic);
-    }
-    c.sat_k = (float)(ldexp(1.0, bits) * (1.0 - ldexp(1.0, -23)));
-    c.s_mid = kMagic + (float)ldexp(1.0, bits - 1);
-    c.s_top = kMagic + (float)(ldexp(1.0, bits) - 1.0);
-    c.cell_center = (float)(0.5 - ldexp(1.0, bits - 1));
-    pack_constants_biased(cb, bits, code_mode == QUEST_CODES_GEMM_OPERAND_E4M3 ? QUEST_CODES_GEMM_OPERAND
-                                    : fp4 ? QUEST_CODES_INT8 : code_mode,
-                          &c.pack2_mult, &c.pack2_add, &c.pack2_xor);
-    c.code_fp8 = code_mode == QUEST_CODES_GEMM_OPERAND_E4M3;
-    c.grid_fp4 = code_mode == QUEST_CODES_FP4_PACKED ? 1 : (code_mode == QUEST_CODES_FP4_OPERAND ? 2 : 0);
-    {   // an 8-field word (one chunk of 8 elements) for cb <= 4
-        const uint32_t rep8 = cb == 1 ? 0xFFu : (cb == 2 ? 0x5555u : 0x11111111u);
-        const uint32_t x8 = cb == 1 ? 0xFFu : (cb == 2 ? 0xAAAAu : 0x88888888u);
-        const uint32_t off = (1u << (cb - 1)) - (1u << (bits - 1));
-        c.pack8_add = (off - kMagicBits) * rep8;
-        c.pack8_xor = x8;
-    }
-    c.trust_ge1 = trust >= 1.0f;
-    c.mask_mode = mask ? (int)mask_mode : -1;
-    c.deq_mode = dequant ? (int)dequant_dtype : -1;
-
+    bool row_mode = false;
+    int cb = 0;
+    const quest_status st = prepare_quantize(x, x_dtype, rows, cols, ld_x, bits, had_block, rms_group, trust,
+                                             code_mode, codes, scales, mask_mode, mask, dequant, dequant_dtype,
+                                             a, row_mode, cb);
+    if (st != QUEST_OK || a.rows == 0) return st;
     cudaError_t e = launch_quantize(a, x_dtype, had_block, cb, bits, row_mode, static_cast<cudaStream_t>(stream));
     if (e == cudaErrorNotSupported)
         return fail(QUEST_EUNSUPPORTED, "the E4M3 operand form and the FP4 grid need rows of whole 128-value slabs, "
                                         "aligned codes and at most 16 slabs per row in row-RMS mode");
     if (e != cudaSuccess) return cuda_fail(e, "quest_quantize_fwd launch");
+    return QUEST_OK;
+}
+
+quest_status quest_quantize_operands(const void* x, int64_t M, const void* w, int64_t N, int64_t K,
+                                     quest_dtype dtype, int bits, int had_block, quest_code_mode code_mode,
+                                     void* x_codes, float* x_scales, void* w_codes, float* w_scales,
+                                     void* stream) {
+    g_last_error.clear();
+    QuantArgs ax, aw;
+    bool rx = false, rw = false;
+    int cb = 0;
+    quest_status st = prepare_quantize(x, dtype, M, K, K, bits, had_block, K, 1.0f, code_mode, x_codes, x_scales,
+                                       QUEST_MASK_BITS, nullptr, nullptr, QUEST_BF16, ax, rx, cb);
+    if (st != QUEST_OK) return st;
+    st = prepare_quantize(w, dtype, N, K, K, bits, had_block, K, 1.0f, code_mode, w_codes, w_scales,
+                          QUEST_MASK_BITS, nullptr, nullptr, QUEST_BF16, aw, rw, cb);
+    if (st != QUEST_OK) return st;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    cudaError_t e = cudaSuccess;
+    if (ax.rows > 0 && aw.rows > 0 && rx && tc_path_ok(ax, dtype, had_block, cb, true) &&
+        tc_path_ok(aw, dtype, had_block, cb, true)) {
+        // one launch: w's rows follow x's in the row-RMS kernel
+        QuantArgs a = ax;
+        a.x2 = aw.x;
+        a.codes2 = aw.codes;
+        a.scales2 = aw.scales;
+        a.rows2 = aw.rows;
+        e = launch_quantize_tc(a, had_block, cb, bits, true, s);
+    } else {
+        if (ax.rows > 0) e = launch_quantize(ax, dtype, had_block, cb, bits, rx, s);
+        if (e == cudaSuccess && aw.rows > 0) e = launch_quantize(aw, dtype, had_block, cb, bits, rw, s);
+    }
+    if (e == cudaErrorNotSupported)
+        return fail(QUEST_EUNSUPPORTED, "the E4M3 operand form and the FP4 grid need rows of whole 128-value slabs, "
+                                        "aligned codes and at most 16 slabs per row in row-RMS mode");
+    if (e != cudaSuccess) return cuda_fail(e, "quest_quantize_operands launch");
     return QUEST_OK;
 }
 

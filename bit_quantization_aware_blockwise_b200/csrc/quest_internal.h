@@ -54,6 +54,13 @@ struct QuantArgs {
     uint8_t* deq;
     int64_t deq_row_bytes;
     QuantConsts c;
+    // Optional second tensor of the same width and constants, quantized by the
+    // same row-RMS launch after the first (rows2 == 0: none): its rows follow
+    // those of x in one virtual row space. No mask or dequant for it.
+    const char* x2;
+    uint8_t* codes2;
+    float* scales2;
+    int64_t rows2;
 };
 
 struct TrustArgs {
@@ -87,11 +94,11 @@ cudaError_t launch_w4a4(const int8_t* A, const float* sa, const int8_t* B, const
 // Reads (synchronising `stream`) and clears the integer linear layer's device
 // status word; returns its value (0 or a quest_status).
 int read_and_clear_gemm_status(cudaStream_t stream, cudaError_t* err);
-// Input gradient of the quantized linear layer with the trust backward fused in:
-// gx = H (mask * (gy wt^T)) / sqrt(128) per 128-column block (w4a4_gemm.cu).
 // dst[c][r] = src[r][c] for bf16 [rows, cols] (transpose.cu).
 cudaError_t launch_transpose_bf16(const uint16_t* src, int64_t rows, int64_t cols, uint16_t* dst,
                                   cudaStream_t stream);
+// Input gradient of the quantized linear layer with the trust backward fused in:
+// gx = H (mask * (gy wt^T)) / sqrt(128) per 128-column block (w4a4_gemm.cu).
 cudaError_t launch_trust_linear(const uint16_t* gy, const uint16_t* wt, const uint8_t* mask, int64_t M,
                                 int64_t N, int64_t K, uint16_t* gx, cudaStream_t stream);
 cudaError_t launch_w4a4_grouped(const int8_t* A, const float* sa, const int8_t* B, const float* sb,

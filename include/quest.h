@@ -166,6 +166,21 @@ quest_status quest_quantize_fwd(const void* x, quest_dtype x_dtype, int64_t rows
                                 void* dequant, quest_dtype dequant_dtype, void* stream);
 
 /*
+ * quest_quantize_operands -- both operands of a QuEST linear layer in one call:
+ * quest_quantize_fwd with rms_group = K (one RMS per row), no mask and no dequant,
+ * on x [M, K] and on w [N, K], both dense (row pitch K elements) and of one dtype.
+ * Where both tensors take the tensor-core row layout (bf16, rows of whole 128-value
+ * slabs, at most 16 slabs per row, aligned codes) the library quantizes them in a
+ * single launch, w's rows after x's; otherwise it issues the two quantizations one
+ * after the other. Outputs and errors as quest_quantize_fwd (codes in code_mode,
+ * scales fp32 [M] and [N], Delta per row); M == 0 or N == 0 skips that tensor.
+ */
+quest_status quest_quantize_operands(const void* x, int64_t M, const void* w, int64_t N, int64_t K,
+                                     quest_dtype dtype, int bits, int had_block, quest_code_mode code_mode,
+                                     void* x_codes, float* x_scales, void* w_codes, float* w_scales,
+                                     void* stream);
+
+/*
  * quest_trust_bwd -- trust-estimator backward.
  *
  * Follows pith.science review, "What carries the argument" (the gradient is

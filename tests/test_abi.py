@@ -171,3 +171,17 @@ def test_trust_bwd_linear_rejects_invalid_arguments():
     assert lib.quest_transpose_bf16(FAKE, -1, 4, FAKE, None) == 1
     assert lib.quest_transpose_bf16(FAKE, 4, 4, FAKE + 8, None) == 1      # overlapping
     assert lib.quest_transpose_bf16(None, 0, 4, None, None) == 0
+
+
+def test_quantize_operands_rejects_invalid_arguments():
+    lib = q.load_library()
+    ok = dict(x=FAKE, M=4, w=FAKE, N=8, K=256, dt=0, bits=4, had=128, mode=2, cx=FAKE, sx=FAKE, cw=FAKE, sw=FAKE)
+
+    def call(**kw):
+        a = dict(ok)
+        a.update(kw)
+        return lib.quest_quantize_operands(*a.values(), None)
+    for kw in [dict(bits=9), dict(K=200), dict(had=100), dict(mode=7), dict(x=None), dict(cw=None),
+               dict(sw=None), dict(w=FAKE + 4), dict(mode=5, bits=3), dict(dt=4)]:
+        assert call(**kw) == 1, kw
+    assert call(M=0, N=0, x=None, w=None, cx=None, sx=None, cw=None, sw=None) == 0

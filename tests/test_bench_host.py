@@ -19,6 +19,7 @@ def test_part_bytes_by_hand():
     p = bench.part_bytes()
     assert p["quantize_fwd"] == 2 * e + e // 2 + e // 8 + 4 * (e // 128)
     assert p["trust_bwd"] == int(4.125 * e)
+    assert p["quantize_operands"] == 3 * e + 4 * 16384 + 3 * 5632 * 2048 + 4 * 5632
     assert p["w4a4_linear"] == 16384 * 2048 + 5632 * 2048 + 4 * (16384 + 5632) + 2 * 16384 * 5632
     assert bench.GEMM_OPS == 2 * 16384 * 5632 * 2048
     assert 590e6 < sum(p.values()) < 595e6
