@@ -490,45 +490,59 @@ def run_e2e(args, dev, step, parts, x_cpu, g_cpu, w_cpu, flush, world):
 # ---------------------------------------------------------------------------
 # CPU oracle (cpu_baseline leg and the reference arm)
 # ---------------------------------------------------------------------------
-def oracle_sample(rows_x=256, rows_w=88, gemm_rows=16):
-    """Runs the oracle on a bounded row sample of one step; returns (seconds, bytes)."""
+def oracle_legs(rows_x=256, rows_w=88, gemm_rows=16):
+    """Runs the oracle on a bounded row sample of each leg of one step. Returns the seconds
+    each leg took and the rows it covered, per leg: the activation legs (quantize, trust
+    backward, operand quantize of X) on rows_x rows, the weight operand quantize on rows_w
+    rows, and the GEMM (with its dequantisation) on gemm_rows output rows against all
+    NW weight rows."""
     import oracle
     from bit_quantization_aware_blockwise_b200 import inputs
     x = inputs.to_f64(inputs.activation_input(rows=rows_x))
     g = inputs.to_f64(inputs.grad_input(rows=rows_x))
     w = inputs.to_f64(inputs.weight_up(rows=rows_w))
-    w_full_rows = NW
     t0 = time.perf_counter()
     o = oracle.quantize(x, bits=BITS, had=HB)
     oracle.trust_bwd(g, o["mask"], had=HB)
     ox = oracle.quantize(x, bits=BITS, had=HB, rms_group=C)
+    t1 = time.perf_counter()
     ow = oracle.quantize(w, bits=BITS, had=HB, rms_group=C)
+    t2 = time.perf_counter()
     cx = (2 * ox["q"][:gemm_rows] + 1).astype(np.int8)
     cw = (2 * ow["q"] + 1).astype(np.int8)
-    # the GEMM sample: gemm_rows output rows against all NW weight rows (codes of the
-    # sampled weight rows are tiled to the full width: the cost is the triple loop)
-    cw_full = np.resize(cw, (w_full_rows, C))
+    # the sampled weight rows' codes tiled to the full width: the cost is the triple loop
+    cw_full = np.resize(cw, (NW, C))
     acc = oracle.gemm_i8(cx, cw_full)
-    sw = np.resize(ow["scale"][:, 0], w_full_rows)
-    oracle.dequant_linear(acc, ox["scale"][:gemm_rows, 0], sw)
-    dt = time.perf_counter() - t0
-    e = rows_x * C
-    nbytes = ((2 * e + e // 2 + e // 8 + 4 * (e // HB)) + (2 * e + e // 8 + 2 * e) + (3 * e + 4 * rows_x)
-              + (3 * rows_w * C + 4 * rows_w)
-              + (gemm_rows * C + NW * C + 4 * (gemm_rows + NW) + 2 * gemm_rows * NW))
-    sample = (f"oracle on {rows_x} activation/gradient rows (quantize + trust backward + operand "
-              f"quantize), {rows_w} weight rows, and a {gemm_rows}x{NW}x{C} GEMM block; "
-              f"single-threaded C, fp64/int64")
-    return dt, nbytes, sample
+    oracle.dequant_linear(acc, ox["scale"][:gemm_rows, 0], np.resize(ow["scale"][:, 0], NW))
+    t3 = time.perf_counter()
+    return {"act": (t1 - t0, rows_x, R), "weight": (t2 - t1, rows_w, NW), "gemm": (t3 - t2, gemm_rows, R)}
+
+
+def _sample_text(rows_x, rows_w, gemm_rows, how):
+    return (f"oracle on {rows_x} of {R} activation/gradient rows (quantize + trust backward + operand "
+            f"quantize), {rows_w} of {NW} weight rows and {gemm_rows} of {R} GEMM output rows "
+            f"({gemm_rows}x{NW}x{C}); each leg's time scaled to the full step by its sampled fraction; {how}")
+
+
+def oracle_step_estimate(rows_x=256, rows_w=88, gemm_rows=16):
+    """Seconds of one full step on one core, from a bounded sample of every leg; returns
+    (seconds for a full step, bytes of a full step, seconds spent, description)."""
+    legs = oracle_legs(rows_x, rows_w, gemm_rows)
+    full = sum(t * total / rows for t, rows, total in legs.values())
+    spent = sum(t for t, _, _ in legs.values())
+    return full, sum(part_bytes().values()), spent, _sample_text(rows_x, rows_w, gemm_rows,
+                                                                  "single-threaded C, fp64/int64")
 
 
 def _oracle_shard(shape):
-    return oracle_sample(*shape)[:2]
+    legs = oracle_legs(*shape)
+    return {k: v[0] for k, v in legs.items()}
 
 
 def oracle_all_cores(rows_x, rows_w, gemm_rows):
-    """The same sample split into row shards over every host core (one process per
-    core, spawned; the oracle itself unchanged). Returns (seconds, bytes, cores)."""
+    """The same legs split into row shards over every host core (one spawned process per
+    core, the oracle itself unchanged); each leg's rate is n shards over the mean shard
+    time. Returns (seconds for a full step, bytes of a full step, wall seconds, cores)."""
     import multiprocessing as mp
     n = max(1, os.cpu_count() or 1)
     shard = (max(1, rows_x // n), max(1, rows_w // n), max(1, gemm_rows // n))
@@ -536,22 +550,27 @@ def oracle_all_cores(rows_x, rows_w, gemm_rows):
         pool.map(_oracle_shard, [(2, 2, 1)] * n)          # start-up and imports, untimed
         t0 = time.perf_counter()
         res = pool.map(_oracle_shard, [shard] * n)
-        dt = time.perf_counter() - t0
-    return dt, sum(b for _, b in res), n
+        wall = time.perf_counter() - t0
+    rows = {"act": (shard[0], R), "weight": (shard[1], NW), "gemm": (shard[2], R)}
+    full = 0.0
+    for k, (r, total) in rows.items():
+        t_mean = sum(d[k] for d in res) / n
+        full += total / (n * r / t_mean)
+    return full, sum(part_bytes().values()), wall, n
 
 
 def cpu_baseline(args):
     import oracle
     oracle.build()
-    # the full activation, gradient and weight legs and a 512-row block of the GEMM:
-    # about 10-20 s of single-threaded CPU work
-    dt, nbytes, sample = oracle_sample(rows_x=R, rows_w=NW, gemm_rows=512)
-    out = {"value": round(nbytes / dt / 1e9, 5), "unit": "GB/s", "cores": 1, "kind": "oracle",
-           "sample": sample, "seconds": round(dt, 3)}
-    dt_n, bytes_n, n = oracle_all_cores(R, NW, 512)
-    out["all_cores"] = {"value": round(bytes_n / dt_n / 1e9, 5), "unit": "GB/s", "cores": n,
-                        "seconds": round(dt_n, 3),
-                        "sample": "the same sample split into row shards, one spawned process per core"}
+    # the full activation and weight legs and a 512-row block of the GEMM: about 10-20 s
+    # of single-threaded CPU work
+    full, nbytes, spent, sample = oracle_step_estimate(rows_x=R, rows_w=NW, gemm_rows=512)
+    out = {"value": round(nbytes / full / 1e9, 5), "unit": "GB/s", "cores": 1, "kind": "oracle",
+           "sample": sample, "seconds": round(spent, 3), "seconds_per_full_step": round(full, 3)}
+    full_n, bytes_n, wall_n, n = oracle_all_cores(R, NW, 512)
+    out["all_cores"] = {"value": round(bytes_n / full_n / 1e9, 5), "unit": "GB/s", "cores": n,
+                        "seconds": round(wall_n, 3), "seconds_per_full_step": round(full_n, 3),
+                        "sample": "the same legs split into row shards, one spawned process per core"}
     return out
 
 
@@ -562,10 +581,10 @@ def run_reference(args, world, rank):
     oracle.build()
     times, nb, sample = [], 0, ""
     if args.warmup > 0:
-        oracle_sample(rows_x=64, rows_w=22, gemm_rows=4)
+        oracle_step_estimate(rows_x=64, rows_w=22, gemm_rows=4)
     for _ in range(args.steps):
-        dt, nb, sample = oracle_sample(rows_x=64, rows_w=22, gemm_rows=4)
-        times.append(dt)
+        full, nb, _, sample = oracle_step_estimate(rows_x=64, rows_w=22, gemm_rows=4)
+        times.append(full)
     ms = 1e3 * sum(times) / len(times)
     value = nb / (ms * 1e-3) / 1e9
     line = {
@@ -574,7 +593,8 @@ def run_reference(args, world, rank):
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "f64/int64 (CPU oracle)", "data": "synthetic",
         "config": {"workload": WORKLOAD, "bits": BITS, "had_block": HB,
-                   "note": "each step is a bounded row sample of the workload"},
+                   "note": "each step runs a bounded row sample of every leg of the workload and "
+                           "scales each leg's time to the full step (ms_per_step is that estimate)"},
         "cpu_baseline": {"value": round(value, 5), "unit": "GB/s", "cores": 1, "kind": "oracle",
                          "sample": sample},
         "e2e": {"value": round(value, 5), "unit": "GB/s", "h2d_bytes_per_step": 0,
