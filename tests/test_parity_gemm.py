@@ -190,3 +190,14 @@ def test_w1a1_linear_end_to_end(cuda_device):
     yv = oracle.bf16_bits_to_f64(yb)
     corr = np.sum(yv * exact) / (np.linalg.norm(yv) * np.linalg.norm(exact))
     assert corr > 0.5
+
+
+@pytest.mark.parametrize("M,N,K", [(64, 8, 131056), (200, 16, 65536)])
+def test_longest_reduction(cuda_device, M, N, K):
+    # K up to the largest the library accepts (< 131072, a multiple of 16), with codes at
+    # the b = 4 extremes so |acc| reaches K * 225: the int32 accumulator stays exact
+    a = np.full((M, K), 15, np.int8)
+    b = np.full((N, K), -15, np.int8)
+    a[1::2] = inputs.gemm_codes(M // 2, K, seed=41)
+    b[1::2] = inputs.gemm_codes(N // 2, K, seed=42)
+    check(a, b, inputs.positive_scales(M, seed=43), inputs.positive_scales(N, seed=44))
