@@ -532,6 +532,15 @@ quest_status quest_trust_bwd_linear(const void* grad_y, const void* w_hat_t, con
         if (N > 0 && (!grad_y || !w_hat_t)) return fail(QUEST_EINVAL, "grad_y and w_hat_t must be non-NULL");
         if (!aligned(grad_x, 16) || !aligned(mask, 16) || (N > 0 && (!aligned(grad_y, 16) || !aligned(w_hat_t, 16))))
             return fail(QUEST_EINVAL, "grad_y, w_hat_t, mask and grad_x must be 16-byte aligned");
+        // grad_x is written while the other three are read
+        const char* gx = static_cast<const char*>(grad_x);
+        const int64_t gx_bytes = M * K * 2;
+        auto overlaps = [&](const void* p, int64_t bytes) {
+            const char* c = static_cast<const char*>(p);
+            return c != nullptr && bytes > 0 && c < gx + gx_bytes && gx < c + bytes;
+        };
+        if (overlaps(grad_y, M * N * 2) || overlaps(w_hat_t, K * N * 2) || overlaps(mask, M * K / 8))
+            return fail(QUEST_EINVAL, "grad_x must not overlap grad_y, w_hat_t or mask");
     }
     cudaError_t e = launch_trust_linear(static_cast<const uint16_t*>(grad_y), static_cast<const uint16_t*>(w_hat_t),
                                         static_cast<const uint8_t*>(mask), M, N, K, static_cast<uint16_t*>(grad_x),

@@ -165,7 +165,8 @@ def test_trust_bwd_linear_rejects_invalid_arguments():
                                           a["gx"], None)
     for kw, st in [(dict(M=-1), 1), (dict(K=200), 1), (dict(N=12), 1), (dict(had=64), 2), (dict(had=100), 1),
                    (dict(gx=None), 1), (dict(mask=None), 1), (dict(gy=None), 1), (dict(gy=FAKE + 8), 1),
-                   (dict(mask=FAKE + 4), 1), (dict(M=1 << 31), 1)]:
+                   (dict(mask=FAKE + 4), 1), (dict(M=1 << 31), 1),
+                   (dict(gx=FAKE + 64), 1)]:                                  # grad_x overlapping grad_y
         assert call(**kw) == st, kw
     assert call(M=0, gy=None, wt=None, mask=None, gx=None) == 0
     assert lib.quest_transpose_bf16(FAKE, -1, 4, FAKE, None) == 1
