@@ -65,23 +65,31 @@ NOMINAL_HBM_GBS = 8000.0     # nominal B200 HBM3e bandwidth (about 8 TB/s); the 
 # DRAM traffic per launch of the dominant kernel, from one ncu capture of the full
 # workload (dram__bytes_read.sum + dram__bytes_write.sum, one pass; the summary is in
 # profiles/launches_hot_path_16384x2048.md). Reported only while the kernel's source
-# file is byte-identical to the one that was captured; otherwise null.
+# files are byte-identical to the ones that were captured; otherwise null.
 NCU_TRAFFIC = {
-    "w4a4_linear": {"source": "bit_quantization_aware_blockwise_b200/csrc/w4a4_gemm.cu",
-                    "sha256": "747a9bf4a9f2430d821282a5f35dcb6815f80a7ff304b7c2832382999935302f",
-                    "dram_read": 66429056, "dram_write": 145147520},
+    "w4a4_linear": {"sources": ["bit_quantization_aware_blockwise_b200/csrc/w4a4_gemm.cu",
+                                "bit_quantization_aware_blockwise_b200/csrc/tc_common.cuh"],
+                    "sha256": "c2fce9adadc06d9d12b7102f12b7cd0e4f3ddbb31af6eb9b4bcea9fabffc833d",
+                    "dram_read": 65093504, "dram_write": 146637824},
 }
 
 
-def ncu_traffic(part):
+def sources_sha256(paths):
     import hashlib
+    h = hashlib.sha256()
+    for p in paths:
+        with open(os.path.join(ROOT, p), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()
+
+
+def ncu_traffic(part):
     rec = NCU_TRAFFIC.get(part)
     if rec is None:
         return None
     try:
-        with open(os.path.join(ROOT, rec["source"]), "rb") as f:
-            if hashlib.sha256(f.read()).hexdigest() != rec["sha256"]:
-                return None
+        if sources_sha256(rec["sources"]) != rec["sha256"]:
+            return None
     except OSError:
         return None
     return rec["dram_read"] + rec["dram_write"]

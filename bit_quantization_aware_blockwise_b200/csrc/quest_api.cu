@@ -571,9 +571,16 @@ quest_status quest_device_status(void* stream) {
     g_last_error.clear();
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     cudaError_t e = cudaSuccess;
+    // every status word is read and cleared, so a later call starts clean
     const int vg = read_and_clear_gemm_status(s, &e);
     if (e != cudaSuccess) return cuda_fail(e, "quest_device_status");
+    const int vgr = read_and_clear_grouped_status(s, &e);
+    if (e != cudaSuccess) return cuda_fail(e, "quest_device_status");
+    const int vtl = read_and_clear_trust_linear_status(s, &e);
+    if (e != cudaSuccess) return cuda_fail(e, "quest_device_status");
     if (vg != 0) return fail((quest_status)vg, "a bounded device-side wait in quest_w4a4_linear gave up");
+    if (vgr != 0) return fail((quest_status)vgr, "a bounded device-side wait in quest_w4a4_linear_grouped gave up");
+    if (vtl != 0) return fail((quest_status)vtl, "a bounded device-side wait in quest_trust_bwd_linear gave up");
     return QUEST_OK;
 }
 

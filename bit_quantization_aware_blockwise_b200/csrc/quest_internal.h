@@ -91,14 +91,17 @@ cudaError_t launch_w4a4(const int8_t* A, const float* sa, const int8_t* B, const
                         int64_t M, int64_t N, int64_t K, uint16_t* y, int32_t* acc,
                         cudaStream_t stream);
 
-// Reads (synchronising `stream`) and clears the integer linear layer's device
-// status word; returns its value (0 or a quest_status).
+// Read (synchronising `stream`) and clear the device status word of the integer
+// linear layer (w4a4_gemm.cu), the grouped layer (w4a4_grouped.cu) and the fused
+// input gradient (trust_linear.cu); each returns its value (0 or a quest_status).
 int read_and_clear_gemm_status(cudaStream_t stream, cudaError_t* err);
+int read_and_clear_grouped_status(cudaStream_t stream, cudaError_t* err);
+int read_and_clear_trust_linear_status(cudaStream_t stream, cudaError_t* err);
 // dst[c][r] = src[r][c] for bf16 [rows, cols] (transpose.cu).
 cudaError_t launch_transpose_bf16(const uint16_t* src, int64_t rows, int64_t cols, uint16_t* dst,
                                   cudaStream_t stream);
 // Input gradient of the quantized linear layer with the trust backward fused in:
-// gx = H (mask * (gy wt^T)) / sqrt(128) per 128-column block (w4a4_gemm.cu).
+// gx = H (mask * (gy wt^T)) / sqrt(128) per 128-column block (trust_linear.cu).
 cudaError_t launch_trust_linear(const uint16_t* gy, const uint16_t* wt, const uint8_t* mask, int64_t M,
                                 int64_t N, int64_t K, uint16_t* gx, cudaStream_t stream);
 cudaError_t launch_w4a4_grouped(const int8_t* A, const float* sa, const int8_t* B, const float* sb,

@@ -1,0 +1,416 @@
+// Linear layer on QuEST codes with per-group scales along K (one scale per row and
+// per 128-wide K group on both operands): CTA-pair tcgen05 kind::f8f6f4 kernel on
+// E4M3 codes with a per-group TMEM round trip (see the kernel's comment).
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace quest {
+namespace {
+// Device-side status word of this file's kernels (0 = fine). Written only when a
+// bounded wait gives up; read and cleared by quest_device_status().
+__device__ int g_tc_status = 0;
+}  // namespace
+}  // namespace quest
+
+#include "tc_common.cuh"
+
+namespace quest {
+namespace {
+
+// ---------------------------------------------------------------------------
+// Per-group scales along K (one scale per row and per 128-wide K group on both
+// operands): Y[m][n] = sum_g (sa[m][g]/2)(sb[n][g]/2) * P_g[m][n], P_g the
+// product of group g's codes. The codes come as FP8 E4M3 (c = 2q + 1, odd,
+// |c| <= 15, exact in E4M3), so tcgen05 kind::f8f6f4 with fp32 accumulation
+// gives every P_g exactly (integers below 2^24) with no int -> float step.
+// CTA pairs as above, tiles of 256 x 128, one stage per group; the MMA cycles
+// four 128-column TMEM slots, one group each, and eight epilogue warps (two per
+// TMEM lane quarter, 64 columns each) fold every group into fp32 accumulators
+// held in registers: acc += P_g * (sa/2)(sb/2), two packed FMA-class
+// instructions per pair of outputs per group. A group's completion is read off
+// its stage's empty barrier (one commit per group). This layer is bounded by the
+// TMEM round trip, not the tensor cores: four slots hold about 1000 cycles of
+// MMA work per SM, while a slot takes about 3000 cycles from the commit to its
+// release by both CTAs' epilogues (clock64 counters on B200).
+
+constexpr int kGThreads = 320;               // producer, MMA, 8 epilogue warps
+constexpr int kGEpiThreads = 256;
+constexpr int kGBN = 128;                    // output columns per pair tile
+constexpr int kGStages = 6;
+constexpr int kGSlots = 4;                   // TMEM slots of kGBN columns
+constexpr int kGroup = 128;                  // K group = one stage
+constexpr int kGScaleBlock = 16;             // groups of scales staged at a time
+constexpr uint32_t kGStageA = 128 * BK, kGStageB = (kGBN / 2) * BK;   // per CTA
+constexpr uint32_t kGTxBytes = 2 * (kGStageA + kGStageB);
+constexpr uint32_t kGSmemA = 0;
+constexpr uint32_t kGSmemB = kGSmemA + kGStages * kGStageA;
+constexpr uint32_t kGScaleBytes = kGScaleBlock * (kGBN + 128) * 4;    // one block: sb [16][128], sa [16][128]
+constexpr uint32_t kGSmemS = kGSmemB + kGStages * kGStageB;           // two blocks (double buffer)
+constexpr uint32_t kGSmemC = kGSmemS + 2 * kGScaleBytes;              // 8 warps x 2 x 2 KB
+constexpr uint32_t kGCBytes = 32 * 32 * 2;                            // 32 rows x 32 bf16
+constexpr uint32_t kGSmemBar = kGSmemC + 8 * 2 * kGCBytes;
+constexpr uint32_t kGNumBars = 2 * kGStages + kGSlots + 1;
+constexpr uint32_t kGSmemTmemSlot = kGSmemBar + kGNumBars * 8;
+constexpr uint32_t kGSmemAbort = kGSmemTmemSlot + 4;
+constexpr uint32_t kGSmemUsed = kGSmemAbort + 4;
+constexpr uint32_t kGSmemTotal = kGSmemUsed + 1024;
+static_assert(kGSmemTotal <= 227 * 1024, "grouped kernel shared memory");
+static_assert(kGSlots * kGBN == kTmemCols, "TMEM slots");
+static_assert(kGSlots < kGStages, "the epilogue reads group completion off the stage barriers");
+
+// kind::f8f6f4, f32 accumulator, A and B E4M3, K-major, M = 256, N = 128.
+constexpr uint32_t kIdescGrouped = (1u << 4) | (0u << 7) | (0u << 10) | (uint32_t(kGBN >> 3) << 17) |
+                                   (uint32_t(256 >> 4) << 24);
+
+__device__ __forceinline__ void tc_mma_f8_pair(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
+                                               uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::2.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(adesc), "l"(bdesc), "r"(kIdescGrouped), "r"(accumulate)
+        : "memory");
+}
+
+__device__ __forceinline__ void gepi_bar() {
+    asm volatile("bar.sync 1, %0;" ::"n"(kGEpiThreads) : "memory");
+}
+__device__ __forceinline__ bool gepi_any(bool pred) {
+    uint32_t out;
+    asm volatile(
+        "{\n\t.reg .pred p, q;\n\t"
+        "setp.ne.u32 p, %1, 0;\n\t"
+        "bar.red.or.pred q, 1, %2, p;\n\t"
+        "selp.u32 %0, 1, 0, q;\n\t}"
+        : "=r"(out)
+        : "r"((uint32_t)pred), "n"(kGEpiThreads)
+        : "memory");
+    return out != 0;
+}
+
+__device__ __forceinline__ void cp_async4(uint32_t dst, const float* src, bool valid) {
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;" ::"r"(dst), "l"(src), "r"(valid ? 4 : 0)
+                 : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
+
+struct GroupedParams {
+    const float* sa;    // [M, K / 128]
+    const float* sb;    // [N, K / 128]
+    float* y32;         // optional fp32 copy of Y [M, N]
+    int M, N, K;
+    int num_m2, num_n, num_k;   // 256-row pair tiles, 128-column tiles, K groups
+};
+
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGThreads, 1)
+w4a4_gemm_grouped_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_b,
+                         const __grid_constant__ CUtensorMap map_y, const GroupedParams p) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const uint32_t sbase = smem_u32(smem);
+    const uint32_t bar_full = sbase + kGSmemBar;                 // [kGStages], used in the even CTA
+    const uint32_t bar_empty = bar_full + 8 * kGStages;          // [kGStages]
+    const uint32_t bar_tempty = bar_empty + 8 * kGStages;        // [kGSlots], used in the even CTA
+    const uint32_t bar_drain = bar_tempty + 8 * kGSlots;
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + kGSmemAbort);
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kGSmemTmemSlot);
+    // scale blocks (double buffer): [16][128] sb[n0 + n][g0 + gg], then [16][128] sa[m0 + r][g0 + gg]
+    float* s_sc = reinterpret_cast<float*>(smem + kGSmemS);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const uint32_t rank = cluster_rank();
+    const bool even = rank == 0;
+    const int pair = blockIdx.x >> 1, num_pairs = gridDim.x >> 1;
+    const int num_tiles = p.num_m2 * p.num_n;
+    const int G = p.num_k;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kGStages; ++s) {
+            mbar_init(bar_full + 8 * s, 1);
+            mbar_init(bar_empty + 8 * s, 1);
+        }
+        for (int b = 0; b < kGSlots; ++b) mbar_init(bar_tempty + 8 * b, 16);   // 8 epilogue warps x 2 CTAs
+        mbar_init(bar_drain, 1);
+        *abort_flag = 0;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&map_a)) : "memory");
+        asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&map_b)) : "memory");
+        asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&map_y)) : "memory");
+    }
+    if (warp == 1) {
+        asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                         smem_u32(tmem_slot)),
+                     "r"(kTmemCols)
+                     : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+    }
+    tc_fence_before();
+    cluster_sync();
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+
+    if (warp == 0) {
+        // ------------------------------------------------------------ TMA producer (both CTAs)
+        if (lane == 0) {
+            const uint32_t full_even = map_to_rank(bar_full, 0);
+            uint32_t stage = 0, phase = 0;
+            uint64_t issued = 0;
+            bool ok = true;
+            for (int tile = pair; tile < num_tiles && ok; tile += num_pairs) {
+                const int m0 = (tile % p.num_m2) * 256 + 128 * int(rank);
+                const int n0 = (tile / p.num_m2) * kGBN + (kGBN / 2) * int(rank);
+                for (int kb = 0; kb < G; ++kb) {
+                    if (!mbar_wait(bar_empty + 8 * stage, phase ^ 1, abort_flag)) { ok = false; break; }
+                    if (even) mbar_arrive_expect_tx(bar_full + 8 * stage, kGTxBytes);
+                    const uint32_t fb = full_even + 8 * stage;
+                    tma_load_2d_pair(sbase + kGSmemA + stage * kGStageA, &map_a, kb * BK, m0, fb);
+                    tma_load_2d_pair(sbase + kGSmemB + stage * kGStageB, &map_b, kb * BK, n0, fb);
+                    ++issued;
+                    if (++stage == kGStages) { stage = 0; phase ^= 1; }
+                }
+            }
+            if (!ok && even) {
+                const uint64_t n = issued < kGStages ? issued : kGStages;
+                for (uint64_t i = issued - n; i < issued; ++i) {
+                    const uint32_t st = uint32_t(i % kGStages), ph = uint32_t((i / kGStages) & 1);
+                    const uint64_t t0 = global_timer_ns();
+                    while (!mbar_try_wait(bar_full + 8 * st, ph) && global_timer_ns() - t0 < kWaitLimitNs) {
+                    }
+                }
+            } else if (!ok) {
+                const uint64_t t0 = global_timer_ns();
+                while (global_timer_ns() - t0 < 10000000ull) {
+                }
+            }
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------------------ MMA issuer (even CTA)
+        if (even && lane == 0) {
+            uint32_t stage = 0, phase = 0;
+            uint32_t gcount = 0;   // groups issued so far: TMEM slot = gcount % kGSlots
+            bool ok = true;
+            for (int tile = pair; tile < num_tiles && ok; tile += num_pairs) {
+                for (int kb = 0; kb < G; ++kb, ++gcount) {
+                    const uint32_t slot = gcount % kGSlots, sphase = (gcount / kGSlots) & 1;
+                    if (!mbar_wait(bar_tempty + 8 * slot, sphase ^ 1, abort_flag)) { ok = false; break; }
+                    if (!mbar_wait(bar_full + 8 * stage, phase, abort_flag)) { ok = false; break; }
+                    tc_fence_after();
+                    const uint32_t d_tmem = tmem_base + slot * kGBN;
+                    const uint32_t a_addr = sbase + kGSmemA + stage * kGStageA;
+                    const uint32_t b_addr = sbase + kGSmemB + stage * kGStageB;
+#pragma unroll
+                    for (int kk = 0; kk < BK / kUmmaK; ++kk) {
+                        tc_mma_f8_pair(d_tmem, smem_desc_k128(a_addr + kk * kUmmaK),
+                                       smem_desc_k128(b_addr + kk * kUmmaK), kk != 0);
+                    }
+                    // frees the stage in both CTAs and, the same event, marks this group's
+                    // partials ready for the epilogue (which waits on this stage's barrier)
+                    tc_commit_pair_mc(bar_empty + 8 * stage);
+                    if (++stage == kGStages) { stage = 0; phase ^= 1; }
+                }
+            }
+            tc_commit_pair(bar_drain);
+            const uint64_t t0 = global_timer_ns();
+            while (!mbar_try_wait(bar_drain, 0) && global_timer_ns() - t0 < kWaitLimitNs) {
+            }
+        }
+    } else {
+        // ------------------------------------------------------------ epilogue (warps 2..9, both CTAs)
+        const int et = threadIdx.x - 64;                   // 0..255
+        const int ew = et >> 5;                            // epilogue warp 0..7
+        const int quarter = warp & 3;                      // TMEM lanes 32*quarter .. +31
+        const int half = ew >> 2;                          // columns 64*half .. +63 of the tile
+        const int row_in_tile = quarter * 32 + lane;
+        const uint32_t lane_addr = uint32_t(quarter * 32) << 16;
+        const uint32_t tempty_even = map_to_rank(bar_tempty, 0);
+        const uint32_t stg0 = sbase + kGSmemC + uint32_t(ew) * 2 * kGCBytes;
+        const int Gs = p.K / kGroup;                       // scale columns per row
+        // issue the copies of scale block (tile, g0) into buffer b: transposed to [group][column]
+        auto prefetch = [&](int tile, int g0, int b) {
+            if (tile < num_tiles) {
+                const int pm0 = (tile % p.num_m2) * 256 + 128 * int(rank), pn0 = (tile / p.num_m2) * kGBN;
+                const int nb = (G - g0) < kGScaleBlock ? (G - g0) : kGScaleBlock;
+                const uint32_t base = sbase + kGSmemS + uint32_t(b) * kGScaleBytes;
+#pragma unroll
+                for (int k = 0; k < kGScaleBlock * kGBN / kGEpiThreads; ++k) {
+                    const int i = et + k * kGEpiThreads, n = i / kGScaleBlock, gg = i % kGScaleBlock;
+                    const bool v = gg < nb && pn0 + n < p.N;
+                    cp_async4(base + 4 * (gg * kGBN + n), p.sb + (v ? int64_t(pn0 + n) * Gs + g0 + gg : 0), v);
+                }
+#pragma unroll
+                for (int k = 0; k < kGScaleBlock * 128 / kGEpiThreads; ++k) {
+                    const int i = et + k * kGEpiThreads, r = i / kGScaleBlock, gg = i % kGScaleBlock;
+                    const bool v = gg < nb && pm0 + r < p.M;
+                    cp_async4(base + 4 * (kGScaleBlock * kGBN + gg * 128 + r),
+                              p.sa + (v ? int64_t(pm0 + r) * Gs + g0 + gg : 0), v);
+                }
+            }
+            cp_async_commit();
+        };
+        uint32_t gcount = 0;
+        int cbuf = 0, sbuf = 0;
+        bool aborted = false;
+        prefetch(pair, 0, 0);
+        for (int tile = pair; tile < num_tiles && !aborted; tile += num_pairs) {
+            const int m0 = (tile % p.num_m2) * 256 + 128 * int(rank), n0 = (tile / p.num_m2) * kGBN;
+            float2 acc[32];   // columns 64*half + 2j, +1
+#pragma unroll
+            for (int j = 0; j < 32; ++j) acc[j] = make_float2(0.0f, 0.0f);
+            for (int g = 0; g < G; ++g, ++gcount) {
+                if ((g % kGScaleBlock) == 0) {
+                    // a thread whose wait gave up stops the whole epilogue here (uniform exit)
+                    if (gepi_any(aborted)) break;
+                    // this block's scales have landed, and every thread is done with the other
+                    // buffer: start copying the next block into it (one tile ahead at most)
+                    cp_async_wait_all();
+                    gepi_bar();
+                    if (g + kGScaleBlock < G) prefetch(tile, g + kGScaleBlock, sbuf ^ 1);
+                    else prefetch(tile + num_pairs, 0, sbuf ^ 1);
+                }
+                // group gcount's MMAs are complete when its stage's empty barrier completes
+                // that use; the epilogue trails the MMA by at most kGSlots < kGStages groups,
+                // so the parity cannot alias
+                const uint32_t slot = gcount % kGSlots;
+                const uint32_t gst = gcount % kGStages, gph = (gcount / kGStages) & 1;
+                if (!mbar_wait(bar_empty + 8 * gst, gph, abort_flag)) aborted = true;
+                if (aborted) continue;   // later waits return at once (abort flag); exit at the next check
+                tc_fence_after();
+                const uint32_t t_grp = tmem_base + lane_addr + slot * kGBN + 64 * half;
+                uint32_t r0[32], r1[32];
+                QUEST_TMEM_LD32(t_grp, r0);
+                QUEST_TMEM_LD32(t_grp + 32, r1);
+                tmem_wait_ld();
+                // the group's partials are in registers: hand the slot back
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive_remote(tempty_even + 8 * slot);
+                // (sa/2)(sb/2): the factor 1/4 rides on the row scale
+                const float* sblk = s_sc + sbuf * (kGScaleBytes / 4);
+                const float sx = 0.25f * sblk[kGScaleBlock * kGBN + (g % kGScaleBlock) * 128 + row_in_tile];
+                const float4* sw4 = reinterpret_cast<const float4*>(sblk + (g % kGScaleBlock) * kGBN + 64 * half);
+                if ((g % kGScaleBlock) == kGScaleBlock - 1 || g == G - 1) sbuf ^= 1;   // next block, other buffer
+#pragma unroll
+                for (int q4 = 0; q4 < 16; ++q4) {
+                    const float4 w4 = sw4[q4];
+                    const uint32_t* r = q4 < 8 ? r0 : r1;
+                    const int i = (q4 & 7) * 4;
+                    const float2 w01 = __fmul2_rn(make_float2(sx, sx), make_float2(w4.x, w4.y));
+                    const float2 w23 = __fmul2_rn(make_float2(sx, sx), make_float2(w4.z, w4.w));
+                    acc[2 * q4] = __ffma2_rn(make_float2(__uint_as_float(r[i]), __uint_as_float(r[i + 1])), w01,
+                                             acc[2 * q4]);
+                    acc[2 * q4 + 1] = __ffma2_rn(make_float2(__uint_as_float(r[i + 2]), __uint_as_float(r[i + 3])),
+                                                 w23, acc[2 * q4 + 1]);
+                }
+            }
+            if (gepi_any(aborted)) { aborted = true; break; }
+            // ---- output: this warp's 32 rows x 64 columns, in 2 chunks of 32 columns
+            const int m = m0 + row_in_tile;
+            if (p.y32 != nullptr && m < p.M) {
+                float* yrow = p.y32 + int64_t(m) * p.N + n0 + 64 * half;
+#pragma unroll
+                for (int j = 0; j < 32; ++j) {
+                    const int n = n0 + 64 * half + 2 * j;
+                    if (n < p.N) yrow[2 * j] = acc[j].x;
+                    if (n + 1 < p.N) yrow[2 * j + 1] = acc[j].y;
+                }
+            }
+            const uint32_t swz = (lane >> 1) & 3;
+#pragma unroll
+            for (int c = 0; c < 2; ++c) {
+                if (lane == 0) bulk_wait_read_le1();   // the buffer used two chunks ago is free
+                __syncwarp();
+                const uint32_t stg = stg0 + cbuf * kGCBytes + lane * 64;
+#pragma unroll
+                for (int q16 = 0; q16 < 4; ++q16) {
+                    uint32_t w[4];
+#pragma unroll
+                    for (int h = 0; h < 4; ++h) {
+                        const float2 v = acc[c * 16 + q16 * 4 + h];
+                        __nv_bfloat162 hb = __floats2bfloat162_rn(v.x, v.y);
+                        w[h] = *reinterpret_cast<uint32_t*>(&hb);
+                    }
+                    asm volatile("st.shared.v4.u32 [%0], {%1,%2,%3,%4};" ::"r"(stg + ((q16 ^ swz) << 4)),
+                                 "r"(w[0]), "r"(w[1]), "r"(w[2]), "r"(w[3])
+                                 : "memory");
+                }
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) {
+                    tma_store_2d(&map_y, stg0 + cbuf * kGCBytes, n0 + 64 * half + c * kChunkCols, m0 + 32 * quarter);
+                    bulk_commit();
+                }
+                cbuf ^= 1;
+            }
+        }
+        cp_async_wait_all();   // no copy may still target shared memory at exit
+        if (lane == 0) bulk_wait_all();
+    }
+
+    tc_fence_before();
+    cluster_sync();
+    if (warp == 1) {
+        tc_fence_after();
+        asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem_base), "r"(kTmemCols)
+                     : "memory");
+    }
+}
+
+cudaError_t launch_grouped(const int8_t* A, const float* sa, const int8_t* B, const float* sb, int64_t M,
+                           int64_t N, int64_t K, uint16_t* y, float* y32, cudaStream_t stream) {
+    CUtensorMap ma, mb, my;
+    if (!make_map_2d(&ma, CU_TENSOR_MAP_DATA_TYPE_UINT8, A, K, M, K, BK, 128, CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !make_map_2d(&mb, CU_TENSOR_MAP_DATA_TYPE_UINT8, B, K, N, K, BK, kGBN / 2, CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !make_map_2d(&my, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, y, N, M, N * 2, kChunkCols, 32,
+                     CU_TENSOR_MAP_SWIZZLE_64B))
+        return cudaErrorInvalidValue;
+    GroupedParams p;
+    p.sa = sa; p.sb = sb; p.y32 = y32;
+    p.M = (int)M; p.N = (int)N; p.K = (int)K;
+    p.num_m2 = (int)((M + 255) / 256);
+    p.num_n = (int)((N + kGBN - 1) / kGBN);
+    p.num_k = (int)(K / kGroup);
+    static thread_local int attr_dev = -1;
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (attr_dev != dev) {
+        cudaError_t e = cudaFuncSetAttribute(w4a4_gemm_grouped_kernel,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize, kGSmemTotal);
+        if (e != cudaSuccess) return e;
+        attr_dev = dev;
+    }
+    const int tiles = p.num_m2 * p.num_n;
+    const int pairs = pair_clusters(dev, (const void*)w4a4_gemm_grouped_kernel, kGThreads, kGSmemTotal);
+    const int grid_pairs = tiles < pairs ? tiles : pairs;
+    w4a4_gemm_grouped_kernel<<<2 * grid_pairs, kGThreads, kGSmemTotal, stream>>>(ma, mb, my, p);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_w4a4_grouped(const int8_t* A, const float* sa, const int8_t* B, const float* sb,
+                                int64_t M, int64_t N, int64_t K, uint16_t* y, float* y32,
+                                cudaStream_t stream) {
+    if (M == 0 || N == 0) return cudaSuccess;
+    if (K == 0) {
+        const int64_t n = M * N;
+        if (y32) cudaMemsetAsync(y32, 0, size_t(n) * sizeof(float), stream);
+        return launch_zero_fill(y, nullptr, n, stream);
+    }
+    return launch_grouped(A, sa, B, sb, M, N, K, y, y32, stream);
+}
+
+int read_and_clear_grouped_status(cudaStream_t stream, cudaError_t* err) {
+    int v = 0, zero = 0;
+    cudaError_t e = cudaMemcpyFromSymbolAsync(&v, g_tc_status, sizeof(int), 0, cudaMemcpyDeviceToHost, stream);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(stream);
+    if (e == cudaSuccess && v != 0)
+        e = cudaMemcpyToSymbolAsync(g_tc_status, &zero, sizeof(int), 0, cudaMemcpyHostToDevice, stream);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(stream);
+    *err = e;
+    return v;
+}
+
+}  // namespace quest
