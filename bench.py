@@ -338,12 +338,11 @@ def run_b200(args, world, rank, local):
     part_ms = {n: [] for n in names}
     step_ms = []
     for k in range(args.steps):
-        tot = 0.0
         for i, n in enumerate(names):
-            t = evs[k][i][0].elapsed_time(evs[k][i][1])
-            part_ms[n].append(t)
-            tot += t
-        step_ms.append(tot)
+            part_ms[n].append(evs[k][i][0].elapsed_time(evs[k][i][1]))
+        # the step: from the start of its first kernel to the end of its last, on the
+        # device (the gaps between its launches included, the L2 flush before it not)
+        step_ms.append(evs[k][0][0].elapsed_time(evs[k][-1][1]))
     my_ms = sum(step_ms) / args.steps
     ms = dist_max(my_ms, world)
     pbytes = part_bytes()
@@ -397,6 +396,9 @@ def run_b200(args, world, rank, local):
         "config": {"workload": WORKLOAD, "bits": BITS, "had_block": HB,
                    "shapes": {"x": [R, C], "grad": [R, C], "w_up": [NW, C], "y": [R, NW]},
                    "l2": L2Flush.describe,
+                   "timing": "per step: CUDA events on the launching stream from the start of the "
+                             "step's first kernel to the end of its last (launch gaps included), "
+                             "mean over the timed steps, max over ranks",
                    "parallelism": f"dp{world} (independent row shards, no collective)"},
         "parts": breakdown,
         "w4a4_tops": breakdown["w4a4_linear"]["tops"],
