@@ -319,8 +319,11 @@ def run_b200(args, world, rank, local):
     torch.cuda.synchronize()
     q.device_status()
 
-    evs = [[[torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)]
-            for _ in parts] for _ in range(args.steps)]
+    # the timed steps: one CUDA event before the step's first kernel and one after its
+    # last, nothing recorded between its kernels (so each kernel's launch may overlap
+    # the tail of the one before it)
+    span = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+            for _ in range(args.steps)]
     clocks = ClockSampler(local)
     dist_barrier(world)
     torch.cuda.synchronize()
@@ -328,21 +331,31 @@ def run_b200(args, world, rank, local):
     t0 = time.perf_counter()
     for k in range(args.steps):
         flush.zero_()  # L2 flush between timed steps (outside the per-step events)
-        one_step(evs[k])
+        span[k][0].record(stream)
+        one_step()
+        span[k][1].record(stream)
     torch.cuda.synchronize()
     wall = time.perf_counter() - t0
     clocks.stop()
     dist_barrier(world)
     q.device_status()
+    step_ms = [a.elapsed_time(b) for a, b in span]
 
+    # the per-kernel breakdown: the same steps again with events around every kernel
+    evs = [[[torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)]
+            for _ in parts] for _ in range(args.steps)]
+    dist_barrier(world)
+    torch.cuda.synchronize()
+    for k in range(args.steps):
+        flush.zero_()
+        one_step(evs[k])
+    torch.cuda.synchronize()
+    dist_barrier(world)
+    q.device_status()
     part_ms = {n: [] for n in names}
-    step_ms = []
     for k in range(args.steps):
         for i, n in enumerate(names):
             part_ms[n].append(evs[k][i][0].elapsed_time(evs[k][i][1]))
-        # the step: from the start of its first kernel to the end of its last, on the
-        # device (the gaps between its launches included, the L2 flush before it not)
-        step_ms.append(evs[k][0][0].elapsed_time(evs[k][-1][1]))
     my_ms = sum(step_ms) / args.steps
     ms = dist_max(my_ms, world)
     pbytes = part_bytes()
@@ -396,9 +409,10 @@ def run_b200(args, world, rank, local):
         "config": {"workload": WORKLOAD, "bits": BITS, "had_block": HB,
                    "shapes": {"x": [R, C], "grad": [R, C], "w_up": [NW, C], "y": [R, NW]},
                    "l2": L2Flush.describe,
-                   "timing": "per step: CUDA events on the launching stream from the start of the "
-                             "step's first kernel to the end of its last (launch gaps included), "
-                             "mean over the timed steps, max over ranks",
+                   "timing": "per step: one CUDA event on the launching stream before the step's "
+                             "first kernel and one after its last (launch gaps included, nothing "
+                             "recorded between kernels), mean over the timed steps, max over ranks; "
+                             "parts: a second pass with events around every kernel",
                    "parallelism": f"dp{world} (independent row shards, no collective)"},
         "parts": breakdown,
         "w4a4_tops": breakdown["w4a4_linear"]["tops"],
@@ -839,7 +853,8 @@ def run_profile_kernels(args):
     torch.cuda.synchronize()
     out = q.quantize_fwd(x, BITS, mask_mode=q.MASK_BITS)                               # 1
     gi = q.trust_bwd(g, out["mask"])                                                   # 2
-    op = q.quantize_fwd(x, BITS, rms_group=C, code_mode=q.CODES_GEMM_OPERAND, mask_mode=None)  # 3
+    w_up = inputs.weight_up().to(dev)
+    op, _ = q.quantize_operands(x, w_up, BITS, HB, q.CODES_GEMM_OPERAND)                 # 3
     y = q.w4a4_linear(a, sa, b, sb)                                                    # 4
     a8, b8 = a.float().to(torch.float8_e4m3fn), b.float().to(torch.float8_e4m3fn)
     sag = sa[:, None].repeat(1, C // HB).contiguous()

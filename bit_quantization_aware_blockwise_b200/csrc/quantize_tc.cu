@@ -182,6 +182,8 @@ constexpr int kDepth = 1;
 
 template <int HB, int CB, int FMT, bool SAT>
 __global__ void __launch_bounds__(kThreads) quantize_tc_groups(const QuantArgs A) {
+    pdl_wait();      // the previous kernel on the stream has completed
+    pdl_trigger();   // the next one may be scheduled as CTAs of this one leave
     const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
     const int64_t spr = A.cols / 128;
     const int64_t total = A.rows * spr;
@@ -225,6 +227,8 @@ __global__ void __launch_bounds__(kThreads) quantize_tc_groups(const QuantArgs A
 // follow those of the first in one virtual row space, so both take one launch.
 template <int HB, int CB, int FMT, bool SAT, int SUB>
 __global__ void __launch_bounds__(kThreads, 3) quantize_tc_rows(const QuantArgs A, int spr) {
+    pdl_wait();      // the previous kernel on the stream has completed
+    pdl_trigger();   // the next one may be scheduled as CTAs of this one leave
     constexpr int NBL = Blk<HB>::NBL, PPB = Blk<HB>::PPB;
     const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
     const int rps = SUB > 1 ? 1 : 8 / spr;          // rows per warp step
@@ -287,26 +291,25 @@ __global__ void __launch_bounds__(kThreads, 3) quantize_tc_rows(const QuantArgs 
 template <int HB, int CB, int FMT, bool SAT>
 cudaError_t launch_t(const QuantArgs& a, bool row_mode, cudaStream_t s) {
     const int sms = sm_count();
+    // grids never exceed the resident capacity (persistent, grid-stride)
     if (row_mode) {
         const int spr = (int)(a.cols / 128);
         auto go = [&](auto fn, int64_t rows_per_warp) {
             const int64_t warps = (a.rows + a.rows2 + rows_per_warp - 1) / rows_per_warp;
             const int64_t cap = int64_t(sms) * max_ctas_per_sm((const void*)fn, kThreads, 0);
             const int64_t want = (warps + kThreads / 32 - 1) / (kThreads / 32);
-            fn<<<(int)(want < cap ? want : cap), kThreads, 0, s>>>(a, spr);
+            return launch_pdl(fn, dim3((unsigned)(want < cap ? want : cap)), dim3(kThreads), 0, s, a, spr);
         };
-        if (spr == 16) go(quantize_tc_rows<HB, CB, FMT, SAT, 2>, 1);
-        else if (spr == 8) go(quantize_tc_rows<HB, CB, FMT, SAT, 1>, 1);
-        else go(quantize_tc_rows<HB, CB, FMT, SAT, 1>, 8 / spr);
-    } else {
-        const int64_t slabs = a.rows * (a.cols / 128);
-        const int64_t warps = (slabs + 7) / 8;
-        auto fn = quantize_tc_groups<HB, CB, FMT, SAT>;
-        const int64_t cap = int64_t(sms) * max_ctas_per_sm((const void*)fn, kThreads, 0);
-        const int64_t want = (warps + kThreads / 32 - 1) / (kThreads / 32);
-        fn<<<(int)(want < cap ? want : cap), kThreads, 0, s>>>(a);
+        if (spr == 16) return go(quantize_tc_rows<HB, CB, FMT, SAT, 2>, 1);
+        if (spr == 8) return go(quantize_tc_rows<HB, CB, FMT, SAT, 1>, 1);
+        return go(quantize_tc_rows<HB, CB, FMT, SAT, 1>, 8 / spr);
     }
-    return cudaGetLastError();
+    const int64_t slabs = a.rows * (a.cols / 128);
+    const int64_t warps = (slabs + 7) / 8;
+    auto fn = quantize_tc_groups<HB, CB, FMT, SAT>;
+    const int64_t cap = int64_t(sms) * max_ctas_per_sm((const void*)fn, kThreads, 0);
+    const int64_t want = (warps + kThreads / 32 - 1) / (kThreads / 32);
+    return launch_pdl(fn, dim3((unsigned)(want < cap ? want : cap)), dim3(kThreads), 0, s, a);
 }
 
 template <int HB, int CB, int FMT>

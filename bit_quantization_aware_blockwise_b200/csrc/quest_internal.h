@@ -112,4 +112,32 @@ cudaError_t launch_w4a4_grouped(const int8_t* A, const float* sa, const int8_t* 
 int sm_count();
 int max_ctas_per_sm(const void* func, int threads, size_t smem);
 
+// Programmatic dependent launch. A kernel launched by launch_pdl may be scheduled
+// while the kernel before it on the stream is still finishing (once every CTA of
+// that kernel has called pdl_trigger() or exited); it must call pdl_wait() before
+// it reads or writes global memory: pdl_wait() returns once the previous kernel
+// has completed and its writes are visible. The kernels of the hot path call
+// pdl_wait() and then pdl_trigger() before their first global access, so the
+// launch and prologue of the next kernel overlap the tail of the current one.
+#ifdef __CUDACC__
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+#endif
+
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
+                              Args... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
+}
+
 }  // namespace quest

@@ -76,6 +76,8 @@ __device__ __forceinline__ void mask_chunk(uint4& w, uint32_t m) {
 
 template <int HB>
 __global__ void __launch_bounds__(kThreads) trust_tc_kernel(const TrustArgs a) {
+    pdl_wait();      // the previous kernel on the stream (the mask's producer) has completed
+    pdl_trigger();   // the next one may be scheduled as CTAs of this one leave
     const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
     const int64_t total = a.rows * (a.cols / 128);
     const int64_t warp0 = (int64_t(blockIdx.x) * kThreads + threadIdx.x) >> 5;
@@ -121,8 +123,7 @@ cudaError_t launch_hb(const TrustArgs& a, cudaStream_t stream) {
     auto fn = trust_tc_kernel<HB>;
     const int64_t cap = int64_t(sm_count()) * max_ctas_per_sm((const void*)fn, kThreads, 0);
     const int64_t want = (warps + kThreads / 32 - 1) / (kThreads / 32);
-    fn<<<(int)(want < cap ? want : cap), kThreads, 0, stream>>>(a);
-    return cudaGetLastError();
+    return launch_pdl(fn, dim3((unsigned)(want < cap ? want : cap)), dim3(kThreads), 0, stream, a);
 }
 
 }  // namespace tc

@@ -348,6 +348,10 @@ w4a4_gemm_pair_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_co
     cluster_sync();   // barrier initialisation and the TMEM address are visible across the pair
     tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
+    // the prologue above touched no global memory: wait here for the kernel that
+    // produced the operand codes, then let the next kernel be scheduled
+    pdl_wait();
+    pdl_trigger();
 
     if (warp == 0) {
         // ------------------------------------------------------------ TMA producer (both CTAs)
@@ -525,8 +529,8 @@ cudaError_t launch_pair(const int8_t* A, const float* sa, const int8_t* B, const
     const int tiles = p.num_m2 * p.num_n;
     const int pairs = pair_clusters(dev, (const void*)w4a4_gemm_pair_kernel, kThreads, kPSmemTotal);
     const int grid_pairs = tiles < pairs ? tiles : pairs;
-    w4a4_gemm_pair_kernel<<<2 * grid_pairs, kThreads, kPSmemTotal, stream>>>(ma, mb, my, p);
-    return cudaGetLastError();
+    return launch_pdl(w4a4_gemm_pair_kernel, dim3(2 * grid_pairs), dim3(kThreads), kPSmemTotal, stream, ma, mb, my,
+                      p);
 }
 
 }  // namespace
