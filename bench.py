@@ -69,8 +69,8 @@ NOMINAL_HBM_GBS = 8000.0     # nominal B200 HBM3e bandwidth (about 8 TB/s); the 
 NCU_TRAFFIC = {
     "w4a4_linear": {"sources": ["bit_quantization_aware_blockwise_b200/csrc/w4a4_gemm.cu",
                                 "bit_quantization_aware_blockwise_b200/csrc/tc_common.cuh"],
-                    "sha256": "c2fce9adadc06d9d12b7102f12b7cd0e4f3ddbb31af6eb9b4bcea9fabffc833d",
-                    "dram_read": 65093504, "dram_write": 146637824},
+                    "sha256": "bf7189f0aed2174798abfe645287e9756496f22aef2b5a106c455f2a32cb1e49",
+                    "dram_read": 65594624, "dram_write": 147340928},
 }
 
 

@@ -131,6 +131,8 @@ __device__ __forceinline__ void group_consts(const QuantConsts& c, float ss, flo
 // bounds are warp-uniform so every shuffle has all 32 lanes.
 template <typename Tin, int HB, int CB>
 __global__ void __launch_bounds__(kThreads) quantize_groups_kernel(const QuantArgs a) {
+    pdl_wait();      // the previous kernel on the stream has completed
+    pdl_trigger();   // the next one may be scheduled as CTAs of this one leave
     using S = TeamShape<HB>;
     constexpr int K = S::K, LPB = S::LPB, TPW = 32 / LPB;
     constexpr int kElem = sizeof(Tin);
@@ -185,6 +187,8 @@ __global__ void __launch_bounds__(kThreads) quantize_groups_kernel(const QuantAr
 // registers, so that the whole row is read once. Row sums meet in shared memory.
 template <typename Tin, int HB, int CB, int P>
 __global__ void __launch_bounds__(kThreads) quantize_rows_kernel(const QuantArgs a, int wpr) {
+    pdl_wait();      // the previous kernel on the stream has completed
+    pdl_trigger();   // the next one may be scheduled as CTAs of this one leave
     using S = TeamShape<HB>;
     constexpr int K = S::K, LPB = S::LPB, TPW = 32 / LPB;
     constexpr int kElem = sizeof(Tin);
@@ -261,8 +265,7 @@ cudaError_t launch_groups(const QuantArgs& a, cudaStream_t stream) {
     auto fn = quantize_groups_kernel<Tin, HB, CB>;
     const int64_t cap = int64_t(sm_count()) * max_ctas_per_sm((const void*)fn, kThreads, 0);
     const int grid = (int)(want < cap ? want : cap);
-    fn<<<grid, kThreads, 0, stream>>>(a);
-    return cudaGetLastError();
+    return launch_pdl(fn, dim3((unsigned)grid), dim3(kThreads), 0, stream, a);
 }
 
 template <typename Tin, int HB, int CB>
@@ -281,10 +284,9 @@ cudaError_t launch_rows(const QuantArgs& a, cudaStream_t stream) {
     const int64_t cap = int64_t(sm_count()) * max_ctas_per_sm(fnp, kThreads, 0);
     const int grid = (int)(want < cap ? want : cap);
     if (one_pass)
-        quantize_rows_kernel<Tin, HB, CB, 1><<<grid, kThreads, 0, stream>>>(a, wpr);
-    else
-        quantize_rows_kernel<Tin, HB, CB, 2><<<grid, kThreads, 0, stream>>>(a, wpr);
-    return cudaGetLastError();
+        return launch_pdl(quantize_rows_kernel<Tin, HB, CB, 1>, dim3((unsigned)grid), dim3(kThreads), 0, stream, a,
+                          wpr);
+    return launch_pdl(quantize_rows_kernel<Tin, HB, CB, 2>, dim3((unsigned)grid), dim3(kThreads), 0, stream, a, wpr);
 }
 
 template <typename Tin, int HB>

@@ -256,6 +256,8 @@ __device__ __forceinline__ void block_sums(const float2 (&P)[32], float (&ss)[32
 
 template <typename Tin, int HB, int CB, int FMT, bool SAT>
 __global__ void __launch_bounds__(kThreads, Pipe<Tin>::kMinBlocks) quantize_hs_groups(const QuantArgs A) {
+    pdl_wait();      // the previous kernel on the stream has completed
+    pdl_trigger();   // the next one may be scheduled as CTAs of this one leave
     constexpr int PPB = (HB >= 128 ? 128 : HB) / 4;   // pairs of one block in this lane
     constexpr int BPL = 32 / PPB;
     const int lane = threadIdx.x & 31, h = lane & 1, pw = lane >> 1;
@@ -318,6 +320,8 @@ __global__ void __launch_bounds__(kThreads, Pipe<Tin>::kMinBlocks) quantize_hs_g
 
 template <typename Tin, int HB, int CB, int FMT, bool SAT>
 __global__ void __launch_bounds__(kThreads, Pipe<Tin>::kMinBlocks) quantize_hs_rows(const QuantArgs A, int spr) {
+    pdl_wait();      // the previous kernel on the stream has completed
+    pdl_trigger();   // the next one may be scheduled as CTAs of this one leave
     constexpr int PPB = (HB >= 128 ? 128 : HB) / 4;
     constexpr int BPL = 32 / PPB;
     const int lane = threadIdx.x & 31, h = lane & 1;
@@ -374,16 +378,15 @@ cudaError_t launch_t(const QuantArgs& a, bool row_mode, cudaStream_t s) {
         auto fn = quantize_hs_rows<Tin, HB, CB, FMT, SAT>;
         const int64_t cap = int64_t(sms) * max_ctas_per_sm((const void*)fn, kThreads, 0);
         const int64_t want = (warps + kThreads / 32 - 1) / (kThreads / 32);
-        fn<<<(int)(want < cap ? want : cap), kThreads, 0, s>>>(a, spr);
+        return launch_pdl(fn, dim3((unsigned)(want < cap ? want : cap)), dim3(kThreads), 0, s, a, spr);
     } else {
         const int64_t slabs = a.rows * (a.cols / 128);
         const int64_t warps = (slabs + 15) / 16;
         auto fn = quantize_hs_groups<Tin, HB, CB, FMT, SAT>;
         const int64_t cap = int64_t(sms) * max_ctas_per_sm((const void*)fn, kThreads, 0);
         const int64_t want = (warps + kThreads / 32 - 1) / (kThreads / 32);
-        fn<<<(int)(want < cap ? want : cap), kThreads, 0, s>>>(a);
+        return launch_pdl(fn, dim3((unsigned)(want < cap ? want : cap)), dim3(kThreads), 0, s, a);
     }
-    return cudaGetLastError();
 }
 
 template <typename Tin, int HB, int CB, int FMT>

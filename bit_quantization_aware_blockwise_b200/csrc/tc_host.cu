@@ -14,6 +14,8 @@ namespace {
 
 // Writes zeros (K == 0: the empty sum).
 __global__ void zero_fill_kernel(uint16_t* y, int32_t* acc, int64_t n) {
+    pdl_wait();      // the previous kernel on the stream has completed
+    pdl_trigger();   // the next one may be scheduled as CTAs of this one leave
     for (int64_t i = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; i < n;
          i += int64_t(gridDim.x) * blockDim.x) {
         y[i] = 0;
@@ -88,8 +90,7 @@ cudaError_t launch_zero_fill(uint16_t* y, int32_t* acc, int64_t n, cudaStream_t 
     int64_t blocks = (n + 255) / 256;
     if (blocks > 4096) blocks = 4096;
     if (blocks < 1) return cudaSuccess;
-    zero_fill_kernel<<<(int)blocks, 256, 0, stream>>>(y, acc, n);
-    return cudaGetLastError();
+    return launch_pdl(zero_fill_kernel, dim3((unsigned)blocks), dim3(256), 0, stream, y, acc, n);
 }
 
 }  // namespace quest

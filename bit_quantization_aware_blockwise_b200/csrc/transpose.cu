@@ -16,6 +16,8 @@ constexpr int kT = 32, kRowsPerPass = 8;
 __global__ void __launch_bounds__(kT * kRowsPerPass) transpose_bf16_kernel(const uint16_t* __restrict__ src,
                                                                           int64_t rows, int64_t cols,
                                                                           uint16_t* __restrict__ dst) {
+    pdl_wait();      // the previous kernel on the stream has completed
+    pdl_trigger();   // the next one may be scheduled as CTAs of this one leave
     __shared__ uint16_t tile[kT][kT + 1];
     const int64_t tr = (rows + kT - 1) / kT, tc = (cols + kT - 1) / kT;
     const int tx = threadIdx.x, ty = threadIdx.y;
@@ -44,6 +46,8 @@ constexpr int kT2 = 64;
 __global__ void __launch_bounds__(32 * kRowsPerPass) transpose_bf16x2_kernel(const uint32_t* __restrict__ src,
                                                                             int64_t rows, int64_t cols,
                                                                             uint32_t* __restrict__ dst) {
+    pdl_wait();      // the previous kernel on the stream has completed
+    pdl_trigger();   // the next one may be scheduled as CTAs of this one leave
     __shared__ uint16_t tile[kT2][kT2 + 2];
     const int64_t tr = (rows + kT2 - 1) / kT2, tc = (cols + kT2 - 1) / kT2;
     const int tx = threadIdx.x, ty = threadIdx.y;
@@ -79,14 +83,13 @@ cudaError_t launch_transpose_bf16(const uint16_t* src, int64_t rows, int64_t col
     if (rows % 2 == 0 && cols % 2 == 0 && (reinterpret_cast<uintptr_t>(src) & 3) == 0 &&
         (reinterpret_cast<uintptr_t>(dst) & 3) == 0) {
         const int64_t tiles = ((rows + kT2 - 1) / kT2) * ((cols + kT2 - 1) / kT2);
-        transpose_bf16x2_kernel<<<(int)(tiles < cap ? tiles : cap), dim3(32, kRowsPerPass), 0, stream>>>(
-            reinterpret_cast<const uint32_t*>(src), rows, cols, reinterpret_cast<uint32_t*>(dst));
-        return cudaGetLastError();
+        return launch_pdl(transpose_bf16x2_kernel, dim3((unsigned)(tiles < cap ? tiles : cap)), dim3(32, kRowsPerPass),
+                          0, stream, reinterpret_cast<const uint32_t*>(src), rows, cols,
+                          reinterpret_cast<uint32_t*>(dst));
     }
     const int64_t tiles = ((rows + kT - 1) / kT) * ((cols + kT - 1) / kT);
-    transpose_bf16_kernel<<<(int)(tiles < cap ? tiles : cap), dim3(kT, kRowsPerPass), 0, stream>>>(src, rows, cols,
-                                                                                                 dst);
-    return cudaGetLastError();
+    return launch_pdl(transpose_bf16_kernel, dim3((unsigned)(tiles < cap ? tiles : cap)), dim3(kT, kRowsPerPass), 0,
+                      stream, src, rows, cols, dst);
 }
 
 }  // namespace quest

@@ -44,6 +44,8 @@ __device__ __forceinline__ uint32_t ld_mask_bytes8(const uint8_t* p) {
 
 template <int HB>
 __global__ void __launch_bounds__(kThreads) trust_bwd_kernel(const TrustArgs a) {
+    pdl_wait();      // the previous kernel on the stream has completed
+    pdl_trigger();   // the next one may be scheduled as CTAs of this one leave
     using S = TeamShape<HB>;
     constexpr int K = S::K, LPB = S::LPB, TPW = 32 / LPB;
     const int lane = threadIdx.x & 31, sub = lane % LPB;
@@ -94,8 +96,7 @@ cudaError_t launch_hb(const TrustArgs& a, cudaStream_t stream) {
     auto fn = trust_bwd_kernel<HB>;
     const int64_t cap = int64_t(sm_count()) * max_ctas_per_sm((const void*)fn, kThreads, 0);
     const int grid = (int)(want < cap ? want : cap);
-    fn<<<grid, kThreads, 0, stream>>>(a);
-    return cudaGetLastError();
+    return launch_pdl(fn, dim3((unsigned)grid), dim3(kThreads), 0, stream, a);
 }
 
 }  // namespace

@@ -119,6 +119,10 @@ trust_linear_pair_kernel(const __grid_constant__ CUtensorMap map_a, const __grid
     cluster_sync();
     tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
+    // the prologue above touched no global memory: wait here for the previous
+    // kernel on the stream, then let the next kernel be scheduled
+    pdl_wait();
+    pdl_trigger();
 
     if (warp == 0) {
         // ------------------------------------------------------------ TMA producer (both CTAs)
@@ -304,8 +308,8 @@ cudaError_t launch_trust_linear_pair(const uint16_t* gy, const uint16_t* wt, con
     const int tiles = p.num_m2 * p.num_n;
     const int pairs = pair_clusters(dev, (const void*)trust_linear_pair_kernel, kThreads, kPSmemTotal);
     const int grid_pairs = tiles < pairs ? tiles : pairs;
-    trust_linear_pair_kernel<<<2 * grid_pairs, kThreads, kPSmemTotal, stream>>>(ma, mb, my, p);
-    return cudaGetLastError();
+    return launch_pdl(trust_linear_pair_kernel, dim3(2 * grid_pairs), dim3(kThreads), kPSmemTotal, stream, ma, mb,
+                      my, p);
 }
 
 }  // namespace

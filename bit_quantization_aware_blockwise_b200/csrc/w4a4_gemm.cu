@@ -122,6 +122,10 @@ w4a4_gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constan
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
+    // the prologue above touched no global memory: wait here for the previous
+    // kernel on the stream, then let the next kernel be scheduled
+    pdl_wait();
+    pdl_trigger();
 
     if (warp == 0) {
         // ------------------------------------------------------------ TMA producer
@@ -568,8 +572,7 @@ cudaError_t launch_w4a4(const int8_t* A, const float* sa, const int8_t* B, const
     const int tiles = p.num_m * p.num_n;
     const int sms = sm_count();
     const int grid = tiles < sms ? tiles : sms;
-    w4a4_gemm_kernel<<<grid, kThreads, kSmemTotal, stream>>>(ma, mb, my, p);
-    return cudaGetLastError();
+    return launch_pdl(w4a4_gemm_kernel, dim3(grid), dim3(kThreads), kSmemTotal, stream, ma, mb, my, p);
 }
 
 int read_and_clear_gemm_status(cudaStream_t stream, cudaError_t* err) {

@@ -151,6 +151,10 @@ w4a4_gemm_grouped_kernel(const __grid_constant__ CUtensorMap map_a, const __grid
     cluster_sync();
     tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
+    // the prologue above touched no global memory: wait here for the previous
+    // kernel on the stream, then let the next kernel be scheduled
+    pdl_wait();
+    pdl_trigger();
 
     if (warp == 0) {
         // ------------------------------------------------------------ TMA producer (both CTAs)
@@ -384,8 +388,8 @@ cudaError_t launch_grouped(const int8_t* A, const float* sa, const int8_t* B, co
     const int tiles = p.num_m2 * p.num_n;
     const int pairs = pair_clusters(dev, (const void*)w4a4_gemm_grouped_kernel, kGThreads, kGSmemTotal);
     const int grid_pairs = tiles < pairs ? tiles : pairs;
-    w4a4_gemm_grouped_kernel<<<2 * grid_pairs, kGThreads, kGSmemTotal, stream>>>(ma, mb, my, p);
-    return cudaGetLastError();
+    return launch_pdl(w4a4_gemm_grouped_kernel, dim3(2 * grid_pairs), dim3(kGThreads), kGSmemTotal, stream, ma, mb,
+                      my, p);
 }
 
 }  // namespace
