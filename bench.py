@@ -727,46 +727,46 @@ def run_configs(args):
             + (deq.numel() * deq.element_size() if deq is not None else 0)
         return f, nbytes, (codes, scales, mask)
 
-    # config 1: fp32 256 x 512, int8 codes, fp32 dequant, byte mask
+    # the fp32 256 x 512 N(0,1) tensor: int8 codes, fp32 dequant, byte mask
     x1 = inputs.smoke_input().to(dev)
     f, nb, _ = quant(x1, 4, HB, q.CODES_INT8, q.MASK_BYTES, q.FP32)
-    add("cfg1 quantize fp32 256x512 b4 int8+fp32 deq+byte mask", f, nb)
-    # config 2: activations 16384 x 2048
+    add("quantize fp32 256x512 N(0,1) b4 int8 codes+fp32 deq+byte mask", f, nb)
+    # the activations 16384 x 2048
     x2 = inputs.activation_input().to(dev)
     for bits in (1, 2, 3, 4, 8):
         f, nb, _ = quant(x2, bits, HB, q.CODES_PACKED, q.MASK_BITS)
-        add(f"cfg2 quantize 16384x2048 b{bits} codes+mask", f, nb)
+        add(f"quantize activations 16384x2048 b{bits} codes+mask", f, nb)
     f, nb, _ = quant(x2, 4, HB, q.CODES_PACKED, q.MASK_BITS, q.BF16)
-    add("cfg2 quantize 16384x2048 b4 codes+mask+bf16 yhat", f, nb)
-    # config 3: weights, with the CUDA-graph batch over rotated buffers
+    add("quantize activations 16384x2048 b4 codes+mask+bf16 yhat", f, nb)
+    # the weights, with the CUDA-graph batch over rotated buffers
     for wname, wt in (("W_up 5632x2048", inputs.weight_up()), ("W_down 2048x5632", inputs.weight_down())):
         w = wt.to(dev)
         for bits in (1, 4):
             f, nb, _ = quant(w, bits, HB, q.CODES_PACKED, q.MASK_BITS)
             sets = [quant(w.clone(), bits, HB, q.CODES_PACKED, q.MASK_BITS)[0] for _ in range(16)]
             g_us = _graph_us(lambda fn: fn, sets, stream)
-            add(f"cfg3 quantize {wname} b{bits} codes+mask", f, nb,
+            add(f"quantize {wname} b{bits} codes+mask", f, nb,
                 extra={"graph_us_per_launch": round(g_us, 2),
                        "graph_gbs": round(nb / (g_us * 1e-6) / 1e9, 1)})
             del sets
-    # config 4: trust backward with config 2's b = 4 mask
+    # trust backward of the 16384 x 2048 gradient with the activations' b = 4 mask
     fq, _, (codes, scales, mask) = quant(x2, 4, HB, q.CODES_PACKED, q.MASK_BITS)
     fq()
     g = inputs.grad_input().to(dev)
     gi = torch.empty_like(g)
     f = lambda: q.trust_bwd_raw(g.data_ptr(), mask.data_ptr(), q.MASK_BITS, R, C, HB, gi.data_ptr(), s)
-    add("cfg4 trust backward 16384x2048", f, 4 * R * C + R * C // 8)
-    # config 5: operand codes (one RMS per row) and the linear layer
+    add("trust backward 16384x2048", f, 4 * R * C + R * C // 8)
+    # the linear layer's operand codes (one RMS per row) and the layer
     fx, nbx, (cx, sx, _) = quant(x2, 4, C, q.CODES_GEMM_OPERAND, None)
-    add("cfg5 operand quantize X 16384x2048 (row RMS)", fx, nbx)
+    add("operand quantize X 16384x2048 (row RMS)", fx, nbx)
     w = inputs.weight_up().to(dev)
     fw, nbw, (cw, sw, _) = quant(w, 4, C, q.CODES_GEMM_OPERAND, None)
-    add("cfg5 operand quantize W_up 5632x2048 (row RMS)", fw, nbw)
+    add("operand quantize W_up 5632x2048 (row RMS)", fw, nbw)
     fx(); fw()
     y = torch.empty((R, NW), dtype=torch.bfloat16, device=dev)
     f = lambda: q.w4a4_linear_raw(cx.data_ptr(), sx.data_ptr(), cw.data_ptr(), sw.data_ptr(), R, NW, C,
                                   y.data_ptr(), None, s)
-    add("cfg5 W4A4 linear 16384x5632x2048", f, R * C + NW * C + 4 * (R + NW) + 2 * R * NW, unit_ops=GEMM_OPS)
+    add("W4A4 linear 16384x5632x2048", f, R * C + NW * C + 4 * (R + NW) + 2 * R * NW, unit_ops=GEMM_OPS)
     # the 1-bit path: b = 1 operand codes (c in {-1, +1}) through the same GEMM
     fx1, nbx1, (cx1, sx1, _) = quant(x2, 1, C, q.CODES_GEMM_OPERAND, None)
     fw1, nbw1, (cw1, sw1, _) = quant(w, 1, C, q.CODES_GEMM_OPERAND, None)
@@ -803,7 +803,7 @@ def run_configs(args):
         R * C + NW * C + 4 * (R + NW) + 2 * R * NW, unit_ops=GEMM_OPS)
     # the input gradient of the layer with the trust backward fused into the bf16
     # product: w_hat from the weight quantizer's bf16 dequant, laid out [K, N] by the
-    # library's transpose, X's trust mask from config 4
+    # library's transpose, X's trust mask from the trust backward case above
     fwq, _, _ = quant(w, 4, C, q.CODES_GEMM_OPERAND, None)
     w_hat = torch.empty((NW, C), dtype=torch.bfloat16, device=dev)
     cwq = torch.empty(NW * C, dtype=torch.uint8, device=dev)
@@ -830,7 +830,7 @@ def run_configs(args):
         q.trust_bwd_raw(G.data_ptr(), mask.data_ptr(), q.MASK_BITS, R, C, HB, gx2.data_ptr(), s)
     add("comparison: cuBLAS bf16 product then trust backward (unfused, G through HBM)", unfused,
         2 * R * NW + 2 * C * NW + R * C // 8 + 2 * R * C, unit_ops=GEMM_OPS, bf16=True)
-    gemm_tops = next(r["tops"] for r in rows if r["case"].startswith("cfg5 W4A4 linear"))
+    gemm_tops = next(r["tops"] for r in rows if r["case"].startswith("W4A4 linear"))
     q.device_status()
     probe = mma_probe(dev, gemm_tops)
     print(json.dumps({"configs": rows, "int8_mma_probe": probe, "peaks": peaks}), flush=True)
