@@ -30,7 +30,9 @@ namespace {
 // shared-memory ring, barriers and TMEM accumulators are the same. The epilogue
 // thread that owns an accumulator row (one TMEM lane) holds a whole 128-column
 // block in registers: the mask and the 128-point transform are register work with
-// no exchange, and G never reaches HBM.
+// no exchange, and G never reaches HBM. Tiles run output-column-fastest: the pairs in
+// flight share a few 256-row blocks of grad_y (which, at 16384 x 5632 bf16, is larger
+// than L2) and all of w_hat_t, so grad_y streams from HBM about once.
 constexpr uint32_t kIdescBf16Pair = (1u << 4)     // D: fp32
                                   | (1u << 7)     // A: bf16
                                   | (1u << 10)    // B: bf16
@@ -132,8 +134,8 @@ trust_linear_pair_kernel(const __grid_constant__ CUtensorMap map_a, const __grid
             uint64_t issued = 0;
             bool ok = true;
             for (int tile = pair; tile < num_tiles && ok; tile += num_pairs) {
-                const int m0 = (tile % p.num_m2) * 256 + 128 * int(rank);
-                const int k0 = (tile / p.num_m2) * BN + 128 * int(rank);
+                const int m0 = (tile / p.num_n) * 256 + 128 * int(rank);
+                const int k0 = (tile % p.num_n) * BN + 128 * int(rank);
                 for (int kb = 0; kb < p.num_k; ++kb) {
                     if (!mbar_wait(bar_empty + 8 * stage, phase ^ 1, abort_flag)) { ok = false; break; }
                     if (even) mbar_arrive_expect_tx(bar_full + 8 * stage, kPTxBytes);
@@ -201,7 +203,7 @@ trust_linear_pair_kernel(const __grid_constant__ CUtensorMap map_a, const __grid
         int local = 0;
         int cbuf = 0;
         for (int tile = pair; tile < num_tiles; tile += num_pairs, ++local) {
-            const int m0 = (tile % p.num_m2) * 256 + 128 * int(rank), k0 = (tile / p.num_m2) * BN;
+            const int m0 = (tile / p.num_n) * 256 + 128 * int(rank), k0 = (tile % p.num_n) * BN;
             const uint32_t buf = local & 1, bphase = (local >> 1) & 1;
             const int m = m0 + row_in_tile;
             // this row's mask bits for the tile's two blocks, fetched before the wait
