@@ -830,6 +830,23 @@ def run_configs(args):
         q.trust_bwd_raw(G.data_ptr(), mask.data_ptr(), q.MASK_BITS, R, C, HB, gx2.data_ptr(), s)
     add("comparison: cuBLAS bf16 product then trust backward (unfused, G through HBM)", unfused,
         2 * R * NW + 2 * C * NW + R * C // 8 + 2 * R * C, unit_ops=GEMM_OPS, bf16=True)
+    # the QAT forward on dequantised operands: X and W_up quantized with RMS per 128-group
+    # and bf16 yhat, then the bf16 layer (the per-group-scaled product on yhat)
+    xh = torch.empty((R, C), dtype=torch.bfloat16, device=dev)
+    wh = torch.empty((NW, C), dtype=torch.bfloat16, device=dev)
+    for src, dst in ((x2, xh), (w, wh)):
+        rr = src.shape[0]
+        cq = torch.empty(rr * C, dtype=torch.uint8, device=dev)
+        sq = torch.empty(rr * (C // HB), dtype=torch.float32, device=dev)
+        q.quantize_fwd_raw(src.data_ptr(), q.BF16, rr, C, C, 4, HB, HB, 1.0, q.CODES_INT8, cq.data_ptr(),
+                           sq.data_ptr(), 0, None, dst.data_ptr(), q.BF16, s)
+    f = lambda: q.linear_bf16_raw(xh.data_ptr(), wh.data_ptr(), R, NW, C, y.data_ptr(), s)
+    add("QAT forward linear on bf16 yhat 16384x5632x2048 (RMS per 128-group)", f,
+        2 * R * C + 2 * NW * C + 2 * R * NW, unit_ops=GEMM_OPS, bf16=True)
+    y2 = torch.empty_like(y)
+    f = lambda: torch.matmul(xh, wh.t(), out=y2)
+    add("comparison: cuBLAS bf16 product on the same yhat", f, 2 * R * C + 2 * NW * C + 2 * R * NW,
+        unit_ops=GEMM_OPS, bf16=True)
     gemm_tops = next(r["tops"] for r in rows if r["case"].startswith("W4A4 linear"))
     q.device_status()
     probe = mma_probe(dev, gemm_tops)

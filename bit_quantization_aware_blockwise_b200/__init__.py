@@ -39,6 +39,8 @@ from ._binding import (  # noqa: F401
     trust_bwd_linear_raw,
     transpose_bf16,
     transpose_bf16_raw,
+    linear_bf16,
+    linear_bf16_raw,
     device_status,
     probe_mma_i8,
     probe_status,
@@ -50,5 +52,6 @@ __all__ = [
     "MASK_BYTES", "BF16", "FP32", "library_path", "load_library", "alpha", "alpha_fp4", "codes_bytes", "mask_bytes",
     "container_bits", "quantize_fwd", "quantize_operands", "quantize_operands_raw", "trust_bwd", "w4a4_linear", "quantize_fwd_raw",
     "trust_bwd_raw", "w4a4_linear_raw", "w4a4_linear_grouped", "w4a4_linear_grouped_raw",
-    "trust_bwd_linear", "trust_bwd_linear_raw", "transpose_bf16", "transpose_bf16_raw", "device_status", "probe_mma_i8", "probe_status",
+    "trust_bwd_linear", "trust_bwd_linear_raw", "transpose_bf16", "transpose_bf16_raw",
+    "linear_bf16", "linear_bf16_raw", "device_status", "probe_mma_i8", "probe_status",
 ]

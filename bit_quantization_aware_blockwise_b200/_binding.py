@@ -32,6 +32,7 @@ SIGNATURES = {
     "quest_w4a4_linear_grouped": (_int, [_p, _p, _p, _p, _i64, _i64, _i64, _i64, _p, _p, _p]),
     "quest_trust_bwd_linear": (_int, [_p, _p, _p, _i64, _i64, _i64, _int, _p, _p]),
     "quest_transpose_bf16": (_int, [_p, _i64, _i64, _p, _p]),
+    "quest_linear_bf16": (_int, [_p, _p, _i64, _i64, _i64, _p, _p]),
     "quest_device_status": (_int, [_p]),
     "quest_alpha": (_f64, [_int]),
     "quest_alpha_fp4": (_f64, []),
@@ -120,6 +121,10 @@ def w4a4_linear_raw(a_codes, a_scales, w_codes, w_scales, M, N, K, y, acc=None, 
 def trust_bwd_linear_raw(grad_y, w_hat_t, mask, M, N, K, had_block, grad_x, stream=0):
     _check(load_library().quest_trust_bwd_linear(grad_y, w_hat_t, mask, M, N, K, had_block, grad_x, stream),
            "quest_trust_bwd_linear")
+
+
+def linear_bf16_raw(x_hat, w_hat, M, N, K, y, stream=0):
+    _check(load_library().quest_linear_bf16(x_hat, w_hat, M, N, K, y, stream), "quest_linear_bf16")
 
 
 def transpose_bf16_raw(src, rows, cols, dst, stream=0):
@@ -286,6 +291,24 @@ def trust_bwd_linear(grad_y, w_hat_t, mask, had_block: int = 128, out=None, stre
         out = torch.empty((M, K), dtype=torch.bfloat16, device=grad_y.device)
     trust_bwd_linear_raw(grad_y.data_ptr(), w_hat_t.data_ptr(), mask.data_ptr(), M, N, K, had_block,
                          out.data_ptr(), _stream_handle(stream, grad_y.device))
+    return out
+
+
+def linear_bf16(x_hat, w_hat, out=None, stream=None):
+    """y = x_hat @ w_hat^T on bf16 operands [M, K] and [N, K] (fp32 accumulation, bf16 out)."""
+    torch = _torch()
+    _require_cuda(x_hat, "x_hat")
+    _require_cuda(w_hat, "w_hat")
+    if x_hat.dtype != torch.bfloat16 or w_hat.dtype != torch.bfloat16:
+        raise QuestError("x_hat and w_hat must be bfloat16")
+    if x_hat.dim() != 2 or w_hat.dim() != 2 or x_hat.shape[1] != w_hat.shape[1]:
+        raise QuestError("x_hat [M, K] and w_hat [N, K] expected")
+    if not (x_hat.is_contiguous() and w_hat.is_contiguous()):
+        raise QuestError("x_hat and w_hat must be contiguous")
+    (M, K), N = x_hat.shape, w_hat.shape[0]
+    if out is None:
+        out = torch.empty((M, N), dtype=torch.bfloat16, device=x_hat.device)
+    linear_bf16_raw(x_hat.data_ptr(), w_hat.data_ptr(), M, N, K, out.data_ptr(), _stream_handle(stream, x_hat.device))
     return out
 
 

@@ -550,6 +550,34 @@ quest_status quest_trust_bwd_linear(const void* grad_y, const void* w_hat_t, con
     return QUEST_OK;
 }
 
+quest_status quest_linear_bf16(const void* x_hat, const void* w_hat, int64_t M, int64_t N, int64_t K, void* y,
+                               void* stream) {
+    g_last_error.clear();
+    if (M < 0 || N < 0 || K < 0) return fail(QUEST_EINVAL, "M, N and K must be >= 0");
+    if (M >= (int64_t(1) << 31) || N >= (int64_t(1) << 31) || K >= (int64_t(1) << 31))
+        return fail(QUEST_EINVAL, "M, N and K must be < 2^31");
+    if (K % 8 != 0 || N % 8 != 0) return fail(QUEST_EINVAL, "K and N must be multiples of 8 (16-byte rows)");
+    if (M > 0 && N > 0) {
+        if (!y) return fail(QUEST_EINVAL, "y must be non-NULL");
+        if (K > 0 && (!x_hat || !w_hat)) return fail(QUEST_EINVAL, "x_hat and w_hat must be non-NULL");
+        if (!aligned(y, 16) || (K > 0 && (!aligned(x_hat, 16) || !aligned(w_hat, 16))))
+            return fail(QUEST_EINVAL, "x_hat, w_hat and y must be 16-byte aligned");
+        const char* yc = static_cast<const char*>(y);
+        const int64_t y_bytes = M * N * 2;
+        auto overlaps = [&](const void* p, int64_t bytes) {
+            const char* c = static_cast<const char*>(p);
+            return c != nullptr && bytes > 0 && c < yc + y_bytes && yc < c + bytes;
+        };
+        if (overlaps(x_hat, M * K * 2) || overlaps(w_hat, N * K * 2))
+            return fail(QUEST_EINVAL, "y must not overlap x_hat or w_hat");
+    }
+    cudaError_t e = launch_linear_bf16(static_cast<const uint16_t*>(x_hat), static_cast<const uint16_t*>(w_hat), M,
+                                       N, K, static_cast<uint16_t*>(y), static_cast<cudaStream_t>(stream));
+    if (e == cudaErrorInvalidValue) return fail(QUEST_ECUDA, "quest_linear_bf16: tensor map encoding failed");
+    if (e != cudaSuccess) return cuda_fail(e, "quest_linear_bf16 launch");
+    return QUEST_OK;
+}
+
 quest_status quest_transpose_bf16(const void* src, int64_t rows, int64_t cols, void* dst, void* stream) {
     g_last_error.clear();
     if (rows < 0 || cols < 0) return fail(QUEST_EINVAL, "rows and cols must be >= 0");
@@ -580,7 +608,8 @@ quest_status quest_device_status(void* stream) {
     if (e != cudaSuccess) return cuda_fail(e, "quest_device_status");
     if (vg != 0) return fail((quest_status)vg, "a bounded device-side wait in quest_w4a4_linear gave up");
     if (vgr != 0) return fail((quest_status)vgr, "a bounded device-side wait in quest_w4a4_linear_grouped gave up");
-    if (vtl != 0) return fail((quest_status)vtl, "a bounded device-side wait in quest_trust_bwd_linear gave up");
+    if (vtl != 0)
+        return fail((quest_status)vtl, "a bounded device-side wait in quest_trust_bwd_linear or quest_linear_bf16 gave up");
     return QUEST_OK;
 }
 

@@ -104,6 +104,9 @@ cudaError_t launch_transpose_bf16(const uint16_t* src, int64_t rows, int64_t col
 // gx = H (mask * (gy wt^T)) / sqrt(128) per 128-column block (trust_linear.cu).
 cudaError_t launch_trust_linear(const uint16_t* gy, const uint16_t* wt, const uint8_t* mask, int64_t M,
                                 int64_t N, int64_t K, uint16_t* gx, cudaStream_t stream);
+// y [M, N] = x_hat [M, K] w_hat [N, K]^T on bf16 operands, fp32 accumulation (trust_linear.cu).
+cudaError_t launch_linear_bf16(const uint16_t* x_hat, const uint16_t* w_hat, int64_t M, int64_t N, int64_t K,
+                               uint16_t* y, cudaStream_t stream);
 cudaError_t launch_w4a4_grouped(const int8_t* A, const float* sa, const int8_t* B, const float* sb,
                                 int64_t M, int64_t N, int64_t K, uint16_t* y, float* y32,
                                 cudaStream_t stream);

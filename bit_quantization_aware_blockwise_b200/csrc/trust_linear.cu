@@ -1,5 +1,6 @@
-// Input gradient of the quantized linear layer with the trust backward fused into
-// the epilogue of a CTA-pair tcgen05 bf16 product (see the kernel's comment).
+// CTA-pair tcgen05 bf16 products: the input gradient of the quantized linear layer
+// with the trust backward fused into the epilogue, and the linear layer on bf16
+// dequantised operands (see the kernel's comment).
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -30,7 +31,9 @@ namespace {
 // shared-memory ring, barriers and TMEM accumulators are the same. The epilogue
 // thread that owns an accumulator row (one TMEM lane) holds a whole 128-column
 // block in registers: the mask and the 128-point transform are register work with
-// no exchange, and G never reaches HBM. Tiles run output-column-fastest: the pairs in
+// no exchange, and G never reaches HBM. The same kernel without the mask and the
+// transform is the linear layer on bf16 dequantised operands, y = x_hat w_hat^T
+// (yhat = (q + 1/2) Delta rounded to bf16, any RMS grouping). Tiles run output-column-fastest: the pairs in
 // flight share a few 256-row blocks of grad_y (which, at 16384 x 5632 bf16, is larger
 // than L2) and all of w_hat_t, so grad_y streams from HBM about once.
 constexpr uint32_t kIdescBf16Pair = (1u << 4)     // D: fp32
@@ -74,9 +77,12 @@ __device__ __forceinline__ void fwht128_regs(float2 (&w)[64]) {
     }
 }
 
+// TRUST: the epilogue masks and transforms each 128-column block (the input gradient);
+// otherwise it stores the product as it is (the linear layer on bf16 yhat operands).
+template <bool TRUST>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
-trust_linear_pair_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_b,
-                         const __grid_constant__ CUtensorMap map_y, const TrustLinearParams p) {
+bf16_pair_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_b,
+                 const __grid_constant__ CUtensorMap map_y, const TrustLinearParams p) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const uint32_t sbase = smem_u32(smem);
@@ -207,13 +213,14 @@ trust_linear_pair_kernel(const __grid_constant__ CUtensorMap map_a, const __grid
             const uint32_t buf = local & 1, bphase = (local >> 1) & 1;
             const int m = m0 + row_in_tile;
             // this row's mask bits for the tile's two blocks, fetched before the wait
-            uint4 mw[2];
+            uint4 mw[2] = {make_uint4(0u, 0u, 0u, 0u), make_uint4(0u, 0u, 0u, 0u)};
+            if constexpr (TRUST) {
 #pragma unroll
-            for (int b = 0; b < 2; ++b) {
-                const int kb0 = k0 + 128 * b;
-                mw[b] = (m < p.M && kb0 < p.K)
-                            ? *reinterpret_cast<const uint4*>(p.mask + int64_t(m) * mask_row_bytes + kb0 / 8)
-                            : make_uint4(0u, 0u, 0u, 0u);
+                for (int b = 0; b < 2; ++b) {
+                    const int kb0 = k0 + 128 * b;
+                    if (m < p.M && kb0 < p.K)
+                        mw[b] = *reinterpret_cast<const uint4*>(p.mask + int64_t(m) * mask_row_bytes + kb0 / 8);
+                }
             }
             const bool got = mbar_wait(bar_tfull + 8 * buf, bphase, abort_flag);
             if (epi_any(!got)) break;
@@ -232,13 +239,18 @@ trust_linear_pair_kernel(const __grid_constant__ CUtensorMap map_a, const __grid
                     const uint32_t bits = c == 0 ? mb.x : c == 1 ? mb.y : c == 2 ? mb.z : mb.w;
 #pragma unroll
                     for (int i = 0; i < 16; ++i) {
-                        // keep G where the mask bit is 1 (bit j of the word = column 32c + j)
-                        const uint32_t k0m = 0u - ((bits >> (2 * i)) & 1u);
-                        const uint32_t k1m = 0u - ((bits >> (2 * i + 1)) & 1u);
-                        w[16 * c + i] = make_float2(__uint_as_float(r[2 * i] & k0m), __uint_as_float(r[2 * i + 1] & k1m));
+                        if constexpr (TRUST) {
+                            // keep G where the mask bit is 1 (bit j of the word = column 32c + j)
+                            const uint32_t k0m = 0u - ((bits >> (2 * i)) & 1u);
+                            const uint32_t k1m = 0u - ((bits >> (2 * i + 1)) & 1u);
+                            w[16 * c + i] =
+                                make_float2(__uint_as_float(r[2 * i] & k0m), __uint_as_float(r[2 * i + 1] & k1m));
+                        } else {
+                            w[16 * c + i] = make_float2(__uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1]));
+                        }
                     }
                 }
-                fwht128_regs(w);
+                if constexpr (TRUST) fwht128_regs(w);
 #pragma unroll
                 for (int c = 0; c < 4; ++c) {
                     const uint32_t stg = sbase + kPSmemC + cbuf * kCBytes + row_in_tile * (kChunkCols * 2);
@@ -249,7 +261,8 @@ trust_linear_pair_kernel(const __grid_constant__ CUtensorMap map_a, const __grid
 #pragma unroll
                         for (int h = 0; h < 4; ++h) {
                             const float2 v = w[16 * c + 4 * q16 + h];
-                            __nv_bfloat162 hb = __floats2bfloat162_rn(v.x * p.scale, v.y * p.scale);
+                            __nv_bfloat162 hb = TRUST ? __floats2bfloat162_rn(v.x * p.scale, v.y * p.scale)
+                                                      : __floats2bfloat162_rn(v.x, v.y);
                             o[h] = *reinterpret_cast<uint32_t*>(&hb);
                         }
                         asm volatile("st.shared.v4.u32 [%0], {%1,%2,%3,%4};" ::"r"(stg + ((q16 ^ swz) << 4)),
@@ -283,8 +296,11 @@ trust_linear_pair_kernel(const __grid_constant__ CUtensorMap map_a, const __grid
     }
 }
 
-cudaError_t launch_trust_linear_pair(const uint16_t* gy, const uint16_t* wt, const uint8_t* mask, int64_t M,
-                                     int64_t N, int64_t K, uint16_t* gx, cudaStream_t stream) {
+// out [M, K] = a [M, N] b [K, N]^T (both N-contiguous), with the trust epilogue when
+// TRUST (mask bits [M, K / 8]).
+template <bool TRUST>
+cudaError_t launch_bf16_pair(const uint16_t* gy, const uint16_t* wt, const uint8_t* mask, int64_t M, int64_t N,
+                             int64_t K, uint16_t* gx, cudaStream_t stream) {
     CUtensorMap ma, mb, my;
     if (!make_map_2d(&ma, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, gy, N, M, N * 2, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B) ||
         !make_map_2d(&mb, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, wt, N, K, N * 2, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B) ||
@@ -293,7 +309,7 @@ cudaError_t launch_trust_linear_pair(const uint16_t* gy, const uint16_t* wt, con
         return cudaErrorInvalidValue;
     TrustLinearParams p;
     p.mask = mask;
-    p.scale = 0.08838834764831845f;   // 1 / sqrt(128)
+    p.scale = TRUST ? 0.08838834764831845f : 1.0f;   // 1 / sqrt(128) for the inverse transform
     p.M = (int)M; p.N = (int)N; p.K = (int)K;
     p.num_m2 = (int)((M + 255) / 256);
     p.num_n = (int)((K + BN - 1) / BN);
@@ -302,15 +318,15 @@ cudaError_t launch_trust_linear_pair(const uint16_t* gy, const uint16_t* wt, con
     int dev = 0;
     cudaGetDevice(&dev);
     if (attr_dev != dev) {
-        cudaError_t e = cudaFuncSetAttribute(trust_linear_pair_kernel,
+        cudaError_t e = cudaFuncSetAttribute(bf16_pair_kernel<TRUST>,
                                              cudaFuncAttributeMaxDynamicSharedMemorySize, kPSmemTotal);
         if (e != cudaSuccess) return e;
         attr_dev = dev;
     }
     const int tiles = p.num_m2 * p.num_n;
-    const int pairs = pair_clusters(dev, (const void*)trust_linear_pair_kernel, kThreads, kPSmemTotal);
+    const int pairs = pair_clusters(dev, (const void*)bf16_pair_kernel<TRUST>, kThreads, kPSmemTotal);
     const int grid_pairs = tiles < pairs ? tiles : pairs;
-    return launch_pdl(trust_linear_pair_kernel, dim3(2 * grid_pairs), dim3(kThreads), kPSmemTotal, stream, ma, mb,
+    return launch_pdl(bf16_pair_kernel<TRUST>, dim3(2 * grid_pairs), dim3(kThreads), kPSmemTotal, stream, ma, mb,
                       my, p);
 }
 
@@ -322,7 +338,15 @@ cudaError_t launch_trust_linear(const uint16_t* gy, const uint16_t* wt, const ui
     if (N == 0) {   // the empty sum: G = 0, so the gradient is 0
         return launch_zero_fill(gx, nullptr, M * K, stream);
     }
-    return launch_trust_linear_pair(gy, wt, mask, M, N, K, gx, stream);
+    return launch_bf16_pair<true>(gy, wt, mask, M, N, K, gx, stream);
+}
+
+cudaError_t launch_linear_bf16(const uint16_t* x_hat, const uint16_t* w_hat, int64_t M, int64_t N, int64_t K,
+                               uint16_t* y, cudaStream_t stream) {
+    if (M == 0 || N == 0) return cudaSuccess;
+    if (K == 0) return launch_zero_fill(y, nullptr, M * N, stream);   // the empty sum
+    // the pair kernel's product runs over its second dimension: y [M, N] = x_hat [M, K] w_hat [N, K]^T
+    return launch_bf16_pair<false>(x_hat, w_hat, nullptr, M, K, N, y, stream);
 }
 
 int read_and_clear_trust_linear_status(cudaStream_t stream, cudaError_t* err) {

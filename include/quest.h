@@ -294,6 +294,27 @@ quest_status quest_trust_bwd_linear(const void* grad_y, const void* w_hat_t, con
                                     int64_t N, int64_t K, int had_block, void* grad_x, void* stream);
 
 /*
+ * quest_linear_bf16 -- the linear layer of QuEST training on dequantised operands.
+ *
+ * The forward pass multiplies the quantized operands in the Hadamard domain
+ * (pith.science review, "Assumptions & free parameters": the transform applied to
+ * both operands leaves the product unchanged; Figure 2 caption: two Hadamard
+ * transforms on the forward pass):
+ *     y = x_hat w_hat^T        x_hat [M, K], w_hat [N, K] bf16 (e.g. quest_quantize_fwd's
+ *                              bf16 `dequant` of each operand, any RMS grouping),
+ *                              fp32 accumulation, y bf16 [M, N] (RNE).
+ * With per-128-group scales this is the layer of quest_w4a4_linear_grouped computed on
+ * yhat rounded to bf16 instead of on the exact codes.
+ *
+ * Arguments: M, N, K >= 0, K and N multiples of 8, M, N, K < 2^31; x_hat, w_hat and y
+ * device pointers, 16-byte aligned, y not overlapping the operands. K == 0 writes zeros.
+ * Returns QUEST_OK, QUEST_EINVAL or QUEST_ECUDA (a bounded wait that gives up is
+ * reported by quest_device_status, like quest_trust_bwd_linear's).
+ */
+quest_status quest_linear_bf16(const void* x_hat, const void* w_hat, int64_t M, int64_t N, int64_t K, void* y,
+                               void* stream);
+
+/*
  * quest_transpose_bf16 -- dst[c][r] = src[r][c] for a bf16 [rows, cols] matrix
  * (row-major, dense); dst is [cols, rows]. Produces the w_hat_t operand of
  * quest_trust_bwd_linear from a dequantised weight. src and dst must not overlap.

@@ -221,6 +221,18 @@ def trust_bwd_linear(g_y, w_hat, mask, had: int = 128) -> np.ndarray:
     return trust_bwd(g_y @ w_hat, mask, had)
 
 
+def linear_bf16(x_hat, w_hat) -> np.ndarray:
+    """y = x_hat @ w_hat^T in fp64 (numpy's matmul): the linear layer on dequantised
+    operands in the Hadamard domain (pith.science review, "Assumptions & free
+    parameters": the transform applied to both operands leaves the product unchanged).
+    x_hat [M, K], w_hat [N, K]; bf16 inputs are exact in fp64."""
+    x_hat = np.asarray(x_hat, dtype=np.float64)
+    w_hat = np.asarray(w_hat, dtype=np.float64)
+    if x_hat.ndim != 2 or w_hat.ndim != 2 or x_hat.shape[1] != w_hat.shape[1]:
+        raise ValueError("x_hat [M, K] and w_hat [N, K] expected")
+    return x_hat @ w_hat.T
+
+
 def gemm_i8(a, b) -> np.ndarray:
     """acc = A @ B^T in int64 by a triple loop; A [M,K], B [N,K] int8."""
     a = np.ascontiguousarray(np.asarray(a, dtype=np.int8))

@@ -186,3 +186,14 @@ def test_quantize_operands_rejects_invalid_arguments():
                dict(sw=None), dict(w=FAKE + 4), dict(mode=5, bits=3), dict(dt=4)]:
         assert call(**kw) == 1, kw
     assert call(M=0, N=0, x=None, w=None, cx=None, sx=None, cw=None, sw=None) == 0
+
+
+def test_linear_bf16_rejects_invalid_arguments():
+    lib = q.load_library()
+
+    def call(x=FAKE, w=FAKE + (1 << 24), M=4, N=16, K=64, y=FAKE + (1 << 25)):
+        return lib.quest_linear_bf16(x, w, M, N, K, y, None)
+    for kw in [dict(M=-1), dict(K=12), dict(N=12), dict(y=None), dict(x=None), dict(w=FAKE + 8),
+               dict(y=FAKE + 64), dict(M=1 << 31)]:
+        assert call(**kw) == 1, kw
+    assert call(M=0, x=None, w=None, y=None) == 0

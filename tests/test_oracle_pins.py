@@ -528,3 +528,17 @@ def test_one_bit_outer_trust_from_the_pages():
     p = 2 * scipy.stats.norm.sf(edge * a1)
     rate = 1 - o["mask"].mean()
     assert abs(rate - p) < 4 * math.sqrt(p * (1 - p) / x.size)
+
+
+def test_linear_bf16_pins():
+    # brute-force triple loop on a tiny case, and the Hadamard-invariance the pages state:
+    # transforming both operands' rows by the same orthogonal H leaves the product unchanged
+    g = np.random.default_rng(23)
+    x = g.standard_normal((3, 8))
+    w = g.standard_normal((5, 8))
+    y = oracle.linear_bf16(x, w)
+    for i in range(3):
+        for j in range(5):
+            assert abs(y[i, j] - sum(x[i, k] * w[j, k] for k in range(8))) < 1e-12
+    H = scipy.linalg.hadamard(8) / np.sqrt(8)
+    assert np.allclose(oracle.linear_bf16(x @ H.T, w @ H.T), y, rtol=0, atol=1e-12)
