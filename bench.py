@@ -881,12 +881,13 @@ def run_profile_kernels(args):
     gyl = inputs.upstream_grad(8192, NW, seed=5).to(dev)
     wt = q.transpose_bf16(inputs.weight_up().to(dev))                                  # 7
     gx = q.trust_bwd_linear(gyl, wt, out["mask"][: 8192 * C // 8])                     # 8
+    yf = q.linear_bf16(x[:8192], w_up)                                                 # 9
     torch.cuda.synchronize()
     q.device_status()
     print(json.dumps({"profile_kernels": "ok", "rows": rows, "checksum": [
         float(out["scales"].sum()), float(gi.float().abs().sum()), float(op["scales"].sum()),
         float(y.float().abs().sum()), float(yg.float().abs().sum()), float(f4["scales"].sum()),
-        float(gx.float().abs().sum())]}))
+        float(gx.float().abs().sum()), float(yf.float().abs().sum())]}))
 
 
 def main():
