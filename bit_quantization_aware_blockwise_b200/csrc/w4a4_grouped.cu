@@ -1,6 +1,7 @@
 // Linear layer on QuEST codes with per-group scales along K (one scale per row and
 // per 128-wide K group on both operands): CTA-pair tcgen05 kind::f8f6f4 kernel on
-// E4M3 codes with a per-group TMEM round trip (see the kernel's comment).
+// E4M3 codes with a per-group TMEM round trip into two ping-pong epilogue teams
+// (see the kernel's comment).
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -25,40 +26,55 @@ namespace {
 // product of group g's codes. The codes come as FP8 E4M3 (c = 2q + 1, odd,
 // |c| <= 15, exact in E4M3), so tcgen05 kind::f8f6f4 with fp32 accumulation
 // gives every P_g exactly (integers below 2^24) with no int -> float step.
-// CTA pairs as above, tiles of 256 x 128, one stage per group; the MMA cycles
-// four 128-column TMEM slots, one group each, and eight epilogue warps (two per
-// TMEM lane quarter, 64 columns each) fold every group into fp32 accumulators
-// held in registers: acc += P_g * (sa/2)(sb/2), two packed FMA-class
-// instructions per pair of outputs per group. A group's completion is read off
-// its stage's empty barrier (one commit per group). This layer is bounded by the
-// TMEM round trip, not the tensor cores: four slots hold about 1000 cycles of
-// MMA work per SM, while a slot takes about 3000 cycles from the commit to its
-// release by both CTAs' epilogues (clock64 counters on B200).
+//
+// Every group's product makes a round trip through TMEM to registers, where it
+// is scaled and added: acc += P_g * (sa/2)(sb/2), two packed FP instructions per
+// pair of outputs per group. The epilogue runs as two teams of four warps (one
+// warp per TMEM lane quarter on each team), each team owning the whole 128 x 128
+// accumulator of its own output tile in registers: the CTA pair takes its tiles
+// two at a time, and the MMA issuer alternates between them group by group
+// (tile 2c group g, tile 2c+1 group g, tile 2c group g+1, ...), so the two
+// warps on a scheduler are at different points of their groups. Each team has
+// two of the four 128-column TMEM slots; a slot's full barrier (committed by the
+// MMA issuer in both CTAs) says that its group's product is complete, its empty
+// barrier (8 warp arrivals) that the team has read it. A slot is never reissued
+// before its team has read it, so its full barrier is at most one phase ahead of
+// the team's wait. An epilogue thread holds its row of the accumulator (128
+// registers) and two 16-column TMEM load buffers, so the load of the next 16
+// columns overlaps the arithmetic on the current ones.
+//
+// What bounds it (16384 x 5632 x 2048, scratch variants timed on B200): 400 us
+// as built; 393 us with half the MMAs; 330 us with the FP work removed; 254 us
+// with neither MMAs nor FP work. The layer is bound by moving every group's fp32
+// product from TMEM to registers (5.9 GB per launch): with one 16-column load in
+// flight per warp and two warps per scheduler (the accumulator leaves no
+// registers for more) that runs at about 83 B per clock per SM alone and 64 with
+// the MMAs running. A lockstep layout (eight warps on the same group, 64
+// columns each, two 32-column loads per wait) measured the same 403 us.
 
-constexpr int kGThreads = 320;               // producer, MMA, 8 epilogue warps
-constexpr int kGEpiThreads = 256;
+constexpr int kGThreads = 384;               // warpgroup 0: producer, MMA (2 warps idle); 1, 2: the teams
+constexpr int kGTeamThreads = 128;
 constexpr int kGBN = 128;                    // output columns per pair tile
 constexpr int kGStages = 6;
-constexpr int kGSlots = 4;                   // TMEM slots of kGBN columns
+constexpr int kGSlots = 4;                   // TMEM slots of kGBN columns, two per team
 constexpr int kGroup = 128;                  // K group = one stage
-constexpr int kGScaleBlock = 16;             // groups of scales staged at a time
+constexpr int kGScaleBlock = 8;              // groups of scales staged at a time
 constexpr uint32_t kGStageA = 128 * BK, kGStageB = (kGBN / 2) * BK;   // per CTA
 constexpr uint32_t kGTxBytes = 2 * (kGStageA + kGStageB);
 constexpr uint32_t kGSmemA = 0;
 constexpr uint32_t kGSmemB = kGSmemA + kGStages * kGStageA;
-constexpr uint32_t kGScaleBytes = kGScaleBlock * (kGBN + 128) * 4;    // one block: sb [16][128], sa [16][128]
-constexpr uint32_t kGSmemS = kGSmemB + kGStages * kGStageB;           // two blocks (double buffer)
-constexpr uint32_t kGSmemC = kGSmemS + 2 * kGScaleBytes;              // 8 warps x 2 x 2 KB
+constexpr uint32_t kGScaleBytes = kGScaleBlock * (kGBN + 128) * 4;    // one block: sb [8][128], sa [8][128]
+constexpr uint32_t kGSmemS = kGSmemB + kGStages * kGStageB;           // 2 teams x 2 blocks (double buffer)
+constexpr uint32_t kGSmemC = kGSmemS + 4 * kGScaleBytes;              // 8 warps x 2 x 2 KB
 constexpr uint32_t kGCBytes = 32 * 32 * 2;                            // 32 rows x 32 bf16
 constexpr uint32_t kGSmemBar = kGSmemC + 8 * 2 * kGCBytes;
-constexpr uint32_t kGNumBars = 2 * kGStages + kGSlots + 1;
+constexpr uint32_t kGNumBars = 2 * kGStages + 2 * kGSlots + 1;
 constexpr uint32_t kGSmemTmemSlot = kGSmemBar + kGNumBars * 8;
 constexpr uint32_t kGSmemAbort = kGSmemTmemSlot + 4;
 constexpr uint32_t kGSmemUsed = kGSmemAbort + 4;
 constexpr uint32_t kGSmemTotal = kGSmemUsed + 1024;
 static_assert(kGSmemTotal <= 227 * 1024, "grouped kernel shared memory");
 static_assert(kGSlots * kGBN == kTmemCols, "TMEM slots");
-static_assert(kGSlots < kGStages, "the epilogue reads group completion off the stage barriers");
 
 // kind::f8f6f4, f32 accumulator, A and B E4M3, K-major, M = 256, N = 128.
 constexpr uint32_t kIdescGrouped = (1u << 4) | (0u << 7) | (0u << 10) | (uint32_t(kGBN >> 3) << 17) |
@@ -74,21 +90,32 @@ __device__ __forceinline__ void tc_mma_f8_pair(uint32_t d_tmem, uint64_t adesc, 
         : "memory");
 }
 
-__device__ __forceinline__ void gepi_bar() {
-    asm volatile("bar.sync 1, %0;" ::"n"(kGEpiThreads) : "memory");
+// Named barrier 1 + team over the team's 128 threads, and an OR-vote on it.
+__device__ __forceinline__ void team_bar(int team) {
+    asm volatile("bar.sync %0, %1;" ::"r"(1 + team), "n"(kGTeamThreads) : "memory");
 }
-__device__ __forceinline__ bool gepi_any(bool pred) {
+__device__ __forceinline__ bool team_any(int team, bool pred) {
     uint32_t out;
     asm volatile(
         "{\n\t.reg .pred p, q;\n\t"
         "setp.ne.u32 p, %1, 0;\n\t"
-        "bar.red.or.pred q, 1, %2, p;\n\t"
+        "bar.red.or.pred q, %2, %3, p;\n\t"
         "selp.u32 %0, 1, 0, q;\n\t}"
         : "=r"(out)
-        : "r"((uint32_t)pred), "n"(kGEpiThreads)
+        : "r"((uint32_t)pred), "r"(1 + team), "n"(kGTeamThreads)
         : "memory");
     return out != 0;
 }
+
+// tcgen05.wait::ld that names the loaded registers as read-write operands, so no
+// use of them can be scheduled above the wait.
+#define QUEST_TMEM_WAIT16(r)                                                                   \
+    asm volatile("tcgen05.wait::ld.sync.aligned;"                                             \
+                 : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]),     \
+                   "+r"(r[6]), "+r"(r[7]), "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]),   \
+                   "+r"(r[12]), "+r"(r[13]), "+r"(r[14]), "+r"(r[15])                          \
+                 :                                                                             \
+                 : "memory")
 
 __device__ __forceinline__ void cp_async4(uint32_t dst, const float* src, bool valid) {
     asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;" ::"r"(dst), "l"(src), "r"(valid ? 4 : 0)
@@ -113,12 +140,11 @@ w4a4_gemm_grouped_kernel(const __grid_constant__ CUtensorMap map_a, const __grid
     const uint32_t sbase = smem_u32(smem);
     const uint32_t bar_full = sbase + kGSmemBar;                 // [kGStages], used in the even CTA
     const uint32_t bar_empty = bar_full + 8 * kGStages;          // [kGStages]
-    const uint32_t bar_tempty = bar_empty + 8 * kGStages;        // [kGSlots], used in the even CTA
+    const uint32_t bar_tfull = bar_empty + 8 * kGStages;         // [kGSlots]
+    const uint32_t bar_tempty = bar_tfull + 8 * kGSlots;         // [kGSlots], used in the even CTA
     const uint32_t bar_drain = bar_tempty + 8 * kGSlots;
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + kGSmemAbort);
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kGSmemTmemSlot);
-    // scale blocks (double buffer): [16][128] sb[n0 + n][g0 + gg], then [16][128] sa[m0 + r][g0 + gg]
-    float* s_sc = reinterpret_cast<float*>(smem + kGSmemS);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const uint32_t rank = cluster_rank();
@@ -126,13 +152,19 @@ w4a4_gemm_grouped_kernel(const __grid_constant__ CUtensorMap map_a, const __grid
     const int pair = blockIdx.x >> 1, num_pairs = gridDim.x >> 1;
     const int num_tiles = p.num_m2 * p.num_n;
     const int G = p.num_k;
+    // this pair's tiles: pair + i * num_pairs for i < ntl, taken two at a time
+    // (couple c = tiles 2c and 2c + 1; the last couple may hold one tile)
+    const int ntl = (num_tiles - pair + num_pairs - 1) / num_pairs;
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < kGStages; ++s) {
             mbar_init(bar_full + 8 * s, 1);
             mbar_init(bar_empty + 8 * s, 1);
         }
-        for (int b = 0; b < kGSlots; ++b) mbar_init(bar_tempty + 8 * b, 16);   // 8 epilogue warps x 2 CTAs
+        for (int b = 0; b < kGSlots; ++b) {
+            mbar_init(bar_tfull + 8 * b, 1);
+            mbar_init(bar_tempty + 8 * b, 8);   // 4 team warps x 2 CTAs
+        }
         mbar_init(bar_drain, 1);
         *abort_flag = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -163,17 +195,21 @@ w4a4_gemm_grouped_kernel(const __grid_constant__ CUtensorMap map_a, const __grid
             uint32_t stage = 0, phase = 0;
             uint64_t issued = 0;
             bool ok = true;
-            for (int tile = pair; tile < num_tiles && ok; tile += num_pairs) {
-                const int m0 = (tile % p.num_m2) * 256 + 128 * int(rank);
-                const int n0 = (tile / p.num_m2) * kGBN + (kGBN / 2) * int(rank);
-                for (int kb = 0; kb < G; ++kb) {
-                    if (!mbar_wait(bar_empty + 8 * stage, phase ^ 1, abort_flag)) { ok = false; break; }
-                    if (even) mbar_arrive_expect_tx(bar_full + 8 * stage, kGTxBytes);
-                    const uint32_t fb = full_even + 8 * stage;
-                    tma_load_2d_pair(sbase + kGSmemA + stage * kGStageA, &map_a, kb * BK, m0, fb);
-                    tma_load_2d_pair(sbase + kGSmemB + stage * kGStageB, &map_b, kb * BK, n0, fb);
-                    ++issued;
-                    if (++stage == kGStages) { stage = 0; phase ^= 1; }
+            for (int c = 0; 2 * c < ntl && ok; ++c) {
+                const int nt = 2 * c + 1 < ntl ? 2 : 1;
+                for (int kb = 0; kb < G && ok; ++kb) {
+                    for (int t = 0; t < nt; ++t) {
+                        const int tile = pair + (2 * c + t) * num_pairs;
+                        const int m0 = (tile % p.num_m2) * 256 + 128 * int(rank);
+                        const int n0 = (tile / p.num_m2) * kGBN + (kGBN / 2) * int(rank);
+                        if (!mbar_wait(bar_empty + 8 * stage, phase ^ 1, abort_flag)) { ok = false; break; }
+                        if (even) mbar_arrive_expect_tx(bar_full + 8 * stage, kGTxBytes);
+                        const uint32_t fb = full_even + 8 * stage;
+                        tma_load_2d_pair(sbase + kGSmemA + stage * kGStageA, &map_a, kb * BK, m0, fb);
+                        tma_load_2d_pair(sbase + kGSmemB + stage * kGStageB, &map_b, kb * BK, n0, fb);
+                        ++issued;
+                        if (++stage == kGStages) { stage = 0; phase ^= 1; }
+                    }
                 }
             }
             if (!ok && even) {
@@ -194,26 +230,31 @@ w4a4_gemm_grouped_kernel(const __grid_constant__ CUtensorMap map_a, const __grid
         // ------------------------------------------------------------ MMA issuer (even CTA)
         if (even && lane == 0) {
             uint32_t stage = 0, phase = 0;
-            uint32_t gcount = 0;   // groups issued so far: TMEM slot = gcount % kGSlots
+            uint32_t gcount0 = 0, gcount1 = 0;   // groups issued per team: slot 2 t + (count & 1)
             bool ok = true;
-            for (int tile = pair; tile < num_tiles && ok; tile += num_pairs) {
-                for (int kb = 0; kb < G; ++kb, ++gcount) {
-                    const uint32_t slot = gcount % kGSlots, sphase = (gcount / kGSlots) & 1;
-                    if (!mbar_wait(bar_tempty + 8 * slot, sphase ^ 1, abort_flag)) { ok = false; break; }
-                    if (!mbar_wait(bar_full + 8 * stage, phase, abort_flag)) { ok = false; break; }
-                    tc_fence_after();
-                    const uint32_t d_tmem = tmem_base + slot * kGBN;
-                    const uint32_t a_addr = sbase + kGSmemA + stage * kGStageA;
-                    const uint32_t b_addr = sbase + kGSmemB + stage * kGStageB;
+            for (int c = 0; 2 * c < ntl && ok; ++c) {
+                const int nt = 2 * c + 1 < ntl ? 2 : 1;
+                for (int kb = 0; kb < G && ok; ++kb) {
+                    for (int t = 0; t < nt; ++t) {
+                        const uint32_t gc = t ? gcount1 : gcount0;
+                        const uint32_t slot = 2 * t + (gc & 1), sphase = (gc >> 1) & 1;
+                        if (!mbar_wait(bar_tempty + 8 * slot, sphase ^ 1, abort_flag)) { ok = false; break; }
+                        if (!mbar_wait(bar_full + 8 * stage, phase, abort_flag)) { ok = false; break; }
+                        tc_fence_after();
+                        const uint32_t d_tmem = tmem_base + slot * kGBN;
+                        const uint32_t a_addr = sbase + kGSmemA + stage * kGStageA;
+                        const uint32_t b_addr = sbase + kGSmemB + stage * kGStageB;
 #pragma unroll
-                    for (int kk = 0; kk < BK / kUmmaK; ++kk) {
-                        tc_mma_f8_pair(d_tmem, smem_desc_k128(a_addr + kk * kUmmaK),
-                                       smem_desc_k128(b_addr + kk * kUmmaK), kk != 0);
+                        for (int kk = 0; kk < BK / kUmmaK; ++kk) {
+                            tc_mma_f8_pair(d_tmem, smem_desc_k128(a_addr + kk * kUmmaK),
+                                           smem_desc_k128(b_addr + kk * kUmmaK), kk != 0);
+                        }
+                        tc_commit_pair_mc(bar_empty + 8 * stage);   // frees the stage in both CTAs
+                        tc_commit_pair_mc(bar_tfull + 8 * slot);    // the group's product is ready
+                        if (t) gcount1 = gc + 1;
+                        else gcount0 = gc + 1;
+                        if (++stage == kGStages) { stage = 0; phase ^= 1; }
                     }
-                    // frees the stage in both CTAs and, the same event, marks this group's
-                    // partials ready for the epilogue (which waits on this stage's barrier)
-                    tc_commit_pair_mc(bar_empty + 8 * stage);
-                    if (++stage == kGStages) { stage = 0; phase ^= 1; }
                 }
             }
             tc_commit_pair(bar_drain);
@@ -221,32 +262,35 @@ w4a4_gemm_grouped_kernel(const __grid_constant__ CUtensorMap map_a, const __grid
             while (!mbar_try_wait(bar_drain, 0) && global_timer_ns() - t0 < kWaitLimitNs) {
             }
         }
-    } else {
-        // ------------------------------------------------------------ epilogue (warps 2..9, both CTAs)
-        const int et = threadIdx.x - 64;                   // 0..255
-        const int ew = et >> 5;                            // epilogue warp 0..7
+    } else if (warp >= 4) {
+        // ------------------------------------------------------------ epilogue (warps 4..11, both CTAs)
+        const int ew = warp - 4;                           // epilogue warp 0..7
+        const int team = ew >> 2;                          // tiles 2c + team
+        const int tt = (ew & 3) * 32 + lane;               // thread in team 0..127
         const int quarter = warp & 3;                      // TMEM lanes 32*quarter .. +31
-        const int half = ew >> 2;                          // columns 64*half .. +63 of the tile
         const int row_in_tile = quarter * 32 + lane;
         const uint32_t lane_addr = uint32_t(quarter * 32) << 16;
         const uint32_t tempty_even = map_to_rank(bar_tempty, 0);
         const uint32_t stg0 = sbase + kGSmemC + uint32_t(ew) * 2 * kGCBytes;
+        const uint32_t sc_base = kGSmemS + uint32_t(team) * 2 * kGScaleBytes;   // this team's two blocks
         const int Gs = p.K / kGroup;                       // scale columns per row
-        // issue the copies of scale block (tile, g0) into buffer b: transposed to [group][column]
-        auto prefetch = [&](int tile, int g0, int b) {
-            if (tile < num_tiles) {
+        // issue the copies of the scales of groups g0 .. g0+7 of local tile i into buffer b,
+        // transposed to [group][column] and [group][row]
+        auto prefetch = [&](int i, int g0, int b) {
+            if (i < ntl) {
+                const int tile = pair + i * num_pairs;
                 const int pm0 = (tile % p.num_m2) * 256 + 128 * int(rank), pn0 = (tile / p.num_m2) * kGBN;
                 const int nb = (G - g0) < kGScaleBlock ? (G - g0) : kGScaleBlock;
-                const uint32_t base = sbase + kGSmemS + uint32_t(b) * kGScaleBytes;
+                const uint32_t base = sbase + sc_base + uint32_t(b) * kGScaleBytes;
 #pragma unroll
-                for (int k = 0; k < kGScaleBlock * kGBN / kGEpiThreads; ++k) {
-                    const int i = et + k * kGEpiThreads, n = i / kGScaleBlock, gg = i % kGScaleBlock;
+                for (int k = 0; k < kGScaleBlock * kGBN / kGTeamThreads; ++k) {
+                    const int e = tt + k * kGTeamThreads, n = e / kGScaleBlock, gg = e % kGScaleBlock;
                     const bool v = gg < nb && pn0 + n < p.N;
                     cp_async4(base + 4 * (gg * kGBN + n), p.sb + (v ? int64_t(pn0 + n) * Gs + g0 + gg : 0), v);
                 }
 #pragma unroll
-                for (int k = 0; k < kGScaleBlock * 128 / kGEpiThreads; ++k) {
-                    const int i = et + k * kGEpiThreads, r = i / kGScaleBlock, gg = i % kGScaleBlock;
+                for (int k = 0; k < kGScaleBlock * 128 / kGTeamThreads; ++k) {
+                    const int e = tt + k * kGTeamThreads, r = e / kGScaleBlock, gg = e % kGScaleBlock;
                     const bool v = gg < nb && pm0 + r < p.M;
                     cp_async4(base + 4 * (kGScaleBlock * kGBN + gg * 128 + r),
                               p.sa + (v ? int64_t(pm0 + r) * Gs + g0 + gg : 0), v);
@@ -254,76 +298,84 @@ w4a4_gemm_grouped_kernel(const __grid_constant__ CUtensorMap map_a, const __grid
             }
             cp_async_commit();
         };
-        uint32_t gcount = 0;
         int cbuf = 0, sbuf = 0;
         bool aborted = false;
-        prefetch(pair, 0, 0);
-        for (int tile = pair; tile < num_tiles && !aborted; tile += num_pairs) {
+        prefetch(team, 0, 0);
+        for (int i = team; i < ntl && !aborted; i += 2) {
+            const int tile = pair + i * num_pairs;
             const int m0 = (tile % p.num_m2) * 256 + 128 * int(rank), n0 = (tile / p.num_m2) * kGBN;
-            float2 acc[32];   // columns 64*half + 2j, +1
+            const int c = i >> 1;
+            float2 acc[64];   // columns 2j, 2j + 1 of the tile
 #pragma unroll
-            for (int j = 0; j < 32; ++j) acc[j] = make_float2(0.0f, 0.0f);
-            for (int g = 0; g < G; ++g, ++gcount) {
+            for (int j = 0; j < 64; ++j) acc[j] = make_float2(0.0f, 0.0f);
+            for (int g = 0; g < G; ++g) {
                 if ((g % kGScaleBlock) == 0) {
-                    // a thread whose wait gave up stops the whole epilogue here (uniform exit)
-                    if (gepi_any(aborted)) break;
-                    // this block's scales have landed, and every thread is done with the other
-                    // buffer: start copying the next block into it (one tile ahead at most)
+                    // a thread whose wait gave up stops the whole team here (uniform exit)
+                    if (team_any(team, aborted)) break;
+                    // this block's scales have landed, and every thread of the team is done
+                    // with the other buffer: start copying the next block into it
                     cp_async_wait_all();
-                    gepi_bar();
-                    if (g + kGScaleBlock < G) prefetch(tile, g + kGScaleBlock, sbuf ^ 1);
-                    else prefetch(tile + num_pairs, 0, sbuf ^ 1);
+                    team_bar(team);
+                    if (g + kGScaleBlock < G) prefetch(i, g + kGScaleBlock, sbuf ^ 1);
+                    else prefetch(i + 2, 0, sbuf ^ 1);
                 }
-                // group gcount's MMAs are complete when its stage's empty barrier completes
-                // that use; the epilogue trails the MMA by at most kGSlots < kGStages groups,
-                // so the parity cannot alias
-                const uint32_t slot = gcount % kGSlots;
-                const uint32_t gst = gcount % kGStages, gph = (gcount / kGStages) & 1;
-                if (!mbar_wait(bar_empty + 8 * gst, gph, abort_flag)) aborted = true;
+                // the team has G groups in every couple before c
+                const uint32_t ga = uint32_t(G) * uint32_t(c) + uint32_t(g);   // the team's group count
+                const uint32_t slot = 2 * team + (ga & 1);
+                if (!mbar_wait(bar_tfull + 8 * slot, (ga >> 1) & 1, abort_flag)) aborted = true;
                 if (aborted) continue;   // later waits return at once (abort flag); exit at the next check
                 tc_fence_after();
-                const uint32_t t_grp = tmem_base + lane_addr + slot * kGBN + 64 * half;
-                uint32_t r0[32], r1[32];
-                QUEST_TMEM_LD32(t_grp, r0);
-                QUEST_TMEM_LD32(t_grp + 32, r1);
-                tmem_wait_ld();
-                // the group's partials are in registers: hand the slot back
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive_remote(tempty_even + 8 * slot);
+                const uint32_t t_grp = tmem_base + lane_addr + slot * kGBN;
                 // (sa/2)(sb/2): the factor 1/4 rides on the row scale
-                const float* sblk = s_sc + sbuf * (kGScaleBytes / 4);
+                const float* sblk = reinterpret_cast<const float*>(smem + sc_base) + sbuf * (kGScaleBytes / 4);
                 const float sx = 0.25f * sblk[kGScaleBlock * kGBN + (g % kGScaleBlock) * 128 + row_in_tile];
-                const float4* sw4 = reinterpret_cast<const float4*>(sblk + (g % kGScaleBlock) * kGBN + 64 * half);
+                const float4* sw4 = reinterpret_cast<const float4*>(sblk + (g % kGScaleBlock) * kGBN);
                 if ((g % kGScaleBlock) == kGScaleBlock - 1 || g == G - 1) sbuf ^= 1;   // next block, other buffer
+                // 16 columns per TMEM load, two buffers: the load of columns 16 (q + 1) ..
+                // is in flight while columns 16 q .. are scaled and added
+                uint32_t rbuf[2][16];
+                QUEST_TMEM_LD16(t_grp, rbuf[0]);
+                QUEST_TMEM_WAIT16(rbuf[0]);
 #pragma unroll
-                for (int q4 = 0; q4 < 16; ++q4) {
-                    const float4 w4 = sw4[q4];
-                    const uint32_t* r = q4 < 8 ? r0 : r1;
-                    const int i = (q4 & 7) * 4;
-                    const float2 w01 = __fmul2_rn(make_float2(sx, sx), make_float2(w4.x, w4.y));
-                    const float2 w23 = __fmul2_rn(make_float2(sx, sx), make_float2(w4.z, w4.w));
-                    acc[2 * q4] = __ffma2_rn(make_float2(__uint_as_float(r[i]), __uint_as_float(r[i + 1])), w01,
-                                             acc[2 * q4]);
-                    acc[2 * q4 + 1] = __ffma2_rn(make_float2(__uint_as_float(r[i + 2]), __uint_as_float(r[i + 3])),
-                                                 w23, acc[2 * q4 + 1]);
+                for (int q = 0; q < 8; ++q) {
+                    uint32_t (&r)[16] = rbuf[q & 1];
+                    if (q < 7) QUEST_TMEM_LD16(t_grp + 16 * (q + 1), rbuf[(q + 1) & 1]);
+                    if (q == 7) {
+                        // the group's partials are all in registers: hand the slot back
+                        tc_fence_before();
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive_remote(tempty_even + 8 * slot);
+                    }
+#pragma unroll
+                    for (int v = 0; v < 4; ++v) {
+                        const float4 w4 = sw4[4 * q + v];
+                        const float2 w01 = __fmul2_rn(make_float2(sx, sx), make_float2(w4.x, w4.y));
+                        const float2 w23 = __fmul2_rn(make_float2(sx, sx), make_float2(w4.z, w4.w));
+                        float2& a0 = acc[8 * q + 2 * v];
+                        float2& a1 = acc[8 * q + 2 * v + 1];
+                        a0 = __ffma2_rn(make_float2(__uint_as_float(r[4 * v]), __uint_as_float(r[4 * v + 1])), w01,
+                                        a0);
+                        a1 = __ffma2_rn(make_float2(__uint_as_float(r[4 * v + 2]), __uint_as_float(r[4 * v + 3])),
+                                        w23, a1);
+                    }
+                    if (q < 7) QUEST_TMEM_WAIT16(rbuf[(q + 1) & 1]);
                 }
             }
-            if (gepi_any(aborted)) { aborted = true; break; }
-            // ---- output: this warp's 32 rows x 64 columns, in 2 chunks of 32 columns
+            if (team_any(team, aborted)) { aborted = true; break; }
+            // ---- output: this warp's 32 rows x 128 columns, in 4 chunks of 32 columns
             const int m = m0 + row_in_tile;
             if (p.y32 != nullptr && m < p.M) {
-                float* yrow = p.y32 + int64_t(m) * p.N + n0 + 64 * half;
+                float* yrow = p.y32 + int64_t(m) * p.N + n0;
 #pragma unroll
-                for (int j = 0; j < 32; ++j) {
-                    const int n = n0 + 64 * half + 2 * j;
+                for (int j = 0; j < 64; ++j) {
+                    const int n = n0 + 2 * j;
                     if (n < p.N) yrow[2 * j] = acc[j].x;
                     if (n + 1 < p.N) yrow[2 * j + 1] = acc[j].y;
                 }
             }
             const uint32_t swz = (lane >> 1) & 3;
 #pragma unroll
-            for (int c = 0; c < 2; ++c) {
+            for (int q = 0; q < 4; ++q) {
                 if (lane == 0) bulk_wait_read_le1();   // the buffer used two chunks ago is free
                 __syncwarp();
                 const uint32_t stg = stg0 + cbuf * kGCBytes + lane * 64;
@@ -332,7 +384,7 @@ w4a4_gemm_grouped_kernel(const __grid_constant__ CUtensorMap map_a, const __grid
                     uint32_t w[4];
 #pragma unroll
                     for (int h = 0; h < 4; ++h) {
-                        const float2 v = acc[c * 16 + q16 * 4 + h];
+                        const float2 v = acc[q * 16 + q16 * 4 + h];
                         __nv_bfloat162 hb = __floats2bfloat162_rn(v.x, v.y);
                         w[h] = *reinterpret_cast<uint32_t*>(&hb);
                     }
@@ -343,7 +395,7 @@ w4a4_gemm_grouped_kernel(const __grid_constant__ CUtensorMap map_a, const __grid
                 fence_proxy_async_smem();
                 __syncwarp();
                 if (lane == 0) {
-                    tma_store_2d(&map_y, stg0 + cbuf * kGCBytes, n0 + 64 * half + c * kChunkCols, m0 + 32 * quarter);
+                    tma_store_2d(&map_y, stg0 + cbuf * kGCBytes, n0 + q * kChunkCols, m0 + 32 * quarter);
                     bulk_commit();
                 }
                 cbuf ^= 1;

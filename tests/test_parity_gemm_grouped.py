@@ -60,6 +60,14 @@ def test_grouped_shapes(cuda_device, M, N, K):
     check(*_case(M, N, K, seed=M + N + K))
 
 
+@pytest.mark.parametrize("M,N,K", [(2560, 2080, 640), (9400, 1272, 128), (7424, 1016, 384)])
+def test_grouped_several_tiles_per_pair(cuda_device, M, N, K):
+    # more pair tiles than CTA pairs on the part (148 SMs: 74 pairs): each pair takes
+    # 2-3, 5 or 3-4 tiles, two at a time (odd counts leave a last tile alone), with an
+    # odd number of K groups (5, 1, 3) and ragged rows or columns
+    check(*_case(M, N, K, seed=M + N + K))
+
+
 def test_grouped_largest_codes(cuda_device):
     # |c| = 15 everywhere: every group's product is +-128 * 225 = +-28800
     M, N, K = 256, 256, 512
