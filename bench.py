@@ -689,7 +689,7 @@ def run_configs(args):
     flush = L2Flush(dev)
     rows = []
 
-    def add(name, f, nbytes, unit_ops=None, extra=None, bf16=False):
+    def add(name, f, nbytes, unit_ops=None, extra=None, bf16=False, fp4=False):
         med, p10 = _timed(f, flush, stream)
         r = {"case": name, "median_us": round(med, 2), "p10_us": round(p10, 2), "bytes": nbytes,
              "gbs": round(nbytes / (med * 1e-6) / 1e9, 1)}
@@ -701,6 +701,8 @@ def run_configs(args):
         elif unit_ops:
             r["tops"] = round(unit_ops / (med * 1e-6) / 1e12, 1)
             r["frac_int8_peak"] = round(r["tops"] / (peaks["bf16_tflops"] * 2.0), 4)
+            if fp4:   # nominal dense FP4 : bf16 ratio 9 : 2.25
+                r["frac_fp4_peak"] = round(r["tops"] / (peaks["bf16_tflops"] * 4.0), 4)
         if extra:
             r.update(extra)
         rows.append(r)
@@ -801,6 +803,15 @@ def run_configs(args):
                                   y.data_ptr(), None, s)
     add("FP4 linear 16384x5632x2048 (c=2Q codes, int8 tensor cores)", f,
         R * C + NW * C + 4 * (R + NW) + 2 * R * NW, unit_ops=GEMM_OPS)
+    # the same layer on the block-scaled FP4 tensor cores: packed E2M1 codes, one RMS per row
+    fxp, nbxp, (cxp, sxp, _) = quant(x2, 4, C, F4, None)
+    fwp, nbwp, (cwp, swp, _) = quant(w, 4, C, F4, None)
+    add("FP4 packed quantize X 16384x2048 E2M1 (row RMS)", fxp, nbxp)
+    fxp(); fwp()
+    f = lambda: q.fp4_linear_raw(cxp.data_ptr(), sxp.data_ptr(), cwp.data_ptr(), swp.data_ptr(), R, NW, C,
+                                 y.data_ptr(), None, s)
+    add("FP4 linear 16384x5632x2048 (packed E2M1, block-scaled FP4 tensor cores)", f,
+        R * C // 2 + NW * C // 2 + 4 * (R + NW) + 2 * R * NW, unit_ops=GEMM_OPS, fp4=True)
     # the input gradient of the layer with the trust backward fused into the bf16
     # product: w_hat from the weight quantizer's bf16 dequant, laid out [K, N] by the
     # library's transpose, X's trust mask from the trust backward case above

@@ -33,6 +33,7 @@ SIGNATURES = {
     "quest_trust_bwd_linear": (_int, [_p, _p, _p, _i64, _i64, _i64, _int, _p, _p]),
     "quest_transpose_bf16": (_int, [_p, _i64, _i64, _p, _p]),
     "quest_linear_bf16": (_int, [_p, _p, _i64, _i64, _i64, _p, _p]),
+    "quest_fp4_linear": (_int, [_p, _p, _p, _p, _i64, _i64, _i64, _p, _p, _p]),
     "quest_device_status": (_int, [_p]),
     "quest_alpha": (_f64, [_int]),
     "quest_alpha_fp4": (_f64, []),
@@ -125,6 +126,11 @@ def trust_bwd_linear_raw(grad_y, w_hat_t, mask, M, N, K, had_block, grad_x, stre
 
 def linear_bf16_raw(x_hat, w_hat, M, N, K, y, stream=0):
     _check(load_library().quest_linear_bf16(x_hat, w_hat, M, N, K, y, stream), "quest_linear_bf16")
+
+
+def fp4_linear_raw(a_codes, a_scales, w_codes, w_scales, M, N, K, y, acc=None, stream=0):
+    _check(load_library().quest_fp4_linear(a_codes, a_scales, w_codes, w_scales, M, N, K, y, acc, stream),
+           "quest_fp4_linear")
 
 
 def transpose_bf16_raw(src, rows, cols, dst, stream=0):
@@ -346,6 +352,29 @@ def w4a4_linear(a_codes, a_scales, w_codes, w_scales, out=None, acc: bool = Fals
     w4a4_linear_raw(a_codes.data_ptr(), a_scales.data_ptr(), w_codes.data_ptr(), w_scales.data_ptr(),
                     M, N, K, out.data_ptr(), acc_t.data_ptr() if acc_t is not None else None,
                     _stream_handle(stream, dev))
+    return (out, acc_t) if acc else out
+
+
+def fp4_linear(a_codes, a_scales, w_codes, w_scales, K: int, out=None, acc: bool = False, stream=None):
+    """y = bf16((Q_a @ Q_w^T) * a_scales[:, None] * w_scales[None, :]) on packed E2M1 codes
+    (uint8 [M, K/2] and [N, K/2], the CODES_FP4_PACKED form with one scale per row).
+    Returns y (and the fp32 accumulator sum_k Q_a Q_w if acc)."""
+    torch = _torch()
+    for t, n in ((a_codes, "a_codes"), (w_codes, "w_codes"), (a_scales, "a_scales"), (w_scales, "w_scales")):
+        _require_cuda(t, n)
+    if a_codes.dtype not in (torch.int8, torch.uint8) or w_codes.dtype not in (torch.int8, torch.uint8):
+        raise QuestError("packed codes must be uint8")
+    if not (a_codes.is_contiguous() and w_codes.is_contiguous()):
+        raise QuestError("codes must be contiguous")
+    M, N = a_scales.numel(), w_scales.numel()   # one scale per row
+    if a_codes.numel() < M * (K // 2) or w_codes.numel() < N * (K // 2):
+        raise QuestError("codes must hold K/2 bytes per row")
+    dev = a_codes.device
+    if out is None:
+        out = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+    acc_t = torch.empty((M, N), dtype=torch.float32, device=dev) if acc else None
+    fp4_linear_raw(a_codes.data_ptr(), a_scales.data_ptr(), w_codes.data_ptr(), w_scales.data_ptr(), M, N, K,
+                   out.data_ptr(), acc_t.data_ptr() if acc_t is not None else None, _stream_handle(stream, dev))
     return (out, acc_t) if acc else out
 
 

@@ -16,7 +16,7 @@ ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(HERE, "libquest_b200.so")
-SOURCES = ["quest_api.cu", "quantize_fwd.cu", "quantize_hs.cu", "quantize_tc.cu", "trust_bwd.cu", "trust_tc.cu", "w4a4_gemm.cu", "w4a4_grouped.cu", "trust_linear.cu", "tc_host.cu", "transpose.cu",
+SOURCES = ["quest_api.cu", "quantize_fwd.cu", "quantize_hs.cu", "quantize_tc.cu", "trust_bwd.cu", "trust_tc.cu", "w4a4_gemm.cu", "w4a4_grouped.cu", "trust_linear.cu", "fp4_gemm.cu", "tc_host.cu", "transpose.cu",
            "probe_mma.cu"]
 HEADERS = ["quest_device.cuh", "quest_internal.h", "quest_emit.cuh", "quest_tc.cuh", "tc_common.cuh"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]

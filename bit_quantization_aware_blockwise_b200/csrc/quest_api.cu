@@ -487,6 +487,32 @@ quest_status quest_w4a4_linear(const int8_t* a_codes, const float* a_scales,
     return QUEST_OK;
 }
 
+quest_status quest_fp4_linear(const uint8_t* a_codes, const float* a_scales, const uint8_t* w_codes,
+                              const float* w_scales, int64_t M, int64_t N, int64_t K, void* y, float* acc,
+                              void* stream) {
+    g_last_error.clear();
+    if (M < 0 || N < 0 || K < 0) return fail(QUEST_EINVAL, "M, N and K must be >= 0");
+    if (M >= (int64_t(1) << 31) || N >= (int64_t(1) << 31)) return fail(QUEST_EINVAL, "M and N must be < 2^31");
+    if (K % 32 != 0) return fail(QUEST_EINVAL, "K must be a multiple of 32");
+    if (K > 16384) return fail(QUEST_EINVAL, "K must be <= 16384 (exact fp32 accumulation bound)");
+    if (N % 8 != 0) return fail(QUEST_EINVAL, "N must be a multiple of 8");
+    if (M > 0 && N > 0) {
+        if (!y) return fail(QUEST_EINVAL, "y must be non-NULL");
+        if (K > 0 && (!a_codes || !w_codes || !a_scales || !w_scales))
+            return fail(QUEST_EINVAL, "codes and scales must be non-NULL");
+        if (K > 0 && (!aligned(a_codes, 16) || !aligned(w_codes, 16)))
+            return fail(QUEST_EINVAL, "codes must be 16-byte aligned");
+        if (!aligned(y, 16)) return fail(QUEST_EINVAL, "y must be 16-byte aligned");
+        if ((a_scales && !aligned(a_scales, 4)) || (w_scales && !aligned(w_scales, 4)) || (acc && !aligned(acc, 4)))
+            return fail(QUEST_EINVAL, "scales and acc must be 4-byte aligned");
+    }
+    cudaError_t e = launch_fp4_linear(a_codes, a_scales, w_codes, w_scales, M, N, K, static_cast<uint16_t*>(y), acc,
+                                      static_cast<cudaStream_t>(stream));
+    if (e == cudaErrorInvalidValue) return fail(QUEST_ECUDA, "quest_fp4_linear: tensor map encoding failed");
+    if (e != cudaSuccess) return cuda_fail(e, "quest_fp4_linear launch");
+    return QUEST_OK;
+}
+
 quest_status quest_w4a4_linear_grouped(const uint8_t* a_codes, const float* a_scales,
                                        const uint8_t* w_codes, const float* w_scales, int64_t M,
                                        int64_t N, int64_t K, int64_t group, void* y, float* y_f32,
@@ -606,10 +632,13 @@ quest_status quest_device_status(void* stream) {
     if (e != cudaSuccess) return cuda_fail(e, "quest_device_status");
     const int vtl = read_and_clear_trust_linear_status(s, &e);
     if (e != cudaSuccess) return cuda_fail(e, "quest_device_status");
+    const int vf4 = read_and_clear_fp4_status(s, &e);
+    if (e != cudaSuccess) return cuda_fail(e, "quest_device_status");
     if (vg != 0) return fail((quest_status)vg, "a bounded device-side wait in quest_w4a4_linear gave up");
     if (vgr != 0) return fail((quest_status)vgr, "a bounded device-side wait in quest_w4a4_linear_grouped gave up");
     if (vtl != 0)
         return fail((quest_status)vtl, "a bounded device-side wait in quest_trust_bwd_linear or quest_linear_bf16 gave up");
+    if (vf4 != 0) return fail((quest_status)vf4, "a bounded device-side wait in quest_fp4_linear gave up");
     return QUEST_OK;
 }
 

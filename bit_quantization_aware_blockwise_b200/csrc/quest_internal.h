@@ -92,11 +92,13 @@ cudaError_t launch_w4a4(const int8_t* A, const float* sa, const int8_t* B, const
                         cudaStream_t stream);
 
 // Read (synchronising `stream`) and clear the device status word of the integer
-// linear layer (w4a4_gemm.cu), the grouped layer (w4a4_grouped.cu) and the fused
-// input gradient (trust_linear.cu); each returns its value (0 or a quest_status).
+// linear layer (w4a4_gemm.cu), the grouped layer (w4a4_grouped.cu), the fused
+// input gradient (trust_linear.cu) and the FP4 layer (fp4_gemm.cu); each returns
+// its value (0 or a quest_status).
 int read_and_clear_gemm_status(cudaStream_t stream, cudaError_t* err);
 int read_and_clear_grouped_status(cudaStream_t stream, cudaError_t* err);
 int read_and_clear_trust_linear_status(cudaStream_t stream, cudaError_t* err);
+int read_and_clear_fp4_status(cudaStream_t stream, cudaError_t* err);
 // dst[c][r] = src[r][c] for bf16 [rows, cols] (transpose.cu).
 cudaError_t launch_transpose_bf16(const uint16_t* src, int64_t rows, int64_t cols, uint16_t* dst,
                                   cudaStream_t stream);
@@ -107,6 +109,9 @@ cudaError_t launch_trust_linear(const uint16_t* gy, const uint16_t* wt, const ui
 // y [M, N] = x_hat [M, K] w_hat [N, K]^T on bf16 operands, fp32 accumulation (trust_linear.cu).
 cudaError_t launch_linear_bf16(const uint16_t* x_hat, const uint16_t* w_hat, int64_t M, int64_t N, int64_t K,
                                uint16_t* y, cudaStream_t stream);
+// y [M, N] = (sum_k Q_a Q_w) sa[m] sb[n] on packed E2M1 codes, block-scaled FP4 MMA (fp4_gemm.cu).
+cudaError_t launch_fp4_linear(const uint8_t* A, const float* sa, const uint8_t* B, const float* sb, int64_t M,
+                              int64_t N, int64_t K, uint16_t* y, float* acc, cudaStream_t stream);
 cudaError_t launch_w4a4_grouped(const int8_t* A, const float* sa, const int8_t* B, const float* sb,
                                 int64_t M, int64_t N, int64_t K, uint16_t* y, float* y32,
                                 cudaStream_t stream);

@@ -97,6 +97,12 @@ def gemm_codes(rows: int, cols: int, seed: int, bits: int = 4) -> np.ndarray:
     return (2 * q + 1).astype(np.int8)
 
 
+def fp4_codes(rows: int, cols: int, seed: int) -> np.ndarray:
+    """Packed 4-bit codes [rows, cols/2] bytes, every nibble uniform over its 16 values
+    (two per byte, element 2j in the low nibble)."""
+    return rng(seed).integers(0, 256, size=(rows, cols // 2)).astype(np.uint8)
+
+
 def positive_scales(n: int, seed: int, lo: float = 1e-3, hi: float = 5e-2) -> np.ndarray:
     """Positive fp32 per-row scale factors, log-uniform in [lo, hi]."""
     u = rng(seed).random(n)

@@ -266,6 +266,41 @@ quest_status quest_w4a4_linear_grouped(const uint8_t* a_codes, const float* a_sc
                                        void* stream);
 
 /*
+ * quest_fp4_linear -- linear layer on FP4 (E2M1) QuEST codes on the block-scaled
+ * FP4 tensor cores.
+ *
+ * The FP4-grid variant of the quantizer (pith.science review, Figure 4a and
+ * "Assumptions & free parameters"; the codes of a quantize_fwd call with
+ * code_mode QUEST_CODES_FP4_PACKED and rms_group = cols, so one step Delta per
+ * row) feeds the layer directly:
+ *     acc[m][n] = sum_k Q_a[m][k] * Q_w[n][k]     (Q the E2M1 grid values)
+ *     y[m][n]   = bf16_rne( acc[m][n] * a_scales[m] * w_scales[n] )
+ * Every product of two E2M1 values is a multiple of 1/4 of magnitude <= 36, so
+ * for K <= 16384 every partial sum is a multiple of 1/4 below 2^20 and the fp32
+ * accumulation is exact. Same result as quest_w4a4_linear on the operand form
+ * c = 2Q (QUEST_CODES_FP4_OPERAND), at twice its tensor-core rate and half its
+ * operand bytes.
+ *
+ * Arguments
+ *   a_codes    device, packed E2M1 [M, K/2] bytes (element 2j in the low nibble
+ *              of byte j); 16-byte aligned.
+ *   a_scales   device, fp32 [M] (Delta of each row).
+ *   w_codes    device, packed E2M1 [N, K/2] bytes; 16-byte aligned.
+ *   w_scales   device, fp32 [N].
+ *   M >= 0, N >= 0 (0 = no-op); N a multiple of 8; K >= 0, a multiple of 32,
+ *   K <= 16384.
+ *   y          device, bf16 [M, N]; 16-byte aligned.
+ *   acc        device, optional fp32 [M, N] copy of the accumulator (NULL = not
+ *              written); meant for exactness checks.
+ * Errors: QUEST_EINVAL on bad sizes, NULL or misaligned pointers (checked before
+ * any launch); QUEST_ECUDA on a launch failure. A bounded device-side wait that
+ * gives up is reported by quest_device_status as QUEST_ETIMEOUT.
+ */
+quest_status quest_fp4_linear(const uint8_t* a_codes, const float* a_scales, const uint8_t* w_codes,
+                              const float* w_scales, int64_t M, int64_t N, int64_t K, void* y, float* acc,
+                              void* stream);
+
+/*
  * quest_trust_bwd_linear -- input gradient of a QuEST linear layer with the
  * trust backward fused into the product.
  *

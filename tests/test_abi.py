@@ -197,3 +197,15 @@ def test_linear_bf16_rejects_invalid_arguments():
                dict(y=FAKE + 64), dict(M=1 << 31)]:
         assert call(**kw) == 1, kw
     assert call(M=0, x=None, w=None, y=None) == 0
+
+
+def test_fp4_linear_rejects_invalid_arguments():
+    lib = q.load_library()
+
+    def call(a=FAKE, sa=FAKE + (1 << 20), w=FAKE + (1 << 24), sw=FAKE + (1 << 21), M=4, N=16, K=64,
+             y=FAKE + (1 << 25), acc=None):
+        return lib.quest_fp4_linear(a, sa, w, sw, M, N, K, y, acc, None)
+    for kw in [dict(M=-1), dict(K=48), dict(K=16416), dict(N=12), dict(y=None), dict(a=None), dict(sw=None),
+               dict(w=FAKE + 8), dict(sa=FAKE + 2), dict(acc=FAKE + 6), dict(y=FAKE + 8), dict(M=1 << 31)]:
+        assert call(**kw) == 1, kw
+    assert call(M=0, a=None, w=None, sa=None, sw=None, y=None) == 0
