@@ -893,12 +893,15 @@ def run_profile_kernels(args):
     wt = q.transpose_bf16(inputs.weight_up().to(dev))                                  # 7
     gx = q.trust_bwd_linear(gyl, wt, out["mask"][: 8192 * C // 8])                     # 8
     yf = q.linear_bf16(x[:8192], w_up)                                                 # 9
+    pa4 = torch.from_numpy(inputs.fp4_codes(8192, 2048, seed=35)).to(dev)
+    pw4 = torch.from_numpy(inputs.fp4_codes(NW, 2048, seed=36)).to(dev)
+    y4 = q.fp4_linear(pa4, sa.repeat(2), pw4, sb, 2048)                                # 10
     torch.cuda.synchronize()
     q.device_status()
     print(json.dumps({"profile_kernels": "ok", "rows": rows, "checksum": [
         float(out["scales"].sum()), float(gi.float().abs().sum()), float(op["scales"].sum()),
         float(y.float().abs().sum()), float(yg.float().abs().sum()), float(f4["scales"].sum()),
-        float(gx.float().abs().sum()), float(yf.float().abs().sum())]}))
+        float(gx.float().abs().sum()), float(yf.float().abs().sum()), float(y4.float().abs().sum())]}))
 
 
 def main():
