@@ -22,8 +22,13 @@
 // (256 FP4 values per row per stage); four tcgen05.mma (K = 64 each) per stage;
 // two 224-column fp32 accumulators (TMEM columns 0 and 256) alternate so the
 // epilogue of one tile overlaps the mainloop of the next; TMEM columns 480-511
-// hold the scale bytes. Epilogue as in the integer layer: 32 columns per TMEM
-// load, scale, round to bf16, 64-byte-swizzled staging, TMA store. Every
+// hold the scale bytes. Epilogue: eight warps, two per TMEM lane quarter, each
+// taking half of the tile's columns of its 32 accumulator rows, 32 columns at a
+// time: scale, round to bf16, store through its own 64-byte-swizzled staging
+// buffers and TMA stores (warp-level syncs only). At the FP4 rate a tile's
+// mainloop is short (about 3.8K cycles), and with one warp per lane quarter the
+// epilogue did not fit in it (16384 x 5632 x 2048: 94.7 us, against 75.8 us with
+// the epilogue skipped). Every
 // mbarrier wait is bounded; a timeout records QUEST_ETIMEOUT in the device
 // status word and the CTA drains its copies, frees TMEM and returns.
 #include <cuda.h>
@@ -45,6 +50,10 @@ namespace quest {
 namespace {
 
 constexpr int kFBN = 224;                                   // output columns per pair tile
+constexpr int kFThreads = 320;                              // producer, MMA, 8 epilogue warps
+constexpr int kFEpiThreads = 256;
+constexpr int kFChunks = kFBN / kChunkCols;                 // 7 column chunks: warps of half 0 take 4, half 1 take 3
+constexpr int kFHalfChunks = (kFChunks + 1) / 2;
 constexpr int kFStages = 6;
 constexpr uint32_t kFStageA = 128 * BK;                     // 128 rows x 128 bytes (256 FP4 values)
 constexpr uint32_t kFStageB = (kFBN / 2) * BK;              // 112 rows x 128 bytes
@@ -52,7 +61,8 @@ constexpr uint32_t kFTxBytes = 2 * (kFStageA + kFStageB);   // both CTAs land on
 constexpr uint32_t kFSmemA = 0;
 constexpr uint32_t kFSmemB = kFSmemA + kFStages * kFStageA;
 constexpr uint32_t kFSmemC = kFSmemB + kFStages * kFStageB;
-constexpr uint32_t kFSmemScale = kFSmemC + 2 * kCBytes;     // float[kFBN]
+constexpr uint32_t kFWarpCBytes = 32 * kChunkCols * 2;      // one warp's 32 x 32 bf16 staging chunk
+constexpr uint32_t kFSmemScale = kFSmemC + 8 * 2 * kFWarpCBytes;   // float[kFBN]
 constexpr uint32_t kFSmemBar = kFSmemScale + kFBN * 4;
 constexpr uint32_t kFNumBars = 2 * kFStages + 4 + 1;
 constexpr uint32_t kFSmemTmemSlot = kFSmemBar + kFNumBars * 8;
@@ -81,6 +91,21 @@ __device__ __forceinline__ void tc_mma_fp4_pair(uint32_t d_tmem, uint64_t adesc,
         : "memory");
 }
 
+// Named barrier 1 over the 256 epilogue threads, and an OR-vote on it.
+__device__ __forceinline__ void fepi_bar() { asm volatile("bar.sync 1, %0;" ::"n"(kFEpiThreads) : "memory"); }
+__device__ __forceinline__ bool fepi_any(bool pred) {
+    uint32_t out;
+    asm volatile(
+        "{\n\t.reg .pred p, q;\n\t"
+        "setp.ne.u32 p, %1, 0;\n\t"
+        "bar.red.or.pred q, 1, %2, p;\n\t"
+        "selp.u32 %0, 1, 0, q;\n\t}"
+        : "=r"(out)
+        : "r"((uint32_t)pred), "n"(kFEpiThreads)
+        : "memory");
+    return out != 0;
+}
+
 // 32 consecutive TMEM columns of this warp's 32 lanes <- the same 32-bit word.
 __device__ __forceinline__ void tmem_fill32(uint32_t taddr, uint32_t v) {
     asm volatile(
@@ -100,7 +125,7 @@ struct Fp4Params {
     int num_m2, num_n, num_k;   // 256-row pair tiles, 224-column tiles, 256-value K steps
 };
 
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kFThreads, 1)
 fp4_gemm_pair_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_b,
                      const __grid_constant__ CUtensorMap map_y, const Fp4Params p) {
     extern __shared__ uint8_t smem_raw[];
@@ -128,7 +153,7 @@ fp4_gemm_pair_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_con
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(bar_tfull + 8 * b, 1);
-            mbar_init(bar_tempty + 8 * b, 2);   // one arrival from each CTA's epilogue
+            mbar_init(bar_tempty + 8 * b, 16);   // one arrival from each epilogue warp of both CTAs
         }
         mbar_init(bar_drain, 1);
         *abort_flag = 0;
@@ -229,9 +254,11 @@ fp4_gemm_pair_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_con
             }
         }
     } else {
-        // ------------------------------------------------------------ epilogue (warps 2..5, both CTAs)
-        const int et = threadIdx.x - 64;
-        const int quarter = warp & 3;
+        // ------------------------------------------------------------ epilogue (warps 2..9, both CTAs)
+        const int et = threadIdx.x - 64;             // 0..255
+        const int quarter = warp & 3;                // TMEM lanes 32*quarter .. +31
+        const int half = (warp - 2) >> 2;            // column chunks [0, 4) or [4, 7)
+        const int c_lo = half * kFHalfChunks, c_hi = half ? kFChunks : kFHalfChunks;
         const int row_in_tile = quarter * 32 + lane;
         const uint32_t lane_addr = uint32_t(quarter * 32) << 16;
         const uint32_t tempty_even = map_to_rank(bar_tempty, 0);
@@ -240,25 +267,36 @@ fp4_gemm_pair_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_con
         for (int tile = pair; tile < num_tiles; tile += num_pairs, ++local) {
             const int m0 = (tile % p.num_m2) * 256 + 128 * int(rank), n0 = (tile / p.num_m2) * kFBN;
             const uint32_t buf = local & 1, bphase = (local >> 1) & 1;
-            epi_bar();   // everyone is done with the previous tile's column scales
-            for (int c = et; c < kFBN; c += kEpiThreads) {
+            fepi_bar();   // everyone is done with the previous tile's column scales
+            for (int c = et; c < kFBN; c += kFEpiThreads) {
                 const int n = n0 + c;
                 s_scale[c] = n < p.N ? p.sb[n] : 0.0f;
             }
             const int m = m0 + row_in_tile;
             const float sa_m = m < p.M ? p.sa[m] : 0.0f;
             const bool got = mbar_wait(bar_tfull + 8 * buf, bphase, abort_flag);
-            if (epi_any(!got)) break;
+            if (fepi_any(!got)) break;
             tc_fence_after();
             const uint32_t t_acc = tmem_base + lane_addr + buf * kFAccStride;
+            // each warp stores its own 32 rows: 32 x 32 bf16 chunks through two staging
+            // buffers of its own, so no chunk waits on the other warps
+            const uint32_t stg_w = sbase + kFSmemC + uint32_t(warp - 2) * 2 * kFWarpCBytes;
+            const uint32_t swz = (lane >> 1) & 3;
 #pragma unroll 1
-            for (int c = 0; c < kFBN / kChunkCols; ++c) {
+            for (int c = c_lo; c < c_hi; ++c) {
                 uint32_t r[32];
                 QUEST_TMEM_LD32(t_acc + c * kChunkCols, r);
                 tmem_wait_ld();
+                if (c == c_hi - 1) {
+                    // this warp's part of the accumulator is read: hand it back to the MMA
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive_remote(tempty_even + 8 * buf);
+                }
                 const float* sc = s_scale + c * kChunkCols;
-                const uint32_t stg = sbase + kFSmemC + cbuf * kCBytes + row_in_tile * (kChunkCols * 2);
-                const uint32_t swz = (row_in_tile >> 1) & 3;
+                if (lane == 0) bulk_wait_read_le1();   // the buffer used two chunks ago is free
+                __syncwarp();
+                const uint32_t stg = stg_w + cbuf * kFWarpCBytes + lane * (kChunkCols * 2);
 #pragma unroll
                 for (int q16 = 0; q16 < 4; ++q16) {
                     uint32_t w[4];
@@ -283,20 +321,15 @@ fp4_gemm_pair_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_con
                     }
                 }
                 fence_proxy_async_smem();
-                epi_bar();
-                if (et == 0) {
-                    tma_store_2d(&map_y, sbase + kFSmemC + cbuf * kCBytes, n0 + c * kChunkCols, m0);
+                __syncwarp();
+                if (lane == 0) {
+                    tma_store_2d(&map_y, stg_w + cbuf * kFWarpCBytes, n0 + c * kChunkCols, m0 + 32 * quarter);
                     bulk_commit();
-                    bulk_wait_read_le1();   // the other staging buffer is free again
                 }
-                epi_bar();
                 cbuf ^= 1;
             }
-            tc_fence_before();
-            epi_bar();
-            if (et == 0) mbar_arrive_remote(tempty_even + 8 * buf);
         }
-        if (et == 0) bulk_wait_all();
+        if (lane == 0) bulk_wait_all();
     }
 
     tc_fence_before();
@@ -321,7 +354,7 @@ cudaError_t launch_fp4_linear(const uint8_t* A, const float* sa, const uint8_t* 
     CUtensorMap ma, mb, my;
     if (!make_map_2d(&ma, CU_TENSOR_MAP_DATA_TYPE_UINT8, A, kb, M, kb, BK, 128, CU_TENSOR_MAP_SWIZZLE_128B) ||
         !make_map_2d(&mb, CU_TENSOR_MAP_DATA_TYPE_UINT8, B, kb, N, kb, BK, kFBN / 2, CU_TENSOR_MAP_SWIZZLE_128B) ||
-        !make_map_2d(&my, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, y, N, M, N * 2, kChunkCols, 128,
+        !make_map_2d(&my, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, y, N, M, N * 2, kChunkCols, 32,
                      CU_TENSOR_MAP_SWIZZLE_64B))
         return cudaErrorInvalidValue;
     Fp4Params p;
@@ -340,9 +373,10 @@ cudaError_t launch_fp4_linear(const uint8_t* A, const float* sa, const uint8_t* 
         attr_dev = dev;
     }
     const int tiles = p.num_m2 * p.num_n;
-    const int pairs = pair_clusters(dev, (const void*)fp4_gemm_pair_kernel, kThreads, kFSmemTotal);
+    const int pairs = pair_clusters(dev, (const void*)fp4_gemm_pair_kernel, kFThreads, kFSmemTotal);
     const int grid_pairs = tiles < pairs ? tiles : pairs;
-    return launch_pdl(fp4_gemm_pair_kernel, dim3(2 * grid_pairs), dim3(kThreads), kFSmemTotal, stream, ma, mb, my, p);
+    return launch_pdl(fp4_gemm_pair_kernel, dim3(2 * grid_pairs), dim3(kFThreads), kFSmemTotal, stream, ma, mb, my,
+                      p);
 }
 
 int read_and_clear_fp4_status(cudaStream_t stream, cudaError_t* err) {
