@@ -40,7 +40,7 @@ extern "C" {
 typedef enum quest_status {
     QUEST_OK = 0,
     QUEST_EINVAL = 1,         /* an argument is out of range, NULL or misaligned */
-    QUEST_EUNSUPPORTED = 2,   /* a valid request this build does not implement */
+    QUEST_EUNSUPPORTED = 2,   /* a valid request the library does not implement */
     QUEST_ECUDA = 3,          /* CUDA launch / driver error */
     QUEST_ETIMEOUT = 4        /* a bounded device-side wait gave up */
 } quest_status;
