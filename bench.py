@@ -428,25 +428,27 @@ def run_b200(args, world, rank, local):
         print(json.dumps(result), flush=True)
 
 
-def mma_probe(dev, gemm_tops, iters=20000, reps=5):
-    """int8 tensor-core rate with no memory traffic (back-to-back tcgen05.mma
-    kind::i8, M 128 N 256 K 32, one CTA per SM): context for the GEMM's fraction."""
+def mma_probe(dev, gemm_tops, iters=20000, reps=5, fp4=False):
+    """Tensor-core rate with no memory traffic (back-to-back tcgen05.mma, one CTA per
+    SM): kind::i8 M 128 N 256 K 32, or with fp4 kind::mxf4 M 128 N 256 K 64 with unit
+    block scales; context for the linear layers' fractions."""
     import statistics
     import torch
     import bit_quantization_aware_blockwise_b200 as q
     stream = torch.cuda.current_stream(dev)
-    q.probe_mma_i8(iters, stream.cuda_stream)
+    launch = q.probe_mma_fp4 if fp4 else q.probe_mma_i8
+    launch(iters, stream.cuda_stream)
     ts, ctas = [], 0
     for _ in range(reps):
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         a.record(stream)
-        ctas = q.probe_mma_i8(iters, stream.cuda_stream)
+        ctas = launch(iters, stream.cuda_stream)
         b.record(stream)
         torch.cuda.synchronize()
         ts.append(a.elapsed_time(b))
     q.probe_status(stream.cuda_stream)
     ms = statistics.median(ts)
-    tops = 2.0 * 128 * 256 * 32 * iters * ctas / (ms * 1e-3) / 1e12
+    tops = 2.0 * 128 * 256 * (64 if fp4 else 32) * iters * ctas / (ms * 1e-3) / 1e12
     return {"tops": round(tops, 1), "iters": iters, "ctas": ctas,
             "gemm_frac_of_probe": round(gemm_tops / tops, 4),
             "note": "timed alone right after the bench loop; the roofline peak stays the measured bf16 x 2"}
@@ -861,7 +863,11 @@ def run_configs(args):
     gemm_tops = next(r["tops"] for r in rows if r["case"].startswith("W4A4 linear"))
     q.device_status()
     probe = mma_probe(dev, gemm_tops)
-    print(json.dumps({"configs": rows, "int8_mma_probe": probe, "peaks": peaks}), flush=True)
+    fp4_tops = next(r["tops"] for r in rows if "block-scaled FP4" in r["case"])
+    probe4 = mma_probe(dev, fp4_tops, fp4=True)
+    probe4["note"] = "timed alone after the configs; the FP4 layer's fraction stays of 4 x the measured bf16 peak"
+    print(json.dumps({"configs": rows, "int8_mma_probe": probe, "fp4_mma_probe": probe4, "peaks": peaks}),
+          flush=True)
 
 
 def run_profile_kernels(args):

@@ -45,6 +45,7 @@ from ._binding import (  # noqa: F401
     fp4_linear_raw,
     device_status,
     probe_mma_i8,
+    probe_mma_fp4,
     probe_status,
 )
 
@@ -55,5 +56,5 @@ __all__ = [
     "container_bits", "quantize_fwd", "quantize_operands", "quantize_operands_raw", "trust_bwd", "w4a4_linear", "quantize_fwd_raw",
     "trust_bwd_raw", "w4a4_linear_raw", "w4a4_linear_grouped", "w4a4_linear_grouped_raw",
     "trust_bwd_linear", "trust_bwd_linear_raw", "transpose_bf16", "transpose_bf16_raw",
-    "linear_bf16", "linear_bf16_raw", "fp4_linear", "fp4_linear_raw", "device_status", "probe_mma_i8", "probe_status",
+    "linear_bf16", "linear_bf16_raw", "fp4_linear", "fp4_linear_raw", "device_status", "probe_mma_i8", "probe_mma_fp4", "probe_status",
 ]

@@ -44,6 +44,7 @@ SIGNATURES = {
     "quest_last_error_message": (ctypes.c_char_p, []),
     "quest_version": (_int, []),
     "quest_probe_mma_i8": (_int, [_int, _p, _p]),
+    "quest_probe_mma_fp4": (_int, [_int, _p, _p]),
     "quest_probe_status": (_int, [_p]),
 }
 
@@ -413,6 +414,13 @@ def probe_mma_i8(iters, stream=0):
     """Enqueue the int8 tensor-core peak probe; returns the number of CTAs launched."""
     ctas = ctypes.c_int(0)
     _check(load_library().quest_probe_mma_i8(iters, ctypes.byref(ctas), stream), "quest_probe_mma_i8")
+    return ctas.value
+
+
+def probe_mma_fp4(iters, stream=0):
+    """Enqueue the FP4 (kind::mxf4) tensor-core peak probe; returns the number of CTAs launched."""
+    ctas = ctypes.c_int(0)
+    _check(load_library().quest_probe_mma_fp4(iters, ctypes.byref(ctas), stream), "quest_probe_mma_fp4")
     return ctas.value
 
 

@@ -97,8 +97,108 @@ __global__ void __launch_bounds__(kProbeThreads, 1) probe_mma_i8_kernel(int iter
     }
 }
 
+// The same probe for the block-scaled FP4 kind: tcgen05.mma kind::mxf4 (M = 128,
+// N = 256, K = 64) with unit UE8M0 block scales (byte 0x7F) held in TMEM columns
+// 480-511, the scale arrangement of the FP4 linear layer.
+constexpr uint32_t kIdescProbeFp4 = (1u << 7) | (1u << 10) | (uint32_t(256 >> 3) << 17) | (1u << 23) |
+                                    (uint32_t(128 >> 4) << 24);
+
+__global__ void __launch_bounds__(kProbeThreads, 1) probe_mma_fp4_kernel(int iters) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const uint32_t sbase = static_cast<uint32_t>(__cvta_generic_to_shared(smem));
+    for (uint32_t i = threadIdx.x * 16; i < kBar; i += kProbeThreads * 16)
+        *reinterpret_cast<uint4*>(smem + i) = make_uint4(0x22222222u, 0x22222222u, 0x22222222u, 0x22222222u);
+    const uint32_t bar = sbase + kBar;
+    if (threadIdx.x == 0) {
+        asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(bar) : "memory");
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    const int warp = threadIdx.x >> 5;
+    if (warp == 0) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], 512;" ::"r"(sbase + kSlot)
+                     : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    }
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+    __syncthreads();
+    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+    const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(smem + kSlot);
+    {
+        // unit block scales in this warp's lane quarter, columns 480-511
+        const uint32_t v = 0x7F7F7F7Fu, taddr = tmem + (uint32_t(warp * 32) << 16) + 480;
+        asm volatile(
+            "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
+            "{%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,"
+            "%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1};" ::"r"(taddr),
+            "r"(v)
+            : "memory");
+        asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+    }
+    asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+    __syncthreads();
+    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+
+    if (threadIdx.x == 0) {
+        const uint64_t a = probe_desc(sbase + kA), b = probe_desc(sbase + kB);
+        const uint32_t sfa = tmem + 480, sfb = tmem + 496;
+        for (int i = 0; i < iters; ++i) {
+            asm volatile(
+                "{\n\t.reg .pred p;\n\t"
+                "setp.ne.b32 p, %4, 0;\n\t"
+                "tcgen05.mma.cta_group::1.kind::mxf4.block_scale.block32 [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::"r"(
+                    tmem),
+                "l"(a), "l"(b), "r"(kIdescProbeFp4), "r"(i), "r"(sfa), "r"(sfb)
+                : "memory");
+        }
+        asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
+                     : "memory");
+        uint64_t t0, t;
+        asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t0));
+        for (;;) {
+            uint32_t ok;
+            asm volatile(
+                "{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], 0;\n\t"
+                "selp.u32 %0, 1, 0, p;\n\t}"
+                : "=r"(ok)
+                : "r"(bar)
+                : "memory");
+            if (ok) break;
+            asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+            if (t - t0 > 2000000000ull) {
+                atomicExch(&g_probe_status, (int)QUEST_ETIMEOUT);
+                break;
+            }
+        }
+    }
+    asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+    __syncthreads();
+    if (warp == 0) {
+        asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, 512;" ::"r"(tmem) : "memory");
+    }
+}
+
 }  // namespace
 }  // namespace quest
+
+extern "C" quest_status quest_probe_mma_fp4(int iters, int* ctas, void* stream) {
+    using namespace quest;
+    if (iters < 1 || iters > (1 << 24) || ctas == nullptr) return QUEST_EINVAL;
+    static thread_local int attr_dev = -1;
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (attr_dev != dev) {
+        if (cudaFuncSetAttribute(probe_mma_fp4_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 kProbeSmem + 1024) != cudaSuccess)
+            return QUEST_ECUDA;
+        attr_dev = dev;
+    }
+    *ctas = sm_count();
+    probe_mma_fp4_kernel<<<*ctas, kProbeThreads, kProbeSmem + 1024, static_cast<cudaStream_t>(stream)>>>(iters);
+    return cudaGetLastError() == cudaSuccess ? QUEST_OK : QUEST_ECUDA;
+}
 
 extern "C" quest_status quest_probe_mma_i8(int iters, int* ctas, void* stream) {
     using namespace quest;

@@ -3,9 +3,9 @@
  * integer linear layer on B200 (sm_100a).
  *
  * The pages define no such operation: the entry points below exist only so a
- * benchmark can measure the int8 MMA rate of the part it runs on, the
- * denominator of the linear layer's tensor-core fraction besides the nominal
- * dense figure.
+ * benchmark can measure the int8 and FP4 MMA rates of the part it runs on, the
+ * denominators of the linear layers' tensor-core fractions besides the nominal
+ * dense figures.
  */
 #ifndef QUEST_B200_PROBE_H
 #define QUEST_B200_PROBE_H
@@ -25,6 +25,12 @@ extern "C" {
  * Errors: QUEST_EINVAL if iters is outside [1, 2^24] or ctas is NULL;
  * QUEST_ECUDA on a launch error. */
 quest_status quest_probe_mma_i8(int iters, int* ctas, void* stream);
+
+/* The same for the block-scaled FP4 kind of the FP4 linear layer: back-to-back
+ * tcgen05.mma kind::mxf4 (M = 128, N = 256, K = 64, E2M1 operands in shared
+ * memory, unit UE8M0 block scales in TMEM, fp32 accumulator); the caller
+ * computes 2 * 128 * 256 * 64 * iters * ctas / seconds. Errors as above. */
+quest_status quest_probe_mma_fp4(int iters, int* ctas, void* stream);
 
 /* Synchronise `stream`; QUEST_ETIMEOUT if a probe's bounded completion wait
  * (2 s) gave up since the last call (the flag is then cleared). */

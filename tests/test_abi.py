@@ -152,6 +152,10 @@ def test_probe_rejects_invalid_arguments():
     assert lib.quest_probe_mma_i8(0, ctypes.byref(n), None) == 1
     assert lib.quest_probe_mma_i8(1 << 25, ctypes.byref(n), None) == 1
     assert lib.quest_probe_mma_i8(100, None, None) == 1
+    for fn in (lib.quest_probe_mma_fp4,):
+        assert fn(0, ctypes.byref(n), None) == 1
+        assert fn(1 << 25, ctypes.byref(n), None) == 1
+        assert fn(100, None, None) == 1
 
 
 def test_trust_bwd_linear_rejects_invalid_arguments():
