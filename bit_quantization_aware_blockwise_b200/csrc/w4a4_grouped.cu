@@ -45,12 +45,13 @@ namespace {
 //
 // What bounds it (16384 x 5632 x 2048, scratch variants timed on B200): 400 us
 // as built; 393 us with half the MMAs; 330 us with the FP work removed; 254 us
-// with neither MMAs nor FP work. The layer is bound by moving every group's fp32
-// product from TMEM to registers (5.9 GB per launch): with one 16-column load in
-// flight per warp and two warps per scheduler (the accumulator leaves no
-// registers for more) that runs at about 83 B per clock per SM alone and 64 with
-// the MMAs running. A lockstep layout (eight warps on the same group, 64
-// columns each, two 32-column loads per wait) measured the same 403 us.
+// with neither MMAs nor FP work. That last floor is the operand feed: 128-wide
+// pair tiles load 48 KB per 256 x 128 x 128 group, twice the bytes per MMA of
+// the integer layer's 256-wide tiles, and 2.16 GB in 254 us is 8.5 TB/s of TMA
+// loads, near the 11-12 TB/s the other tensor-core layers reach. TMEM reads are
+// not the limit (a probe of back-to-back tcgen05.ld reads 460-935 B per clock
+// per SM; this layer needs about 64). A lockstep layout (eight warps on the same
+// group, 64 columns each, two 32-column loads per wait) measured the same 403 us.
 
 constexpr int kGThreads = 384;               // warpgroup 0: producer, MMA (2 warps idle); 1, 2: the teams
 constexpr int kGTeamThreads = 128;
