@@ -50,7 +50,7 @@ namespace {
 // the integer layer's 256-wide tiles, and 2.16 GB in 254 us is 8.5 TB/s of TMA
 // loads, near the 11-12 TB/s the other tensor-core layers reach. TMEM reads are
 // not the limit (a probe of back-to-back tcgen05.ld reads 460-935 B per clock
-// per SM; this layer needs about 64). A lockstep layout (eight warps on the same
+// per SM; this layer moves about 50). A lockstep layout (eight warps on the same
 // group, 64 columns each, two 32-column loads per wait) measured the same 403 us.
 
 constexpr int kGThreads = 384;               // warpgroup 0: producer, MMA (2 warps idle); 1, 2: the teams
