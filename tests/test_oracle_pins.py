@@ -289,25 +289,111 @@ def test_trust_region_edges(bits, trust):
         inner = (frac >= (1 - trust) / 2) & (frac <= (1 + trust) / 2)
         expect = np.where(np.abs(t) < half, inner, 0).astype(np.uint8)
         # outer region: beyond the clip t lies further from the level than 1/2
-    safe = o["d_mask"] > 1e-9
+    safe = _flip_distance(t, bits, trust) > 1e-9   # closed form, not the oracle's d_mask
     assert np.array_equal(m[safe], expect[safe])
 
 
-def test_exemption_distances_are_honest():
-    # Moving t by less than d_round must not change the code, and by less than
-    # d_mask must not change the mask: checked by re-quantising scaled copies.
-    g = np.random.default_rng(12)
-    x = g.standard_normal((4, 128))
-    base = oracle.quantize(x, bits=3)
-    d = np.repeat(base["scale"], 128, axis=1)
-    t = base["t"]
-    lo, hi = -4, 3
-    for eps_frac in (0.5, 0.99):
-        for sgn in (-1, 1):
-            tt = t + sgn * eps_frac * np.minimum(base["d_round"], 0.25)
-            qq = np.clip(np.floor(tt), lo, hi)
-            assert np.array_equal(qq, base["q"])
-    assert np.all(np.isfinite(d))
+# ---------------------------------------------------------------------------
+# Mask-exemption distance d_mask. The parity checks exempt a mask bit whose t
+# lies within 1e-5 relative of a flip point of the mask, so d_mask must be the
+# true distance: were it 0 everywhere, every mask comparison would be skipped.
+# The flip points come from the rule's closed form (half-interval mask,
+# pith.science review, "What carries the argument"): for T >= 1 only the outer
+# edge |t| = 2^(b-1) + (T-1)/2 flips; for T < 1 each cell k of the clamped grid
+# flips at k + (1-T)/2 and k + (1+T)/2.
+# ---------------------------------------------------------------------------
+
+def _flip_points(bits, trust):
+    half = 1 << (bits - 1)
+    if trust >= 1:
+        e = half + (trust - 1) / 2
+        return np.array([-e, e])
+    k = np.arange(-half, half, dtype=np.float64)
+    return np.sort(np.concatenate([k + (1 - trust) / 2, k + (1 + trust) / 2]))
+
+
+def _flip_distance(t, bits, trust):
+    f = _flip_points(bits, trust)
+    return np.abs(np.asarray(t)[..., None] - f).min(axis=-1)
+
+
+def _mask_rule(t, bits, trust):
+    """The mask as a function of t alone (closed form of m = [|t - (q+1/2)| <= T/2])."""
+    half = 1 << (bits - 1)
+    t = np.asarray(t, dtype=np.float64)
+    if trust >= 1:
+        return (np.abs(t) <= half + (trust - 1) / 2).astype(np.uint8)
+    frac = t - np.floor(t)
+    inner = (frac >= (1 - trust) / 2) & (frac <= (1 + trust) / 2)
+    return np.where((t >= -half) & (t < half), inner, False).astype(np.uint8)
+
+
+_DMASK_CASES = [(4, 1.0), (3, 0.8), (2, 1.3), (1, 1.0), (8, 1.0), (4, 0.5), (3, 2.0), (1, "s*")]
+
+
+def _edge_input(bits, trust, seed, rows=6, cols=512):
+    """x whose transformed groups put many t values within 0.3 of the mask's flip
+    points. Each group's t = y half / (alpha r) is chosen first; r = rms(y) then
+    equals half / alpha exactly when sum(y^2) = 128 (half / alpha)^2, which the
+    last value of the group makes true; x = H y / sqrt(128) (H symmetric)."""
+    g = np.random.default_rng(seed)
+    half = 1 << (bits - 1)
+    a, _, _ = oracle.alpha(bits)
+    budget = 128 * (half / a) ** 2
+    f = _flip_points(bits, trust)
+    H = scipy.linalg.hadamard(128).astype(np.float64) / math.sqrt(128)
+    y = np.empty((rows, cols))
+    for r in range(rows):
+        for b0 in range(0, cols, 128):
+            v = g.standard_normal(128) * 0.2 * (half / a)
+            n_near = int(min(48, 0.5 * budget / (np.max(np.abs(f)) + 0.3) ** 2))
+            pts = g.choice(f, n_near) + g.uniform(-0.3, 0.3, n_near)
+            v[:n_near] = pts
+            rest = budget - np.sum(v[:127] ** 2)
+            assert rest > 0
+            v[127] = math.sqrt(rest)
+            y[r, b0:b0 + 128] = g.permutation(v)
+    return (y.reshape(rows, cols // 128, 128) @ H).reshape(rows, cols)
+
+
+@pytest.mark.parametrize("bits,trust", _DMASK_CASES)
+def test_mask_flip_distance_closed_form(bits, trust):
+    # The oracle searches an element's own cell and both neighbours, which holds
+    # every flip point within distance 1 of t (the clamped edge cells reach to
+    # infinity), so the two agree exactly once capped at 1.
+    if trust == "s*":
+        trust = _golden("outer_trust_scale_1bit")
+    x = _edge_input(bits, trust, 70 + bits)
+    x[1, :128] = 0.0                                    # an all-zero group: no flips
+    o = oracle.quantize(x, bits=bits, had=128, trust=trust)
+    t, d = o["t"], o["d_mask"]
+    zero = np.repeat(o["scale"] == 0, 128, axis=1)
+    assert np.all(np.isinf(d[zero]))
+    ref = _flip_distance(t[~zero], bits, trust)
+    np.testing.assert_allclose(np.minimum(d[~zero], 1.0), np.minimum(ref, 1.0), rtol=0, atol=1e-12)
+    # the data reach the flip points often enough for this to bite
+    assert np.sum(ref < 0.3) > 50
+
+
+@pytest.mark.parametrize("bits,trust", _DMASK_CASES)
+def test_mask_flip_distance_is_tight(bits, trust):
+    # Moving t by less than d_mask leaves the mask as the oracle set it; moving it
+    # by just more than a finite d_mask changes it in one of the two directions.
+    if trust == "s*":
+        trust = _golden("outer_trust_scale_1bit")
+    x = _edge_input(bits, trust, 80 + bits)
+    o = oracle.quantize(x, bits=bits, had=128, trust=trust)
+    t, m, d = o["t"], o["mask"], np.minimum(o["d_mask"], 1.0)
+    assert np.array_equal(_mask_rule(t, bits, trust), m)
+    for s in (-1.0, 1.0):
+        assert np.array_equal(_mask_rule(t + s * 0.999 * d, bits, trust), m)
+    near = o["d_mask"] < 0.5
+    assert near.sum() > 50
+    up = _mask_rule(t + 1.001 * d, bits, trust) != m
+    down = _mask_rule(t - 1.001 * d, bits, trust) != m
+    assert np.all((up | down)[near])
+    # both mask values occur near the flips
+    assert 0 < m[near].mean() < 1
 
 
 def test_mse_of_quantizer_matches_closed_form():

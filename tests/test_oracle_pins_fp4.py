@@ -162,3 +162,66 @@ def test_fp4_boundary_distances():
     d = np.minimum(a, np.abs(a[..., None] - mids).min(axis=-1))
     assert np.allclose(o["d_round"], d, atol=1e-15)
     assert np.allclose(o["d_mask"], np.abs(a - 7.0), atol=1e-15)
+
+
+# Mask-exemption distance on the FP4 grid. The mask m = [|t - Q| <= (T/2) w(t)]
+# (the half-interval rule read on the local interval width) changes value only at
+# |t| = 6 + T beyond the grid and, for T < 1, at v_k + (T/2) w_k and
+# v_(k+1) - (T/2) w_k inside each interval [v_k, v_(k+1)] of width w_k. d_mask must
+# be the distance to the nearest of them, or the parity checks' exemption band
+# would hide mask mismatches.
+
+def _fp4_flip_points(trust):
+    pts = [6.0 + trust]
+    if trust < 1.0:
+        for k in range(7):
+            w = GRID[k + 1] - GRID[k]
+            pts += [GRID[k] + 0.5 * trust * w, GRID[k + 1] - 0.5 * trust * w]
+    return np.array(pts)
+
+
+def _fp4_edge_input(trust, seed, rows=6, cols=512):
+    """x whose groups put many |t| within 0.3 of the flip points: with t = y / (s* r)
+    and r = rms(y), t = y exactly when sum(y^2) = 128 / s*^2 (the last value of each
+    group makes it so); x = H y / sqrt(128)."""
+    g = np.random.default_rng(seed)
+    s, _ = oracle.alpha_fp4()
+    budget = 128 / s ** 2
+    f = _fp4_flip_points(trust)
+    H = linalg.hadamard(128).astype(np.float64) / math.sqrt(128)
+    y = np.empty((rows, cols))
+    for r in range(rows):
+        for b0 in range(0, cols, 128):
+            v = g.standard_normal(128) * 0.3
+            n_near = int(min(48, 0.5 * budget / (np.max(f) + 0.3) ** 2))
+            v[:n_near] = (g.choice(f, n_near) + g.uniform(-0.3, 0.3, n_near)) * np.sign(g.standard_normal(n_near))
+            rest = budget - np.sum(v[:127] ** 2)
+            assert rest > 0
+            v[127] = math.sqrt(rest)
+            y[r, b0:b0 + 128] = g.permutation(v)
+    return (y.reshape(rows, cols // 128, 128) @ H).reshape(rows, cols)
+
+
+def _fp4_mask_rule(t, trust):
+    a = np.abs(t)
+    q = GRID[np.abs(a[..., None] - GRID).argmin(axis=-1)]   # nearest magnitude (no ties here)
+    w = np.where(a < 2, 0.5, np.where(a < 4, 1.0, 2.0))
+    return (np.abs(a - q) <= 0.5 * trust * w).astype(np.uint8)
+
+
+@pytest.mark.parametrize("trust", [0.5, 0.8, 1.0, 1.3, 2.0])
+def test_fp4_mask_flip_distance(trust):
+    x = _fp4_edge_input(trust, 90 + int(10 * trust))
+    o = oracle.quantize_fp4(x, had=128, trust=trust)
+    a, d = np.abs(o["t"]), o["d_mask"]
+    ref = np.abs(a[..., None] - _fp4_flip_points(trust)).min(axis=-1)
+    np.testing.assert_allclose(d, ref, rtol=0, atol=1e-12)
+    assert np.sum(ref < 0.3) > 50
+    # the distance is tight: less than d keeps the mask, just more flips it one way
+    m = o["mask"]
+    assert np.array_equal(_fp4_mask_rule(o["t"], trust), m)
+    for sg in (-1.0, 1.0):
+        assert np.array_equal(_fp4_mask_rule(o["t"] + sg * 0.999 * d, trust), m)
+    near = d < 0.2
+    flips = (_fp4_mask_rule(o["t"] + 1.001 * d, trust) != m) | (_fp4_mask_rule(o["t"] - 1.001 * d, trust) != m)
+    assert np.all(flips[near])

@@ -15,7 +15,8 @@ import torch
 import oracle
 import bit_quantization_aware_blockwise_b200 as q
 from bit_quantization_aware_blockwise_b200 import inputs
-from parity import check_bf16, check_f32, check_mask, exempt_codes, unpack_mask_bits
+from parity import (MASK_EXEMPT_FRAC, MASK_EXEMPT_FRAC_TRUST_BELOW_1, check_bf16, check_f32, check_mask,
+                    exempt_codes, unpack_mask_bits)
 
 pytestmark = pytest.mark.gpu
 
@@ -61,7 +62,7 @@ def neighbours(v, w):
     return np.abs(iv - iw) <= 1
 
 
-def check_fp4(res, o):
+def check_fp4(res, o, trust=1.0):
     ex = exempt_codes(o)
     if "code" in res:
         bad = (res["code"] != o["code"]) & ~ex
@@ -71,7 +72,7 @@ def check_fp4(res, o):
     assert np.all(neighbours(res["value"][ex], o["value"][ex]))
     check_f32(res["scales"], o["scale"], SCALE_REL, what="scales")
     if "mask" in res:
-        check_mask(res["mask"], o)
+        check_mask(res["mask"], o, MASK_EXEMPT_FRAC if trust >= 1 else MASK_EXEMPT_FRAC_TRUST_BELOW_1)
     diff = res["value"] != o["value"]
     if "deq_bits" in res:
         check_bf16(res["deq_bits"], o["yhat"], skip=diff, what="dequant bf16")
@@ -106,7 +107,7 @@ def test_fp4_trust_forms_byte_mask_fp32_dequant(cuda_device, trust, code_mode):
     x = inputs.activations(21, 1024, seed=int(trust * 10), dtype="bf16")
     o = oracle.quantize_fp4(inputs.to_f64(x), had=64, trust=trust)
     res = run_gpu(x, had=64, trust=trust, code_mode=code_mode, mask_mode=q.MASK_BYTES, dequant="fp32")
-    check_fp4(res, o)
+    check_fp4(res, o, trust)
     assert 0 < res["mask"].mean() <= 1
 
 

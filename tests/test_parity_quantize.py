@@ -12,8 +12,8 @@ import torch
 import oracle
 import bit_quantization_aware_blockwise_b200 as q
 from bit_quantization_aware_blockwise_b200 import inputs
-from parity import (check_bf16, check_codes, check_codes_operand, check_f32, check_mask,
-                    unpack_codes, unpack_mask_bits)
+from parity import (MASK_EXEMPT_FRAC, MASK_EXEMPT_FRAC_TRUST_BELOW_1, check_bf16, check_codes,
+                    check_codes_operand, check_f32, check_mask, unpack_codes, unpack_mask_bits)
 
 pytestmark = pytest.mark.gpu
 
@@ -46,7 +46,7 @@ def run_gpu(x_cpu, bits, had=128, rms_group=None, trust=1.0, code_mode=q.CODES_P
     return res
 
 
-def check_all(res, o, bits, code_mode=q.CODES_PACKED, rms_group=None):
+def check_all(res, o, bits, code_mode=q.CODES_PACKED, rms_group=None, trust=1.0):
     if code_mode == q.CODES_GEMM_OPERAND:
         n_ex = check_codes_operand(res["codes"], o)
         exq = (res["codes"] - 1) // 2 != o["q"]
@@ -55,7 +55,7 @@ def check_all(res, o, bits, code_mode=q.CODES_PACKED, rms_group=None):
         exq = res["codes"] != o["q"]
     check_f32(res["scales"], o["scale"], SCALE_REL, what="scales")
     if "mask" in res:
-        check_mask(res["mask"], o)
+        check_mask(res["mask"], o, MASK_EXEMPT_FRAC if trust >= 1 else MASK_EXEMPT_FRAC_TRUST_BELOW_1)
     if "deq_bits" in res:
         check_bf16(res["deq_bits"], o["yhat"], skip=exq, what="dequant bf16")
     if "deq" in res:
@@ -129,7 +129,7 @@ def test_row_rms_other_blocks(cuda_device, had, cols):
 def test_trust_factors(cuda_device, bits, trust):
     x = inputs.activations(64, 1024, seed=11)
     o = oracle.quantize(inputs.to_f64(x), bits=bits, had=128, trust=trust)
-    check_all(run_gpu(x, bits, trust=trust), o, bits)
+    check_all(run_gpu(x, bits, trust=trust), o, bits, trust=trust)
 
 
 def test_zero_groups_and_rows(cuda_device):
@@ -138,9 +138,9 @@ def test_zero_groups_and_rows(cuda_device):
     x[3, 128:256] = 0
     for trust in (1.0, 0.5):
         o = oracle.quantize(inputs.to_f64(x), bits=4, had=128, trust=trust)
-        check_all(run_gpu(x, 4, trust=trust), o, 4)
+        check_all(run_gpu(x, 4, trust=trust), o, 4, trust=trust)
         o = oracle.quantize(inputs.to_f64(x), bits=4, had=128, rms_group=512, trust=trust)
-        check_all(run_gpu(x, 4, rms_group=512, trust=trust), o, 4)
+        check_all(run_gpu(x, 4, rms_group=512, trust=trust), o, 4, trust=trust)
 
 
 def test_empty_input(cuda_device):
