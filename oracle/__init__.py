@@ -80,6 +80,13 @@ def _load():
         lib.oracle_quantize_fp4.argtypes = [_p, _i64, _i64, _i64, _int, _i64, _dbl, _dbl,
                                             _p, _p, _p, _p, _p, _p, _p, _p, _p]
         lib.oracle_quantize_fp4.restype = _int
+        lib.oracle_sparse24_mse.argtypes = [_int, _dbl]
+        lib.oracle_sparse24_mse.restype = _dbl
+        lib.oracle_sparse24_alpha.argtypes = [_int, _p, _p, _p]
+        lib.oracle_sparse24_alpha.restype = _int
+        lib.oracle_quantize_sparse24.argtypes = [_p, _i64, _i64, _i64, _int, _i64, _int, _dbl, _dbl,
+                                                 _p, _p, _p, _p, _p, _p, _p, _p, _p, _p]
+        lib.oracle_quantize_sparse24.restype = _int
         lib.oracle_trust_bwd.argtypes = [_p, _p, _i64, _i64, _int, _p]
         lib.oracle_trust_bwd.restype = _int
         lib.oracle_gemm_i8.argtypes = [_p, _p, _i64, _i64, _i64, _p]
@@ -192,6 +199,50 @@ def quantize_fp4(x, had: int = 128, rms_group: int | None = None, trust: float =
         _ptr(out["y"]), _ptr(out["t"]), _ptr(out["code"]), _ptr(out["value"]), _ptr(out["yhat"]),
         _ptr(out["mask"]), _ptr(out["scale"]), _ptr(out["d_round"]), _ptr(out["d_mask"]))
     _check(rc, "quantize_fp4")
+    return out
+
+
+def sparse24_mse(bits: int, delta: float) -> float:
+    """E[(X - Q(X))^2 | X kept] for the 2:4-sparse format: of four iid N(0,1) values the
+    two of largest magnitude are kept; Q the 2^bits-level midrise grid of step delta."""
+    return float(_load().oracle_sparse24_mse(bits, delta))
+
+
+_sparse_alpha_cache = {}
+
+
+def alpha_sparse24(bits: int):
+    """(alpha_b, optimal step, minimal MSE of the kept values) of the 2:4-sparse format."""
+    if bits not in _sparse_alpha_cache:
+        a, d, m = _dbl(), _dbl(), _dbl()
+        _check(_load().oracle_sparse24_alpha(bits, ctypes.byref(a), ctypes.byref(d), ctypes.byref(m)),
+               "sparse24_alpha")
+        _sparse_alpha_cache[bits] = (a.value, d.value, m.value)
+    return _sparse_alpha_cache[bits]
+
+
+def quantize_sparse24(x, bits: int, had: int = 128, rms_group: int | None = None, trust: float = 1.0):
+    """2:4-sparse quantizer of the rows of ``x`` (see ``quest_oracle.c``). Returns a dict of
+    numpy arrays: y, t, q (0 where pruned), kept (1 = survives), yhat, mask, scale, d_round,
+    d_mask, d_prune."""
+    x = np.ascontiguousarray(np.asarray(x, dtype=np.float64))
+    if x.ndim != 2:
+        raise ValueError("x must be 2-D")
+    rows, cols = x.shape
+    rms_group = had if rms_group is None else int(rms_group)
+    a, _, _ = alpha_sparse24(bits)
+    out = {
+        "y": np.empty((rows, cols)), "t": np.empty((rows, cols)),
+        "q": np.empty((rows, cols), dtype=np.int32), "kept": np.empty((rows, cols), dtype=np.uint8),
+        "yhat": np.empty((rows, cols)), "mask": np.empty((rows, cols), dtype=np.uint8),
+        "scale": np.empty((rows, cols // rms_group if rms_group else 0)),
+        "d_round": np.empty((rows, cols)), "d_mask": np.empty((rows, cols)), "d_prune": np.empty((rows, cols)),
+    }
+    rc = _load().oracle_quantize_sparse24(
+        _ptr(x), rows, cols, cols, had, rms_group, bits, float(trust), a,
+        _ptr(out["y"]), _ptr(out["t"]), _ptr(out["q"]), _ptr(out["kept"]), _ptr(out["yhat"]),
+        _ptr(out["mask"]), _ptr(out["scale"]), _ptr(out["d_round"]), _ptr(out["d_mask"]), _ptr(out["d_prune"]))
+    _check(rc, "quantize_sparse24")
     return out
 
 

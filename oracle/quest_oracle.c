@@ -260,6 +260,191 @@ int oracle_quantize(const double* x, int64_t rows, int64_t cols, int64_t ld, int
 }
 
 /* ------------------------------------------------------------------------- */
+/* 2:4-sparse INT4 variant.                                                   */
+/*                                                                           */
+/* The pages evaluate QuEST on 2:4-sparse INT4 (atlas.scime.ai summary,        */
+/* ablation table: adding 2:4 sparsity to QuEST INT4 hurts accuracy;           */
+/* pith.science review, results list and Figure 4a: INT, FP and INT+sparse     */
+/* formats at 4 bits) without spelling the format out. Reading: the same       */
+/* Hadamard transform and RMS (over every value of the rms group); then, in    */
+/* each run of four consecutive transformed values along the row, the two of   */
+/* largest magnitude are kept (on equal magnitudes the lower index wins) and   */
+/* the other two become zero; kept values go onto the b-bit midrise grid whose */
+/* step minimises the MSE of the KEPT values when the input is N(0,1) (the     */
+/* Gaussian fit of this format); the trust mask applies the half-interval rule */
+/* to each value's total error, so a pruned value (rebuilt as 0) keeps its     */
+/* gradient iff |t| <= T/2.                                                   */
+/* ------------------------------------------------------------------------- */
+
+/* Density of the magnitude a of a kept value: four iid N(0,1) values, the two
+ * largest magnitudes kept. With F(a) = erf(a / sqrt 2) the half-normal CDF and
+ * f(a) = 2 phi(a) its density, the k-th smallest of four magnitudes has density
+ * 4!/((k-1)!(4-k)!) F^(k-1) (1-F)^(4-k) f; a kept value is the 3rd or the 4th
+ * with probability 1/2 each: (12 F^2 (1-F) + 4 F^3) f / 2 = (6 F^2 - 4 F^3) f. */
+static double kept_density(double a) {
+    double F = erf(a / sqrt(2.0));
+    return (6.0 * F * F - 4.0 * F * F * F) * 2.0 * phi(a);
+}
+
+/* Integral over [a, b] of (x - c)^2 kept_density(x) dx, composite Simpson. */
+static double kept_cell_sq_error(double a, double b, double c) {
+    const int n = 2000;                       /* even */
+    const double h = (b - a) / n;
+    double acc = 0.0;
+    for (int i = 0; i <= n; ++i) {
+        double x = a + i * h;
+        double w = (i == 0 || i == n) ? 1.0 : ((i & 1) ? 4.0 : 2.0);
+        acc += w * (x - c) * (x - c) * kept_density(x);
+    }
+    return acc * h / 3.0;
+}
+
+/* E[(X - Q(X))^2 | X kept], Q the 2^bits-level midrise quantizer of step delta
+ * (levels (i + 1/2) delta, thresholds at multiples of delta, outer cells open).
+ * The grid and the kept-value law are both symmetric, so the integral runs over
+ * magnitudes; the open outer cell is cut 40 beyond its start (the density there
+ * is below 1e-300). */
+double oracle_sparse24_mse(int bits, double delta) {
+    if (bits < 1 || bits > 8 || !(delta > 0.0)) return NAN;
+    const int half = 1 << (bits - 1);
+    double total = 0.0;
+    for (int i = 0; i < half; ++i) {
+        double a = i * delta;
+        double b = (i == half - 1) ? a + 40.0 : (i + 1) * delta;
+        total += kept_cell_sq_error(a, b, (i + 0.5) * delta);
+    }
+    return total;
+}
+
+/* alpha_b of the 2:4-sparse format: 2^(b-1) times the step minimising
+ * oracle_sparse24_mse (golden section). */
+int oracle_sparse24_alpha(int bits, double* alpha, double* delta_opt, double* mse_opt) {
+    if (bits < 1 || bits > 8) return ORACLE_EINVAL;
+    const double g = (sqrt(5.0) - 1.0) / 2.0;
+    double a = 1e-3, b = 6.0;
+    double c = b - g * (b - a), d = a + g * (b - a);
+    double fc = oracle_sparse24_mse(bits, c), fd = oracle_sparse24_mse(bits, d);
+    while (b - a > 1e-11) {
+        if (fc < fd) {
+            b = d; d = c; fd = fc;
+            c = b - g * (b - a); fc = oracle_sparse24_mse(bits, c);
+        } else {
+            a = c; c = d; fc = fd;
+            d = a + g * (b - a); fd = oracle_sparse24_mse(bits, d);
+        }
+    }
+    double dopt = 0.5 * (a + b);
+    if (alpha) *alpha = ldexp(dopt, bits - 1);
+    if (delta_opt) *delta_opt = dopt;
+    if (mse_opt) *mse_opt = oracle_sparse24_mse(bits, dopt);
+    return ORACLE_OK;
+}
+
+/*
+ * 2:4-sparse quantizer of x [rows, cols] (row stride ld), cols a multiple of 4.
+ * Outputs as oracle_quantize, plus:
+ *   kept    [rows, cols]  1 where the value survives the pruning  (required)
+ *   q       [rows, cols]  the code of a kept value, 0 for a pruned one (required)
+ *   yhat    [rows, cols]  (q + 1/2) Delta for kept values, 0 for pruned ones
+ *   d_round [rows, cols]  kept: distance of t to the nearest code boundary; pruned: inf
+ *   d_mask  [rows, cols]  distance of t to the nearest flip point of its mask rule
+ *   d_prune [rows, cols]  for every value of a run of four: the gap between the
+ *                         2nd and 3rd largest |t| of the run (where the choice of
+ *                         kept values would change)
+ */
+int oracle_quantize_sparse24(const double* x, int64_t rows, int64_t cols, int64_t ld, int had,
+                             int64_t rms_group, int bits, double trust, double alpha, double* y_out,
+                             double* t_out, int32_t* q, uint8_t* kept, double* yhat, uint8_t* mask,
+                             double* scale, double* d_round, double* d_mask, double* d_prune) {
+    if (rows < 0 || cols <= 0 || ld < cols || !is_pow2(had) || had < 4 || cols % had != 0) return ORACLE_EINVAL;
+    if (rms_group <= 0 || rms_group % had != 0 || cols % rms_group != 0) return ORACLE_EINVAL;
+    if (bits < 1 || bits > 8 || !(trust > 0.0) || !(alpha > 0.0) || q == NULL || kept == NULL)
+        return ORACLE_EINVAL;
+
+    const int lo = -(1 << (bits - 1)), hi = (1 << (bits - 1)) - 1;
+    const double levels_half = ldexp(1.0, bits - 1);
+    double* H = (double*)malloc(sizeof(double) * had * had);
+    double* y = (double*)malloc(sizeof(double) * cols);
+    if (!H || !y) { free(H); free(y); return ORACLE_EINVAL; }
+    oracle_hadamard(had, H);
+
+    for (int64_t r = 0; r < rows; ++r) {
+        const double* xr = x + r * ld;
+        /* Step 1: blockwise Hadamard transform of the row. */
+        for (int64_t b0 = 0; b0 < cols; b0 += had) hadamard_block(H, had, xr + b0, y + b0);
+        for (int64_t g0 = 0; g0 < cols; g0 += rms_group) {
+            /* Step 2: RMS over every transformed value of the group. */
+            double ss = 0.0;
+            for (int64_t j = 0; j < rms_group; ++j) ss += y[g0 + j] * y[g0 + j];
+            double rms = sqrt(ss / (double)rms_group);
+            /* Step 3: the step fitted to the kept values of a Gaussian input. */
+            double delta = alpha * rms / levels_half;
+            if (scale) scale[r * (cols / rms_group) + g0 / rms_group] = delta;
+            for (int64_t j0 = 0; j0 < rms_group; j0 += 4) {
+                /* Step 4: in the run of four, keep the two largest magnitudes. An
+                 * element is kept when fewer than two others beat it (a larger
+                 * magnitude, or an equal one at a lower index). */
+                double mag[4];
+                for (int i = 0; i < 4; ++i) mag[i] = fabs(y[g0 + j0 + i]);
+                int keep[4];
+                for (int i = 0; i < 4; ++i) {
+                    int beaten = 0;
+                    for (int k = 0; k < 4; ++k)
+                        if (k != i && (mag[k] > mag[i] || (mag[k] == mag[i] && k < i))) ++beaten;
+                    keep[i] = beaten < 2;
+                }
+                /* the 2nd and 3rd largest magnitudes, for the exemption distance */
+                double srt[4];
+                for (int i = 0; i < 4; ++i) srt[i] = mag[i];
+                for (int i = 0; i < 4; ++i)
+                    for (int k = i + 1; k < 4; ++k)
+                        if (srt[k] > srt[i]) { double tmp = srt[i]; srt[i] = srt[k]; srt[k] = tmp; }
+                double gap = (delta == 0.0) ? INFINITY : (srt[1] - srt[2]) / delta;
+                /* Step 5: project the kept values onto the grid; step 6: trust mask. */
+                for (int i = 0; i < 4; ++i) {
+                    int64_t idx = r * cols + g0 + j0 + i;
+                    double yv = y[g0 + j0 + i];
+                    double tv = 0.0, dr = INFINITY, dm = INFINITY, yh = 0.0;
+                    int qv = 0;
+                    uint8_t mv = 1;
+                    if (delta != 0.0) {
+                        tv = yv / delta;
+                        if (keep[i]) {
+                            double fl = floor(tv);
+                            if (fl < lo) fl = lo;
+                            if (fl > hi) fl = hi;
+                            qv = (int)fl;
+                            mv = (fabs(tv - (qv + 0.5)) <= 0.5 * trust) ? 1 : 0;
+                            double k = nearbyint(tv);
+                            if (k < lo + 1) k = lo + 1;
+                            if (k > hi) k = hi;
+                            dr = (hi > lo) ? fabs(tv - k) : INFINITY;
+                            dm = mask_flip_distance(tv, qv, lo, hi, trust);
+                            yh = (qv + 0.5) * delta;
+                        } else {
+                            mv = (fabs(tv) <= 0.5 * trust) ? 1 : 0;
+                            dm = fabs(fabs(tv) - 0.5 * trust);
+                        }
+                    }
+                    if (y_out) y_out[idx] = yv;
+                    if (t_out) t_out[idx] = tv;
+                    q[idx] = qv;
+                    kept[idx] = (uint8_t)keep[i];
+                    if (yhat) yhat[idx] = yh;
+                    if (mask) mask[idx] = mv;
+                    if (d_round) d_round[idx] = dr;
+                    if (d_mask) d_mask[idx] = dm;
+                    if (d_prune) d_prune[idx] = gap;
+                }
+            }
+        }
+    }
+    free(H);
+    free(y);
+    return ORACLE_OK;
+}
+
+/* ------------------------------------------------------------------------- */
 /* FP4 (E2M1) grid variant.                                                   */
 /*                                                                           */
 /* The pages evaluate QuEST on an FP4 grid as well as the INT4 one (pith.science */
