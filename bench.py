@@ -61,11 +61,12 @@ def part_bytes():
 
 GEMM_OPS = 2 * R * NW * C
 NOMINAL_HBM_GBS = 8000.0     # nominal B200 HBM3e bandwidth (about 8 TB/s); the roofline peak is the measured copy
+NOMINAL_INT8_TOPS = 4500.0   # nominal B200 dense int8 tensor-core rate (used only when the probe is skipped)
 
 # DRAM traffic per launch of the dominant kernel, from one ncu capture of the full
-# workload (dram__bytes_read.sum + dram__bytes_write.sum, one pass; the summary is in
-# profiles/launches_hot_path_16384x2048.md). Reported only while the kernel's source
-# files are byte-identical to the ones that were captured; otherwise null.
+# workload (dram__bytes_read.sum + dram__bytes_write.sum, one pass). Reported only
+# while the kernel's source files are byte-identical to the ones that were
+# captured; otherwise null.
 NCU_TRAFFIC = {
     "w4a4_linear": {"sources": ["bit_quantization_aware_blockwise_b200/csrc/w4a4_gemm.cu",
                                 "bit_quantization_aware_blockwise_b200/csrc/tc_common.cuh"],
@@ -363,7 +364,14 @@ def run_b200(args, world, rank, local):
     value = aggregate_throughput(step_bytes, world, ms)
 
     hbm = peaks["hbm_gbs"]
-    int8_peak = peaks["bf16_tflops"] * 2.0   # nominal int8 : bf16 dense ratio 4.5 : 2.25
+    derived_int8 = peaks["bf16_tflops"] * 2.0   # nominal int8 : bf16 dense ratio 4.5 : 2.25
+    # the int8 tensor-core peak: the rate of back-to-back kind::i8 MMAs measured on this
+    # part (no memory traffic), else the nominal dense figure
+    probe = None if args.no_probe else mma_probe(dev)
+    if probe is not None:
+        int8_peak, int8_src = probe["tops"], "measured: back-to-back tcgen05 kind::i8 MMAs, one CTA per SM"
+    else:
+        int8_peak, int8_src = NOMINAL_INT8_TOPS, "nominal B200 dense int8 (probe skipped)"
     breakdown = {}
     for n in names:
         m = statistics.median(part_ms[n])
@@ -373,6 +381,7 @@ def run_b200(args, world, rank, local):
         if n == "w4a4_linear":
             d["tops"] = round(GEMM_OPS / (m * 1e-3) / 1e12, 1)
             d["frac_int8_peak"] = round(d["tops"] / int8_peak, 4)
+            d["frac_bf16x2"] = round(d["tops"] / derived_int8, 4)
         breakdown[n] = d
     dominant = max(names, key=lambda n: breakdown[n]["ms"])
     avg = {n: sum(part_ms[n]) / len(part_ms[n]) for n in names}
@@ -381,7 +390,9 @@ def run_b200(args, world, rank, local):
         roofline = {"kernel": "w4a4_gemm_pair_kernel", "bound": "tensor", "achieved": round(achieved, 1),
                     "peak": round(int8_peak, 1), "unit": "TOPS",
                     "frac": round(achieved / int8_peak, 4),
-                    "peak_source": f"{peaks['source']} bf16 burst x 2 (nominal int8/bf16 dense ratio)",
+                    "peak_source": int8_src,
+                    "frac_of_bf16x2": round(achieved / derived_int8, 4),
+                    "bf16x2_source": f"{peaks['source']} bf16 burst x 2 (nominal int8/bf16 dense ratio)",
                     "traffic": ncu_traffic(dominant), "traffic_unit": "bytes per launch (ncu DRAM read+write)"}
     else:
         achieved = pbytes[dominant] / (avg[dominant] * 1e-3) / 1e9
@@ -395,7 +406,8 @@ def run_b200(args, world, rank, local):
     if not args.no_e2e:
         e2e = run_e2e(args, dev, step, parts, x_cpu, g_cpu, w_cpu, flush, world)
 
-    probe = None if args.no_probe else mma_probe(dev, breakdown["w4a4_linear"]["tops"])
+    if probe is not None:
+        probe["gemm_frac_of_probe"] = round(breakdown["w4a4_linear"]["tops"] / probe["tops"], 4)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -428,7 +440,7 @@ def run_b200(args, world, rank, local):
         print(json.dumps(result), flush=True)
 
 
-def mma_probe(dev, gemm_tops, iters=20000, reps=5, fp4=False):
+def mma_probe(dev, gemm_tops=None, iters=20000, reps=5, fp4=False):
     """Tensor-core rate with no memory traffic (back-to-back tcgen05.mma, one CTA per
     SM): kind::i8 M 128 N 256 K 32, or with fp4 kind::mxf4 M 128 N 256 K 64 with unit
     block scales; context for the linear layers' fractions."""
@@ -449,9 +461,11 @@ def mma_probe(dev, gemm_tops, iters=20000, reps=5, fp4=False):
     q.probe_status(stream.cuda_stream)
     ms = statistics.median(ts)
     tops = 2.0 * 128 * 256 * (64 if fp4 else 32) * iters * ctas / (ms * 1e-3) / 1e12
-    return {"tops": round(tops, 1), "iters": iters, "ctas": ctas,
-            "gemm_frac_of_probe": round(gemm_tops / tops, 4),
-            "note": "timed alone right after the bench loop; the roofline peak stays the measured bf16 x 2"}
+    out = {"tops": round(tops, 1), "iters": iters, "ctas": ctas,
+           "note": "timed alone right after the bench loop (burst); the GEMM's roofline peak"}
+    if gemm_tops is not None:
+        out["gemm_frac_of_probe"] = round(gemm_tops / tops, 4)
+    return out
 
 
 def run_e2e(args, dev, step, parts, x_cpu, g_cpu, w_cpu, flush, world):

@@ -47,6 +47,10 @@ from ._binding import (  # noqa: F401
     probe_mma_i8,
     probe_mma_fp4,
     probe_status,
+    debug_inject_fault,
+    FAULT_NONE,
+    FAULT_LAUNCH,
+    FAULT_WAIT_TIMEOUT,
 )
 
 __all__ = [
@@ -57,4 +61,5 @@ __all__ = [
     "trust_bwd_raw", "w4a4_linear_raw", "w4a4_linear_grouped", "w4a4_linear_grouped_raw",
     "trust_bwd_linear", "trust_bwd_linear_raw", "transpose_bf16", "transpose_bf16_raw",
     "linear_bf16", "linear_bf16_raw", "fp4_linear", "fp4_linear_raw", "device_status", "probe_mma_i8", "probe_mma_fp4", "probe_status",
+    "debug_inject_fault", "FAULT_NONE", "FAULT_LAUNCH", "FAULT_WAIT_TIMEOUT",
 ]

@@ -43,13 +43,22 @@ SIGNATURES = {
     "quest_status_string": (ctypes.c_char_p, [_int]),
     "quest_last_error_message": (ctypes.c_char_p, []),
     "quest_version": (_int, []),
+    "quest_debug_inject_fault": (_int, [_int]),
+}
+
+# The benchmark's tensor-core rate probes (include/quest_probe.h), in their own library.
+_PROBE_LIB_NAME = "libquest_probe.so"
+PROBE_SIGNATURES = {
     "quest_probe_mma_i8": (_int, [_int, _p, _p]),
     "quest_probe_mma_fp4": (_int, [_int, _p, _p]),
     "quest_probe_status": (_int, [_p]),
 }
 
+FAULT_NONE, FAULT_LAUNCH, FAULT_WAIT_TIMEOUT = 0, 1, 2   # include/quest_debug.h
+
 _lock = threading.Lock()
 _lib = None
+_probe_lib = None
 
 
 class QuestError(RuntimeError):
@@ -83,6 +92,29 @@ def load_library():
             f.restype = res
             f.argtypes = args
         _lib = lib
+        return lib
+
+
+def load_probe_library():
+    """Load the benchmark's probe library (once). Raises QuestError if it is not built."""
+    global _probe_lib
+    load_library()
+    with _lock:
+        if _probe_lib is not None:
+            return _probe_lib
+        path = os.path.join(os.path.dirname(library_path()), _PROBE_LIB_NAME)
+        if not os.path.exists(path):
+            raise QuestError(f"{path} not found: build it with "
+                             "`python -m bit_quantization_aware_blockwise_b200.build`")
+        try:
+            lib = ctypes.CDLL(path)
+        except OSError as e:
+            raise QuestError(f"cannot load {path}: {e}") from e
+        for name, (res, args) in PROBE_SIGNATURES.items():
+            f = getattr(lib, name)
+            f.restype = res
+            f.argtypes = args
+        _probe_lib = lib
         return lib
 
 
@@ -410,19 +442,29 @@ def w4a4_linear_grouped(a_codes, a_scales, w_codes, w_scales, out=None, y_f32: b
     return (out, y32) if y_f32 else out
 
 
+def _check_probe(status: int, what: str):
+    if status != 0:
+        raise QuestError(f"{what}: {_STATUS.get(status, status)}", status)
+
+
 def probe_mma_i8(iters, stream=0):
     """Enqueue the int8 tensor-core peak probe; returns the number of CTAs launched."""
     ctas = ctypes.c_int(0)
-    _check(load_library().quest_probe_mma_i8(iters, ctypes.byref(ctas), stream), "quest_probe_mma_i8")
+    _check_probe(load_probe_library().quest_probe_mma_i8(iters, ctypes.byref(ctas), stream), "quest_probe_mma_i8")
     return ctas.value
 
 
 def probe_mma_fp4(iters, stream=0):
     """Enqueue the FP4 (kind::mxf4) tensor-core peak probe; returns the number of CTAs launched."""
     ctas = ctypes.c_int(0)
-    _check(load_library().quest_probe_mma_fp4(iters, ctypes.byref(ctas), stream), "quest_probe_mma_fp4")
+    _check_probe(load_probe_library().quest_probe_mma_fp4(iters, ctypes.byref(ctas), stream), "quest_probe_mma_fp4")
     return ctas.value
 
 
 def probe_status(stream=0):
-    _check(load_library().quest_probe_status(stream), "quest_probe_status")
+    _check_probe(load_probe_library().quest_probe_status(stream), "quest_probe_status")
+
+
+def debug_inject_fault(fault):
+    """Arm a fault for the next launching call on this thread (include/quest_debug.h)."""
+    _check(load_library().quest_debug_inject_fault(fault), "quest_debug_inject_fault")

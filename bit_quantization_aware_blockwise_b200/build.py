@@ -1,4 +1,5 @@
-"""Builds the C-ABI library ``libquest_b200.so`` in-tree with nvcc for sm_100a.
+"""Builds the C-ABI library ``libquest_b200.so`` in-tree with nvcc for sm_100a, and
+the benchmark's tensor-core rate probes as a separate ``libquest_probe.so``.
 
 Usage: ``python -m bit_quantization_aware_blockwise_b200.build [--force]``.
 The CUDA runtime is linked statically so the library does not depend on the
@@ -16,8 +17,10 @@ ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(HERE, "libquest_b200.so")
-SOURCES = ["quest_api.cu", "quantize_fwd.cu", "quantize_hs.cu", "quantize_tc.cu", "trust_bwd.cu", "trust_tc.cu", "w4a4_gemm.cu", "w4a4_grouped.cu", "trust_linear.cu", "fp4_gemm.cu", "tc_host.cu", "transpose.cu",
-           "probe_mma.cu"]
+PROBE_LIB = os.path.join(HERE, "libquest_probe.so")
+SOURCES = ["quest_api.cu", "quantize_fwd.cu", "quantize_hs.cu", "quantize_tc.cu", "trust_bwd.cu", "trust_tc.cu",
+           "w4a4_gemm.cu", "w4a4_grouped.cu", "trust_linear.cu", "fp4_gemm.cu", "tc_host.cu", "transpose.cu"]
+PROBE_SOURCES = ["bench_probe/probe_mma.cu"]
 HEADERS = ["quest_device.cuh", "quest_internal.h", "quest_emit.cuh", "quest_tc.cuh", "tc_common.cuh"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
@@ -31,15 +34,16 @@ def nvcc() -> str:
 
 def _inputs():
     files = [os.path.join(CSRC, f) for f in SOURCES + HEADERS]
-    files.append(os.path.join(INCLUDE, "quest.h"))
+    files += [os.path.join(CSRC, f) for f in PROBE_SOURCES]
+    files += [os.path.join(INCLUDE, h) for h in ("quest.h", "quest_debug.h", "quest_probe.h")]
     files.append(os.path.abspath(__file__))
     return files
 
 
 def stale() -> bool:
-    if not os.path.exists(LIB):
+    if not os.path.exists(LIB) or not os.path.exists(PROBE_LIB):
         return True
-    t = os.path.getmtime(LIB)
+    t = min(os.path.getmtime(LIB), os.path.getmtime(PROBE_LIB))
     return any(os.path.getmtime(f) > t for f in _inputs())
 
 
@@ -54,8 +58,8 @@ def build(force: bool = False, verbose: bool = False) -> str:
               "-I", INCLUDE, "-I", CSRC, "--expt-relaxed-constexpr"]
     if verbose:
         common += ["-Xptxas", "-v"]
-    for src in SOURCES:
-        obj = os.path.join(out_dir, src + ".o")
+    for src in SOURCES + PROBE_SOURCES:
+        obj = os.path.join(out_dir, os.path.basename(src) + ".o")
         objs.append(obj)
         cmd = common + ["-c", os.path.join(CSRC, src), "-o", obj]
         procs.append((cmd, subprocess.Popen(cmd, stdout=subprocess.PIPE, stderr=subprocess.STDOUT)))
@@ -69,10 +73,11 @@ def build(force: bool = False, verbose: bool = False) -> str:
             sys.stderr.write("nvcc failed: " + " ".join(cmd) + "\n")
     if failed:
         raise RuntimeError("building libquest_b200.so failed")
-    tmp = LIB + f".{os.getpid()}.tmp"
-    link = [nvcc(), *ARCH, "-shared", "-cudart", "static", "-o", tmp, *objs]
-    subprocess.run(link, check=True)
-    os.replace(tmp, LIB)
+    n = len(SOURCES)
+    for lib, lib_objs in ((LIB, objs[:n]), (PROBE_LIB, objs[n:])):
+        tmp = lib + f".{os.getpid()}.tmp"
+        subprocess.run([nvcc(), *ARCH, "-shared", "-cudart", "static", "-o", tmp, *lib_objs], check=True)
+        os.replace(tmp, lib)
     return LIB
 
 

@@ -4,11 +4,14 @@
 // The caller times a launch; 2 * 128 * 256 * 32 * iters * SMs / time is the
 // int8 MMA rate this part sustains at its current clocks, the denominator the
 // GEMM's tensor-core fraction can be read against besides the nominal figure.
+//
+// Built into its own library (libquest_probe.so) for the benchmark: it is a
+// measurement aid, not part of the QuEST path, so the product library does not
+// export it.
 #include <cuda_runtime.h>
 #include <stdint.h>
 
 #include "quest.h"
-#include "quest_internal.h"
 #include "quest_probe.h"
 
 namespace quest {
@@ -16,6 +19,18 @@ namespace quest {
 __device__ int g_probe_status = 0;
 
 namespace {
+
+// At most 2^20 MMAs per CTA: tens of milliseconds at any clock, far inside the
+// kernel's 2 s completion wait, so that wait never gives up (and never frees
+// TMEM) while MMAs are still in flight.
+constexpr int kMaxIters = 1 << 20;
+
+int probe_sm_count() {
+    int dev = 0, n = 0;
+    cudaGetDevice(&dev);
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 1;
+    return n;
+}
 
 constexpr int kProbeThreads = 128;
 constexpr uint32_t kProbeSmem = 120 * 1024;   // more than half an SM: one CTA per SM
@@ -185,7 +200,7 @@ __global__ void __launch_bounds__(kProbeThreads, 1) probe_mma_fp4_kernel(int ite
 
 extern "C" quest_status quest_probe_mma_fp4(int iters, int* ctas, void* stream) {
     using namespace quest;
-    if (iters < 1 || iters > (1 << 24) || ctas == nullptr) return QUEST_EINVAL;
+    if (iters < 1 || iters > kMaxIters || ctas == nullptr) return QUEST_EINVAL;
     static thread_local int attr_dev = -1;
     int dev = 0;
     cudaGetDevice(&dev);
@@ -195,14 +210,14 @@ extern "C" quest_status quest_probe_mma_fp4(int iters, int* ctas, void* stream) 
             return QUEST_ECUDA;
         attr_dev = dev;
     }
-    *ctas = sm_count();
+    *ctas = probe_sm_count();
     probe_mma_fp4_kernel<<<*ctas, kProbeThreads, kProbeSmem + 1024, static_cast<cudaStream_t>(stream)>>>(iters);
     return cudaGetLastError() == cudaSuccess ? QUEST_OK : QUEST_ECUDA;
 }
 
 extern "C" quest_status quest_probe_mma_i8(int iters, int* ctas, void* stream) {
     using namespace quest;
-    if (iters < 1 || iters > (1 << 24) || ctas == nullptr) return QUEST_EINVAL;
+    if (iters < 1 || iters > kMaxIters || ctas == nullptr) return QUEST_EINVAL;
     static thread_local int attr_dev = -1;
     int dev = 0;
     cudaGetDevice(&dev);
@@ -212,7 +227,7 @@ extern "C" quest_status quest_probe_mma_i8(int iters, int* ctas, void* stream) {
             return QUEST_ECUDA;
         attr_dev = dev;
     }
-    *ctas = sm_count();
+    *ctas = probe_sm_count();
     probe_mma_i8_kernel<<<*ctas, kProbeThreads, kProbeSmem + 1024, static_cast<cudaStream_t>(stream)>>>(iters);
     return cudaGetLastError() == cudaSuccess ? QUEST_OK : QUEST_ECUDA;
 }

@@ -12,6 +12,7 @@
 #include <utility>
 
 #include "quest.h"
+#include "quest_debug.h"
 #include "quest_device.cuh"
 #include "quest_internal.h"
 
@@ -27,6 +28,21 @@ quest_status fail(quest_status s, const std::string& msg) {
 
 quest_status cuda_fail(cudaError_t e, const char* where) {
     g_last_error = std::string(where) + ": " + cudaGetErrorString(e);
+    return QUEST_ECUDA;
+}
+
+// Fault armed by quest_debug_inject_fault for this host thread (QUEST_FAULT_NONE
+// normally). take_fault consumes it when it is the one asked for.
+thread_local int g_fault = QUEST_FAULT_NONE;
+
+bool take_fault(quest_fault f) {
+    if (g_fault != (int)f) return false;
+    g_fault = QUEST_FAULT_NONE;
+    return true;
+}
+
+quest_status injected_launch_failure(const char* where) {
+    g_last_error = std::string(where) + " launch: injected launch failure (quest_debug_inject_fault); nothing launched";
     return QUEST_ECUDA;
 }
 
@@ -385,6 +401,7 @@ quest_status quest_quantize_fwd(const void* x, quest_dtype x_dtype, int64_t rows
                                              code_mode, codes, scales, mask_mode, mask, dequant, dequant_dtype,
                                              a, row_mode, cb);
     if (st != QUEST_OK || a.rows == 0) return st;
+    if (take_fault(QUEST_FAULT_LAUNCH)) return injected_launch_failure("quest_quantize_fwd");
     cudaError_t e = launch_quantize(a, x_dtype, had_block, cb, bits, row_mode, static_cast<cudaStream_t>(stream));
     if (e == cudaErrorNotSupported)
         return fail(QUEST_EUNSUPPORTED, "the E4M3 operand form and the FP4 grid need rows of whole 128-value slabs, "
@@ -407,6 +424,7 @@ quest_status quest_quantize_operands(const void* x, int64_t M, const void* w, in
     st = prepare_quantize(w, dtype, N, K, K, bits, had_block, K, 1.0f, code_mode, w_codes, w_scales,
                           QUEST_MASK_BITS, nullptr, nullptr, QUEST_BF16, aw, rw, cb);
     if (st != QUEST_OK) return st;
+    if (take_fault(QUEST_FAULT_LAUNCH)) return injected_launch_failure("quest_quantize_operands");
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     cudaError_t e = cudaSuccess;
     if (ax.rows > 0 && aw.rows > 0 && rx && tc_path_ok(ax, dtype, had_block, cb, true) &&
@@ -457,6 +475,7 @@ quest_status quest_trust_bwd(const void* grad_out, const void* mask, quest_mask_
     a.cols = cols;
     a.out = static_cast<uint16_t*>(grad_in);
     a.inv_sqrt_hb = (float)(1.0 / sqrt((double)had_block));
+    if (take_fault(QUEST_FAULT_LAUNCH)) return injected_launch_failure("quest_trust_bwd");
     cudaError_t e = launch_trust_bwd(a, had_block, static_cast<cudaStream_t>(stream));
     if (e != cudaSuccess) return cuda_fail(e, "quest_trust_bwd launch");
     return QUEST_OK;
@@ -480,8 +499,10 @@ quest_status quest_w4a4_linear(const int8_t* a_codes, const float* a_scales,
         if (!aligned(a_scales, 4) || !aligned(w_scales, 4) || (acc && !aligned(acc, 4)))
             return fail(QUEST_EINVAL, "scales and acc must be 4-byte aligned");
     }
+    if (take_fault(QUEST_FAULT_LAUNCH)) return injected_launch_failure("quest_w4a4_linear");
+    const bool inject_timeout = take_fault(QUEST_FAULT_WAIT_TIMEOUT);
     cudaError_t e = launch_w4a4(a_codes, a_scales, w_codes, w_scales, M, N, K,
-                                static_cast<uint16_t*>(y), acc, static_cast<cudaStream_t>(stream));
+                                static_cast<uint16_t*>(y), acc, static_cast<cudaStream_t>(stream), inject_timeout);
     if (e == cudaErrorInvalidValue) return fail(QUEST_ECUDA, "quest_w4a4_linear: tensor map encoding failed");
     if (e != cudaSuccess) return cuda_fail(e, "quest_w4a4_linear launch");
     return QUEST_OK;
@@ -506,6 +527,7 @@ quest_status quest_fp4_linear(const uint8_t* a_codes, const float* a_scales, con
         if ((a_scales && !aligned(a_scales, 4)) || (w_scales && !aligned(w_scales, 4)) || (acc && !aligned(acc, 4)))
             return fail(QUEST_EINVAL, "scales and acc must be 4-byte aligned");
     }
+    if (take_fault(QUEST_FAULT_LAUNCH)) return injected_launch_failure("quest_fp4_linear");
     cudaError_t e = launch_fp4_linear(a_codes, a_scales, w_codes, w_scales, M, N, K, static_cast<uint16_t*>(y), acc,
                                       static_cast<cudaStream_t>(stream));
     if (e == cudaErrorInvalidValue) return fail(QUEST_ECUDA, "quest_fp4_linear: tensor map encoding failed");
@@ -535,6 +557,7 @@ quest_status quest_w4a4_linear_grouped(const uint8_t* a_codes, const float* a_sc
             (y_f32 && !aligned(y_f32, 4)))
             return fail(QUEST_EINVAL, "scales and y_f32 must be 4-byte aligned");
     }
+    if (take_fault(QUEST_FAULT_LAUNCH)) return injected_launch_failure("quest_w4a4_linear_grouped");
     cudaError_t e = launch_w4a4_grouped(reinterpret_cast<const int8_t*>(a_codes), a_scales,
                                         reinterpret_cast<const int8_t*>(w_codes), w_scales, M, N, K,
                                         static_cast<uint16_t*>(y), y_f32, static_cast<cudaStream_t>(stream));
@@ -568,6 +591,7 @@ quest_status quest_trust_bwd_linear(const void* grad_y, const void* w_hat_t, con
         if (overlaps(grad_y, M * N * 2) || overlaps(w_hat_t, K * N * 2) || overlaps(mask, M * K / 8))
             return fail(QUEST_EINVAL, "grad_x must not overlap grad_y, w_hat_t or mask");
     }
+    if (take_fault(QUEST_FAULT_LAUNCH)) return injected_launch_failure("quest_trust_bwd_linear");
     cudaError_t e = launch_trust_linear(static_cast<const uint16_t*>(grad_y), static_cast<const uint16_t*>(w_hat_t),
                                         static_cast<const uint8_t*>(mask), M, N, K, static_cast<uint16_t*>(grad_x),
                                         static_cast<cudaStream_t>(stream));
@@ -597,6 +621,7 @@ quest_status quest_linear_bf16(const void* x_hat, const void* w_hat, int64_t M, 
         if (overlaps(x_hat, M * K * 2) || overlaps(w_hat, N * K * 2))
             return fail(QUEST_EINVAL, "y must not overlap x_hat or w_hat");
     }
+    if (take_fault(QUEST_FAULT_LAUNCH)) return injected_launch_failure("quest_linear_bf16");
     cudaError_t e = launch_linear_bf16(static_cast<const uint16_t*>(x_hat), static_cast<const uint16_t*>(w_hat), M,
                                        N, K, static_cast<uint16_t*>(y), static_cast<cudaStream_t>(stream));
     if (e == cudaErrorInvalidValue) return fail(QUEST_ECUDA, "quest_linear_bf16: tensor map encoding failed");
@@ -615,9 +640,18 @@ quest_status quest_transpose_bf16(const void* src, int64_t rows, int64_t cols, v
         const int64_t bytes = rows * cols * 2;
         if (a < b + bytes && b < a + bytes) return fail(QUEST_EINVAL, "src and dst must not overlap");
     }
+    if (take_fault(QUEST_FAULT_LAUNCH)) return injected_launch_failure("quest_transpose_bf16");
     cudaError_t e = launch_transpose_bf16(static_cast<const uint16_t*>(src), rows, cols, static_cast<uint16_t*>(dst),
                                           static_cast<cudaStream_t>(stream));
     if (e != cudaSuccess) return cuda_fail(e, "quest_transpose_bf16 launch");
+    return QUEST_OK;
+}
+
+quest_status quest_debug_inject_fault(quest_fault fault) {
+    g_last_error.clear();
+    if (fault != QUEST_FAULT_NONE && fault != QUEST_FAULT_LAUNCH && fault != QUEST_FAULT_WAIT_TIMEOUT)
+        return fail(QUEST_EINVAL, "unknown fault");
+    g_fault = (int)fault;
     return QUEST_OK;
 }
 

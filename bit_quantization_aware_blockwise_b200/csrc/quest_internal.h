@@ -87,9 +87,11 @@ cudaError_t launch_trust_bwd(const TrustArgs& a, int had_block, cudaStream_t str
 // Trust backward with the tensor-core Hadamard factor (trust_tc.cu).
 bool trust_tc_ok(const TrustArgs& a, int had_block);
 cudaError_t launch_trust_tc(const TrustArgs& a, int had_block, cudaStream_t stream);
+// inject_timeout: the launch withholds its operand loads and bounds its waits at
+// 1 ms (quest_debug_inject_fault, QUEST_FAULT_WAIT_TIMEOUT); false on every normal call.
 cudaError_t launch_w4a4(const int8_t* A, const float* sa, const int8_t* B, const float* sb,
                         int64_t M, int64_t N, int64_t K, uint16_t* y, int32_t* acc,
-                        cudaStream_t stream);
+                        cudaStream_t stream, bool inject_timeout = false);
 
 // Read (synchronising `stream`) and clear the device status word of the integer
 // linear layer (w4a4_gemm.cu), the grouped layer (w4a4_grouped.cu), the fused

@@ -39,6 +39,9 @@ __device__ int g_tc_status = 0;
 namespace quest {
 namespace {
 
+// Wait bound of a launch that carries the injected timeout fault.
+constexpr uint64_t kInjectedWaitLimitNs = 1000000ull;   // 1 ms
+
 // Shared-memory layout of the single-CTA kernel.
 constexpr int kStages = 4;
 constexpr uint32_t kStageA = BM * BK, kStageB = BN * BK, kStageBytes = kStageA + kStageB;
@@ -75,6 +78,10 @@ struct GemmParams {
     int32_t* acc;       // optional int32 copy of the accumulator
     int M, N, K;
     int num_m, num_n, num_k;
+    // Injected fault (tests of the timeout path): the producer issues no copies,
+    // so nothing is ever in flight and the pipeline waits run out after limit_ns.
+    int withhold;
+    uint64_t limit_ns;  // bound of each pipeline wait (kWaitLimitNs normally)
 };
 
 __global__ void __launch_bounds__(kThreads, 1)
@@ -133,10 +140,10 @@ w4a4_gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constan
             uint32_t stage = 0, phase = 0;
             uint64_t issued = 0;
             bool ok = true;
-            for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
+            for (int tile = blockIdx.x; tile < num_tiles && ok && !p.withhold; tile += gridDim.x) {
                 const int m0 = (tile % p.num_m) * BM, n0 = (tile / p.num_m) * BN;
                 for (int kb = 0; kb < p.num_k; ++kb) {
-                    if (!mbar_wait(bar_empty + 8 * stage, phase ^ 1, abort_flag)) { ok = false; break; }
+                    if (!mbar_wait(bar_empty + 8 * stage, phase ^ 1, abort_flag, p.limit_ns)) { ok = false; break; }
                     const uint32_t fb = bar_full + 8 * stage;
                     mbar_arrive_expect_tx(fb, kStageBytes);
                     tma_load_2d(sbase + kSmemA + stage * kStageA, &map_a, kb * BK, m0, fb);
@@ -164,11 +171,11 @@ w4a4_gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constan
             int local = 0;
             for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x, ++local) {
                 const uint32_t buf = local & 1, bphase = (local >> 1) & 1;
-                if (!mbar_wait(bar_tempty + 8 * buf, bphase ^ 1, abort_flag)) { ok = false; break; }
+                if (!mbar_wait(bar_tempty + 8 * buf, bphase ^ 1, abort_flag, p.limit_ns)) { ok = false; break; }
                 tc_fence_after();
                 const uint32_t d_tmem = tmem_base + buf * BN;
                 for (int kb = 0; kb < p.num_k; ++kb) {
-                    if (!mbar_wait(bar_full + 8 * stage, phase, abort_flag)) { ok = false; break; }
+                    if (!mbar_wait(bar_full + 8 * stage, phase, abort_flag, p.limit_ns)) { ok = false; break; }
                     tc_fence_after();
                     const uint32_t a_addr = sbase + kSmemA + stage * kStageA;
                     const uint32_t b_addr = sbase + kSmemB + stage * kStageB;
@@ -207,7 +214,7 @@ w4a4_gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constan
             }
             const int m = m0 + row_in_tile;
             const float sa_half = m < p.M ? p.sa[m] * 0.5f : 0.0f;
-            const bool got = mbar_wait(bar_tfull + 8 * buf, bphase, abort_flag);
+            const bool got = mbar_wait(bar_tfull + 8 * buf, bphase, abort_flag, p.limit_ns);
             if (epi_any(!got)) break;  // all 128 threads leave together
             tc_fence_after();
             const uint32_t t_acc = tmem_base + lane_addr + buf * BN;
@@ -541,13 +548,14 @@ cudaError_t launch_pair(const int8_t* A, const float* sa, const int8_t* B, const
 
 cudaError_t launch_w4a4(const int8_t* A, const float* sa, const int8_t* B, const float* sb,
                         int64_t M, int64_t N, int64_t K, uint16_t* y, int32_t* acc,
-                        cudaStream_t stream) {
+                        cudaStream_t stream, bool inject_timeout) {
     if (M == 0 || N == 0) return cudaSuccess;
     if (K == 0) {
         return launch_zero_fill(y, acc, M * N, stream);
     }
-    // more than one 128-row block: CTA pairs (M = 256 tiles); otherwise one CTA per tile
-    if (M > BM) return launch_pair(A, sa, B, sb, M, N, K, y, acc, stream);
+    // more than one 128-row block: CTA pairs (M = 256 tiles); otherwise one CTA per
+    // tile (which also handles any M, and carries the injected timeout)
+    if (M > BM && !inject_timeout) return launch_pair(A, sa, B, sb, M, N, K, y, acc, stream);
     CUtensorMap ma, mb, my;
     if (!make_map_2d(&ma, CU_TENSOR_MAP_DATA_TYPE_UINT8, A, K, M, K, BK, BM, CU_TENSOR_MAP_SWIZZLE_128B) ||
         !make_map_2d(&mb, CU_TENSOR_MAP_DATA_TYPE_UINT8, B, K, N, K, BK, BN, CU_TENSOR_MAP_SWIZZLE_128B) ||
@@ -560,6 +568,8 @@ cudaError_t launch_w4a4(const int8_t* A, const float* sa, const int8_t* B, const
     p.num_m = (int)((M + BM - 1) / BM);
     p.num_n = (int)((N + BN - 1) / BN);
     p.num_k = (int)((K + BK - 1) / BK);
+    p.withhold = inject_timeout ? 1 : 0;
+    p.limit_ns = inject_timeout ? kInjectedWaitLimitNs : kWaitLimitNs;
     static thread_local int attr_dev = -1;
     int dev = 0;
     cudaGetDevice(&dev);

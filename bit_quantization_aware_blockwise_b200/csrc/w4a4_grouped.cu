@@ -323,7 +323,9 @@ w4a4_gemm_grouped_kernel(const __grid_constant__ CUtensorMap map_a, const __grid
                 // the team has G groups in every couple before c
                 const uint32_t ga = uint32_t(G) * uint32_t(c) + uint32_t(g);   // the team's group count
                 const uint32_t slot = 2 * team + (ga & 1);
-                if (!mbar_wait(bar_tfull + 8 * slot, (ga >> 1) & 1, abort_flag)) aborted = true;
+                // the warp decides together: the TMEM loads below are warp-collective
+                if (!__all_sync(0xFFFFFFFFu, mbar_wait(bar_tfull + 8 * slot, (ga >> 1) & 1, abort_flag)))
+                    aborted = true;
                 if (aborted) continue;   // later waits return at once (abort flag); exit at the next check
                 tc_fence_after();
                 const uint32_t t_grp = tmem_base + lane_addr + slot * kGBN;

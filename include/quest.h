@@ -368,13 +368,19 @@ quest_status quest_transpose_bf16(const void* src, int64_t rows, int64_t cols, v
 quest_status quest_device_status(void* stream);
 
 /* alpha_b, the clip edge of the b-bit grid (2^(b-1) times the step that minimises
- * the MSE of the midrise uniform quantizer for X ~ N(0,1)); bits 1..8. Computed on
- * the host at first use. Returns NaN for an invalid bit-width. */
+ * the MSE of the midrise uniform quantizer for X ~ N(0,1)); bits 1..8. Follows
+ * pith.science review, "What carries the argument" (the grid's scale minimises the
+ * L2 error against a standard Gaussian) and "Assumptions & free parameters" (alpha
+ * is fixed from an N(0,1) target, not fitted to data). Computed on the host at
+ * first use. Returns NaN for an invalid bit-width. */
 double quest_alpha(int bits);
 
 /* s*, the scale of the OCP E2M1 (FP4) grid {0, +-0.5, +-1, +-1.5, +-2, +-3, +-4, +-6}
  * that minimises E[(X - s Q(X / s))^2] for X ~ N(0,1), Q round-to-nearest onto the
- * grid (the FP4 code modes use Delta = s* r). Computed on the host at first use. */
+ * grid (the FP4 code modes use Delta = s* r). The same Gaussian-MSE fit as alpha_b
+ * (pith.science review, "What carries the argument"; "Assumptions & free
+ * parameters") applied to the FP4 grid the review's results list and Figure 4a
+ * compare against INT4. Computed on the host at first use. */
 double quest_alpha_fp4(void);
 
 /* Bits of the storage container of a b-bit packed code: 1, 2, 4, 4, 8, 8, 8, 8. 0 if invalid. */

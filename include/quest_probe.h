@@ -1,6 +1,7 @@
 /*
  * quest_probe.h -- measurement aid for the tensor-core roofline of the QuEST
- * integer linear layer on B200 (sm_100a).
+ * integer linear layer on B200 (sm_100a). Exported by the benchmark's own
+ * library, libquest_probe.so, not by the product library libquest_b200.so.
  *
  * The pages define no such operation: the entry points below exist only so a
  * benchmark can measure the int8 and FP4 MMA rates of the part it runs on, the
@@ -22,7 +23,8 @@ extern "C" {
  * traffic. `*ctas` receives the number of CTAs launched (host pointer). The
  * caller times the launch on `stream` (CUDA events) and computes
  * 2 * 128 * 256 * 32 * iters * ctas / seconds.
- * Errors: QUEST_EINVAL if iters is outside [1, 2^24] or ctas is NULL;
+ * Errors: QUEST_EINVAL if iters is outside [1, 2^20] (so a launch stays far
+ * inside the kernel's 2 s completion wait) or ctas is NULL;
  * QUEST_ECUDA on a launch error. */
 quest_status quest_probe_mma_i8(int iters, int* ctas, void* stream);
 

@@ -15,10 +15,13 @@ from bit_quantization_aware_blockwise_b200 import _binding
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
 
-def _declared_functions():
+PROBE_HEADER = "quest_probe.h"   # the benchmark's own library, libquest_probe.so
+
+
+def _declared_functions(probe=False):
     names = set()
     for fn in os.listdir(os.path.join(ROOT, "include")):
-        if fn.endswith(".h"):
+        if fn.endswith(".h") and (fn == PROBE_HEADER) == probe:
             text = open(os.path.join(ROOT, "include", fn)).read()
             text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
             names |= set(re.findall(r"\b(quest_\w+)\s*\(", text))
@@ -29,10 +32,23 @@ def test_library_exports_every_declared_symbol():
     lib = q.load_library()
     declared = _declared_functions()
     assert "quest_quantize_fwd" in declared and "quest_w4a4_linear" in declared
+    assert "quest_debug_inject_fault" in declared
     for name in sorted(declared):
         assert hasattr(lib, name), name
     # and the binding knows the signature of each
     assert declared == set(_binding.SIGNATURES)
+
+
+def test_probe_library_is_separate():
+    declared = _declared_functions(probe=True)
+    assert declared == set(_binding.PROBE_SIGNATURES) and declared
+    probe = _binding.load_probe_library()
+    for name in sorted(declared):
+        assert hasattr(probe, name), name
+    # the product library exports only the method's calls (and the debug hook)
+    lib = q.load_library()
+    for name in sorted(declared):
+        assert not hasattr(lib, name), name
 
 
 def test_version_and_status_strings():
@@ -147,14 +163,11 @@ def test_w4a4_rejects_invalid_arguments():
 
 
 def test_probe_rejects_invalid_arguments():
-    lib = q.load_library()
+    lib = _binding.load_probe_library()
     n = ctypes.c_int(0)
-    assert lib.quest_probe_mma_i8(0, ctypes.byref(n), None) == 1
-    assert lib.quest_probe_mma_i8(1 << 25, ctypes.byref(n), None) == 1
-    assert lib.quest_probe_mma_i8(100, None, None) == 1
-    for fn in (lib.quest_probe_mma_fp4,):
+    for fn in (lib.quest_probe_mma_i8, lib.quest_probe_mma_fp4):
         assert fn(0, ctypes.byref(n), None) == 1
-        assert fn(1 << 25, ctypes.byref(n), None) == 1
+        assert fn((1 << 20) + 1, ctypes.byref(n), None) == 1   # cap: far inside the 2 s wait
         assert fn(100, None, None) == 1
 
 

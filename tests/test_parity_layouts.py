@@ -54,7 +54,7 @@ def test_row_rms_all_slab_counts(cuda_device, dtype, had, spr):
     check_all(res, o, 4, q.CODES_GEMM_OPERAND)
     o = oracle.quantize(inputs.to_f64(x), bits=2, had=had, rms_group=cols, trust=0.7)
     res = run_gpu(x, 2, had=had, rms_group=cols, trust=0.7, mask_mode=q.MASK_BYTES, dequant="fp32")
-    check_all(res, o, 2)
+    check_all(res, o, 2, trust=0.7)
 
 
 @pytest.mark.parametrize("dtype", ["bf16", "fp32"])
