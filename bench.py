@@ -828,6 +828,23 @@ def run_configs(args):
                                  y.data_ptr(), None, s)
     add("FP4 linear 16384x5632x2048 (packed E2M1, block-scaled FP4 tensor cores)", f,
         R * C // 2 + NW * C // 2 + 4 * (R + NW) + 2 * R * NW, unit_ops=GEMM_OPS, fp4=True)
+    # the 2:4-sparse format: W_up quantized with pruning (one RMS per row), the layer
+    # with the sparse weights on the sparse tensor cores against X's operand codes;
+    # TOPS count the logical (dense-equivalent) 2 M N K
+    wsp = {"codes": torch.empty((NW, C // 2), dtype=torch.int8, device=dev),
+           "meta": torch.empty((NW, C // 8), dtype=torch.uint8, device=dev),
+           "scales": torch.empty(NW, dtype=torch.float32, device=dev)}
+    f = lambda: q.quantize_sparse24_raw(w.data_ptr(), NW, C, 4, HB, C, 1.0, wsp["codes"].data_ptr(),
+                                        wsp["meta"].data_ptr(), wsp["scales"].data_ptr(), None, None, s)
+    add("2:4-sparse quantize W_up 5632x2048 b4 (row RMS, survivors + metadata)", f,
+        2 * NW * C + NW * C // 2 + NW * C // 8 + 4 * NW)
+    f()
+    fx(); q.device_status()
+    f = lambda: q.w4a4_linear_sparse24_raw(cx.data_ptr(), sx.data_ptr(), wsp["codes"].data_ptr(),
+                                           wsp["meta"].data_ptr(), wsp["scales"].data_ptr(), R, NW, C,
+                                           y.data_ptr(), None, s)
+    add("2:4-sparse W4A4 linear 16384x5632x2048 (sparse tensor cores, logical ops)", f,
+        R * C + NW * C // 2 + NW * C // 8 + 4 * (R + NW) + 2 * R * NW, unit_ops=GEMM_OPS)
     # the input gradient of the layer with the trust backward fused into the bf16
     # product: w_hat from the weight quantizer's bf16 dequant, laid out [K, N] by the
     # library's transpose, X's trust mask from the trust backward case above
@@ -877,6 +894,9 @@ def run_configs(args):
     gemm_tops = next(r["tops"] for r in rows if r["case"].startswith("W4A4 linear"))
     q.device_status()
     probe = mma_probe(dev, gemm_tops)
+    for r in rows:   # int8 layers against the measured int8 MMA rate too
+        if "tops" in r and "frac_fp4_peak" not in r and "tflops" not in r:
+            r["frac_int8_probe"] = round(r["tops"] / probe["tops"], 4)
     fp4_tops = next(r["tops"] for r in rows if "block-scaled FP4" in r["case"])
     probe4 = mma_probe(dev, fp4_tops, fp4=True)
     probe4["note"] = "timed alone after the configs; the FP4 layer's fraction stays of 4 x the measured bf16 peak"

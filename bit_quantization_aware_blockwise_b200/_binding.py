@@ -44,6 +44,9 @@ SIGNATURES = {
     "quest_last_error_message": (ctypes.c_char_p, []),
     "quest_version": (_int, []),
     "quest_debug_inject_fault": (_int, [_int]),
+    "quest_quantize_sparse24": (_int, [_p, _i64, _i64, _int, _int, _i64, _f32, _p, _p, _p, _p, _p, _p]),
+    "quest_alpha_sparse24": (_f64, [_int]),
+    "quest_w4a4_linear_sparse24": (_int, [_p, _p, _p, _p, _p, _i64, _i64, _i64, _p, _p, _p]),
 }
 
 # The benchmark's tensor-core rate probes (include/quest_probe.h), in their own library.
@@ -265,6 +268,68 @@ def quantize_fwd(x, bits: int, had_block: int = 128, rms_group: int | None = Non
                      deq.data_ptr() if deq is not None else None, deq_dtype,
                      _stream_handle(stream, dev))
     return {"codes": codes, "scales": scales, "mask": mask, "dequant": deq}
+
+
+def quantize_sparse24_raw(x, rows, cols, bits, had_block, rms_group, trust, codes, meta, scales, mask=None,
+                          dequant=None, stream=0):
+    _check(load_library().quest_quantize_sparse24(x, rows, cols, bits, had_block, rms_group, trust, codes, meta,
+                                                  scales, mask, dequant, stream), "quest_quantize_sparse24")
+
+
+def quantize_sparse24(x, bits: int = 4, rms_group: int | None = None, trust: float = 1.0, mask: bool = True,
+                      dequant: bool = False, stream=None) -> dict:
+    """2:4-sparse quantizer of the rows of a dense bf16 CUDA tensor ``x`` (Hadamard block
+    128). Returns ``{"codes": int8 [rows, cols/2], "meta": uint8 [rows, cols/8],
+    "scales": fp32 [rows, cols/rms_group], "mask": uint32 [rows, cols/32] or None,
+    "dequant": bf16 [rows, cols] or None}`` (see include/quest.h)."""
+    torch = _torch()
+    _require_cuda(x, "x")
+    if x.dim() != 2 or x.dtype != torch.bfloat16 or not x.is_contiguous():
+        raise QuestError("x must be a contiguous 2-D bf16 tensor")
+    rows, cols = x.shape
+    rg = 128 if rms_group is None else int(rms_group)
+    dev = x.device
+    codes = torch.empty((rows, cols // 2), dtype=torch.int8, device=dev)
+    meta = torch.empty((rows, cols // 8), dtype=torch.uint8, device=dev)
+    scales = torch.empty((rows, cols // rg if rg else 0), dtype=torch.float32, device=dev)
+    m = torch.empty((rows, cols // 32), dtype=torch.int32, device=dev) if mask else None
+    deq = torch.empty((rows, cols), dtype=torch.bfloat16, device=dev) if dequant else None
+    quantize_sparse24_raw(x.data_ptr(), rows, cols, bits, 128, rg, trust, codes.data_ptr(), meta.data_ptr(),
+                          scales.data_ptr(), m.data_ptr() if m is not None else None,
+                          deq.data_ptr() if deq is not None else None, _stream_handle(stream, dev))
+    return {"codes": codes, "meta": meta, "scales": scales, "mask": m, "dequant": deq}
+
+
+def w4a4_linear_sparse24_raw(x_codes, x_scales, w_codes, w_meta, w_scales, M, N, K, y, acc=None, stream=0):
+    _check(load_library().quest_w4a4_linear_sparse24(x_codes, x_scales, w_codes, w_meta, w_scales, M, N, K, y, acc,
+                                                     stream), "quest_w4a4_linear_sparse24")
+
+
+def w4a4_linear_sparse24(x_codes, x_scales, w_codes, w_meta, w_scales, out=None, acc: bool = False, stream=None):
+    """y [M, N] bf16 = (x_codes @ w^T) * (x_scales/2)[:, None] * (w_scales/2)[None, :] with w the
+    2:4-sparse weight codes given compressed (w_codes [N, K/2], w_meta [N, K/8]). Returns y, or
+    (y, acc int32) with ``acc=True``."""
+    torch = _torch()
+    for t, name in ((x_codes, "x_codes"), (w_codes, "w_codes"), (w_meta, "w_meta"), (x_scales, "x_scales"),
+                    (w_scales, "w_scales")):
+        _require_cuda(t, name)
+        if not t.is_contiguous():
+            raise QuestError(f"{name} must be contiguous")
+    M, K = x_codes.shape
+    N = w_codes.shape[0]
+    if w_codes.shape[1] * 2 != K or w_meta.shape != (N, K // 8):
+        raise QuestError("w_codes must be [N, K/2] and w_meta [N, K/8]")
+    dev = x_codes.device
+    y = out if out is not None else torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+    a = torch.empty((M, N), dtype=torch.int32, device=dev) if acc else None
+    w4a4_linear_sparse24_raw(x_codes.data_ptr(), x_scales.data_ptr(), w_codes.data_ptr(), w_meta.data_ptr(),
+                             w_scales.data_ptr(), M, N, K, y.data_ptr(), a.data_ptr() if a is not None else None,
+                             _stream_handle(stream, dev))
+    return (y, a) if acc else y
+
+
+def alpha_sparse24(bits: int) -> float:
+    return float(load_library().quest_alpha_sparse24(bits))
 
 
 def quantize_operands(x, w, bits: int = 4, had_block: int = 128, code_mode: int = CODES_GEMM_OPERAND,

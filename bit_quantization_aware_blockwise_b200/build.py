@@ -19,7 +19,8 @@ INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(HERE, "libquest_b200.so")
 PROBE_LIB = os.path.join(HERE, "libquest_probe.so")
 SOURCES = ["quest_api.cu", "quantize_fwd.cu", "quantize_hs.cu", "quantize_tc.cu", "trust_bwd.cu", "trust_tc.cu",
-           "w4a4_gemm.cu", "w4a4_grouped.cu", "trust_linear.cu", "fp4_gemm.cu", "tc_host.cu", "transpose.cu"]
+           "w4a4_gemm.cu", "w4a4_grouped.cu", "trust_linear.cu", "fp4_gemm.cu", "tc_host.cu", "transpose.cu",
+           "quantize_sparse.cu", "w4a4_sparse.cu"]
 PROBE_SOURCES = ["bench_probe/probe_mma.cu"]
 HEADERS = ["quest_device.cuh", "quest_internal.h", "quest_emit.cuh", "quest_tc.cuh", "tc_common.cuh"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]

@@ -137,6 +137,89 @@ void init_alpha_fp4() {
     g_alpha_fp4 = 0.5 * (lo + hi);
 }
 
+// alpha_b of the 2:4-sparse format: the step that minimises the MSE of the values
+// that survive 2:4 pruning of an N(0,1) input. A survivor's magnitude has density
+// (6F^2 - 4F^3) f (F the half-normal CDF, f its density; the mean of the 3rd and 4th
+// order statistics of four samples), so a cell [a, b) holds mass G(b) - G(a) with
+// G = 2F^3 - F^4; its first moment has no closed form and is taken by 64-point
+// Gauss-Legendre quadrature (the last cell cut 12 beyond its start, where the
+// density is below 1e-30). As for the dense grid the thresholds sit midway between
+// levels, so the optimum is the root of
+//   g(D) = sum_i (i+1/2) (M1_i - (i+1/2) D M0_i),
+// positive below it; found by bisection.
+constexpr int kGL = 64;
+double g_gl_x[kGL], g_gl_w[kGL];
+std::once_flag g_gl_once;
+
+void init_gauss_legendre() {
+    // nodes: roots of P_n by Newton's method from the Chebyshev guesses; weights
+    // 2 / ((1 - x^2) P_n'(x)^2)
+    for (int i = 0; i < kGL; ++i) {
+        double x = cos(M_PI * (i + 0.75) / (kGL + 0.5)), dp = 1.0;
+        for (int it = 0; it < 100; ++it) {
+            double p0 = 1.0, p1 = x;
+            for (int n = 2; n <= kGL; ++n) {
+                const double pn = ((2.0 * n - 1.0) * x * p1 - (n - 1.0) * p0) / n;
+                p0 = p1;
+                p1 = pn;
+            }
+            dp = kGL * (x * p1 - p0) / (x * x - 1.0);
+            const double dx = p1 / dp;
+            x -= dx;
+            if (fabs(dx) < 1e-16) break;
+        }
+        g_gl_x[i] = x;
+        g_gl_w[i] = 2.0 / ((1.0 - x * x) * dp * dp);
+    }
+}
+
+double halfnormal_cdf(double a) { return erf(a * 0.7071067811865476); }
+double kept_mass_antiderivative(double a) {
+    if (isinf(a)) return 1.0;
+    const double F = halfnormal_cdf(a);
+    return 2.0 * F * F * F - F * F * F * F;
+}
+double kept_first_moment(double a, double b) {
+    const double h = 0.5 * (b - a), m = 0.5 * (a + b);
+    double acc = 0.0;
+    for (int i = 0; i < kGL; ++i) {
+        const double x = m + h * g_gl_x[i], F = halfnormal_cdf(x);
+        acc += g_gl_w[i] * x * (6.0 * F * F - 4.0 * F * F * F) * 2.0 * std_normal_pdf(x);
+    }
+    return acc * h;
+}
+
+double sparse_stationarity_residual(int bits, double d) {
+    const int L = 1 << (bits - 1);
+    double g = 0.0;
+    for (int i = 0; i < L; ++i) {
+        const double a = i * d, b = (i == L - 1) ? a + 12.0 : (i + 1) * d, c = i + 0.5;
+        const double m0 = kept_mass_antiderivative(i == L - 1 ? INFINITY : b) - kept_mass_antiderivative(a);
+        g += c * (kept_first_moment(a, b) - c * d * m0);
+    }
+    return g;
+}
+
+double g_alpha_sparse[9];
+std::once_flag g_alpha_sparse_once;
+
+void init_alpha_sparse() {
+    std::call_once(g_gl_once, init_gauss_legendre);
+    g_alpha_sparse[0] = NAN;
+    for (int b = 1; b <= 8; ++b) {
+        double lo = 1e-3, hi = 6.0;
+        for (int it = 0; it < 200; ++it) {
+            const double mid = 0.5 * (lo + hi);
+            if (mid <= lo || mid >= hi) break;
+            if (sparse_stationarity_residual(b, mid) > 0.0)
+                lo = mid;
+            else
+                hi = mid;
+        }
+        g_alpha_sparse[b] = ldexp(0.5 * (lo + hi), b - 1);
+    }
+}
+
 bool is_fp4_mode(quest_code_mode m) { return m == QUEST_CODES_FP4_PACKED || m == QUEST_CODES_FP4_OPERAND; }
 
 int container_bits_of(int bits) {
@@ -237,7 +320,7 @@ static quest_status prepare_quantize(const void* x, quest_dtype x_dtype, int64_t
                               int bits, int had_block, int64_t rms_group, float trust,
                               quest_code_mode code_mode, void* codes, float* scales,
                               quest_mask_mode mask_mode, void* mask, void* dequant, quest_dtype dequant_dtype,
-                              QuantArgs& a, bool& row_mode, int& cb) {
+                              QuantArgs& a, bool& row_mode, int& cb, double alpha_override = 0.0) {
     a = QuantArgs{};
     if (x_dtype != QUEST_BF16 && x_dtype != QUEST_FP32) return fail(QUEST_EINVAL, "x_dtype must be QUEST_BF16 or QUEST_FP32");
     if (rows < 0) return fail(QUEST_EINVAL, "rows must be >= 0");
@@ -279,7 +362,7 @@ static quest_status prepare_quantize(const void* x, quest_dtype x_dtype, int64_t
     }
     if (rows == 0) return QUEST_OK;
 
-    const double alpha = quest_alpha(bits);
+    const double alpha = alpha_override > 0.0 ? alpha_override : quest_alpha(bits);
     const int lo = -(1 << (bits - 1)), hi = (1 << (bits - 1)) - 1;
     // the FP4 grid: Delta = s* r, mask edge 6 + T for T >= 1 (the last grid
     // interval [4, 6] is 2 wide, so T of its halves reach 6 + T)
@@ -348,6 +431,56 @@ double quest_alpha(int bits) {
     if (bits < 1 || bits > 8) return NAN;
     std::call_once(g_alpha_once, init_alpha);
     return g_alpha[bits];
+}
+
+double quest_alpha_sparse24(int bits) {
+    if (bits < 1 || bits > 8) return NAN;
+    std::call_once(g_alpha_sparse_once, init_alpha_sparse);
+    return g_alpha_sparse[bits];
+}
+
+quest_status quest_quantize_sparse24(const void* x, int64_t rows, int64_t cols, int bits, int had_block,
+                                     int64_t rms_group, float trust, void* codes, void* meta, float* scales,
+                                     void* mask, void* dequant, void* stream) {
+    g_last_error.clear();
+    if (bits < 1 || bits > 7) return fail(QUEST_EINVAL, "bits must be in 1..7 (c = 2q+1 in int8)");
+    if (had_block != 128) {
+        if (!valid_had(had_block)) return fail(QUEST_EINVAL, "had_block must be 16, 32, 64, 128 or 256");
+        return fail(QUEST_EUNSUPPORTED, "quest_quantize_sparse24: had_block must be 128");
+    }
+    if (rows < 0) return fail(QUEST_EINVAL, "rows must be >= 0");
+    if (cols <= 0 || cols % 128 != 0) return fail(QUEST_EINVAL, "cols must be a positive multiple of 128");
+    if (rms_group != 128 && rms_group != cols) return fail(QUEST_EINVAL, "rms_group must equal had_block or cols");
+    const bool row_mode = rms_group != 128;
+    const int64_t spr = cols / 128;
+    if (row_mode && !(spr == 1 || spr == 2 || spr == 4 || spr == 8 || spr == 16))
+        return fail(QUEST_EUNSUPPORTED, "quest_quantize_sparse24: one RMS per row needs cols in 128, 256, 512, 1024, 2048");
+    if (rows > 0) {
+        if (!x || !codes || !meta || !scales) return fail(QUEST_EINVAL, "x, codes, meta and scales must be non-NULL");
+        if (!aligned(x, 16)) return fail(QUEST_EINVAL, "x must be 16-byte aligned");
+        if (!aligned(codes, 8) || !aligned(meta, 4) || !aligned(scales, 4) || (mask && !aligned(mask, 4)))
+            return fail(QUEST_EINVAL, "codes must be 8-byte aligned, meta, scales and mask 4-byte aligned");
+        if (dequant && !aligned(dequant, 16)) return fail(QUEST_EINVAL, "dequant must be 16-byte aligned");
+    }
+    SparseArgs sa;
+    bool rm = false;
+    int cb = 0;
+    const quest_status st = prepare_quantize(x, QUEST_BF16, rows, cols, cols, bits, 128, rms_group, trust,
+                                             QUEST_CODES_GEMM_OPERAND, codes, scales, QUEST_MASK_BITS, mask, dequant,
+                                             QUEST_BF16, sa.q, rm, cb, quest_alpha_sparse24(bits));
+    if (st != QUEST_OK || sa.q.rows == 0) return st;
+    sa.q.codes_row_bytes = cols / 2;
+    sa.meta = static_cast<uint8_t*>(meta);
+    sa.meta_row_bytes = cols / 8;
+    sa.bits = bits;
+    {
+        const double edge = ldexp(1.0, bits - 1) + 0.5 * ((double)trust - 1.0), half_t = 0.5 * (double)trust;
+        sa.prune_ratio = (float)((half_t * half_t) / (edge * edge));
+    }
+    if (take_fault(QUEST_FAULT_LAUNCH)) return injected_launch_failure("quest_quantize_sparse24");
+    cudaError_t e = launch_quantize_sparse24(sa, row_mode, static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "quest_quantize_sparse24 launch");
+    return QUEST_OK;
 }
 
 double quest_alpha_fp4(void) {
@@ -505,6 +638,32 @@ quest_status quest_w4a4_linear(const int8_t* a_codes, const float* a_scales,
                                 static_cast<uint16_t*>(y), acc, static_cast<cudaStream_t>(stream), inject_timeout);
     if (e == cudaErrorInvalidValue) return fail(QUEST_ECUDA, "quest_w4a4_linear: tensor map encoding failed");
     if (e != cudaSuccess) return cuda_fail(e, "quest_w4a4_linear launch");
+    return QUEST_OK;
+}
+
+quest_status quest_w4a4_linear_sparse24(const int8_t* x_codes, const float* x_scales, const int8_t* w_codes,
+                                        const uint8_t* w_meta, const float* w_scales, int64_t M, int64_t N, int64_t K,
+                                        void* y, int32_t* acc, void* stream) {
+    g_last_error.clear();
+    if (M < 0 || N < 0 || K < 0) return fail(QUEST_EINVAL, "M, N and K must be >= 0");
+    if (M >= (int64_t(1) << 31) || N >= (int64_t(1) << 31)) return fail(QUEST_EINVAL, "M and N must be < 2^31");
+    if (K % 128 != 0) return fail(QUEST_EINVAL, "K must be a multiple of 128");
+    if (K >= 131072) return fail(QUEST_EINVAL, "K must be < 131072 (int32 accumulator bound)");
+    if (N % 8 != 0) return fail(QUEST_EINVAL, "N must be a multiple of 8");
+    if (M > 0 && N > 0) {
+        if (!y || !x_scales || !w_scales) return fail(QUEST_EINVAL, "y and the scales must be non-NULL");
+        if (K > 0 && (!x_codes || !w_codes || !w_meta)) return fail(QUEST_EINVAL, "codes and meta must be non-NULL");
+        if (K > 0 && (!aligned(x_codes, 16) || !aligned(w_codes, 16) || !aligned(w_meta, 16)))
+            return fail(QUEST_EINVAL, "codes and meta must be 16-byte aligned");
+        if (!aligned(y, 16)) return fail(QUEST_EINVAL, "y must be 16-byte aligned");
+        if (!aligned(x_scales, 4) || !aligned(w_scales, 4) || (acc && !aligned(acc, 4)))
+            return fail(QUEST_EINVAL, "scales and acc must be 4-byte aligned");
+    }
+    if (take_fault(QUEST_FAULT_LAUNCH)) return injected_launch_failure("quest_w4a4_linear_sparse24");
+    cudaError_t e = launch_w4a4_sparse24(x_codes, x_scales, w_codes, w_meta, w_scales, M, N, K,
+                                         static_cast<uint16_t*>(y), acc, static_cast<cudaStream_t>(stream));
+    if (e == cudaErrorInvalidValue) return fail(QUEST_ECUDA, "quest_w4a4_linear_sparse24: tensor map encoding failed");
+    if (e != cudaSuccess) return cuda_fail(e, "quest_w4a4_linear_sparse24 launch");
     return QUEST_OK;
 }
 
@@ -668,11 +827,14 @@ quest_status quest_device_status(void* stream) {
     if (e != cudaSuccess) return cuda_fail(e, "quest_device_status");
     const int vf4 = read_and_clear_fp4_status(s, &e);
     if (e != cudaSuccess) return cuda_fail(e, "quest_device_status");
+    const int vsp = read_and_clear_sparse_status(s, &e);
+    if (e != cudaSuccess) return cuda_fail(e, "quest_device_status");
     if (vg != 0) return fail((quest_status)vg, "a bounded device-side wait in quest_w4a4_linear gave up");
     if (vgr != 0) return fail((quest_status)vgr, "a bounded device-side wait in quest_w4a4_linear_grouped gave up");
     if (vtl != 0)
         return fail((quest_status)vtl, "a bounded device-side wait in quest_trust_bwd_linear or quest_linear_bf16 gave up");
     if (vf4 != 0) return fail((quest_status)vf4, "a bounded device-side wait in quest_fp4_linear gave up");
+    if (vsp != 0) return fail((quest_status)vsp, "a bounded device-side wait in quest_w4a4_linear_sparse24 gave up");
     return QUEST_OK;
 }
 

@@ -63,6 +63,16 @@ struct QuantArgs {
     int64_t rows2;
 };
 
+// 2:4-sparse quantizer (quantize_sparse.cu): the dense quantizer's arguments with
+// the compressed code rows (cols / 2 bytes), the metadata and the pruned mask rule.
+struct SparseArgs {
+    QuantArgs q;
+    uint8_t* meta;           // [rows, cols / 8]: per run of four a nibble of the two kept indices
+    int64_t meta_row_bytes;
+    float prune_ratio;       // (T/2)^2 / edge^2: a pruned value's threshold on y^2, relative to thr2
+    int bits;
+};
+
 struct TrustArgs {
     const uint16_t* g;       // bf16 [rows, cols]
     const uint8_t* mask;     // bits or bytes
@@ -84,6 +94,7 @@ bool tc_path_ok(const QuantArgs& a, quest_dtype x_dtype, int had_block, int cbit
 cudaError_t launch_quantize_tc(const QuantArgs& a, int had_block, int cbits, int bits, bool row_mode,
                                cudaStream_t stream);
 cudaError_t launch_trust_bwd(const TrustArgs& a, int had_block, cudaStream_t stream);
+cudaError_t launch_quantize_sparse24(const SparseArgs& s, bool row_mode, cudaStream_t stream);
 // Trust backward with the tensor-core Hadamard factor (trust_tc.cu).
 bool trust_tc_ok(const TrustArgs& a, int had_block);
 cudaError_t launch_trust_tc(const TrustArgs& a, int had_block, cudaStream_t stream);
@@ -97,7 +108,11 @@ cudaError_t launch_w4a4(const int8_t* A, const float* sa, const int8_t* B, const
 // linear layer (w4a4_gemm.cu), the grouped layer (w4a4_grouped.cu), the fused
 // input gradient (trust_linear.cu) and the FP4 layer (fp4_gemm.cu); each returns
 // its value (0 or a quest_status).
+cudaError_t launch_w4a4_sparse24(const int8_t* X, const float* sx, const int8_t* W, const uint8_t* E,
+                                 const float* sw, int64_t M, int64_t N, int64_t K, uint16_t* y, int32_t* acc,
+                                 cudaStream_t stream);
 int read_and_clear_gemm_status(cudaStream_t stream, cudaError_t* err);
+int read_and_clear_sparse_status(cudaStream_t stream, cudaError_t* err);
 int read_and_clear_grouped_status(cudaStream_t stream, cudaError_t* err);
 int read_and_clear_trust_linear_status(cudaStream_t stream, cudaError_t* err);
 int read_and_clear_fp4_status(cudaStream_t stream, cudaError_t* err);

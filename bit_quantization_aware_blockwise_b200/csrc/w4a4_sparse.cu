@@ -1,0 +1,349 @@
+// Linear layer on 2:4-sparse QuEST weight codes: tcgen05.mma.sp kind::i8 with
+// the weights as the sparse operand (sm_100a).
+//
+//   acc[m][n] = sum_k X[m][k] * W[n][k]      (W 2:4-sparse along k; int8 -> int32, exact)
+//   y[m][n]   = bf16_rne(acc * (sx[m]/2) * (sw[n]/2))
+//
+// The pages evaluate QuEST with 2:4 sparsity added to INT4 (atlas.scime.ai summary
+// of QuEST, ablation table; pith.science review, Figure 4a). The sparse tensor
+// cores take the sparse operand as A (the M side of the MMA), so the product runs
+// transposed: A = the compressed weight codes (128 weight rows per tile), B = the
+// activation codes (224 tokens per tile), D[n][m] in TMEM, and the epilogue writes
+// y[m][n] through a transposed shared-memory stage.
+//
+// Operands per stage (128 logical K values):
+//   A  compressed weights, 128 rows x 64 bytes (the two survivors of each run of
+//      four), 64-byte swizzle;
+//   B  activation codes, 224 rows x 128 bytes, 128-byte swizzle;
+//   E  metadata, 128 rows x 16 bytes (a nibble per run: the lower survivor's index
+//      in bits 0-1, the higher one's in bits 2-3), no swizzle, copied into TMEM
+//      (tcgen05.cp 128x128b: lane = weight row, four 32-bit columns).
+// Each stage is two sparse MMAs (M = 128, N = 224, K = 64 logical); MMA j reads
+// its metadata from columns 2j, 2j+1 of the stage's slot.
+//
+// Structure (one persistent CTA per SM, 192 threads): warp 0 TMA producer, warp 1
+// TMEM allocator, metadata copies and MMA issuer, warps 2-5 epilogue. Two
+// 224-column accumulators alternate (the epilogue of tile i overlaps the mainloop
+// of tile i + 1); the metadata slots sit after them. No cluster, no multicast.
+// Every wait is bounded in time; on timeout the CTA records QUEST_ETIMEOUT,
+// drains its copies and MMAs, frees TMEM and returns.
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace quest {
+namespace {
+// Device-side status word of this file's kernel (0 = fine); read and cleared by
+// quest_device_status().
+__device__ int g_tc_status = 0;
+}  // namespace
+}  // namespace quest
+
+#include "tc_common.cuh"
+
+namespace quest {
+namespace {
+
+constexpr int SBM = 128;                 // weight rows per tile (MMA M)
+constexpr int SBN = 224;                 // tokens per tile (MMA N)
+constexpr int SBK = 128;                 // logical K per stage
+constexpr int kSStages = 5;
+constexpr uint32_t kSStageA = SBM * SBK / 2;        // 8 KB: compressed weights
+constexpr uint32_t kSStageB = SBN * SBK;            // 28 KB: activation codes
+constexpr uint32_t kSStageE = SBM * SBK / 8;        // 2 KB: metadata
+constexpr uint32_t kSTx = kSStageA + kSStageB + kSStageE;
+constexpr uint32_t kSSmemA = 0;
+constexpr uint32_t kSSmemB = kSSmemA + kSStages * kSStageA;
+constexpr uint32_t kSSmemE = kSSmemB + kSStages * kSStageB;
+constexpr uint32_t kSCBytes = 32 * SBM * 2;         // transposed stage: 32 tokens x 128 weight rows, bf16
+constexpr uint32_t kSSmemC = kSSmemE + kSStages * kSStageE;
+constexpr uint32_t kSSmemScale = kSSmemC + 2 * kSCBytes;   // float[SBN]: the tokens' scales
+constexpr uint32_t kSSmemBar = kSSmemScale + SBN * 4;
+constexpr uint32_t kSNumBars = 2 * kSStages + 4 + 1;
+constexpr uint32_t kSSmemTmemSlot = kSSmemBar + kSNumBars * 8;
+constexpr uint32_t kSSmemAbort = kSSmemTmemSlot + 4;
+constexpr uint32_t kSSmemUsed = kSSmemAbort + 4;
+constexpr uint32_t kSSmemTotal = kSSmemUsed + 1024;
+static_assert(kSSmemTotal <= 227 * 1024, "sparse kernel shared memory");
+static_assert(kSStageA % 1024 == 0 && kSStageB % 1024 == 0 && kSStageE % 1024 == 0, "stage alignment");
+constexpr uint32_t kSAccCols = SBN;                  // accumulator buffers at columns 0 and SBN
+constexpr uint32_t kSMetaCol = 2 * SBN;              // metadata slots: 4 columns per stage
+static_assert(kSMetaCol + 4 * kSStages <= kTmemCols, "TMEM columns");
+
+// tcgen05 kind::i8 with sparse A: D int32, A and B signed int8, K-major,
+// M = 128, N = 224, sparsity flag (bit 2).
+constexpr uint32_t kIdescSp = (1u << 2) | (2u << 4) | (1u << 7) | (1u << 10) | (uint32_t(SBN >> 3) << 17) |
+                              (uint32_t(SBM >> 4) << 24);
+
+__device__ __forceinline__ void tc_mma_sp_i8(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t e_tmem,
+                                             uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %5, 0;\n\t"
+        "tcgen05.mma.sp.cta_group::1.kind::i8 [%0], %1, %2, [%3], %4, p;\n\t}" ::"r"(d_tmem),
+        "l"(adesc), "l"(bdesc), "r"(e_tmem), "r"(kIdescSp), "r"(accumulate)
+        : "memory");
+}
+
+// K-major operand with 64-byte rows and the 64-byte swizzle written by TMA:
+// 8-row core groups 512 bytes apart.
+__device__ __forceinline__ uint64_t smem_desc_k64(uint32_t addr) {
+    uint64_t d = 0;
+    d |= uint64_t((addr >> 4) & 0x3FFFu);   // start address
+    d |= uint64_t(1) << 16;                 // leading byte offset (unused for swizzled K-major)
+    d |= uint64_t(512 >> 4) << 32;          // stride byte offset: 8 rows x 64 B
+    d |= uint64_t(1) << 46;                 // descriptor version (sm_100)
+    d |= uint64_t(4) << 61;                 // layout: 64-byte swizzle
+    return d;
+}
+// The metadata stage: 128 rows of 16 bytes, no swizzle: 8-row core matrices of
+// 128 contiguous bytes, 128 bytes apart.
+__device__ __forceinline__ uint64_t smem_desc_meta(uint32_t addr) {
+    uint64_t d = 0;
+    d |= uint64_t((addr >> 4) & 0x3FFFu);
+    d |= uint64_t(kSStageE >> 4) << 16;     // leading byte offset (a second 16-byte column; unused)
+    d |= uint64_t(128 >> 4) << 32;          // stride byte offset: 8 rows x 16 B
+    d |= uint64_t(1) << 46;
+    return d;                               // layout 0: no swizzle
+}
+__device__ __forceinline__ void tc_cp_meta(uint32_t taddr, uint64_t sdesc) {
+    asm volatile("tcgen05.cp.cta_group::1.128x128b [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
+}
+
+struct SparseParams {
+    const float* sx;    // token scales [M]
+    const float* sw;    // weight row scales [N]
+    int32_t* acc;       // optional int32 copy of the accumulator [M][N]
+    int M, N, K;
+    int num_n, num_m, num_k;   // weight-row tiles (128), token tiles (224), K stages (128)
+};
+
+__global__ void __launch_bounds__(kThreads, 1)
+w4a4_sparse_kernel(const __grid_constant__ CUtensorMap map_w, const __grid_constant__ CUtensorMap map_x,
+                   const __grid_constant__ CUtensorMap map_e, const __grid_constant__ CUtensorMap map_y,
+                   const SparseParams p) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const uint32_t sbase = smem_u32(smem);
+    const uint32_t bar_full = sbase + kSSmemBar;             // [kSStages]
+    const uint32_t bar_empty = bar_full + 8 * kSStages;      // [kSStages]
+    const uint32_t bar_tfull = bar_empty + 8 * kSStages;     // [2]
+    const uint32_t bar_tempty = bar_tfull + 16;              // [2]
+    const uint32_t bar_drain = bar_tempty + 16;              // [1]
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + kSSmemAbort);
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kSSmemTmemSlot);
+    float* s_scale = reinterpret_cast<float*>(smem + kSSmemScale);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int num_tiles = p.num_n * p.num_m;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kSStages; ++s) {
+            mbar_init(bar_full + 8 * s, 1);
+            mbar_init(bar_empty + 8 * s, 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(bar_tfull + 8 * b, 1);
+            mbar_init(bar_tempty + 8 * b, kEpiThreads);
+        }
+        mbar_init(bar_drain, 1);
+        *abort_flag = 0;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&map_w)) : "memory");
+        asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&map_x)) : "memory");
+        asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&map_e)) : "memory");
+        asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&map_y)) : "memory");
+    }
+    if (warp == 1) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                         smem_u32(tmem_slot)),
+                     "r"(kTmemCols)
+                     : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+    pdl_wait();
+    pdl_trigger();
+
+    if (warp == 0) {
+        // ------------------------------------------------------------ TMA producer
+        if (lane == 0) {
+            uint32_t stage = 0, phase = 0;
+            uint64_t issued = 0;
+            bool ok = true;
+            for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
+                const int n0 = (tile % p.num_n) * SBM, m0 = (tile / p.num_n) * SBN;
+                for (int kb = 0; kb < p.num_k; ++kb) {
+                    if (!mbar_wait(bar_empty + 8 * stage, phase ^ 1, abort_flag)) { ok = false; break; }
+                    const uint32_t fb = bar_full + 8 * stage;
+                    mbar_arrive_expect_tx(fb, kSTx);
+                    tma_load_2d(sbase + kSSmemA + stage * kSStageA, &map_w, kb * (SBK / 2), n0, fb);
+                    tma_load_2d(sbase + kSSmemB + stage * kSStageB, &map_x, kb * SBK, m0, fb);
+                    tma_load_2d(sbase + kSSmemE + stage * kSStageE, &map_e, kb * (SBK / 8), n0, fb);
+                    ++issued;
+                    if (++stage == kSStages) { stage = 0; phase ^= 1; }
+                }
+            }
+            if (!ok) {
+                const uint64_t n = issued < kSStages ? issued : kSStages;
+                for (uint64_t i = issued - n; i < issued; ++i) {
+                    const uint32_t st = uint32_t(i % kSStages), ph = uint32_t((i / kSStages) & 1);
+                    const uint64_t t0 = global_timer_ns();
+                    while (!mbar_try_wait(bar_full + 8 * st, ph) && global_timer_ns() - t0 < kWaitLimitNs) {
+                    }
+                }
+            }
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------------------ metadata copies and MMAs
+        if (lane == 0) {
+            uint32_t stage = 0, phase = 0;
+            bool ok = true;
+            int local = 0;
+            for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x, ++local) {
+                const uint32_t buf = local & 1, bphase = (local >> 1) & 1;
+                if (!mbar_wait(bar_tempty + 8 * buf, bphase ^ 1, abort_flag)) { ok = false; break; }
+                tc_fence_after();
+                const uint32_t d_tmem = tmem_base + buf * kSAccCols;
+                for (int kb = 0; kb < p.num_k; ++kb) {
+                    if (!mbar_wait(bar_full + 8 * stage, phase, abort_flag)) { ok = false; break; }
+                    tc_fence_after();
+                    const uint32_t a_addr = sbase + kSSmemA + stage * kSStageA;
+                    const uint32_t b_addr = sbase + kSSmemB + stage * kSStageB;
+                    const uint32_t e_tmem = tmem_base + kSMetaCol + 4 * stage;
+                    // the copy and the MMAs after it run in issue order
+                    tc_cp_meta(e_tmem, smem_desc_meta(sbase + kSSmemE + stage * kSStageE));
+#pragma unroll
+                    for (int kk = 0; kk < SBK / 64; ++kk) {
+                        tc_mma_sp_i8(d_tmem, smem_desc_k64(a_addr + kk * 32), smem_desc_k128(b_addr + kk * 64),
+                                     e_tmem + 2 * kk, (kb | kk) != 0);
+                    }
+                    tc_commit(bar_empty + 8 * stage);   // frees the stage (and its metadata slot)
+                    if (++stage == kSStages) { stage = 0; phase ^= 1; }
+                }
+                if (!ok) break;
+                tc_commit(bar_tfull + 8 * buf);
+            }
+            tc_commit(bar_drain);
+            const uint64_t t0 = global_timer_ns();
+            while (!mbar_try_wait(bar_drain, 0) && global_timer_ns() - t0 < kWaitLimitNs) {
+            }
+        }
+    } else {
+        // ------------------------------------------------------------ epilogue (warps 2..5)
+        const int et = threadIdx.x - 64;              // 0..127
+        const int quarter = warp & 3;                 // TMEM lanes 32*quarter .. +31
+        const int row = quarter * 32 + lane;          // weight row within the tile = TMEM lane
+        const uint32_t lane_addr = uint32_t(quarter * 32) << 16;
+        int local = 0, cbuf = 0;
+        for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++local) {
+            const int n0 = (tile % p.num_n) * SBM, m0 = (tile / p.num_n) * SBN;
+            const uint32_t buf = local & 1, bphase = (local >> 1) & 1;
+            epi_bar();   // everyone is done with the previous tile's token scales
+            for (int c = et; c < SBN; c += kEpiThreads) {
+                const int m = m0 + c;
+                s_scale[c] = m < p.M ? p.sx[m] * 0.5f : 0.0f;
+            }
+            const int n = n0 + row;
+            const float sw_half = n < p.N ? p.sw[n] * 0.5f : 0.0f;
+            const bool got = mbar_wait(bar_tfull + 8 * buf, bphase, abort_flag);
+            if (epi_any(!got)) break;   // also orders the token scales above (bar.red)
+            tc_fence_after();
+            const uint32_t t_acc = tmem_base + lane_addr + buf * kSAccCols;
+#pragma unroll 1
+            for (int c = 0; c < SBN / 32; ++c) {
+                uint32_t r[32];
+                QUEST_TMEM_LD32(t_acc + c * 32, r);
+                tmem_wait_ld();
+                const float* sc = s_scale + c * 32;
+                // transposed stage: token i of the chunk is row i, this weight row its column
+                uint16_t* stg = reinterpret_cast<uint16_t*>(smem + kSSmemC + cbuf * kSCBytes) + row;
+#pragma unroll
+                for (int i = 0; i < 32; ++i) {
+                    const float y = (float)(int32_t)r[i] * sw_half * sc[i];
+                    stg[i * SBM] = __bfloat16_as_ushort(__float2bfloat16_rn(y));
+                }
+                if (p.acc != nullptr && n < p.N) {
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) {
+                        const int m = m0 + c * 32 + i;
+                        if (m < p.M) p.acc[int64_t(m) * p.N + n] = (int32_t)r[i];
+                    }
+                }
+                fence_proxy_async_smem();
+                epi_bar();
+                if (et == 0) {
+                    tma_store_2d(&map_y, sbase + kSSmemC + cbuf * kSCBytes, n0, m0 + c * 32);
+                    bulk_commit();
+                    bulk_wait_read_le1();   // the other staging buffer is free again
+                }
+                epi_bar();
+                cbuf ^= 1;
+            }
+            tc_fence_before();
+            mbar_arrive(bar_tempty + 8 * buf);
+        }
+        if (et == 0) bulk_wait_all();
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base), "r"(kTmemCols)
+                     : "memory");
+    }
+}
+
+}  // namespace
+
+cudaError_t launch_w4a4_sparse24(const int8_t* X, const float* sx, const int8_t* W, const uint8_t* E,
+                                 const float* sw, int64_t M, int64_t N, int64_t K, uint16_t* y, int32_t* acc,
+                                 cudaStream_t stream) {
+    if (M == 0 || N == 0) return cudaSuccess;
+    if (K == 0) return launch_zero_fill(y, acc, M * N, stream);
+    CUtensorMap mw, mx, me, my;
+    if (!make_map_2d(&mw, CU_TENSOR_MAP_DATA_TYPE_UINT8, W, K / 2, N, K / 2, SBK / 2, SBM,
+                     CU_TENSOR_MAP_SWIZZLE_64B) ||
+        !make_map_2d(&mx, CU_TENSOR_MAP_DATA_TYPE_UINT8, X, K, M, K, SBK, SBN, CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !make_map_2d(&me, CU_TENSOR_MAP_DATA_TYPE_UINT8, E, K / 8, N, K / 8, SBK / 8, SBM,
+                     CU_TENSOR_MAP_SWIZZLE_NONE) ||
+        !make_map_2d(&my, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, y, N, M, N * 2, SBM, 32, CU_TENSOR_MAP_SWIZZLE_NONE))
+        return cudaErrorInvalidValue;
+    SparseParams p;
+    p.sx = sx; p.sw = sw; p.acc = acc;
+    p.M = (int)M; p.N = (int)N; p.K = (int)K;
+    p.num_n = (int)((N + SBM - 1) / SBM);
+    p.num_m = (int)((M + SBN - 1) / SBN);
+    p.num_k = (int)((K + SBK - 1) / SBK);
+    static thread_local int attr_dev = -1;
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (attr_dev != dev) {
+        cudaError_t e = cudaFuncSetAttribute(w4a4_sparse_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             kSSmemTotal);
+        if (e != cudaSuccess) return e;
+        attr_dev = dev;
+    }
+    const int tiles = p.num_n * p.num_m;
+    const int sms = sm_count();
+    const int grid = tiles < sms ? tiles : sms;
+    return launch_pdl(w4a4_sparse_kernel, dim3(grid), dim3(kThreads), kSSmemTotal, stream, mw, mx, me, my, p);
+}
+
+int read_and_clear_sparse_status(cudaStream_t stream, cudaError_t* err) {
+    int v = 0, zero = 0;
+    cudaError_t e = cudaMemcpyFromSymbolAsync(&v, g_tc_status, sizeof(int), 0, cudaMemcpyDeviceToHost, stream);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(stream);
+    if (e == cudaSuccess && v != 0)
+        e = cudaMemcpyToSymbolAsync(g_tc_status, &zero, sizeof(int), 0, cudaMemcpyHostToDevice, stream);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(stream);
+    *err = e;
+    return v;
+}
+
+}  // namespace quest

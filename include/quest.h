@@ -181,6 +181,44 @@ quest_status quest_quantize_operands(const void* x, int64_t M, const void* w, in
                                      void* stream);
 
 /*
+ * quest_quantize_sparse24 -- the 2:4-sparse INT variant of the QuEST quantizer.
+ *
+ * The pages evaluate QuEST on a 2:4-sparse INT4 format and report that adding 2:4
+ * sparsity to QuEST INT4 costs accuracy (atlas.scime.ai summary, ablation table;
+ * pith.science review, results list and Figure 4a: INT, FP and INT+sparse formats
+ * at 4 bits), without spelling the format out. This library reads it as the
+ * transform and RMS of quest_quantize_fwd (Hadamard block 128, r over every value
+ * of the rms group), then, in every run of four consecutive transformed values:
+ *     keep the two values of largest |y| (on equal magnitudes the lower index wins),
+ *     Delta = quest_alpha_sparse24(bits) * r / 2^(b-1),  t = y / Delta,
+ *     kept:   q = clamp(floor(t), -2^(b-1), 2^(b-1)-1), yhat = (q + 1/2) Delta,
+ *             m = [ |t - (q + 1/2)| <= trust / 2 ]
+ *     pruned: yhat = 0, m = [ |t| <= trust / 2 ]   (the half-interval rule on the
+ *             value's total error)
+ * A group with r == 0 keeps the lower two indices of each run with q = 0, m = 1.
+ *
+ * Arguments
+ *   x          device bf16 [rows, cols], dense (row pitch cols), 16-byte aligned.
+ *   rows >= 0; cols a positive multiple of 128.   bits 1..7.
+ *   had_block  must be 128 (QUEST_EUNSUPPORTED otherwise).
+ *   rms_group  128, or cols (one RMS per row; then cols in 128, 256, 512, 1024, 2048).
+ *   trust      T > 0.
+ *   codes      device int8 [rows, cols / 2], 8-byte aligned: per run of four the two
+ *              kept values' c = 2q + 1 in index order (the compressed operand of
+ *              quest_w4a4_linear_sparse24).
+ *   meta       device uint8 [rows, cols / 8], 4-byte aligned: per run a nibble with
+ *              the lower kept index in bits 0-1 and the higher in bits 2-3; byte j
+ *              holds runs 2j (low nibble) and 2j + 1.
+ *   scales     device fp32 [rows, cols / rms_group], Delta per group.
+ *   mask       device, optional: uint32 mask words [rows, cols / 32] as QUEST_MASK_BITS.
+ *   dequant    device, optional: bf16 [rows, cols] yhat (0 where pruned), 16-byte aligned.
+ * Returns QUEST_OK, QUEST_EINVAL, QUEST_EUNSUPPORTED or QUEST_ECUDA.
+ */
+quest_status quest_quantize_sparse24(const void* x, int64_t rows, int64_t cols, int bits, int had_block,
+                                     int64_t rms_group, float trust, void* codes, void* meta, float* scales,
+                                     void* mask, void* dequant, void* stream);
+
+/*
  * quest_trust_bwd -- trust-estimator backward.
  *
  * Follows pith.science review, "What carries the argument" (the gradient is
@@ -264,6 +302,38 @@ quest_status quest_w4a4_linear_grouped(const uint8_t* a_codes, const float* a_sc
                                        const uint8_t* w_codes, const float* w_scales, int64_t M,
                                        int64_t N, int64_t K, int64_t group, void* y, float* y_f32,
                                        void* stream);
+
+/*
+ * quest_w4a4_linear_sparse24 -- integer linear layer with 2:4-sparse weight codes
+ * on the sparse tensor cores.
+ *
+ * The layer of quest_w4a4_linear (pith.science review, Figure 5; "Assumptions &
+ * free parameters": a transform on both operands leaves the product unchanged)
+ * with the weights in the 2:4-sparse format the pages evaluate (atlas.scime.ai
+ * summary, ablation table; pith.science review, Figure 4a), as
+ * quest_quantize_sparse24 writes them with rms_group = K (one step per row):
+ *     acc[m][n] = sum_k x_codes[m][k] * w[n][k]    (w = the weight codes with the
+ *                                                   pruned values zero; exact, int32)
+ *     y[m][n]   = bf16_rne( acc[m][n] * (x_scales[m] / 2) * (w_scales[n] / 2) )
+ * The weights are the sparse operand of tcgen05.mma.sp (kind::i8): each run of four
+ * K values contributes its two survivors.
+ *
+ * Arguments
+ *   x_codes    device int8 [M, K] (c = 2q + 1, as quest_quantize_operands writes), 16-byte aligned.
+ *   x_scales   device fp32 [M].
+ *   w_codes    device int8 [N, K / 2]: the survivors' codes, 16-byte aligned.
+ *   w_meta     device uint8 [N, K / 8]: the survivors' indices (quest_quantize_sparse24's
+ *              meta), 16-byte aligned.
+ *   w_scales   device fp32 [N].
+ *   M, N >= 0 (0 = no-op); N a multiple of 8; K a multiple of 128, K < 131072.
+ *   y          device bf16 [M, N], 16-byte aligned.
+ *   acc        device, optional int32 [M, N] copy of the accumulator (NULL = not written).
+ * Returns QUEST_OK, QUEST_EINVAL or QUEST_ECUDA; a bounded device-side wait that gives
+ * up is reported by quest_device_status as QUEST_ETIMEOUT.
+ */
+quest_status quest_w4a4_linear_sparse24(const int8_t* x_codes, const float* x_scales, const int8_t* w_codes,
+                                        const uint8_t* w_meta, const float* w_scales, int64_t M, int64_t N, int64_t K,
+                                        void* y, int32_t* acc, void* stream);
 
 /*
  * quest_fp4_linear -- linear layer on FP4 (E2M1) QuEST codes on the block-scaled
@@ -382,6 +452,14 @@ double quest_alpha(int bits);
  * parameters") applied to the FP4 grid the review's results list and Figure 4a
  * compare against INT4. Computed on the host at first use. */
 double quest_alpha_fp4(void);
+
+/* alpha_b of the 2:4-sparse format (quest_quantize_sparse24): 2^(b-1) times the step
+ * of the midrise grid that minimises the MSE of the values surviving 2:4 pruning of
+ * an N(0,1) input (of four values, the two of largest magnitude). The Gaussian fit of
+ * pith.science review, "What carries the argument" and "Assumptions & free
+ * parameters", taken on the sparse format the ablation table of the atlas.scime.ai
+ * summary evaluates. bits 1..8; NaN otherwise. Computed on the host at first use. */
+double quest_alpha_sparse24(int bits);
 
 /* Bits of the storage container of a b-bit packed code: 1, 2, 4, 4, 8, 8, 8, 8. 0 if invalid. */
 int quest_container_bits(int bits);

@@ -68,6 +68,32 @@ def test_alpha_table_matches_oracle(bits):
     assert a_lib == pytest.approx(a_ref, rel=3e-7)
 
 
+def test_alpha_sparse24_matches_oracle():
+    # library: closed-form cell masses, Gauss-Legendre first moments and bisection on
+    # the stationarity condition; oracle: Simpson quadrature of the MSE and a
+    # golden-section search, which resolves the argmin of a flat minimum to about
+    # sqrt(machine epsilon)
+    for bits in range(1, 9):
+        assert q.alpha_sparse24(bits) == pytest.approx(oracle.alpha_sparse24(bits)[0], rel=1e-7)
+    assert math.isnan(q.alpha_sparse24(0)) and math.isnan(q.alpha_sparse24(9))
+
+
+def test_quantize_sparse24_rejects_invalid_arguments():
+    lib = q.load_library()
+    ok = dict(x=FAKE, rows=4, cols=256, bits=4, had=128, rg=128, trust=1.0, codes=FAKE, meta=FAKE, scales=FAKE)
+
+    def call(**kw):
+        a = dict(ok)
+        a.update(kw)
+        return lib.quest_quantize_sparse24(a["x"], a["rows"], a["cols"], a["bits"], a["had"], a["rg"], a["trust"],
+                                           a["codes"], a["meta"], a["scales"], None, None, None)
+    for kw, st in [(dict(bits=8), 1), (dict(bits=0), 1), (dict(had=64), 2), (dict(had=100), 1), (dict(cols=200), 1),
+                   (dict(rg=512), 1), (dict(cols=384, rg=384), 2), (dict(trust=0.0), 1), (dict(x=None), 1),
+                   (dict(meta=None), 1), (dict(x=FAKE + 8), 1), (dict(codes=FAKE + 4), 1), (dict(rows=-1), 1)]:
+        assert call(**kw) == st, kw
+    assert call(rows=0, x=None, codes=None, meta=None, scales=None) == 0
+
+
 def test_alpha_fp4_matches_oracle():
     # library: bisection on the stationarity condition of the E2M1 grid; oracle:
     # golden section on its closed-form Gaussian MSE
