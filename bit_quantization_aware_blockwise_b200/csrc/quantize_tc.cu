@@ -46,12 +46,19 @@ __device__ __forceinline__ void lane_sums(const float2 (&P)[16], float (&ss)[Blk
 
 // Quantise and store this lane's 32 values: chunks c = t + 4f of the slab whose
 // first element is `e_slab` in row `row`.
-template <int PPB, int CB, int FMT, bool SAT>
+// OUT selects the outputs at compile time for the common calls, so that the
+// unrolled chunk loop is one straight block: 0 = as the call's flags say (mask,
+// dequant and the trust form read at run time), 1 = codes + mask bits with T >= 1,
+// no dequant, 2 = codes only.
+template <int PPB, int CB, int FMT, bool SAT, int OUT>
 __device__ __forceinline__ void emit(const QuantArgs& A, const float2 (&P)[16], const GroupK* G, int64_t row,
                                      int64_t e_slab, int t, bool valid) {
     const QuantConsts& k = A.c;
     uint8_t* codes = A.codes + row * A.codes_row_bytes + e_slab * CB / 8;
-    const bool do_mask = k.mask_mode >= 0, do_deq = valid && k.deq_mode >= 0;
+    const bool do_mask = OUT == 1 ? true : (OUT == 2 ? false : k.mask_mode >= 0);
+    const bool do_deq = OUT != 0 ? false : (valid && k.deq_mode >= 0);
+    const bool trust_ge1 = OUT == 1 ? true : k.trust_ge1 != 0;
+    const bool mask_bits = OUT == 1 ? true : k.mask_mode == 0;
     uint32_t cbytes = 0, mbytes = 0;
 #pragma unroll
     for (int f = 0; f < 4; ++f) {
@@ -65,7 +72,7 @@ __device__ __forceinline__ void emit(const QuantArgs& A, const float2 (&P)[16], 
             } else {
                 if (valid) *reinterpret_cast<uint2*>(codes + 8 * c) = fp4_operand_i8(w4);
             }
-            if (do_mask && !k.trust_ge1) mbytes |= mask_byte_fp4_cell<PPB>(P, G, f, w4, k) << (8 * f);
+            if (do_mask && !trust_ge1) mbytes |= mask_byte_fp4_cell<PPB>(P, G, f, w4, k) << (8 * f);
             if (do_deq) fp4_dequant<PPB>(w4, G, f, y);
         } else {
             float2 s[4];
@@ -107,7 +114,7 @@ __device__ __forceinline__ void emit(const QuantArgs& A, const float2 (&P)[16], 
     // trust mask bytes: one loop per form of the test, so that neither is predicated
     // into the other's path (the FP4 grid's general form was taken with its codes)
     if (do_mask) {
-        if (k.trust_ge1) {
+        if (trust_ge1) {
 #pragma unroll
             for (int f = 0; f < 4; ++f) mbytes |= mask_byte_edge<PPB>(P, G, f) << (8 * f);
         } else if constexpr (FMT < 3) {
@@ -120,7 +127,7 @@ __device__ __forceinline__ void emit(const QuantArgs& A, const float2 (&P)[16], 
         if (valid) *reinterpret_cast<uint32_t*>(codes + 4 * t) = w;
     }
     if (do_mask) {
-        if (k.mask_mode == 0) {
+        if (mask_bits) {
             const uint32_t w = quad_transpose_bytes(mbytes, t);
             if (valid) *reinterpret_cast<uint32_t*>(A.mask + row * A.mask_row_bytes + e_slab / 8 + 4 * t) = w;
         } else if (valid) {
@@ -139,7 +146,7 @@ __device__ __forceinline__ void emit(const QuantArgs& A, const float2 (&P)[16], 
 
 
 // Everything after the MMA for one slab of the group-RMS kernel.
-template <int HB, int CB, int FMT, bool SAT>
+template <int HB, int CB, int FMT, bool SAT, int OUT>
 __device__ __forceinline__ void group_slab(const QuantArgs& A, float2 (&P)[16], int64_t slab, bool valid,
                                            int lane) {
     constexpr int NBL = Blk<HB>::NBL, PPB = Blk<HB>::PPB;
@@ -156,7 +163,7 @@ __device__ __forceinline__ void group_slab(const QuantArgs& A, float2 (&P)[16], 
         G[b] = make_group(A.c, v);
     }
     const int64_t E = slab * 128;   // dense outputs: row 0 with a flat offset
-    emit<PPB, CB, FMT, SAT>(A, P, G, 0, E, t, valid);
+    emit<PPB, CB, FMT, SAT, OUT>(A, P, G, 0, E, t, valid);
     if (valid) {
         float* sp = A.scales + E / HB;
         if constexpr (HB == 256) {
@@ -180,7 +187,7 @@ __device__ __forceinline__ void group_slab(const QuantArgs& A, float2 (&P)[16], 
 // flight costs more in registers, and so in resident warps, than it hides).
 constexpr int kDepth = 1;
 
-template <int HB, int CB, int FMT, bool SAT>
+template <int HB, int CB, int FMT, bool SAT, int OUT>
 __global__ void __launch_bounds__(kThreads) quantize_tc_groups(const QuantArgs A) {
     pdl_wait();      // the previous kernel on the stream has completed
     pdl_trigger();   // the next one may be scheduled as CTAs of this one leave
@@ -214,7 +221,7 @@ __global__ void __launch_bounds__(kThreads) quantize_tc_groups(const QuantArgs A
             const int64_t next = slab + kDepth * step;
             if (next < total) load_slab(src_of(next), t, raw[d]);
             else zero4(raw[d]);
-            group_slab<HB, CB, FMT, SAT>(A, P, slab, slab < total, lane);
+            group_slab<HB, CB, FMT, SAT, OUT>(A, P, slab, slab < total, lane);
         }
     }
 }
@@ -225,7 +232,7 @@ __global__ void __launch_bounds__(kThreads) quantize_tc_groups(const QuantArgs A
 // MMA has consumed the current row's registers, so they land during its arithmetic.
 // The rows of a second tensor (A.rows2 > 0, the other operand of a linear layer)
 // follow those of the first in one virtual row space, so both take one launch.
-template <int HB, int CB, int FMT, bool SAT, int SUB>
+template <int HB, int CB, int FMT, bool SAT, int SUB, int OUT>
 __global__ void __launch_bounds__(kThreads, 3) quantize_tc_rows(const QuantArgs A, int spr) {
     pdl_wait();      // the previous kernel on the stream has completed
     pdl_trigger();   // the next one may be scheduled as CTAs of this one leave
@@ -283,13 +290,13 @@ __global__ void __launch_bounds__(kThreads, 3) quantize_tc_rows(const QuantArgs 
         }
 #pragma unroll
         for (int u = 0; u < SUB; ++u)
-            emit<PPB, CB, FMT, SAT>(T, P[u], G, row, int64_t(sc0 + 8 * u) * 128, t, valid);
+            emit<PPB, CB, FMT, SAT, OUT>(T, P[u], G, row, int64_t(sc0 + 8 * u) * 128, t, valid);
         if (valid && sc0 == 0 && t == 0) T.scales[row] = G[0].delta;
     }
 }
 
-template <int HB, int CB, int FMT, bool SAT>
-cudaError_t launch_t(const QuantArgs& a, bool row_mode, cudaStream_t s) {
+template <int HB, int CB, int FMT, bool SAT, int OUT>
+cudaError_t launch_out(const QuantArgs& a, bool row_mode, cudaStream_t s) {
     const int sms = sm_count();
     // grids never exceed the resident capacity (persistent, grid-stride)
     if (row_mode) {
@@ -300,16 +307,28 @@ cudaError_t launch_t(const QuantArgs& a, bool row_mode, cudaStream_t s) {
             const int64_t want = (warps + kThreads / 32 - 1) / (kThreads / 32);
             return launch_pdl(fn, dim3((unsigned)(want < cap ? want : cap)), dim3(kThreads), 0, s, a, spr);
         };
-        if (spr == 16) return go(quantize_tc_rows<HB, CB, FMT, SAT, 2>, 1);
-        if (spr == 8) return go(quantize_tc_rows<HB, CB, FMT, SAT, 1>, 1);
-        return go(quantize_tc_rows<HB, CB, FMT, SAT, 1>, 8 / spr);
+        if (spr == 16) return go(quantize_tc_rows<HB, CB, FMT, SAT, 2, OUT>, 1);
+        if (spr == 8) return go(quantize_tc_rows<HB, CB, FMT, SAT, 1, OUT>, 1);
+        return go(quantize_tc_rows<HB, CB, FMT, SAT, 1, OUT>, 8 / spr);
     }
     const int64_t slabs = a.rows * (a.cols / 128);
     const int64_t warps = (slabs + 7) / 8;
-    auto fn = quantize_tc_groups<HB, CB, FMT, SAT>;
+    auto fn = quantize_tc_groups<HB, CB, FMT, SAT, OUT>;
     const int64_t cap = int64_t(sms) * max_ctas_per_sm((const void*)fn, kThreads, 0);
     const int64_t want = (warps + kThreads / 32 - 1) / (kThreads / 32);
     return launch_pdl(fn, dim3((unsigned)(want < cap ? want : cap)), dim3(kThreads), 0, s, a);
+}
+
+// The compile-time output sets (OUT 1, 2) for Hadamard block 128; everything else
+// reads its flags at run time (OUT 0).
+template <int HB, int CB, int FMT, bool SAT>
+cudaError_t launch_t(const QuantArgs& a, bool row_mode, cudaStream_t s) {
+    if constexpr (HB == 128 && FMT < 3) {
+        const QuantConsts& k = a.c;
+        if (k.deq_mode < 0 && k.mask_mode == 0 && k.trust_ge1) return launch_out<HB, CB, FMT, SAT, 1>(a, row_mode, s);
+        if (k.deq_mode < 0 && k.mask_mode < 0) return launch_out<HB, CB, FMT, SAT, 2>(a, row_mode, s);
+    }
+    return launch_out<HB, CB, FMT, SAT, 0>(a, row_mode, s);
 }
 
 template <int HB, int CB, int FMT>

@@ -43,7 +43,7 @@ def decompress(codes, meta, rows, cols):
     return dense.reshape(rows, cols), kept.reshape(rows, cols)
 
 
-def check_sparse(res, o, rows, cols, trust=1.0):
+def check_sparse(res, o, rows, cols, trust=1.0, bits=4):
     dense, kept = decompress(res["codes"], res["meta"], rows, cols)
     t = o["t"]
     # a run is exempt when its 2nd and 3rd largest |t| are within the band
@@ -60,7 +60,11 @@ def check_sparse(res, o, rows, cols, trust=1.0):
     assert np.all(np.abs(q_gpu - o["q"])[surv & ex_code] <= 1)
     assert np.all(dense[kept == 0] == 0) and np.all(np.abs(dense[kept == 1]) % 2 == 1)
     check_f32(res["scales"], o["scale"], SCALE_REL, what="scales")
-    n_ex = int((surv & ex_code).sum())
+    # exempt codes: the band is 2e-5 |t| wide at every integer, and the spread of t
+    # grows as 2^(b-1) / alpha_b, so the allowance does too
+    n_code = int((surv & ex_code).sum())
+    assert n_code <= max(1e-4, 5e-5 * 2 ** (bits - 1)) * rows * cols + 2, f"{n_code} exempt codes"
+    n_ex = 0
     if res.get("mask") is not None:
         m = unpack_mask_bits(res["mask"], rows, cols)
         ex_mask = o["d_mask"] <= EXEMPT_REL * np.maximum(np.abs(t), 1.0)
@@ -70,13 +74,13 @@ def check_sparse(res, o, rows, cols, trust=1.0):
     if res.get("deq_bits") is not None:
         skip = ex_run | (surv & ex_code)
         check_bf16(res["deq_bits"], o["yhat"], skip=skip, what="dequant bf16")
-    # exempt values outside exempt runs, as for the dense quantizer; and exempt runs (a
-    # prune tie exempts its four values) at most 1e-4 of the runs
+    # exempt mask bits outside exempt runs, as for the dense quantizer; and exempt runs
+    # (a prune tie exempts its four values) at most 1e-4 of the runs
     frac = 1e-4 if trust >= 1 else 5e-4
-    assert n_ex <= frac * rows * cols + 2, f"{n_ex} exempt values of {rows * cols}"
+    assert n_ex <= frac * rows * cols + 2, f"{n_ex} exempt mask bits of {rows * cols}"
     n_runs = int(ex_run.sum()) // 4
     assert n_runs <= 1e-4 * rows * cols / 4 + 2, f"{n_runs} exempt runs of {rows * cols // 4}"
-    return n_ex + 4 * n_runs
+    return n_code + n_ex + 4 * n_runs
 
 
 def run(x, bits, rms_group=128, trust=1.0, dequant=True):
@@ -94,7 +98,7 @@ def test_activations_group_rms(cuda_device, bits, trust):
     # Student-t(3) activations with outlier channels; 37 rows x 768 (ragged last warp step)
     x = inputs.activations(37, 768, seed=40 + bits)
     o = oracle.quantize_sparse24(inputs.to_f64(x), bits=bits, had=128, trust=trust)
-    check_sparse(run(x, bits, trust=trust), o, 37, 768, trust)
+    check_sparse(run(x, bits, trust=trust), o, 37, 768, trust, bits)
 
 
 @pytest.mark.parametrize("spr", [1, 2, 4, 8, 16])
