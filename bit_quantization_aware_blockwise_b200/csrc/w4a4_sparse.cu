@@ -299,6 +299,249 @@ w4a4_sparse_kernel(const __grid_constant__ CUtensorMap map_w, const __grid_const
     }
 }
 
+// ---------------------------------------------------------------------------
+// CTA-pair variant (cluster of 2, tcgen05 cta_group::2): one sparse MMA of
+// M = 256 weight rows (128 per CTA, each CTA's own compressed rows and metadata),
+// N = 224 tokens (112 rows of B per CTA), K = 64 logical per instruction, issued by
+// the even CTA. A stage stages 24 KB per CTA instead of 38 KB for the same tensor
+// work per SM: the activation tile is split between the two CTAs. The metadata copy
+// (tcgen05.cp cta_group::2, issued by the even CTA) fills each CTA's TMEM slot from
+// its own shared memory. Barriers as the dense CTA-pair layer: both producers
+// signal the even CTA's full barrier, the even CTA's commits (multicast to both
+// CTAs) free stages and hand each CTA its half of the accumulator, each epilogue
+// returns its buffer with one arrival on the even CTA's barrier.
+constexpr int kPSStages = 7;
+constexpr int PBN = SBN / 2;                             // B rows per CTA
+constexpr uint32_t kPSStageB = PBN * SBK;                // 14 KB
+constexpr uint32_t kPSTx = 2 * (kSStageA + kPSStageB + kSStageE);   // both CTAs land on one barrier
+constexpr uint32_t kPSSmemA = 0;
+constexpr uint32_t kPSSmemB = kPSSmemA + kPSStages * kSStageA;
+constexpr uint32_t kPSSmemE = kPSSmemB + kPSStages * kPSStageB;
+constexpr uint32_t kPSSmemC = kPSSmemE + kPSStages * kSStageE;
+constexpr uint32_t kPSSmemScale = kPSSmemC + 2 * kSCBytes;
+constexpr uint32_t kPSSmemBar = kPSSmemScale + SBN * 4;
+constexpr uint32_t kPSNumBars = 2 * kPSStages + 4 + 1;
+constexpr uint32_t kPSSmemTmemSlot = kPSSmemBar + kPSNumBars * 8;
+constexpr uint32_t kPSSmemAbort = kPSSmemTmemSlot + 4;
+constexpr uint32_t kPSSmemTotal = kPSSmemAbort + 4 + 1024;
+static_assert(kPSSmemTotal <= 227 * 1024, "sparse pair kernel shared memory");
+static_assert(kPSStageB % 1024 == 0, "stage alignment");
+static_assert(kSMetaCol + 4 * kPSStages <= kTmemCols, "TMEM columns");
+
+constexpr uint32_t kIdescSpPair = (1u << 2) | (2u << 4) | (1u << 7) | (1u << 10) | (uint32_t(SBN >> 3) << 17) |
+                                  (uint32_t(256 >> 4) << 24);
+
+__device__ __forceinline__ void tc_mma_sp_i8_pair(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t e_tmem,
+                                                  uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %5, 0;\n\t"
+        "tcgen05.mma.sp.cta_group::2.kind::i8 [%0], %1, %2, [%3], %4, p;\n\t}" ::"r"(d_tmem),
+        "l"(adesc), "l"(bdesc), "r"(e_tmem), "r"(kIdescSpPair), "r"(accumulate)
+        : "memory");
+}
+__device__ __forceinline__ void tc_cp_meta_pair(uint32_t taddr, uint64_t sdesc) {
+    asm volatile("tcgen05.cp.cta_group::2.128x128b [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
+}
+
+struct SparsePairParams {
+    const float* sx;
+    const float* sw;
+    int32_t* acc;
+    int M, N, K;
+    int num_n2, num_m, num_k;   // 256-row weight pair tiles, token tiles (224), K stages (128)
+};
+
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
+w4a4_sparse_pair_kernel(const __grid_constant__ CUtensorMap map_w, const __grid_constant__ CUtensorMap map_x,
+                        const __grid_constant__ CUtensorMap map_e, const __grid_constant__ CUtensorMap map_y,
+                        const SparsePairParams p) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const uint32_t sbase = smem_u32(smem);
+    const uint32_t bar_full = sbase + kPSSmemBar;            // [kPSStages], used in the even CTA
+    const uint32_t bar_empty = bar_full + 8 * kPSStages;     // [kPSStages]
+    const uint32_t bar_tfull = bar_empty + 8 * kPSStages;    // [2]
+    const uint32_t bar_tempty = bar_tfull + 16;              // [2], used in the even CTA
+    const uint32_t bar_drain = bar_tempty + 16;              // [1]
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + kPSSmemAbort);
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kPSSmemTmemSlot);
+    float* s_scale = reinterpret_cast<float*>(smem + kPSSmemScale);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const uint32_t rank = cluster_rank();
+    const bool even = rank == 0;
+    const int pair = blockIdx.x >> 1, num_pairs = gridDim.x >> 1;
+    const int num_tiles = p.num_n2 * p.num_m;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kPSStages; ++s) {
+            mbar_init(bar_full + 8 * s, 1);
+            mbar_init(bar_empty + 8 * s, 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(bar_tfull + 8 * b, 1);
+            mbar_init(bar_tempty + 8 * b, 2);
+        }
+        mbar_init(bar_drain, 1);
+        *abort_flag = 0;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&map_w)) : "memory");
+        asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&map_x)) : "memory");
+        asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&map_e)) : "memory");
+        asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&map_y)) : "memory");
+    }
+    if (warp == 1) {
+        asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                         smem_u32(tmem_slot)),
+                     "r"(kTmemCols)
+                     : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+    }
+    tc_fence_before();
+    cluster_sync();
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+    pdl_wait();
+    pdl_trigger();
+
+    if (warp == 0) {
+        // ------------------------------------------------------------ TMA producer (both CTAs)
+        if (lane == 0) {
+            const uint32_t full_even = map_to_rank(bar_full, 0);
+            uint32_t stage = 0, phase = 0;
+            uint64_t issued = 0;
+            bool ok = true;
+            for (int tile = pair; tile < num_tiles && ok; tile += num_pairs) {
+                const int n0 = (tile % p.num_n2) * 256 + 128 * int(rank);
+                const int m0 = (tile / p.num_n2) * SBN + PBN * int(rank);
+                for (int kb = 0; kb < p.num_k; ++kb) {
+                    if (!mbar_wait(bar_empty + 8 * stage, phase ^ 1, abort_flag)) { ok = false; break; }
+                    if (even) mbar_arrive_expect_tx(bar_full + 8 * stage, kPSTx);
+                    const uint32_t fb = full_even + 8 * stage;
+                    tma_load_2d_pair(sbase + kPSSmemA + stage * kSStageA, &map_w, kb * (SBK / 2), n0, fb);
+                    tma_load_2d_pair(sbase + kPSSmemB + stage * kPSStageB, &map_x, kb * SBK, m0, fb);
+                    tma_load_2d_pair(sbase + kPSSmemE + stage * kSStageE, &map_e, kb * (SBK / 8), n0, fb);
+                    ++issued;
+                    if (++stage == kPSStages) { stage = 0; phase ^= 1; }
+                }
+            }
+            if (!ok && even) {
+                const uint64_t n = issued < kPSStages ? issued : kPSStages;
+                for (uint64_t i = issued - n; i < issued; ++i) {
+                    const uint32_t st = uint32_t(i % kPSStages), ph = uint32_t((i / kPSStages) & 1);
+                    const uint64_t t0 = global_timer_ns();
+                    while (!mbar_try_wait(bar_full + 8 * st, ph) && global_timer_ns() - t0 < kWaitLimitNs) {
+                    }
+                }
+            } else if (!ok) {
+                // the odd CTA cannot observe the even CTA's barrier: give its copies time to land
+                const uint64_t t0 = global_timer_ns();
+                while (global_timer_ns() - t0 < 10000000ull) {
+                }
+            }
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------------------ metadata copies and MMAs (even CTA)
+        if (even && lane == 0) {
+            uint32_t stage = 0, phase = 0;
+            bool ok = true;
+            int local = 0;
+            for (int tile = pair; tile < num_tiles && ok; tile += num_pairs, ++local) {
+                const uint32_t buf = local & 1, bphase = (local >> 1) & 1;
+                if (!mbar_wait(bar_tempty + 8 * buf, bphase ^ 1, abort_flag)) { ok = false; break; }
+                tc_fence_after();
+                const uint32_t d_tmem = tmem_base + buf * kSAccCols;
+                for (int kb = 0; kb < p.num_k; ++kb) {
+                    if (!mbar_wait(bar_full + 8 * stage, phase, abort_flag)) { ok = false; break; }
+                    tc_fence_after();
+                    const uint32_t a_addr = sbase + kPSSmemA + stage * kSStageA;
+                    const uint32_t b_addr = sbase + kPSSmemB + stage * kPSStageB;
+                    const uint32_t e_tmem = tmem_base + kSMetaCol + 4 * stage;
+                    tc_cp_meta_pair(e_tmem, smem_desc_meta(sbase + kPSSmemE + stage * kSStageE));
+#pragma unroll
+                    for (int kk = 0; kk < SBK / 64; ++kk) {
+                        tc_mma_sp_i8_pair(d_tmem, smem_desc_k64(a_addr + kk * 32), smem_desc_k128(b_addr + kk * 64),
+                                          e_tmem + 2 * kk, (kb | kk) != 0);
+                    }
+                    tc_commit_pair_mc(bar_empty + 8 * stage);
+                    if (++stage == kPSStages) { stage = 0; phase ^= 1; }
+                }
+                if (!ok) break;
+                tc_commit_pair_mc(bar_tfull + 8 * buf);
+            }
+            tc_commit_pair(bar_drain);
+            const uint64_t t0 = global_timer_ns();
+            while (!mbar_try_wait(bar_drain, 0) && global_timer_ns() - t0 < kWaitLimitNs) {
+            }
+        }
+    } else {
+        // ------------------------------------------------------------ epilogue (warps 2..5, both CTAs)
+        const int et = threadIdx.x - 64;
+        const int quarter = warp & 3;
+        const int row = quarter * 32 + lane;          // weight row within this CTA's half = TMEM lane
+        const uint32_t lane_addr = uint32_t(quarter * 32) << 16;
+        const uint32_t tempty_even = map_to_rank(bar_tempty, 0);
+        int local = 0, cbuf = 0;
+        for (int tile = pair; tile < num_tiles; tile += num_pairs, ++local) {
+            const int n0 = (tile % p.num_n2) * 256 + 128 * int(rank), m0 = (tile / p.num_n2) * SBN;
+            const uint32_t buf = local & 1, bphase = (local >> 1) & 1;
+            epi_bar();
+            for (int c = et; c < SBN; c += kEpiThreads) {
+                const int m = m0 + c;
+                s_scale[c] = m < p.M ? p.sx[m] * 0.5f : 0.0f;
+            }
+            const int n = n0 + row;
+            const float sw_half = n < p.N ? p.sw[n] * 0.5f : 0.0f;
+            const bool got = mbar_wait(bar_tfull + 8 * buf, bphase, abort_flag);
+            if (epi_any(!got)) break;   // also orders the token scales above (bar.red)
+            tc_fence_after();
+            const uint32_t t_acc = tmem_base + lane_addr + buf * kSAccCols;
+#pragma unroll 1
+            for (int c = 0; c < SBN / 32; ++c) {
+                uint32_t r[32];
+                QUEST_TMEM_LD32(t_acc + c * 32, r);
+                tmem_wait_ld();
+                const float* sc = s_scale + c * 32;
+                uint16_t* stg = reinterpret_cast<uint16_t*>(smem + kPSSmemC + cbuf * kSCBytes) + row;
+#pragma unroll
+                for (int i = 0; i < 32; ++i) {
+                    const float y = (float)(int32_t)r[i] * sw_half * sc[i];
+                    stg[i * SBM] = __bfloat16_as_ushort(__float2bfloat16_rn(y));
+                }
+                if (p.acc != nullptr && n < p.N) {
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) {
+                        const int m = m0 + c * 32 + i;
+                        if (m < p.M) p.acc[int64_t(m) * p.N + n] = (int32_t)r[i];
+                    }
+                }
+                fence_proxy_async_smem();
+                epi_bar();
+                if (et == 0) {
+                    tma_store_2d(&map_y, sbase + kPSSmemC + cbuf * kSCBytes, n0, m0 + c * 32);
+                    bulk_commit();
+                    bulk_wait_read_le1();
+                }
+                epi_bar();
+                cbuf ^= 1;
+            }
+            tc_fence_before();
+            epi_bar();
+            if (et == 0) mbar_arrive_remote(tempty_even + 8 * buf);
+        }
+        if (et == 0) bulk_wait_all();
+    }
+
+    tc_fence_before();
+    cluster_sync();
+    if (warp == 1) {
+        tc_fence_after();
+        asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem_base), "r"(kTmemCols)
+                     : "memory");
+    }
+}
+
 }  // namespace
 
 cudaError_t launch_w4a4_sparse24(const int8_t* X, const float* sx, const int8_t* W, const uint8_t* E,
@@ -307,13 +550,38 @@ cudaError_t launch_w4a4_sparse24(const int8_t* X, const float* sx, const int8_t*
     if (M == 0 || N == 0) return cudaSuccess;
     if (K == 0) return launch_zero_fill(y, acc, M * N, stream);
     CUtensorMap mw, mx, me, my;
+    // more than one 128-row block of weights: CTA pairs (M = 256 weight rows per MMA)
+    const bool pairs = N > SBM;
     if (!make_map_2d(&mw, CU_TENSOR_MAP_DATA_TYPE_UINT8, W, K / 2, N, K / 2, SBK / 2, SBM,
                      CU_TENSOR_MAP_SWIZZLE_64B) ||
-        !make_map_2d(&mx, CU_TENSOR_MAP_DATA_TYPE_UINT8, X, K, M, K, SBK, SBN, CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !make_map_2d(&mx, CU_TENSOR_MAP_DATA_TYPE_UINT8, X, K, M, K, SBK, pairs ? PBN : SBN,
+                     CU_TENSOR_MAP_SWIZZLE_128B) ||
         !make_map_2d(&me, CU_TENSOR_MAP_DATA_TYPE_UINT8, E, K / 8, N, K / 8, SBK / 8, SBM,
                      CU_TENSOR_MAP_SWIZZLE_NONE) ||
         !make_map_2d(&my, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, y, N, M, N * 2, SBM, 32, CU_TENSOR_MAP_SWIZZLE_NONE))
         return cudaErrorInvalidValue;
+    if (pairs) {
+        SparsePairParams pp;
+        pp.sx = sx; pp.sw = sw; pp.acc = acc;
+        pp.M = (int)M; pp.N = (int)N; pp.K = (int)K;
+        pp.num_n2 = (int)((N + 255) / 256);
+        pp.num_m = (int)((M + SBN - 1) / SBN);
+        pp.num_k = (int)((K + SBK - 1) / SBK);
+        static thread_local int pair_attr_dev = -1;
+        int dev = 0;
+        cudaGetDevice(&dev);
+        if (pair_attr_dev != dev) {
+            cudaError_t e = cudaFuncSetAttribute(w4a4_sparse_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                 kPSSmemTotal);
+            if (e != cudaSuccess) return e;
+            pair_attr_dev = dev;
+        }
+        const int tiles = pp.num_n2 * pp.num_m;
+        const int npairs = pair_clusters(dev, (const void*)w4a4_sparse_pair_kernel, kThreads, kPSSmemTotal);
+        const int grid_pairs = tiles < npairs ? tiles : npairs;
+        return launch_pdl(w4a4_sparse_pair_kernel, dim3(2 * grid_pairs), dim3(kThreads), kPSSmemTotal, stream, mw, mx,
+                          me, my, pp);
+    }
     SparseParams p;
     p.sx = sx; p.sw = sw; p.acc = acc;
     p.M = (int)M; p.N = (int)N; p.K = (int)K;
