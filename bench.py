@@ -468,15 +468,20 @@ def run_b200(args, world, rank, local):
         print(json.dumps(result), flush=True)
 
 
-def mma_probe(dev, gemm_tops=None, iters=20000, reps=5, fp4=False):
+def mma_probe(dev, gemm_tops=None, iters=20000, reps=5, fp4=False, sparse=False, cp_every=0):
     """Tensor-core rate with no memory traffic (back-to-back tcgen05.mma, one CTA per
-    SM): kind::i8 M 128 N 256 K 32, or with fp4 kind::mxf4 M 128 N 256 K 64 with unit
-    block scales; context for the linear layers' fractions."""
+    SM): kind::i8 M 128 N 256 K 32; with fp4 kind::mxf4 M 128 N 256 K 64 with unit
+    block scales; with sparse the 2:4-sparse kind::i8 M 128 N 256 K 64 (logical, the
+    dense-equivalent rate), metadata resident or copied every cp_every MMAs; context
+    for the linear layers' fractions."""
     import statistics
     import torch
     import bit_quantization_aware_blockwise_b200 as q
     stream = torch.cuda.current_stream(dev)
-    launch = q.probe_mma_fp4 if fp4 else q.probe_mma_i8
+    if sparse:
+        launch = lambda n, st: q.probe_mma_sp_i8(n, cp_every, st)
+    else:
+        launch = q.probe_mma_fp4 if fp4 else q.probe_mma_i8
     launch(iters, stream.cuda_stream)
     ts, ctas = [], 0
     for _ in range(reps):
@@ -488,7 +493,7 @@ def mma_probe(dev, gemm_tops=None, iters=20000, reps=5, fp4=False):
         ts.append(a.elapsed_time(b))
     q.probe_status(stream.cuda_stream)
     ms = statistics.median(ts)
-    tops = 2.0 * 128 * 256 * (64 if fp4 else 32) * iters * ctas / (ms * 1e-3) / 1e12
+    tops = 2.0 * 128 * 256 * (64 if (fp4 or sparse) else 32) * iters * ctas / (ms * 1e-3) / 1e12
     out = {"tops": round(tops, 1), "iters": iters, "ctas": ctas,
            "note": "timed alone right after the bench loop (burst); the GEMM's roofline peak"}
     if gemm_tops is not None:
@@ -940,7 +945,14 @@ def run_configs(args):
     fp4_tops = next(r["tops"] for r in rows if "block-scaled FP4" in r["case"])
     probe4 = mma_probe(dev, fp4_tops, fp4=True)
     probe4["note"] = "timed alone after the configs; the FP4 layer's fraction stays of 4 x the measured bf16 peak"
-    print(json.dumps({"configs": rows, "int8_mma_probe": probe, "fp4_mma_probe": probe4, "peaks": peaks}),
+    sp_row = next(r for r in rows if r["case"].startswith("2:4-sparse W4A4 linear"))
+    probe_sp = mma_probe(dev, sp_row["tops"], sparse=True)
+    probe_sp["note"] = "2:4-sparse kind::i8, metadata resident in TMEM, dense-equivalent ops"
+    sp_row["frac_sparse_probe"] = probe_sp["gemm_frac_of_probe"]
+    probe_sp_cp = mma_probe(dev, None, sparse=True, cp_every=2)
+    probe_sp_cp["note"] = "the same with a tcgen05.cp of metadata before every second MMA"
+    print(json.dumps({"configs": rows, "int8_mma_probe": probe, "fp4_mma_probe": probe4,
+                      "sparse_mma_probe": probe_sp, "sparse_mma_probe_cp2": probe_sp_cp, "peaks": peaks}),
           flush=True)
 
 

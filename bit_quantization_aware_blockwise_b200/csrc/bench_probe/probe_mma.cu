@@ -195,6 +195,113 @@ __global__ void __launch_bounds__(kProbeThreads, 1) probe_mma_fp4_kernel(int ite
     }
 }
 
+// The same for the 2:4-sparse integer kind of the sparse linear layer:
+// tcgen05.mma.sp kind::i8 (M = 128, N = 256, K = 64 logical, 32 bytes of the
+// compressed A per row), metadata in TMEM (byte 0x44: every run keeps indices
+// 0 and 1). With cp_every = c > 0, a tcgen05.cp (128x128b, four columns of
+// metadata from shared memory) precedes every c-th MMA and that MMA and the
+// next c - 1 read the copied columns, the pattern of a layer that stages its
+// metadata through shared memory with its operands (c = 2 per 128-value stage).
+constexpr uint32_t kIdescProbeSp = (1u << 2) | (2u << 4) | (1u << 7) | (1u << 10) | (uint32_t(256 >> 3) << 17) |
+                                   (uint32_t(128 >> 4) << 24);
+constexpr uint32_t kMetaSmem = kSlot + 1024 - (kSlot % 1024);   // 2 KB: 128 rows x 16 bytes
+constexpr int kMetaSlots = 8;                                    // rotating 4-column slots from column 288
+static_assert(kMetaSmem + 2048 <= kProbeSmem, "probe shared memory");
+
+__global__ void __launch_bounds__(kProbeThreads, 1) probe_mma_sp_i8_kernel(int iters, int cp_every) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const uint32_t sbase = static_cast<uint32_t>(__cvta_generic_to_shared(smem));
+    for (uint32_t i = threadIdx.x * 16; i < kBar; i += kProbeThreads * 16)
+        *reinterpret_cast<uint4*>(smem + i) = make_uint4(0x01010101u, 0x01010101u, 0x01010101u, 0x01010101u);
+    for (uint32_t i = threadIdx.x * 16; i < 2048; i += kProbeThreads * 16)
+        *reinterpret_cast<uint4*>(smem + kMetaSmem + i) = make_uint4(0x44444444u, 0x44444444u, 0x44444444u,
+                                                                     0x44444444u);
+    const uint32_t bar = sbase + kBar;
+    if (threadIdx.x == 0) {
+        asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(bar) : "memory");
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    const int warp = threadIdx.x >> 5;
+    if (warp == 0) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], 512;" ::"r"(sbase + kSlot)
+                     : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    }
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+    __syncthreads();
+    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+    const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(smem + kSlot);
+    {
+        // metadata 0x44 in this warp's lane quarter, columns 256-287 (the resident set)
+        // and 288-319 (the copy slots, so the first reads before any copy are valid too)
+        const uint32_t v = 0x44444444u;
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            const uint32_t taddr = tmem + (uint32_t(warp * 32) << 16) + 256 + 32 * h;
+            asm volatile(
+                "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
+                "{%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,"
+                "%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1};" ::"r"(taddr),
+                "r"(v)
+                : "memory");
+        }
+        asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+    }
+    asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+    __syncthreads();
+    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+
+    if (threadIdx.x == 0) {
+        const uint64_t a = probe_desc(sbase + kA), b = probe_desc(sbase + kB);
+        uint64_t md = 0;
+        md |= uint64_t(((sbase + kMetaSmem) >> 4) & 0x3FFFu);
+        md |= uint64_t(2048 >> 4) << 16;
+        md |= uint64_t(128 >> 4) << 32;
+        md |= uint64_t(1) << 46;
+        uint32_t e = tmem + 256;
+        for (int i = 0; i < iters; ++i) {
+            if (cp_every > 0 && i % cp_every == 0) {
+                e = tmem + 288 + 4 * uint32_t((i / cp_every) % kMetaSlots);
+                asm volatile("tcgen05.cp.cta_group::1.128x128b [%0], %1;" ::"r"(e), "l"(md) : "memory");
+            }
+            const uint32_t ei = cp_every > 0 ? e + 2 * uint32_t((i % cp_every) & 1) : e;
+            asm volatile(
+                "{\n\t.reg .pred p;\n\t"
+                "setp.ne.b32 p, %5, 0;\n\t"
+                "tcgen05.mma.sp.cta_group::1.kind::i8 [%0], %1, %2, [%3], %4, p;\n\t}" ::"r"(tmem),
+                "l"(a), "l"(b), "r"(ei), "r"(kIdescProbeSp), "r"(i)
+                : "memory");
+        }
+        asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
+                     : "memory");
+        uint64_t t0, t;
+        asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t0));
+        for (;;) {
+            uint32_t ok;
+            asm volatile(
+                "{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], 0;\n\t"
+                "selp.u32 %0, 1, 0, p;\n\t}"
+                : "=r"(ok)
+                : "r"(bar)
+                : "memory");
+            if (ok) break;
+            asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+            if (t - t0 > 2000000000ull) {
+                atomicExch(&g_probe_status, (int)QUEST_ETIMEOUT);
+                break;
+            }
+        }
+    }
+    asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+    __syncthreads();
+    if (warp == 0) {
+        asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, 512;" ::"r"(tmem) : "memory");
+    }
+}
+
 }  // namespace
 }  // namespace quest
 
@@ -244,4 +351,22 @@ extern "C" quest_status quest_probe_status(void* stream) {
         cudaStreamSynchronize(s);
     }
     return static_cast<quest_status>(v);
+}
+
+extern "C" quest_status quest_probe_mma_sp_i8(int iters, int cp_every, int* ctas, void* stream) {
+    using namespace quest;
+    if (iters < 1 || iters > kMaxIters || cp_every < 0 || cp_every > 64 || ctas == nullptr) return QUEST_EINVAL;
+    static thread_local int attr_dev = -1;
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (attr_dev != dev) {
+        if (cudaFuncSetAttribute(probe_mma_sp_i8_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 kProbeSmem + 1024) != cudaSuccess)
+            return QUEST_ECUDA;
+        attr_dev = dev;
+    }
+    *ctas = probe_sm_count();
+    probe_mma_sp_i8_kernel<<<*ctas, kProbeThreads, kProbeSmem + 1024, static_cast<cudaStream_t>(stream)>>>(iters,
+                                                                                                       cp_every);
+    return cudaGetLastError() == cudaSuccess ? QUEST_OK : QUEST_ECUDA;
 }

@@ -59,6 +59,7 @@ constexpr uint32_t kSSmemE = kSSmemB + kSStages * kSStageB;
 constexpr uint32_t kSCBytes = 32 * SBM * 2;         // transposed stage: 32 tokens x 128 weight rows, bf16
 constexpr uint32_t kSSmemC = kSSmemE + kSStages * kSStageE;
 constexpr uint32_t kSSmemScale = kSSmemC + 2 * kSCBytes;   // float[SBN]: the tokens' scales
+static_assert(kSSmemScale % 16 == 0, "16-byte scale loads");
 constexpr uint32_t kSSmemBar = kSSmemScale + SBN * 4;
 constexpr uint32_t kSNumBars = 2 * kSStages + 4 + 1;
 constexpr uint32_t kSSmemTmemSlot = kSSmemBar + kSNumBars * 8;
@@ -109,6 +110,30 @@ __device__ __forceinline__ uint64_t smem_desc_meta(uint32_t addr) {
 }
 __device__ __forceinline__ void tc_cp_meta(uint32_t taddr, uint64_t sdesc) {
     asm volatile("tcgen05.cp.cta_group::1.128x128b [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
+}
+
+// One 32-token chunk of a weight row (TMEM lane): scale, round to bf16 and store
+// the 32 values down the transposed stage (token i of the chunk at row i, this
+// weight row at its column). The chunk's token scales are read into registers
+// (as float4) before any store: the 16-bit stores and the scale loads both go
+// to shared memory, and interleaved the compiler has to keep every store ahead
+// of the next load, which chained the 32 conversions one after another.
+__device__ __forceinline__ void stage_chunk_transposed(const uint32_t (&r)[32], float sw_half, const float* sc,
+                                                       uint16_t* stg) {
+    float s[32];
+#pragma unroll
+    for (int i = 0; i < 32; i += 4) {
+        const float4 v = *reinterpret_cast<const float4*>(sc + i);
+        s[i] = v.x;
+        s[i + 1] = v.y;
+        s[i + 2] = v.z;
+        s[i + 3] = v.w;
+    }
+    uint16_t h[32];
+#pragma unroll
+    for (int i = 0; i < 32; ++i) h[i] = __bfloat16_as_ushort(__float2bfloat16_rn((float)(int32_t)r[i] * sw_half * s[i]));
+#pragma unroll
+    for (int i = 0; i < 32; ++i) stg[i * SBM] = h[i];
 }
 
 struct SparseParams {
@@ -259,14 +284,9 @@ w4a4_sparse_kernel(const __grid_constant__ CUtensorMap map_w, const __grid_const
                 uint32_t r[32];
                 QUEST_TMEM_LD32(t_acc + c * 32, r);
                 tmem_wait_ld();
-                const float* sc = s_scale + c * 32;
                 // transposed stage: token i of the chunk is row i, this weight row its column
-                uint16_t* stg = reinterpret_cast<uint16_t*>(smem + kSSmemC + cbuf * kSCBytes) + row;
-#pragma unroll
-                for (int i = 0; i < 32; ++i) {
-                    const float y = (float)(int32_t)r[i] * sw_half * sc[i];
-                    stg[i * SBM] = __bfloat16_as_ushort(__float2bfloat16_rn(y));
-                }
+                stage_chunk_transposed(r, sw_half, s_scale + c * 32,
+                                       reinterpret_cast<uint16_t*>(smem + kSSmemC + cbuf * kSCBytes) + row);
                 if (p.acc != nullptr && n < p.N) {
 #pragma unroll
                     for (int i = 0; i < 32; ++i) {
@@ -310,23 +330,45 @@ w4a4_sparse_kernel(const __grid_constant__ CUtensorMap map_w, const __grid_const
 // signal the even CTA's full barrier, the even CTA's commits (multicast to both
 // CTAs) free stages and hand each CTA its half of the accumulator, each epilogue
 // returns its buffer with one arrival on the even CTA's barrier.
+//
+// Metadata, two forms. Staged (any K): a 2 KB slab rides in every stage of the
+// ring and one tcgen05.cp per stage moves it into a rotating 4-column slot just
+// before the stage's two MMAs. Resident (K <= 2048): the 64 TMEM columns after
+// the two accumulators hold the metadata of the whole reduction for this CTA's
+// 128 weight rows; the pair walks its tiles in weight-major order, so the block
+// (K/8 bytes per row) is loaded and copied into TMEM once per weight tile, and
+// the ring carries only operand codes. Before overwriting the columns for the
+// next weight tile the issuer waits for the previous tile's accumulator commit
+// (its MMAs have read the old metadata); the copies' own commit frees the
+// shared-memory block for the producer.
 constexpr int kPSStages = 7;
 constexpr int PBN = SBN / 2;                             // B rows per CTA
 constexpr uint32_t kPSStageB = PBN * SBK;                // 14 KB
-constexpr uint32_t kPSTx = 2 * (kSStageA + kPSStageB + kSStageE);   // both CTAs land on one barrier
-constexpr uint32_t kPSSmemA = 0;
-constexpr uint32_t kPSSmemB = kPSSmemA + kPSStages * kSStageA;
-constexpr uint32_t kPSSmemE = kPSSmemB + kPSStages * kPSStageB;
-constexpr uint32_t kPSSmemC = kPSSmemE + kPSStages * kSStageE;
-constexpr uint32_t kPSSmemScale = kPSSmemC + 2 * kSCBytes;
-constexpr uint32_t kPSSmemBar = kPSSmemScale + SBN * 4;
-constexpr uint32_t kPSNumBars = 2 * kPSStages + 4 + 1;
-constexpr uint32_t kPSSmemTmemSlot = kPSSmemBar + kPSNumBars * 8;
-constexpr uint32_t kPSSmemAbort = kPSSmemTmemSlot + 4;
-constexpr uint32_t kPSSmemTotal = kPSSmemAbort + 4 + 1024;
-static_assert(kPSSmemTotal <= 227 * 1024, "sparse pair kernel shared memory");
+// Shared memory of the pair kernel. Staged metadata: a 2 KB slab per stage in the
+// ring. Resident metadata (K <= kResidentMaxK): no metadata in the ring, one slab
+// per 128-value K stage of the whole reduction, loaded once per weight tile.
+constexpr int kResidentMaxK = (kTmemCols - kSMetaCol) / 4 * SBK;   // 16 stages of 4 columns: K <= 2048
+template <bool R>
+struct PairLayout {
+    static constexpr uint32_t kStageE = R ? 0u : kSStageE;
+    static constexpr uint32_t kTx = 2 * (kSStageA + kPSStageB + kStageE);   // both CTAs land on one barrier
+    static constexpr uint32_t kA = 0;
+    static constexpr uint32_t kB = kA + kPSStages * kSStageA;
+    static constexpr uint32_t kE = kB + kPSStages * kPSStageB;     // staged slabs, or the resident block
+    static constexpr uint32_t kEBytes = R ? uint32_t(kResidentMaxK / SBK) * kSStageE : kPSStages * kSStageE;
+    static constexpr uint32_t kC = kE + kEBytes;
+    static constexpr uint32_t kScale = kC + 2 * kSCBytes;
+    static constexpr uint32_t kBar = kScale + SBN * 4;
+    static constexpr uint32_t kNumBars = 2 * kPSStages + 4 + 1 + 2;   // + metadata full / empty
+    static constexpr uint32_t kTmemSlot = kBar + kNumBars * 8;
+    static constexpr uint32_t kAbort = kTmemSlot + 4;
+    static constexpr uint32_t kTotal = kAbort + 4 + 1024;
+    static_assert(kTotal <= 227 * 1024, "sparse pair kernel shared memory");
+    static_assert(kScale % 16 == 0, "16-byte scale loads");
+};
 static_assert(kPSStageB % 1024 == 0, "stage alignment");
 static_assert(kSMetaCol + 4 * kPSStages <= kTmemCols, "TMEM columns");
+static_assert(kResidentMaxK >= SBK, "resident metadata");
 
 constexpr uint32_t kIdescSpPair = (1u << 2) | (2u << 4) | (1u << 7) | (1u << 10) | (uint32_t(SBN >> 3) << 17) |
                                   (uint32_t(256 >> 4) << 24);
@@ -352,27 +394,41 @@ struct SparsePairParams {
     int num_n2, num_m, num_k;   // 256-row weight pair tiles, token tiles (224), K stages (128)
 };
 
+template <bool kResident>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 w4a4_sparse_pair_kernel(const __grid_constant__ CUtensorMap map_w, const __grid_constant__ CUtensorMap map_x,
                         const __grid_constant__ CUtensorMap map_e, const __grid_constant__ CUtensorMap map_y,
                         const SparsePairParams p) {
+    using L = PairLayout<kResident>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const uint32_t sbase = smem_u32(smem);
-    const uint32_t bar_full = sbase + kPSSmemBar;            // [kPSStages], used in the even CTA
+    const uint32_t bar_full = sbase + L::kBar;               // [kPSStages], used in the even CTA
     const uint32_t bar_empty = bar_full + 8 * kPSStages;     // [kPSStages]
     const uint32_t bar_tfull = bar_empty + 8 * kPSStages;    // [2]
     const uint32_t bar_tempty = bar_tfull + 16;              // [2], used in the even CTA
     const uint32_t bar_drain = bar_tempty + 16;              // [1]
-    volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + kPSSmemAbort);
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kPSSmemTmemSlot);
-    float* s_scale = reinterpret_cast<float*>(smem + kPSSmemScale);
+    const uint32_t bar_mfull = bar_drain + 8;                // resident metadata landed (even CTA)
+    const uint32_t bar_mempty = bar_mfull + 8;               // resident metadata copied into TMEM
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kAbort);
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kTmemSlot);
+    float* s_scale = reinterpret_cast<float*>(smem + L::kScale);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const uint32_t rank = cluster_rank();
     const bool even = rank == 0;
     const int pair = blockIdx.x >> 1, num_pairs = gridDim.x >> 1;
     const int num_tiles = p.num_n2 * p.num_m;
+    // Tiles of this pair. Staged metadata: every num_pairs-th tile, token tiles
+    // fastest within a weight tile's column of the grid (tile = n2 + num_n2 * mt).
+    // Resident metadata: a contiguous run of tiles in weight-major order
+    // (tile = mt + num_m * n2), so a pair meets one or two weight tiles and
+    // copies each one's metadata into TMEM once.
+    const int t_begin = kResident ? int((int64_t(pair) * num_tiles) / num_pairs) : pair;
+    const int t_end = kResident ? int((int64_t(pair + 1) * num_tiles) / num_pairs) : num_tiles;
+    const int t_step = kResident ? 1 : num_pairs;
+    auto tile_n2 = [&](int tile) { return kResident ? tile / p.num_m : tile % p.num_n2; };
+    auto tile_mt = [&](int tile) { return kResident ? tile % p.num_m : tile / p.num_n2; };
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < kPSStages; ++s) {
@@ -384,6 +440,8 @@ w4a4_sparse_pair_kernel(const __grid_constant__ CUtensorMap map_w, const __grid_
             mbar_init(bar_tempty + 8 * b, 2);
         }
         mbar_init(bar_drain, 1);
+        mbar_init(bar_mfull, 1);
+        mbar_init(bar_mempty, 1);
         *abort_flag = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
         asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&map_w)) : "memory");
@@ -409,21 +467,41 @@ w4a4_sparse_pair_kernel(const __grid_constant__ CUtensorMap map_w, const __grid_
         // ------------------------------------------------------------ TMA producer (both CTAs)
         if (lane == 0) {
             const uint32_t full_even = map_to_rank(bar_full, 0);
-            uint32_t stage = 0, phase = 0;
+            uint32_t stage = 0, phase = 0, mphase = 0;
             uint64_t issued = 0;
-            bool ok = true;
-            for (int tile = pair; tile < num_tiles && ok; tile += num_pairs) {
-                const int n0 = (tile % p.num_n2) * 256 + 128 * int(rank);
-                const int m0 = (tile / p.num_n2) * SBN + PBN * int(rank);
+            bool ok = true, mphase_issued = false;
+            int cur_n2 = -1;
+            for (int tile = t_begin; tile < t_end && ok; tile += t_step) {
+                const int n0 = tile_n2(tile) * 256 + 128 * int(rank);
+                const int m0 = tile_mt(tile) * SBN + PBN * int(rank);
+                if (kResident && tile_n2(tile) != cur_n2) {
+                    // the whole reduction's metadata of this CTA's 128 weight rows, once
+                    // the previous weight tile's block has been copied into TMEM
+                    if (!mbar_wait(bar_mempty, mphase ^ 1, abort_flag)) { ok = false; break; }
+                    if (even) mbar_arrive_expect_tx(bar_mfull, 2u * uint32_t(p.num_k) * kSStageE);
+                    const uint32_t mb = map_to_rank(bar_mfull, 0);
+                    for (int kb = 0; kb < p.num_k; ++kb)
+                        tma_load_2d_pair(sbase + L::kE + kb * kSStageE, &map_e, kb * (SBK / 8), n0, mb);
+                    mphase ^= 1;
+                    mphase_issued = true;
+                    cur_n2 = tile_n2(tile);
+                }
                 for (int kb = 0; kb < p.num_k; ++kb) {
                     if (!mbar_wait(bar_empty + 8 * stage, phase ^ 1, abort_flag)) { ok = false; break; }
-                    if (even) mbar_arrive_expect_tx(bar_full + 8 * stage, kPSTx);
+                    if (even) mbar_arrive_expect_tx(bar_full + 8 * stage, L::kTx);
                     const uint32_t fb = full_even + 8 * stage;
-                    tma_load_2d_pair(sbase + kPSSmemA + stage * kSStageA, &map_w, kb * (SBK / 2), n0, fb);
-                    tma_load_2d_pair(sbase + kPSSmemB + stage * kPSStageB, &map_x, kb * SBK, m0, fb);
-                    tma_load_2d_pair(sbase + kPSSmemE + stage * kSStageE, &map_e, kb * (SBK / 8), n0, fb);
+                    tma_load_2d_pair(sbase + L::kA + stage * kSStageA, &map_w, kb * (SBK / 2), n0, fb);
+                    tma_load_2d_pair(sbase + L::kB + stage * kPSStageB, &map_x, kb * SBK, m0, fb);
+                    if (!kResident)
+                        tma_load_2d_pair(sbase + L::kE + stage * kSStageE, &map_e, kb * (SBK / 8), n0, fb);
                     ++issued;
                     if (++stage == kPSStages) { stage = 0; phase ^= 1; }
+                }
+            }
+            if (!ok && even && kResident && mphase_issued) {
+                // the last metadata block may still be landing
+                const uint64_t t0 = global_timer_ns();
+                while (!mbar_try_wait(bar_mfull, mphase ^ 1) && global_timer_ns() - t0 < kWaitLimitNs) {
                 }
             }
             if (!ok && even) {
@@ -444,21 +522,36 @@ w4a4_sparse_pair_kernel(const __grid_constant__ CUtensorMap map_w, const __grid_
     } else if (warp == 1) {
         // ------------------------------------------------------------ metadata copies and MMAs (even CTA)
         if (even && lane == 0) {
-            uint32_t stage = 0, phase = 0;
+            uint32_t stage = 0, phase = 0, mphase = 0;
             bool ok = true;
-            int local = 0;
-            for (int tile = pair; tile < num_tiles && ok; tile += num_pairs, ++local) {
+            int local = 0, cur_n2 = -1;
+            for (int tile = t_begin; tile < t_end && ok; tile += t_step, ++local) {
                 const uint32_t buf = local & 1, bphase = (local >> 1) & 1;
                 if (!mbar_wait(bar_tempty + 8 * buf, bphase ^ 1, abort_flag)) { ok = false; break; }
+                if (kResident && tile_n2(tile) != cur_n2) {
+                    if (cur_n2 >= 0) {
+                        // the previous tile's MMAs (its accumulator commit) must have read
+                        // the old metadata before the copies overwrite those columns
+                        const uint32_t pb = (local - 1) & 1, pph = ((local - 1) >> 1) & 1;
+                        if (!mbar_wait(bar_tfull + 8 * pb, pph, abort_flag)) { ok = false; break; }
+                    }
+                    if (!mbar_wait(bar_mfull, mphase, abort_flag)) { ok = false; break; }
+                    tc_fence_after();
+                    for (int kb = 0; kb < p.num_k; ++kb)
+                        tc_cp_meta_pair(tmem_base + kSMetaCol + 4 * kb, smem_desc_meta(sbase + L::kE + kb * kSStageE));
+                    tc_commit_pair_mc(bar_mempty);   // both CTAs' blocks are free once copied
+                    mphase ^= 1;
+                    cur_n2 = tile_n2(tile);
+                }
                 tc_fence_after();
                 const uint32_t d_tmem = tmem_base + buf * kSAccCols;
                 for (int kb = 0; kb < p.num_k; ++kb) {
                     if (!mbar_wait(bar_full + 8 * stage, phase, abort_flag)) { ok = false; break; }
                     tc_fence_after();
-                    const uint32_t a_addr = sbase + kPSSmemA + stage * kSStageA;
-                    const uint32_t b_addr = sbase + kPSSmemB + stage * kPSStageB;
-                    const uint32_t e_tmem = tmem_base + kSMetaCol + 4 * stage;
-                    tc_cp_meta_pair(e_tmem, smem_desc_meta(sbase + kPSSmemE + stage * kSStageE));
+                    const uint32_t a_addr = sbase + L::kA + stage * kSStageA;
+                    const uint32_t b_addr = sbase + L::kB + stage * kPSStageB;
+                    const uint32_t e_tmem = tmem_base + kSMetaCol + 4 * (kResident ? uint32_t(kb) : stage);
+                    if (!kResident) tc_cp_meta_pair(e_tmem, smem_desc_meta(sbase + L::kE + stage * kSStageE));
 #pragma unroll
                     for (int kk = 0; kk < SBK / 64; ++kk) {
                         tc_mma_sp_i8_pair(d_tmem, smem_desc_k64(a_addr + kk * 32), smem_desc_k128(b_addr + kk * 64),
@@ -483,8 +576,8 @@ w4a4_sparse_pair_kernel(const __grid_constant__ CUtensorMap map_w, const __grid_
         const uint32_t lane_addr = uint32_t(quarter * 32) << 16;
         const uint32_t tempty_even = map_to_rank(bar_tempty, 0);
         int local = 0, cbuf = 0;
-        for (int tile = pair; tile < num_tiles; tile += num_pairs, ++local) {
-            const int n0 = (tile % p.num_n2) * 256 + 128 * int(rank), m0 = (tile / p.num_n2) * SBN;
+        for (int tile = t_begin; tile < t_end; tile += t_step, ++local) {
+            const int n0 = tile_n2(tile) * 256 + 128 * int(rank), m0 = tile_mt(tile) * SBN;
             const uint32_t buf = local & 1, bphase = (local >> 1) & 1;
             epi_bar();
             for (int c = et; c < SBN; c += kEpiThreads) {
@@ -502,13 +595,8 @@ w4a4_sparse_pair_kernel(const __grid_constant__ CUtensorMap map_w, const __grid_
                 uint32_t r[32];
                 QUEST_TMEM_LD32(t_acc + c * 32, r);
                 tmem_wait_ld();
-                const float* sc = s_scale + c * 32;
-                uint16_t* stg = reinterpret_cast<uint16_t*>(smem + kPSSmemC + cbuf * kSCBytes) + row;
-#pragma unroll
-                for (int i = 0; i < 32; ++i) {
-                    const float y = (float)(int32_t)r[i] * sw_half * sc[i];
-                    stg[i * SBM] = __bfloat16_as_ushort(__float2bfloat16_rn(y));
-                }
+                stage_chunk_transposed(r, sw_half, s_scale + c * 32,
+                                       reinterpret_cast<uint16_t*>(smem + L::kC + cbuf * kSCBytes) + row);
                 if (p.acc != nullptr && n < p.N) {
 #pragma unroll
                     for (int i = 0; i < 32; ++i) {
@@ -519,7 +607,7 @@ w4a4_sparse_pair_kernel(const __grid_constant__ CUtensorMap map_w, const __grid_
                 fence_proxy_async_smem();
                 epi_bar();
                 if (et == 0) {
-                    tma_store_2d(&map_y, sbase + kPSSmemC + cbuf * kSCBytes, n0, m0 + c * 32);
+                    tma_store_2d(&map_y, sbase + L::kC + cbuf * kSCBytes, n0, m0 + c * 32);
                     bulk_commit();
                     bulk_wait_read_le1();
                 }
@@ -540,6 +628,26 @@ w4a4_sparse_pair_kernel(const __grid_constant__ CUtensorMap map_w, const __grid_
         asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem_base), "r"(kTmemCols)
                      : "memory");
     }
+}
+
+template <bool kResident>
+cudaError_t launch_sparse_pair(const CUtensorMap& mw, const CUtensorMap& mx, const CUtensorMap& me,
+                               const CUtensorMap& my, const SparsePairParams& pp, cudaStream_t stream) {
+    constexpr uint32_t smem = PairLayout<kResident>::kTotal;
+    static thread_local int attr_dev = -1;
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (attr_dev != dev) {
+        cudaError_t e = cudaFuncSetAttribute(w4a4_sparse_pair_kernel<kResident>,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+        if (e != cudaSuccess) return e;
+        attr_dev = dev;
+    }
+    const int tiles = pp.num_n2 * pp.num_m;
+    const int npairs = pair_clusters(dev, (const void*)w4a4_sparse_pair_kernel<kResident>, kThreads, smem);
+    const int grid_pairs = tiles < npairs ? tiles : npairs;
+    return launch_pdl(w4a4_sparse_pair_kernel<kResident>, dim3(2 * grid_pairs), dim3(kThreads), smem, stream, mw, mx,
+                      me, my, pp);
 }
 
 }  // namespace
@@ -567,20 +675,8 @@ cudaError_t launch_w4a4_sparse24(const int8_t* X, const float* sx, const int8_t*
         pp.num_n2 = (int)((N + 255) / 256);
         pp.num_m = (int)((M + SBN - 1) / SBN);
         pp.num_k = (int)((K + SBK - 1) / SBK);
-        static thread_local int pair_attr_dev = -1;
-        int dev = 0;
-        cudaGetDevice(&dev);
-        if (pair_attr_dev != dev) {
-            cudaError_t e = cudaFuncSetAttribute(w4a4_sparse_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                                 kPSSmemTotal);
-            if (e != cudaSuccess) return e;
-            pair_attr_dev = dev;
-        }
-        const int tiles = pp.num_n2 * pp.num_m;
-        const int npairs = pair_clusters(dev, (const void*)w4a4_sparse_pair_kernel, kThreads, kPSSmemTotal);
-        const int grid_pairs = tiles < npairs ? tiles : npairs;
-        return launch_pdl(w4a4_sparse_pair_kernel, dim3(2 * grid_pairs), dim3(kThreads), kPSSmemTotal, stream, mw, mx,
-                          me, my, pp);
+        return K <= kResidentMaxK ? launch_sparse_pair<true>(mw, mx, me, my, pp, stream)
+                                  : launch_sparse_pair<false>(mw, mx, me, my, pp, stream);
     }
     SparseParams p;
     p.sx = sx; p.sw = sw; p.acc = acc;

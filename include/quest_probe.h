@@ -6,7 +6,7 @@
  * The pages define no such operation: the entry points below exist only so a
  * benchmark can measure the int8 and FP4 MMA rates of the part it runs on, the
  * denominators of the linear layers' tensor-core fractions besides the nominal
- * dense figures.
+ * dense figures (and the 2:4-sparse rate of the sparse layer).
  */
 #ifndef QUEST_B200_PROBE_H
 #define QUEST_B200_PROBE_H
@@ -33,6 +33,17 @@ quest_status quest_probe_mma_i8(int iters, int* ctas, void* stream);
  * memory, unit UE8M0 block scales in TMEM, fp32 accumulator); the caller
  * computes 2 * 128 * 256 * 64 * iters * ctas / seconds. Errors as above. */
 quest_status quest_probe_mma_fp4(int iters, int* ctas, void* stream);
+
+/* The same for the 2:4-sparse integer kind of the sparse linear layer:
+ * back-to-back tcgen05.mma.sp kind::i8 (M = 128, N = 256, K = 64 logical
+ * values, 32 bytes of compressed A per row, metadata in TMEM). With
+ * cp_every = c > 0 a tcgen05.cp of four metadata columns from shared memory
+ * precedes every c-th MMA, whose group of c MMAs then reads the copied columns;
+ * cp_every = 0 keeps the metadata resident. The caller computes the
+ * dense-equivalent rate 2 * 128 * 256 * 64 * iters * ctas / seconds.
+ * Errors: QUEST_EINVAL if iters is outside [1, 2^20], cp_every outside
+ * [0, 64] or ctas is NULL; QUEST_ECUDA on a launch error. */
+quest_status quest_probe_mma_sp_i8(int iters, int cp_every, int* ctas, void* stream);
 
 /* Synchronise `stream`; QUEST_ETIMEOUT if a probe's bounded completion wait
  * (2 s) gave up since the last call (the flag is then cleared). */

@@ -195,6 +195,11 @@ def test_probe_rejects_invalid_arguments():
         assert fn(0, ctypes.byref(n), None) == 1
         assert fn((1 << 20) + 1, ctypes.byref(n), None) == 1   # cap: far inside the 2 s wait
         assert fn(100, None, None) == 1
+    sp = lib.quest_probe_mma_sp_i8
+    assert sp(0, 0, ctypes.byref(n), None) == 1
+    assert sp((1 << 20) + 1, 2, ctypes.byref(n), None) == 1
+    assert sp(100, -1, ctypes.byref(n), None) == 1 and sp(100, 65, ctypes.byref(n), None) == 1
+    assert sp(100, 2, None, None) == 1
 
 
 def test_trust_bwd_linear_rejects_invalid_arguments():

@@ -173,9 +173,10 @@ def run_sparse_layer(xc, sx, wc, meta, sw):
 
 
 @pytest.mark.parametrize("M,N,K", [(224, 128, 128), (300, 136, 384), (17, 8, 128), (450, 264, 1024),
-                                   (1000, 520, 2048)])
+                                   (1000, 520, 2048), (300, 264, 2304), (600, 520, 4096)])
 def test_sparse_layer_accumulator_exact(cuda_device, M, N, K):
-    # ragged tiles in both directions, several waves, K of one to sixteen stages
+    # ragged tiles in both directions, several waves, K of one to sixteen stages (the
+    # metadata resident in TMEM) and beyond (2304, 4096: the metadata staged per stage)
     g = np.random.default_rng(M + N + K)
     xc = (2 * g.integers(-8, 8, (M, K)) + 1).astype(np.int8)
     wd, kept = random_sparse_codes(N, K, seed=K)
@@ -186,6 +187,24 @@ def test_sparse_layer_accumulator_exact(cuda_device, M, N, K):
     ref = oracle.gemm_i8(xc, wd.astype(np.int8))
     assert np.array_equal(acc, ref)
     check_bf16(y, oracle.dequant_linear(ref, sx.astype(np.float64), sw.astype(np.float64)), what="y")
+
+
+@pytest.mark.parametrize("M,N,K", [(4000, 1288, 640), (3600, 1096, 2048)])
+def test_sparse_layer_weight_tile_changes(cuda_device, M, N, K):
+    # more tiles than CTA pairs: each pair walks a run of tiles in weight-major order
+    # and reloads the resident metadata where the run crosses into the next 256 weight
+    # rows; rows sampled from every token tile, against the exact product
+    g = np.random.default_rng(M + K)
+    xc = (2 * g.integers(-8, 8, (M, K)) + 1).astype(np.int8)
+    wd, kept = random_sparse_codes(N, K, seed=K + 1)
+    wc, meta = compress(wd, kept)
+    sx = g.uniform(0.5, 2.0, M).astype(np.float32)
+    sw = g.uniform(0.5, 2.0, N).astype(np.float32)
+    y, acc = run_sparse_layer(xc, sx, wc, meta, sw)
+    rows = np.unique(np.concatenate([np.arange(0, M, 224), np.arange(223, M, 224), g.integers(0, M, 64), [M - 1]]))
+    ref = oracle.gemm_i8(np.ascontiguousarray(xc[rows]), wd.astype(np.int8))
+    assert np.array_equal(acc[rows], ref)
+    check_bf16(y[rows], oracle.dequant_linear(ref, sx[rows].astype(np.float64), sw.astype(np.float64)), what="y")
 
 
 def test_sparse_layer_extreme_codes(cuda_device):
