@@ -468,7 +468,7 @@ def run_b200(args, world, rank, local):
         print(json.dumps(result), flush=True)
 
 
-def mma_probe(dev, gemm_tops=None, iters=20000, reps=5, fp4=False, sparse=False, cp_every=0):
+def mma_probe(dev, gemm_tops=None, iters=20000, reps=5, fp4=False, sparse=False, cp_every=0, bf16=False):
     """Tensor-core rate with no memory traffic (back-to-back tcgen05.mma, one CTA per
     SM): kind::i8 M 128 N 256 K 32; with fp4 kind::mxf4 M 128 N 256 K 64 with unit
     block scales; with sparse the 2:4-sparse kind::i8 M 128 N 256 K 64 (logical, the
@@ -480,6 +480,8 @@ def mma_probe(dev, gemm_tops=None, iters=20000, reps=5, fp4=False, sparse=False,
     stream = torch.cuda.current_stream(dev)
     if sparse:
         launch = lambda n, st: q.probe_mma_sp_i8(n, cp_every, st)
+    elif bf16:
+        launch = q.probe_mma_bf16
     else:
         launch = q.probe_mma_fp4 if fp4 else q.probe_mma_i8
     launch(iters, stream.cuda_stream)
@@ -493,7 +495,7 @@ def mma_probe(dev, gemm_tops=None, iters=20000, reps=5, fp4=False, sparse=False,
         ts.append(a.elapsed_time(b))
     q.probe_status(stream.cuda_stream)
     ms = statistics.median(ts)
-    tops = 2.0 * 128 * 256 * (64 if (fp4 or sparse) else 32) * iters * ctas / (ms * 1e-3) / 1e12
+    tops = 2.0 * 128 * 256 * (64 if (fp4 or sparse) else 16 if bf16 else 32) * iters * ctas / (ms * 1e-3) / 1e12
     out = {"tops": round(tops, 1), "iters": iters, "ctas": ctas,
            "note": "timed alone right after the bench loop (burst); the GEMM's roofline peak"}
     if gemm_tops is not None:
@@ -951,9 +953,14 @@ def run_configs(args):
     sp_row["frac_sparse_probe"] = probe_sp["gemm_frac_of_probe"]
     probe_sp_cp = mma_probe(dev, None, sparse=True, cp_every=2)
     probe_sp_cp["note"] = "the same with a tcgen05.cp of metadata before every second MMA"
+    probe_bf = mma_probe(dev, None, bf16=True)
+    probe_bf["note"] = "kind::f16 bf16, measured the same way: the denominator for cuBLAS and the f3 kernels"
+    for r in rows:
+        if "tflops" in r:
+            r["frac_bf16_probe"] = round(r["tflops"] / probe_bf["tops"], 4)
     print(json.dumps({"configs": rows, "int8_mma_probe": probe, "fp4_mma_probe": probe4,
-                      "sparse_mma_probe": probe_sp, "sparse_mma_probe_cp2": probe_sp_cp, "peaks": peaks}),
-          flush=True)
+                      "sparse_mma_probe": probe_sp, "sparse_mma_probe_cp2": probe_sp_cp,
+                      "bf16_mma_probe": probe_bf, "peaks": peaks}), flush=True)
 
 
 def run_profile_kernels(args):

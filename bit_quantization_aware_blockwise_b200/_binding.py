@@ -54,6 +54,7 @@ _PROBE_LIB_NAME = "libquest_probe.so"
 PROBE_SIGNATURES = {
     "quest_probe_mma_i8": (_int, [_int, _p, _p]),
     "quest_probe_mma_fp4": (_int, [_int, _p, _p]),
+    "quest_probe_mma_bf16": (_int, [_int, _p, _p]),
     "quest_probe_mma_sp_i8": (_int, [_int, _int, _p, _p]),
     "quest_probe_status": (_int, [_p]),
 }
@@ -524,6 +525,13 @@ def probe_mma_fp4(iters, stream=0):
     """Enqueue the FP4 (kind::mxf4) tensor-core peak probe; returns the number of CTAs launched."""
     ctas = ctypes.c_int(0)
     _check_probe(load_probe_library().quest_probe_mma_fp4(iters, ctypes.byref(ctas), stream), "quest_probe_mma_fp4")
+    return ctas.value
+
+
+def probe_mma_bf16(iters, stream=0):
+    """Enqueue the bf16 (kind::f16) tensor-core probe; returns the number of CTAs launched."""
+    ctas = ctypes.c_int(0)
+    _check_probe(load_probe_library().quest_probe_mma_bf16(iters, ctypes.byref(ctas), stream), "quest_probe_mma_bf16")
     return ctas.value
 
 

@@ -4,6 +4,8 @@
 // The caller times a launch; 2 * 128 * 256 * 32 * iters * SMs / time is the
 // int8 MMA rate this part sustains at its current clocks, the denominator the
 // GEMM's tensor-core fraction can be read against besides the nominal figure.
+// The same kernel with kind::f16 (bf16 operands, K = 16) gives the bf16 rate
+// measured the same way, against which a library bf16 GEMM can be read.
 //
 // Built into its own library (libquest_probe.so) for the benchmark: it is a
 // measurement aid, not part of the QuEST path, so the product library does not
@@ -50,7 +52,13 @@ __device__ __forceinline__ uint64_t probe_desc(uint32_t addr) {
     return d;
 }
 
-__global__ void __launch_bounds__(kProbeThreads, 1) probe_mma_i8_kernel(int iters) {
+// kind::f16 with bf16 A and B, fp32 accumulator (M = 128, N = 256, K = 16: the
+// same 32 bytes per operand row as the int8 instruction), for the bf16 layers.
+constexpr uint32_t kIdescProbeBf16 = (1u << 4) | (1u << 7) | (1u << 10) | (uint32_t(256 >> 3) << 17) |
+                                     (uint32_t(128 >> 4) << 24);
+
+template <bool kBf16>
+__global__ void __launch_bounds__(kProbeThreads, 1) probe_mma_dense_kernel(int iters) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const uint32_t sbase = static_cast<uint32_t>(__cvta_generic_to_shared(smem));
@@ -76,12 +84,20 @@ __global__ void __launch_bounds__(kProbeThreads, 1) probe_mma_i8_kernel(int iter
     if (threadIdx.x == 0) {
         const uint64_t a = probe_desc(sbase + kA), b = probe_desc(sbase + kB);
         for (int i = 0; i < iters; ++i) {
-            asm volatile(
-                "{\n\t.reg .pred p;\n\t"
-                "setp.ne.b32 p, %4, 0;\n\t"
-                "tcgen05.mma.cta_group::1.kind::i8 [%0], %1, %2, %3, p;\n\t}" ::"r"(tmem),
-                "l"(a), "l"(b), "r"(kIdescProbe), "r"(i)
-                : "memory");
+            if (kBf16)
+                asm volatile(
+                    "{\n\t.reg .pred p;\n\t"
+                    "setp.ne.b32 p, %4, 0;\n\t"
+                    "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(tmem),
+                    "l"(a), "l"(b), "r"(kIdescProbeBf16), "r"(i)
+                    : "memory");
+            else
+                asm volatile(
+                    "{\n\t.reg .pred p;\n\t"
+                    "setp.ne.b32 p, %4, 0;\n\t"
+                    "tcgen05.mma.cta_group::1.kind::i8 [%0], %1, %2, %3, p;\n\t}" ::"r"(tmem),
+                    "l"(a), "l"(b), "r"(kIdescProbe), "r"(i)
+                    : "memory");
         }
         asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
                      : "memory");
@@ -322,21 +338,36 @@ extern "C" quest_status quest_probe_mma_fp4(int iters, int* ctas, void* stream) 
     return cudaGetLastError() == cudaSuccess ? QUEST_OK : QUEST_ECUDA;
 }
 
-extern "C" quest_status quest_probe_mma_i8(int iters, int* ctas, void* stream) {
-    using namespace quest;
+namespace quest {
+namespace {
+
+template <bool kBf16>
+quest_status launch_probe_dense(int iters, int* ctas, void* stream) {
     if (iters < 1 || iters > kMaxIters || ctas == nullptr) return QUEST_EINVAL;
     static thread_local int attr_dev = -1;
     int dev = 0;
     cudaGetDevice(&dev);
     if (attr_dev != dev) {
-        if (cudaFuncSetAttribute(probe_mma_i8_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        if (cudaFuncSetAttribute(probe_mma_dense_kernel<kBf16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  kProbeSmem + 1024) != cudaSuccess)
             return QUEST_ECUDA;
         attr_dev = dev;
     }
     *ctas = probe_sm_count();
-    probe_mma_i8_kernel<<<*ctas, kProbeThreads, kProbeSmem + 1024, static_cast<cudaStream_t>(stream)>>>(iters);
+    probe_mma_dense_kernel<kBf16>
+        <<<*ctas, kProbeThreads, kProbeSmem + 1024, static_cast<cudaStream_t>(stream)>>>(iters);
     return cudaGetLastError() == cudaSuccess ? QUEST_OK : QUEST_ECUDA;
+}
+
+}  // namespace
+}  // namespace quest
+
+extern "C" quest_status quest_probe_mma_i8(int iters, int* ctas, void* stream) {
+    return quest::launch_probe_dense<false>(iters, ctas, stream);
+}
+
+extern "C" quest_status quest_probe_mma_bf16(int iters, int* ctas, void* stream) {
+    return quest::launch_probe_dense<true>(iters, ctas, stream);
 }
 
 extern "C" quest_status quest_probe_status(void* stream) {

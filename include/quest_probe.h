@@ -28,6 +28,11 @@ extern "C" {
  * QUEST_ECUDA on a launch error. */
 quest_status quest_probe_mma_i8(int iters, int* ctas, void* stream);
 
+/* The same for bf16: back-to-back tcgen05.mma kind::f16 (M = 128, N = 256,
+ * K = 16, bf16 operands, fp32 accumulator); the caller computes
+ * 2 * 128 * 256 * 16 * iters * ctas / seconds. Errors as above. */
+quest_status quest_probe_mma_bf16(int iters, int* ctas, void* stream);
+
 /* The same for the block-scaled FP4 kind of the FP4 linear layer: back-to-back
  * tcgen05.mma kind::mxf4 (M = 128, N = 256, K = 64, E2M1 operands in shared
  * memory, unit UE8M0 block scales in TMEM, fp32 accumulator); the caller
