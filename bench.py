@@ -149,6 +149,16 @@ class ClockSampler:
                 pass
             time.sleep(self.period)
 
+    def sample_now(self):
+        """One synchronous sample from the calling thread (the sampling thread can be
+        starved while the launching thread holds the interpreter)."""
+        if self.ok:
+            try:
+                self.samples.append((self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM),
+                                     self.nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)))
+            except Exception:
+                pass
+
     def start(self):
         if self.ok:
             self._thr = threading.Thread(target=self._run, daemon=True)
@@ -350,11 +360,14 @@ def run_b200(args, world, rank, local):
     torch.cuda.synchronize()
     clocks.start()
     t0 = time.perf_counter()
+    every = max(1, args.steps // 8)
     for k in range(args.steps):
         flush.zero_()  # L2 flush between timed steps (outside the per-step events)
         span[k][0].record(stream)
         one_step()
         span[k][1].record(stream)
+        if k % every == every - 1:
+            clocks.sample_now()   # the queue ahead of the GPU holds this and earlier steps
     torch.cuda.synchronize()
     wall = time.perf_counter() - t0
     clocks.stop()
@@ -1009,7 +1022,7 @@ def run_profile_kernels(args):
 def main():
     ap = argparse.ArgumentParser(description=__doc__)
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--steps", type=int, default=1000)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["b200", "reference"], default="b200")
     ap.add_argument("--no-e2e", action="store_true")
