@@ -56,9 +56,13 @@ constexpr uint32_t kSTx = kSStageA + kSStageB + kSStageE;
 constexpr uint32_t kSSmemA = 0;
 constexpr uint32_t kSSmemB = kSSmemA + kSStages * kSStageA;
 constexpr uint32_t kSSmemE = kSSmemB + kSStages * kSStageB;
-constexpr uint32_t kSCBytes = 32 * SBM * 2;         // transposed stage: 32 tokens x 128 weight rows, bf16
+// Transposed output stage: every epilogue warp owns kStgBufs buffers of 32 tokens x its 32
+// weight rows (bf16, 2 KB), each written back by the warp's own TMA store.
+constexpr int kStgBufs = 4;
+constexpr uint32_t kStgBytes = 32 * 32 * 2;
+constexpr uint32_t kSCBytes = 4 * kStgBufs * kStgBytes;   // 32 KB per CTA
 constexpr uint32_t kSSmemC = kSSmemE + kSStages * kSStageE;
-constexpr uint32_t kSSmemScale = kSSmemC + 2 * kSCBytes;   // float[SBN]: the tokens' scales
+constexpr uint32_t kSSmemScale = kSSmemC + kSCBytes;       // float[SBN]: the tokens' scales
 static_assert(kSSmemScale % 16 == 0, "16-byte scale loads");
 constexpr uint32_t kSSmemBar = kSSmemScale + SBN * 4;
 constexpr uint32_t kSNumBars = 2 * kSStages + 4 + 1;
@@ -113,8 +117,8 @@ __device__ __forceinline__ void tc_cp_meta(uint32_t taddr, uint64_t sdesc) {
 }
 
 // One 32-token chunk of a weight row (TMEM lane): scale, round to bf16 and store
-// the 32 values down the transposed stage (token i of the chunk at row i, this
-// weight row at its column). The chunk's token scales are read into registers
+// the 32 values down the warp's transposed stage (token i of the chunk at row i,
+// this weight row at column lane). The chunk's token scales are read into registers
 // (as float4) before any store: the 16-bit stores and the scale loads both go
 // to shared memory, and interleaved the compiler has to keep every store ahead
 // of the next load, which chained the 32 conversions one after another.
@@ -133,7 +137,47 @@ __device__ __forceinline__ void stage_chunk_transposed(const uint32_t (&r)[32], 
 #pragma unroll
     for (int i = 0; i < 32; ++i) h[i] = __bfloat16_as_ushort(__float2bfloat16_rn((float)(int32_t)r[i] * sw_half * s[i]));
 #pragma unroll
-    for (int i = 0; i < 32; ++i) stg[i * SBM] = h[i];
+    for (int i = 0; i < 32; ++i) stg[i * 32] = h[i];
+}
+
+__device__ __forceinline__ void bulk_wait_read_stg() {
+    asm volatile("cp.async.bulk.wait_group.read %0;" ::"n"(kStgBufs - 1) : "memory");
+}
+
+// This warp's 32 weight rows x SBN tokens of a finished accumulator out to y[m][n]:
+// per 32-token chunk one TMEM load, the scaled bf16 values down a staging buffer of the
+// warp's own, and one TMA store of that 32 x 32 box (no barrier with the other warps;
+// the buffer is reused once at most kStgBufs - 1 of the warp's stores are still reading).
+// n_w: the warp's first weight row; n = n_w + lane. Lane 0 issues and tracks the stores.
+__device__ __forceinline__ void store_tile_transposed(const CUtensorMap& map_y, uint32_t t_acc, uint8_t* stg,
+                                                      uint32_t stg_addr, int& cbuf, int lane, int n_w, int m0,
+                                                      float sw_half, const float* s_scale, int32_t* acc, int M,
+                                                      int N) {
+    const int n = n_w + lane;
+#pragma unroll 1
+    for (int c = 0; c < SBN / 32; ++c) {
+        uint32_t r[32];
+        QUEST_TMEM_LD32(t_acc + c * 32, r);
+        tmem_wait_ld();
+        if (lane == 0) bulk_wait_read_stg();
+        __syncwarp();
+        stage_chunk_transposed(r, sw_half, s_scale + c * 32,
+                               reinterpret_cast<uint16_t*>(stg + cbuf * kStgBytes) + lane);
+        if (acc != nullptr && n < N) {
+#pragma unroll
+            for (int i = 0; i < 32; ++i) {
+                const int m = m0 + c * 32 + i;
+                if (m < M) acc[int64_t(m) * N + n] = (int32_t)r[i];
+            }
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+            tma_store_2d(&map_y, stg_addr + cbuf * kStgBytes, n_w, m0 + c * 32);
+            bulk_commit();
+        }
+        cbuf = cbuf + 1 == kStgBufs ? 0 : cbuf + 1;
+    }
 }
 
 struct SparseParams {
@@ -264,6 +308,8 @@ w4a4_sparse_kernel(const __grid_constant__ CUtensorMap map_w, const __grid_const
         const int quarter = warp & 3;                 // TMEM lanes 32*quarter .. +31
         const int row = quarter * 32 + lane;          // weight row within the tile = TMEM lane
         const uint32_t lane_addr = uint32_t(quarter * 32) << 16;
+        uint8_t* stg_w = smem + kSSmemC + (warp - 2) * kStgBufs * kStgBytes;
+        const uint32_t stg_w_addr = sbase + kSSmemC + (warp - 2) * kStgBufs * kStgBytes;
         int local = 0, cbuf = 0;
         for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++local) {
             const int n0 = (tile % p.num_n) * SBM, m0 = (tile / p.num_n) * SBN;
@@ -279,35 +325,12 @@ w4a4_sparse_kernel(const __grid_constant__ CUtensorMap map_w, const __grid_const
             if (epi_any(!got)) break;   // also orders the token scales above (bar.red)
             tc_fence_after();
             const uint32_t t_acc = tmem_base + lane_addr + buf * kSAccCols;
-#pragma unroll 1
-            for (int c = 0; c < SBN / 32; ++c) {
-                uint32_t r[32];
-                QUEST_TMEM_LD32(t_acc + c * 32, r);
-                tmem_wait_ld();
-                // transposed stage: token i of the chunk is row i, this weight row its column
-                stage_chunk_transposed(r, sw_half, s_scale + c * 32,
-                                       reinterpret_cast<uint16_t*>(smem + kSSmemC + cbuf * kSCBytes) + row);
-                if (p.acc != nullptr && n < p.N) {
-#pragma unroll
-                    for (int i = 0; i < 32; ++i) {
-                        const int m = m0 + c * 32 + i;
-                        if (m < p.M) p.acc[int64_t(m) * p.N + n] = (int32_t)r[i];
-                    }
-                }
-                fence_proxy_async_smem();
-                epi_bar();
-                if (et == 0) {
-                    tma_store_2d(&map_y, sbase + kSSmemC + cbuf * kSCBytes, n0, m0 + c * 32);
-                    bulk_commit();
-                    bulk_wait_read_le1();   // the other staging buffer is free again
-                }
-                epi_bar();
-                cbuf ^= 1;
-            }
+            store_tile_transposed(map_y, t_acc, stg_w, stg_w_addr, cbuf, lane, n0 + 32 * quarter, m0, sw_half,
+                                  s_scale, p.acc, p.M, p.N);
             tc_fence_before();
             mbar_arrive(bar_tempty + 8 * buf);
         }
-        if (et == 0) bulk_wait_all();
+        if (lane == 0) bulk_wait_all();
     }
 
     tc_fence_before();
@@ -357,7 +380,7 @@ struct PairLayout {
     static constexpr uint32_t kE = kB + kPSStages * kPSStageB;     // staged slabs, or the resident block
     static constexpr uint32_t kEBytes = R ? uint32_t(kResidentMaxK / SBK) * kSStageE : kPSStages * kSStageE;
     static constexpr uint32_t kC = kE + kEBytes;
-    static constexpr uint32_t kScale = kC + 2 * kSCBytes;
+    static constexpr uint32_t kScale = kC + kSCBytes;
     static constexpr uint32_t kBar = kScale + SBN * 4;
     static constexpr uint32_t kNumBars = 2 * kPSStages + 4 + 1 + 2;   // + metadata full / empty
     static constexpr uint32_t kTmemSlot = kBar + kNumBars * 8;
@@ -575,6 +598,8 @@ w4a4_sparse_pair_kernel(const __grid_constant__ CUtensorMap map_w, const __grid_
         const int row = quarter * 32 + lane;          // weight row within this CTA's half = TMEM lane
         const uint32_t lane_addr = uint32_t(quarter * 32) << 16;
         const uint32_t tempty_even = map_to_rank(bar_tempty, 0);
+        uint8_t* stg_w = smem + L::kC + (warp - 2) * kStgBufs * kStgBytes;
+        const uint32_t stg_w_addr = sbase + L::kC + (warp - 2) * kStgBufs * kStgBytes;
         int local = 0, cbuf = 0;
         for (int tile = t_begin; tile < t_end; tile += t_step, ++local) {
             const int n0 = tile_n2(tile) * 256 + 128 * int(rank), m0 = tile_mt(tile) * SBN;
@@ -590,35 +615,13 @@ w4a4_sparse_pair_kernel(const __grid_constant__ CUtensorMap map_w, const __grid_
             if (epi_any(!got)) break;   // also orders the token scales above (bar.red)
             tc_fence_after();
             const uint32_t t_acc = tmem_base + lane_addr + buf * kSAccCols;
-#pragma unroll 1
-            for (int c = 0; c < SBN / 32; ++c) {
-                uint32_t r[32];
-                QUEST_TMEM_LD32(t_acc + c * 32, r);
-                tmem_wait_ld();
-                stage_chunk_transposed(r, sw_half, s_scale + c * 32,
-                                       reinterpret_cast<uint16_t*>(smem + L::kC + cbuf * kSCBytes) + row);
-                if (p.acc != nullptr && n < p.N) {
-#pragma unroll
-                    for (int i = 0; i < 32; ++i) {
-                        const int m = m0 + c * 32 + i;
-                        if (m < p.M) p.acc[int64_t(m) * p.N + n] = (int32_t)r[i];
-                    }
-                }
-                fence_proxy_async_smem();
-                epi_bar();
-                if (et == 0) {
-                    tma_store_2d(&map_y, sbase + L::kC + cbuf * kSCBytes, n0, m0 + c * 32);
-                    bulk_commit();
-                    bulk_wait_read_le1();
-                }
-                epi_bar();
-                cbuf ^= 1;
-            }
+            store_tile_transposed(map_y, t_acc, stg_w, stg_w_addr, cbuf, lane, n0 + 32 * quarter, m0, sw_half,
+                                  s_scale, p.acc, p.M, p.N);
             tc_fence_before();
             epi_bar();
             if (et == 0) mbar_arrive_remote(tempty_even + 8 * buf);
         }
-        if (et == 0) bulk_wait_all();
+        if (lane == 0) bulk_wait_all();
     }
 
     tc_fence_before();
@@ -666,7 +669,7 @@ cudaError_t launch_w4a4_sparse24(const int8_t* X, const float* sx, const int8_t*
                      CU_TENSOR_MAP_SWIZZLE_128B) ||
         !make_map_2d(&me, CU_TENSOR_MAP_DATA_TYPE_UINT8, E, K / 8, N, K / 8, SBK / 8, SBM,
                      CU_TENSOR_MAP_SWIZZLE_NONE) ||
-        !make_map_2d(&my, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, y, N, M, N * 2, SBM, 32, CU_TENSOR_MAP_SWIZZLE_NONE))
+        !make_map_2d(&my, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, y, N, M, N * 2, 32, 32, CU_TENSOR_MAP_SWIZZLE_NONE))
         return cudaErrorInvalidValue;
     if (pairs) {
         SparsePairParams pp;

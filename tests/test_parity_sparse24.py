@@ -207,6 +207,24 @@ def test_sparse_layer_weight_tile_changes(cuda_device, M, N, K):
     check_bf16(y[rows], oracle.dequant_linear(ref, sx[rows].astype(np.float64), sw.astype(np.float64)), what="y")
 
 
+def test_sparse_layer_full_shape_sampled(cuda_device):
+    # 16384 x 5632 x 2048, the launch the configs time: seeded b = 4 activation codes and
+    # random 2:4-sparse weight codes; the oracle recomputes a 24 x 24 grid of outputs
+    M, N, K = inputs.TOKENS, inputs.MLP_WIDTH, inputs.HIDDEN
+    xc = inputs.gemm_codes(M, K, seed=41)
+    wd, kept = random_sparse_codes(N, K, seed=42)
+    wc, meta = compress(wd, kept)
+    sx, sw = inputs.positive_scales(M, 43), inputs.positive_scales(N, 44)
+    y, acc = run_sparse_layer(xc, sx, wc, meta, sw)
+    g = np.random.default_rng(45)
+    rows = np.unique(np.concatenate([[0, M - 1], g.choice(M, 22, replace=False)]))
+    cols = np.unique(np.concatenate([[0, N - 1], g.choice(N, 22, replace=False)]))
+    ref = oracle.gemm_i8(np.ascontiguousarray(xc[rows]), np.ascontiguousarray(wd[cols].astype(np.int8)))
+    assert np.array_equal(acc[np.ix_(rows, cols)].astype(np.int64), ref)
+    check_bf16(y[np.ix_(rows, cols)], oracle.dequant_linear(ref, sx[rows].astype(np.float64),
+                                                            sw[cols].astype(np.float64)), what="y (sampled)")
+
+
 def test_sparse_layer_extreme_codes(cuda_device):
     # every survivor +-127 against +-127: |acc| = 127^2 K / 2 at K = 2048 (no overflow)
     M, N, K = 256, 128, 2048
