@@ -60,8 +60,10 @@ __device__ __forceinline__ uint32_t mask_byte_thr(const float2 (&P)[16], int f, 
 }
 
 // Quantise, prune and store this lane's 32 values (chunks c = t + 4f of the slab
-// whose first element is e_slab in row `row`).
-template <bool SAT>
+// whose first element is e_slab in row `row`). OUT = 0 reads the optional outputs
+// (mask, dequant) from the arguments; OUT = 1 writes codes and metadata only, the
+// set the sparse layer consumes, with the optional paths compiled out.
+template <bool SAT, int OUT>
 __device__ __forceinline__ void emit_sparse(const SparseArgs& S, const float2 (&P)[16], const GroupK& G,
                                             int64_t row, int64_t e_slab, int t, bool valid) {
     const QuantArgs& A = S.q;
@@ -69,7 +71,7 @@ __device__ __forceinline__ void emit_sparse(const SparseArgs& S, const float2 (&
     uint8_t* codes = A.codes + row * A.codes_row_bytes + e_slab / 2;
     const int coff = 1 - (1 << S.bits);   // c = 2 q_b + 1 - 2^b
     const float thr2p = G.thr2 * S.prune_ratio;
-    const bool do_mask = k.mask_mode >= 0, do_deq = valid && k.deq_mode >= 0;
+    const bool do_mask = OUT == 0 && k.mask_mode >= 0, do_deq = OUT == 0 && valid && k.deq_mode >= 0;
     uint32_t mbytes = 0, metab = 0;
 #pragma unroll
     for (int f = 0; f < 4; ++f) {
@@ -135,7 +137,7 @@ __device__ __forceinline__ float lane_sum_sq(const float2 (&P)[16]) {
 }
 
 // One RMS per 128-value slab (Hadamard block 128): a warp step covers 8 slabs.
-template <bool SAT>
+template <bool SAT, int OUT>
 __global__ void __launch_bounds__(kThreads) quantize_sparse_groups(const SparseArgs S) {
     pdl_wait();
     pdl_trigger();
@@ -165,7 +167,7 @@ __global__ void __launch_bounds__(kThreads) quantize_sparse_groups(const SparseA
         const GroupK G = make_group(A.c, v);
         const bool valid = slab < total;
         const int64_t row = valid ? slab / spr : 0, e_slab = (slab - row * spr) * 128;
-        emit_sparse<SAT>(S, P, G, row, e_slab, t, valid);
+        emit_sparse<SAT, OUT>(S, P, G, row, e_slab, t, valid);
         if (valid && t == 0) A.scales[slab] = G.delta;
     }
 }
@@ -173,8 +175,10 @@ __global__ void __launch_bounds__(kThreads) quantize_sparse_groups(const SparseA
 // One RMS per row of spr = cols / 128 slabs (spr in 1, 2, 4, 8, 16). SUB slabs per
 // lane group (spr / 8 when spr >= 8: a warp holds a row); for spr < 8 a warp step
 // covers 8 / spr rows.
-template <bool SAT, int SUB>
-__global__ void __launch_bounds__(kThreads, 3) quantize_sparse_rows(const SparseArgs S, int spr) {
+// Four CTAs per SM for the codes-and-metadata set (124 registers at SUB = 2, no spill);
+// three with the optional outputs.
+template <bool SAT, int SUB, int OUT>
+__global__ void __launch_bounds__(kThreads, OUT == 1 ? 4 : 3) quantize_sparse_rows(const SparseArgs S, int spr) {
     pdl_wait();
     pdl_trigger();
     const QuantArgs& A = S.q;
@@ -212,13 +216,14 @@ __global__ void __launch_bounds__(kThreads, 3) quantize_sparse_rows(const Sparse
         for (int sh = 4; sh < 4 * gspan; sh <<= 1) v += __shfl_xor_sync(0xFFFFFFFFu, v, sh);
         const GroupK G = make_group(A.c, v);
 #pragma unroll
-        for (int u = 0; u < SUB; ++u) emit_sparse<SAT>(S, P[u], G, valid ? row : 0, int64_t(sc0 + 8 * u) * 128, t, valid);
+        for (int u = 0; u < SUB; ++u)
+            emit_sparse<SAT, OUT>(S, P[u], G, valid ? row : 0, int64_t(sc0 + 8 * u) * 128, t, valid);
         if (valid && sc0 == 0 && t == 0) A.scales[row] = G.delta;
     }
 }
 
-template <bool SAT>
-cudaError_t launch_sat(const SparseArgs& s, bool row_mode, cudaStream_t stream) {
+template <bool SAT, int OUT>
+cudaError_t launch_out(const SparseArgs& s, bool row_mode, cudaStream_t stream) {
     const QuantArgs& a = s.q;
     const int sms = sm_count();
     if (row_mode) {
@@ -229,12 +234,12 @@ cudaError_t launch_sat(const SparseArgs& s, bool row_mode, cudaStream_t stream) 
             const int64_t want = (warps + kThreads / 32 - 1) / (kThreads / 32);
             return launch_pdl(fn, dim3((unsigned)(want < cap ? want : cap)), dim3(kThreads), 0, stream, s, spr);
         };
-        if (spr == 16) return go(quantize_sparse_rows<SAT, 2>, 1);
-        if (spr == 8) return go(quantize_sparse_rows<SAT, 1>, 1);
-        return go(quantize_sparse_rows<SAT, 1>, 8 / spr);
+        if (spr == 16) return go(quantize_sparse_rows<SAT, 2, OUT>, 1);
+        if (spr == 8) return go(quantize_sparse_rows<SAT, 1, OUT>, 1);
+        return go(quantize_sparse_rows<SAT, 1, OUT>, 8 / spr);
     }
     const int64_t warps = (a.rows * (a.cols / 128) + 7) / 8;
-    auto fn = quantize_sparse_groups<SAT>;
+    auto fn = quantize_sparse_groups<SAT, OUT>;
     const int64_t cap = int64_t(sms) * max_ctas_per_sm((const void*)fn, kThreads, 0);
     const int64_t want = (warps + kThreads / 32 - 1) / (kThreads / 32);
     return launch_pdl(fn, dim3((unsigned)(want < cap ? want : cap)), dim3(kThreads), 0, stream, s);
@@ -243,7 +248,11 @@ cudaError_t launch_sat(const SparseArgs& s, bool row_mode, cudaStream_t stream) 
 }  // namespace sp
 
 cudaError_t launch_quantize_sparse24(const SparseArgs& s, bool row_mode, cudaStream_t stream) {
-    return s.bits <= 6 ? sp::launch_sat<true>(s, row_mode, stream) : sp::launch_sat<false>(s, row_mode, stream);
+    // codes and metadata only (no mask, no dequant): the output set compiled in
+    const bool lean = s.q.c.mask_mode < 0 && s.q.c.deq_mode < 0;
+    if (s.bits <= 6)
+        return lean ? sp::launch_out<true, 1>(s, row_mode, stream) : sp::launch_out<true, 0>(s, row_mode, stream);
+    return lean ? sp::launch_out<false, 1>(s, row_mode, stream) : sp::launch_out<false, 0>(s, row_mode, stream);
 }
 
 }  // namespace quest

@@ -109,6 +109,25 @@ def test_row_rms_all_slab_counts(cuda_device, spr):
     check_sparse(run(x, 4, rms_group=cols), o, 45, cols)
 
 
+@pytest.mark.parametrize("rms", ["group", 1, 2, 4, 8, 16])
+def test_codes_and_metadata_only(cuda_device, rms):
+    # without mask and dequant the kernels run with the optional outputs compiled out;
+    # codes, metadata and scales must match the oracle and, bit for bit, the run that
+    # writes every output
+    cols = 768 if rms == "group" else 128 * rms
+    rg = 128 if rms == "group" else cols
+    x = inputs.activations(45, cols, seed=50 + cols)
+    o = oracle.quantize_sparse24(inputs.to_f64(x), bits=4, had=128, rms_group=rg)
+    lean = q.quantize_sparse24(x.cuda(), 4, rms_group=rg, mask=False, dequant=False)
+    full = q.quantize_sparse24(x.cuda(), 4, rms_group=rg, mask=True, dequant=True)
+    torch.cuda.synchronize()
+    assert lean["mask"] is None and lean["dequant"] is None
+    for k in ("codes", "meta", "scales"):
+        assert torch.equal(lean[k], full[k]), k
+    check_sparse({"codes": lean["codes"].cpu().numpy(), "meta": lean["meta"].cpu().numpy(),
+                  "scales": lean["scales"].cpu().numpy()}, o, 45, cols)
+
+
 def test_activation_slice_full_width(cuda_device):
     # 512 rows of the 16384 x 2048 activation workload
     x = inputs.activations(512, 2048, seed=1)
