@@ -21,12 +21,15 @@
 // Each stage is two sparse MMAs (M = 128, N = 224, K = 64 logical); MMA j reads
 // its metadata from columns 2j, 2j+1 of the stage's slot.
 //
-// Structure (one persistent CTA per SM, 192 threads): warp 0 TMA producer, warp 1
-// TMEM allocator, metadata copies and MMA issuer, warps 2-5 epilogue. Two
-// 224-column accumulators alternate (the epilogue of tile i overlaps the mainloop
-// of tile i + 1); the metadata slots sit after them. No cluster, no multicast.
-// Every wait is bounded in time; on timeout the CTA records QUEST_ETIMEOUT,
-// drains its copies and MMAs, frees TMEM and returns.
+// Two kernels. With at most 128 weight rows (N <= 128), one persistent CTA per SM
+// (192 threads: warp 0 TMA producer, warp 1 TMEM allocator, metadata copies and
+// MMA issuer, warps 2-5 epilogue), the structure above. Otherwise CTA pairs
+// (cluster of two, cta_group::2, M = 256 weight rows per MMA; see below). In both,
+// two 224-column accumulators alternate (the epilogue of tile i overlaps the
+// mainloop of tile i + 1) and the metadata columns sit after them; each epilogue
+// warp stores its own 32 weight rows through staging buffers of its own. No TMA
+// multicast. Every wait is bounded in time; on timeout the CTA records
+// QUEST_ETIMEOUT, drains its copies and MMAs, frees TMEM and returns.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
