@@ -17,14 +17,17 @@
 // (2^0 in UE8M0) in every lane is written once per CTA, and every MMA points its
 // A and B scale operands into it, so no scale ever leaves the chip.
 //
-// Structure: CTA pairs (cluster of 2, cta_group::2), M = 256 x N = 224 pair
-// tiles; per CTA a 6-stage ring of A [128 x 128 B] and B [112 x 128 B] tiles
+// Structure: CTA pairs (cluster of 2, cta_group::2), M = 256 x N = 240 pair
+// tiles; per CTA a 6-stage ring of A [128 x 128 B] and B [120 x 128 B] tiles
 // (256 FP4 values per row per stage); four tcgen05.mma (K = 64 each) per stage;
-// two 224-column fp32 accumulators (TMEM columns 0 and 256) alternate so the
+// two 240-column fp32 accumulators (TMEM columns 0 and 240) alternate so the
 // epilogue of one tile overlaps the mainloop of the next; TMEM columns 480-511
-// hold the scale bytes. Epilogue: eight warps, two per TMEM lane quarter, each
-// taking half of the tile's columns of its 32 accumulator rows, 32 columns at a
-// time: scale, round to bf16, store through its own 64-byte-swizzled staging
+// hold the scale bytes. N = 240 is the widest tile two accumulators and the
+// scale columns leave room for, and it divides N = 5632 into 23.5 tiles (224
+// gave 25.1, so every pair ran a mostly empty 26th column of tiles). Epilogue:
+// eight warps, two per TMEM lane quarter, each taking half of the tile's columns
+// of its 32 accumulator rows, 32 columns at a time (the last 16 with a
+// 16-column load and store): scale, round to bf16, store through its own staging
 // buffers and TMA stores (warp-level syncs only). At the FP4 rate a tile's
 // mainloop is short (about 3.8K cycles), and with one warp per lane quarter the
 // epilogue did not fit in it (16384 x 5632 x 2048: 94.7 us, against 75.8 us with
@@ -49,14 +52,15 @@ __device__ int g_tc_status = 0;
 namespace quest {
 namespace {
 
-constexpr int kFBN = 224;                                   // output columns per pair tile
+constexpr int kFBN = 240;                                   // output columns per pair tile
 constexpr int kFThreads = 320;                              // producer, MMA, 8 epilogue warps
 constexpr int kFEpiThreads = 256;
-constexpr int kFChunks = kFBN / kChunkCols;                 // 7 column chunks: warps of half 0 take 4, half 1 take 3
-constexpr int kFHalfChunks = (kFChunks + 1) / 2;
+constexpr int kFChunks = kFBN / kChunkCols;                 // 7 whole 32-column chunks and a 16-column tail
+constexpr int kFTailCols = kFBN - kFChunks * kChunkCols;    // 16
+constexpr int kFHalfChunks = 4;                             // half 0: chunks 0-3; half 1: 4-6 and the tail
 constexpr int kFStages = 6;
 constexpr uint32_t kFStageA = 128 * BK;                     // 128 rows x 128 bytes (256 FP4 values)
-constexpr uint32_t kFStageB = (kFBN / 2) * BK;              // 112 rows x 128 bytes
+constexpr uint32_t kFStageB = (kFBN / 2) * BK;              // 120 rows x 128 bytes
 constexpr uint32_t kFTxBytes = 2 * (kFStageA + kFStageB);   // both CTAs land on the even CTA's barrier
 constexpr uint32_t kFSmemA = 0;
 constexpr uint32_t kFSmemB = kFSmemA + kFStages * kFStageA;
@@ -71,12 +75,13 @@ constexpr uint32_t kFSmemUsed = kFSmemAbort + 4;
 constexpr uint32_t kFSmemTotal = kFSmemUsed + 1024;
 static_assert(kFStageB % 1024 == 0, "128-byte-swizzled stages start on 1 KB boundaries");
 static_assert(kFSmemTotal <= 227 * 1024, "FP4 pair kernel shared memory");
-constexpr uint32_t kFAccStride = 256;                       // accumulator buffers at TMEM columns 0 and 256
+constexpr uint32_t kFAccStride = kFBN;                      // accumulator buffers at TMEM columns 0 and 240
 constexpr uint32_t kFScaleCol = 480;                        // 32 columns of 0x7F bytes: A scales at 480, B at 496
 static_assert(kFAccStride + kFBN <= kFScaleCol && kFScaleCol + 32 <= kTmemCols, "TMEM columns");
+static_assert(kFTailCols == 16, "one 16-column tail chunk");
 
 // Block-scaled instruction descriptor: A and B E2M1 (format 1 of the FP4 kind),
-// K-major, N = 224, UE8M0 scales (bit 23), M = 256, scale-factor ids 0, K = 64.
+// K-major, N = 240, UE8M0 scales (bit 23), M = 256, scale-factor ids 0, K = 64.
 constexpr uint32_t kIdescFp4 = (1u << 7) | (1u << 10) | (uint32_t(kFBN >> 3) << 17) | (1u << 23) |
                                (uint32_t(256 >> 4) << 24);
 
@@ -122,12 +127,13 @@ struct Fp4Params {
     const float* sb;    // [N]
     float* acc;         // optional fp32 [M, N] copy of the accumulator
     int M, N, K;
-    int num_m2, num_n, num_k;   // 256-row pair tiles, 224-column tiles, 256-value K steps
+    int num_m2, num_n, num_k;   // 256-row pair tiles, 240-column tiles, 256-value K steps
 };
 
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kFThreads, 1)
 fp4_gemm_pair_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_b,
-                     const __grid_constant__ CUtensorMap map_y, const Fp4Params p) {
+                     const __grid_constant__ CUtensorMap map_y, const __grid_constant__ CUtensorMap map_y16,
+                     const Fp4Params p) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const uint32_t sbase = smem_u32(smem);
@@ -161,6 +167,7 @@ fp4_gemm_pair_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_con
         asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&map_a)) : "memory");
         asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&map_b)) : "memory");
         asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&map_y)) : "memory");
+        asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&map_y16)) : "memory");
     }
     if (warp == 1) {
         asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
@@ -258,7 +265,7 @@ fp4_gemm_pair_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_con
         const int et = threadIdx.x - 64;             // 0..255
         const int quarter = warp & 3;                // TMEM lanes 32*quarter .. +31
         const int half = (warp - 2) >> 2;            // column chunks [0, 4) or [4, 7)
-        const int c_lo = half * kFHalfChunks, c_hi = half ? kFChunks : kFHalfChunks;
+        const int c_lo = half * kFHalfChunks, c_hi = half ? kFChunks + 1 : kFHalfChunks;   // chunk 7: the tail
         const int row_in_tile = quarter * 32 + lane;
         const uint32_t lane_addr = uint32_t(quarter * 32) << 16;
         const uint32_t tempty_even = map_to_rank(bar_tempty, 0);
@@ -285,7 +292,12 @@ fp4_gemm_pair_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_con
 #pragma unroll 1
             for (int c = c_lo; c < c_hi; ++c) {
                 uint32_t r[32];
-                QUEST_TMEM_LD32(t_acc + c * kChunkCols, r);
+                if (c == kFChunks) {
+                    // the last 16 columns: a 16-column load (nothing past the tile is read)
+                    QUEST_TMEM_LD16(t_acc + c * kChunkCols, r);
+                } else {
+                    QUEST_TMEM_LD32(t_acc + c * kChunkCols, r);
+                }
                 tmem_wait_ld();
                 if (c == c_hi - 1) {
                     // this warp's part of the accumulator is read: hand it back to the MMA
@@ -296,6 +308,41 @@ fp4_gemm_pair_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_con
                 const float* sc = s_scale + c * kChunkCols;
                 if (lane == 0) bulk_wait_read_le1();   // the buffer used two chunks ago is free
                 __syncwarp();
+                if (c == kFChunks) {
+                    // tail: 32 rows x 16 bf16, unswizzled, one 16-column TMA box
+                    const uint32_t stg = stg_w + cbuf * kFWarpCBytes + lane * (kFTailCols * 2);
+#pragma unroll
+                    for (int q16 = 0; q16 < 2; ++q16) {
+                        uint32_t w[4];
+#pragma unroll
+                        for (int h = 0; h < 4; ++h) {
+                            const int i = q16 * 8 + h * 2;
+                            const float y0 = __uint_as_float(r[i]) * sa_m * sc[i];
+                            const float y1 = __uint_as_float(r[i + 1]) * sa_m * sc[i + 1];
+                            __nv_bfloat162 hb = __floats2bfloat162_rn(y0, y1);
+                            w[h] = *reinterpret_cast<uint32_t*>(&hb);
+                        }
+                        asm volatile("st.shared.v4.u32 [%0], {%1,%2,%3,%4};" ::"r"(stg + (q16 << 4)), "r"(w[0]),
+                                     "r"(w[1]), "r"(w[2]), "r"(w[3])
+                                     : "memory");
+                    }
+                    if (p.acc != nullptr && m < p.M) {
+                        float* arow = p.acc + int64_t(m) * p.N;
+#pragma unroll
+                        for (int i = 0; i < kFTailCols; ++i) {
+                            const int n = n0 + c * kChunkCols + i;
+                            if (n < p.N) arow[n] = __uint_as_float(r[i]);
+                        }
+                    }
+                    fence_proxy_async_smem();
+                    __syncwarp();
+                    if (lane == 0) {
+                        tma_store_2d(&map_y16, stg_w + cbuf * kFWarpCBytes, n0 + c * kChunkCols, m0 + 32 * quarter);
+                        bulk_commit();
+                    }
+                    cbuf ^= 1;
+                    continue;
+                }
                 const uint32_t stg = stg_w + cbuf * kFWarpCBytes + lane * (kChunkCols * 2);
 #pragma unroll
                 for (int q16 = 0; q16 < 4; ++q16) {
@@ -351,11 +398,13 @@ cudaError_t launch_fp4_linear(const uint8_t* A, const float* sa, const uint8_t* 
         return launch_zero_fill(y, nullptr, M * N, stream);
     }
     const int64_t kb = K / 2;   // bytes per row of packed codes
-    CUtensorMap ma, mb, my;
+    CUtensorMap ma, mb, my, my16;
     if (!make_map_2d(&ma, CU_TENSOR_MAP_DATA_TYPE_UINT8, A, kb, M, kb, BK, 128, CU_TENSOR_MAP_SWIZZLE_128B) ||
         !make_map_2d(&mb, CU_TENSOR_MAP_DATA_TYPE_UINT8, B, kb, N, kb, BK, kFBN / 2, CU_TENSOR_MAP_SWIZZLE_128B) ||
         !make_map_2d(&my, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, y, N, M, N * 2, kChunkCols, 32,
-                     CU_TENSOR_MAP_SWIZZLE_64B))
+                     CU_TENSOR_MAP_SWIZZLE_64B) ||
+        !make_map_2d(&my16, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, y, N, M, N * 2, kFTailCols, 32,
+                     CU_TENSOR_MAP_SWIZZLE_NONE))
         return cudaErrorInvalidValue;
     Fp4Params p;
     p.sa = sa; p.sb = sb; p.acc = acc;
@@ -376,7 +425,7 @@ cudaError_t launch_fp4_linear(const uint8_t* A, const float* sa, const uint8_t* 
     const int pairs = pair_clusters(dev, (const void*)fp4_gemm_pair_kernel, kFThreads, kFSmemTotal);
     const int grid_pairs = tiles < pairs ? tiles : pairs;
     return launch_pdl(fp4_gemm_pair_kernel, dim3(2 * grid_pairs), dim3(kFThreads), kFSmemTotal, stream, ma, mb, my,
-                      p);
+                      my16, p);
 }
 
 int read_and_clear_fp4_status(cudaStream_t stream, cudaError_t* err) {
