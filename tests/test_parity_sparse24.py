@@ -192,10 +192,12 @@ def run_sparse_layer(xc, sx, wc, meta, sw):
 
 
 @pytest.mark.parametrize("M,N,K", [(224, 128, 128), (300, 136, 384), (17, 8, 128), (450, 264, 1024),
-                                   (1000, 520, 2048), (300, 264, 2304), (600, 520, 4096)])
+                                   (1000, 520, 2048), (300, 264, 2304), (600, 520, 4096), (256, 264, 16384),
+                                   (40, 64, 8192)])
 def test_sparse_layer_accumulator_exact(cuda_device, M, N, K):
     # ragged tiles in both directions, several waves, K of one to sixteen stages (the
-    # metadata resident in TMEM) and beyond (2304, 4096: the metadata staged per stage)
+    # metadata resident in TMEM) and beyond (2304 to 16384: the metadata staged per
+    # stage, in the CTA-pair and the one-CTA kernel)
     g = np.random.default_rng(M + N + K)
     xc = (2 * g.integers(-8, 8, (M, K)) + 1).astype(np.int8)
     wd, kept = random_sparse_codes(N, K, seed=K)
