@@ -70,8 +70,8 @@ NOMINAL_INT8_TOPS = 4500.0   # nominal B200 dense int8 tensor-core rate (used on
 NCU_TRAFFIC = {
     "w4a4_linear": {"sources": ["bit_quantization_aware_blockwise_b200/csrc/w4a4_gemm.cu",
                                 "bit_quantization_aware_blockwise_b200/csrc/tc_common.cuh"],
-                    "sha256": "70cb34708642a11377a2708ed66233d7f146d6f4ffa4ff47fda3a213d1b89a28",
-                    "dram_read": 65655296, "dram_write": 146501888},
+                    "sha256": "cfbca22a76b949f761c98afe5bc39339a414144f54c04d83fdd1c0c884f20141",
+                    "dram_read": 64602368, "dram_write": 146513024},
 }
 
 

@@ -317,9 +317,11 @@ fp4_gemm_pair_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_con
 #pragma unroll
                         for (int h = 0; h < 4; ++h) {
                             const int i = q16 * 8 + h * 2;
-                            const float y0 = __uint_as_float(r[i]) * sa_m * sc[i];
-                            const float y1 = __uint_as_float(r[i + 1]) * sa_m * sc[i + 1];
-                            __nv_bfloat162 hb = __floats2bfloat162_rn(y0, y1);
+                            const float2 y = __fmul2_rn(
+                                __fmul2_rn(make_float2(__uint_as_float(r[i]), __uint_as_float(r[i + 1])),
+                                           make_float2(sa_m, sa_m)),
+                                *reinterpret_cast<const float2*>(sc + i));
+                            __nv_bfloat162 hb = __floats2bfloat162_rn(y.x, y.y);
                             w[h] = *reinterpret_cast<uint32_t*>(&hb);
                         }
                         asm volatile("st.shared.v4.u32 [%0], {%1,%2,%3,%4};" ::"r"(stg + (q16 << 4)), "r"(w[0]),
@@ -350,9 +352,11 @@ fp4_gemm_pair_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_con
 #pragma unroll
                     for (int h = 0; h < 4; ++h) {
                         const int i = q16 * 8 + h * 2;
-                        const float y0 = __uint_as_float(r[i]) * sa_m * sc[i];
-                        const float y1 = __uint_as_float(r[i + 1]) * sa_m * sc[i + 1];
-                        __nv_bfloat162 hb = __floats2bfloat162_rn(y0, y1);
+                        const float2 y = __fmul2_rn(
+                            __fmul2_rn(make_float2(__uint_as_float(r[i]), __uint_as_float(r[i + 1])),
+                                       make_float2(sa_m, sa_m)),
+                            *reinterpret_cast<const float2*>(sc + i));
+                        __nv_bfloat162 hb = __floats2bfloat162_rn(y.x, y.y);
                         w[h] = *reinterpret_cast<uint32_t*>(&hb);
                     }
                     asm volatile("st.shared.v4.u32 [%0], {%1,%2,%3,%4};" ::"r"(stg + ((q16 ^ swz) << 4)),

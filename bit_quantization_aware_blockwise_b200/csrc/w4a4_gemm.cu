@@ -232,9 +232,13 @@ w4a4_gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constan
 #pragma unroll
                     for (int h = 0; h < 4; ++h) {
                         const int i = q16 * 8 + h * 2;
-                        const float y0 = (float)(int32_t)r[i] * sa_half * sc[i];
-                        const float y1 = (float)(int32_t)r[i + 1] * sa_half * sc[i + 1];
-                        __nv_bfloat162 hb = __floats2bfloat162_rn(y0, y1);
+                        // (acc * sa/2) * sb/2 per column, two columns per packed multiply
+                        const float2 s01 = *reinterpret_cast<const float2*>(sc + i);
+                        const float2 y = __fmul2_rn(
+                            __fmul2_rn(make_float2((float)(int32_t)r[i], (float)(int32_t)r[i + 1]),
+                                       make_float2(sa_half, sa_half)),
+                            s01);
+                        __nv_bfloat162 hb = __floats2bfloat162_rn(y.x, y.y);
                         w[h] = *reinterpret_cast<uint32_t*>(&hb);
                     }
                     const uint32_t dst = stg + ((q16 ^ swz) << 4);
@@ -469,9 +473,13 @@ w4a4_gemm_pair_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_co
 #pragma unroll
                     for (int h = 0; h < 4; ++h) {
                         const int i = q16 * 8 + h * 2;
-                        const float y0 = (float)(int32_t)r[i] * sa_half * sc[i];
-                        const float y1 = (float)(int32_t)r[i + 1] * sa_half * sc[i + 1];
-                        __nv_bfloat162 hb = __floats2bfloat162_rn(y0, y1);
+                        // (acc * sa/2) * sb/2 per column, two columns per packed multiply
+                        const float2 s01 = *reinterpret_cast<const float2*>(sc + i);
+                        const float2 y = __fmul2_rn(
+                            __fmul2_rn(make_float2((float)(int32_t)r[i], (float)(int32_t)r[i + 1]),
+                                       make_float2(sa_half, sa_half)),
+                            s01);
+                        __nv_bfloat162 hb = __floats2bfloat162_rn(y.x, y.y);
                         w[h] = *reinterpret_cast<uint32_t*>(&hb);
                     }
                     const uint32_t dst = stg + ((q16 ^ swz) << 4);

@@ -138,7 +138,14 @@ __device__ __forceinline__ void stage_chunk_transposed(const uint32_t (&r)[32], 
     }
     uint16_t h[32];
 #pragma unroll
-    for (int i = 0; i < 32; ++i) h[i] = __bfloat16_as_ushort(__float2bfloat16_rn((float)(int32_t)r[i] * sw_half * s[i]));
+    for (int i = 0; i < 32; i += 2) {
+        // (acc * sw/2) * sx/2 per token, two tokens per packed multiply
+        const float2 y = __fmul2_rn(__fmul2_rn(make_float2((float)(int32_t)r[i], (float)(int32_t)r[i + 1]),
+                                               make_float2(sw_half, sw_half)),
+                                    make_float2(s[i], s[i + 1]));
+        h[i] = __bfloat16_as_ushort(__float2bfloat16_rn(y.x));
+        h[i + 1] = __bfloat16_as_ushort(__float2bfloat16_rn(y.y));
+    }
 #pragma unroll
     for (int i = 0; i < 32; ++i) stg[i * 32] = h[i];
 }
