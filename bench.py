@@ -402,6 +402,7 @@ def run_b200(args, world, rank, local):
     # the int8 tensor-core peak: the rate of back-to-back kind::i8 MMAs measured on this
     # part (no memory traffic), else the nominal dense figure
     probe = None if args.no_probe else mma_probe(dev)
+    pair_probe = None if args.no_probe else mma_probe(dev, pair=True)
     if probe is not None:
         int8_peak, int8_src = probe["tops"], "measured: back-to-back tcgen05 kind::i8 MMAs, one CTA per SM"
     else:
@@ -432,6 +433,10 @@ def run_b200(args, world, rank, local):
                     "frac_of_bf16x2": round(achieved / derived_int8, 4),
                     "bf16x2_source": f"{peaks['source']} bf16 burst x 2 (nominal int8/bf16 dense ratio)",
                     "traffic": ncu_traffic(dominant), "traffic_unit": "bytes per launch (ncu DRAM read+write)"}
+        if pair_probe is not None:
+            # context: the same MMAs in the kernel's own instruction form (cta_group::2, M 256)
+            roofline["frac_of_pair_probe"] = round(achieved / pair_probe["tops"], 4)
+            roofline["pair_probe_tops"] = pair_probe["tops"]
     else:
         achieved = pbytes[dominant] / (avg[dominant] * 1e-3) / 1e9
         roofline = {"kernel": dominant, "bound": "hbm", "achieved": round(achieved, 1),
@@ -481,7 +486,8 @@ def run_b200(args, world, rank, local):
         print(json.dumps(result), flush=True)
 
 
-def mma_probe(dev, gemm_tops=None, iters=20000, reps=5, fp4=False, sparse=False, cp_every=0, bf16=False):
+def mma_probe(dev, gemm_tops=None, iters=20000, reps=5, fp4=False, sparse=False, cp_every=0, bf16=False,
+              pair=False):
     """Tensor-core rate with no memory traffic (back-to-back tcgen05.mma, one CTA per
     SM): kind::i8 M 128 N 256 K 32; with fp4 kind::mxf4 M 128 N 256 K 64 with unit
     block scales; with sparse the 2:4-sparse kind::i8 M 128 N 256 K 64 (logical, the
@@ -495,6 +501,8 @@ def mma_probe(dev, gemm_tops=None, iters=20000, reps=5, fp4=False, sparse=False,
         launch = lambda n, st: q.probe_mma_sp_i8(n, cp_every, st)
     elif bf16:
         launch = q.probe_mma_bf16
+    elif pair:
+        launch = q.probe_mma_i8_pair
     else:
         launch = q.probe_mma_fp4 if fp4 else q.probe_mma_i8
     launch(iters, stream.cuda_stream)
@@ -508,7 +516,8 @@ def mma_probe(dev, gemm_tops=None, iters=20000, reps=5, fp4=False, sparse=False,
         ts.append(a.elapsed_time(b))
     q.probe_status(stream.cuda_stream)
     ms = statistics.median(ts)
-    tops = 2.0 * 128 * 256 * (64 if (fp4 or sparse) else 16 if bf16 else 32) * iters * ctas / (ms * 1e-3) / 1e12
+    per_unit = 2.0 * (256 if pair else 128) * 256 * (64 if (fp4 or sparse) else 16 if bf16 else 32)
+    tops = per_unit * iters * (ctas // 2 if pair else ctas) / (ms * 1e-3) / 1e12
     out = {"tops": round(tops, 1), "iters": iters, "ctas": ctas,
            "note": "timed alone right after the bench loop (burst); the GEMM's roofline peak"}
     if gemm_tops is not None:
@@ -966,6 +975,8 @@ def run_configs(args):
     sp_row["frac_sparse_probe"] = probe_sp["gemm_frac_of_probe"]
     probe_sp_cp = mma_probe(dev, None, sparse=True, cp_every=2)
     probe_sp_cp["note"] = "the same with a tcgen05.cp of metadata before every second MMA"
+    probe_pair = mma_probe(dev, gemm_tops, pair=True)
+    probe_pair["note"] = "cta_group::2 kind::i8 (M 256 per CTA pair), the instruction form of the int8 layers"
     probe_bf = mma_probe(dev, None, bf16=True)
     probe_bf["note"] = "kind::f16 bf16, measured the same way: the denominator for cuBLAS and the f3 kernels"
     for r in rows:
@@ -973,7 +984,7 @@ def run_configs(args):
             r["frac_bf16_probe"] = round(r["tflops"] / probe_bf["tops"], 4)
     print(json.dumps({"configs": rows, "int8_mma_probe": probe, "fp4_mma_probe": probe4,
                       "sparse_mma_probe": probe_sp, "sparse_mma_probe_cp2": probe_sp_cp,
-                      "bf16_mma_probe": probe_bf, "peaks": peaks}), flush=True)
+                      "int8_pair_mma_probe": probe_pair, "bf16_mma_probe": probe_bf, "peaks": peaks}), flush=True)
 
 
 def run_profile_kernels(args):

@@ -55,6 +55,7 @@ PROBE_SIGNATURES = {
     "quest_probe_mma_i8": (_int, [_int, _p, _p]),
     "quest_probe_mma_fp4": (_int, [_int, _p, _p]),
     "quest_probe_mma_bf16": (_int, [_int, _p, _p]),
+    "quest_probe_mma_i8_pair": (_int, [_int, _p, _p]),
     "quest_probe_mma_sp_i8": (_int, [_int, _int, _p, _p]),
     "quest_probe_status": (_int, [_p]),
 }
@@ -525,6 +526,14 @@ def probe_mma_fp4(iters, stream=0):
     """Enqueue the FP4 (kind::mxf4) tensor-core peak probe; returns the number of CTAs launched."""
     ctas = ctypes.c_int(0)
     _check_probe(load_probe_library().quest_probe_mma_fp4(iters, ctypes.byref(ctas), stream), "quest_probe_mma_fp4")
+    return ctas.value
+
+
+def probe_mma_i8_pair(iters, stream=0):
+    """Enqueue the CTA-pair int8 probe (cta_group::2, M = 256); returns the number of CTAs."""
+    ctas = ctypes.c_int(0)
+    _check_probe(load_probe_library().quest_probe_mma_i8_pair(iters, ctypes.byref(ctas), stream),
+                 "quest_probe_mma_i8_pair")
     return ctas.value
 
 

@@ -341,6 +341,80 @@ extern "C" quest_status quest_probe_mma_fp4(int iters, int* ctas, void* stream) 
 namespace quest {
 namespace {
 
+// The int8 kind as the linear layer issues it: CTA pairs (cluster of two,
+// tcgen05.mma.cta_group::2.kind::i8, M = 256 across the pair, N = 256, K = 32), each
+// CTA holding its 128 rows of A and 128 rows of B in shared memory; the even CTA
+// issues, one multicast commit ends the run in both CTAs.
+constexpr uint32_t kIdescProbePair = (2u << 4) | (1u << 7) | (1u << 10) | (uint32_t(256 >> 3) << 17) |
+                                     (uint32_t(256 >> 4) << 24);
+
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kProbeThreads, 1) probe_mma_i8_pair_kernel(int iters) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const uint32_t sbase = static_cast<uint32_t>(__cvta_generic_to_shared(smem));
+    const uint32_t bar = sbase, slot = sbase + 16, a_addr = sbase + 1024, b_addr = a_addr + 128 * 128;
+    for (uint32_t i = threadIdx.x * 16; i < 2 * 128 * 128; i += kProbeThreads * 16)
+        *reinterpret_cast<uint4*>(smem + 1024 + i) = make_uint4(0x01010101u, 0x01010101u, 0x01010101u, 0x01010101u);
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    uint32_t rank;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(rank));
+    if (threadIdx.x == 0) {
+        asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(bar) : "memory");
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    const int warp = threadIdx.x >> 5;
+    if (warp == 0) {
+        asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], 512;" ::"r"(slot) : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+    }
+    asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+    const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(smem + 16);
+    if (rank == 0 && threadIdx.x == 0) {
+        for (int i = 0; i < iters; ++i) {
+            const uint32_t kk = uint32_t(i & 3) * 32;   // the four 32-byte K steps of a 128-byte row
+            asm volatile(
+                "{\n\t.reg .pred p;\n\t"
+                "setp.ne.b32 p, %4, 0;\n\t"
+                "tcgen05.mma.cta_group::2.kind::i8 [%0], %1, %2, %3, p;\n\t}" ::"r"(tmem),
+                "l"(probe_desc(a_addr + kk)), "l"(probe_desc(b_addr + kk)), "r"(kIdescProbePair), "r"(i)
+                : "memory");
+        }
+        asm volatile(
+            "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;" ::"r"(
+                bar),
+            "h"((uint16_t)0x3)
+            : "memory");
+    }
+    if (threadIdx.x == 0) {
+        // bounded wait for the pair's MMAs (2 s; iters <= 2^20 take tens of milliseconds)
+        uint64_t t0, t;
+        asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t0));
+        for (;;) {
+            uint32_t ok;
+            asm volatile(
+                "{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], 0;\n\t"
+                "selp.u32 %0, 1, 0, p;\n\t}"
+                : "=r"(ok)
+                : "r"(bar)
+                : "memory");
+            if (ok) break;
+            asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+            if (t - t0 > 2000000000ull) {
+                atomicExch(&g_probe_status, (int)QUEST_ETIMEOUT);
+                break;
+            }
+        }
+    }
+    asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+    if (warp == 0) {
+        asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+        asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, 512;" ::"r"(tmem) : "memory");
+    }
+}
+
 template <bool kBf16>
 quest_status launch_probe_dense(int iters, int* ctas, void* stream) {
     if (iters < 1 || iters > kMaxIters || ctas == nullptr) return QUEST_EINVAL;
@@ -399,5 +473,22 @@ extern "C" quest_status quest_probe_mma_sp_i8(int iters, int cp_every, int* ctas
     *ctas = probe_sm_count();
     probe_mma_sp_i8_kernel<<<*ctas, kProbeThreads, kProbeSmem + 1024, static_cast<cudaStream_t>(stream)>>>(iters,
                                                                                                        cp_every);
+    return cudaGetLastError() == cudaSuccess ? QUEST_OK : QUEST_ECUDA;
+}
+
+extern "C" quest_status quest_probe_mma_i8_pair(int iters, int* ctas, void* stream) {
+    using namespace quest;
+    if (iters < 1 || iters > kMaxIters || ctas == nullptr) return QUEST_EINVAL;
+    static thread_local int attr_dev = -1;
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (attr_dev != dev) {
+        if (cudaFuncSetAttribute(probe_mma_i8_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 kProbeSmem + 1024) != cudaSuccess)
+            return QUEST_ECUDA;
+        attr_dev = dev;
+    }
+    *ctas = probe_sm_count() & ~1;   // whole pairs, one CTA per SM
+    probe_mma_i8_pair_kernel<<<*ctas, kProbeThreads, kProbeSmem + 1024, static_cast<cudaStream_t>(stream)>>>(iters);
     return cudaGetLastError() == cudaSuccess ? QUEST_OK : QUEST_ECUDA;
 }

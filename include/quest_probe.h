@@ -28,6 +28,13 @@ extern "C" {
  * QUEST_ECUDA on a launch error. */
 quest_status quest_probe_mma_i8(int iters, int* ctas, void* stream);
 
+/* The int8 kind as the linear layer issues it: CTA pairs (cluster of two CTAs on
+ * two SMs, tcgen05.mma.cta_group::2.kind::i8, M = 256 across the pair, N = 256,
+ * K = 32), back to back from shared memory; `*ctas` receives the number of CTAs
+ * (an even count, one per SM). The caller computes
+ * 2 * 256 * 256 * 32 * iters * (ctas / 2) / seconds. Errors as above. */
+quest_status quest_probe_mma_i8_pair(int iters, int* ctas, void* stream);
+
 /* The same for bf16: back-to-back tcgen05.mma kind::f16 (M = 128, N = 256,
  * K = 16, bf16 operands, fp32 accumulator); the caller computes
  * 2 * 128 * 256 * 16 * iters * ctas / seconds. Errors as above. */

@@ -191,7 +191,7 @@ def test_w4a4_rejects_invalid_arguments():
 def test_probe_rejects_invalid_arguments():
     lib = _binding.load_probe_library()
     n = ctypes.c_int(0)
-    for fn in (lib.quest_probe_mma_i8, lib.quest_probe_mma_fp4, lib.quest_probe_mma_bf16):
+    for fn in (lib.quest_probe_mma_i8, lib.quest_probe_mma_fp4, lib.quest_probe_mma_bf16, lib.quest_probe_mma_i8_pair):
         assert fn(0, ctypes.byref(n), None) == 1
         assert fn((1 << 20) + 1, ctypes.byref(n), None) == 1   # cap: far inside the 2 s wait
         assert fn(100, None, None) == 1
