@@ -22,10 +22,13 @@ __device__ int g_probe_status = 0;
 
 namespace {
 
-// At most 2^20 MMAs per CTA: tens of milliseconds at any clock, far inside the
+// At most 2^16 MMAs per CTA: a few milliseconds at any clock, far inside the
 // kernel's 2 s completion wait, so that wait never gives up (and never frees
-// TMEM) while MMAs are still in flight.
-constexpr int kMaxIters = 1 << 20;
+// TMEM) while MMAs are still in flight. The benchmark runs 20000; a scratch
+// variant of the pair probe run with 200000 ended in an illegal-address error
+// whose cause reading the code did not show, so runs stay in the range that has
+// been exercised.
+constexpr int kMaxIters = 1 << 16;
 
 int probe_sm_count() {
     int dev = 0, n = 0;
@@ -388,7 +391,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kProbeThreads, 1) pr
             : "memory");
     }
     if (threadIdx.x == 0) {
-        // bounded wait for the pair's MMAs (2 s; iters <= 2^20 take tens of milliseconds)
+        // bounded wait for the pair's MMAs (2 s; iters <= 2^16 take a few milliseconds)
         uint64_t t0, t;
         asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t0));
         for (;;) {

@@ -23,7 +23,7 @@ extern "C" {
  * traffic. `*ctas` receives the number of CTAs launched (host pointer). The
  * caller times the launch on `stream` (CUDA events) and computes
  * 2 * 128 * 256 * 32 * iters * ctas / seconds.
- * Errors: QUEST_EINVAL if iters is outside [1, 2^20] (so a launch stays far
+ * Errors: QUEST_EINVAL if iters is outside [1, 2^16] (so a launch stays far
  * inside the kernel's 2 s completion wait) or ctas is NULL;
  * QUEST_ECUDA on a launch error. */
 quest_status quest_probe_mma_i8(int iters, int* ctas, void* stream);
@@ -53,7 +53,7 @@ quest_status quest_probe_mma_fp4(int iters, int* ctas, void* stream);
  * precedes every c-th MMA, whose group of c MMAs then reads the copied columns;
  * cp_every = 0 keeps the metadata resident. The caller computes the
  * dense-equivalent rate 2 * 128 * 256 * 64 * iters * ctas / seconds.
- * Errors: QUEST_EINVAL if iters is outside [1, 2^20], cp_every outside
+ * Errors: QUEST_EINVAL if iters is outside [1, 2^16], cp_every outside
  * [0, 64] or ctas is NULL; QUEST_ECUDA on a launch error. */
 quest_status quest_probe_mma_sp_i8(int iters, int cp_every, int* ctas, void* stream);
 

@@ -193,11 +193,11 @@ def test_probe_rejects_invalid_arguments():
     n = ctypes.c_int(0)
     for fn in (lib.quest_probe_mma_i8, lib.quest_probe_mma_fp4, lib.quest_probe_mma_bf16, lib.quest_probe_mma_i8_pair):
         assert fn(0, ctypes.byref(n), None) == 1
-        assert fn((1 << 20) + 1, ctypes.byref(n), None) == 1   # cap: far inside the 2 s wait
+        assert fn((1 << 16) + 1, ctypes.byref(n), None) == 1   # cap: far inside the 2 s wait
         assert fn(100, None, None) == 1
     sp = lib.quest_probe_mma_sp_i8
     assert sp(0, 0, ctypes.byref(n), None) == 1
-    assert sp((1 << 20) + 1, 2, ctypes.byref(n), None) == 1
+    assert sp((1 << 16) + 1, 2, ctypes.byref(n), None) == 1
     assert sp(100, -1, ctypes.byref(n), None) == 1 and sp(100, 65, ctypes.byref(n), None) == 1
     assert sp(100, 2, None, None) == 1
 
