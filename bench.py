@@ -1033,7 +1033,8 @@ def run_profile_kernels(args):
 def main():
     ap = argparse.ArgumentParser(description=__doc__)
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=1000)
+    ap.add_argument("--steps", type=int, default=None,
+                    help="timed steps (default: 1000 for the B200 arm, 20 for the CPU oracle arm)")
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["b200", "reference"], default="b200")
     ap.add_argument("--no-e2e", action="store_true")
@@ -1045,6 +1046,9 @@ def main():
     ap.add_argument("--configs", action="store_true",
                     help="time every workload configuration (median / p10 per kernel) and exit")
     args = ap.parse_args()
+    if args.steps is None:
+        # the oracle arm samples each step on the host cores (about half a second a step)
+        args.steps = 1000 if args.impl == "b200" else 20
     if args.profile_kernels:
         run_profile_kernels(args)
         return
