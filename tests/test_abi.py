@@ -22,7 +22,8 @@ def _declared_functions(probe=False):
     names = set()
     for fn in os.listdir(os.path.join(ROOT, "include")):
         if fn.endswith(".h") and (fn == PROBE_HEADER) == probe:
-            text = open(os.path.join(ROOT, "include", fn)).read()
+            with open(os.path.join(ROOT, "include", fn)) as f:
+                text = f.read()
             text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
             names |= set(re.findall(r"\b(quest_\w+)\s*\(", text))
     return names
