@@ -119,71 +119,99 @@ __device__ __forceinline__ void tc_cp_meta(uint32_t taddr, uint64_t sdesc) {
     asm volatile("tcgen05.cp.cta_group::1.128x128b [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
 }
 
-// One 32-token chunk of a weight row (TMEM lane): scale, round to bf16 and store
-// the 32 values down the warp's transposed stage (token i of the chunk at row i,
-// this weight row at column lane). The chunk's token scales are read into registers
-// (as float4) before any store: the 16-bit stores and the scale loads both go
-// to shared memory, and interleaved the compiler has to keep every store ahead
-// of the next load, which chained the 32 conversions one after another.
-__device__ __forceinline__ void stage_chunk_transposed(const uint32_t (&r)[32], float sw_half, const float* sc,
-                                                       uint16_t* stg) {
-    float s[32];
-#pragma unroll
-    for (int i = 0; i < 32; i += 4) {
-        const float4 v = *reinterpret_cast<const float4*>(sc + i);
-        s[i] = v.x;
-        s[i + 1] = v.y;
-        s[i + 2] = v.z;
-        s[i + 3] = v.w;
-    }
-    uint16_t h[32];
-#pragma unroll
-    for (int i = 0; i < 32; i += 2) {
-        // (acc * sw/2) * sx/2 per token, two tokens per packed multiply
-        const float2 y = __fmul2_rn(__fmul2_rn(make_float2((float)(int32_t)r[i], (float)(int32_t)r[i + 1]),
-                                               make_float2(sw_half, sw_half)),
-                                    make_float2(s[i], s[i + 1]));
-        h[i] = __bfloat16_as_ushort(__float2bfloat16_rn(y.x));
-        h[i + 1] = __bfloat16_as_ushort(__float2bfloat16_rn(y.y));
-    }
-#pragma unroll
-    for (int i = 0; i < 32; ++i) stg[i * 32] = h[i];
-}
-
 __device__ __forceinline__ void bulk_wait_read_stg() {
     asm volatile("cp.async.bulk.wait_group.read %0;" ::"n"(kStgBufs - 1) : "memory");
 }
 
-// This warp's 32 weight rows x SBN tokens of a finished accumulator out to y[m][n]:
-// per 32-token chunk one TMEM load, the scaled bf16 values down a staging buffer of the
-// warp's own, and one TMA store of that 32 x 32 box (no barrier with the other warps;
-// the buffer is reused once at most kStgBufs - 1 of the warp's stores are still reading).
-// n_w: the warp's first weight row; n = n_w + lane. Lane 0 issues and tracks the stores.
-__device__ __forceinline__ void store_tile_transposed(const CUtensorMap& map_y, uint32_t t_acc, uint8_t* stg,
-                                                      uint32_t stg_addr, int& cbuf, int lane, int n_w, int m0,
-                                                      float sw_half, const float* s_scale, int32_t* acc, int M,
-                                                      int N) {
-    const int n = n_w + lane;
+// 16 TMEM lanes x 32 columns in the 16x256b pattern: thread t receives, for k = 0..3,
+// r[4k], r[4k+1] = lane t/4, columns 8k + 2(t%4), 8k + 2(t%4) + 1 and r[4k+2], r[4k+3] =
+// lane t/4 + 8, the same columns (the fragment layout of an 8 x 8 matrix pair).
+#define QUEST_TMEM_LD16X256_X4(taddr, r)                                                       \
+    asm volatile(                                                                              \
+        "tcgen05.ld.sync.aligned.16x256b.x4.b32 "                                             \
+        "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"                      \
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), \
+          "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),          \
+          "=r"(r[13]), "=r"(r[14]), "=r"(r[15])                                                \
+        : "r"(taddr))
+
+// Four 8 x 8 bf16 matrices, each stored transposed (rows of the fragment become columns).
+__device__ __forceinline__ void stmatrix_x4_trans(uint32_t addr, uint32_t r0, uint32_t r1, uint32_t r2,
+                                                  uint32_t r3) {
+    asm volatile("stmatrix.sync.aligned.m8n8.x4.trans.shared.b16 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(r0),
+                 "r"(r1), "r"(r2), "r"(r3)
+                 : "memory");
+}
+
+// This warp's 32 weight rows x SBN tokens of a finished accumulator out to y[m][n]. The
+// accumulator holds D[n][m] (lane = weight row), y wants rows of tokens, so each 32-token
+// chunk is read in the 16x256b pattern, in which a thread holds two adjacent tokens of two
+// weight rows: scaled, rounded to bf16 pairs, these are the fragments of 8 x 8 matrices that
+// stmatrix.trans writes transposed into a staging buffer laid out as y's rows ([token][32
+// weight rows], 64-byte swizzle); the warp's own TMA store writes the 32 x 32 box. Four
+// stmatrix per chunk replace 32 16-bit stores of a thread-per-row layout. The buffer is
+// reused once at most kStgBufs - 1 of the warp's stores are still reading. n_w: the warp's
+// first weight row; sw_half: the scale of weight row n_w + lane. Lane 0 issues the stores.
+__device__ __forceinline__ void store_tile_transposed(const CUtensorMap& map_y, uint32_t t_acc, uint32_t stg_addr,
+                                                      int& cbuf, int lane, int n_w, int m0, float sw_half,
+                                                      const float* s_scale, int32_t* acc, int M, int N) {
+    const int g = lane >> 2, t = lane & 3, q = lane >> 3, rr = lane & 7;
+    // scales of the weight rows this thread holds: n_w + 16h + 8rb + g
+    float swr[2][2];
+#pragma unroll
+    for (int h = 0; h < 2; ++h)
+#pragma unroll
+        for (int rb = 0; rb < 2; ++rb) swr[h][rb] = __shfl_sync(0xFFFFFFFFu, sw_half, 16 * h + 8 * rb + g);
 #pragma unroll 1
     for (int c = 0; c < SBN / 32; ++c) {
-        uint32_t r[32];
-        QUEST_TMEM_LD32(t_acc + c * 32, r);
+        uint32_t ra[2][16];   // lanes 0-15 and 16-31 of the warp's quarter
+        QUEST_TMEM_LD16X256_X4(t_acc + c * 32, ra[0]);
+        QUEST_TMEM_LD16X256_X4(t_acc + (16u << 16) + c * 32, ra[1]);
         tmem_wait_ld();
         if (lane == 0) bulk_wait_read_stg();
         __syncwarp();
-        stage_chunk_transposed(r, sw_half, s_scale + c * 32,
-                               reinterpret_cast<uint16_t*>(stg + cbuf * kStgBytes) + lane);
-        if (acc != nullptr && n < N) {
+        const uint32_t base = stg_addr + cbuf * kStgBytes;
 #pragma unroll
-            for (int i = 0; i < 32; ++i) {
-                const int m = m0 + c * 32 + i;
-                if (m < M) acc[int64_t(m) * N + n] = (int32_t)r[i];
+        for (int h = 0; h < 2; ++h) {
+            uint32_t P[4][2];   // [8-token block k][weight-row block rb]: a bf16 pair
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                const float2 s = *reinterpret_cast<const float2*>(s_scale + c * 32 + 8 * k + 2 * t);
+#pragma unroll
+                for (int rb = 0; rb < 2; ++rb) {
+                    // (acc * sw/2) * sx/2 per token, two tokens per packed multiply
+                    const float2 v = __fmul2_rn(__fmul2_rn(make_float2((float)(int32_t)ra[h][4 * k + 2 * rb],
+                                                                       (float)(int32_t)ra[h][4 * k + 2 * rb + 1]),
+                                                           make_float2(swr[h][rb], swr[h][rb])),
+                                                s);
+                    __nv_bfloat162 hb = __floats2bfloat162_rn(v.x, v.y);
+                    P[k][rb] = *reinterpret_cast<uint32_t*>(&hb);
+                }
+            }
+            // matrix j of an x4 takes its row addresses from threads 8j .. 8j + 7: token
+            // 8k + rr of the chunk, weight-row block nb (16 bytes), 64-byte swizzle
+#pragma unroll
+            for (int kp = 0; kp < 2; ++kp) {
+                const int k = 2 * kp + (q >> 1), nb = 2 * h + (q & 1), m = 8 * k + rr;
+                const uint32_t addr = base + uint32_t(m) * 64u + (uint32_t(nb ^ ((m >> 1) & 3)) << 4);
+                stmatrix_x4_trans(addr, P[2 * kp][0], P[2 * kp][1], P[2 * kp + 1][0], P[2 * kp + 1][1]);
+            }
+            if (acc != nullptr) {
+#pragma unroll
+                for (int k = 0; k < 4; ++k)
+#pragma unroll
+                    for (int rb = 0; rb < 2; ++rb)
+#pragma unroll
+                        for (int e = 0; e < 2; ++e) {
+                            const int n = n_w + 16 * h + 8 * rb + g, m = m0 + c * 32 + 8 * k + 2 * t + e;
+                            if (n < N && m < M) acc[int64_t(m) * N + n] = (int32_t)ra[h][4 * k + 2 * rb + e];
+                        }
             }
         }
         fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) {
-            tma_store_2d(&map_y, stg_addr + cbuf * kStgBytes, n_w, m0 + c * 32);
+            tma_store_2d(&map_y, base, n_w, m0 + c * 32);
             bulk_commit();
         }
         cbuf = cbuf + 1 == kStgBufs ? 0 : cbuf + 1;
@@ -318,7 +346,6 @@ w4a4_sparse_kernel(const __grid_constant__ CUtensorMap map_w, const __grid_const
         const int quarter = warp & 3;                 // TMEM lanes 32*quarter .. +31
         const int row = quarter * 32 + lane;          // weight row within the tile = TMEM lane
         const uint32_t lane_addr = uint32_t(quarter * 32) << 16;
-        uint8_t* stg_w = smem + kSSmemC + (warp - 2) * kStgBufs * kStgBytes;
         const uint32_t stg_w_addr = sbase + kSSmemC + (warp - 2) * kStgBufs * kStgBytes;
         int local = 0, cbuf = 0;
         for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++local) {
@@ -335,8 +362,8 @@ w4a4_sparse_kernel(const __grid_constant__ CUtensorMap map_w, const __grid_const
             if (epi_any(!got)) break;   // also orders the token scales above (bar.red)
             tc_fence_after();
             const uint32_t t_acc = tmem_base + lane_addr + buf * kSAccCols;
-            store_tile_transposed(map_y, t_acc, stg_w, stg_w_addr, cbuf, lane, n0 + 32 * quarter, m0, sw_half,
-                                  s_scale, p.acc, p.M, p.N);
+            store_tile_transposed(map_y, t_acc, stg_w_addr, cbuf, lane, n0 + 32 * quarter, m0, sw_half, s_scale,
+                                  p.acc, p.M, p.N);
             tc_fence_before();
             mbar_arrive(bar_tempty + 8 * buf);
         }
@@ -608,7 +635,6 @@ w4a4_sparse_pair_kernel(const __grid_constant__ CUtensorMap map_w, const __grid_
         const int row = quarter * 32 + lane;          // weight row within this CTA's half = TMEM lane
         const uint32_t lane_addr = uint32_t(quarter * 32) << 16;
         const uint32_t tempty_even = map_to_rank(bar_tempty, 0);
-        uint8_t* stg_w = smem + L::kC + (warp - 2) * kStgBufs * kStgBytes;
         const uint32_t stg_w_addr = sbase + L::kC + (warp - 2) * kStgBufs * kStgBytes;
         int local = 0, cbuf = 0;
         for (int tile = t_begin; tile < t_end; tile += t_step, ++local) {
@@ -625,8 +651,8 @@ w4a4_sparse_pair_kernel(const __grid_constant__ CUtensorMap map_w, const __grid_
             if (epi_any(!got)) break;   // also orders the token scales above (bar.red)
             tc_fence_after();
             const uint32_t t_acc = tmem_base + lane_addr + buf * kSAccCols;
-            store_tile_transposed(map_y, t_acc, stg_w, stg_w_addr, cbuf, lane, n0 + 32 * quarter, m0, sw_half,
-                                  s_scale, p.acc, p.M, p.N);
+            store_tile_transposed(map_y, t_acc, stg_w_addr, cbuf, lane, n0 + 32 * quarter, m0, sw_half, s_scale,
+                                  p.acc, p.M, p.N);
             tc_fence_before();
             epi_bar();
             if (et == 0) mbar_arrive_remote(tempty_even + 8 * buf);
@@ -679,7 +705,7 @@ cudaError_t launch_w4a4_sparse24(const int8_t* X, const float* sx, const int8_t*
                      CU_TENSOR_MAP_SWIZZLE_128B) ||
         !make_map_2d(&me, CU_TENSOR_MAP_DATA_TYPE_UINT8, E, K / 8, N, K / 8, SBK / 8, SBM,
                      CU_TENSOR_MAP_SWIZZLE_NONE) ||
-        !make_map_2d(&my, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, y, N, M, N * 2, 32, 32, CU_TENSOR_MAP_SWIZZLE_NONE))
+        !make_map_2d(&my, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, y, N, M, N * 2, 32, 32, CU_TENSOR_MAP_SWIZZLE_64B))
         return cudaErrorInvalidValue;
     if (pairs) {
         SparsePairParams pp;
