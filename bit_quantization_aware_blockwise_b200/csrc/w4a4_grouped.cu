@@ -29,38 +29,45 @@ namespace {
 //
 // Every group's product makes a round trip through TMEM to registers, where it
 // is scaled and added: acc += P_g * (sa/2)(sb/2), two packed FP instructions per
-// pair of outputs per group. The epilogue runs as two teams of four warps (one
-// warp per TMEM lane quarter on each team), each team owning the whole 128 x 128
-// accumulator of its own output tile in registers: the CTA pair takes its tiles
-// two at a time, and the MMA issuer alternates between them group by group
-// (tile 2c group g, tile 2c+1 group g, tile 2c group g+1, ...), so the two
-// warps on a scheduler are at different points of their groups. Each team has
-// two of the four 128-column TMEM slots; a slot's full barrier (committed by the
-// MMA issuer in both CTAs) says that its group's product is complete, its empty
-// barrier (8 warp arrivals) that the team has read it. A slot is never reissued
-// before its team has read it, so its full barrier is at most one phase ahead of
-// the team's wait. An epilogue thread holds its row of the accumulator (128
-// registers) and two 16-column TMEM load buffers, so the load of the next 16
-// columns overlaps the arithmetic on the current ones.
+// pair of outputs per group. A pair tile is 256 rows x 256 columns, computed as two
+// 128-column halves: every operand stage holds one group of the tile's A rows and
+// of the B rows of both halves, and the MMA issuer runs both halves' MMAs off it
+// (half 0 into one TMEM slot, half 1 into another), so A crosses from L2 once per
+// group for both. The epilogue runs as two teams of four warps (one warp per TMEM
+// lane quarter on each team), team h owning the 128 x 128 accumulator of half h in
+// registers; the two warps on a scheduler read alternate slots. Each team has two
+// of the four 128-column TMEM slots (groups alternate between them); a slot's full
+// barrier (committed by the MMA issuer in both CTAs) says that its group's product
+// is complete, its empty barrier (8 warp arrivals) that the team has read it. A slot
+// is never reissued before its team has read it, so its full barrier is at most one
+// phase ahead of the team's wait. An epilogue thread holds its row of the
+// accumulator (128 registers) and two 16-column TMEM load buffers, so the load of
+// the next 16 columns overlaps the arithmetic on the current ones.
 //
-// What bounds it (16384 x 5632 x 2048, scratch variants timed on B200): 400 us
-// as built; 393 us with half the MMAs; 330 us with the FP work removed; 254 us
-// with neither MMAs nor FP work. That last floor is the operand feed: 128-wide
-// pair tiles load 48 KB per 256 x 128 x 128 group, twice the bytes per MMA of
-// the integer layer's 256-wide tiles, and 2.16 GB in 254 us is 8.5 TB/s of TMA
-// loads, near the 11-12 TB/s the other tensor-core layers reach. TMEM reads are
-// not the limit (a probe of back-to-back tcgen05.ld reads 460-935 B per clock
-// per SM; this layer moves about 50). A lockstep layout (eight warps on the same
-// group, 64 columns each, two 32-column loads per wait) measured the same 403 us.
+// What bounds it (16384 x 5632 x 2048, scratch variants of the earlier layout,
+// in which the two teams took two different 256 x 128 tiles and every stage held
+// one tile's group, timed on B200): 400 us as built; 393 us with half the MMAs;
+// 330 us with the FP work removed; 254 us with neither MMAs nor FP work, the
+// operand feed of 48 KB per 256 x 128 x 128 group (2.16 GB in 254 us, 8.5 TB/s
+// of TMA loads). Sharing A between the two halves cuts that feed by a third
+// (64 KB per 256 x 256 x 128 group), yet the layer gained only 1-2 % (387 us
+// against 390 us in an interleaved A/B, outputs identical): the hand-off of the
+// TMEM slots (the MMA's commit, the team's reads, the arrivals from both CTAs,
+// the polling on both sides) sets the pace, not the feed. TMEM reads are not the
+// limit (a probe of back-to-back tcgen05.ld reads 460-935 B per clock per SM;
+// this layer moves about 50). A lockstep layout (eight warps on the same group,
+// 64 columns each, two 32-column loads per wait) measured the same 403 us.
 
 constexpr int kGThreads = 384;               // warpgroup 0: producer, MMA (2 warps idle); 1, 2: the teams
 constexpr int kGTeamThreads = 128;
-constexpr int kGBN = 128;                    // output columns per pair tile
-constexpr int kGStages = 6;
+constexpr int kGBN = 128;                    // output columns per team (one half of a pair tile)
+constexpr int kGWide = 2 * kGBN;             // output columns per pair tile
+constexpr int kGStages = 5;
 constexpr int kGSlots = 4;                   // TMEM slots of kGBN columns, two per team
 constexpr int kGroup = 128;                  // K group = one stage
 constexpr int kGScaleBlock = 8;              // groups of scales staged at a time
-constexpr uint32_t kGStageA = 128 * BK, kGStageB = (kGBN / 2) * BK;   // per CTA
+// per CTA and stage: 128 A rows; the B rows of half 0, then of half 1 (kGBN / 2 each)
+constexpr uint32_t kGStageA = 128 * BK, kGStageBHalf = (kGBN / 2) * BK, kGStageB = 2 * kGStageBHalf;
 constexpr uint32_t kGTxBytes = 2 * (kGStageA + kGStageB);
 constexpr uint32_t kGSmemA = 0;
 constexpr uint32_t kGSmemB = kGSmemA + kGStages * kGStageA;
@@ -130,7 +137,7 @@ struct GroupedParams {
     const float* sb;    // [N, K / 128]
     float* y32;         // optional fp32 copy of Y [M, N]
     int M, N, K;
-    int num_m2, num_n, num_k;   // 256-row pair tiles, 128-column tiles, K groups
+    int num_m2, num_n, num_k;   // 256-row and 256-column pair tiles, K groups
 };
 
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGThreads, 1)
@@ -153,8 +160,7 @@ w4a4_gemm_grouped_kernel(const __grid_constant__ CUtensorMap map_a, const __grid
     const int pair = blockIdx.x >> 1, num_pairs = gridDim.x >> 1;
     const int num_tiles = p.num_m2 * p.num_n;
     const int G = p.num_k;
-    // this pair's tiles: pair + i * num_pairs for i < ntl, taken two at a time
-    // (couple c = tiles 2c and 2c + 1; the last couple may hold one tile)
+    // this pair's tiles: pair + i * num_pairs for i < ntl
     const int ntl = (num_tiles - pair + num_pairs - 1) / num_pairs;
 
     if (threadIdx.x == 0) {
@@ -196,21 +202,21 @@ w4a4_gemm_grouped_kernel(const __grid_constant__ CUtensorMap map_a, const __grid
             uint32_t stage = 0, phase = 0;
             uint64_t issued = 0;
             bool ok = true;
-            for (int c = 0; 2 * c < ntl && ok; ++c) {
-                const int nt = 2 * c + 1 < ntl ? 2 : 1;
+            for (int i = 0; i < ntl && ok; ++i) {
+                const int tile = pair + i * num_pairs;
+                const int m0 = (tile % p.num_m2) * 256 + 128 * int(rank);
+                // half h's B rows: n0 + h * kGBN .. + kGBN / 2 - 1 in this CTA
+                const int n0 = (tile / p.num_m2) * kGWide + (kGBN / 2) * int(rank);
                 for (int kb = 0; kb < G && ok; ++kb) {
-                    for (int t = 0; t < nt; ++t) {
-                        const int tile = pair + (2 * c + t) * num_pairs;
-                        const int m0 = (tile % p.num_m2) * 256 + 128 * int(rank);
-                        const int n0 = (tile / p.num_m2) * kGBN + (kGBN / 2) * int(rank);
-                        if (!mbar_wait(bar_empty + 8 * stage, phase ^ 1, abort_flag)) { ok = false; break; }
-                        if (even) mbar_arrive_expect_tx(bar_full + 8 * stage, kGTxBytes);
-                        const uint32_t fb = full_even + 8 * stage;
-                        tma_load_2d_pair(sbase + kGSmemA + stage * kGStageA, &map_a, kb * BK, m0, fb);
-                        tma_load_2d_pair(sbase + kGSmemB + stage * kGStageB, &map_b, kb * BK, n0, fb);
-                        ++issued;
-                        if (++stage == kGStages) { stage = 0; phase ^= 1; }
-                    }
+                    if (!mbar_wait(bar_empty + 8 * stage, phase ^ 1, abort_flag)) { ok = false; break; }
+                    if (even) mbar_arrive_expect_tx(bar_full + 8 * stage, kGTxBytes);
+                    const uint32_t fb = full_even + 8 * stage;
+                    const uint32_t b_st = sbase + kGSmemB + stage * kGStageB;
+                    tma_load_2d_pair(sbase + kGSmemA + stage * kGStageA, &map_a, kb * BK, m0, fb);
+                    tma_load_2d_pair(b_st, &map_b, kb * BK, n0, fb);
+                    tma_load_2d_pair(b_st + kGStageBHalf, &map_b, kb * BK, n0 + kGBN, fb);
+                    ++issued;
+                    if (++stage == kGStages) { stage = 0; phase ^= 1; }
                 }
             }
             if (!ok && even) {
@@ -231,31 +237,31 @@ w4a4_gemm_grouped_kernel(const __grid_constant__ CUtensorMap map_a, const __grid
         // ------------------------------------------------------------ MMA issuer (even CTA)
         if (even && lane == 0) {
             uint32_t stage = 0, phase = 0;
-            uint32_t gcount0 = 0, gcount1 = 0;   // groups issued per team: slot 2 t + (count & 1)
+            uint32_t gc = 0;   // groups issued (the same for both halves): half h's slot is 2 h + (gc & 1)
             bool ok = true;
-            for (int c = 0; 2 * c < ntl && ok; ++c) {
-                const int nt = 2 * c + 1 < ntl ? 2 : 1;
+            for (int i = 0; i < ntl && ok; ++i) {
                 for (int kb = 0; kb < G && ok; ++kb) {
-                    for (int t = 0; t < nt; ++t) {
-                        const uint32_t gc = t ? gcount1 : gcount0;
-                        const uint32_t slot = 2 * t + (gc & 1), sphase = (gc >> 1) & 1;
+                    if (!mbar_wait(bar_full + 8 * stage, phase, abort_flag)) { ok = false; break; }
+                    const uint32_t a_addr = sbase + kGSmemA + stage * kGStageA;
+                    const uint32_t b_st = sbase + kGSmemB + stage * kGStageB;
+                    const uint32_t sphase = (gc >> 1) & 1;
+#pragma unroll 1
+                    for (int h = 0; h < 2; ++h) {
+                        const uint32_t slot = 2 * h + (gc & 1);
                         if (!mbar_wait(bar_tempty + 8 * slot, sphase ^ 1, abort_flag)) { ok = false; break; }
-                        if (!mbar_wait(bar_full + 8 * stage, phase, abort_flag)) { ok = false; break; }
                         tc_fence_after();
                         const uint32_t d_tmem = tmem_base + slot * kGBN;
-                        const uint32_t a_addr = sbase + kGSmemA + stage * kGStageA;
-                        const uint32_t b_addr = sbase + kGSmemB + stage * kGStageB;
+                        const uint32_t b_addr = b_st + h * kGStageBHalf;
 #pragma unroll
                         for (int kk = 0; kk < BK / kUmmaK; ++kk) {
                             tc_mma_f8_pair(d_tmem, smem_desc_k128(a_addr + kk * kUmmaK),
                                            smem_desc_k128(b_addr + kk * kUmmaK), kk != 0);
                         }
-                        tc_commit_pair_mc(bar_empty + 8 * stage);   // frees the stage in both CTAs
-                        tc_commit_pair_mc(bar_tfull + 8 * slot);    // the group's product is ready
-                        if (t) gcount1 = gc + 1;
-                        else gcount0 = gc + 1;
-                        if (++stage == kGStages) { stage = 0; phase ^= 1; }
+                        if (h == 1) tc_commit_pair_mc(bar_empty + 8 * stage);   // frees the stage in both CTAs
+                        tc_commit_pair_mc(bar_tfull + 8 * slot);                 // the half's product is ready
                     }
+                    ++gc;
+                    if (++stage == kGStages) { stage = 0; phase ^= 1; }
                 }
             }
             tc_commit_pair(bar_drain);
@@ -266,7 +272,7 @@ w4a4_gemm_grouped_kernel(const __grid_constant__ CUtensorMap map_a, const __grid
     } else if (warp >= 4) {
         // ------------------------------------------------------------ epilogue (warps 4..11, both CTAs)
         const int ew = warp - 4;                           // epilogue warp 0..7
-        const int team = ew >> 2;                          // tiles 2c + team
+        const int team = ew >> 2;                          // half of every tile: columns kGBN * team ..
         const int tt = (ew & 3) * 32 + lane;               // thread in team 0..127
         const int quarter = warp & 3;                      // TMEM lanes 32*quarter .. +31
         const int row_in_tile = quarter * 32 + lane;
@@ -280,7 +286,8 @@ w4a4_gemm_grouped_kernel(const __grid_constant__ CUtensorMap map_a, const __grid
         auto prefetch = [&](int i, int g0, int b) {
             if (i < ntl) {
                 const int tile = pair + i * num_pairs;
-                const int pm0 = (tile % p.num_m2) * 256 + 128 * int(rank), pn0 = (tile / p.num_m2) * kGBN;
+                const int pm0 = (tile % p.num_m2) * 256 + 128 * int(rank);
+                const int pn0 = (tile / p.num_m2) * kGWide + kGBN * team;
                 const int nb = (G - g0) < kGScaleBlock ? (G - g0) : kGScaleBlock;
                 const uint32_t base = sbase + sc_base + uint32_t(b) * kGScaleBytes;
 #pragma unroll
@@ -301,11 +308,11 @@ w4a4_gemm_grouped_kernel(const __grid_constant__ CUtensorMap map_a, const __grid
         };
         int cbuf = 0, sbuf = 0;
         bool aborted = false;
-        prefetch(team, 0, 0);
-        for (int i = team; i < ntl && !aborted; i += 2) {
+        prefetch(0, 0, 0);
+        for (int i = 0; i < ntl && !aborted; ++i) {
             const int tile = pair + i * num_pairs;
-            const int m0 = (tile % p.num_m2) * 256 + 128 * int(rank), n0 = (tile / p.num_m2) * kGBN;
-            const int c = i >> 1;
+            const int m0 = (tile % p.num_m2) * 256 + 128 * int(rank);
+            const int n0 = (tile / p.num_m2) * kGWide + kGBN * team;
             float2 acc[64];   // columns 2j, 2j + 1 of the tile
 #pragma unroll
             for (int j = 0; j < 64; ++j) acc[j] = make_float2(0.0f, 0.0f);
@@ -318,10 +325,10 @@ w4a4_gemm_grouped_kernel(const __grid_constant__ CUtensorMap map_a, const __grid
                     cp_async_wait_all();
                     team_bar(team);
                     if (g + kGScaleBlock < G) prefetch(i, g + kGScaleBlock, sbuf ^ 1);
-                    else prefetch(i + 2, 0, sbuf ^ 1);
+                    else prefetch(i + 1, 0, sbuf ^ 1);
                 }
-                // the team has G groups in every couple before c
-                const uint32_t ga = uint32_t(G) * uint32_t(c) + uint32_t(g);   // the team's group count
+                // G groups in every tile before i
+                const uint32_t ga = uint32_t(G) * uint32_t(i) + uint32_t(g);   // the team's group count
                 const uint32_t slot = 2 * team + (ga & 1);
                 // the warp decides together: the TMEM loads below are warp-collective
                 if (!__all_sync(0xFFFFFFFFu, mbar_wait(bar_tfull + 8 * slot, (ga >> 1) & 1, abort_flag)))
@@ -429,7 +436,7 @@ cudaError_t launch_grouped(const int8_t* A, const float* sa, const int8_t* B, co
     p.sa = sa; p.sb = sb; p.y32 = y32;
     p.M = (int)M; p.N = (int)N; p.K = (int)K;
     p.num_m2 = (int)((M + 255) / 256);
-    p.num_n = (int)((N + kGBN - 1) / kGBN);
+    p.num_n = (int)((N + kGWide - 1) / kGWide);
     p.num_k = (int)(K / kGroup);
     static thread_local int attr_dev = -1;
     int dev = 0;
