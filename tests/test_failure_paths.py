@@ -1,6 +1,6 @@
 """The library's error paths, exercised without faulting a GPU.
 
-SURVEY-planned failure handling: every entry point reports a status; a launch
+The library's own failure handling: every entry point reports a status; a launch
 failure maps to QUEST_ECUDA with the outputs untouched; a bounded device-side
 wait that runs out leaves QUEST_ETIMEOUT for quest_device_status. The faults are
 armed on the host (include/quest_debug.h): a simulated launch failure launches
