@@ -70,8 +70,8 @@ NOMINAL_INT8_TOPS = 4500.0   # nominal B200 dense int8 tensor-core rate (used on
 NCU_TRAFFIC = {
     "w4a4_linear": {"sources": ["bit_quantization_aware_blockwise_b200/csrc/w4a4_gemm.cu",
                                 "bit_quantization_aware_blockwise_b200/csrc/tc_common.cuh"],
-                    "sha256": "cfbca22a76b949f761c98afe5bc39339a414144f54c04d83fdd1c0c884f20141",
-                    "dram_read": 64602368, "dram_write": 146513024},
+                    "sha256": "1c75746fed44389d0acabf3c34564f0990dde41d1b696c16a2954f95f582a6c2",
+                    "dram_read": 65882752, "dram_write": 146098816},
 }
 
 

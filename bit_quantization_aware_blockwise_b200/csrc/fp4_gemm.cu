@@ -204,7 +204,10 @@ fp4_gemm_pair_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_con
                 const int m0 = (tile % p.num_m2) * 256 + 128 * int(rank);
                 const int n0 = (tile / p.num_m2) * kFBN + (kFBN / 2) * int(rank);
                 for (int kb = 0; kb < p.num_k; ++kb) {
-                    if (!mbar_wait(bar_empty + 8 * stage, phase ^ 1, abort_flag)) { ok = false; break; }
+                    if (!mbar_wait(bar_empty + 8 * stage, phase ^ 1, abort_flag, kWaitLimitNs, kSuspendProducerNs)) {
+                        ok = false;
+                        break;
+                    }
                     if (even) mbar_arrive_expect_tx(bar_full + 8 * stage, kFTxBytes);
                     const uint32_t fb = full_even + 8 * stage;
                     tma_load_2d_pair(sbase + kFSmemA + stage * kFStageA, &map_a, kb * BK, m0, fb);
@@ -236,11 +239,17 @@ fp4_gemm_pair_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_con
             int local = 0;
             for (int tile = pair; tile < num_tiles && ok; tile += num_pairs, ++local) {
                 const uint32_t buf = local & 1, bphase = (local >> 1) & 1;
-                if (!mbar_wait(bar_tempty + 8 * buf, bphase ^ 1, abort_flag)) { ok = false; break; }
+                if (!mbar_wait(bar_tempty + 8 * buf, bphase ^ 1, abort_flag, kWaitLimitNs, kSuspendMmaNs)) {
+                    ok = false;
+                    break;
+                }
                 tc_fence_after();
                 const uint32_t d_tmem = tmem_base + buf * kFAccStride;
                 for (int kb = 0; kb < p.num_k; ++kb) {
-                    if (!mbar_wait(bar_full + 8 * stage, phase, abort_flag)) { ok = false; break; }
+                    if (!mbar_wait(bar_full + 8 * stage, phase, abort_flag, kWaitLimitNs, kSuspendMmaNs)) {
+                        ok = false;
+                        break;
+                    }
                     tc_fence_after();
                     const uint32_t a_addr = sbase + kFSmemA + stage * kFStageA;
                     const uint32_t b_addr = sbase + kFSmemB + stage * kFStageB;
@@ -281,7 +290,7 @@ fp4_gemm_pair_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_con
             }
             const int m = m0 + row_in_tile;
             const float sa_m = m < p.M ? p.sa[m] : 0.0f;
-            const bool got = mbar_wait(bar_tfull + 8 * buf, bphase, abort_flag);
+            const bool got = mbar_wait(bar_tfull + 8 * buf, bphase, abort_flag, kWaitLimitNs, kSuspendEpilogueNs);
             if (fepi_any(!got)) break;
             tc_fence_after();
             const uint32_t t_acc = tmem_base + lane_addr + buf * kFAccStride;

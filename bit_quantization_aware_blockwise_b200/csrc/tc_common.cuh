@@ -40,6 +40,14 @@ constexpr int kChunkCols = 32;                // epilogue columns per TMEM load 
 constexpr uint32_t kTmemCols = 512;           // two 256-column accumulators
 constexpr uint32_t kCBytes = BM * kChunkCols * 2;  // one bf16 staging chunk (8 KB)
 constexpr uint64_t kWaitLimitNs = 2000000000ull;            // 2 s per wait
+// Suspend-time hints (ns) of the bounded waits by role; 0 polls. With the MMA
+// issuer polling its full barrier (it waits on the operand feed most of the time)
+// the integer, FP4, 2:4-sparse and bf16 pair layers ran 4-8 % slower than with
+// every role parked (hints on the producer and epilogue alone changed nothing);
+// the grouped layer, whose per-group TMEM hand-off is latency-bound, polls.
+constexpr uint32_t kSuspendProducerNs = 2000;
+constexpr uint32_t kSuspendMmaNs = 2000;
+constexpr uint32_t kSuspendEpilogueNs = 2000;
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
     return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -66,6 +74,21 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
         : "memory");
     return ok != 0;
 }
+// The same test with a suspend-time hint: while the phase is incomplete the thread
+// is parked, up to hint_ns, and woken when the phase completes, instead of returning
+// at once. A polling warp issues a few instructions per try on a scheduler it shares
+// with warps doing the work (and draws power under the cap).
+__device__ __forceinline__ bool mbar_try_wait_hint(uint32_t bar, uint32_t parity, uint32_t hint_ns) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity), "r"(hint_ns)
+        : "memory");
+    return ok != 0;
+}
 __device__ __forceinline__ uint64_t global_timer_ns() {
     uint64_t t;
     asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
@@ -74,12 +97,14 @@ __device__ __forceinline__ uint64_t global_timer_ns() {
 
 // Bounded wait for the phase of `bar` with parity `parity`. Returns false when
 // the CTA is aborting (another role timed out) or this wait timed out.
+// suspend_ns > 0: each try parks the thread up to suspend_ns (see mbar_try_wait_hint).
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag,
-                                          uint64_t limit_ns = kWaitLimitNs) {
-    if (mbar_try_wait(bar, parity)) return true;
+                                          uint64_t limit_ns = kWaitLimitNs, uint32_t suspend_ns = 0) {
+    auto test = [&]() { return suspend_ns ? mbar_try_wait_hint(bar, parity, suspend_ns) : mbar_try_wait(bar, parity); };
+    if (test()) return true;
     const uint64_t t0 = global_timer_ns();
     for (uint32_t it = 1;; ++it) {
-        if (mbar_try_wait(bar, parity)) return true;
+        if (test()) return true;
         if ((it & 63u) == 0) {
             if (*abort_flag) return false;
             if (global_timer_ns() - t0 > limit_ns) {

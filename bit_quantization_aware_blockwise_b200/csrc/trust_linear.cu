@@ -143,7 +143,10 @@ bf16_pair_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constan
                 const int m0 = (tile / p.num_n) * 256 + 128 * int(rank);
                 const int k0 = (tile % p.num_n) * BN + 128 * int(rank);
                 for (int kb = 0; kb < p.num_k; ++kb) {
-                    if (!mbar_wait(bar_empty + 8 * stage, phase ^ 1, abort_flag)) { ok = false; break; }
+                    if (!mbar_wait(bar_empty + 8 * stage, phase ^ 1, abort_flag, kWaitLimitNs, kSuspendProducerNs)) {
+                        ok = false;
+                        break;
+                    }
                     if (even) mbar_arrive_expect_tx(bar_full + 8 * stage, kPTxBytes);
                     const uint32_t fb = full_even + 8 * stage;
                     tma_load_2d_pair(sbase + kPSmemA + stage * kPStageA, &map_a, kb * 64, m0, fb);
@@ -174,11 +177,17 @@ bf16_pair_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constan
             int local = 0;
             for (int tile = pair; tile < num_tiles && ok; tile += num_pairs, ++local) {
                 const uint32_t buf = local & 1, bphase = (local >> 1) & 1;
-                if (!mbar_wait(bar_tempty + 8 * buf, bphase ^ 1, abort_flag)) { ok = false; break; }
+                if (!mbar_wait(bar_tempty + 8 * buf, bphase ^ 1, abort_flag, kWaitLimitNs, kSuspendMmaNs)) {
+                    ok = false;
+                    break;
+                }
                 tc_fence_after();
                 const uint32_t d_tmem = tmem_base + buf * BN;
                 for (int kb = 0; kb < p.num_k; ++kb) {
-                    if (!mbar_wait(bar_full + 8 * stage, phase, abort_flag)) { ok = false; break; }
+                    if (!mbar_wait(bar_full + 8 * stage, phase, abort_flag, kWaitLimitNs, kSuspendMmaNs)) {
+                        ok = false;
+                        break;
+                    }
                     tc_fence_after();
                     const uint32_t a_addr = sbase + kPSmemA + stage * kPStageA;
                     const uint32_t b_addr = sbase + kPSmemB + stage * kPStageB;
@@ -222,7 +231,7 @@ bf16_pair_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constan
                         mw[b] = *reinterpret_cast<const uint4*>(p.mask + int64_t(m) * mask_row_bytes + kb0 / 8);
                 }
             }
-            const bool got = mbar_wait(bar_tfull + 8 * buf, bphase, abort_flag);
+            const bool got = mbar_wait(bar_tfull + 8 * buf, bphase, abort_flag, kWaitLimitNs, kSuspendEpilogueNs);
             if (epi_any(!got)) break;
             tc_fence_after();
             const uint32_t t_acc = tmem_base + lane_addr + buf * BN;

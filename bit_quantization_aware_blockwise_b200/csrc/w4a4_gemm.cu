@@ -143,7 +143,10 @@ w4a4_gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constan
             for (int tile = blockIdx.x; tile < num_tiles && ok && !p.withhold; tile += gridDim.x) {
                 const int m0 = (tile % p.num_m) * BM, n0 = (tile / p.num_m) * BN;
                 for (int kb = 0; kb < p.num_k; ++kb) {
-                    if (!mbar_wait(bar_empty + 8 * stage, phase ^ 1, abort_flag, p.limit_ns)) { ok = false; break; }
+                    if (!mbar_wait(bar_empty + 8 * stage, phase ^ 1, abort_flag, p.limit_ns, kSuspendProducerNs)) {
+                        ok = false;
+                        break;
+                    }
                     const uint32_t fb = bar_full + 8 * stage;
                     mbar_arrive_expect_tx(fb, kStageBytes);
                     tma_load_2d(sbase + kSmemA + stage * kStageA, &map_a, kb * BK, m0, fb);
@@ -171,11 +174,17 @@ w4a4_gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constan
             int local = 0;
             for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x, ++local) {
                 const uint32_t buf = local & 1, bphase = (local >> 1) & 1;
-                if (!mbar_wait(bar_tempty + 8 * buf, bphase ^ 1, abort_flag, p.limit_ns)) { ok = false; break; }
+                if (!mbar_wait(bar_tempty + 8 * buf, bphase ^ 1, abort_flag, p.limit_ns, kSuspendMmaNs)) {
+                    ok = false;
+                    break;
+                }
                 tc_fence_after();
                 const uint32_t d_tmem = tmem_base + buf * BN;
                 for (int kb = 0; kb < p.num_k; ++kb) {
-                    if (!mbar_wait(bar_full + 8 * stage, phase, abort_flag, p.limit_ns)) { ok = false; break; }
+                    if (!mbar_wait(bar_full + 8 * stage, phase, abort_flag, p.limit_ns, kSuspendMmaNs)) {
+                        ok = false;
+                        break;
+                    }
                     tc_fence_after();
                     const uint32_t a_addr = sbase + kSmemA + stage * kStageA;
                     const uint32_t b_addr = sbase + kSmemB + stage * kStageB;
@@ -214,7 +223,7 @@ w4a4_gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constan
             }
             const int m = m0 + row_in_tile;
             const float sa_half = m < p.M ? p.sa[m] * 0.5f : 0.0f;
-            const bool got = mbar_wait(bar_tfull + 8 * buf, bphase, abort_flag, p.limit_ns);
+            const bool got = mbar_wait(bar_tfull + 8 * buf, bphase, abort_flag, p.limit_ns, kSuspendEpilogueNs);
             if (epi_any(!got)) break;  // all 128 threads leave together
             tc_fence_after();
             const uint32_t t_acc = tmem_base + lane_addr + buf * BN;
@@ -379,7 +388,10 @@ w4a4_gemm_pair_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_co
                 const int m0 = (tile % p.num_m2) * 256 + 128 * int(rank);
                 const int n0 = (tile / p.num_m2) * BN + 128 * int(rank);
                 for (int kb = 0; kb < p.num_k; ++kb) {
-                    if (!mbar_wait(bar_empty + 8 * stage, phase ^ 1, abort_flag)) { ok = false; break; }
+                    if (!mbar_wait(bar_empty + 8 * stage, phase ^ 1, abort_flag, kWaitLimitNs, kSuspendProducerNs)) {
+                        ok = false;
+                        break;
+                    }
                     if (even) mbar_arrive_expect_tx(bar_full + 8 * stage, kPTxBytes);
                     const uint32_t fb = full_even + 8 * stage;
                     tma_load_2d_pair(sbase + kPSmemA + stage * kPStageA, &map_a, kb * BK, m0, fb);
@@ -412,11 +424,17 @@ w4a4_gemm_pair_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_co
             int local = 0;
             for (int tile = pair; tile < num_tiles && ok; tile += num_pairs, ++local) {
                 const uint32_t buf = local & 1, bphase = (local >> 1) & 1;
-                if (!mbar_wait(bar_tempty + 8 * buf, bphase ^ 1, abort_flag)) { ok = false; break; }
+                if (!mbar_wait(bar_tempty + 8 * buf, bphase ^ 1, abort_flag, kWaitLimitNs, kSuspendMmaNs)) {
+                    ok = false;
+                    break;
+                }
                 tc_fence_after();
                 const uint32_t d_tmem = tmem_base + buf * BN;
                 for (int kb = 0; kb < p.num_k; ++kb) {
-                    if (!mbar_wait(bar_full + 8 * stage, phase, abort_flag)) { ok = false; break; }
+                    if (!mbar_wait(bar_full + 8 * stage, phase, abort_flag, kWaitLimitNs, kSuspendMmaNs)) {
+                        ok = false;
+                        break;
+                    }
                     tc_fence_after();
                     const uint32_t a_addr = sbase + kPSmemA + stage * kPStageA;
                     const uint32_t b_addr = sbase + kPSmemB + stage * kPStageB;
@@ -455,7 +473,7 @@ w4a4_gemm_pair_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_co
             }
             const int m = m0 + row_in_tile;
             const float sa_half = m < p.M ? p.sa[m] * 0.5f : 0.0f;
-            const bool got = mbar_wait(bar_tfull + 8 * buf, bphase, abort_flag);
+            const bool got = mbar_wait(bar_tfull + 8 * buf, bphase, abort_flag, kWaitLimitNs, kSuspendEpilogueNs);
             if (epi_any(!got)) break;  // all 128 threads leave together
             tc_fence_after();
             const uint32_t t_acc = tmem_base + lane_addr + buf * BN;

@@ -58,6 +58,9 @@ namespace {
 // this layer moves about 50). A lockstep layout (eight warps on the same group,
 // 64 columns each, two 32-column loads per wait) measured the same 403 us.
 
+// Every wait of this kernel polls: the hand-off of its TMEM slots is a latency chain,
+// and parking the waiting threads (the other tensor-core layers' setting) cost 1 %.
+constexpr uint32_t kGPollNs = 0;
 constexpr int kGThreads = 384;               // warpgroup 0: producer, MMA (2 warps idle); 1, 2: the teams
 constexpr int kGTeamThreads = 128;
 constexpr int kGBN = 128;                    // output columns per team (one half of a pair tile)
@@ -208,7 +211,10 @@ w4a4_gemm_grouped_kernel(const __grid_constant__ CUtensorMap map_a, const __grid
                 // half h's B rows: n0 + h * kGBN .. + kGBN / 2 - 1 in this CTA
                 const int n0 = (tile / p.num_m2) * kGWide + (kGBN / 2) * int(rank);
                 for (int kb = 0; kb < G && ok; ++kb) {
-                    if (!mbar_wait(bar_empty + 8 * stage, phase ^ 1, abort_flag)) { ok = false; break; }
+                    if (!mbar_wait(bar_empty + 8 * stage, phase ^ 1, abort_flag, kWaitLimitNs, kGPollNs)) {
+                        ok = false;
+                        break;
+                    }
                     if (even) mbar_arrive_expect_tx(bar_full + 8 * stage, kGTxBytes);
                     const uint32_t fb = full_even + 8 * stage;
                     const uint32_t b_st = sbase + kGSmemB + stage * kGStageB;
@@ -241,14 +247,20 @@ w4a4_gemm_grouped_kernel(const __grid_constant__ CUtensorMap map_a, const __grid
             bool ok = true;
             for (int i = 0; i < ntl && ok; ++i) {
                 for (int kb = 0; kb < G && ok; ++kb) {
-                    if (!mbar_wait(bar_full + 8 * stage, phase, abort_flag)) { ok = false; break; }
+                    if (!mbar_wait(bar_full + 8 * stage, phase, abort_flag, kWaitLimitNs, kGPollNs)) {
+                        ok = false;
+                        break;
+                    }
                     const uint32_t a_addr = sbase + kGSmemA + stage * kGStageA;
                     const uint32_t b_st = sbase + kGSmemB + stage * kGStageB;
                     const uint32_t sphase = (gc >> 1) & 1;
 #pragma unroll 1
                     for (int h = 0; h < 2; ++h) {
                         const uint32_t slot = 2 * h + (gc & 1);
-                        if (!mbar_wait(bar_tempty + 8 * slot, sphase ^ 1, abort_flag)) { ok = false; break; }
+                        if (!mbar_wait(bar_tempty + 8 * slot, sphase ^ 1, abort_flag, kWaitLimitNs, kGPollNs)) {
+                            ok = false;
+                            break;
+                        }
                         tc_fence_after();
                         const uint32_t d_tmem = tmem_base + slot * kGBN;
                         const uint32_t b_addr = b_st + h * kGStageBHalf;
@@ -331,8 +343,8 @@ w4a4_gemm_grouped_kernel(const __grid_constant__ CUtensorMap map_a, const __grid
                 const uint32_t ga = uint32_t(G) * uint32_t(i) + uint32_t(g);   // the team's group count
                 const uint32_t slot = 2 * team + (ga & 1);
                 // the warp decides together: the TMEM loads below are warp-collective
-                if (!__all_sync(0xFFFFFFFFu, mbar_wait(bar_tfull + 8 * slot, (ga >> 1) & 1, abort_flag)))
-                    aborted = true;
+                const bool got = mbar_wait(bar_tfull + 8 * slot, (ga >> 1) & 1, abort_flag, kWaitLimitNs, kGPollNs);
+                if (!__all_sync(0xFFFFFFFFu, got)) aborted = true;
                 if (aborted) continue;   // later waits return at once (abort flag); exit at the next check
                 tc_fence_after();
                 const uint32_t t_grp = tmem_base + lane_addr + slot * kGBN;

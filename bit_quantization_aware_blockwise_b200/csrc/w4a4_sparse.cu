@@ -285,7 +285,10 @@ w4a4_sparse_kernel(const __grid_constant__ CUtensorMap map_w, const __grid_const
             for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
                 const int n0 = (tile % p.num_n) * SBM, m0 = (tile / p.num_n) * SBN;
                 for (int kb = 0; kb < p.num_k; ++kb) {
-                    if (!mbar_wait(bar_empty + 8 * stage, phase ^ 1, abort_flag)) { ok = false; break; }
+                    if (!mbar_wait(bar_empty + 8 * stage, phase ^ 1, abort_flag, kWaitLimitNs, kSuspendProducerNs)) {
+                        ok = false;
+                        break;
+                    }
                     const uint32_t fb = bar_full + 8 * stage;
                     mbar_arrive_expect_tx(fb, kSTx);
                     tma_load_2d(sbase + kSSmemA + stage * kSStageA, &map_w, kb * (SBK / 2), n0, fb);
@@ -313,11 +316,17 @@ w4a4_sparse_kernel(const __grid_constant__ CUtensorMap map_w, const __grid_const
             int local = 0;
             for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x, ++local) {
                 const uint32_t buf = local & 1, bphase = (local >> 1) & 1;
-                if (!mbar_wait(bar_tempty + 8 * buf, bphase ^ 1, abort_flag)) { ok = false; break; }
+                if (!mbar_wait(bar_tempty + 8 * buf, bphase ^ 1, abort_flag, kWaitLimitNs, kSuspendMmaNs)) {
+                    ok = false;
+                    break;
+                }
                 tc_fence_after();
                 const uint32_t d_tmem = tmem_base + buf * kSAccCols;
                 for (int kb = 0; kb < p.num_k; ++kb) {
-                    if (!mbar_wait(bar_full + 8 * stage, phase, abort_flag)) { ok = false; break; }
+                    if (!mbar_wait(bar_full + 8 * stage, phase, abort_flag, kWaitLimitNs, kSuspendMmaNs)) {
+                        ok = false;
+                        break;
+                    }
                     tc_fence_after();
                     const uint32_t a_addr = sbase + kSSmemA + stage * kSStageA;
                     const uint32_t b_addr = sbase + kSSmemB + stage * kSStageB;
@@ -358,7 +367,7 @@ w4a4_sparse_kernel(const __grid_constant__ CUtensorMap map_w, const __grid_const
             }
             const int n = n0 + row;
             const float sw_half = n < p.N ? p.sw[n] * 0.5f : 0.0f;
-            const bool got = mbar_wait(bar_tfull + 8 * buf, bphase, abort_flag);
+            const bool got = mbar_wait(bar_tfull + 8 * buf, bphase, abort_flag, kWaitLimitNs, kSuspendEpilogueNs);
             if (epi_any(!got)) break;   // also orders the token scales above (bar.red)
             tc_fence_after();
             const uint32_t t_acc = tmem_base + lane_addr + buf * kSAccCols;
@@ -537,7 +546,10 @@ w4a4_sparse_pair_kernel(const __grid_constant__ CUtensorMap map_w, const __grid_
                 if (kResident && tile_n2(tile) != cur_n2) {
                     // the whole reduction's metadata of this CTA's 128 weight rows, once
                     // the previous weight tile's block has been copied into TMEM
-                    if (!mbar_wait(bar_mempty, mphase ^ 1, abort_flag)) { ok = false; break; }
+                    if (!mbar_wait(bar_mempty, mphase ^ 1, abort_flag, kWaitLimitNs, kSuspendProducerNs)) {
+                        ok = false;
+                        break;
+                    }
                     if (even) mbar_arrive_expect_tx(bar_mfull, 2u * uint32_t(p.num_k) * kSStageE);
                     const uint32_t mb = map_to_rank(bar_mfull, 0);
                     for (int kb = 0; kb < p.num_k; ++kb)
@@ -547,7 +559,10 @@ w4a4_sparse_pair_kernel(const __grid_constant__ CUtensorMap map_w, const __grid_
                     cur_n2 = tile_n2(tile);
                 }
                 for (int kb = 0; kb < p.num_k; ++kb) {
-                    if (!mbar_wait(bar_empty + 8 * stage, phase ^ 1, abort_flag)) { ok = false; break; }
+                    if (!mbar_wait(bar_empty + 8 * stage, phase ^ 1, abort_flag, kWaitLimitNs, kSuspendProducerNs)) {
+                        ok = false;
+                        break;
+                    }
                     if (even) mbar_arrive_expect_tx(bar_full + 8 * stage, L::kTx);
                     const uint32_t fb = full_even + 8 * stage;
                     tma_load_2d_pair(sbase + L::kA + stage * kSStageA, &map_w, kb * (SBK / 2), n0, fb);
@@ -587,15 +602,21 @@ w4a4_sparse_pair_kernel(const __grid_constant__ CUtensorMap map_w, const __grid_
             int local = 0, cur_n2 = -1;
             for (int tile = t_begin; tile < t_end && ok; tile += t_step, ++local) {
                 const uint32_t buf = local & 1, bphase = (local >> 1) & 1;
-                if (!mbar_wait(bar_tempty + 8 * buf, bphase ^ 1, abort_flag)) { ok = false; break; }
+                if (!mbar_wait(bar_tempty + 8 * buf, bphase ^ 1, abort_flag, kWaitLimitNs, kSuspendMmaNs)) {
+                    ok = false;
+                    break;
+                }
                 if (kResident && tile_n2(tile) != cur_n2) {
                     if (cur_n2 >= 0) {
                         // the previous tile's MMAs (its accumulator commit) must have read
                         // the old metadata before the copies overwrite those columns
                         const uint32_t pb = (local - 1) & 1, pph = ((local - 1) >> 1) & 1;
-                        if (!mbar_wait(bar_tfull + 8 * pb, pph, abort_flag)) { ok = false; break; }
+                        if (!mbar_wait(bar_tfull + 8 * pb, pph, abort_flag, kWaitLimitNs, kSuspendMmaNs)) {
+                            ok = false;
+                            break;
+                        }
                     }
-                    if (!mbar_wait(bar_mfull, mphase, abort_flag)) { ok = false; break; }
+                    if (!mbar_wait(bar_mfull, mphase, abort_flag, kWaitLimitNs, kSuspendMmaNs)) { ok = false; break; }
                     tc_fence_after();
                     for (int kb = 0; kb < p.num_k; ++kb)
                         tc_cp_meta_pair(tmem_base + kSMetaCol + 4 * kb, smem_desc_meta(sbase + L::kE + kb * kSStageE));
@@ -606,7 +627,10 @@ w4a4_sparse_pair_kernel(const __grid_constant__ CUtensorMap map_w, const __grid_
                 tc_fence_after();
                 const uint32_t d_tmem = tmem_base + buf * kSAccCols;
                 for (int kb = 0; kb < p.num_k; ++kb) {
-                    if (!mbar_wait(bar_full + 8 * stage, phase, abort_flag)) { ok = false; break; }
+                    if (!mbar_wait(bar_full + 8 * stage, phase, abort_flag, kWaitLimitNs, kSuspendMmaNs)) {
+                        ok = false;
+                        break;
+                    }
                     tc_fence_after();
                     const uint32_t a_addr = sbase + L::kA + stage * kSStageA;
                     const uint32_t b_addr = sbase + L::kB + stage * kPSStageB;
@@ -647,7 +671,7 @@ w4a4_sparse_pair_kernel(const __grid_constant__ CUtensorMap map_w, const __grid_
             }
             const int n = n0 + row;
             const float sw_half = n < p.N ? p.sw[n] * 0.5f : 0.0f;
-            const bool got = mbar_wait(bar_tfull + 8 * buf, bphase, abort_flag);
+            const bool got = mbar_wait(bar_tfull + 8 * buf, bphase, abort_flag, kWaitLimitNs, kSuspendEpilogueNs);
             if (epi_any(!got)) break;   // also orders the token scales above (bar.red)
             tc_fence_after();
             const uint32_t t_acc = tmem_base + lane_addr + buf * kSAccCols;
