@@ -258,3 +258,29 @@ def test_fp4_linear_rejects_invalid_arguments():
                dict(w=FAKE + 8), dict(sa=FAKE + 2), dict(acc=FAKE + 6), dict(y=FAKE + 8), dict(M=1 << 31)]:
         assert call(**kw) == 1, kw
     assert call(M=0, a=None, w=None, sa=None, sw=None, y=None) == 0
+
+
+def test_grouped_linear_rejects_invalid_arguments():
+    lib = q.load_library()
+
+    def call(a=FAKE, sa=FAKE + (1 << 20), w=FAKE + (1 << 24), sw=FAKE + (1 << 21), M=4, N=16, K=256, group=128,
+             y=FAKE + (1 << 25), y32=None):
+        return lib.quest_w4a4_linear_grouped(a, sa, w, sw, M, N, K, group, y, y32, None)
+    for kw in [dict(M=-1), dict(K=200), dict(K=1 << 24), dict(N=12), dict(y=None), dict(a=None), dict(sw=None),
+               dict(w=FAKE + 8), dict(sa=FAKE + 2), dict(y32=FAKE + 6), dict(y=FAKE + 8), dict(M=1 << 31)]:
+        assert call(**kw) == 1, kw
+    assert call(group=64) == 2 and call(group=256) == 2      # the layer takes 128-value groups only
+    assert call(M=0, a=None, w=None, sa=None, sw=None, y=None) == 0
+
+
+def test_sparse24_linear_rejects_invalid_arguments():
+    lib = q.load_library()
+
+    def call(x=FAKE, sx=FAKE + (1 << 20), w=FAKE + (1 << 24), meta=FAKE + (1 << 23), sw=FAKE + (1 << 21), M=4,
+             N=16, K=256, y=FAKE + (1 << 25), acc=None):
+        return lib.quest_w4a4_linear_sparse24(x, sx, w, meta, sw, M, N, K, y, acc, None)
+    for kw in [dict(M=-1), dict(K=192), dict(K=131072), dict(N=12), dict(y=None), dict(x=None), dict(meta=None),
+               dict(sw=None), dict(w=FAKE + 8), dict(meta=FAKE + 4), dict(sx=FAKE + 2), dict(acc=FAKE + 6),
+               dict(y=FAKE + 8), dict(N=1 << 31)]:
+        assert call(**kw) == 1, kw
+    assert call(N=0, x=None, w=None, meta=None, sx=None, sw=None, y=None) == 0

@@ -25,6 +25,19 @@ def test_part_bytes_by_hand():
     assert 590e6 < sum(p.values()) < 595e6
 
 
+def test_traffic_is_reported_only_for_the_captured_sources(monkeypatch):
+    rec = bench.NCU_TRAFFIC["w4a4_linear"]
+    # the record's hash is of the sources as they stand, so its bytes are reported
+    assert bench.ncu_traffic("w4a4_linear") == rec["dram_read"] + rec["dram_write"]
+    assert 200e6 < bench.ncu_traffic("w4a4_linear") < 240e6      # about the 229.7 MB algorithmic
+    # any change to the kernel's sources withdraws it
+    monkeypatch.setitem(bench.NCU_TRAFFIC, "w4a4_linear", dict(rec, sha256="0" * 64))
+    assert bench.ncu_traffic("w4a4_linear") is None
+    monkeypatch.setitem(bench.NCU_TRAFFIC, "w4a4_linear", dict(rec, sources=rec["sources"] + ["missing.cu"]))
+    assert bench.ncu_traffic("w4a4_linear") is None
+    assert bench.ncu_traffic("quantize_fwd") is None
+
+
 def _free_port():
     with socket.socket() as s:
         s.bind(("127.0.0.1", 0))
