@@ -38,6 +38,45 @@ def test_traffic_is_reported_only_for_the_captured_sources(monkeypatch):
     assert bench.ncu_traffic("quantize_fwd") is None
 
 
+class _FakeNvml:
+    """The NVML names the clock sampler reads, with the bit values NVML defines."""
+    NVML_CLOCK_SM = 1
+    nvmlClocksEventReasonGpuIdle = 0x1
+    nvmlClocksEventReasonApplicationsClocksSetting = 0x2
+    nvmlClocksEventReasonSwPowerCap = 0x4
+    nvmlClocksEventReasonHwSlowdown = 0x8
+    nvmlClocksEventReasonSyncBoost = 0x10
+    nvmlClocksEventReasonSwThermalSlowdown = 0x20
+    nvmlClocksEventReasonHwThermalSlowdown = 0x40
+    nvmlClocksEventReasonHwPowerBrakeSlowdown = 0x80
+
+    def __init__(self, seq):
+        self.seq = list(seq)
+
+    def nvmlDeviceGetClockInfo(self, h, which):
+        return self.seq[0][0]
+
+    def nvmlDeviceGetCurrentClocksEventReasons(self, h):
+        return self.seq.pop(0)[1]
+
+
+def test_clock_summary_from_samples():
+    cs = bench.ClockSampler.__new__(bench.ClockSampler)
+    cs.ok, cs.samples, cs.max_mhz, cs.h = True, [], 1965, None
+    cs.nv = _FakeNvml([(1965, 0x1), (1875, 0x4), (1852, 0x4), (1965, 0x0), (1900, 0x4 | 0x1)])
+    for _ in range(5):
+        cs.sample_now()
+    out = cs.summary()
+    assert out == {"sm_mhz": 1900, "sm_max_mhz": 1965, "reasons": ["sw_power_cap"], "samples": 5}
+    cs.nv.seq = [(1500, 0x40 | 0x8)]
+    cs.sample_now()
+    # reasons are the union over the timed region: one throttled sample marks the run
+    assert cs.summary()["reasons"] == ["hw_slowdown", "hw_thermal_slowdown", "sw_power_cap"]
+    # without NVML the line says so instead of guessing a clock
+    cs.ok = False
+    assert cs.summary()["sm_mhz"] is None and "NVML" in cs.summary()["note"]
+
+
 def _free_port():
     with socket.socket() as s:
         s.bind(("127.0.0.1", 0))
